@@ -1,0 +1,271 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test ties one oracle function to a library routine, a closed form, an invariant
+or an independent formulation, chosen so that a plausible slip (a dropped term, a sign,
+a transposed operand, an off-by-one position, a wrong head mapping) fails.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+from bandwidth_bound_stream_b200 import synth
+from oracle import oracle as orc
+
+FP16, BF16 = 0, 1
+
+
+# ---------------------------------------------------------------- storage types
+
+def test_fp16_values_match_numpy_for_every_pattern():
+    bits = np.arange(65536, dtype=np.uint16)
+    got = orc.value(bits, FP16)
+    want = bits.view(np.float16).astype(np.float64)
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    assert np.array_equal(got[ok], want[ok])
+
+
+def test_bf16_values_match_torch_for_every_pattern():
+    bits = np.arange(65536, dtype=np.uint16)
+    got = orc.value(bits, BF16)
+    want = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    ok = ~np.isnan(want)
+    assert np.array_equal(np.isnan(got), ~ok)
+    assert np.array_equal(got[ok], want[ok])
+
+
+def test_store_fp16_matches_numpy_rounding():
+    rng = np.random.default_rng(0)
+    v = np.concatenate([rng.normal(0, 1, 4000), rng.normal(0, 1e-5, 2000), rng.normal(0, 2e4, 1000),
+                        rng.normal(0, 1e-7, 1000), [0.0, -0.0, 65504.0, 65519.99, 65520.0, 1e9, 2.0**-24, 2.0**-25,
+                                                    3 * 2.0**-26, 1 + 2.0**-11, 1 + 3 * 2.0**-11]])
+    want = v.astype(np.float32).astype(np.float16).view(np.uint16)
+    assert np.array_equal(orc.store(v, FP16), want)
+
+
+def test_store_bf16_matches_torch_rounding():
+    rng = np.random.default_rng(1)
+    v = np.concatenate([rng.normal(0, 1, 4000), rng.normal(0, 1e-30, 500), [0.0, 1.0 + 2.0**-8, 1.0 + 3 * 2.0**-8]])
+    want = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(orc.store(v, BF16), want)
+
+
+# ---------------------------------------------------------------- building blocks
+
+def test_matvec_matches_numpy_matmul_and_orientation():
+    rng = np.random.default_rng(2)
+    W = synth.normal_u16(5, 0x333, 37 * 131, FP16).reshape(37, 131)
+    x = rng.normal(size=131)
+    want = W.view(np.float16).astype(np.float64) @ x
+    got = orc.matvec(W, FP16, x)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-15)
+    # a transposed operand would not even have the right length
+    assert got.shape == (37,)
+
+
+def test_rmsnorm_closed_forms():
+    g = synth.gain_u16(64, BF16)
+    x = np.full(64, 3.0)
+    np.testing.assert_allclose(orc.rmsnorm(x, g, BF16, 1e-5), 3.0 / np.sqrt(9.0 + 1e-5), rtol=1e-15)
+    rng = np.random.default_rng(3)
+    x = rng.normal(0, 7, 256)
+    y = orc.rmsnorm(x, synth.gain_u16(256, FP16), FP16, 0.0)
+    assert abs(np.sqrt(np.mean(y * y)) - 1.0) < 1e-14
+    # the gain multiplies element-wise (fp16 0x4000 = 2.0)
+    g2 = synth.gain_u16(256, FP16)
+    g2[7] = 0x4000
+    y2 = orc.rmsnorm(x, g2, FP16, 0.0)
+    assert y2[7] == pytest.approx(2 * y[7], rel=1e-15) and np.array_equal(np.delete(y2, 7), np.delete(y, 7))
+
+
+def _rope_complex(v, pos, theta):
+    """Rotate-half RoPE as complex multiplication: (v_i + i v_{i+D/2}) * exp(i pos theta^(-2i/D))."""
+    D = v.size
+    half = D // 2
+    z = v[:half] + 1j * v[half:]
+    ang = pos * theta ** (-2.0 * np.arange(half) / D)
+    r = z * np.exp(1j * ang)
+    return np.concatenate([r.real, r.imag])
+
+
+def test_rope_equals_complex_rotation():
+    rng = np.random.default_rng(4)
+    for D, pos, theta in [(128, 0, 1e4), (128, 1, 1e4), (128, 4095, 5e5), (64, 17, 1e4), (2, 3, 1e4)]:
+        v = rng.normal(size=D)
+        np.testing.assert_allclose(orc.rope(v, pos, theta), _rope_complex(v, pos, theta), rtol=0, atol=1e-12)
+
+
+def test_rope_invariants():
+    rng = np.random.default_rng(5)
+    q, k = rng.normal(size=128), rng.normal(size=128)
+    assert np.array_equal(orc.rope(q, 0, 1e4), q)
+    for p in (1, 100, 32000):
+        assert np.linalg.norm(orc.rope(q, p, 1e4)) == pytest.approx(np.linalg.norm(q), rel=1e-13)
+    # <R_p q, R_p' k> depends only on p - p'
+    a = orc.rope(q, 1000, 1e4) @ orc.rope(k, 990, 1e4)
+    b = orc.rope(q, 10, 1e4) @ orc.rope(k, 0, 1e4)
+    assert a == pytest.approx(b, rel=1e-9)
+    # D = 2 is a plane rotation by pos radians
+    c, s = np.cos(3.0), np.sin(3.0)
+    np.testing.assert_allclose(orc.rope(np.array([1.0, 0.0]), 3, 1e4), [c, s], atol=1e-15)
+
+
+def _kv(rng, n, D, dtype):
+    K = orc.store(rng.normal(0, 1, (n, D)), dtype)
+    V = orc.store(rng.normal(0, 1, (n, D)), dtype)
+    return K, V
+
+
+def test_attention_single_key_returns_v_exactly():
+    rng = np.random.default_rng(6)
+    K, V = _kv(rng, 1, 128, FP16)
+    out = orc.attention(rng.normal(size=128) * 10, K, V, FP16)
+    assert np.array_equal(out, orc.value(V[0], FP16))
+
+
+def test_attention_matches_scipy_softmax():
+    rng = np.random.default_rng(7)
+    for n, D, dt in [(5, 64, FP16), (300, 128, BF16)]:
+        K, V = _kv(rng, n, D, dt)
+        q = rng.normal(size=D)
+        Kf, Vf = orc.value(K, dt), orc.value(V, dt)
+        w = scipy.special.softmax(Kf @ q / np.sqrt(D))
+        assert w.sum() == pytest.approx(1.0, abs=1e-12)
+        np.testing.assert_allclose(orc.attention(q, K, V, dt), w @ Vf, rtol=1e-11, atol=1e-13)
+
+
+def test_attention_uniform_scores_average_values():
+    rng = np.random.default_rng(8)
+    _, V = _kv(rng, 9, 64, FP16)
+    K = np.tile(orc.store(rng.normal(size=64), FP16), (9, 1))
+    out = orc.attention(rng.normal(size=64), K, V, FP16)
+    np.testing.assert_allclose(out, orc.value(V, FP16).mean(axis=0), rtol=1e-13, atol=1e-15)
+
+
+def test_silu_and_argmax():
+    for z in (-20.0, -1.0, 0.0, 0.5, 3.0, 30.0):
+        assert orc.silu(z) == pytest.approx(z * scipy.special.expit(z), rel=1e-14, abs=1e-300)
+    assert orc.argmax(np.array([1.0, 5.0, 2.0, 5.0])) == 1
+    assert orc.argmax(np.array([-3.0, -3.0])) == 0
+
+
+# ---------------------------------------------------------------- the whole step
+
+MINI = synth.ModelConfig("mini", 2, 128, 4, 2, 32, 192, 97, FP16, rope_theta=1e4)
+
+
+def _weights(cfg, seed=0):
+    return synth.model_weights(cfg, seed)
+
+
+def test_incremental_decode_equals_full_recompute():
+    for cfg in (MINI, dataclasses.replace(MINI, dtype=BF16, n_kv_heads=4, rope_theta=5e5)):
+        w = _weights(cfg)
+        toks = synth.prompt(cfg, 13)
+        m = orc.OracleModel(cfg, w, max_ctx=16)
+        inc = np.stack([m.step(t) for t in toks])
+        full = orc.OracleModel(cfg, w, max_ctx=16).forward_sequence(toks)
+        np.testing.assert_allclose(inc, full, rtol=0, atol=1e-12)
+
+
+def test_gqa_equals_mha_with_repeated_kv_heads():
+    cfg = MINI
+    w = _weights(cfg)
+    mha_cfg = dataclasses.replace(cfg, n_kv_heads=cfg.n_heads)
+    rep = cfg.n_heads // cfg.n_kv_heads
+    w_mha = {k: v for k, v in w.items() if k != "layers"}
+    w_mha["layers"] = []
+    D = cfg.head_dim
+    for L in w["layers"]:
+        L2 = dict(L)
+        for name in ("wk", "wv"):
+            heads = L[name].reshape(cfg.n_kv_heads, D, cfg.d_model)
+            L2[name] = np.repeat(heads, rep, axis=0).reshape(cfg.n_heads * D, cfg.d_model)
+        w_mha["layers"].append(L2)
+    toks = synth.prompt(cfg, 6)
+    a = orc.OracleModel(cfg, w, 8)
+    b = orc.OracleModel(mha_cfg, w_mha, 8)
+    for t in toks:
+        np.testing.assert_array_equal(a.step(t), b.step(t))
+
+
+def _f(bits, dt):
+    return orc.value(bits, dt)
+
+
+def test_identity_blocks_reduce_to_embedding_times_head():
+    """With Wo = 0 and Wd = 0 the residual stays E[tok]: logits = W_lm rmsnorm(E[tok])."""
+    cfg = MINI
+    w = _weights(cfg)
+    for L in w["layers"]:
+        L["wo"] = np.zeros_like(L["wo"])
+        L["w_down"] = np.zeros_like(L["w_down"])
+    m = orc.OracleModel(cfg, w, 4)
+    tok = 11
+    e = _f(w["tok_emb"][tok], cfg.dtype)
+    h = e / np.sqrt(np.mean(e * e) + cfg.rms_eps)
+    want = _f(w["lm_head"], cfg.dtype) @ h
+    np.testing.assert_allclose(m.step(tok), want, rtol=1e-12, atol=1e-14)
+
+
+def test_first_position_value_path_and_cache_write():
+    """One layer at position 0: attention returns the stored v, so x = E + Wo v (+ MLP)."""
+    cfg = dataclasses.replace(MINI, n_layers=1)
+    w = _weights(cfg)
+    L = w["layers"][0]
+    L["w_down"] = np.zeros_like(L["w_down"])
+    m = orc.OracleModel(cfg, w, 4)
+    tok, pos = 5, 0
+    dt, D = cfg.dtype, cfg.head_dim
+    e = _f(w["tok_emb"][tok], dt)
+    h = e / np.sqrt(np.mean(e * e) + cfg.rms_eps)
+    k = _f(L["wk"], dt) @ h
+    v = _f(L["wv"], dt) @ h
+    v_st = v.astype(np.float32).astype(np.float16)
+    k_st = np.concatenate([_rope_complex(k[g * D:(g + 1) * D], pos, cfg.rope_theta)
+                           for g in range(cfg.n_kv_heads)]).astype(np.float32).astype(np.float16)
+    o = np.concatenate([v_st[(hh * cfg.n_kv_heads // cfg.n_heads) * D:][:D].astype(np.float64)
+                        for hh in range(cfg.n_heads)])
+    x = e + _f(L["wo"], dt) @ o
+    hf = x / np.sqrt(np.mean(x * x) + cfg.rms_eps)
+    want = _f(w["lm_head"], dt) @ hf
+    got = m.step(tok, pos)
+    np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-13)
+    assert np.array_equal(m.k_cache[0, :, pos].ravel(), k_st.view(np.uint16))
+    assert np.array_equal(m.v_cache[0, :, pos].ravel(), v_st.view(np.uint16))
+
+
+def test_cache_append_at_later_position_uses_that_position():
+    """Layer-0 K at position p depends on token p only: rotated by p, stored rounded."""
+    cfg = MINI
+    w = _weights(cfg)
+    m = orc.OracleModel(cfg, w, 8)
+    toks = synth.prompt(cfg, 5)
+    for t in toks:
+        m.step(t, want_logits=False)
+    p = 4
+    e = _f(w["tok_emb"][toks[p]], cfg.dtype)
+    h = e / np.sqrt(np.mean(e * e) + cfg.rms_eps)
+    k = _f(w["layers"][0]["wk"], cfg.dtype) @ h
+    D = cfg.head_dim
+    k_rot = np.concatenate([_rope_complex(k[g * D:(g + 1) * D], p, cfg.rope_theta) for g in range(cfg.n_kv_heads)])
+    assert np.array_equal(m.k_cache[0, :, p].ravel(), k_rot.astype(np.float32).astype(np.float16).view(np.uint16))
+
+
+def test_bad_arguments_rejected():
+    m = orc.OracleModel(MINI, _weights(MINI), 2)
+    with pytest.raises(ValueError):
+        m.step(MINI.vocab)
+    with pytest.raises(ValueError):
+        m.step(1, pos=2)
+
+
+def test_logit_scale_of_synthetic_model():
+    """N(0, 0.02) weights give logits of std ~0.02*sqrt(d) after the final unit-RMS norm."""
+    cfg = synth.TINY
+    m = orc.OracleModel(cfg, _weights(cfg), 4)
+    lg = m.step(int(synth.prompt(cfg, 1)[0]))
+    assert 0.5 * 0.02 * np.sqrt(cfg.d_model) < lg.std() < 2.0 * 0.02 * np.sqrt(cfg.d_model)
