@@ -16,8 +16,8 @@ INCLUDE = os.path.join(ROOT, "include")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
-KIE_SOURCES = ["kie_engine.cu", "kie_b1.cu", "kie_mr.cu", "kie_attn.cu"]
-KIE_HEADERS = ["kie_device.cuh", "kie_internal.h"]
+KIE_SOURCES = ["kie_engine.cu", "kie_b1.cu", "kie_attn.cu"]
+KIE_HEADERS = ["kie_device.cuh", "kie_internal.h", "kie_attn.cuh"]
 
 
 def _run(cmd):
@@ -51,17 +51,25 @@ def build_kie(force: bool = False, verbose_ptxas: bool = False) -> str:
         return out
     objdir = os.path.join(HERE, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
+    objs, procs = [], []
     for s in srcs:
         o = os.path.join(objdir, os.path.basename(s) + ".o")
         cmd = [NVCC, *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-rdc=false",
                "-I", INCLUDE, "-I", CSRC, "-c", s, "-o", o]
         if verbose_ptxas:
             cmd.insert(1, "-Xptxas=-v")
-        log = _run(cmd)
-        if verbose_ptxas:
-            sys.stdout.write(log)
+        procs.append((cmd, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)))
         objs.append(o)
+    failed = False
+    for cmd, pr in procs:
+        log, _ = pr.communicate()
+        if pr.returncode != 0:
+            sys.stderr.write(log)
+            failed = True
+        elif verbose_ptxas:
+            sys.stdout.write(log)
+    if failed:
+        raise RuntimeError("nvcc failed")
     _run([NVCC, *ARCH, "-shared", "-o", out, *objs, "-lcuda"])
     return out
 

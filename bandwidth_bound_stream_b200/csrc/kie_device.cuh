@@ -1,0 +1,173 @@
+// Device-side building blocks for sm_100a: mbarriers, bulk async copies, scoped
+// atomics, bounded waits, storage-type conversions.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "kie_internal.h"
+
+#define KIE_DEV __device__ __forceinline__
+
+// ------------------------------------------------------------------ clocks, fences, barriers
+
+KIE_DEV uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+KIE_DEV void named_bar_sync(int id, int count) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory"); }
+
+KIE_DEV uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+KIE_DEV unsigned long long ld_acquire_gpu_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+KIE_DEV void red_release_gpu_add_u64(unsigned long long *p, unsigned long long v) {
+    asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+KIE_DEV uint32_t ld_acquire_sys_u32(const volatile uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+KIE_DEV void st_release_sys_u32(volatile uint32_t *p, uint32_t v) {
+    asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+KIE_DEV unsigned ld_volatile_u32(const unsigned *p) { return *(const volatile unsigned *)p; }
+
+// Records the first device error (code, where). Later errors keep the first.
+KIE_DEV void set_error(unsigned *err, unsigned code, unsigned where) {
+    atomicCAS(err, 0u, (code << 8) | (where & 0xFFu));
+}
+
+// ------------------------------------------------------------------ mbarrier
+
+KIE_DEV void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+KIE_DEV void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+
+KIE_DEV void mbar_arrive(uint64_t *bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+KIE_DEV void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
+                     smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+KIE_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait on an mbarrier phase. Returns false on timeout or when *abort becomes set.
+KIE_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, long long timeout_ns, const volatile int *abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    uint64_t t0 = globaltimer();
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (abort && *abort) return false;
+        if ((long long)(globaltimer() - t0) > timeout_ns) return false;
+    }
+}
+
+// ------------------------------------------------------------------ bulk async copy (TMA, 1-D, no multicast)
+
+// Global -> this CTA's shared memory; completion is signalled as transaction bytes on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+KIE_DEV void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+// ------------------------------------------------------------------ storage types
+
+// 8 stored elements (one 16-byte vector) -> 8 floats.
+template <int DT>
+KIE_DEV void cvt8(const uint4 &v, float *f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        if (DT == KIE_BF16) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        } else {
+            __half2 h = *reinterpret_cast<const __half2 *>(&w[i]);
+            float2 t = __half22float2(h);
+            f[2 * i] = t.x;
+            f[2 * i + 1] = t.y;
+        }
+    }
+}
+
+template <int DT>
+KIE_DEV float cvt1(uint16_t b) {
+    if (DT == KIE_BF16) return __uint_as_float((uint32_t)b << 16);
+    return __half2float(__ushort_as_half(b));
+}
+
+// float -> storage element, round to nearest even.
+template <int DT>
+KIE_DEV uint16_t store1(float f) {
+    if (DT == KIE_BF16) return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+    return __half_as_ushort(__float2half_rn(f));
+}
+
+KIE_DEV float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+KIE_DEV float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Reduces R partial sums (R in 1,2,4,8) across the warp. Afterwards lane l holds the full
+// sum of row l / (32 / R) (every lane of that row group holds it).
+template <int R>
+KIE_DEV float warp_reduce_rows(float (&acc)[8]) {
+    const int lane = threadIdx.x & 31;
+    int n = R;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        if (n > 1) {
+            const bool hi = (lane & off) != 0;
+            const int h = n >> 1;
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                if (j < h) {
+                    float send = hi ? acc[j] : acc[j + h];
+                    float keep = hi ? acc[j + h] : acc[j];
+                    acc[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                }
+            }
+            n = h;
+        } else {
+            acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], off);
+        }
+    }
+    return acc[0];
+}

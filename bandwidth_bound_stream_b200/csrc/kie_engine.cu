@@ -1,0 +1,674 @@
+// Host side of the decode engine: validation, the fixed (ahead-of-time) schedule and
+// memory layout, the weight repack, sessions, the doorbell and kernel launches.
+//
+// Everything the kernels will touch is allocated in kie_create and laid out once: the
+// schedule and addresses are fixed before the first token, with no allocator or scheduler
+// at run time ("实时AI推理为何贵56倍？…", section 把一切提前决定好). Per call the host only
+// writes input tokens into a mapped mailbox and reads output tokens back (same page,
+// section 让工作常驻 GPU).
+#include <cuda_runtime.h>
+#include <emmintrin.h>
+
+#include <algorithm>
+#include <atomic>
+#include <chrono>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "kie_internal.h"
+
+// kernels of the other translation units
+size_t kie_b1_smem_bytes();
+int kie_b1_vec_per_lane(int K);
+cudaError_t kie_b1_prepare(int dtype);
+cudaError_t kie_b1_occupancy(int dtype, int *blocks_per_sm);
+cudaError_t kie_b1_launch(const KieParams &P, const KieCmd &one, int resident, cudaStream_t stream);
+
+namespace {
+
+struct RowCopy {
+    long long dst;
+    const uint8_t *src;
+    long long bytes;
+};
+
+__global__ void gather_rows_kernel(const RowCopy *rc, long long n, uint8_t *arena) {
+    for (long long i = blockIdx.x; i < n; i += gridDim.x) {
+        const RowCopy r = rc[i];
+        for (long long b = (long long)threadIdx.x * 16; b < r.bytes; b += (long long)blockDim.x * 16)
+            *reinterpret_cast<uint4 *>(arena + r.dst + b) = *reinterpret_cast<const uint4 *>(r.src + b);
+    }
+}
+
+enum { KIND_NONE = 0, KIND_B1 = 1, KIND_MR = 2 };
+
+double now_s() {
+    return std::chrono::duration<double>(std::chrono::steady_clock::now().time_since_epoch()).count();
+}
+
+}  // namespace
+
+struct kie_engine {
+    kie_config cfg{};
+    int dev = 0, nblk = 0;
+    KieParams P{};
+    std::vector<void *> dev_allocs;
+    KieMailbox *mbox_host = nullptr;
+    KieMailbox *mbox_dev = nullptr;
+    int64_t io_ints = 0;
+    cudaStream_t stream = nullptr;
+    cudaEvent_t ev_done = nullptr;
+    int resident = KIND_NONE;  // which kernel currently sits resident on the GPU
+    uint32_t seq = 0;
+    std::vector<int> sess_len;
+    std::vector<char> sess_used;
+    bool poisoned = false;
+    std::string err;
+
+    kie_status fail(kie_status s, const char *fmt, ...) {
+        char buf[512];
+        va_list ap;
+        va_start(ap, fmt);
+        vsnprintf(buf, sizeof buf, fmt, ap);
+        va_end(ap);
+        err = buf;
+        if (s == KIE_ERR_TIMEOUT || s == KIE_ERR_DEVICE) poisoned = true;
+        return s;
+    }
+    kie_status cuda_fail(cudaError_t e, const char *what) {
+        return fail(KIE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    }
+    template <class T>
+    cudaError_t alloc(T **p, size_t bytes) {
+        void *q = nullptr;
+        cudaError_t e = cudaMalloc(&q, bytes < 16 ? 16 : bytes);
+        if (e == cudaSuccess) {
+            dev_allocs.push_back(q);
+            *p = static_cast<T *>(q);
+        }
+        return e;
+    }
+};
+
+#define CK(expr, what)                                        \
+    do {                                                      \
+        cudaError_t _e = (expr);                              \
+        if (_e != cudaSuccess) return eng->cuda_fail(_e, what); \
+    } while (0)
+
+// ---------------------------------------------------------------- small C-ABI helpers
+
+extern "C" void kie_config_defaults(kie_config *c) {
+    if (!c) return;
+    memset(c, 0, sizeof *c);
+    c->rms_eps = 1e-5f;
+    c->rope_theta = 1e4f;
+    c->dtype = KIE_FP16;
+    c->max_sessions = 1;
+    c->max_ctx = 4096;
+    c->timeout_ms = 10000;
+    c->idle_ms = 200;
+    c->modes = KIE_MODE_BATCH1;
+    c->device = 0;
+}
+
+extern "C" const char *kie_status_string(kie_status s) {
+    switch (s) {
+        case KIE_OK: return "ok";
+        case KIE_ERR_ARG: return "bad argument";
+        case KIE_ERR_CAPACITY: return "capacity exceeded";
+        case KIE_ERR_CUDA: return "CUDA error";
+        case KIE_ERR_TIMEOUT: return "timeout";
+        case KIE_ERR_STATE: return "engine poisoned";
+        case KIE_ERR_DEVICE: return "device error";
+        case KIE_ERR_UNSUPPORTED: return "mode not enabled";
+        default: return "unknown status";
+    }
+}
+
+extern "C" kie_status kie_last_error(kie_engine *eng, char *buf, int32_t len) {
+    if (!eng || !buf || len <= 0) return KIE_ERR_ARG;
+    snprintf(buf, (size_t)len, "%s", eng->err.c_str());
+    return KIE_OK;
+}
+
+// ---------------------------------------------------------------- validation and plan
+
+static const char *shape_error(const kie_config &c) {
+    if (c.n_layers <= 0 || c.d_model <= 0 || c.n_heads <= 0 || c.n_kv_heads <= 0 || c.head_dim <= 0 || c.ffn <= 0 ||
+        c.vocab <= 0)
+        return "all shape fields must be positive";
+    if (c.dtype != KIE_FP16 && c.dtype != KIE_BF16) return "dtype must be KIE_FP16 or KIE_BF16";
+    if (c.d_model % 64 || (c.n_heads * c.head_dim) % 64 || c.ffn % 64)
+        return "d_model, n_heads*head_dim and ffn must be multiples of 64";
+    if (c.head_dim != 8 && c.head_dim != 16 && c.head_dim != 32 && c.head_dim != 64 && c.head_dim != 128)
+        return "head_dim must be 8, 16, 32, 64 or 128";
+    if (c.n_heads % c.n_kv_heads || c.n_heads / c.n_kv_heads > KIE_GMAX)
+        return "n_heads must be a multiple of n_kv_heads, at most 8 query heads per kv head";
+    if (c.d_model > 8192) return "d_model above 8192 is not supported";
+    if (c.ffn > 16384 || c.n_heads * c.head_dim > 16384) return "ffn and n_heads*head_dim must be <= 16384";
+    if (c.max_sessions <= 0 || c.max_ctx <= 0) return "max_sessions and max_ctx must be positive";
+    if (c.timeout_ms <= 0 || c.idle_ms <= 0) return "timeouts must be positive";
+    if (!(c.modes & (KIE_MODE_BATCH1 | KIE_MODE_TICK))) return "modes must enable at least one kernel";
+    return nullptr;
+}
+
+// Units [c*n/nblk, (c+1)*n/nblk) of `unit` rows each.
+static void partition(int *row0, int n_units, int unit, int nblk) {
+    for (int c = 0; c <= nblk; c++) row0[c] = (int)((long long)c * n_units / nblk) * unit;
+}
+
+// Source row of logical row r of each phase (rotation pairs and gate/up pairs interleaved).
+static const uint8_t *qkv_src(const kie_config &c, const void *const *L, int r) {
+    const int D = c.head_dim, qd = c.n_heads * D, kvd = c.n_kv_heads * D;
+    const int j = r % D, dim = (j >> 1) + (j & 1) * (D >> 1);
+    const void *m;
+    int head;
+    if (r < qd) { m = L[1]; head = r / D; }
+    else if (r < qd + kvd) { m = L[2]; head = (r - qd) / D; }
+    else { m = L[3]; head = (r - qd - kvd) / D; }
+    return static_cast<const uint8_t *>(m) + ((size_t)head * D + dim) * c.d_model * 2;
+}
+
+extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, kie_engine **out) {
+    if (!out) return KIE_ERR_ARG;
+    *out = nullptr;
+    if (!cfg || !w || !w->tok_emb || !w->layers || !w->final_norm || !w->lm_head) return KIE_ERR_ARG;
+    if (shape_error(*cfg)) return KIE_ERR_ARG;
+    kie_engine *eng = new kie_engine();
+    eng->cfg = *cfg;
+    const kie_config &c = eng->cfg;
+    kie_status st = KIE_OK;
+    auto bail = [&](kie_status s) {
+        kie_destroy(eng);
+        return s;
+    };
+    if (!(c.modes & KIE_MODE_BATCH1)) {
+        delete eng;
+        return KIE_ERR_UNSUPPORTED;  // the tick kernel is built separately
+    }
+    cudaError_t e = cudaSetDevice(c.device);
+    if (e != cudaSuccess) return bail(eng->cuda_fail(e, "cudaSetDevice"));
+    int sms = 0, coop = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, c.device);
+    cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, c.device);
+    if (!coop || sms <= 0 || sms > KIE_MAX_CTAS) {
+        eng->fail(KIE_ERR_CUDA, "device lacks cooperative launch");
+        return bail(KIE_ERR_CUDA);
+    }
+    e = kie_b1_prepare(c.dtype);
+    if (e != cudaSuccess) return bail(eng->cuda_fail(e, "kernel attributes"));
+    int occ = 0;
+    e = kie_b1_occupancy(c.dtype, &occ);
+    if (e != cudaSuccess || occ < 1) return bail(eng->cuda_fail(e == cudaSuccess ? cudaErrorInvalidConfiguration : e,
+                                                                "megakernel does not fit on an SM"));
+    const int nblk = sms;
+    eng->nblk = nblk;
+    const int L = c.n_layers, d = c.d_model, D = c.head_dim, Hq = c.n_heads, Hkv = c.n_kv_heads, F = c.ffn,
+              V = c.vocab;
+    const int G = Hq / Hkv, qd = Hq * D, kvd = Hkv * D;
+    KieParams &P = eng->P;
+    P.L = L; P.d = d; P.Hq = Hq; P.Hkv = Hkv; P.D = D; P.F = F; P.V = V; P.dtype = c.dtype; P.G = G;
+    P.eps = c.rms_eps;
+    P.max_ctx = c.max_ctx;
+    P.max_sessions = c.max_sessions;
+    P.nblk = nblk;
+    P.timeout_ns = (long long)c.timeout_ms * 1000000ll;
+    P.idle_ns = (long long)c.idle_ms * 1000000ll;
+
+    // ---- the static schedule: row partition per phase
+    const int Kph[KIE_NPH] = {d, qd, d, F, d};
+    std::vector<int> row0((size_t)KIE_NPH * (nblk + 1));
+    partition(&row0[PH_QKV * (nblk + 1)], (qd + 2 * kvd) / 2, 2, nblk);
+    partition(&row0[PH_O * (nblk + 1)], d, 1, nblk);
+    partition(&row0[PH_GU * (nblk + 1)], F, 2, nblk);
+    partition(&row0[PH_DOWN * (nblk + 1)], d, 1, nblk);
+    partition(&row0[PH_HEAD * (nblk + 1)], V, 1, nblk);
+    for (int ph = 0; ph < KIE_NPH; ph++) {
+        P.K[ph] = Kph[ph];
+        const int nv = kie_b1_vec_per_lane(Kph[ph]);
+        P.cr[ph] = nv == 1 ? 8 : nv == 2 ? 4 : nv == 4 ? 2 : 1;
+        if ((ph == PH_QKV || ph == PH_GU) && P.cr[ph] < 2) {
+            eng->fail(KIE_ERR_ARG, "paired rows need two rows per chunk");
+            return bail(KIE_ERR_ARG);
+        }
+        for (int cc = 0; cc < nblk; cc++)
+            if (row0[ph * (nblk + 1) + cc + 1] - row0[ph * (nblk + 1) + cc] > KIE_ROWACC_MAX) {
+                eng->fail(KIE_ERR_ARG, "phase %d gives a CTA more than %d rows", ph, KIE_ROWACC_MAX);
+                return bail(KIE_ERR_ARG);
+            }
+    }
+    // attention splits: about one unit per CTA, and no split longer than the score buffer
+    {
+        int s = std::max(1, nblk / Hkv);
+        const int cap = KIE_SCORE_MAX / G;
+        s = std::max(s, (c.max_ctx + cap - 1) / cap);
+        P.splits = s;
+    }
+
+    // ---- packed weights: CTA c's stream is one contiguous segment
+    std::vector<long long> seg_off(nblk + 1, 0);
+    for (int cc = 0; cc < nblk; cc++) {
+        long long lb = 0;
+        for (int ph = 0; ph < PH_HEAD; ph++)
+            lb += (long long)(row0[ph * (nblk + 1) + cc + 1] - row0[ph * (nblk + 1) + cc]) * Kph[ph] * 2;
+        const long long hb = (long long)(row0[PH_HEAD * (nblk + 1) + cc + 1] - row0[PH_HEAD * (nblk + 1) + cc]) * d * 2;
+        seg_off[cc + 1] = seg_off[cc] + (long long)L * lb + hb;
+    }
+    uint8_t *wpack = nullptr;
+    CK(eng->alloc(&wpack, (size_t)seg_off[nblk]), "cudaMalloc packed weights");
+    P.wpack = wpack;
+    {
+        std::vector<RowCopy> rc;
+        rc.reserve((size_t)L * (qd + 2 * kvd + d + 2 * F + d) + V);
+        for (int cc = 0; cc < nblk; cc++) {
+            long long off = seg_off[cc];
+            for (int l = 0; l <= L; l++) {
+                const void *const *Lw = w->layers + (size_t)9 * (l < L ? l : 0);
+                for (int ph = (l < L ? 0 : PH_HEAD); ph < (l < L ? PH_HEAD : KIE_NPH); ph++) {
+                    const int K = Kph[ph];
+                    for (int r = row0[ph * (nblk + 1) + cc]; r < row0[ph * (nblk + 1) + cc + 1]; r++) {
+                        const uint8_t *src;
+                        switch (ph) {
+                            case PH_QKV: src = qkv_src(c, Lw, r); break;
+                            case PH_O: src = static_cast<const uint8_t *>(Lw[4]) + (size_t)r * K * 2; break;
+                            case PH_GU: src = static_cast<const uint8_t *>(Lw[(r & 1) ? 7 : 6]) + (size_t)(r >> 1) * K * 2; break;
+                            case PH_DOWN: src = static_cast<const uint8_t *>(Lw[8]) + (size_t)r * K * 2; break;
+                            default: src = static_cast<const uint8_t *>(w->lm_head) + (size_t)r * K * 2; break;
+                        }
+                        rc.push_back({off, src, (long long)K * 2});
+                        off += (long long)K * 2;
+                    }
+                }
+            }
+            if (off != seg_off[cc + 1]) {
+                eng->fail(KIE_ERR_ARG, "internal: segment size mismatch");
+                return bail(KIE_ERR_ARG);
+            }
+        }
+        RowCopy *d_rc = nullptr;
+        CK(cudaMalloc(&d_rc, rc.size() * sizeof(RowCopy)), "cudaMalloc repack list");
+        e = cudaMemcpy(d_rc, rc.data(), rc.size() * sizeof(RowCopy), cudaMemcpyHostToDevice);
+        if (e == cudaSuccess) {
+            gather_rows_kernel<<<4 * nblk, 256>>>(d_rc, (long long)rc.size(), wpack);
+            e = cudaGetLastError();
+        }
+        if (e == cudaSuccess) e = cudaDeviceSynchronize();
+        cudaFree(d_rc);
+        if (e != cudaSuccess) return bail(eng->cuda_fail(e, "weight repack"));
+    }
+    int *d_row0 = nullptr;
+    long long *d_seg = nullptr;
+    CK(eng->alloc(&d_row0, row0.size() * sizeof(int)), "cudaMalloc plan");
+    CK(eng->alloc(&d_seg, seg_off.size() * sizeof(long long)), "cudaMalloc plan");
+    CK(cudaMemcpy(d_row0, row0.data(), row0.size() * sizeof(int), cudaMemcpyHostToDevice), "upload plan");
+    CK(cudaMemcpy(d_seg, seg_off.data(), seg_off.size() * sizeof(long long), cudaMemcpyHostToDevice), "upload plan");
+    P.row0 = d_row0;
+    P.seg_off = d_seg;
+
+    // ---- small weights: embedding table and norm gains
+    uint16_t *emb = nullptr, *gains = nullptr;
+    CK(eng->alloc(&emb, (size_t)V * d * 2), "cudaMalloc embedding");
+    CK(cudaMemcpy(emb, w->tok_emb, (size_t)V * d * 2, cudaMemcpyDeviceToDevice), "copy embedding");
+    CK(eng->alloc(&gains, (size_t)(2 * L + 1) * d * 2), "cudaMalloc gains");
+    for (int l = 0; l < L; l++) {
+        CK(cudaMemcpy(gains + (size_t)(2 * l) * d, w->layers[9 * l + 0], (size_t)d * 2, cudaMemcpyDeviceToDevice), "gains");
+        CK(cudaMemcpy(gains + (size_t)(2 * l + 1) * d, w->layers[9 * l + 5], (size_t)d * 2, cudaMemcpyDeviceToDevice), "gains");
+    }
+    CK(cudaMemcpy(gains + (size_t)(2 * L) * d, w->final_norm, (size_t)d * 2, cudaMemcpyDeviceToDevice), "gains");
+    P.emb = emb;
+    P.gains = gains;
+
+    // ---- rotary table, computed in double on the host
+    {
+        std::vector<float2> rope((size_t)c.max_ctx * (D / 2));
+        for (int p = 0; p < c.max_ctx; p++)
+            for (int i = 0; i < D / 2; i++) {
+                const double ang = (double)p * std::pow((double)c.rope_theta, -2.0 * i / D);
+                rope[(size_t)p * (D / 2) + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+            }
+        float2 *d_rope = nullptr;
+        CK(eng->alloc(&d_rope, rope.size() * sizeof(float2)), "cudaMalloc rope");
+        CK(cudaMemcpy(d_rope, rope.data(), rope.size() * sizeof(float2), cudaMemcpyHostToDevice), "upload rope");
+        P.rope = d_rope;
+    }
+
+    // ---- KV cache for every session slot
+    P.sess_stride = (long long)L * Hkv * c.max_ctx * D;
+    CK(eng->alloc(&P.kcache, (size_t)c.max_sessions * P.sess_stride * 2), "cudaMalloc K cache");
+    CK(eng->alloc(&P.vcache, (size_t)c.max_sessions * P.sess_stride * 2), "cudaMalloc V cache");
+
+    // ---- activations and scratch
+    CK(eng->alloc(&P.x, (size_t)d * 4), "cudaMalloc x");
+    CK(eng->alloc(&P.q, (size_t)qd * 4), "cudaMalloc q");
+    CK(eng->alloc(&P.o, (size_t)qd * 4), "cudaMalloc o");
+    CK(eng->alloc(&P.u, (size_t)F * 4), "cudaMalloc u");
+    CK(eng->alloc(&P.part, (size_t)Hkv * P.splits * G * (D + 2) * 4), "cudaMalloc partials");
+    CK(eng->alloc(&P.cnt, (size_t)Hkv * 4), "cudaMalloc counters");
+    CK(eng->alloc(&P.cand_val, (size_t)nblk * 4), "cudaMalloc candidates");
+    CK(eng->alloc(&P.cand_idx, (size_t)nblk * 4), "cudaMalloc candidates");
+    CK(eng->alloc(&P.tokbuf, (size_t)c.max_ctx * 4), "cudaMalloc token buffer");
+    CK(eng->alloc(&P.bar, 16), "cudaMalloc barrier");
+    CK(eng->alloc(&P.err, 16), "cudaMalloc error word");
+    CK(eng->alloc(&P.last_seq, 16), "cudaMalloc sequence");
+    CK(eng->alloc(&P.cmd, sizeof(KieCmd)), "cudaMalloc command");
+    CK(cudaMemset(P.cnt, 0, (size_t)Hkv * 4), "memset");
+    CK(cudaMemset(P.bar, 0, 16), "memset");
+    CK(cudaMemset(P.err, 0, 16), "memset");
+    CK(cudaMemset(P.last_seq, 0, 16), "memset");
+    CK(cudaMemset(P.x, 0, (size_t)d * 4), "memset");
+
+    // ---- the doorbell: mapped, pinned host memory
+    eng->io_ints = 2 * (int64_t)c.max_ctx + 64 * 64 + 64;
+    const size_t mb_bytes = sizeof(KieMailbox) + (size_t)eng->io_ints * 4;
+    CK(cudaHostAlloc((void **)&eng->mbox_host, mb_bytes, cudaHostAllocMapped | cudaHostAllocPortable), "cudaHostAlloc mailbox");
+    memset(eng->mbox_host, 0, mb_bytes);
+    CK(cudaHostGetDevicePointer((void **)&eng->mbox_dev, eng->mbox_host, 0), "mailbox device alias");
+    P.mbox = eng->mbox_dev;
+
+    CK(cudaStreamCreateWithFlags(&eng->stream, cudaStreamNonBlocking), "cudaStreamCreate");
+    CK(cudaEventCreateWithFlags(&eng->ev_done, cudaEventDisableTiming), "cudaEventCreate");
+    CK(cudaDeviceSynchronize(), "create");
+    eng->sess_len.assign(c.max_sessions, 0);
+    eng->sess_used.assign(c.max_sessions, 0);
+    (void)st;
+    *out = eng;
+    return KIE_OK;
+}
+
+// ---------------------------------------------------------------- resident kernel control
+
+static bool kernel_running(kie_engine *eng) {
+    if (eng->resident == KIND_NONE) return false;
+    const cudaError_t q = cudaEventQuery(eng->ev_done);
+    if (q == cudaErrorNotReady) return true;
+    eng->resident = KIND_NONE;
+    return false;
+}
+
+static kie_status check_device_error(kie_engine *eng) {
+    unsigned err = 0;
+    cudaError_t e = cudaMemcpy(&err, eng->P.err, 4, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return eng->fail(KIE_ERR_DEVICE, "reading device status: %s", cudaGetErrorString(e));
+    if (err) {
+        const unsigned code = err >> 8, where = err & 0xFF;
+        const char *what = code == DERR_BARRIER_TIMEOUT ? "grid barrier timed out"
+                           : code == DERR_RING_TIMEOUT  ? "weight ring wait timed out"
+                           : code == DERR_BAD_TOKEN     ? "token id out of range"
+                           : code == DERR_MMA_TIMEOUT   ? "tensor-core wait timed out"
+                                                        : "unknown device error";
+        return eng->fail(code == DERR_BARRIER_TIMEOUT || code == DERR_RING_TIMEOUT || code == DERR_MMA_TIMEOUT
+                             ? KIE_ERR_TIMEOUT
+                             : KIE_ERR_DEVICE,
+                         "device: %s (phase %u)", what, where);
+    }
+    return KIE_OK;
+}
+
+static kie_status launch_resident(kie_engine *eng, int kind) {
+    cudaError_t e = cudaMemsetAsync(eng->P.bar, 0, 16, eng->stream);
+    if (e == cudaSuccess) {
+        KieCmd none{};
+        e = kie_b1_launch(eng->P, none, 1, eng->stream);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(eng->ev_done, eng->stream);
+    if (e != cudaSuccess) return eng->cuda_fail(e, "launching the resident kernel");
+    eng->resident = kind;
+    return KIE_OK;
+}
+
+// Posts one command and waits for its completion (relaunching the kernel if it had gone idle).
+static kie_status doorbell(kie_engine *eng, const KieCmd &cmd_in, int kind) {
+    if (kernel_running(eng) && eng->resident != kind) {
+        // another kernel is resident: ask it to leave first (handled by the caller's kind switch)
+    }
+    if (!kernel_running(eng)) {
+        kie_status s = launch_resident(eng, kind);
+        if (s != KIE_OK) return s;
+    }
+    KieMailbox *mb = eng->mbox_host;
+    const uint32_t s = ++eng->seq;
+    KieCmd cmd = cmd_in;
+    cmd.seq = s;
+    memcpy((void *)&mb->cmd, &cmd, sizeof cmd);
+    std::atomic_thread_fence(std::memory_order_release);
+    mb->cmd_seq = s;
+    const double t0 = now_s(), limit = eng->cfg.timeout_ms * 1e-3 + (cmd.op == OP_EXIT ? 0.0 : 0.0);
+    unsigned spins = 0;
+    for (;;) {
+        if (mb->done_seq == s) break;
+        if ((++spins & 1023u) == 0) {
+            if (!kernel_running(eng)) {
+                std::atomic_thread_fence(std::memory_order_acquire);
+                if (mb->done_seq == s) break;
+                const kie_status ds = check_device_error(eng);
+                if (ds != KIE_OK) return ds;
+                const cudaError_t le = cudaGetLastError();
+                if (le != cudaSuccess) return eng->fail(KIE_ERR_DEVICE, "resident kernel: %s", cudaGetErrorString(le));
+                if (cmd.op == OP_EXIT) break;
+                kie_status ls = launch_resident(eng, kind);  // it went idle before taking the command
+                if (ls != KIE_OK) return ls;
+            }
+            // the time limit scales with the work of the command
+            const double budget = limit * (1.0 + (cmd.n > 0 ? cmd.n / 64.0 : 0.0));
+            if (now_s() - t0 > budget) {
+                return eng->fail(KIE_ERR_TIMEOUT, "no answer from the device after %.1f s", now_s() - t0);
+            }
+        } else {
+            _mm_pause();
+        }
+    }
+    std::atomic_thread_fence(std::memory_order_acquire);
+    if (mb->status != 0) {
+        const kie_status ds = check_device_error(eng);
+        return ds != KIE_OK ? ds : eng->fail(KIE_ERR_DEVICE, "device reported a failed command");
+    }
+    return KIE_OK;
+}
+
+static kie_status stop_resident(kie_engine *eng) {
+    if (!kernel_running(eng)) return KIE_OK;
+    KieCmd ex{};
+    ex.op = OP_EXIT;
+    kie_status s = doorbell(eng, ex, eng->resident);
+    const double t0 = now_s();
+    while (kernel_running(eng)) {
+        if (now_s() - t0 > eng->cfg.timeout_ms * 1e-3) return eng->fail(KIE_ERR_TIMEOUT, "resident kernel did not stop");
+    }
+    return s;
+}
+
+extern "C" void kie_destroy(kie_engine *eng) {
+    if (!eng) return;
+    if (!eng->poisoned && eng->stream) stop_resident(eng);
+    if (eng->stream) cudaStreamSynchronize(eng->stream);
+    for (void *p : eng->dev_allocs) cudaFree(p);
+    if (eng->mbox_host) cudaFreeHost(eng->mbox_host);
+    if (eng->ev_done) cudaEventDestroy(eng->ev_done);
+    if (eng->stream) cudaStreamDestroy(eng->stream);
+    delete eng;
+}
+
+// ---------------------------------------------------------------- sessions
+
+static kie_status check_live(kie_engine *eng) {
+    if (!eng) return KIE_ERR_ARG;
+    if (eng->poisoned) return KIE_ERR_STATE;
+    return KIE_OK;
+}
+
+static kie_status check_sid(kie_engine *eng, int32_t sid) {
+    if (sid < 0 || sid >= eng->cfg.max_sessions || !eng->sess_used[sid])
+        return eng->fail(KIE_ERR_ARG, "session %d is not open", sid);
+    return KIE_OK;
+}
+
+extern "C" kie_status kie_session_open(kie_engine *eng, int32_t *sid) {
+    kie_status s = check_live(eng);
+    if (s != KIE_OK) return s;
+    if (!sid) return KIE_ERR_ARG;
+    for (int i = 0; i < eng->cfg.max_sessions; i++)
+        if (!eng->sess_used[i]) {
+            eng->sess_used[i] = 1;
+            eng->sess_len[i] = 0;
+            *sid = i;
+            return KIE_OK;
+        }
+    return eng->fail(KIE_ERR_CAPACITY, "all %d session slots are open", eng->cfg.max_sessions);
+}
+
+extern "C" kie_status kie_session_close(kie_engine *eng, int32_t sid) {
+    kie_status s = check_live(eng);
+    if (s != KIE_OK) return s;
+    if ((s = check_sid(eng, sid)) != KIE_OK) return s;
+    eng->sess_used[sid] = 0;
+    eng->sess_len[sid] = 0;
+    return KIE_OK;
+}
+
+extern "C" kie_status kie_session_length(kie_engine *eng, int32_t sid, int32_t *ctx) {
+    if (!eng || !ctx) return KIE_ERR_ARG;
+    kie_status s = check_sid(eng, sid);
+    if (s != KIE_OK) return s;
+    *ctx = eng->sess_len[sid];
+    return KIE_OK;
+}
+
+extern "C" kie_status kie_session_rewind(kie_engine *eng, int32_t sid, int32_t ctx) {
+    kie_status s = check_live(eng);
+    if (s != KIE_OK) return s;
+    if ((s = check_sid(eng, sid)) != KIE_OK) return s;
+    if (ctx < 0 || ctx > eng->sess_len[sid]) return eng->fail(KIE_ERR_ARG, "rewind past the current length");
+    eng->sess_len[sid] = ctx;
+    return KIE_OK;
+}
+
+extern "C" kie_status kie_session_kv(kie_engine *eng, int32_t sid, void **k_dev, void **v_dev) {
+    if (!eng || !k_dev || !v_dev) return KIE_ERR_ARG;
+    kie_status s = check_sid(eng, sid);
+    if (s != KIE_OK) return s;
+    *k_dev = eng->P.kcache + (size_t)sid * eng->P.sess_stride;
+    *v_dev = eng->P.vcache + (size_t)sid * eng->P.sess_stride;
+    return KIE_OK;
+}
+
+// ---------------------------------------------------------------- decode calls
+
+static kie_status ensure_kind(kie_engine *eng, int kind) {
+    if (kernel_running(eng) && eng->resident != kind) return stop_resident(eng);
+    return KIE_OK;
+}
+
+static kie_status check_tokens(kie_engine *eng, const int32_t *t, int n) {
+    for (int i = 0; i < n; i++)
+        if (t[i] < 0 || t[i] >= eng->cfg.vocab) return eng->fail(KIE_ERR_ARG, "token %d out of range", t[i]);
+    return KIE_OK;
+}
+
+static int32_t *io_dev(kie_engine *eng, int64_t at) { return eng->mbox_dev->io + at; }
+
+extern "C" kie_status kie_prefill(kie_engine *eng, int32_t sid, const int32_t *tokens, int32_t n, int32_t *first_token) {
+    kie_status s = check_live(eng);
+    if (s != KIE_OK) return s;
+    if (!tokens || !first_token || n <= 0) return eng->fail(KIE_ERR_ARG, "prefill needs n >= 1 tokens");
+    if ((s = check_sid(eng, sid)) != KIE_OK) return s;
+    if ((s = check_tokens(eng, tokens, n)) != KIE_OK) return s;
+    const int ctx = eng->sess_len[sid];
+    if ((int64_t)ctx + n > eng->cfg.max_ctx) return eng->fail(KIE_ERR_CAPACITY, "prefill of %d at %d exceeds max_ctx", n, ctx);
+    if ((s = ensure_kind(eng, KIND_B1)) != KIE_OK) return s;
+    memcpy(eng->mbox_host->io, tokens, (size_t)n * 4);
+    KieCmd cmd{};
+    cmd.op = OP_PREFILL;
+    cmd.sid = sid;
+    cmd.pos0 = ctx;
+    cmd.n = n;
+    cmd.tokens = io_dev(eng, 0);
+    cmd.out = io_dev(eng, eng->cfg.max_ctx);
+    s = doorbell(eng, cmd, KIND_B1);
+    if (s != KIE_OK) return s;
+    *first_token = ((volatile int32_t *)eng->mbox_host->io)[eng->cfg.max_ctx];
+    eng->sess_len[sid] = ctx + n;
+    return KIE_OK;
+}
+
+static kie_status decode_doorbell(kie_engine *eng, int32_t sid, int32_t in_token, int32_t n, int32_t *out,
+                                  float *logits_dev) {
+    kie_status s = check_live(eng);
+    if (s != KIE_OK) return s;
+    if (!out || n <= 0) return eng->fail(KIE_ERR_ARG, "need n >= 1 and an output buffer");
+    if ((s = check_sid(eng, sid)) != KIE_OK) return s;
+    if ((s = check_tokens(eng, &in_token, 1)) != KIE_OK) return s;
+    const int ctx = eng->sess_len[sid];
+    if ((int64_t)ctx + n > eng->cfg.max_ctx) return eng->fail(KIE_ERR_CAPACITY, "%d steps at %d exceed max_ctx", n, ctx);
+    if ((int64_t)n > eng->io_ints - eng->cfg.max_ctx) return eng->fail(KIE_ERR_ARG, "n too large for the mailbox");
+    if ((s = ensure_kind(eng, KIND_B1)) != KIE_OK) return s;
+    KieCmd cmd{};
+    cmd.op = OP_DECODE;
+    cmd.sid = sid;
+    cmd.pos0 = ctx;
+    cmd.n = n;
+    cmd.in_tok = in_token;
+    cmd.out = io_dev(eng, eng->cfg.max_ctx);
+    cmd.logits = logits_dev;
+    s = doorbell(eng, cmd, KIND_B1);
+    if (s != KIE_OK) return s;
+    const volatile int32_t *io = eng->mbox_host->io + eng->cfg.max_ctx;
+    for (int i = 0; i < n; i++) out[i] = io[i];
+    eng->sess_len[sid] = ctx + n;
+    return KIE_OK;
+}
+
+extern "C" kie_status kie_decode_step(kie_engine *eng, int32_t sid, int32_t in_token, int32_t *out_token,
+                                      float *logits_dev) {
+    return decode_doorbell(eng, sid, in_token, 1, out_token, logits_dev);
+}
+
+extern "C" kie_status kie_generate(kie_engine *eng, int32_t sid, int32_t in_token, int32_t n, int32_t *out_tokens) {
+    return decode_doorbell(eng, sid, in_token, n, out_tokens, nullptr);
+}
+
+extern "C" kie_status kie_decode_launch(kie_engine *eng, int32_t sid, const int32_t *in_token_dev, int32_t n,
+                                        int32_t *out_tokens_dev, float *logits_dev, void *stream) {
+    kie_status s = check_live(eng);
+    if (s != KIE_OK) return s;
+    if (!in_token_dev || !out_tokens_dev || n <= 0) return eng->fail(KIE_ERR_ARG, "launch needs device buffers and n >= 1");
+    if ((s = check_sid(eng, sid)) != KIE_OK) return s;
+    const int ctx = eng->sess_len[sid];
+    if ((int64_t)ctx + n > eng->cfg.max_ctx) return eng->fail(KIE_ERR_CAPACITY, "%d steps at %d exceed max_ctx", n, ctx);
+    if ((s = stop_resident(eng)) != KIE_OK) return s;
+    cudaStream_t st = stream ? static_cast<cudaStream_t>(stream) : eng->stream;
+    KieCmd cmd{};
+    cmd.op = OP_DECODE;
+    cmd.sid = sid;
+    cmd.pos0 = ctx;
+    cmd.n = n;
+    cmd.tok_dev = in_token_dev;
+    cmd.out = out_tokens_dev;
+    cmd.logits = logits_dev;
+    cudaError_t e = cudaMemsetAsync(eng->P.bar, 0, 16, st);
+    if (e == cudaSuccess) e = kie_b1_launch(eng->P, cmd, 0, st);
+    if (e != cudaSuccess) return eng->cuda_fail(e, "launching the decode kernel");
+    eng->sess_len[sid] = ctx + n;
+    return KIE_OK;
+}
+
+extern "C" kie_status kie_sync(kie_engine *eng) {
+    kie_status s = check_live(eng);
+    if (s != KIE_OK) return s;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return eng->fail(KIE_ERR_DEVICE, "kernel failed: %s", cudaGetErrorString(e));
+    return check_device_error(eng);
+}
+
+extern "C" kie_status kie_tick(kie_engine *eng, int32_t n_sess, const int32_t *sids, const int32_t *in_tokens,
+                               int32_t steps, int32_t *out_tokens, float *logits_dev) {
+    kie_status s = check_live(eng);
+    if (s != KIE_OK) return s;
+    (void)n_sess; (void)sids; (void)in_tokens; (void)steps; (void)out_tokens; (void)logits_dev;
+    if (!(eng->cfg.modes & KIE_MODE_TICK)) return eng->fail(KIE_ERR_UNSUPPORTED, "engine built without KIE_MODE_TICK");
+    return KIE_ERR_UNSUPPORTED;
+}

@@ -1,0 +1,93 @@
+// Internal definitions shared by the engine's host code and its kernels.
+#pragma once
+#include <stdint.h>
+
+#include "kie.h"
+
+#define KIE_MAX_CTAS 256
+#define KIE_CONS_WARPS 8                      // consumer warps per CTA (batch-1 kernel)
+#define KIE_CONS_THREADS (KIE_CONS_WARPS * 32)
+#define KIE_THREADS (KIE_CONS_THREADS + 32)   // + one producer warp
+#define KIE_NSLOT 6                           // weight ring depth
+#define KIE_SLOT_BYTES 32768                  // one ring slot
+#define KIE_ROWACC_MAX 1024                   // output rows one CTA may own in one phase
+#define KIE_SCORE_MAX 4096                    // attention scores one split may hold (floats)
+#define KIE_GMAX 8                            // query heads per kv head
+#define KIE_DMAX 128                          // head_dim
+
+// Phases of the batch-1 weight stream, in stream order within a layer; the LM head follows the last layer.
+enum { PH_QKV = 0, PH_O = 1, PH_GU = 2, PH_DOWN = 3, PH_HEAD = 4, KIE_NPH = 5 };
+
+// Commands of the resident kernel.
+enum { OP_NONE = 0, OP_DECODE = 1, OP_PREFILL = 2, OP_TICK = 3, OP_EXIT = 4 };
+
+// Device error codes (err word = code << 8 | where).
+enum { DERR_BARRIER_TIMEOUT = 1, DERR_RING_TIMEOUT = 2, DERR_BAD_TOKEN = 3, DERR_MMA_TIMEOUT = 4 };
+
+struct KieCmd {
+    int32_t op, sid, pos0, n;
+    int32_t in_tok;          // first input token of OP_DECODE
+    int32_t n_sess;          // OP_TICK: sessions in the tick; OP_PREFILL on the tick kernel: rows
+    uint32_t seq;            // doorbell sequence number
+    int32_t flags;
+    const int32_t *tokens;   // OP_PREFILL: input tokens [n] (device); OP_TICK: first inputs [n_sess]
+    const int32_t *tok_dev;  // OP_DECODE via launch: device pointer to the first input token
+    int32_t *out;            // output tokens (device memory or the mapped mailbox)
+    float *logits;           // optional logits
+    const int32_t *sids;     // OP_TICK: session ids [n_sess] (device)
+    const int32_t *pos;      // OP_TICK: start positions [n_sess] (device)
+};
+
+// Host-mapped doorbell. The host writes `cmd`, then `cmd_seq`; the kernel writes the
+// outputs, then `done_seq`.
+struct KieMailbox {
+    volatile uint32_t cmd_seq;
+    uint32_t pad0[31];
+    KieCmd cmd;
+    uint32_t pad1[32 - (sizeof(KieCmd) / 4) % 32];
+    volatile uint32_t done_seq;
+    volatile int32_t status;
+    uint32_t pad2[30];
+    int32_t io[1];           // inputs then outputs (sized at allocation)
+};
+
+// Everything a kernel needs; passed by value.
+struct KieParams {
+    int L, d, Hq, Hkv, D, F, V, dtype, G;
+    float eps;
+    int max_ctx, max_sessions, nblk;
+    int splits;                     // attention splits per kv head (batch-1)
+    int cr[KIE_NPH];                // rows per ring chunk, per phase
+    int K[KIE_NPH];                 // row length (elements) per phase
+    // batch-1 packed weights: CTA c streams [seg_off[c], seg_off[c+1]) once per token
+    const uint8_t *wpack;
+    const int *row0;                // [KIE_NPH][nblk+1] logical row partition
+    const long long *seg_off;       // [nblk+1]
+    // unpacked small weights
+    const uint16_t *emb;            // [V][d]
+    const uint16_t *gains;          // [2L+1][d]: attn_norm l, mlp_norm l, final
+    const float2 *rope;             // [max_ctx][D/2] (cos, sin)
+    // KV cache [sessions][L][Hkv][max_ctx][D]
+    uint16_t *kcache, *vcache;
+    long long sess_stride;
+    // activations and scratch
+    float *x, *q, *o, *u;
+    float *part;                    // [Hkv*splits*G][D+2]
+    unsigned *cnt;                  // [Hkv]
+    float *cand_val;
+    int *cand_idx;                  // [nblk]
+    int *tokbuf;                    // [max_ctx] device copy of command inputs
+    unsigned long long *bar;        // grid barrier counter
+    unsigned *err;                  // first device error
+    KieMailbox *mbox;               // device alias of the mapped mailbox
+    unsigned *last_seq;             // last doorbell sequence processed
+    KieCmd *cmd;                    // command broadcast slot
+    long long timeout_ns, idle_ns;
+};
+
+#ifdef __cplusplus
+extern "C++" {
+// kernels (defined in kie_b1.cu / kie_mr.cu)
+struct KieMrParams;
+}
+#endif

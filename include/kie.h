@@ -1,0 +1,189 @@
+/*
+ * kie.h — C ABI of the B200 decode engine (libkie.so).
+ *
+ * The engine runs the autoregressive decode step of a dense decoder-only transformer
+ * (pre-norm RMSNorm, rotary positions, grouped-query attention, SwiGLU MLP, untied LM
+ * head, greedy argmax) as one persistent sm_100a kernel per GPU:
+ *
+ *  - Every weight byte and the KV cache are streamed once per generated token; decode is
+ *    bound by memory bandwidth, not compute ("Kog 3000 tok/s 实时推理：内存带宽优化与请求级并发的
+ *    工程权衡", section 内存带宽优化的三层策略; the HN digest of Kog's inference engine,
+ *    section 技术原理, "内存带宽是关键瓶颈").
+ *  - One resident kernel replaces per-op launches (the same digest, 技术原理, 持久化单内核运行时;
+ *    "实时AI推理为何贵56倍？持续推理与常驻内核的破局之道", section 让工作常驻 GPU). The host only
+ *    writes input tokens into a mapped mailbox (the doorbell) and reads output tokens.
+ *  - Sessions due on the same tick advance as one batch, so the weights are read once for
+ *    the whole group (same page, section 让所有活跃会话同步推进): kie_tick.
+ *  - Schedule and memory layout are fixed at kie_create, with no allocator or scheduler
+ *    afterwards (same page, section 把一切提前决定好).
+ *
+ * Conventions for every call:
+ *  - Return KIE_OK (0) or a negative kie_status. No call aborts the process.
+ *  - After KIE_ERR_TIMEOUT or KIE_ERR_DEVICE the engine is poisoned: every later call
+ *    except kie_last_error / kie_destroy returns KIE_ERR_STATE.
+ *  - One host thread per engine; calls on one engine must not overlap.
+ *  - "host" pointers are ordinary CPU memory; "device" pointers are CUDA device memory
+ *    on the engine's device.
+ */
+#ifndef KIE_H
+#define KIE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KIE_ABI_VERSION 1
+
+typedef struct kie_engine kie_engine; /* opaque; owned by the library */
+typedef int32_t kie_status;
+
+enum {
+    KIE_OK = 0,
+    KIE_ERR_ARG = -1,         /* bad argument or unsupported shape                          */
+    KIE_ERR_CAPACITY = -2,    /* context or session capacity exceeded; nothing was written */
+    KIE_ERR_CUDA = -3,        /* a CUDA runtime call failed (message in kie_last_error)    */
+    KIE_ERR_TIMEOUT = -4,     /* a host or device wait ran past timeout_ms                 */
+    KIE_ERR_STATE = -5,       /* engine poisoned by an earlier timeout / device error      */
+    KIE_ERR_DEVICE = -6,      /* the kernel reported an error status                       */
+    KIE_ERR_UNSUPPORTED = -7  /* the engine was created without the mode this call needs  */
+};
+
+enum { KIE_FP16 = 0, KIE_BF16 = 1 };
+
+/* Which kernels and weight layouts kie_create builds (bitmask). */
+enum {
+    KIE_MODE_BATCH1 = 1, /* single-session decode: kie_decode_step / kie_generate / kie_decode_launch */
+    KIE_MODE_TICK = 2    /* multi-session tick and chunked prefill on tcgen05 tensor cores            */
+};
+
+typedef struct {
+    int32_t n_layers, d_model, n_heads, n_kv_heads, head_dim, ffn, vocab;
+    float rms_eps;    /* RMSNorm epsilon (1e-5 in all shipped configs)                 */
+    float rope_theta; /* rotary base (1e4, or 5e5 for the Llama-3-8B shape)            */
+    int32_t dtype;    /* KIE_FP16 or KIE_BF16: weights and KV cache                    */
+    int32_t max_sessions; /* KV slots allocated up front                               */
+    int32_t max_ctx;      /* positions per session allocated up front                  */
+    int32_t timeout_ms;   /* bound on every device spin and host wait of one command   */
+    int32_t idle_ms;      /* the resident kernel exits after this long with no command */
+    int32_t modes;        /* KIE_MODE_* bitmask                                        */
+    int32_t device;       /* CUDA device ordinal                                       */
+} kie_config;
+
+/*
+ * Weights, all DEVICE pointers in row-major [out][in] layout of the storage dtype:
+ *   tok_emb [vocab][d_model], final_norm [d_model], lm_head [vocab][d_model],
+ *   layers[9*l + j] for layer l, j in order: attn_norm [d], wq [Hq*D][d], wk [Hkv*D][d],
+ *   wv [Hkv*D][d], wo [d][Hq*D], mlp_norm [d], w_gate [ffn][d], w_up [ffn][d], w_down [d][ffn].
+ * `layers` itself is a HOST array of 9*n_layers device pointers.
+ * The engine reads them only inside kie_create (it repacks them into its own arena in the
+ * streaming order of its fixed schedule); the caller may free them afterwards.
+ */
+typedef struct {
+    const void *tok_emb;
+    const void *const *layers;
+    const void *final_norm;
+    const void *lm_head;
+} kie_weights;
+
+/* Fills a config with the shape fields zeroed and defaults for the rest
+   (eps 1e-5, theta 1e4, fp16, 1 session, 4096 positions, timeouts 10 s / 200 ms,
+   batch-1 mode, device 0). */
+void kie_config_defaults(kie_config *cfg);
+
+/*
+ * Builds an engine: validates the shape, allocates every device buffer it will ever use
+ * (packed weights, KV cache of max_sessions x max_ctx, activations, split-K scratch,
+ * mapped host mailbox), computes the static work partition for this GPU's SM count and
+ * repacks the weights. Constraints: d_model, n_heads*head_dim and ffn multiples of 64;
+ * head_dim even and <= 128; n_heads a multiple of n_kv_heads with n_heads/n_kv_heads <= 8.
+ * Errors: KIE_ERR_ARG (shape), KIE_ERR_CUDA (allocation or launch). On error *out is NULL.
+ */
+kie_status kie_create(const kie_config *cfg, const kie_weights *w, kie_engine **out);
+
+/* Stops the resident kernel (if running) and frees everything. NULL is ignored. */
+void kie_destroy(kie_engine *eng);
+
+/* Claims a free KV slot with context length 0. KIE_ERR_CAPACITY when all are taken. */
+kie_status kie_session_open(kie_engine *eng, int32_t *sid);
+kie_status kie_session_close(kie_engine *eng, int32_t sid);
+/* Current context length (tokens in the cache) of a session. */
+kie_status kie_session_length(kie_engine *eng, int32_t sid, int32_t *ctx);
+/* Rewinds a session to its first `ctx` positions (ctx <= current length); later steps overwrite the rest. */
+kie_status kie_session_rewind(kie_engine *eng, int32_t sid, int32_t ctx);
+/* DEVICE pointers to the session's K and V cache, each [n_layers][n_kv_heads][max_ctx][head_dim]
+   of the storage dtype. Owned by the engine; valid until kie_destroy. */
+kie_status kie_session_kv(kie_engine *eng, int32_t sid, void **k_dev, void **v_dev);
+
+/*
+ * Appends a prompt: tokens (HOST, n >= 1) are processed teacher-forced at positions
+ * ctx..ctx+n-1, and *first_token (HOST) receives the argmax after the last one.
+ * KIE_ERR_CAPACITY if ctx + n > max_ctx (nothing written). Uses the tick kernel's
+ * chunked path when the engine has KIE_MODE_TICK, else the batch-1 kernel.
+ */
+kie_status kie_prefill(kie_engine *eng, int32_t sid, const int32_t *tokens, int32_t n, int32_t *first_token);
+
+/*
+ * One decode step through the doorbell: in_token at position ctx, *out_token (HOST)
+ * receives the argmax. logits_dev (DEVICE, nullable) receives the fp32 logits [vocab].
+ */
+kie_status kie_decode_step(kie_engine *eng, int32_t sid, int32_t in_token, int32_t *out_token, float *logits_dev);
+
+/*
+ * n greedy steps through the doorbell, the argmax fed back on the GPU with no host round
+ * trip per token: out_tokens (HOST, [n]) receives each step's argmax.
+ */
+kie_status kie_generate(kie_engine *eng, int32_t sid, int32_t in_token, int32_t n, int32_t *out_tokens);
+
+/*
+ * Stream-ordered form of kie_generate: one launch of the same kernel on `stream`
+ * (a cudaStream_t; NULL = the engine's own stream), reading *in_token_dev and writing
+ * out_tokens_dev[n] and, if non-NULL, logits_dev[n][vocab] (all DEVICE). Returns after
+ * the launch is queued; the session length advances immediately. Device errors surface
+ * at the next call that synchronises (or via kie_sync).
+ */
+kie_status kie_decode_launch(kie_engine *eng, int32_t sid, const int32_t *in_token_dev, int32_t n,
+                             int32_t *out_tokens_dev, float *logits_dev, void *stream);
+
+/* Waits for queued launches and reports any device error they raised. */
+kie_status kie_sync(kie_engine *eng);
+
+/*
+ * One tick of the continuous-inference workload: the n_sess sessions sids[] (HOST)
+ * advance together by `steps` greedy tokens each, weights read once per step for all of
+ * them. in_tokens (HOST, [n_sess]) are the first inputs; step s's argmax is the input of
+ * step s+1 on the GPU. out_tokens (HOST, [steps][n_sess]) receive every argmax.
+ * logits_dev (DEVICE, nullable) receives [steps][n_sess][vocab] fp32.
+ * Needs KIE_MODE_TICK; n_sess <= 64, distinct sids.
+ */
+kie_status kie_tick(kie_engine *eng, int32_t n_sess, const int32_t *sids, const int32_t *in_tokens, int32_t steps,
+                    int32_t *out_tokens, float *logits_dev);
+
+/* Copies the engine's last error message (NUL-terminated, truncated to len). */
+kie_status kie_last_error(kie_engine *eng, char *buf, int32_t len);
+
+/* Static text of a status code. */
+const char *kie_status_string(kie_status s);
+
+/*
+ * Split-K single-query attention over a KV cache, as run inside the decode kernel
+ * (the "attention over the KV cache" part of one decode step; see the first section
+ * of this header for the passages). For query head h (kv head g = h*Hkv/Hq):
+ *   out[h] = sum_{j<n_ctx} softmax_j(q[h] . K[g][j] / sqrt(D)) V[g][j].
+ * q_dev [n_heads][head_dim] fp32; k_dev, v_dev [n_kv_heads][kv_stride][head_dim] of
+ * dtype (kv_stride >= n_ctx positions between heads); out_dev [n_heads][head_dim] fp32;
+ * scratch_dev: caller-owned DEVICE buffer of at least kie_flash_decode_scratch_bytes(...)
+ * bytes (split partials and merge counters; contents on entry are ignored).
+ * All DEVICE, stream-ordered on `stream` (cudaStream_t, NULL = legacy default stream).
+ * n_ctx >= 1, head_dim even <= 128, n_heads/n_kv_heads <= 8. Returns KIE_ERR_ARG on bad shapes.
+ */
+kie_status kie_flash_decode(const float *q_dev, const void *k_dev, const void *v_dev, int32_t n_heads,
+                            int32_t n_kv_heads, int32_t head_dim, int32_t n_ctx, int64_t kv_stride, int32_t dtype,
+                            float *out_dev, void *scratch_dev, int64_t scratch_bytes, void *stream);
+int64_t kie_flash_decode_scratch_bytes(int32_t n_heads, int32_t n_kv_heads, int32_t head_dim, int32_t n_ctx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KIE_H */

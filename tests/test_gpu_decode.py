@@ -1,0 +1,251 @@
+"""Parity of the batch-1 decode megakernel with the CPU oracle (GPU tests).
+
+Every test runs the CUDA path through the C ABI (libkie.so via the ctypes binding) and
+compares with the oracle on the same seeded inputs. Tolerances are those of
+``tests/parity.py``: logits max-abs 2e-2 (fp16) / 5e-2 (bf16) at every step, token ids
+exact wherever the oracle's top-1/top-2 margin exceeds 0.05 (teacher forcing keeps both
+sides on the oracle's sequence).
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def kie():
+    from bandwidth_bound_stream_b200 import build
+    build.build_kie()
+    from bandwidth_bound_stream_b200 import kie as k
+    return k
+
+
+def _setup(kie, model, max_ctx, seed=0, **kw):
+    from oracle.oracle import OracleModel
+    dw = kie.DeviceWeights(model, seed=seed, host_copy=True)
+    eng = kie.Engine(kie.config(model, max_ctx=max_ctx, timeout_ms=5000, idle_ms=50, **kw), dw.kie)
+    orc = OracleModel(model, dw.host, max_ctx)
+    return dw, eng, orc
+
+
+def _lockstep(kie, eng, orc, model, prompt, n_steps):
+    """Prefill then n_steps teacher-forced decode steps with logits; returns the step reports."""
+    from tests.parity import compare_step
+    V = model.vocab
+    logits = torch.empty(V, dtype=torch.float32, device="cuda")
+    sid = eng.session_open()
+    first = eng.prefill(sid, prompt)
+    ref = orc.prefill(prompt)
+    reports = [compare_step(ref, first, ref, model.dtype)]  # token only (no logits out of prefill)
+    tok = int(np.argmax(ref))
+    for _ in range(n_steps):
+        out = eng.decode_step(sid, tok, logits.data_ptr())
+        got = logits.cpu().numpy()
+        ref = orc.step(tok)
+        reports.append(compare_step(got, out, ref, model.dtype))
+        tok = int(np.argmax(ref))
+    assert eng.session_length(sid) == len(prompt) + n_steps
+    return reports
+
+
+# ------------------------------------------------------------------ attention op
+
+@pytest.mark.parametrize("Hq,Hkv,D,ctx,dtype", [
+    (4, 4, 64, 1, 0), (16, 8, 128, 7, 0), (16, 8, 128, 129, 0), (32, 8, 128, 1025, 1),
+    (6, 2, 64, 300, 1), (16, 8, 128, 5000, 0), (16, 8, 128, 32768, 0),
+])
+def test_flash_decode_op_matches_oracle(kie, Hq, Hkv, D, ctx, dtype):
+    from bandwidth_bound_stream_b200 import synth
+    from oracle import oracle as orc
+    rng = np.random.default_rng(ctx)
+    q = rng.normal(0, 1, (Hq, D))
+    stride = ctx + 3
+    K = synth.normal_u16(ctx, 0x7001, Hkv * stride * D, dtype, std=1.0).reshape(Hkv, stride, D)
+    Vv = synth.normal_u16(ctx, 0x7002, Hkv * stride * D, dtype, std=1.0).reshape(Hkv, stride, D)
+    q_d = torch.tensor(q, dtype=torch.float32, device="cuda")
+    k_d = torch.from_numpy(K.view(np.int16)).cuda()
+    v_d = torch.from_numpy(Vv.view(np.int16)).cuda()
+    out = torch.full((Hq, D), float("nan"), dtype=torch.float32, device="cuda")
+    nbytes = kie.flash_decode_scratch_bytes(Hq, Hkv, D, ctx)
+    scratch = torch.full((nbytes,), 0x55, dtype=torch.uint8, device="cuda")
+    st = kie.flash_decode(q_d.data_ptr(), k_d.data_ptr(), v_d.data_ptr(), Hq, Hkv, D, ctx, stride, dtype,
+                          out.data_ptr(), scratch.data_ptr(), nbytes)
+    assert st == kie.KIE_OK
+    got = out.cpu().numpy()
+    # the oracle sees the query as the fp32 values the kernel reads
+    qf = q.astype(np.float32).astype(np.float64)
+    for h in range(Hq):
+        g = h * Hkv // Hq
+        want = orc.attention(qf[h], K[g, :ctx], Vv[g, :ctx], dtype)
+        np.testing.assert_allclose(got[h], want, rtol=0, atol=2e-5 * max(1.0, np.abs(want).max()))
+
+
+# ------------------------------------------------------------------ whole-model parity
+
+def test_tiny_parity(kie):
+    from bandwidth_bound_stream_b200 import synth
+    from tests.parity import assert_reports
+    m = synth.TINY
+    dw, eng, orc = _setup(kie, m, 64)
+    with eng:
+        reps = _lockstep(kie, eng, orc, m, synth.prompt(m, 16), 32)
+    assert_reports(reps, m.dtype)
+
+
+def test_tiny_generate_and_launch_match_oracle_chain(kie):
+    """kie_generate (doorbell, argmax fed back on the GPU) and kie_decode_launch (one stream-ordered
+    launch) both follow the oracle's greedy chain while its margins exceed 0.05."""
+    from bandwidth_bound_stream_b200 import synth
+    from tests.parity import MARGIN, margin
+    m = synth.TINY
+    dw, eng, orc = _setup(kie, m, 96)
+    prompt = synth.prompt(m, 16, session=3)
+    n = 24
+    with eng:
+        sid = eng.session_open()
+        first = eng.prefill(sid, prompt)
+        ref = orc.prefill(prompt)
+        assert first == int(np.argmax(ref)) or margin(ref) <= MARGIN
+        chain, margins = [], []
+        tok = first
+        for _ in range(n):
+            ref = orc.step(tok)
+            tok = int(np.argmax(ref))
+            chain.append(tok)
+            margins.append(margin(ref))
+        gen = eng.generate(sid, first, n)
+        # compare up to the first low-margin step (after it the two chains may legitimately differ)
+        k = next((i for i, mg in enumerate(margins) if mg <= MARGIN), n)
+        assert list(gen[:k]) == chain[:k]
+        # the stream-ordered launch from the same prefix gives the same tokens as the doorbell path
+        eng.session_rewind(sid, len(prompt))
+        tok_d = torch.tensor([first], dtype=torch.int32, device="cuda")
+        out_d = torch.zeros(n, dtype=torch.int32, device="cuda")
+        eng.decode_launch(sid, tok_d.data_ptr(), n, out_d.data_ptr())
+        eng.sync()
+        assert np.array_equal(out_d.cpu().numpy(), gen)
+
+
+@pytest.mark.parametrize("name,prompt_len,steps", [("slice-1.9b", 40, 8), ("slice-8b", 24, 6), ("ragged", 33, 10)])
+def test_sliced_shapes_parity(kie, name, prompt_len, steps):
+    """Two-layer slices of the 1.9B (fp16, GQA 2) and 8B (bf16, GQA 4) shapes at full width, and a ragged
+    shape (odd vocab, GQA 3, rows not divisible by the SM count)."""
+    from bandwidth_bound_stream_b200 import synth
+    from tests.parity import assert_reports
+    m = synth.CONFIGS[name]
+    dw, eng, orc = _setup(kie, m, prompt_len + steps + 4)
+    with eng:
+        reps = _lockstep(kie, eng, orc, m, synth.prompt(m, prompt_len), steps)
+    assert_reports(reps, m.dtype)
+
+
+def test_full_1p9b_parity_short_context(kie):
+    """All 28 layers of the 1.9B shape, 64-token prompt, 4 decode steps with logits."""
+    from bandwidth_bound_stream_b200 import synth
+    from tests.parity import assert_reports
+    m = synth.DENSE_1P9B
+    dw, eng, orc = _setup(kie, m, 80)
+    with eng:
+        reps = _lockstep(kie, eng, orc, m, synth.prompt(m, 64), 4)
+    assert_reports(reps, m.dtype)
+
+
+def test_full_1p9b_bench_launch_layer0_cache(kie):
+    """The benchmark's configuration (1.9B, prompt 1024, one launch of 512 steps): layer-0 K/V at sampled
+    positions equal the oracle's projection of that position's token (they depend on it alone)."""
+    from bandwidth_bound_stream_b200 import synth
+    from oracle import oracle as orc
+    m = synth.DENSE_1P9B
+    dw = kie.DeviceWeights(m, host_copy=True)
+    prompt = synth.prompt(m, 1024)
+    with kie.Engine(kie.config(m, max_ctx=1536, timeout_ms=5000, idle_ms=50), dw.kie) as eng:
+        sid = eng.session_open()
+        first = eng.prefill(sid, prompt)
+        tok_d = torch.tensor([first], dtype=torch.int32, device="cuda")
+        out_d = torch.zeros(512, dtype=torch.int32, device="cuda")
+        eng.decode_launch(sid, tok_d.data_ptr(), 512, out_d.data_ptr())
+        eng.sync()
+        gen = out_d.cpu().numpy()
+        assert gen.min() >= 0 and gen.max() < m.vocab
+        kp, vp = eng.session_kv(sid)
+        n = m.n_kv_heads * 1536 * m.head_dim
+        # copy layer 0 of the cache through a torch view of the engine's buffer
+        kt = _device_view(kp, n)
+        vt = _device_view(vp, n)
+        K0 = kt.cpu().numpy().view(np.uint16).reshape(m.n_kv_heads, 1536, m.head_dim)
+        V0 = vt.cpu().numpy().view(np.uint16).reshape(m.n_kv_heads, 1536, m.head_dim)
+    seq = np.concatenate([prompt, [first], gen[:-1]])
+    L0 = dw.host["layers"][0]
+    for p in (0, 1, 777, 1023, 1024, 1300, 1535):
+        e = orc.value(dw.host["tok_emb"][seq[p]], m.dtype)
+        h = orc.rmsnorm(e, L0["attn_norm"], m.dtype, m.rms_eps)
+        k = orc.matvec(L0["wk"], m.dtype, h)
+        v = orc.matvec(L0["wv"], m.dtype, h)
+        D = m.head_dim
+        for g in range(m.n_kv_heads):
+            kr = orc.rope(k[g * D:(g + 1) * D], p, m.rope_theta)
+            want_k = orc.value(orc.store(kr, m.dtype), m.dtype)
+            want_v = orc.value(orc.store(v[g * D:(g + 1) * D], m.dtype), m.dtype)
+            got_k = orc.value(K0[g, p], m.dtype)
+            got_v = orc.value(V0[g, p], m.dtype)
+            # fp32 accumulation vs fp64: at most one rounding step of the stored value apart
+            np.testing.assert_allclose(got_k, want_k, rtol=2e-3, atol=1e-4)
+            np.testing.assert_allclose(got_v, want_v, rtol=2e-3, atol=1e-4)
+
+
+def _device_view(ptr, n):
+    """A torch int16 tensor aliasing n elements of engine-owned device memory (read-only use)."""
+    class _Holder:
+        __cuda_array_interface__ = {"shape": (n,), "typestr": "<i2", "data": (ptr, False), "version": 2}
+    return torch.as_tensor(_Holder(), device="cuda")
+
+
+# ------------------------------------------------------------------ host-side errors and lifecycle
+
+def test_errors_are_reported_not_fatal(kie):
+    from bandwidth_bound_stream_b200 import synth
+    m = synth.TINY
+    dw = kie.DeviceWeights(m)
+    with kie.Engine(kie.config(m, max_ctx=20, max_sessions=1, timeout_ms=5000, idle_ms=50), dw.kie) as eng:
+        sid = eng.session_open()
+        with pytest.raises(kie.KieError) as ei:
+            eng.session_open()
+        assert ei.value.status == kie.KIE_ERR_CAPACITY
+        with pytest.raises(kie.KieError) as ei:
+            eng.prefill(sid, np.zeros(21, dtype=np.int32))
+        assert ei.value.status == kie.KIE_ERR_CAPACITY
+        assert eng.session_length(sid) == 0
+        with pytest.raises(kie.KieError) as ei:
+            eng.decode_step(sid, m.vocab)
+        assert ei.value.status == kie.KIE_ERR_ARG
+        with pytest.raises(kie.KieError) as ei:
+            eng.decode_step(sid + 1, 1)
+        assert ei.value.status == kie.KIE_ERR_ARG
+        # the engine still works afterwards
+        first = eng.prefill(sid, synth.prompt(m, 8))
+        assert 0 <= first < m.vocab
+        with pytest.raises(kie.KieError) as ei:
+            eng.generate(sid, first, 13)
+        assert ei.value.status == kie.KIE_ERR_CAPACITY
+
+
+def test_resident_kernel_idles_out_and_relaunches(kie):
+    """With no command the resident kernel gives up waiting after idle_ms and exits cleanly; the
+    next call relaunches it and the results are unchanged."""
+    import time
+    from bandwidth_bound_stream_b200 import synth
+    m = synth.TINY
+    dw = kie.DeviceWeights(m)
+    prompt = synth.prompt(m, 10)
+    with kie.Engine(kie.config(m, max_ctx=64, timeout_ms=5000, idle_ms=20), dw.kie) as eng:
+        sid = eng.session_open()
+        first = eng.prefill(sid, prompt)
+        a = eng.generate(sid, first, 5)
+        time.sleep(0.3)  # well past idle_ms: the kernel has exited
+        eng.session_rewind(sid, len(prompt))
+        b = eng.generate(sid, first, 5)
+        assert np.array_equal(a, b)
