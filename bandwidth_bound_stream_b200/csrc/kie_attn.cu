@@ -6,22 +6,19 @@
 
 namespace {
 
+constexpr int FD_WARPS = 8;
+
 template <int DT>
-__global__ void __launch_bounds__(ATTN_THREADS) flash_decode_kernel(AttnArgs A, int G) {
+__global__ void __launch_bounds__(FD_WARPS * 32) flash_decode_kernel(AttnArgs A, int G) {
     __shared__ AttnSmem S;
-    attn_smem_init(S, threadIdx.x, ATTN_THREADS);
-    __syncthreads();
-    attn_all_units<DT>(A, S, G, blockIdx.x, gridDim.x);
+    attn_all_units<DT, FD_WARPS>(A, S, G, blockIdx.x, gridDim.x);
 }
 
-// Splits per kv head: about 64 positions per split, at most 64 splits, and never more
-// positions per split than the score buffer holds.
+// Splits per kv head: about 64 positions per split, at most 64 splits.
 int fd_splits(int G, int n_ctx) {
+    (void)G;
     int s = (n_ctx + 63) / 64;
     if (s > 64) s = 64;
-    const int cap = KIE_SCORE_MAX / G;  // positions one split may hold
-    const int need = (n_ctx + cap - 1) / cap;
-    if (s < need) s = need;
     return s < 1 ? 1 : s;
 }
 
@@ -69,7 +66,7 @@ extern "C" kie_status kie_flash_decode(const float *q_dev, const void *k_dev, co
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(A.cnt, 0, (size_t)n_kv_heads * 4, s) != cudaSuccess) return KIE_ERR_CUDA;
     const dim3 grid(n_kv_heads * A.nsplit);
-    if (dtype == KIE_BF16) flash_decode_kernel<KIE_BF16><<<grid, ATTN_THREADS, 0, s>>>(A, G);
-    else flash_decode_kernel<KIE_FP16><<<grid, ATTN_THREADS, 0, s>>>(A, G);
+    if (dtype == KIE_BF16) flash_decode_kernel<KIE_BF16><<<grid, FD_WARPS * 32, 0, s>>>(A, G);
+    else flash_decode_kernel<KIE_FP16><<<grid, FD_WARPS * 32, 0, s>>>(A, G);
     return cudaGetLastError() == cudaSuccess ? KIE_OK : KIE_ERR_CUDA;
 }

@@ -2,20 +2,20 @@
 //
 // Decode reads the whole KV cache once per token ("Kog 3000 tok/s 实时推理…", section
 // 内存带宽优化的三层策略), so the cache range of each kv head is cut into `nsplit` splits
-// and one CTA works on one (kv head, split) unit, for all query heads of the group:
+// and one CTA works on one (kv head, split) unit, for all query heads of the group.
 //
-//   pass 1  s_j = q_h . K_j / sqrt(D) (kept in log2 units) for every position of the split
-//   pass 2  p_j = 2^(s_j - m), l = sum p_j, acc = sum p_j V_j
-//   merge   the last unit to finish a kv head combines the splits' (m, l, acc):
-//           o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s
+// Within a unit, D/8 lanes hold one position's 16-byte slices ("a position group"), so a
+// warp covers 32/(D/8) positions per load and the CTA 8x that. Each position group walks
+// its positions in batches of B, issuing all 2B K/V loads of a batch before using any, and
+// keeps a running softmax per query head (max m, sum l, weighted value sum acc), with
+// scores in log2 units: s_j = q . K_j * log2(e) / sqrt(D), p_j = 2^(s_j - m).
+// Position groups, then warps, are merged by rescaling to the common max. The last unit to
+// finish a kv head combines the splits the same way:
+//     o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s,
+// which equals the one-pass softmax over all positions for any split count.
 //
-// The merge is the usual log-sum-exp combination of partial softmaxes (it equals the
-// one-pass softmax for any number of splits). Lanes: D/8 lanes hold one position's
-// 16-byte slices, so a warp covers 32/(D/8) positions per load; the partial sums over
-// positions in a warp are combined with shuffles, across warps in shared memory.
-//
-// Contract for callers: 256 threads (8 warps) execute attn_all_units together and use
-// named barrier 1; AttnSmem is zero-initialised once with attn_smem_init.
+// Contract for callers: NW warps (8 or 16, threads 0 .. 32*NW-1) execute attn_all_units
+// together and use named barrier 1.
 #pragma once
 #include <math_constants.h>
 
@@ -32,31 +32,46 @@ struct AttnArgs {
 };
 
 struct AttnSmem {
-    float scores[KIE_SCORE_MAX];
-    float accs[KIE_GMAX * KIE_DMAX];
-    float lsum[KIE_GMAX];
+    float wacc[4][KIE_GMAX * KIE_DMAX];  // warp w adds into slot w % 4, in warp order
+    float wl[4][KIE_GMAX];
     float mrow[KIE_GMAX];
-    float red[KIE_GMAX * 8];
+    float red[KIE_GMAX * 16];
     int is_last;
 };
 
-KIE_DEV void attn_smem_init(AttnSmem &S, int tid, int nthreads) {
-    for (int i = tid; i < KIE_GMAX * KIE_DMAX; i += nthreads) S.accs[i] = 0.f;
-    if (tid < KIE_GMAX) S.lsum[tid] = 0.f;
+// Asks L2 for the K and V rows units first, first + step, ... will read (a hint that may be
+// issued before the newest position is written: L2 stays coherent).
+KIE_DEV void attn_prefetch(const uint16_t *k, const uint16_t *v, long long head_stride, int D, int Hkv, int nsplit,
+                           int ctx, int first, int step) {
+    for (int unit = first; unit < Hkv * nsplit; unit += step) {
+        const int g = unit / nsplit, s = unit % nsplit;
+        const long long p0 = (long long)s * ctx / nsplit, p1 = (long long)(s + 1) * ctx / nsplit;
+        for (long long a = p0; a < p1; a += 1024) {
+            const long long n = (p1 - a < 1024 ? p1 - a : 1024) * D * 2;
+            const size_t off = (size_t)g * head_stride + (size_t)a * D;
+            bulk_prefetch_l2(k + off, (uint32_t)n);
+            bulk_prefetch_l2(v + off, (uint32_t)n);
+        }
+    }
 }
 
-#define ATTN_THREADS 256
-#define ATTN_WARPS 8
+// 2^(x - M) with 2^(-inf - M) = 0 (M >= x; M = -inf only when x = -inf)
+KIE_DEV float rescale(float x, float M) { return x == -CUDART_INF_F ? 0.f : exp2f(x - M); }
 
-template <int DT, int G>
-__device__ void attn_unit(const AttnArgs &A, AttnSmem &S, int unit) {
+// Query heads hoff .. hoff+nh-1 (nh <= GC) of the group of kv head `unit / nsplit`, whose
+// group has Gt query heads in all; a kv head with more than 4 query heads is done in chunks
+// of 4 (each chunk re-reads the split's K/V, mostly from L2).
+template <int DT, int GC, int NW>
+__device__ void attn_unit(const AttnArgs &A, AttnSmem &S, int unit, int Gt, int hoff) {
+    constexpr int G = GC;
+    constexpr int B = NW >= 16 ? (G == 1 ? 4 : 2) : (G == 1 ? 8 : G == 2 ? 4 : 2);  // positions per group per batch (register budget)
+    constexpr int ATTN_WARPS = NW, ATTN_THREADS = NW * 32;
+    const int nh = min(GC, Gt - hoff);
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int D = A.D, lpp = D >> 3, ppw = 32 / lpp, sub = lane / lpp, sl = lane % lpp;
     const int nsplit = A.nsplit, ctx = A.ctx;
-    const int SP = KIE_SCORE_MAX / G;
+    const int ngroups = ATTN_WARPS * ppw, gi = w * ppw + sub;
     const float qscale = rsqrtf((float)D) * 1.4426950408889634f;
-    const int stride = ATTN_WARPS * ppw;
-    constexpr int U = 4;
 
     const int g = unit / nsplit, s = unit % nsplit;
     const int p0 = (int)((long long)s * ctx / nsplit), p1 = (int)((long long)(s + 1) * ctx / nsplit);
@@ -68,161 +83,171 @@ __device__ void attn_unit(const AttnArgs &A, AttnSmem &S, int unit) {
     float q[G][8];
 #pragma unroll
     for (int jj = 0; jj < G; jj++) {
-        const float *qp = A.q + (size_t)(g * G + jj) * D + sl * 8;
+        const float *qp = A.q + (size_t)(g * Gt + hoff + min(jj, nh - 1)) * D + sl * 8;
         const float4 a = __ldcg(reinterpret_cast<const float4 *>(qp));
         const float4 b = __ldcg(reinterpret_cast<const float4 *>(qp + 4));
         q[jj][0] = a.x * qscale; q[jj][1] = a.y * qscale; q[jj][2] = a.z * qscale; q[jj][3] = a.w * qscale;
         q[jj][4] = b.x * qscale; q[jj][5] = b.y * qscale; q[jj][6] = b.z * qscale; q[jj][7] = b.w * qscale;
     }
-
-    // pass 1: scores of every position of the split
-    float mx[G];
-#pragma unroll
-    for (int jj = 0; jj < G; jj++) mx[jj] = -CUDART_INF_F;
-    for (int j0 = w * ppw + sub; j0 - sub < np; j0 += stride * U) {
-        uint4 kv[U];
-#pragma unroll
-        for (int u = 0; u < U; u++) {
-            const int j = j0 + u * stride;
-            kv[u] = j < np ? __ldcg(reinterpret_cast<const uint4 *>(Kp + (size_t)j * D)) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < U; u++) {
-            const int j = j0 + u * stride;
-            float f[8];
-            cvt8<DT>(kv[u], f);
-#pragma unroll
-            for (int jj = 0; jj < G; jj++) {
-                float dsum = 0.f;
-#pragma unroll
-                for (int e = 0; e < 8; e++) dsum = fmaf(f[e], q[jj][e], dsum);
-                for (int o = lpp >> 1; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
-                if (j < np) {
-                    if (sl == 0) S.scores[jj * SP + j] = dsum;
-                    mx[jj] = fmaxf(mx[jj], dsum);
-                }
-            }
-        }
-    }
+    float m[G], l[G], acc[G][8];
 #pragma unroll
     for (int jj = 0; jj < G; jj++) {
-        const float m = warp_max(mx[jj]);
-        if (lane == 0) S.red[w * G + jj] = m;
-    }
-    named_bar_sync(1, ATTN_THREADS);
-    if (tid < G) {
-        float m = -CUDART_INF_F;
-        for (int k = 0; k < ATTN_WARPS; k++) m = fmaxf(m, S.red[k * G + tid]);
-        S.mrow[tid] = m;
-    }
-    named_bar_sync(1, ATTN_THREADS);
-    float M[G];
-#pragma unroll
-    for (int jj = 0; jj < G; jj++) M[jj] = S.mrow[jj];
-
-    // pass 2: softmax weights and the weighted sum of values
-    float acc[G][8], ls[G];
-#pragma unroll
-    for (int jj = 0; jj < G; jj++) {
-        ls[jj] = 0.f;
+        m[jj] = -CUDART_INF_F;
+        l[jj] = 0.f;
 #pragma unroll
         for (int e = 0; e < 8; e++) acc[jj][e] = 0.f;
     }
-    for (int j0 = w * ppw + sub; j0 - sub < np; j0 += stride * U) {
-        uint4 vv[U];
+
+    for (int base = 0; base < np; base += ngroups * B) {  // uniform across the CTA
+        uint4 kv[B], vv[B];
 #pragma unroll
-        for (int u = 0; u < U; u++) {
-            const int j = j0 + u * stride;
-            vv[u] = j < np ? __ldcg(reinterpret_cast<const uint4 *>(Vp + (size_t)j * D)) : make_uint4(0, 0, 0, 0);
+        for (int b = 0; b < B; b++) {
+            const int j = base + gi + b * ngroups;
+            const bool ok = j < np;
+            kv[b] = ok ? __ldcg(reinterpret_cast<const uint4 *>(Kp + (size_t)j * D)) : make_uint4(0, 0, 0, 0);
+            vv[b] = ok ? __ldcg(reinterpret_cast<const uint4 *>(Vp + (size_t)j * D)) : make_uint4(0, 0, 0, 0);
+        }
+        float sc[B][G];
+#pragma unroll
+        for (int b = 0; b < B; b++) {
+            const bool ok = base + gi + b * ngroups < np;
+            float f[8];
+            cvt8<DT>(kv[b], f);
+#pragma unroll
+            for (int jj = 0; jj < G; jj++) {
+                float d = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; e++) d = fmaf(f[e], q[jj][e], d);
+                for (int o = lpp >> 1; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+                sc[b][jj] = ok ? d : -CUDART_INF_F;
+            }
         }
 #pragma unroll
-        for (int u = 0; u < U; u++) {
-            const int j = j0 + u * stride;
-            if (j < np) {
-                float f[8];
-                cvt8<DT>(vv[u], f);
+        for (int jj = 0; jj < G; jj++) {
+            float mb = m[jj];
 #pragma unroll
-                for (int jj = 0; jj < G; jj++) {
-                    const float p = exp2f(S.scores[jj * SP + j] - M[jj]);
-                    ls[jj] += p;
+            for (int b = 0; b < B; b++) mb = fmaxf(mb, sc[b][jj]);
+            const float r = rescale(m[jj], mb);
+            l[jj] *= r;
 #pragma unroll
-                    for (int e = 0; e < 8; e++) acc[jj][e] = fmaf(p, f[e], acc[jj][e]);
-                }
+            for (int e = 0; e < 8; e++) acc[jj][e] *= r;
+            m[jj] = mb;
+        }
+#pragma unroll
+        for (int b = 0; b < B; b++) {
+            float f[8];
+            cvt8<DT>(vv[b], f);
+#pragma unroll
+            for (int jj = 0; jj < G; jj++) {
+                const float p = rescale(sc[b][jj], m[jj]);
+                l[jj] += p;
+#pragma unroll
+                for (int e = 0; e < 8; e++) acc[jj][e] = fmaf(p, f[e], acc[jj][e]);
             }
         }
     }
+    // merge the position groups of each warp (lanes with the same sl hold the same dims)
 #pragma unroll
     for (int jj = 0; jj < G; jj++) {
         for (int o = lpp; o < 32; o <<= 1) {
-            ls[jj] += __shfl_xor_sync(0xffffffffu, ls[jj], o);
+            const float m2 = __shfl_xor_sync(0xffffffffu, m[jj], o);
+            const float l2 = __shfl_xor_sync(0xffffffffu, l[jj], o);
+            const float M = fmaxf(m[jj], m2);
+            const float ra = rescale(m[jj], M), rb = rescale(m2, M);
+            l[jj] = l[jj] * ra + l2 * rb;
 #pragma unroll
-            for (int e = 0; e < 8; e++) acc[jj][e] += __shfl_xor_sync(0xffffffffu, acc[jj][e], o);
+            for (int e = 0; e < 8; e++) {
+                const float a2 = __shfl_xor_sync(0xffffffffu, acc[jj][e], o);
+                acc[jj][e] = acc[jj][e] * ra + a2 * rb;
+            }
+            m[jj] = M;
         }
-        if (sub == 0) {
-#pragma unroll
-            for (int e = 0; e < 8; e++) atomicAdd(&S.accs[jj * D + sl * 8 + e], acc[jj][e]);
-            if (sl == 0) atomicAdd(&S.lsum[jj], ls[jj]);
-        }
+        if (lane == 0) S.red[w * G + jj] = m[jj];
     }
     named_bar_sync(1, ATTN_THREADS);
+    if (tid < G) {
+        float M = -CUDART_INF_F;
+        for (int k = 0; k < ATTN_WARPS; k++) M = fmaxf(M, S.red[k * G + tid]);
+        S.mrow[tid] = M;
+    }
+    named_bar_sync(1, ATTN_THREADS);
+    // merge the warps at the common max, in a fixed order (warps w, w+4, ... into slot w % 4,
+    // then slots 0..3)
+    for (int round = 0; round < ATTN_WARPS / 4; round++) {
+        if ((w >> 2) == round && sub == 0) {
+            float *wa = S.wacc[w & 3];
+#pragma unroll
+            for (int jj = 0; jj < G; jj++) {
+                const float r = rescale(m[jj], S.mrow[jj]);
+#pragma unroll
+                for (int e = 0; e < 8; e++) {
+                    const float v = acc[jj][e] * r;
+                    wa[jj * D + sl * 8 + e] = round == 0 ? v : wa[jj * D + sl * 8 + e] + v;
+                }
+                if (sl == 0) S.wl[w & 3][jj] = round == 0 ? l[jj] * r : S.wl[w & 3][jj] + l[jj] * r;
+            }
+        }
+        named_bar_sync(1, ATTN_THREADS);
+    }
 
     // publish this split's partial, then the last split of the kv head merges
-    float *pp = A.part + (size_t)unit * G * (D + 2);
-    for (int i = tid; i < G * (D + 2); i += ATTN_THREADS) {
-        const int jj = i / (D + 2), e = i % (D + 2);
-        float val;
+    float *pp = A.part + ((size_t)unit * Gt + hoff) * (D + 2);
+    for (int i = tid; i < nh * (D + 2) / 2; i += ATTN_THREADS) {  // float2 per thread (D + 2 is even)
+        const int jj = (2 * i) / (D + 2), e = (2 * i) % (D + 2);
+        float2 val;
         if (e == 0) {
-            val = M[jj];
-        } else if (e == 1) {
-            val = S.lsum[jj];
-            S.lsum[jj] = 0.f;
+            val.x = S.mrow[jj];
+            val.y = ((S.wl[0][jj] + S.wl[1][jj]) + S.wl[2][jj]) + S.wl[3][jj];
         } else {
-            val = S.accs[jj * D + e - 2];
-            S.accs[jj * D + e - 2] = 0.f;
+            const int k = jj * D + e - 2;
+            val.x = ((S.wacc[0][k] + S.wacc[1][k]) + S.wacc[2][k]) + S.wacc[3][k];
+            val.y = ((S.wacc[0][k + 1] + S.wacc[1][k + 1]) + S.wacc[2][k + 1]) + S.wacc[3][k + 1];
         }
-        pp[i] = val;
+        reinterpret_cast<float2 *>(pp)[i] = val;
     }
     __threadfence();
     named_bar_sync(1, ATTN_THREADS);
     if (tid == 0) {
+        const unsigned chunks = (unsigned)((Gt + GC - 1) / GC);
         const unsigned prev = atomicAdd(A.cnt + g, 1u);
-        S.is_last = (prev == (unsigned)(nsplit - 1));
+        S.is_last = (prev == (unsigned)nsplit * chunks - 1u);
     }
     named_bar_sync(1, ATTN_THREADS);
     if (S.is_last) {
         __threadfence();
-        const float *pg = A.part + (size_t)g * nsplit * G * (D + 2);
-        for (int i = tid; i < G * D; i += ATTN_THREADS) {
+        const float *pg = A.part + (size_t)g * nsplit * Gt * (D + 2);
+        for (int i = tid; i < Gt * D; i += ATTN_THREADS) {
             const int jj = i / D, e = i % D;
             float mxs = -CUDART_INF_F;
-            for (int k = 0; k < nsplit; k++) mxs = fmaxf(mxs, __ldcg(pg + ((size_t)k * G + jj) * (D + 2)));
+            for (int k = 0; k < nsplit; k++) mxs = fmaxf(mxs, __ldcg(pg + ((size_t)k * Gt + jj) * (D + 2)));
             float num = 0.f, den = 0.f;
             for (int k = 0; k < nsplit; k++) {
-                const float *pk = pg + ((size_t)k * G + jj) * (D + 2);
-                const float wk = exp2f(__ldcg(pk) - mxs);
+                const float *pk = pg + ((size_t)k * Gt + jj) * (D + 2);
+                const float wk = rescale(__ldcg(pk), mxs);
                 den = fmaf(wk, __ldcg(pk + 1), den);
                 num = fmaf(wk, __ldcg(pk + 2 + e), num);
             }
-            A.o[(size_t)(g * G + jj) * D + e] = num / den;
+            A.o[(size_t)(g * Gt + jj) * D + e] = num / den;
         }
         if (tid == 0) A.cnt[g] = 0u;
     }
     named_bar_sync(1, ATTN_THREADS);
 }
 
-// Units first, first + step, ... of the Hkv * nsplit units.
-template <int DT>
+// Units first, first + step, ... of the Hkv * nsplit units. With 16 warps (a smaller
+// register budget per thread) at most 2 query heads are processed per pass, else 4.
+template <int DT, int NW>
 __device__ void attn_all_units(const AttnArgs &A, AttnSmem &S, int G, int first, int step) {
+    constexpr int GCMAX = NW >= 16 ? 2 : 4;
     for (int unit = first; unit < A.Hkv * A.nsplit; unit += step) {
-        switch (G) {
-            case 1: attn_unit<DT, 1>(A, S, unit); break;
-            case 2: attn_unit<DT, 2>(A, S, unit); break;
-            case 3: attn_unit<DT, 3>(A, S, unit); break;
-            case 4: attn_unit<DT, 4>(A, S, unit); break;
-            case 5: attn_unit<DT, 5>(A, S, unit); break;
-            case 6: attn_unit<DT, 6>(A, S, unit); break;
-            case 7: attn_unit<DT, 7>(A, S, unit); break;
-            default: attn_unit<DT, 8>(A, S, unit); break;
+        if (G == 1) {
+            attn_unit<DT, 1, NW>(A, S, unit, 1, 0);
+        } else if (G <= GCMAX) {
+            if (G == 2) attn_unit<DT, 2, NW>(A, S, unit, 2, 0);
+            else if (G == 3) attn_unit<DT, (GCMAX >= 3 ? 3 : 2), NW>(A, S, unit, 3, 0);
+            else attn_unit<DT, GCMAX, NW>(A, S, unit, G, 0);
+        } else {
+            for (int hoff = 0; hoff < G; hoff += GCMAX) attn_unit<DT, GCMAX, NW>(A, S, unit, G, hoff);
         }
     }
 }

@@ -6,14 +6,15 @@
 // byte plus the KV cache once ("Kog 3000 tok/s 实时推理…", section 内存带宽优化的三层策略), so
 // the kernel is organised around that stream:
 //
-//  * Warp 8 (the producer) walks this CTA's fixed weight schedule for the whole command
-//    (all layers, all tokens) and copies it, chunk by chunk, into a 6 x 32 KB shared-memory
-//    ring with 1-D bulk async copies (TMA). The schedule is contiguous in HBM because the
-//    weights were repacked at engine creation in exactly this order, so each SM streams one
-//    disjoint span (the aligned, topology-aware access pattern of the same section). The
-//    producer never waits on grid barriers, so weight streaming runs ahead of compute by up
-//    to the ring size across phase, layer and token boundaries.
-//  * Warps 0-7 (consumers) run the phases of each layer on the staged chunks:
+//  * Warp 16 (the producer) walks this CTA's fixed weight schedule for the whole command
+//    (all layers, all tokens) and copies it, chunk by chunk, into a 3 x 64 KB shared-memory
+//    ring with 1-D bulk async copies (TMA). An optional second cursor runs `pf_chunks`
+//    chunks further ahead and asks for the same chunks to be brought into L2 (off by
+//    default: measured on B200 it lowers throughput). The schedule is contiguous in HBM
+//    because the weights were repacked at engine creation in exactly this order, so each SM
+//    streams one disjoint span (the aligned, topology-aware access of the same section).
+//    The producer never waits on grid barriers.
+//  * Warps 0-15 (consumers) run the phases of each layer on the staged chunks:
 //      QKV  : RMSNorm -> [Wq;Wk;Wv] rows -> RoPE -> q, and the K/V append to the cache
 //      ATTN : split-K single-query attention over the cache, last split merges (LSE)
 //      O    : x += Wo o
@@ -22,11 +23,18 @@
 //    then, per token, HEAD: final RMSNorm -> LM-head rows -> block argmax -> grid argmax.
 //    Phases are separated by a grid-wide barrier with a time limit.
 //
-// GEMV mapping: a ring chunk holds CR whole rows of length K. Warp w owns the column slice
+// GEMV mapping: a ring chunk holds 2*CR whole rows of length K. The 16 consumer warps form
+// two groups of 8; group g takes rows [g*CR, (g+1)*CR) of every chunk. In a group, warp w
+// owns the column slice
 // [w*K/8, (w+1)*K/8); lane l owns 16-byte vectors l, l+32, ... of that slice, so a lane's
 // slice of the input vector sits in registers for the whole phase and each staged weight
-// byte is read from shared memory exactly once. Row sums are reduced across the warp
-// (shuffle butterfly over CR rows) and across warps with shared-memory atomics.
+// byte is read from shared memory exactly once. Row sums are reduced across the warp with
+// a shuffle butterfly over the CR rows; the 8 column-slice partials of a row are added in
+// a fixed order by the phase epilogue, so results are bit-reproducible.
+//
+// RMSNorm: the residual rows are owned by the CTA that updates them (O and DOWN phases);
+// each CTA publishes the sum of squares of its rows when it arrives at the next grid
+// barrier, and every reader adds the per-CTA sums in CTA order.
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
@@ -37,24 +45,26 @@ namespace {
 
 constexpr int RING_BYTES = KIE_NSLOT * KIE_SLOT_BYTES;
 
+constexpr int WPART_FLOATS = 8 * KIE_ROWACC_MAX;  // column-slice partials: [slices][rows] flattened
+
 struct __align__(16) B1Shared {
-    float rowacc[KIE_ROWACC_MAX];
-    AttnSmem at;
+    union {
+        float wpart[WPART_FLOATS];  // column-slice partials of this phase's row sums
+        AttnSmem at;
+    };
     float red[64];
     int redi[32];
+    float ssqw[KIE_CONS_WARPS];
+    float xown[KIE_XOWN_MAX];  // this CTA's residual rows (O and DOWN phases own the same rows)
+    float2 rope_s[KIE_DMAX / 2];  // rotation of the current position, loaded at the start of QKV
     uint64_t full[KIE_NSLOT];
     uint64_t empty[KIE_NSLOT];
     KieCmd cmd;
     volatile int abort;
     int token;
-    int is_last;
     int gb_ok;
     int row0[KIE_NPH], row1[KIE_NPH];
-};
-
-struct Ring {
-    uint8_t *base;
-    uint32_t it;  // chunks consumed (consumers) or issued (producer) so far
+    unsigned long long wait_cons;
 };
 
 // word-wise copies of the command record (volatile: it may live in mapped host memory)
@@ -71,29 +81,46 @@ __device__ __forceinline__ void copy_words_cg(KieCmd *dst, const KieCmd *src) {
     for (int i = 0; i < (int)(sizeof(KieCmd) / 4); i++) d[i] = __ldcg(s + i);
 }
 
-// rows per ring chunk and 16-byte vectors per lane, both fixed by the row length K
-__host__ __device__ inline int vec_per_lane(int K) {
-    return K <= 2048 ? 1 : K <= 4096 ? 2 : K <= 8192 ? 4 : K <= 14336 ? 7 : 8;
+// GEMV geometry fixed by the row length K: column slices per row (8: two warp groups take
+// different rows of a chunk; 16: all warps share each row), 16-byte vectors per lane, and
+// rows per group in one ring chunk. K <= 14336.
+__host__ __device__ inline int col_slices(int K) { return K <= 8192 ? 8 : 16; }
+__host__ __device__ inline int vec_per_lane(int K) { return K <= 2048 ? 1 : K <= 4096 ? 2 : 4; }
+__host__ __device__ inline int rows_per_group(int K) { return K <= 2048 ? 8 : K <= 4096 ? 4 : 2; }
+
+__device__ __forceinline__ void trace_mark(const KieParams &P, int t, int ev, float after = 0.f) {
+    if (P.trace && t < P.trace_tokens && threadIdx.x == 0)
+        P.trace[((size_t)blockIdx.x * P.trace_tokens + t) * P.trace_events + ev] = globaltimer() + (after != after);
 }
 
 // --------------------------------------------------------------- grid barrier
 
-// All consumer threads call this. Returns false if this CTA is aborting.
+// All consumer threads call this. Returns false if this CTA is aborting. With
+// publish_ssq, the sum of squares of the residual rows this CTA just wrote (per-warp
+// partials in S.ssqw) is published before arriving.
 __device__ bool grid_barrier(const KieParams &P, B1Shared &S, unsigned long long &epoch, long long timeout_ns,
-                             unsigned where) {
+                             unsigned where, bool publish_ssq = false) {
     named_bar_sync(1, KIE_CONS_THREADS);
     if (threadIdx.x == 0) {
         int ok = !S.abort;
         if (ok) {
+            if (publish_ssq) {
+                float v = 0.f;
+                for (int k = 0; k < KIE_CONS_WARPS; k++) v += S.ssqw[k];
+                P.ssq[blockIdx.x] = v;
+            }
             epoch += 1;
             const unsigned long long target = epoch * (unsigned long long)P.nblk;
-            __threadfence();
+            // release: this CTA's writes (ordered before by the named barrier) become visible
             red_release_gpu_add_u64(P.bar, 1ull);
             uint64_t t0 = globaltimer();
             unsigned spins = 0;
             while (ld_acquire_gpu_u64(P.bar) < target) {
                 if ((++spins & 255u) == 0) {
-                    if (ld_volatile_u32(P.err) != 0u) { ok = 0; break; }
+                    if (ld_volatile_u32(P.err) != 0u) {
+                        ok = 0;
+                        break;
+                    }
                     if ((long long)(globaltimer() - t0) > timeout_ns) {
                         set_error(P.err, DERR_BARRIER_TIMEOUT, where);
                         ok = 0;
@@ -101,7 +128,6 @@ __device__ bool grid_barrier(const KieParams &P, B1Shared &S, unsigned long long
                     }
                 }
             }
-            __threadfence();
             if (!ok) S.abort = 1;
         }
         S.gb_ok = ok;
@@ -110,54 +136,114 @@ __device__ bool grid_barrier(const KieParams &P, B1Shared &S, unsigned long long
     return S.gb_ok != 0;
 }
 
-// --------------------------------------------------------------- producer
+// --------------------------------------------------------------- the weight schedule
 
-__device__ void produce(const KieParams &P, B1Shared &S, Ring &R, const KieCmd &cmd) {
-    const int c = blockIdx.x;
-    const uint8_t *seg = P.wpack + P.seg_off[c];
-    long long phase_bytes[KIE_NPH];
-    long long layer_bytes = 0;
-    for (int ph = 0; ph < KIE_NPH; ph++) {
-        phase_bytes[ph] = (long long)(S.row1[ph] - S.row0[ph]) * P.K[ph] * 2;
-        if (ph != PH_HEAD) layer_bytes += phase_bytes[ph];
-    }
-    bool ok = true;
-    for (int t = 0; t < cmd.n && ok; t++) {
-        const bool head = (cmd.op != OP_PREFILL) || (t == cmd.n - 1);
-        for (int l = 0; l <= P.L && ok; l++) {
-            const bool is_head = (l == P.L);
-            if (is_head && !head) break;
-            const uint8_t *g = seg + (long long)l * layer_bytes;
-            for (int ph = is_head ? PH_HEAD : 0; ph < (is_head ? KIE_NPH : PH_HEAD) && ok; ph++) {
-                const int rows = S.row1[ph] - S.row0[ph];
-                const int rb = P.K[ph] * 2, cr = P.cr[ph];
-                for (int r = 0; r < rows; r += cr) {
-                    const int nr = min(cr, rows - r);
-                    const uint32_t bytes = (uint32_t)(nr * rb);
-                    const uint32_t slot = R.it % KIE_NSLOT, par = (R.it / KIE_NSLOT) & 1u;
-                    if (S.abort || !mbar_wait(&S.empty[slot], par ^ 1u, P.timeout_ns, &S.abort)) {
-                        if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x80);
-                        S.abort = 1;
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&S.full[slot], bytes);
-                    bulk_g2s(R.base + (size_t)slot * KIE_SLOT_BYTES, g, bytes, &S.full[slot]);
-                    g += bytes;
-                    R.it++;
+// Walks this CTA's chunks in stream order: per token, every layer's QKV, O, GU, DOWN rows,
+// then (when the token needs logits) the LM-head rows. A token restarts at the segment base.
+struct ChunkIter {
+    const uint8_t *seg, *g;
+    int t, l, ph, r;
+};
+
+__device__ __forceinline__ void chunk_begin(ChunkIter &it, const uint8_t *seg) {
+    it.seg = seg;
+    it.g = seg;
+    it.t = 0;
+    it.l = 0;
+    it.ph = 0;
+    it.r = 0;
+}
+
+// Next chunk (address, bytes); false when the command's schedule is exhausted.
+__device__ bool chunk_next(const KieParams &P, const B1Shared &S, const KieCmd &cmd, ChunkIter &it,
+                           const uint8_t *&addr, uint32_t &bytes) {
+    for (;;) {
+        if (it.t >= cmd.n) return false;
+        const int rows = S.row1[it.ph] - S.row0[it.ph];
+        if (it.r < rows) {
+            const int nr = min(P.cr[it.ph], rows - it.r);
+            bytes = (uint32_t)(nr * P.K[it.ph] * 2);
+            addr = it.g;
+            it.g += bytes;
+            it.r += nr;
+            return true;
+        }
+        // phase exhausted: advance
+        it.r = 0;
+        if (it.ph == PH_HEAD) {
+            it.t++;
+            it.l = 0;
+            it.ph = 0;
+            it.g = it.seg;
+        } else if (it.ph == PH_DOWN) {
+            if (++it.l == P.L) {
+                const bool head = (cmd.op != OP_PREFILL) || (it.t == cmd.n - 1);
+                if (head) {
+                    it.ph = PH_HEAD;
+                } else {
+                    it.t++;
+                    it.l = 0;
+                    it.ph = 0;
+                    it.g = it.seg;
                 }
+            } else {
+                it.ph = 0;
             }
+        } else {
+            it.ph++;
         }
     }
+}
+
+// --------------------------------------------------------------- producer
+
+__device__ void produce(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint8_t *ring, const KieCmd &cmd) {
+    const uint8_t *seg = P.wpack + P.seg_off[blockIdx.x];
+    ChunkIter fetch, pref;
+    chunk_begin(fetch, seg);
+    chunk_begin(pref, seg);
+    const uint8_t *a;
+    uint32_t b;
+    for (int k = 0; k < P.pf_chunks && chunk_next(P, S, cmd, pref, a, b); k++) bulk_prefetch_l2(a, b);
+    unsigned long long waited = 0;
+    int tok = 0;
+    while (chunk_next(P, S, cmd, fetch, a, b)) {
+        if (fetch.t != tok) {
+            if (P.trace && tok < P.trace_tokens)
+                P.trace[((size_t)blockIdx.x * P.trace_tokens + tok) * P.trace_events + P.trace_events - 1] = waited;
+            waited = 0;
+            tok = fetch.t;
+        }
+        const uint32_t slot = ring_it % KIE_NSLOT, par = (ring_it / KIE_NSLOT) & 1u;
+        if (!mbar_try_wait(&S.empty[slot], par ^ 1u)) {
+            const uint64_t w0 = globaltimer();
+            const bool ok = !S.abort && mbar_wait(&S.empty[slot], par ^ 1u, P.timeout_ns, &S.abort);
+            waited += globaltimer() - w0;
+            if (!ok) {
+                if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x80);
+                S.abort = 1;
+                break;
+            }
+        }
+        if (S.abort) break;
+        mbar_arrive_expect_tx(&S.full[slot], b);
+        bulk_g2s(ring + (size_t)slot * KIE_SLOT_BYTES, a, b, &S.full[slot]);
+        ring_it++;
+        const uint8_t *a2;
+        uint32_t b2;
+        if (chunk_next(P, S, cmd, pref, a2, b2)) bulk_prefetch_l2(a2, b2);
+    }
+    if (P.trace && tok < P.trace_tokens)
+        P.trace[((size_t)blockIdx.x * P.trace_tokens + tok) * P.trace_events + P.trace_events - 1] = waited;
     // Wait until every copy issued into the ring has landed before anyone may leave.
-    const uint32_t first = R.it > KIE_NSLOT ? R.it - KIE_NSLOT : 0;
-    for (uint32_t k = first; k < R.it; k++)
+    const uint32_t first = ring_it > KIE_NSLOT ? ring_it - KIE_NSLOT : 0;
+    for (uint32_t k = first; k < ring_it; k++)
         mbar_wait(&S.full[k % KIE_NSLOT], (k / KIE_NSLOT) & 1u, P.timeout_ns, nullptr);
 }
 
 // --------------------------------------------------------------- consumer: GEMV phases
 
-// input vector of a phase, element j
+// element j of a phase's input vector (before the norm)
 template <int DT>
 __device__ __forceinline__ float phase_input(const KieParams &P, int ph, bool from_emb, int tok, int j) {
     if (ph == PH_O) return __ldcg(P.o + j);
@@ -166,65 +252,104 @@ __device__ __forceinline__ float phase_input(const KieParams &P, int ph, bool fr
     return __ldcg(P.x + j);
 }
 
-// Runs one GEMV phase over this CTA's rows; row sums land in S.rowacc[0..rows).
-template <int DT, int NV, int CR>
-__device__ void gemv_phase(const KieParams &P, B1Shared &S, Ring &R, int ph, int l, int tok) {
+// 1/sqrt(mean(x^2) + eps) of the residual, from the per-CTA partial sums (every warp
+// computes the same value in the same order).
+__device__ __forceinline__ float rstd_from_partials(const KieParams &P) {
+    const int lane = threadIdx.x & 31;
+    float v = 0.f;
+    for (int c = lane; c < P.nblk; c += 32) v += __ldcg(P.ssq + c);
+    v = warp_sum(v);
+    return rsqrtf(v / (float)P.d + P.eps);
+}
+
+// Runs one GEMV phase over this CTA's rows; row partials land in S.wpart (see rowsum).
+template <int DT, int NV, int CR, int CS>
+__device__ void gemv_phase(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring, int ph, int l,
+                           int tok, int pos, int t) {
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int K = P.K[ph];
     const int rows = S.row1[ph] - S.row0[ph];
     const bool norm = (ph == PH_QKV || ph == PH_GU || ph == PH_HEAD);
     const bool from_emb = (ph == PH_QKV && l == 0);
 
-    float rstd = 1.f;
-    if (norm) {
-        float ss = 0.f;
-        for (int j = tid; j < P.d; j += KIE_CONS_THREADS) {
-            const float v = phase_input<DT>(P, ph, from_emb, tok, j);
-            ss += v * v;
-        }
-        ss = warp_sum(ss);
-        if (lane == 0) S.red[w] = ss;
-        named_bar_sync(1, KIE_CONS_THREADS);
-        if (w == 0) {
-            float v = lane < KIE_CONS_WARPS ? S.red[lane] : 0.f;
-            v = warp_sum(v);
-            if (lane == 0) S.red[KIE_CONS_WARPS] = rsqrtf(v / (float)P.d + P.eps);
-        }
-        named_bar_sync(1, KIE_CONS_THREADS);
-        rstd = S.red[KIE_CONS_WARPS];
-    }
+    // the QKV epilogue needs this position's rotation: fetch it now, under the row work
+    if (ph == PH_QKV && tid < (P.D >> 1)) S.rope_s[tid] = P.rope[(size_t)pos * (P.D >> 1) + tid];
+    // raw inputs first (one round trip together with the norm partials below)
     const uint16_t *gain = P.gains + (size_t)(ph == PH_HEAD ? 2 * P.L : 2 * l + (ph == PH_GU ? 1 : 0)) * P.d;
-
-    const int kslice = K >> 3;       // columns per warp
-    const int nvec = K >> 6;         // 16-byte vectors per warp slice
+    constexpr int GROUPS = KIE_CONS_WARPS / CS;  // warp groups, each taking CR rows of a chunk
+    const int kslice = K / CS;  // columns per warp
+    const int nvec = kslice >> 3;  // 16-byte vectors per warp slice
     float h[NV][8];
 #pragma unroll
     for (int i = 0; i < NV; i++) {
         const int v = lane + 32 * i;
 #pragma unroll
-        for (int e = 0; e < 8; e++) {
-            float val = 0.f;
-            if (v < nvec) {
-                const int col = w * kslice + 8 * v + e;
-                val = phase_input<DT>(P, ph, from_emb, tok, col);
-                if (norm) val = val * rstd * cvt1<DT>(gain[col]);
+        for (int e = 0; e < 8; e++) h[i][e] = 0.f;
+        if (v < nvec) {
+            const int col0 = (w % CS) * kslice + 8 * v;  // 8 consecutive columns, 32-byte aligned
+            if (from_emb) {
+                cvt8<DT>(__ldg(reinterpret_cast<const uint4 *>(P.emb + (size_t)tok * P.d + col0)), h[i]);
+            } else {
+                const float *src = ph == PH_O ? P.o : ph == PH_DOWN ? P.u : P.x;
+                const float4 a = __ldcg(reinterpret_cast<const float4 *>(src + col0));
+                const float4 b = __ldcg(reinterpret_cast<const float4 *>(src + col0 + 4));
+                h[i][0] = a.x; h[i][1] = a.y; h[i][2] = a.z; h[i][3] = a.w;
+                h[i][4] = b.x; h[i][5] = b.y; h[i][6] = b.z; h[i][7] = b.w;
             }
-            h[i][e] = val;
+            if (norm) {
+                float g[8];
+                cvt8<DT>(__ldg(reinterpret_cast<const uint4 *>(gain + col0)), g);
+#pragma unroll
+                for (int e = 0; e < 8; e++) h[i][e] *= g[e];
+            }
         }
     }
+    if (norm) {
+        float rstd;
+        if (from_emb) {
+            float ss = 0.f;
+            for (int j = tid; j < P.d; j += KIE_CONS_THREADS) {
+                const float v = cvt1<DT>(P.emb[(size_t)tok * P.d + j]);
+                ss += v * v;
+            }
+            ss = warp_sum(ss);
+            if (lane == 0) S.red[w] = ss;
+            named_bar_sync(1, KIE_CONS_THREADS);
+            float v = lane < KIE_CONS_WARPS ? S.red[lane] : 0.f;
+            v = warp_sum(v);
+            rstd = rsqrtf(v / (float)P.d + P.eps);
+            named_bar_sync(1, KIE_CONS_THREADS);
+        } else {
+            rstd = rstd_from_partials(P);
+        }
+#pragma unroll
+        for (int i = 0; i < NV; i++)
+#pragma unroll
+            for (int e = 0; e < 8; e++) h[i][e] *= rstd;
+    }
+    if (l < P.L) trace_mark(P, t, 1 + 16 * l + 11 + (ph == PH_QKV ? 0 : ph == PH_O ? 1 : ph == PH_GU ? 2 : 3), h[0][0]);
 
-    for (int r0 = 0; r0 < rows; r0 += CR) {
-        const int nr = min(CR, rows - r0);
-        const uint32_t slot = R.it % KIE_NSLOT, par = (R.it / KIE_NSLOT) & 1u;
-        R.it++;
-        bool have = !S.abort && mbar_wait(&S.full[slot], par, P.timeout_ns, &S.abort);
-        have = __all_sync(0xffffffffu, have);  // one decision per warp (the reduction below needs all lanes)
+    unsigned long long waited = 0;
+    const int grp = w / CS, ws = w % CS;
+    constexpr int STRIDE = WPART_FLOATS / CS;  // row capacity of one slice's partials
+    for (int c0 = 0; c0 < rows; c0 += GROUPS * CR) {
+        const int r0 = c0 + grp * CR;  // this group's first row in the chunk
+        const int nr = max(0, min(CR, rows - r0));
+        const uint32_t slot = ring_it % KIE_NSLOT, par = (ring_it / KIE_NSLOT) & 1u;
+        ring_it++;
+        bool have = !S.abort && mbar_try_wait(&S.full[slot], par);
+        if (!have && !S.abort) {
+            const uint64_t w0 = globaltimer();
+            have = mbar_wait(&S.full[slot], par, P.timeout_ns, &S.abort);
+            waited += globaltimer() - w0;
+        }
+        have = __all_sync(0xffffffffu, have);  // one decision per warp (the reduction needs all lanes)
         if (!have) {
             if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, (unsigned)ph);
             S.abort = 1;
             continue;  // keep the control flow; the command ends at the next barrier
         }
-        const uint8_t *base = R.base + (size_t)slot * KIE_SLOT_BYTES + (size_t)w * kslice * 2;
+        const uint8_t *base = ring + (size_t)slot * KIE_SLOT_BYTES + ((size_t)grp * CR * K + (size_t)ws * kslice) * 2;
         float acc[8];
 #pragma unroll
         for (int r = 0; r < 8; r++) acc[r] = 0.f;
@@ -246,45 +371,50 @@ __device__ void gemv_phase(const KieParams &P, B1Shared &S, Ring &R, int ph, int
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.empty[slot]);
+        if (lane == 0) mbar_arrive(&S.empty[slot]);  // shared-memory reads of the chunk are done
         const float s = warp_reduce_rows<CR>(acc);
         constexpr int LPR = 32 / CR;
-        if ((lane % LPR) == 0) {
-            const int r = lane / LPR;
-            if (r < nr) atomicAdd(&S.rowacc[r0 + r], s);
-        }
+        if ((lane % LPR) == 0 && lane / LPR < nr) S.wpart[ws * STRIDE + r0 + lane / LPR] = s;
     }
+    if (tid == 0) S.wait_cons += waited;
     named_bar_sync(1, KIE_CONS_THREADS);
 }
 
+// the row sum of row r of the current phase (column slices added in a fixed order)
+__device__ __forceinline__ float rowsum(const B1Shared &S, int r, int cs) {
+    float v = 0.f;
+    const int stride = WPART_FLOATS / cs;
+    for (int k = 0; k < cs; k++) v += S.wpart[k * stride + r];
+    return v;
+}
+
 template <int DT>
-__device__ void gemv_dispatch(const KieParams &P, B1Shared &S, Ring &R, int ph, int l, int tok) {
-    switch (vec_per_lane(P.K[ph])) {
-        case 1: gemv_phase<DT, 1, 8>(P, S, R, ph, l, tok); break;
-        case 2: gemv_phase<DT, 2, 4>(P, S, R, ph, l, tok); break;
-        case 4: gemv_phase<DT, 4, 2>(P, S, R, ph, l, tok); break;
-        case 7: gemv_phase<DT, 7, 1>(P, S, R, ph, l, tok); break;
-        default: gemv_phase<DT, 8, 1>(P, S, R, ph, l, tok); break;
-    }
+__device__ __forceinline__ void gemv_dispatch(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring, int ph, int l,
+                              int tok, int pos, int t) {
+    const int K = P.K[ph];
+    if (K <= 2048) gemv_phase<DT, 1, 8, 8>(P, S, ring_it, ring, ph, l, tok, pos, t);
+    else if (K <= 4096) gemv_phase<DT, 2, 4, 8>(P, S, ring_it, ring, ph, l, tok, pos, t);
+    else if (K <= 8192) gemv_phase<DT, 4, 2, 8>(P, S, ring_it, ring, ph, l, tok, pos, t);
+    else gemv_phase<DT, 4, 2, 16>(P, S, ring_it, ring, ph, l, tok, pos, t);
 }
 
 // --------------------------------------------------------------- consumer: epilogues
+
+__device__ __forceinline__ void attention_prefetch(const KieParams &P, int l, int sid, int pos);
 
 // q/k rows come in rotation pairs (dim i, dim i + D/2); v rows use the same pairing.
 template <int DT>
 __device__ void epilogue_qkv(const KieParams &P, B1Shared &S, int l, int sid, int pos, int tok) {
     const int D = P.D, half = D >> 1, qd = P.Hq * D, kvd = P.Hkv * D;
     const int rbeg = S.row0[PH_QKV], npair = (S.row1[PH_QKV] - rbeg) >> 1;
-    const float2 *rope = P.rope + (size_t)pos * half;
     const size_t sess = (size_t)sid * P.sess_stride;
     for (int p = threadIdx.x; p < npair; p += KIE_CONS_THREADS) {
         const int r = rbeg + 2 * p;
-        float a = S.rowacc[2 * p], b = S.rowacc[2 * p + 1];
-        S.rowacc[2 * p] = 0.f;
-        S.rowacc[2 * p + 1] = 0.f;
+        const int cs = col_slices(P.K[PH_QKV]);
+        const float a = rowsum(S, 2 * p, cs), b = rowsum(S, 2 * p + 1, cs);
         const int i = (r % D) >> 1;
         if (r < qd + kvd) {
-            const float2 cs = rope[i];
+            const float2 cs = S.rope_s[i];
             const float ra = a * cs.x - b * cs.y, rb = b * cs.x + a * cs.y;
             if (r < qd) {
                 const int hh = r / D;
@@ -304,31 +434,64 @@ __device__ void epilogue_qkv(const KieParams &P, B1Shared &S, int l, int sid, in
         }
     }
     if (l == 0) {  // the residual starts as the embedding row (rows this CTA owns in the O phase)
-        for (int r = S.row0[PH_O] + threadIdx.x; r < S.row1[PH_O]; r += KIE_CONS_THREADS)
-            P.x[r] = cvt1<DT>(P.emb[(size_t)tok * P.d + r]);
+        for (int r = S.row0[PH_O] + threadIdx.x; r < S.row1[PH_O]; r += KIE_CONS_THREADS) {
+            const float v = cvt1<DT>(P.emb[(size_t)tok * P.d + r]);
+            S.xown[r - S.row0[PH_O]] = v;
+            P.x[r] = v;
+        }
+    }
+    if (l == 0) attention_prefetch(P, l, sid, pos);
+}
+
+// The cache rows this CTA's attention units will read in layer l start moving into L2
+// (older positions are final; L2 stays coherent for the one written in this token).
+__device__ __forceinline__ void attention_prefetch(const KieParams &P, int l, int sid, int pos) {
+    const int D = P.D;
+    const size_t sess = (size_t)sid * P.sess_stride;
+    {
+        const int ctx = pos + 1;
+        for (int unit = blockIdx.x; unit < P.Hkv * P.splits; unit += P.nblk) {
+            const int g = unit / P.splits, s = unit % P.splits;
+            const long long p0 = (long long)s * ctx / P.splits, p1 = (long long)(s + 1) * ctx / P.splits;
+            const size_t off = sess + ((size_t)(l * P.Hkv + g) * P.max_ctx + p0) * D;
+            const int lines = (int)(((p1 - p0) * D * 2 + 127) / 128);
+            for (int j = threadIdx.x; j < 2 * lines; j += KIE_CONS_THREADS) {
+                const uint16_t *base = (j < lines ? P.kcache : P.vcache) + off;
+                prefetch_l2(reinterpret_cast<const uint8_t *>(base) + (size_t)(j % lines) * 128);
+            }
+        }
     }
 }
 
+// x += row sums on the rows this CTA owns; per-warp sums of squares of the new rows
 __device__ void epilogue_residual(const KieParams &P, B1Shared &S, int ph) {
     const int rbeg = S.row0[ph], n = S.row1[ph] - rbeg;
+    float ss = 0.f;
     for (int r = threadIdx.x; r < n; r += KIE_CONS_THREADS) {
-        P.x[rbeg + r] = __ldcg(P.x + rbeg + r) + S.rowacc[r];
-        S.rowacc[r] = 0.f;
+        const float v = S.xown[r] + rowsum(S, r, col_slices(P.K[ph]));
+        S.xown[r] = v;
+        P.x[rbeg + r] = v;
+        ss += v * v;
     }
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) S.ssqw[threadIdx.x >> 5] = ss;
 }
 
-__device__ void epilogue_gu(const KieParams &P, B1Shared &S) {
+__device__ void epilogue_gu(const KieParams &P, B1Shared &S, int l, int sid, int pos) {
+    if (l + 1 < P.L) attention_prefetch(P, l + 1, sid, pos);
     const int rbeg = S.row0[PH_GU], npair = (S.row1[PH_GU] - rbeg) >> 1;
     for (int p = threadIdx.x; p < npair; p += KIE_CONS_THREADS) {
-        const float g = S.rowacc[2 * p], up = S.rowacc[2 * p + 1];
-        S.rowacc[2 * p] = 0.f;
-        S.rowacc[2 * p + 1] = 0.f;
+        const int cs = col_slices(P.K[PH_GU]);
+        const float g = rowsum(S, 2 * p, cs), up = rowsum(S, 2 * p + 1, cs);
         P.u[(rbeg >> 1) + p] = g / (1.f + expf(-g)) * up;
     }
 }
 
 __device__ __forceinline__ void argmax_combine(float &v, int &i, float v2, int i2) {
-    if (v2 > v || (v2 == v && i2 < i)) { v = v2; i = i2; }
+    if (v2 > v || (v2 == v && i2 < i)) {
+        v = v2;
+        i = i2;
+    }
 }
 
 __device__ void warp_argmax(float &v, int &i) {
@@ -347,39 +510,36 @@ __device__ void epilogue_head(const KieParams &P, B1Shared &S, float *logits) {
     float bv = -CUDART_INF_F;
     int bi = 0x7fffffff;
     for (int r = tid; r < n; r += KIE_CONS_THREADS) {
-        const float v = S.rowacc[r];
-        S.rowacc[r] = 0.f;
+        const float v = rowsum(S, r, col_slices(P.K[PH_HEAD]));
         if (logits) logits[rbeg + r] = v;
         argmax_combine(bv, bi, v, rbeg + r);
     }
     warp_argmax(bv, bi);
-    if (lane == 0) { S.red[w] = bv; S.redi[w] = bi; }
+    if (lane == 0) {
+        S.red[w] = bv;
+        S.redi[w] = bi;
+    }
     named_bar_sync(1, KIE_CONS_THREADS);
     if (w == 0) {
         float v = lane < KIE_CONS_WARPS ? S.red[lane] : -CUDART_INF_F;
         int i = lane < KIE_CONS_WARPS ? S.redi[lane] : 0x7fffffff;
         warp_argmax(v, i);
-        if (lane == 0) { P.cand_val[blockIdx.x] = v; P.cand_idx[blockIdx.x] = i; }
+        if (lane == 0) {
+            P.cand_val[blockIdx.x] = v;
+            P.cand_idx[blockIdx.x] = i;
+        }
     }
 }
 
-// after the head barrier: every CTA reduces all candidates to the same token
-__device__ int final_argmax(const KieParams &P, B1Shared &S) {
-    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+// after the head barrier: every warp of every CTA reduces all candidates to the same
+// token, so no further barrier is needed
+__device__ int final_argmax(const KieParams &P) {
+    const int lane = threadIdx.x & 31;
     float v = -CUDART_INF_F;
     int i = 0x7fffffff;
-    for (int c = tid; c < P.nblk; c += KIE_CONS_THREADS) argmax_combine(v, i, __ldcg(P.cand_val + c), __ldcg(P.cand_idx + c));
+    for (int c = lane; c < P.nblk; c += 32) argmax_combine(v, i, __ldcg(P.cand_val + c), __ldcg(P.cand_idx + c));
     warp_argmax(v, i);
-    if (lane == 0) { S.red[w] = v; S.redi[w] = i; }
-    named_bar_sync(1, KIE_CONS_THREADS);
-    if (w == 0) {
-        v = lane < KIE_CONS_WARPS ? S.red[lane] : -CUDART_INF_F;
-        i = lane < KIE_CONS_WARPS ? S.redi[lane] : 0x7fffffff;
-        warp_argmax(v, i);
-        if (lane == 0) S.token = i;
-    }
-    named_bar_sync(1, KIE_CONS_THREADS);
-    return S.token;
+    return i;
 }
 
 // --------------------------------------------------------------- consumer: attention
@@ -398,15 +558,17 @@ __device__ void attention_layer(const KieParams &P, B1Shared &S, int l, int sid,
     A.Hkv = P.Hkv;
     A.nsplit = P.splits;
     A.ctx = pos + 1;
-    attn_all_units<DT>(A, S.at, P.G, blockIdx.x, P.nblk);
+    attn_all_units<DT, KIE_CONS_WARPS>(A, S.at, P.G, blockIdx.x, P.nblk);
 }
 
 // --------------------------------------------------------------- consumer: one command
 
 template <int DT>
-__device__ void consume(const KieParams &P, B1Shared &S, Ring &R, const KieCmd &cmd, unsigned long long &epoch) {
+__device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring, const KieCmd &cmd,
+                        unsigned long long &epoch) {
     int tok = cmd.in_tok;
     if (cmd.op == OP_DECODE && cmd.tok_dev) tok = __ldcg(cmd.tok_dev);
+    const int L = P.L;
     for (int t = 0; t < cmd.n; t++) {
         const int pos = cmd.pos0 + t;
         if (cmd.op == OP_PREFILL) tok = __ldcg(P.tokbuf + t);
@@ -414,32 +576,52 @@ __device__ void consume(const KieParams &P, B1Shared &S, Ring &R, const KieCmd &
             if (threadIdx.x == 0) set_error(P.err, DERR_BAD_TOKEN, 0);
             S.abort = 1;
         }
+        if (threadIdx.x == 0) S.wait_cons = 0;
+        trace_mark(P, t, 0);
         const bool head = (cmd.op != OP_PREFILL) || (t == cmd.n - 1);
-        for (int l = 0; l < P.L; l++) {
-            gemv_dispatch<DT>(P, S, R, PH_QKV, l, tok);
+        for (int l = 0; l < L; l++) {
+            const int e = 1 + 16 * l;
+            gemv_dispatch<DT>(P, S, ring_it, ring, PH_QKV, l, tok, pos, t);
+            trace_mark(P, t, e);
             epilogue_qkv<DT>(P, S, l, cmd.sid, pos, tok);
+            trace_mark(P, t, e + 1);
             grid_barrier(P, S, epoch, P.timeout_ns, 1);
+            trace_mark(P, t, e + 2);
             if (!S.abort) attention_layer<DT>(P, S, l, cmd.sid, pos);
+            trace_mark(P, t, e + 3);
             grid_barrier(P, S, epoch, P.timeout_ns, 2);
-            gemv_dispatch<DT>(P, S, R, PH_O, l, tok);
+            trace_mark(P, t, e + 4);
+            gemv_dispatch<DT>(P, S, ring_it, ring, PH_O, l, tok, pos, t);
             epilogue_residual(P, S, PH_O);
-            grid_barrier(P, S, epoch, P.timeout_ns, 3);
-            gemv_dispatch<DT>(P, S, R, PH_GU, l, tok);
-            epilogue_gu(P, S);
+            trace_mark(P, t, e + 5);
+            grid_barrier(P, S, epoch, P.timeout_ns, 3, true);
+            trace_mark(P, t, e + 6);
+            gemv_dispatch<DT>(P, S, ring_it, ring, PH_GU, l, tok, pos, t);
+            epilogue_gu(P, S, l, cmd.sid, pos);
+            trace_mark(P, t, e + 7);
             grid_barrier(P, S, epoch, P.timeout_ns, 4);
-            gemv_dispatch<DT>(P, S, R, PH_DOWN, l, tok);
+            trace_mark(P, t, e + 8);
+            gemv_dispatch<DT>(P, S, ring_it, ring, PH_DOWN, l, tok, pos, t);
             epilogue_residual(P, S, PH_DOWN);
-            grid_barrier(P, S, epoch, P.timeout_ns, 5);
+            trace_mark(P, t, e + 9);
+            grid_barrier(P, S, epoch, P.timeout_ns, 5, true);
+            trace_mark(P, t, e + 10);
         }
+        const int eh = 1 + 16 * L;
         if (head) {
-            gemv_dispatch<DT>(P, S, R, PH_HEAD, P.L, tok);
+            gemv_dispatch<DT>(P, S, ring_it, ring, PH_HEAD, L, tok, pos, t);
             float *lg = nullptr;
             if (cmd.logits) lg = cmd.logits + (cmd.op == OP_PREFILL ? 0 : (size_t)t * P.V);
             epilogue_head(P, S, lg);
+            trace_mark(P, t, eh);
             grid_barrier(P, S, epoch, P.timeout_ns, 6);
-            tok = final_argmax(P, S);
+            trace_mark(P, t, eh + 1);
+            tok = final_argmax(P);
             if (blockIdx.x == 0 && threadIdx.x == 0 && cmd.out) cmd.out[cmd.op == OP_PREFILL ? 0 : t] = tok;
+            trace_mark(P, t, eh + 2);
         }
+        if (P.trace && t < P.trace_tokens && threadIdx.x == 0)
+            P.trace[((size_t)blockIdx.x * P.trace_tokens + t) * P.trace_events + P.trace_events - 2] = S.wait_cons;
     }
 }
 
@@ -453,20 +635,18 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
     if (tid == 0) {
         for (int i = 0; i < KIE_NSLOT; i++) {
             mbar_init(&S.full[i], 1);
-            mbar_init(&S.empty[i], KIE_CONS_WARPS);
+            mbar_init(&S.empty[i], KIE_CONS_WARPS);  // both groups read every chunk
         }
         fence_mbar_init();
         S.abort = 0;
     }
-    for (int i = tid; i < KIE_ROWACC_MAX; i += KIE_THREADS) S.rowacc[i] = 0.f;
-    attn_smem_init(S.at, tid, KIE_THREADS);
     if (tid < KIE_NPH) {
         S.row0[tid] = P.row0[tid * (P.nblk + 1) + blockIdx.x];
         S.row1[tid] = P.row0[tid * (P.nblk + 1) + blockIdx.x + 1];
     }
     __syncthreads();
 
-    Ring R{smem, 0};
+    uint32_t ring_it = 0;  // chunks consumed (consumers) / issued (producer); both advance identically
     unsigned long long epoch = 0;
     for (;;) {
         if (tid < KIE_CONS_THREADS) {
@@ -511,9 +691,9 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
         const KieCmd cmd = S.cmd;
         if (cmd.op != OP_DECODE && cmd.op != OP_PREFILL) break;
         if (tid >= KIE_CONS_THREADS) {
-            if (tid == KIE_CONS_THREADS) produce(P, S, R, cmd);
+            if (tid == KIE_CONS_THREADS) produce(P, S, ring_it, smem, cmd);
         } else {
-            consume<DT>(P, S, R, cmd, epoch);
+            consume<DT>(P, S, ring_it, smem, cmd, epoch);
         }
         __syncthreads();
         if (resident && blockIdx.x == 0 && tid == 0) {
@@ -533,14 +713,15 @@ extern "C++" {
 
 size_t kie_b1_smem_bytes() { return RING_BYTES + sizeof(B1Shared); }
 
-int kie_b1_vec_per_lane(int K) { return vec_per_lane(K); }
+// rows per ring chunk for row length K, and the most rows one CTA may own in such a phase
+int kie_b1_chunk_rows(int K) { return (KIE_CONS_WARPS / col_slices(K)) * rows_per_group(K); }
+int kie_b1_max_rows(int K) { return WPART_FLOATS / col_slices(K); }
 
 cudaError_t kie_b1_prepare(int dtype) {
-    const size_t smem = kie_b1_smem_bytes();
-    cudaError_t e = dtype == KIE_BF16
-                        ? cudaFuncSetAttribute(kie_b1_kernel<KIE_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
-                        : cudaFuncSetAttribute(kie_b1_kernel<KIE_FP16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    return e;
+    const int smem = (int)kie_b1_smem_bytes();
+    return dtype == KIE_BF16
+               ? cudaFuncSetAttribute(kie_b1_kernel<KIE_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+               : cudaFuncSetAttribute(kie_b1_kernel<KIE_FP16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
 }
 
 cudaError_t kie_b1_occupancy(int dtype, int *blocks_per_sm) {

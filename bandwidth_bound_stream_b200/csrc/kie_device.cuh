@@ -100,24 +100,35 @@ KIE_DEV void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
                  : "memory");
 }
 
+// Hint: bring the 128-byte line holding p into L2 (through the load/store unit).
+KIE_DEV void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
+// Hint: bring [src, src + bytes) into L2 (no completion tracking). bytes a multiple of 16.
+KIE_DEV void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ------------------------------------------------------------------ storage types
+
+// two stored elements packed in a 32-bit word -> two floats (low half first)
+template <int DT>
+KIE_DEV void cvt2(uint32_t w, float &lo, float &hi) {
+    if (DT == KIE_BF16) {
+        lo = __uint_as_float(w << 16);
+        hi = __uint_as_float(w & 0xFFFF0000u);
+    } else {
+        lo = __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu)));
+        hi = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+    }
+}
 
 // 8 stored elements (one 16-byte vector) -> 8 floats.
 template <int DT>
 KIE_DEV void cvt8(const uint4 &v, float *f) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        if (DT == KIE_BF16) {
-            f[2 * i] = __uint_as_float(w[i] << 16);
-            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-        } else {
-            __half2 h = *reinterpret_cast<const __half2 *>(&w[i]);
-            float2 t = __half22float2(h);
-            f[2 * i] = t.x;
-            f[2 * i + 1] = t.y;
-        }
-    }
+    cvt2<DT>(v.x, f[0], f[1]);
+    cvt2<DT>(v.y, f[2], f[3]);
+    cvt2<DT>(v.z, f[4], f[5]);
+    cvt2<DT>(v.w, f[6], f[7]);
 }
 
 template <int DT>

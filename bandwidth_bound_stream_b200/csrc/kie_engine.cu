@@ -23,7 +23,8 @@
 
 // kernels of the other translation units
 size_t kie_b1_smem_bytes();
-int kie_b1_vec_per_lane(int K);
+int kie_b1_chunk_rows(int K);
+int kie_b1_max_rows(int K);
 cudaError_t kie_b1_prepare(int dtype);
 cudaError_t kie_b1_occupancy(int dtype, int *blocks_per_sm);
 cudaError_t kie_b1_launch(const KieParams &P, const KieCmd &one, int resident, cudaStream_t stream);
@@ -114,6 +115,7 @@ extern "C" void kie_config_defaults(kie_config *c) {
     c->idle_ms = 200;
     c->modes = KIE_MODE_BATCH1;
     c->device = 0;
+    c->prefetch_kb = 0;
 }
 
 extern "C" const char *kie_status_string(kie_status s) {
@@ -150,10 +152,13 @@ static const char *shape_error(const kie_config &c) {
     if (c.n_heads % c.n_kv_heads || c.n_heads / c.n_kv_heads > KIE_GMAX)
         return "n_heads must be a multiple of n_kv_heads, at most 8 query heads per kv head";
     if (c.d_model > 8192) return "d_model above 8192 is not supported";
-    if (c.ffn > 16384 || c.n_heads * c.head_dim > 16384) return "ffn and n_heads*head_dim must be <= 16384";
+    if (c.ffn > 14336 || c.n_heads * c.head_dim > 14336) return "ffn and n_heads*head_dim must be <= 14336";
+    if ((c.ffn > 8192 && c.ffn % 128) || (c.n_heads * c.head_dim > 8192 && (c.n_heads * c.head_dim) % 128))
+        return "ffn and n_heads*head_dim above 8192 must be multiples of 128";
     if (c.max_sessions <= 0 || c.max_ctx <= 0) return "max_sessions and max_ctx must be positive";
     if (c.timeout_ms <= 0 || c.idle_ms <= 0) return "timeouts must be positive";
     if (!(c.modes & (KIE_MODE_BATCH1 | KIE_MODE_TICK))) return "modes must enable at least one kernel";
+    if (c.prefetch_kb < 0 || c.prefetch_kb > 65536) return "prefetch_kb must be in [0, 65536]";
     return nullptr;
 }
 
@@ -230,25 +235,21 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
     partition(&row0[PH_HEAD * (nblk + 1)], V, 1, nblk);
     for (int ph = 0; ph < KIE_NPH; ph++) {
         P.K[ph] = Kph[ph];
-        const int nv = kie_b1_vec_per_lane(Kph[ph]);
-        P.cr[ph] = nv == 1 ? 8 : nv == 2 ? 4 : nv == 4 ? 2 : 1;
-        if ((ph == PH_QKV || ph == PH_GU) && P.cr[ph] < 2) {
-            eng->fail(KIE_ERR_ARG, "paired rows need two rows per chunk");
+        P.cr[ph] = kie_b1_chunk_rows(Kph[ph]);  // rows per ring chunk (even for the paired phases)
+        if (ph == PH_O && (d + nblk - 1) / nblk > KIE_XOWN_MAX) {
+            eng->fail(KIE_ERR_ARG, "d_model too large for %d SMs", nblk);
             return bail(KIE_ERR_ARG);
         }
+        const int max_rows = kie_b1_max_rows(Kph[ph]);
         for (int cc = 0; cc < nblk; cc++)
-            if (row0[ph * (nblk + 1) + cc + 1] - row0[ph * (nblk + 1) + cc] > KIE_ROWACC_MAX) {
-                eng->fail(KIE_ERR_ARG, "phase %d gives a CTA more than %d rows", ph, KIE_ROWACC_MAX);
+            if (row0[ph * (nblk + 1) + cc + 1] - row0[ph * (nblk + 1) + cc] > max_rows) {
+                eng->fail(KIE_ERR_ARG, "phase %d gives a CTA more than %d rows", ph, max_rows);
                 return bail(KIE_ERR_ARG);
             }
     }
-    // attention splits: about one unit per CTA, and no split longer than the score buffer
-    {
-        int s = std::max(1, nblk / Hkv);
-        const int cap = KIE_SCORE_MAX / G;
-        s = std::max(s, (c.max_ctx + cap - 1) / cap);
-        P.splits = s;
-    }
+    // attention splits: about one (kv head, split) unit per CTA
+    P.splits = std::max(1, nblk / Hkv);
+    P.pf_chunks = (int)(((long long)c.prefetch_kb * 1024 + KIE_SLOT_BYTES - 1) / KIE_SLOT_BYTES);
 
     // ---- packed weights: CTA c's stream is one contiguous segment
     std::vector<long long> seg_off(nblk + 1, 0);
@@ -356,6 +357,8 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
     CK(eng->alloc(&P.err, 16), "cudaMalloc error word");
     CK(eng->alloc(&P.last_seq, 16), "cudaMalloc sequence");
     CK(eng->alloc(&P.cmd, sizeof(KieCmd)), "cudaMalloc command");
+    CK(eng->alloc(&P.ssq, (size_t)nblk * 4), "cudaMalloc norm partials");
+    CK(cudaMemset(P.ssq, 0, (size_t)nblk * 4), "memset");
     CK(cudaMemset(P.cnt, 0, (size_t)Hkv * 4), "memset");
     CK(cudaMemset(P.bar, 0, 16), "memset");
     CK(cudaMemset(P.err, 0, 16), "memset");
@@ -487,6 +490,7 @@ extern "C" void kie_destroy(kie_engine *eng) {
     if (!eng->poisoned && eng->stream) stop_resident(eng);
     if (eng->stream) cudaStreamSynchronize(eng->stream);
     for (void *p : eng->dev_allocs) cudaFree(p);
+    if (eng->P.trace) cudaFree(eng->P.trace);
     if (eng->mbox_host) cudaFreeHost(eng->mbox_host);
     if (eng->ev_done) cudaEventDestroy(eng->ev_done);
     if (eng->stream) cudaStreamDestroy(eng->stream);
@@ -671,4 +675,50 @@ extern "C" kie_status kie_tick(kie_engine *eng, int32_t n_sess, const int32_t *s
     (void)n_sess; (void)sids; (void)in_tokens; (void)steps; (void)out_tokens; (void)logits_dev;
     if (!(eng->cfg.modes & KIE_MODE_TICK)) return eng->fail(KIE_ERR_UNSUPPORTED, "engine built without KIE_MODE_TICK");
     return KIE_ERR_UNSUPPORTED;
+}
+
+// ---------------------------------------------------------------- phase trace
+
+extern "C" int32_t kie_trace_events(kie_engine *eng) {
+    if (!eng) return 0;
+    return 1 + 16 * eng->cfg.n_layers + 3 + 2;
+}
+
+extern "C" kie_status kie_trace_enable(kie_engine *eng, int32_t tokens) {
+    kie_status s = check_live(eng);
+    if (s != KIE_OK) return s;
+    if (tokens < 0 || tokens > 4096) return eng->fail(KIE_ERR_ARG, "trace tokens must be in [0, 4096]");
+    if ((s = stop_resident(eng)) != KIE_OK) return s;
+    cudaDeviceSynchronize();
+    if (eng->P.trace) {
+        cudaFree(eng->P.trace);
+        eng->P.trace = nullptr;
+    }
+    eng->P.trace_tokens = tokens;
+    eng->P.trace_events = kie_trace_events(eng);
+    if (tokens > 0) {
+        const size_t n = (size_t)eng->nblk * tokens * eng->P.trace_events;
+        cudaError_t e = cudaMalloc(&eng->P.trace, n * 8);
+        if (e == cudaSuccess) e = cudaMemset(eng->P.trace, 0, n * 8);
+        if (e != cudaSuccess) {
+            eng->P.trace = nullptr;
+            eng->P.trace_tokens = 0;
+            return eng->cuda_fail(e, "trace buffer");
+        }
+    }
+    return KIE_OK;
+}
+
+extern "C" kie_status kie_trace_read(kie_engine *eng, uint64_t *host, int64_t max_elems, int64_t *n) {
+    kie_status s = check_live(eng);
+    if (s != KIE_OK) return s;
+    if (!n || (!host && max_elems > 0)) return KIE_ERR_ARG;
+    const int64_t total = eng->P.trace ? (int64_t)eng->nblk * eng->P.trace_tokens * eng->P.trace_events : 0;
+    *n = total;
+    if (!total || max_elems <= 0) return KIE_OK;
+    if ((s = stop_resident(eng)) != KIE_OK) return s;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess)
+        e = cudaMemcpy(host, eng->P.trace, (size_t)std::min(total, max_elems) * 8, cudaMemcpyDeviceToHost);
+    return e == cudaSuccess ? KIE_OK : eng->cuda_fail(e, "reading the trace");
 }

@@ -5,15 +5,15 @@
 #include "kie.h"
 
 #define KIE_MAX_CTAS 256
-#define KIE_CONS_WARPS 8                      // consumer warps per CTA (batch-1 kernel)
+#define KIE_CONS_WARPS 16                     // consumer warps per CTA (batch-1 kernel): two groups of 8
 #define KIE_CONS_THREADS (KIE_CONS_WARPS * 32)
 #define KIE_THREADS (KIE_CONS_THREADS + 32)   // + one producer warp
-#define KIE_NSLOT 6                           // weight ring depth
-#define KIE_SLOT_BYTES 32768                  // one ring slot
+#define KIE_NSLOT 3                           // weight ring depth
+#define KIE_SLOT_BYTES 65536                  // one ring slot (large bulk copies stream best)
 #define KIE_ROWACC_MAX 1024                   // output rows one CTA may own in one phase
-#define KIE_SCORE_MAX 4096                    // attention scores one split may hold (floats)
 #define KIE_GMAX 8                            // query heads per kv head
 #define KIE_DMAX 128                          // head_dim
+#define KIE_XOWN_MAX 64                       // residual rows one CTA may own (d_model / SMs)
 
 // Phases of the batch-1 weight stream, in stream order within a layer; the LM head follows the last layer.
 enum { PH_QKV = 0, PH_O = 1, PH_GU = 2, PH_DOWN = 3, PH_HEAD = 4, KIE_NPH = 5 };
@@ -83,6 +83,10 @@ struct KieParams {
     unsigned *last_seq;             // last doorbell sequence processed
     KieCmd *cmd;                    // command broadcast slot
     long long timeout_ns, idle_ns;
+    int pf_chunks;                  // L2 prefetch lead of the weight stream, in ring chunks
+    float *ssq;                     // [nblk] per-CTA sums of squares of the residual rows it owns
+    unsigned long long *trace;      // phase stamps (null = off)
+    int trace_tokens, trace_events;
 };
 
 #ifdef __cplusplus

@@ -24,7 +24,8 @@ KIE_MODE_BATCH1, KIE_MODE_TICK = 1, 2
 EXPORTS = ("kie_config_defaults", "kie_create", "kie_destroy", "kie_session_open", "kie_session_close",
            "kie_session_length", "kie_session_rewind", "kie_session_kv", "kie_prefill", "kie_decode_step",
            "kie_generate", "kie_decode_launch", "kie_sync", "kie_tick", "kie_last_error", "kie_status_string",
-           "kie_flash_decode", "kie_flash_decode_scratch_bytes")
+           "kie_flash_decode", "kie_flash_decode_scratch_bytes", "kie_trace_enable", "kie_trace_read",
+           "kie_trace_events")
 
 
 class KieConfig(ctypes.Structure):
@@ -32,7 +33,7 @@ class KieConfig(ctypes.Structure):
                                                "vocab")] + \
                [("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float)] + \
                [(n, ctypes.c_int32) for n in ("dtype", "max_sessions", "max_ctx", "timeout_ms", "idle_ms", "modes",
-                                               "device")]
+                                               "device", "prefetch_kb")]
 
 
 class KieWeights(ctypes.Structure):
@@ -71,6 +72,9 @@ def _load():
         "kie_status_string": (ctypes.c_char_p, [i32]),
         "kie_flash_decode": (i32, [vp, vp, vp, i32, i32, i32, i32, i64, i32, vp, vp, i64, vp]),
         "kie_flash_decode_scratch_bytes": (i64, [i32, i32, i32, i32]),
+        "kie_trace_enable": (i32, [vp, i32]),
+        "kie_trace_read": (i32, [vp, vp, i64, P(i64)]),
+        "kie_trace_events": (i32, [vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(h, name)
@@ -88,7 +92,7 @@ def _ptr(a: np.ndarray):
 
 
 def config(model, max_sessions: int = 1, max_ctx: int = 4096, timeout_ms: int = 10000, idle_ms: int = 200,
-           modes: int = KIE_MODE_BATCH1, device: int = 0) -> KieConfig:
+           modes: int = KIE_MODE_BATCH1, device: int = 0, prefetch_kb: int | None = None) -> KieConfig:
     """A kie_config for a model shape (any object with the shape attributes of synth.ModelConfig)."""
     c = KieConfig()
     lib.kie_config_defaults(ctypes.byref(c))
@@ -97,6 +101,8 @@ def config(model, max_sessions: int = 1, max_ctx: int = 4096, timeout_ms: int = 
     c.rms_eps, c.rope_theta = model.rms_eps, model.rope_theta
     c.max_sessions, c.max_ctx, c.timeout_ms, c.idle_ms, c.modes, c.device = (max_sessions, max_ctx, timeout_ms,
                                                                                 idle_ms, modes, device)
+    if prefetch_kb is not None:
+        c.prefetch_kb = prefetch_kb
     return c
 
 
@@ -177,6 +183,19 @@ class Engine:
                       logits_dev_ptr: int | None = None, stream_ptr: int | None = None):
         self._check(lib.kie_decode_launch(self.h, sid, in_tok_dev_ptr, n, out_dev_ptr, logits_dev_ptr, stream_ptr),
                     "kie_decode_launch")
+
+    def trace_enable(self, tokens: int):
+        self._check(lib.kie_trace_enable(self.h, tokens), "kie_trace_enable")
+
+    def trace_read(self, tokens: int) -> np.ndarray:
+        """Phase stamps as [cta][token][event] (uint64 ns; the last two events are ring wait totals)."""
+        ev = lib.kie_trace_events(self.h)
+        n = ctypes.c_int64()
+        self._check(lib.kie_trace_read(self.h, None, 0, ctypes.byref(n)), "kie_trace_read")
+        out = np.zeros(n.value, dtype=np.uint64)
+        if n.value:
+            self._check(lib.kie_trace_read(self.h, out.ctypes.data, n.value, ctypes.byref(n)), "kie_trace_read")
+        return out.reshape(-1, tokens, ev)
 
     def sync(self):
         self._check(lib.kie_sync(self.h), "kie_sync")

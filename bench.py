@@ -1,0 +1,344 @@
+#!/usr/bin/env python3
+"""Benchmark: batch-1 greedy decode of the ~1.9B dense decoder (fp16) on one B200 per rank.
+
+Workload (one "step"): the session holds a 1024-token prompt (prefilled once, before
+timing); a step rewinds it to those 1024 positions and decodes 512 greedy tokens in one
+launch of the persistent megakernel, the argmax fed back on the GPU. Every step streams
+all weights (3.65 GB per token) plus the KV cache, far more than the 126 MB L2, so no
+L2 flush is needed between steps.
+
+  value     tokens/s over all ranks, device-timed (CUDA events around each launch on the
+            launch stream, max over ranks)
+  e2e       the same through kie_generate with HOST buffers (doorbell: input token and
+            command in, 512 output tokens out), host clock
+  roofline  algorithmic bytes per launch / mean launch time, against the measured HBM peak
+  cpu_baseline  the CPU oracle's decode steps at this context length on the host cores
+
+Multi-GPU: launched under torchrun, each rank runs an independent replica on its own GPU
+(sessions do not shard a single decode; there is no data-path collective).
+``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "batch-1 decode tokens/s and HBM GB/s vs roofline; p99 tick latency at 56 sessions"
+PROMPT, DECODE = 1024, 512
+WORKLOAD = "dense-1.9b fp16 batch-1 decode: prompt 1024 uniform tokens, greedy decode 512 (28L d2048 16/8x128 F8192 V32000)"
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def algorithmic_bytes(model, ctx0: int, n: int) -> int:
+    """Bytes one launch must move: all weights except the embedding table plus one embedding row per token,
+    the KV cache read over the attended positions, and the new position's K/V write."""
+    per_pos = model.kv_bytes_per_position()
+    total = 0
+    for t in range(n):
+        attended = ctx0 + t + 1
+        total += model.weight_bytes_per_token() + attended * per_pos + per_pos
+    return total
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        import torch
+        p = torch.cuda.get_device_properties(device_index)
+        self.bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.bus, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], 0.0, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = max(mx, float(parts[1]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_baseline(model, host_weights, ctx0: int, min_s=10.0, max_s=30.0):
+    """Decode steps of the CPU oracle at the workload's context length (cache pre-sized, values zero)."""
+    from oracle.oracle import OracleModel, num_threads
+    orc = OracleModel(model, host_weights, ctx0 + 64)
+    orc.pos = ctx0
+    tok, steps = 1, 0
+    t0 = time.perf_counter()
+    while True:
+        lg = orc.step(tok)
+        tok = int(np.argmax(lg))
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= min_s or (steps >= 1 and el * (steps + 1) / steps > max_s):
+            break
+    return {"value": steps / el, "unit": "tokens/s", "cores": num_threads(), "kind": "oracle",
+            "sample": f"{steps} oracle decode steps of the full 1.9B model at positions {ctx0}..{ctx0 + steps - 1} "
+                      f"(KV cache of that length, zero contents: the per-step cost does not depend on the values)"}
+
+
+def dist_setup():
+    if "RANK" not in os.environ:
+        return 0, 1, 0
+    import torch
+    import torch.distributed as dist
+    rank, world = int(os.environ["RANK"]), int(os.environ["WORLD_SIZE"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    torch.cuda.set_device(local)
+    import datetime
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def run_reference(args, rank):
+    """The CPU oracle on this workload: each step is a bounded sample, one greedy decode token of the
+    full 1.9B model at the workload's mean context length, timed on the host cores."""
+    if rank != 0:
+        return
+    from bandwidth_bound_stream_b200 import synth
+    from oracle.oracle import OracleModel, num_threads
+    m = synth.DENSE_1P9B
+    ctx0 = PROMPT + DECODE // 2
+    orc = OracleModel(m, synth.model_weights(m), ctx0 + args.warmup + args.steps + 1)
+    orc.pos = ctx0
+    tok = 1
+    for _ in range(args.warmup):
+        tok = int(np.argmax(orc.step(tok)))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        tok = int(np.argmax(orc.step(tok)))
+    el = time.perf_counter() - t0
+    value = args.steps / el
+    sample = (f"{args.steps} timed oracle decode steps (after {args.warmup} warm-up) of the full 1.9B model at "
+              f"positions {ctx0 + args.warmup}.. (KV cache of that length, zero contents)")
+    cb = {"value": value, "unit": "tokens/s", "cores": num_threads(), "kind": "oracle", "sample": sample}
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD if headline else f"{m.name} batch-1: prompt {prompt_len}, decode {decode_n}",
+                   "prompt": prompt_len, "decode": decode_n, "batch": 1,
+                       "parallelism": "CPU oracle, OpenMP over output rows",
+                       "step": "one decode token of the workload per step (bounded sample)"},
+            "cpu_baseline": cb,
+            "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="engine", choices=["engine", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--model", default="dense-1.9b", help="workload shape (profiling cases use smaller ones)")
+    ap.add_argument("--prompt", type=int, default=PROMPT)
+    ap.add_argument("--decode", type=int, default=DECODE)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    rank, world, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    import torch
+
+    from bandwidth_bound_stream_b200 import kie, synth
+    m = synth.CONFIGS[args.model]
+    prompt_len, decode_n = args.prompt, args.decode
+    headline = (args.model == "dense-1.9b" and prompt_len == PROMPT and decode_n == DECODE)
+    dev = f"cuda:{local}"
+    torch.cuda.set_device(local)
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    dw = kie.DeviceWeights(m, seed=0, device=dev, host_copy=want_cpu)
+    prompt = synth.prompt(m, prompt_len)
+    eng = kie.Engine(kie.config(m, max_ctx=prompt_len + decode_n, timeout_ms=10000, idle_ms=200, device=local),
+                     dw.kie)
+    host_weights = dw.host
+    dw.free()  # the engine keeps its own repacked copy
+    torch.cuda.empty_cache()
+    sid = eng.session_open()
+    t0 = time.perf_counter()
+    first = eng.prefill(sid, prompt)
+    ttft_ms = (time.perf_counter() - t0) * 1e3
+
+    stream = torch.cuda.Stream(device=dev)
+    tok_d = torch.tensor([first], dtype=torch.int32, device=dev)
+    out_d = torch.zeros(decode_n, dtype=torch.int32, device=dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+
+    def launch():
+        eng.session_rewind(sid, prompt_len)
+        eng.decode_launch(sid, tok_d.data_ptr(), decode_n, out_d.data_ptr(), None, stream.cuda_stream)
+
+    for _ in range(args.warmup):
+        launch()
+    eng.sync()
+    ref_tokens = out_d.cpu().numpy().copy()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_all0 = torch.cuda.Event(enable_timing=True)
+    t_all1 = torch.cuda.Event(enable_timing=True)
+    t_all0.record(stream)
+    for i in range(args.steps):
+        starts[i].record(stream)
+        launch()
+        ends[i].record(stream)
+    t_all1.record(stream)
+    eng.sync()
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    barrier()
+    total_ms = t_all0.elapsed_time(t_all1)
+    per_launch = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    assert np.array_equal(out_d.cpu().numpy(), ref_tokens), "decode is not deterministic across launches"
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # end to end through the doorbell with host buffers
+    out_h = np.empty(decode_n, dtype=np.int32)
+    for _ in range(2):
+        eng.session_rewind(sid, prompt_len)
+        eng.generate(sid, first, decode_n, out_h)
+    barrier()
+    e0 = time.perf_counter()
+    for _ in range(args.steps):
+        eng.session_rewind(sid, prompt_len)
+        eng.generate(sid, first, decode_n, out_h)
+    e_s = time.perf_counter() - e0
+    assert np.array_equal(out_h, ref_tokens), "doorbell and launch paths disagree"
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([e_s], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_s = float(t.item())
+
+    # inter-token latency of single doorbell steps (host clock)
+    eng.session_rewind(sid, prompt_len)
+    itl = []
+    tok = first
+    for _ in range(min(64, decode_n)):
+        a = time.perf_counter()
+        tok = eng.decode_step(sid, tok)
+        itl.append((time.perf_counter() - a) * 1e3)
+    eng.close()
+
+    tokens = world * decode_n * args.steps
+    value = tokens / (total_ms / 1e3)
+    peak, peak_kind = measured_peaks()
+    bytes_launch = algorithmic_bytes(m, prompt_len, decode_n)
+    mean_launch_s = statistics.mean(per_launch) / 1e3
+    achieved = bytes_launch / mean_launch_s / 1e9
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic_b1_dense1p9b.json")
+    if os.path.exists(prof):
+        with open(prof) as f:
+            tr = json.load(f)
+        if headline and tr.get("kernel_rev") == kernel_revision():
+            traffic = tr.get("bytes_per_launch")
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
+        "config": {"workload": WORKLOAD if headline else f"{m.name} batch-1: prompt {prompt_len}, decode {decode_n}",
+                   "prompt": prompt_len, "decode": decode_n, "batch": 1,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (3.65 GB of weights streamed per token); no flush needed",
+                   "weights": "seeded N(0,0.02) fp16, norms 1"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": peak_kind,
+                     "bytes_per_launch": bytes_launch, "kernel": f"kie_b1_kernel (one launch = {decode_n} tokens)"},
+        "e2e": {"value": round(world * decode_n * args.steps / e_s, 2), "unit": "tokens/s",
+                "h2d_bytes_per_step": 4 + 80, "d2h_bytes_per_step": decode_n * 4 + 8,
+                "path": "kie_generate via the mapped-mailbox doorbell (host token + command in, host tokens out)"},
+        "gpu_launches": args.steps,
+        "clocks": clock_info,
+        "latency": {"ttft_ms": round(ttft_ms, 2), "itl_ms_p50": round(statistics.median(itl), 4),
+                    "itl_ms_p99": round(float(np.percentile(itl, 99)), 4),
+                    "per_launch_ms": [round(x, 3) for x in per_launch]},
+    }
+    if want_cpu:
+        line["cpu_baseline"] = oracle_baseline(m, host_weights, prompt_len + decode_n // 2)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def kernel_revision() -> str:
+    """Hash of the kernel sources (traffic counters are valid only for the revision they were taken on)."""
+    import hashlib
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "bandwidth_bound_stream_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.startswith("kie_b1") or name in ("kie_device.cuh", "kie_attn.cuh", "kie_internal.h"):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+if __name__ == "__main__":
+    main()

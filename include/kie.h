@@ -69,6 +69,8 @@ typedef struct {
     int32_t idle_ms;      /* the resident kernel exits after this long with no command */
     int32_t modes;        /* KIE_MODE_* bitmask                                        */
     int32_t device;       /* CUDA device ordinal                                       */
+    int32_t prefetch_kb;  /* per-SM lead of the weight stream requested into L2 ahead of
+                             the shared-memory ring, in KB (default 0 = ring only)       */
 } kie_config;
 
 /*
@@ -89,14 +91,15 @@ typedef struct {
 
 /* Fills a config with the shape fields zeroed and defaults for the rest
    (eps 1e-5, theta 1e4, fp16, 1 session, 4096 positions, timeouts 10 s / 200 ms,
-   batch-1 mode, device 0). */
+   batch-1 mode, device 0, no L2 lead). */
 void kie_config_defaults(kie_config *cfg);
 
 /*
  * Builds an engine: validates the shape, allocates every device buffer it will ever use
  * (packed weights, KV cache of max_sessions x max_ctx, activations, split-K scratch,
  * mapped host mailbox), computes the static work partition for this GPU's SM count and
- * repacks the weights. Constraints: d_model, n_heads*head_dim and ffn multiples of 64;
+ * repacks the weights. Constraints: d_model, n_heads*head_dim and ffn multiples of 64,
+ * d_model <= 8192, ffn and n_heads*head_dim <= 14336;
  * head_dim even and <= 128; n_heads a multiple of n_kv_heads with n_heads/n_kv_heads <= 8.
  * Errors: KIE_ERR_ARG (shape), KIE_ERR_CUDA (allocation or launch). On error *out is NULL.
  */
@@ -159,6 +162,22 @@ kie_status kie_sync(kie_engine *eng);
  */
 kie_status kie_tick(kie_engine *eng, int32_t n_sess, const int32_t *sids, const int32_t *in_tokens, int32_t steps,
                     int32_t *out_tokens, float *logits_dev);
+
+/*
+ * Phase trace (observability). kie_trace_enable(eng, tokens) makes every later decode
+ * command record, for its first `tokens` tokens, a globaltimer stamp (ns) per CTA at each
+ * phase boundary, plus per-token ring wait totals; tokens = 0 turns it off. kie_trace_read
+ * copies the record into `host` (uint64, at most max_elems) and returns the element count
+ * through *n; layout [cta][token][event], events per token = kie_trace_events(eng):
+ *   0: token start; then per layer 16 slots: 11 phase ends (QKV rows, QKV epilogue, barrier,
+ *   attention, barrier, O rows+epilogue, barrier, gate/up rows+epilogue, barrier, down
+ *   rows+epilogue, barrier) and 5 inner stamps (input vectors ready in the QKV, O, gate/up
+ *   and down phases; attention loads done); then 3 for the head (rows+argmax, barrier, final
+ *   argmax); then the consumer's and the producer's total ring wait in ns.
+ */
+kie_status kie_trace_enable(kie_engine *eng, int32_t tokens);
+kie_status kie_trace_read(kie_engine *eng, uint64_t *host, int64_t max_elems, int64_t *n);
+int32_t kie_trace_events(kie_engine *eng);
 
 /* Copies the engine's last error message (NUL-terminated, truncated to len). */
 kie_status kie_last_error(kie_engine *eng, char *buf, int32_t len);
