@@ -70,3 +70,59 @@ extern "C" kie_status kie_flash_decode(const float *q_dev, const void *k_dev, co
     else flash_decode_kernel<KIE_FP16><<<grid, FD_WARPS * 32, 0, s>>>(A, G);
     return cudaGetLastError() == cudaSuccess ? KIE_OK : KIE_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------------------------------
+// Allocation-free variant of kie_flash_decode.
+//
+// Some callers must not allocate device memory while they run: code that works inside a
+// memory budget fixed at start-up (no allocator after initialisation, as in a resident
+// serving loop), code whose device memory belongs to another framework's allocator, and
+// latency-critical loops where cudaMalloc/cudaFree would stall the device. They call this
+// entry point instead: the split partials and merge counters live in one static device
+// array of KIE_FLASH_DECODE_NOALLOC_MAX_BYTES that every GPU loading this library keeps
+// until the process exits.
+// ---------------------------------------------------------------------------------------
+
+#include <mutex>
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[KIE_FLASH_DECODE_NOALLOC_MAX_BYTES];
+
+constexpr int NOALLOC_MAX_DEVICES = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[NOALLOC_MAX_DEVICES];  // device address of the array, per device (set up once)
+
+// The host-side symbol is only a stand-in: the kernel needs the array's device address,
+// looked up once per device with that device current.
+cudaError_t noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" kie_status kie_flash_decode_noalloc(const float *q_dev, const void *k_dev, const void *v_dev,
+                                               int32_t n_heads, int32_t n_kv_heads, int32_t head_dim, int32_t n_ctx,
+                                               int64_t kv_stride, int32_t dtype, float *out_dev, void *stream) {
+    if (!fd_shape_ok(n_heads, n_kv_heads, head_dim, n_ctx, dtype) || kv_stride < n_ctx) return KIE_ERR_ARG;
+    if (!q_dev || !k_dev || !v_dev || !out_dev) return KIE_ERR_ARG;
+    const int64_t need = kie_flash_decode_scratch_bytes(n_heads, n_kv_heads, head_dim, n_ctx);
+    if (need > (int64_t)KIE_FLASH_DECODE_NOALLOC_MAX_BYTES) return KIE_ERR_CAPACITY;
+    void *scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) return KIE_ERR_CUDA;
+    // the same launch as kie_flash_decode, with the static array as its scratch
+    return kie_flash_decode(q_dev, k_dev, v_dev, n_heads, n_kv_heads, head_dim, n_ctx, kv_stride, dtype, out_dev,
+                            scratch, (int64_t)KIE_FLASH_DECODE_NOALLOC_MAX_BYTES, stream);
+}

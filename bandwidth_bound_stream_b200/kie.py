@@ -25,7 +25,7 @@ EXPORTS = ("kie_config_defaults", "kie_create", "kie_destroy", "kie_session_open
            "kie_session_length", "kie_session_rewind", "kie_session_kv", "kie_prefill", "kie_decode_step",
            "kie_generate", "kie_decode_launch", "kie_sync", "kie_tick", "kie_last_error", "kie_status_string",
            "kie_flash_decode", "kie_flash_decode_scratch_bytes", "kie_trace_enable", "kie_trace_read",
-           "kie_trace_events")
+           "kie_trace_events", "kie_flash_decode_noalloc")
 
 
 class KieConfig(ctypes.Structure):
@@ -75,6 +75,7 @@ def _load():
         "kie_trace_enable": (i32, [vp, i32]),
         "kie_trace_read": (i32, [vp, vp, i64, P(i64)]),
         "kie_trace_events": (i32, [vp]),
+        "kie_flash_decode_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, i64, i32, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(h, name)
@@ -212,6 +213,16 @@ def flash_decode(q_ptr, k_ptr, v_ptr, n_heads, n_kv_heads, head_dim, n_ctx, kv_s
                  scratch_ptr, scratch_bytes, stream_ptr=None) -> int:
     return lib.kie_flash_decode(q_ptr, k_ptr, v_ptr, n_heads, n_kv_heads, head_dim, n_ctx, kv_stride, dtype,
                                 out_ptr, scratch_ptr, scratch_bytes, stream_ptr)
+
+
+def flash_decode_noalloc(q_ptr, k_ptr, v_ptr, n_heads, n_kv_heads, head_dim, n_ctx, kv_stride, dtype, out_ptr,
+                         stream_ptr=None) -> int:
+    """kie_flash_decode with its scratch in the library's static device array (allocates nothing)."""
+    return lib.kie_flash_decode_noalloc(q_ptr, k_ptr, v_ptr, n_heads, n_kv_heads, head_dim, n_ctx, kv_stride, dtype,
+                                        out_ptr, stream_ptr)
+
+
+FLASH_DECODE_NOALLOC_MAX_BYTES = 4 << 20
 
 
 def flash_decode_scratch_bytes(n_heads, n_kv_heads, head_dim, n_ctx) -> int:

@@ -202,6 +202,32 @@ kie_status kie_flash_decode(const float *q_dev, const void *k_dev, const void *v
                             float *out_dev, void *scratch_dev, int64_t scratch_bytes, void *stream);
 int64_t kie_flash_decode_scratch_bytes(int32_t n_heads, int32_t n_kv_heads, int32_t head_dim, int32_t n_ctx);
 
+/*
+ * kie_flash_decode without caller-provided scratch (the pages have no counterpart: this
+ * entry point exists for callers of this library that cannot allocate device memory, such
+ * as code running under a memory budget fixed at start-up, code whose device memory is
+ * owned by another framework's allocator, or latency-critical loops that cannot afford the
+ * device-wide stall of cudaMalloc/cudaFree).
+ *
+ * Same arguments and result as kie_flash_decode, minus scratch_dev/scratch_bytes. The
+ * split partials and merge counters live in one static device array of
+ * KIE_FLASH_DECODE_NOALLOC_MAX_BYTES, which every GPU that loads this library keeps until
+ * the process exits. The call allocates nothing. The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture. All calls on one GPU share that GPU's array, and every
+ * call leaves its partials there: calls whose kernels can overlap on the GPU (launched on
+ * different streams, or from host threads without ordering between them) race with each
+ * other and must be serialised by the caller; calls ordered on one stream are safe (each
+ * call clears the merge counters it needs before its kernel runs).
+ * Returns KIE_ERR_CAPACITY when kie_flash_decode_scratch_bytes(...) for this shape exceeds
+ * KIE_FLASH_DECODE_NOALLOC_MAX_BYTES, KIE_ERR_ARG for bad shapes or pointers, KIE_ERR_CUDA
+ * if the address lookup or the launch fails.
+ */
+#define KIE_FLASH_DECODE_NOALLOC_MAX_BYTES (4 << 20)
+kie_status kie_flash_decode_noalloc(const float *q_dev, const void *k_dev, const void *v_dev, int32_t n_heads,
+                                    int32_t n_kv_heads, int32_t head_dim, int32_t n_ctx, int64_t kv_stride,
+                                    int32_t dtype, float *out_dev, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
