@@ -28,6 +28,13 @@ int kie_b1_max_rows(int K);
 cudaError_t kie_b1_prepare(int dtype);
 cudaError_t kie_b1_occupancy(int dtype, int *blocks_per_sm);
 cudaError_t kie_b1_launch(const KieParams &P, const KieCmd &one, int resident, cudaStream_t stream);
+size_t kie_mr_smem_bytes();
+cudaError_t kie_mr_prepare(int dtype);
+cudaError_t kie_mr_occupancy(int dtype, int *blocks_per_sm);
+cudaError_t kie_mr_launch(const KieParams &P, const KieCmd &one, int resident, cudaStream_t stream);
+cudaError_t kie_mr_repack(const void *tiles, long long n, uint8_t *arena, cudaStream_t stream);
+size_t kie_mr_tile_src_bytes();
+void kie_mr_tile_src(void *dst, const void *const *src3, int n0, int n1, long long off, int N, int K, int rb, int ks);
 
 namespace {
 
@@ -192,10 +199,7 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
         kie_destroy(eng);
         return s;
     };
-    if (!(c.modes & KIE_MODE_BATCH1)) {
-        delete eng;
-        return KIE_ERR_UNSUPPORTED;  // the tick kernel is built separately
-    }
+    const bool b1 = (c.modes & KIE_MODE_BATCH1) != 0, mr = (c.modes & KIE_MODE_TICK) != 0;
     cudaError_t e = cudaSetDevice(c.device);
     if (e != cudaSuccess) return bail(eng->cuda_fail(e, "cudaSetDevice"));
     int sms = 0, coop = 0;
@@ -205,12 +209,24 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
         eng->fail(KIE_ERR_CUDA, "device lacks cooperative launch");
         return bail(KIE_ERR_CUDA);
     }
-    e = kie_b1_prepare(c.dtype);
-    if (e != cudaSuccess) return bail(eng->cuda_fail(e, "kernel attributes"));
-    int occ = 0;
-    e = kie_b1_occupancy(c.dtype, &occ);
-    if (e != cudaSuccess || occ < 1) return bail(eng->cuda_fail(e == cudaSuccess ? cudaErrorInvalidConfiguration : e,
-                                                                "megakernel does not fit on an SM"));
+    if (b1) {
+        e = kie_b1_prepare(c.dtype);
+        if (e != cudaSuccess) return bail(eng->cuda_fail(e, "kernel attributes"));
+        int occ = 0;
+        e = kie_b1_occupancy(c.dtype, &occ);
+        if (e != cudaSuccess || occ < 1)
+            return bail(eng->cuda_fail(e == cudaSuccess ? cudaErrorInvalidConfiguration : e,
+                                       "batch-1 megakernel does not fit on an SM"));
+    }
+    if (mr) {
+        e = kie_mr_prepare(c.dtype);
+        if (e != cudaSuccess) return bail(eng->cuda_fail(e, "kernel attributes"));
+        int occ = 0;
+        e = kie_mr_occupancy(c.dtype, &occ);
+        if (e != cudaSuccess || occ < 1)
+            return bail(eng->cuda_fail(e == cudaSuccess ? cudaErrorInvalidConfiguration : e,
+                                       "tick megakernel does not fit on an SM"));
+    }
     const int nblk = sms;
     eng->nblk = nblk;
     const int L = c.n_layers, d = c.d_model, D = c.head_dim, Hq = c.n_heads, Hkv = c.n_kv_heads, F = c.ffn,
@@ -225,7 +241,8 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
     P.timeout_ns = (long long)c.timeout_ms * 1000000ll;
     P.idle_ns = (long long)c.idle_ms * 1000000ll;
 
-    // ---- the static schedule: row partition per phase
+    P.splits = 1;
+    if (b1) {  // ---- batch-1 kernel: static schedule and packed weights
     const int Kph[KIE_NPH] = {d, qd, d, F, d};
     std::vector<int> row0((size_t)KIE_NPH * (nblk + 1));
     partition(&row0[PH_QKV * (nblk + 1)], (qd + 2 * kvd) / 2, 2, nblk);
@@ -310,6 +327,86 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
     CK(cudaMemcpy(d_seg, seg_off.data(), seg_off.size() * sizeof(long long), cudaMemcpyHostToDevice), "upload plan");
     P.row0 = d_row0;
     P.seg_off = d_seg;
+    }  // batch-1 kernel
+
+    if (mr) {  // ---- tick kernel: swizzled 128 x 64 tiles, tile ranges per SM and phase
+        const int NGm = 5;
+        const int Nm[NGm] = {qd + 2 * kvd, d, 2 * F, d, V};
+        const int Km[NGm] = {d, qd, d, F, d};
+        std::vector<int> a0((size_t)NGm * (nblk + 1));
+        for (int g = 0; g < NGm; g++) {
+            const long long atoms = (long long)((Nm[g] + 127) / 128) * (Km[g] / 64);
+            for (int cc = 0; cc <= nblk; cc++) a0[(size_t)g * (nblk + 1) + cc] = (int)(cc * atoms / nblk);
+        }
+        std::vector<long long> mseg(nblk + 1, 0);
+        for (int cc = 0; cc < nblk; cc++) {
+            long long tiles = 0;
+            for (int g = 0; g < NGm; g++) {
+                const long long n = a0[(size_t)g * (nblk + 1) + cc + 1] - a0[(size_t)g * (nblk + 1) + cc];
+                tiles += g < 4 ? n * L : n;
+            }
+            mseg[cc + 1] = mseg[cc] + tiles * 16384;
+        }
+        uint8_t *mpack = nullptr;
+        CK(eng->alloc(&mpack, (size_t)mseg[nblk]), "cudaMalloc tick weights");
+        const size_t tsz = kie_mr_tile_src_bytes();
+        std::vector<uint8_t> desc((size_t)(mseg[nblk] / 16384) * tsz);
+        size_t nt = 0;
+        for (int cc = 0; cc < nblk; cc++) {
+            long long off = mseg[cc];
+            for (int l = 0; l <= L; l++) {
+                const void *const *Lw = w->layers + (size_t)9 * (l < L ? l : 0);
+                for (int g = (l < L ? 0 : 4); g < (l < L ? 4 : 5); g++) {
+                    const void *src3[3] = {nullptr, nullptr, nullptr};
+                    int n0 = Nm[g], n1 = Nm[g];
+                    switch (g) {
+                        case 0: src3[0] = Lw[1]; src3[1] = Lw[2]; src3[2] = Lw[3]; n0 = qd; n1 = qd + kvd; break;
+                        case 1: src3[0] = Lw[4]; break;
+                        case 2: src3[0] = Lw[6]; src3[1] = Lw[7]; n0 = F; n1 = 2 * F; break;
+                        case 3: src3[0] = Lw[8]; break;
+                        default: src3[0] = w->lm_head; break;
+                    }
+                    const int nks = Km[g] / 64;
+                    for (int a = a0[(size_t)g * (nblk + 1) + cc]; a < a0[(size_t)g * (nblk + 1) + cc + 1]; a++) {
+                        kie_mr_tile_src(&desc[nt * tsz], src3, n0, n1, off, Nm[g], Km[g], a / nks, a % nks);
+                        nt++;
+                        off += 16384;
+                    }
+                }
+            }
+        }
+        void *d_desc = nullptr;
+        CK(cudaMalloc(&d_desc, desc.size()), "cudaMalloc tick repack list");
+        e = cudaMemcpy(d_desc, desc.data(), desc.size(), cudaMemcpyHostToDevice);
+        if (e == cudaSuccess) e = kie_mr_repack(d_desc, (long long)nt, mpack, 0);
+        if (e == cudaSuccess) e = cudaDeviceSynchronize();
+        cudaFree(d_desc);
+        if (e != cudaSuccess) return bail(eng->cuda_fail(e, "tick weight repack"));
+        int *d_a0 = nullptr;
+        long long *d_mseg = nullptr;
+        CK(eng->alloc(&d_a0, a0.size() * sizeof(int)), "cudaMalloc tick plan");
+        CK(eng->alloc(&d_mseg, mseg.size() * sizeof(long long)), "cudaMalloc tick plan");
+        CK(cudaMemcpy(d_a0, a0.data(), a0.size() * sizeof(int), cudaMemcpyHostToDevice), "upload tick plan");
+        CK(cudaMemcpy(d_mseg, mseg.data(), mseg.size() * sizeof(long long), cudaMemcpyHostToDevice), "upload tick plan");
+        P.mr_wpack = mpack;
+        P.mr_a0 = d_a0;
+        P.mr_seg_off = d_mseg;
+        const int R = 64;  // rows per step
+        CK(eng->alloc(&P.mr_x, (size_t)R * d * 4), "cudaMalloc tick scratch");
+        CK(eng->alloc(&P.mr_yqkv, (size_t)R * (qd + 2 * kvd) * 4), "cudaMalloc tick scratch");
+        CK(eng->alloc(&P.mr_ygu, (size_t)R * 2 * F * 4), "cudaMalloc tick scratch");
+        CK(eng->alloc(&P.mr_q, (size_t)R * qd * 4), "cudaMalloc tick scratch");
+        CK(eng->alloc(&P.mr_o, (size_t)R * qd * 4), "cudaMalloc tick scratch");
+        CK(eng->alloc(&P.mr_rstd, (size_t)R * 4), "cudaMalloc tick scratch");
+        CK(eng->alloc(&P.mr_logits, (size_t)R * V * 4), "cudaMalloc tick scratch");
+        CK(eng->alloc(&P.mr_part, (size_t)R * Hkv * G * (D + 2) * 4), "cudaMalloc tick scratch");
+        CK(eng->alloc(&P.mr_cnt, (size_t)R * Hkv * 4), "cudaMalloc tick scratch");
+        CK(eng->alloc(&P.mr_sid, (size_t)R * 4), "cudaMalloc tick scratch");
+        CK(eng->alloc(&P.mr_pos, (size_t)R * 4), "cudaMalloc tick scratch");
+        CK(eng->alloc(&P.mr_tok, (size_t)R * 4), "cudaMalloc tick scratch");
+        CK(cudaMemset(P.mr_cnt, 0, (size_t)R * Hkv * 4), "memset");
+        CK(cudaMemset(P.mr_x, 0, (size_t)R * d * 4), "memset");
+    }
 
     // ---- small weights: embedding table and norm gains
     uint16_t *emb = nullptr, *gains = nullptr;
@@ -366,7 +463,7 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
     CK(cudaMemset(P.x, 0, (size_t)d * 4), "memset");
 
     // ---- the doorbell: mapped, pinned host memory
-    eng->io_ints = 2 * (int64_t)c.max_ctx + 64 * 64 + 64;
+    eng->io_ints = 2 * (int64_t)c.max_ctx + 3 * 64 + 64 * 64;
     const size_t mb_bytes = sizeof(KieMailbox) + (size_t)eng->io_ints * 4;
     CK(cudaHostAlloc((void **)&eng->mbox_host, mb_bytes, cudaHostAllocMapped | cudaHostAllocPortable), "cudaHostAlloc mailbox");
     memset(eng->mbox_host, 0, mb_bytes);
@@ -416,7 +513,7 @@ static kie_status launch_resident(kie_engine *eng, int kind) {
     cudaError_t e = cudaMemsetAsync(eng->P.bar, 0, 16, eng->stream);
     if (e == cudaSuccess) {
         KieCmd none{};
-        e = kie_b1_launch(eng->P, none, 1, eng->stream);
+        e = kind == KIND_MR ? kie_mr_launch(eng->P, none, 1, eng->stream) : kie_b1_launch(eng->P, none, 1, eng->stream);
     }
     if (e == cudaSuccess) e = cudaEventRecord(eng->ev_done, eng->stream);
     if (e != cudaSuccess) return eng->cuda_fail(e, "launching the resident kernel");
@@ -583,6 +680,32 @@ extern "C" kie_status kie_prefill(kie_engine *eng, int32_t sid, const int32_t *t
     if ((s = check_tokens(eng, tokens, n)) != KIE_OK) return s;
     const int ctx = eng->sess_len[sid];
     if ((int64_t)ctx + n > eng->cfg.max_ctx) return eng->fail(KIE_ERR_CAPACITY, "prefill of %d at %d exceeds max_ctx", n, ctx);
+    if (eng->cfg.modes & KIE_MODE_TICK) {
+        // chunks of up to 64 consecutive positions run as rows of the tick kernel
+        if ((s = ensure_kind(eng, KIND_MR)) != KIE_OK) return s;
+        for (int c0 = 0; c0 < n; c0 += 64) {
+            const int m = std::min(64, n - c0);
+            int32_t *io = eng->mbox_host->io;
+            for (int j = 0; j < m; j++) {
+                io[j] = sid;
+                io[64 + j] = ctx + c0 + j;
+                io[128 + j] = tokens[c0 + j];
+            }
+            KieCmd cmd{};
+            cmd.op = OP_PREFILL;
+            cmd.sid = sid;
+            cmd.n = 1;
+            cmd.n_sess = m;
+            cmd.flags = (c0 + m == n) ? 1 : 0;  // logits only after the last chunk
+            cmd.tokens = io_dev(eng, 0);
+            cmd.out = io_dev(eng, 192);
+            s = doorbell(eng, cmd, KIND_MR);
+            if (s != KIE_OK) return s;
+            eng->sess_len[sid] = ctx + c0 + m;
+        }
+        *first_token = ((volatile int32_t *)eng->mbox_host->io)[192];
+        return KIE_OK;
+    }
     if ((s = ensure_kind(eng, KIND_B1)) != KIE_OK) return s;
     memcpy(eng->mbox_host->io, tokens, (size_t)n * 4);
     KieCmd cmd{};
@@ -609,6 +732,7 @@ static kie_status decode_doorbell(kie_engine *eng, int32_t sid, int32_t in_token
     const int ctx = eng->sess_len[sid];
     if ((int64_t)ctx + n > eng->cfg.max_ctx) return eng->fail(KIE_ERR_CAPACITY, "%d steps at %d exceed max_ctx", n, ctx);
     if ((int64_t)n > eng->io_ints - eng->cfg.max_ctx) return eng->fail(KIE_ERR_ARG, "n too large for the mailbox");
+    if (!(eng->cfg.modes & KIE_MODE_BATCH1)) return eng->fail(KIE_ERR_UNSUPPORTED, "engine built without KIE_MODE_BATCH1");
     if ((s = ensure_kind(eng, KIND_B1)) != KIE_OK) return s;
     KieCmd cmd{};
     cmd.op = OP_DECODE;
@@ -643,6 +767,7 @@ extern "C" kie_status kie_decode_launch(kie_engine *eng, int32_t sid, const int3
     if ((s = check_sid(eng, sid)) != KIE_OK) return s;
     const int ctx = eng->sess_len[sid];
     if ((int64_t)ctx + n > eng->cfg.max_ctx) return eng->fail(KIE_ERR_CAPACITY, "%d steps at %d exceed max_ctx", n, ctx);
+    if (!(eng->cfg.modes & KIE_MODE_BATCH1)) return eng->fail(KIE_ERR_UNSUPPORTED, "engine built without KIE_MODE_BATCH1");
     if ((s = stop_resident(eng)) != KIE_OK) return s;
     cudaStream_t st = stream ? static_cast<cudaStream_t>(stream) : eng->stream;
     KieCmd cmd{};
@@ -672,9 +797,38 @@ extern "C" kie_status kie_tick(kie_engine *eng, int32_t n_sess, const int32_t *s
                                int32_t steps, int32_t *out_tokens, float *logits_dev) {
     kie_status s = check_live(eng);
     if (s != KIE_OK) return s;
-    (void)n_sess; (void)sids; (void)in_tokens; (void)steps; (void)out_tokens; (void)logits_dev;
     if (!(eng->cfg.modes & KIE_MODE_TICK)) return eng->fail(KIE_ERR_UNSUPPORTED, "engine built without KIE_MODE_TICK");
-    return KIE_ERR_UNSUPPORTED;
+    if (n_sess < 1 || n_sess > 64 || steps < 1 || steps > 64 || !sids || !in_tokens || !out_tokens)
+        return eng->fail(KIE_ERR_ARG, "tick needs 1..64 sessions, 1..64 steps and host buffers");
+    std::vector<char> seen(eng->cfg.max_sessions, 0);
+    for (int i = 0; i < n_sess; i++) {
+        if ((s = check_sid(eng, sids[i])) != KIE_OK) return s;
+        if (seen[sids[i]]) return eng->fail(KIE_ERR_ARG, "session %d appears twice in one tick", sids[i]);
+        seen[sids[i]] = 1;
+        if ((int64_t)eng->sess_len[sids[i]] + steps > eng->cfg.max_ctx)
+            return eng->fail(KIE_ERR_CAPACITY, "session %d: %d steps exceed max_ctx", sids[i], steps);
+    }
+    if ((s = check_tokens(eng, in_tokens, n_sess)) != KIE_OK) return s;
+    if ((s = ensure_kind(eng, KIND_MR)) != KIE_OK) return s;
+    int32_t *io = eng->mbox_host->io;
+    for (int i = 0; i < n_sess; i++) {
+        io[i] = sids[i];
+        io[64 + i] = eng->sess_len[sids[i]];
+        io[128 + i] = in_tokens[i];
+    }
+    KieCmd cmd{};
+    cmd.op = OP_TICK;
+    cmd.n = steps;
+    cmd.n_sess = n_sess;
+    cmd.tokens = io_dev(eng, 0);
+    cmd.out = io_dev(eng, 192);
+    cmd.logits = logits_dev;
+    s = doorbell(eng, cmd, KIND_MR);
+    if (s != KIE_OK) return s;
+    const volatile int32_t *out = eng->mbox_host->io + 192;
+    for (int i = 0; i < steps * n_sess; i++) out_tokens[i] = out[i];
+    for (int i = 0; i < n_sess; i++) eng->sess_len[sids[i]] += steps;
+    return KIE_OK;
 }
 
 // ---------------------------------------------------------------- phase trace

@@ -87,11 +87,13 @@ struct KieParams {
     float *ssq;                     // [nblk] per-CTA sums of squares of the residual rows it owns
     unsigned long long *trace;      // phase stamps (null = off)
     int trace_tokens, trace_events;
+    // multi-row (tick / chunked prefill) kernel: swizzled 128 x 64 weight tiles, CTA c streams
+    // [mr_seg_off[c], mr_seg_off[c+1]); per GEMM phase it owns tiles [mr_a0[g][c], mr_a0[g][c+1])
+    const uint8_t *mr_wpack;
+    const long long *mr_seg_off;
+    const int *mr_a0;               // [5][nblk+1]
+    float *mr_x, *mr_yqkv, *mr_ygu, *mr_q, *mr_o, *mr_rstd, *mr_logits, *mr_part;
+    unsigned *mr_cnt;
+    int *mr_sid, *mr_pos, *mr_tok;  // [64] rows of the current command
 };
 
-#ifdef __cplusplus
-extern "C++" {
-// kernels (defined in kie_b1.cu / kie_mr.cu)
-struct KieMrParams;
-}
-#endif

@@ -1,0 +1,798 @@
+// Multi-row decode megakernel for sm_100a: the continuous-inference tick and chunked prefill.
+//
+// All sessions due on a tick advance as one batch, so every weight byte is read once for
+// the whole group ("实时AI推理为何贵56倍？持续推理与常驻内核的破局之道", section 让所有活跃会话同步推进),
+// by one resident program (section 让工作常驻 GPU) with a schedule fixed ahead of time (section
+// 把一切提前决定好). With up to 64 rows (sessions, or consecutive positions of one session in
+// prefill) per step, each weight contraction Y[rows][N] = X[rows][K] W[N][K]^T runs on the
+// 5th-generation tensor cores:
+//
+//   D[128 weight rows][128] (fp32, TMEM) += A[128 weight rows][64] * B[128][64]^T  per k-step
+//
+// A is a 128 x 64 weight tile, stored in HBM already in the K-major 128-byte-swizzled layout
+// the MMA reads, and streamed by the producer warp with 1-D bulk copies into an 8-slot ring.
+// B holds the activations split into two 16-bit halves: rows 0-63 carry hi(x) and rows
+// 64-127 carry lo(x) = x - hi(x), so D[:, s] + D[:, 64 + s] equals W x_s to about 16 bits of
+// the fp32 activation (the tensor cores take 16-bit operands only). Warps 0-3 build B tiles
+// from the fp32 activations (applying the RMSNorm scale, or silu(gate)*up for the down
+// projection), warp 8 issues tcgen05.mma and commits, warps 4-7 read the accumulator from
+// TMEM and add it into the fp32 outputs with atomics: the weight tiles of one phase are
+// split evenly over the SMs by k-steps, so partial sums of a row block from several SMs meet
+// in global memory.
+//
+// Phases per layer, each ended by a grid barrier: NORM1 (per-row 1/rms, clear the QKV
+// accumulator) | QKV | ROPE (rotate q and k, append K and V) | ATTN | O (+= residual) |
+// NORM2 | GATE/UP | DOWN (+= residual); then NORMF | HEAD | ARGMAX per step.
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include "kie_attn.cuh"
+#include "kie_device.cuh"
+
+namespace {
+
+constexpr int MR_THREADS = 320;           // warps 0-3 B builders, 4-7 epilogue, 8 MMA, 9 producer
+constexpr int MR_WORKERS = 256;           // warps 0-7 also run the non-GEMM phases
+constexpr int A_SLOTS = 8, B_SLOTS = 4;
+constexpr int TILE = 16384;               // one 128 x 64 16-bit tile
+constexpr int MAXR = 64;                  // rows per step (hi half of B; lo half at +64)
+constexpr int TMEM_COLS = 256;            // two 128-column fp32 accumulators
+
+enum { G_QKV = 0, G_O = 1, G_GU = 2, G_DOWN = 3, G_HEAD = 4, NG = 5 };
+
+struct __align__(1024) MrShared {
+    uint8_t a[A_SLOTS][TILE];
+    uint8_t b[B_SLOTS][TILE];
+    AttnSmem at;
+    uint64_t a_full[A_SLOTS], a_empty[A_SLOTS], b_full[B_SLOTS], b_empty[B_SLOTS];
+    uint64_t acc_full[2], acc_empty[2], drain;
+    uint32_t tmem_base;
+    KieCmd cmd;
+    volatile int abort;
+    int gb_ok;
+    int a0[NG], a1[NG];
+    float red[32];
+};
+
+// ------------------------------------------------------------------ tcgen05 / TMEM helpers
+
+KIE_DEV void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+KIE_DEV void tmem_relinquish() { asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory"); }
+KIE_DEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+KIE_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+KIE_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+KIE_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// D[tmem] (+)= A(desc) * B(desc)^T, M = N = 128, K = 16 (16-bit inputs, fp32 accumulate)
+KIE_DEV void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// arrive on `bar` once every tcgen05 operation issued so far by this thread has completed
+KIE_DEV void umma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// 32 lanes x 32 consecutive fp32 columns from TMEM
+KIE_DEV void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+          "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+          "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor of a K-major, 128-byte-swizzled tile (8-row atoms of 1024 B).
+KIE_DEV uint64_t smem_desc_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);       // start address
+    d |= (uint64_t)1u << 16;                        // leading byte offset (unused when swizzled)
+    d |= (uint64_t)(1024u >> 4) << 32;              // stride byte offset: next 8-row atom
+    d |= (uint64_t)1u << 46;                        // descriptor version (sm_100)
+    d |= (uint64_t)2u << 61;                        // layout: 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: fp32 accumulate, A and B 16-bit (f16 or bf16), both K-major, M = N = 128.
+__host__ __device__ constexpr uint32_t idesc_f16(int dtype) {
+    return (1u << 4) | ((uint32_t)(dtype == KIE_BF16) << 7) | ((uint32_t)(dtype == KIE_BF16) << 10) |
+           ((128u >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+// byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled tile
+KIE_DEV uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+// ------------------------------------------------------------------ shared helpers
+
+struct Gemm {
+    int N, K, ldy;
+    float *y;
+};
+
+__device__ __forceinline__ Gemm gemm_of(const KieParams &P, int g) {
+    Gemm G;
+    switch (g) {
+        case G_QKV: G = {P.Hq * P.D + 2 * P.Hkv * P.D, P.d, P.Hq * P.D + 2 * P.Hkv * P.D, P.mr_yqkv}; break;
+        case G_O: G = {P.d, P.Hq * P.D, P.d, P.mr_x}; break;
+        case G_GU: G = {2 * P.F, P.d, 2 * P.F, P.mr_ygu}; break;
+        case G_DOWN: G = {P.d, P.F, P.d, P.mr_x}; break;
+        default: G = {P.V, P.d, P.V, P.mr_logits}; break;
+    }
+    return G;
+}
+
+// words of a command record (volatile: it may live in mapped host memory)
+__device__ __forceinline__ void copy_cmd(KieCmd *dst, const KieCmd *src, bool vol) {
+    uint32_t *d = reinterpret_cast<uint32_t *>(dst);
+    if (vol) {
+        const volatile uint32_t *s = reinterpret_cast<const volatile uint32_t *>(src);
+        for (int i = 0; i < (int)(sizeof(KieCmd) / 4); i++) d[i] = s[i];
+    } else {
+        const uint32_t *s = reinterpret_cast<const uint32_t *>(src);
+        for (int i = 0; i < (int)(sizeof(KieCmd) / 4); i++) d[i] = __ldcg(s + i);
+    }
+}
+
+// grid barrier over warps 0-7 of every CTA (bounded; see the batch-1 kernel)
+__device__ bool mr_barrier(const KieParams &P, MrShared &S, unsigned long long &epoch, long long timeout_ns,
+                           unsigned where) {
+    named_bar_sync(1, MR_WORKERS);
+    if (threadIdx.x == 0) {
+        int ok = !S.abort;
+        if (ok) {
+            epoch += 1;
+            const unsigned long long target = epoch * (unsigned long long)P.nblk;
+            red_release_gpu_add_u64(P.bar, 1ull);
+            const uint64_t t0 = globaltimer();
+            unsigned spins = 0;
+            while (ld_acquire_gpu_u64(P.bar) < target) {
+                if ((++spins & 255u) == 0) {
+                    if (ld_volatile_u32(P.err) != 0u) {
+                        ok = 0;
+                        break;
+                    }
+                    if ((long long)(globaltimer() - t0) > timeout_ns) {
+                        set_error(P.err, DERR_BARRIER_TIMEOUT, 0x40 | where);
+                        ok = 0;
+                        break;
+                    }
+                }
+            }
+            if (!ok) S.abort = 1;
+        }
+        S.gb_ok = ok;
+    }
+    named_bar_sync(1, MR_WORKERS);
+    return S.gb_ok != 0;
+}
+
+__device__ __forceinline__ bool head_needed(const KieCmd &cmd) { return cmd.op == OP_TICK || (cmd.flags & 1); }
+
+// the GEMM phases of one step, in stream order
+__device__ __forceinline__ int steps_of(const KieCmd &cmd) { return cmd.op == OP_TICK ? cmd.n : 1; }
+
+// ------------------------------------------------------------------ producer (warp 9)
+
+__device__ void mr_produce(const KieParams &P, MrShared &S, uint32_t &a_it, const KieCmd &cmd) {
+    const uint8_t *seg = P.mr_wpack + P.mr_seg_off[blockIdx.x];
+    long long layer_bytes = 0;
+    for (int g = 0; g < G_HEAD; g++) layer_bytes += (long long)(S.a1[g] - S.a0[g]) * TILE;
+    const int steps = steps_of(cmd);
+    for (int st = 0; st < steps && !S.abort; st++) {
+        const uint8_t *src = seg;
+        for (int l = 0; l <= P.L && !S.abort; l++) {
+            if (l == P.L && !head_needed(cmd)) break;
+            for (int g = (l < P.L ? 0 : G_HEAD); g < (l < P.L ? G_HEAD : NG); g++) {
+                for (int a = S.a0[g]; a < S.a1[g]; a++) {
+                    const uint32_t slot = a_it % A_SLOTS, par = (a_it / A_SLOTS) & 1u;
+                    if (S.abort || !mbar_wait(&S.a_empty[slot], par ^ 1u, P.timeout_ns, &S.abort)) {
+                        if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x90);
+                        S.abort = 1;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&S.a_full[slot], TILE);
+                    bulk_g2s(S.a[slot], src, TILE, &S.a_full[slot]);
+                    src += TILE;
+                    a_it++;
+                }
+            }
+        }
+    }
+    // every issued copy must land before the CTA may leave
+    const uint32_t first = a_it > A_SLOTS ? a_it - A_SLOTS : 0;
+    for (uint32_t k = first; k < a_it; k++) mbar_wait(&S.a_full[k % A_SLOTS], (k / A_SLOTS) & 1u, P.timeout_ns, nullptr);
+}
+
+// ------------------------------------------------------------------ MMA issuer (warp 8, one lane)
+
+__device__ void mr_mma(const KieParams &P, MrShared &S, uint32_t &a_it, uint32_t &b_it, uint32_t &u_it,
+                       const KieCmd &cmd) {
+    const uint32_t idesc = idesc_f16(P.dtype);
+    const int steps = steps_of(cmd);
+    bool ok = true;
+    for (int st = 0; st < steps && ok; st++) {
+        for (int l = 0; l <= P.L && ok; l++) {
+            if (l == P.L && !head_needed(cmd)) break;
+            for (int g = (l < P.L ? 0 : G_HEAD); g < (l < P.L ? G_HEAD : NG) && ok; g++) {
+                const int nks = gemm_of(P, g).K / 64;
+                int cur_rb = -1;
+                uint32_t ab = 0;
+                for (int a = S.a0[g]; a < S.a1[g] && ok; a++) {
+                    const int rb = a / nks;
+                    const bool first = (rb != cur_rb);
+                    if (first) {  // new unit: take a free accumulator
+                        cur_rb = rb;
+                        ab = u_it & 1u;
+                        if (!mbar_wait(&S.acc_empty[ab], ((u_it >> 1) & 1u) ^ 1u, P.timeout_ns, &S.abort)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
+                    const uint32_t as = a_it % A_SLOTS, bs = b_it % B_SLOTS;
+                    if (!mbar_wait(&S.a_full[as], (a_it / A_SLOTS) & 1u, P.timeout_ns, &S.abort) ||
+                        !mbar_wait(&S.b_full[bs], (b_it / B_SLOTS) & 1u, P.timeout_ns, &S.abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(S.a[as]), sb = smem_u32(S.b[bs]);
+                    const uint32_t tmem_d = S.tmem_base + ab * 128u;
+#pragma unroll
+                    for (int kk = 0; kk < 4; kk++)
+                        umma_f16(tmem_d, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32), idesc,
+                                 (first && kk == 0) ? 0u : 1u);
+                    umma_commit(&S.a_empty[as]);
+                    umma_commit(&S.b_empty[bs]);
+                    a_it++;
+                    b_it++;
+                    const bool last = (a + 1 == S.a1[g]) || ((a + 1) / nks != rb);
+                    if (last) {
+                        umma_commit(&S.acc_full[ab]);
+                        u_it++;
+                    }
+                }
+            }
+        }
+    }
+    if (!ok) {
+        if (!S.abort) set_error(P.err, DERR_MMA_TIMEOUT, 0x91);
+        S.abort = 1;
+    }
+    // all MMAs issued by this thread must finish before TMEM or the rings are released
+    umma_commit(&S.drain);
+}
+
+// ------------------------------------------------------------------ B-tile builders (warps 0-3)
+
+// Builds the B tile of k-step ks of GEMM g: rows m < M of the 16-bit hi half, rows 64 + m of
+// the lo half, 64 columns, in the swizzled K-major layout.
+template <int DT>
+__device__ void build_b(const KieParams &P, uint8_t *tile, int g, int l, int ks, int M) {
+    const int t = threadIdx.x;  // 0..127
+    const int m = t >> 1, h = t & 1;
+    const int k0 = ks * 64 + h * 32;
+    float v[32];
+    if (m < M) {
+        if (g == G_O) {
+            const float4 *src = reinterpret_cast<const float4 *>(P.mr_o + (size_t)m * P.Hq * P.D + k0);
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const float4 q = __ldcg(src + i);
+                v[4 * i] = q.x; v[4 * i + 1] = q.y; v[4 * i + 2] = q.z; v[4 * i + 3] = q.w;
+            }
+        } else if (g == G_DOWN) {
+            const float4 *gs = reinterpret_cast<const float4 *>(P.mr_ygu + (size_t)m * 2 * P.F + k0);
+            const float4 *us = reinterpret_cast<const float4 *>(P.mr_ygu + (size_t)m * 2 * P.F + P.F + k0);
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const float4 a = __ldcg(gs + i), b = __ldcg(us + i);
+                const float ga[4] = {a.x, a.y, a.z, a.w}, ub[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int e = 0; e < 4; e++) v[4 * i + e] = ga[e] / (1.f + expf(-ga[e])) * ub[e];
+            }
+        } else {  // normalised residual
+            const float r = __ldcg(P.mr_rstd + m);
+            const uint16_t *gain = P.gains + (size_t)(g == G_HEAD ? 2 * P.L : 2 * l + (g == G_GU ? 1 : 0)) * P.d;
+            const float4 *src = reinterpret_cast<const float4 *>(P.mr_x + (size_t)m * P.d + k0);
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const float4 q = __ldcg(src + i);
+                const uint2 gw = __ldg(reinterpret_cast<const uint2 *>(gain + k0 + 4 * i));
+                float g0, g1, g2, g3;
+                cvt2<DT>(gw.x, g0, g1);
+                cvt2<DT>(gw.y, g2, g3);
+                v[4 * i] = q.x * r * g0; v[4 * i + 1] = q.y * r * g1; v[4 * i + 2] = q.z * r * g2; v[4 * i + 3] = q.w * r * g3;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; i++) v[i] = 0.f;
+    }
+    // hi / lo halves, 8 values per 16-byte chunk
+#pragma unroll
+    for (int c = 0; c < 4; c++) {
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const float x0 = v[8 * c + 2 * j], x1 = v[8 * c + 2 * j + 1];
+            const uint16_t h0 = store1<DT>(x0), h1 = store1<DT>(x1);
+            const uint16_t l0 = store1<DT>(x0 - cvt1<DT>(h0)), l1 = store1<DT>(x1 - cvt1<DT>(h1));
+            hw[j] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+            lw[j] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+        }
+        const int chunk = h * 4 + c;
+        *reinterpret_cast<uint4 *>(tile + sw128(m, chunk)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4 *>(tile + sw128(MAXR + m, chunk)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+}
+
+template <int DT>
+__device__ void mr_builders(const KieParams &P, MrShared &S, uint32_t &b_it, int g, int l, int M) {
+    const int nks = gemm_of(P, g).K / 64;
+    const int lane = threadIdx.x & 31;
+    for (int a = S.a0[g]; a < S.a1[g]; a++) {
+        const uint32_t bs = b_it % B_SLOTS;
+        bool ok = !S.abort && mbar_wait(&S.b_empty[bs], ((b_it / B_SLOTS) & 1u) ^ 1u, P.timeout_ns, &S.abort);
+        ok = __all_sync(0xffffffffu, ok);
+        b_it++;
+        if (!ok) {
+            if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x92);
+            S.abort = 1;
+            continue;
+        }
+        build_b<DT>(P, S.b[bs], g, l, a % nks, M);
+        fence_proxy_async_smem();  // generic-proxy writes become visible to the tensor cores
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.b_full[bs]);
+    }
+}
+
+// ------------------------------------------------------------------ epilogue (warps 4-7)
+
+__device__ void mr_epilogue(const KieParams &P, MrShared &S, uint32_t &u_it, int g, int M) {
+    const Gemm G = gemm_of(P, g);
+    const int nks = G.K / 64;
+    const int wq = (threadIdx.x >> 5) & 3, lane = threadIdx.x & 31;
+    int cur_rb = -1;
+    for (int a = S.a0[g]; a < S.a1[g]; a++) {
+        const int rb = a / nks;
+        if (rb == cur_rb) continue;
+        cur_rb = rb;
+        const uint32_t ab = u_it & 1u;
+        bool ok = !S.abort && mbar_wait(&S.acc_full[ab], (u_it >> 1) & 1u, P.timeout_ns, &S.abort);
+        ok = __all_sync(0xffffffffu, ok);
+        u_it++;
+        if (!ok) {
+            if (!S.abort) set_error(P.err, DERR_MMA_TIMEOUT, 0x93);
+            S.abort = 1;
+            continue;
+        }
+        tc_fence_after();
+        const int row = rb * 128 + wq * 32 + lane;
+        const uint32_t taddr = S.tmem_base + ab * 128u + ((uint32_t)(wq * 32) << 16);
+#pragma unroll 1
+        for (int half = 0; half < 2; half++) {
+            float hi[32], lo[32];
+            tmem_ld32(taddr + half * 32, hi);
+            tmem_ld32(taddr + 64 + half * 32, lo);
+            if (row < G.N) {
+#pragma unroll
+                for (int j = 0; j < 32; j++) {
+                    const int s = half * 32 + j;
+                    if (s < M) atomicAdd(G.y + (size_t)s * G.ldy + row, hi[j] + lo[j]);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.acc_empty[ab]);
+    }
+}
+
+// ------------------------------------------------------------------ worker phases (warps 0-7)
+
+// per-row 1/rms of the residual (one CTA per row), and clear the next GEMM's accumulator
+template <int DT>
+__device__ void phase_norm(const KieParams &P, MrShared &S, int g_next, bool load_emb, int M) {
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    if (g_next != G_O) {  // clear rows 0..M-1 of the accumulator of the next GEMM
+        const Gemm G = gemm_of(P, g_next);
+        const size_t n = (size_t)M * G.ldy;
+        for (size_t i = (size_t)blockIdx.x * MR_WORKERS + tid; i < n; i += (size_t)P.nblk * MR_WORKERS) G.y[i] = 0.f;
+    }
+    for (int m = blockIdx.x; m < M; m += P.nblk) {
+        float *x = P.mr_x + (size_t)m * P.d;
+        float ss = 0.f;
+        if (load_emb) {  // a new step starts from the embedding rows of its input tokens
+            const int tok = __ldcg(P.mr_tok + m);
+            for (int j = tid; j < P.d; j += MR_WORKERS) {
+                const float v = cvt1<DT>(P.emb[(size_t)tok * P.d + j]);
+                x[j] = v;
+                ss += v * v;
+            }
+        } else {
+            for (int j = tid; j < P.d; j += MR_WORKERS) {
+                const float v = __ldcg(x + j);
+                ss += v * v;
+            }
+        }
+        ss = warp_sum(ss);
+        if (lane == 0) S.red[w] = ss;
+        named_bar_sync(1, MR_WORKERS);
+        if (tid == 0) {
+            float v = 0.f;
+            for (int k = 0; k < MR_WORKERS / 32; k++) v += S.red[k];
+            P.mr_rstd[m] = rsqrtf(v / (float)P.d + P.eps);
+        }
+        named_bar_sync(1, MR_WORKERS);
+    }
+}
+
+// rotate q and k of every row, store q, append k and v to each row's cache at its position
+template <int DT>
+__device__ void phase_rope(const KieParams &P, int l, int M) {
+    const int D = P.D, half = D >> 1, qd = P.Hq * D, kvd = P.Hkv * D, ldy = qd + 2 * kvd;
+    const int pairs = (P.Hq + P.Hkv) * half + P.Hkv * half;  // q pairs, k pairs, v pairs
+    for (int m = blockIdx.x; m < M; m += P.nblk) {
+        const int sid = __ldcg(P.mr_sid + m), pos = __ldcg(P.mr_pos + m);
+        const float *y = P.mr_yqkv + (size_t)m * ldy;
+        const size_t sess = (size_t)sid * P.sess_stride;
+        for (int p = threadIdx.x; p < pairs; p += MR_WORKERS) {
+            const int head = p / half, i = p % half;  // heads: q 0..Hq-1, k Hq.., v Hq+Hkv..
+            const int base = head * D;                 // column of the head in y (q | k | v)
+            const float a = __ldcg(y + base + i), b = __ldcg(y + base + i + half);
+            if (head < P.Hq + P.Hkv) {
+                const float2 cs = P.rope[(size_t)pos * half + i];
+                const float ra = a * cs.x - b * cs.y, rb = b * cs.x + a * cs.y;
+                if (head < P.Hq) {
+                    float *q = P.mr_q + (size_t)m * qd + base;
+                    q[i] = ra;
+                    q[i + half] = rb;
+                } else {
+                    const int g = head - P.Hq;
+                    uint16_t *kp = P.kcache + sess + ((size_t)(l * P.Hkv + g) * P.max_ctx + pos) * D;
+                    kp[i] = store1<DT>(ra);
+                    kp[i + half] = store1<DT>(rb);
+                }
+            } else {
+                const int g = head - P.Hq - P.Hkv;
+                uint16_t *vp = P.vcache + sess + ((size_t)(l * P.Hkv + g) * P.max_ctx + pos) * D;
+                vp[i] = store1<DT>(a);
+                vp[i + half] = store1<DT>(b);
+            }
+        }
+    }
+}
+
+template <int DT>
+__device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M) {
+    const int G = P.G;
+    for (int u = blockIdx.x; u < M * P.Hkv; u += P.nblk) {
+        const int m = u / P.Hkv, g = u % P.Hkv;
+        const int sid = __ldcg(P.mr_sid + m), pos = __ldcg(P.mr_pos + m);
+        AttnArgs A;
+        A.q = P.mr_q + (size_t)m * P.Hq * P.D;
+        A.k = P.kcache + (size_t)sid * P.sess_stride + (size_t)l * P.Hkv * P.max_ctx * P.D;
+        A.v = P.vcache + (size_t)sid * P.sess_stride + (size_t)l * P.Hkv * P.max_ctx * P.D;
+        A.head_stride = (long long)P.max_ctx * P.D;
+        A.part = P.mr_part + (size_t)m * P.Hkv * G * (P.D + 2);
+        A.cnt = P.mr_cnt + (size_t)m * P.Hkv;
+        A.o = P.mr_o + (size_t)m * P.Hq * P.D;
+        A.D = P.D;
+        A.Hkv = P.Hkv;
+        A.nsplit = 1;
+        A.ctx = pos + 1;
+        if (G <= 4) {
+            switch (G) {
+                case 1: attn_unit<DT, 1, 8>(A, S.at, g, 1, 0); break;
+                case 2: attn_unit<DT, 2, 8>(A, S.at, g, 2, 0); break;
+                case 3: attn_unit<DT, 3, 8>(A, S.at, g, 3, 0); break;
+                default: attn_unit<DT, 4, 8>(A, S.at, g, 4, 0); break;
+            }
+        } else {
+            for (int hoff = 0; hoff < G; hoff += 4) attn_unit<DT, 4, 8>(A, S.at, g, G, hoff);
+        }
+    }
+}
+
+__device__ __forceinline__ void amax(float &v, int &i, float v2, int i2) {
+    if (v2 > v || (v2 == v && i2 < i)) {
+        v = v2;
+        i = i2;
+    }
+}
+
+// argmax of each row's logits (one CTA per row); outputs and the next step's inputs
+__device__ void phase_argmax(const KieParams &P, MrShared &S, const KieCmd &cmd, int step, int M) {
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    for (int m = blockIdx.x; m < M; m += P.nblk) {
+        const float *lg = P.mr_logits + (size_t)m * P.V;
+        float bv = -CUDART_INF_F;
+        int bi = 0x7fffffff;
+        const bool copy = cmd.logits && (cmd.op == OP_TICK || m == M - 1);
+        float *dst = nullptr;
+        if (copy) dst = cmd.logits + (cmd.op == OP_TICK ? ((size_t)step * M + m) * P.V : 0);
+        for (int r = tid; r < P.V; r += MR_WORKERS) {
+            const float v = __ldcg(lg + r);
+            if (dst) dst[r] = v;
+            amax(bv, bi, v, r);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax(bv, bi, __shfl_xor_sync(0xffffffffu, bv, o), __shfl_xor_sync(0xffffffffu, bi, o));
+        if (lane == 0) {
+            S.red[w] = bv;
+            S.red[8 + w] = __int_as_float(bi);
+        }
+        named_bar_sync(1, MR_WORKERS);
+        if (tid == 0) {
+            float v = S.red[0];
+            int i = __float_as_int(S.red[8]);
+            for (int k = 1; k < MR_WORKERS / 32; k++) amax(v, i, S.red[k], __float_as_int(S.red[8 + k]));
+            P.mr_tok[m] = i;                          // input of the next step
+            P.mr_pos[m] = __ldcg(P.mr_pos + m) + 1;
+            if (cmd.out) {
+                if (cmd.op == OP_TICK) cmd.out[step * M + m] = i;
+                else if (m == M - 1) cmd.out[0] = i;
+            }
+        }
+        named_bar_sync(1, MR_WORKERS);
+    }
+}
+
+// ------------------------------------------------------------------ one command, workers' view
+
+template <int DT>
+__device__ void mr_work(const KieParams &P, MrShared &S, uint32_t &b_it, uint32_t &u_it, const KieCmd &cmd,
+                        unsigned long long &epoch) {
+    const int M = cmd.n_sess;
+    const bool builder = threadIdx.x < 128;
+    const int steps = steps_of(cmd);
+    for (int st = 0; st < steps; st++) {
+        for (int l = 0; l < P.L; l++) {
+            if (!S.abort) phase_norm<DT>(P, S, G_QKV, l == 0, M);
+            mr_barrier(P, S, epoch, P.timeout_ns, 1);
+            if (builder) mr_builders<DT>(P, S, b_it, G_QKV, l, M);
+            else mr_epilogue(P, S, u_it, G_QKV, M);
+            mr_barrier(P, S, epoch, P.timeout_ns, 2);
+            if (!S.abort) phase_rope<DT>(P, l, M);
+            mr_barrier(P, S, epoch, P.timeout_ns, 3);
+            if (!S.abort) phase_attn<DT>(P, S, l, M);
+            mr_barrier(P, S, epoch, P.timeout_ns, 4);
+            if (builder) mr_builders<DT>(P, S, b_it, G_O, l, M);
+            else mr_epilogue(P, S, u_it, G_O, M);
+            mr_barrier(P, S, epoch, P.timeout_ns, 5);
+            if (!S.abort) phase_norm<DT>(P, S, G_GU, false, M);
+            mr_barrier(P, S, epoch, P.timeout_ns, 6);
+            if (builder) mr_builders<DT>(P, S, b_it, G_GU, l, M);
+            else mr_epilogue(P, S, u_it, G_GU, M);
+            mr_barrier(P, S, epoch, P.timeout_ns, 7);
+            if (builder) mr_builders<DT>(P, S, b_it, G_DOWN, l, M);
+            else mr_epilogue(P, S, u_it, G_DOWN, M);
+            mr_barrier(P, S, epoch, P.timeout_ns, 8);
+        }
+        if (head_needed(cmd)) {
+            if (!S.abort) phase_norm<DT>(P, S, G_HEAD, false, M);
+            mr_barrier(P, S, epoch, P.timeout_ns, 9);
+            if (builder) mr_builders<DT>(P, S, b_it, G_HEAD, P.L, M);
+            else mr_epilogue(P, S, u_it, G_HEAD, M);
+            mr_barrier(P, S, epoch, P.timeout_ns, 10);
+            if (!S.abort) phase_argmax(P, S, cmd, st, M);
+            mr_barrier(P, S, epoch, P.timeout_ns, 11);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ the kernel
+
+template <int DT>
+__global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieCmd one, int resident) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // the swizzled MMA operands need 1024-byte aligned tiles: align the base by hand
+    const uint32_t mis = smem_u32(smem_raw) & 1023u;
+    MrShared &S = *reinterpret_cast<MrShared *>(smem_raw + ((1024u - mis) & 1023u));
+    const int tid = threadIdx.x, warp = tid >> 5;
+    if (tid == 0) {
+        for (int i = 0; i < A_SLOTS; i++) {
+            mbar_init(&S.a_full[i], 1);
+            mbar_init(&S.a_empty[i], 1);
+        }
+        for (int i = 0; i < B_SLOTS; i++) {
+            mbar_init(&S.b_full[i], 4);
+            mbar_init(&S.b_empty[i], 1);
+        }
+        for (int i = 0; i < 2; i++) {
+            mbar_init(&S.acc_full[i], 1);
+            mbar_init(&S.acc_empty[i], 4);
+        }
+        mbar_init(&S.drain, 1);
+        fence_mbar_init();
+        S.abort = 0;
+    }
+    if (tid < NG) {
+        S.a0[tid] = P.mr_a0[tid * (P.nblk + 1) + blockIdx.x];
+        S.a1[tid] = P.mr_a0[tid * (P.nblk + 1) + blockIdx.x + 1];
+    }
+    if (warp == 8) {
+        tmem_alloc(&S.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    uint32_t a_it = 0, b_it = 0, u_it = 0, drains = 0;
+    unsigned long long epoch = 0;
+    for (;;) {
+        if (tid < MR_WORKERS) {
+            if (!resident) {
+                if (tid == 0) S.cmd = one;
+            } else {
+                if (blockIdx.x == 0) {
+                    if (tid == 0) {
+                        const unsigned last = *P.last_seq;
+                        const uint64_t t0 = globaltimer();
+                        KieCmd c{};
+                        c.op = OP_EXIT;
+                        for (;;) {
+                            const uint32_t s = ld_acquire_sys_u32(&P.mbox->cmd_seq);
+                            if (s != last) {
+                                copy_cmd(&c, &P.mbox->cmd, true);
+                                c.seq = s;
+                                *P.last_seq = s;
+                                break;
+                            }
+                            if ((long long)(globaltimer() - t0) > P.idle_ns) break;
+                            __nanosleep(256);
+                        }
+                        *P.cmd = c;
+                        S.cmd = c;
+                    }
+                    named_bar_sync(1, MR_WORKERS);
+                    // rows of the command arrive in the mailbox: sessions, positions, tokens
+                    if (S.cmd.op == OP_TICK || S.cmd.op == OP_PREFILL) {
+                        const volatile int32_t *io = (const volatile int32_t *)S.cmd.tokens;
+                        for (int m = tid; m < S.cmd.n_sess; m += MR_WORKERS) {
+                            P.mr_sid[m] = io[m];
+                            P.mr_pos[m] = io[MAXR + m];
+                            P.mr_tok[m] = io[2 * MAXR + m];
+                        }
+                    }
+                }
+                mr_barrier(P, S, epoch, P.idle_ns + P.timeout_ns, 0);
+                if (tid == 0) {
+                    copy_cmd(&S.cmd, P.cmd, false);
+                    if (S.abort) S.cmd.op = OP_EXIT;
+                }
+            }
+        }
+        __syncthreads();
+        const KieCmd cmd = S.cmd;
+        if (cmd.op != OP_TICK && cmd.op != OP_PREFILL) break;
+        if (warp == 9) {
+            if ((tid & 31) == 0) mr_produce(P, S, a_it, cmd);
+        } else if (warp == 8) {
+            if ((tid & 31) == 0) {
+                mr_mma(P, S, a_it, b_it, u_it, cmd);
+                mbar_wait(&S.drain, drains & 1u, P.timeout_ns, nullptr);
+            }
+            drains++;
+        } else {
+            mr_work<DT>(P, S, b_it, u_it, cmd, epoch);
+        }
+        __syncthreads();
+        if (resident && blockIdx.x == 0 && tid == 0) {
+            __threadfence_system();
+            P.mbox->status = S.abort ? -1 : 0;
+            st_release_sys_u32(&P.mbox->done_seq, cmd.seq);
+        }
+        if (!resident || S.abort) break;
+    }
+    // release TMEM (warp 8 allocated it; every MMA has drained)
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(S.tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ host-side launch helpers
+
+extern "C++" {
+
+size_t kie_mr_smem_bytes() { return sizeof(MrShared) + 1024; }
+
+cudaError_t kie_mr_prepare(int dtype) {
+    const int smem = (int)kie_mr_smem_bytes();
+    return dtype == KIE_BF16
+               ? cudaFuncSetAttribute(kie_mr_kernel<KIE_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+               : cudaFuncSetAttribute(kie_mr_kernel<KIE_FP16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+}
+
+cudaError_t kie_mr_occupancy(int dtype, int *blocks_per_sm) {
+    const size_t smem = kie_mr_smem_bytes();
+    return dtype == KIE_BF16
+               ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, kie_mr_kernel<KIE_BF16>, MR_THREADS, smem)
+               : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, kie_mr_kernel<KIE_FP16>, MR_THREADS, smem);
+}
+
+cudaError_t kie_mr_launch(const KieParams &P, const KieCmd &one, int resident, cudaStream_t stream) {
+    KieParams p = P;
+    KieCmd c = one;
+    int r = resident;
+    void *args[] = {&p, &c, &r};
+    const void *fn = P.dtype == KIE_BF16 ? (const void *)kie_mr_kernel<KIE_BF16> : (const void *)kie_mr_kernel<KIE_FP16>;
+    return cudaLaunchCooperativeKernel(fn, dim3(P.nblk), dim3(MR_THREADS), args, kie_mr_smem_bytes(), stream);
+}
+
+// Swizzled 128 x 64 tile image of rows [128 rb, 128 rb + 128) and columns [64 ks, 64 ks + 64) of
+// a row-major [N][K] matrix that is the row concatenation of up to three row-major parts
+// (rows [0, n0) from src[0], [n0, n1) from src[1], [n1, N) from src[2]); rows past N are
+// zero. The repack kernel below writes it.
+struct TileSrc {
+    const uint8_t *src[3];
+    long long dst;
+    int n0, n1, N, K, rb, ks;
+};
+
+__global__ void mr_repack_kernel(const TileSrc *t, long long n, uint8_t *arena) {
+    for (long long i = blockIdx.x; i < n; i += gridDim.x) {
+        const TileSrc s = t[i];
+        for (int c16 = threadIdx.x; c16 < 128 * 8; c16 += blockDim.x) {
+            const int r = c16 >> 3, c = c16 & 7;
+            const int row = s.rb * 128 + r;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (row < s.N) {
+                const int part = row < s.n0 ? 0 : row < s.n1 ? 1 : 2;
+                const int prow = row - (part == 0 ? 0 : part == 1 ? s.n0 : s.n1);
+                v = *reinterpret_cast<const uint4 *>(s.src[part] + ((size_t)prow * s.K + s.ks * 64 + c * 8) * 2);
+            }
+            *reinterpret_cast<uint4 *>(arena + s.dst + r * 128 + ((c ^ (r & 7)) << 4)) = v;
+        }
+    }
+}
+
+cudaError_t kie_mr_repack(const void *tiles, long long n, uint8_t *arena, cudaStream_t stream) {
+    mr_repack_kernel<<<1184, 256, 0, stream>>>(static_cast<const TileSrc *>(tiles), n, arena);
+    return cudaGetLastError();
+}
+
+size_t kie_mr_tile_src_bytes() { return sizeof(TileSrc); }
+
+void kie_mr_tile_src(void *dst, const void *const *src3, int n0, int n1, long long off, int N, int K, int rb, int ks) {
+    TileSrc t;
+    for (int i = 0; i < 3; i++) t.src[i] = static_cast<const uint8_t *>(src3[i]);
+    t.dst = off;
+    t.n0 = n0;
+    t.n1 = n1;
+    t.N = N;
+    t.K = K;
+    t.rb = rb;
+    t.ks = ks;
+    *static_cast<TileSrc *>(dst) = t;
+}
+
+}  // extern "C++"

@@ -1,0 +1,123 @@
+"""Parity of the multi-session tick kernel (tcgen05 weight contractions) with the CPU oracle.
+
+Each session of a tick is an independent decode step, so the oracle runs every sampled
+session on its own. Tolerances are those of tests/parity.py. Within one tick the first
+step's argmax feeds the second step on the GPU; the oracle follows its own argmax, so the
+second step is compared only where the first step's tokens are the oracle's (always, when
+the oracle's margin exceeds 0.05).
+"""
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def kie():
+    from bandwidth_bound_stream_b200 import build
+    build.build_kie()
+    from bandwidth_bound_stream_b200 import kie as k
+    return k
+
+
+def _run_tick_parity(kie, model, n_sess, prompt_lens, checked, ticks, max_ctx, modes=None):
+    from bandwidth_bound_stream_b200 import synth
+    from oracle.oracle import OracleModel
+    from tests.parity import MARGIN, assert_reports, compare_step, margin
+    modes = kie.KIE_MODE_TICK if modes is None else modes
+    dw = kie.DeviceWeights(model, host_copy=True)
+    eng = kie.Engine(kie.config(model, max_sessions=n_sess, max_ctx=max_ctx, timeout_ms=20000, idle_ms=100,
+                                modes=modes), dw.kie)
+    V = model.vocab
+    reports = []
+    checked = list(checked)
+    with eng:
+        sids = [eng.session_open() for _ in range(n_sess)]
+        prompts = [synth.prompt(model, prompt_lens[i], session=i) for i in range(n_sess)]
+        firsts = [eng.prefill(sids[i], prompts[i]) for i in range(n_sess)]
+        orcs = {i: OracleModel(model, dw.host, max_ctx) for i in checked}
+        toks = {}
+        for i in checked:
+            ref = orcs[i].prefill(prompts[i])
+            reports.append(compare_step(ref, firsts[i], ref, model.dtype))
+            toks[i] = int(np.argmax(ref))
+        inputs = np.array(firsts, dtype=np.int32)
+        for i in checked:
+            inputs[i] = toks[i]  # teacher-force the checked sessions with the oracle's token
+        logits = torch.empty((2, n_sess, V), dtype=torch.float32, device="cuda")
+        for _ in range(ticks):
+            # one teacher-forced step (logits compared for every checked session) ...
+            out = eng.tick(sids, inputs, 1, logits.data_ptr())
+            got = logits[0].cpu().numpy()
+            for i in checked:
+                ref = orcs[i].step(int(inputs[i]))
+                reports.append(compare_step(got[i], int(out[0, i]), ref, model.dtype))
+                inputs[i] = int(np.argmax(ref))
+            for i in range(n_sess):
+                if i not in checked:
+                    inputs[i] = out[0, i]
+            # ... then a two-step tick: step 1's argmax feeds step 2 on the GPU
+            out = eng.tick(sids, inputs, 2, logits.data_ptr())
+            got = logits.cpu().numpy()
+            for i in list(checked):
+                ref1 = orcs[i].step(int(inputs[i]))
+                reports.append(compare_step(got[0, i], int(out[0, i]), ref1, model.dtype))
+                t1 = int(np.argmax(ref1))
+                if int(out[0, i]) != t1:  # a low-margin step: the two chains part here
+                    assert margin(ref1) <= MARGIN
+                    checked.remove(i)
+                    continue
+                ref2 = orcs[i].step(t1)
+                reports.append(compare_step(got[1, i], int(out[1, i]), ref2, model.dtype))
+                inputs[i] = int(np.argmax(ref2))
+            for i in range(n_sess):
+                if i not in checked:
+                    inputs[i] = out[1, i]
+            assert out.min() >= 0 and out.max() < V
+        for i in range(n_sess):
+            assert eng.session_length(sids[i]) == prompt_lens[i] + 3 * ticks
+    return assert_reports(reports, model.dtype)
+
+
+def test_tick_tiny_parity(kie):
+    """fp16 tiny model, 5 sessions, prompts spanning one and two prefill chunks."""
+    from bandwidth_bound_stream_b200 import synth
+    _run_tick_parity(kie, synth.TINY, 5, [9, 17, 33, 69, 100], checked=[0, 1, 2, 3, 4], ticks=2, max_ctx=128)
+
+
+def test_tick_ragged_parity(kie):
+    """bf16, odd vocabulary (row blocks padded), 3 query heads per kv head, d = 384."""
+    from bandwidth_bound_stream_b200 import synth
+    _run_tick_parity(kie, synth.RAGGED, 7, [5, 12, 64, 65, 3, 30, 20], checked=[0, 3, 6], ticks=2, max_ctx=96)
+
+
+def test_tick_slice_10p8b_56_sessions(kie):
+    """Two layers of the 10.8B tick shape at full width (bf16, GQA 4), 56 sessions; 5 sampled
+    sessions are checked against the oracle."""
+    from bandwidth_bound_stream_b200 import synth
+    lens = [4 + (7 * i) % 61 for i in range(56)]
+    _run_tick_parity(kie, synth.SLICE_TICK, 56, lens, checked=[0, 13, 27, 41, 55], ticks=1, max_ctx=80)
+
+
+def test_tick_errors(kie):
+    from bandwidth_bound_stream_b200 import synth
+    m = synth.TINY
+    dw = kie.DeviceWeights(m)
+    with kie.Engine(kie.config(m, max_sessions=3, max_ctx=16, timeout_ms=5000, idle_ms=50,
+                               modes=kie.KIE_MODE_TICK), dw.kie) as eng:
+        a, b = eng.session_open(), eng.session_open()
+        eng.prefill(a, synth.prompt(m, 4))
+        eng.prefill(b, synth.prompt(m, 14))
+        with pytest.raises(kie.KieError) as ei:
+            eng.tick([a, a], [1, 2], 1)
+        assert ei.value.status == kie.KIE_ERR_ARG
+        with pytest.raises(kie.KieError) as ei:
+            eng.tick([a, b], [1, 2], 3)  # b has 14 of 16 positions
+        assert ei.value.status == kie.KIE_ERR_CAPACITY
+        with pytest.raises(kie.KieError) as ei:
+            eng.decode_step(a, 1)  # no batch-1 kernel in this engine
+        assert ei.value.status == kie.KIE_ERR_UNSUPPORTED
+        out = eng.tick([a, b], [1, 2], 2)
+        assert out.shape == (2, 2) and eng.session_length(a) == 6
