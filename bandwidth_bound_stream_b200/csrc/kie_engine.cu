@@ -793,14 +793,13 @@ extern "C" kie_status kie_sync(kie_engine *eng) {
     return check_device_error(eng);
 }
 
-extern "C" kie_status kie_tick(kie_engine *eng, int32_t n_sess, const int32_t *sids, const int32_t *in_tokens,
-                               int32_t steps, int32_t *out_tokens, float *logits_dev) {
-    kie_status s = check_live(eng);
-    if (s != KIE_OK) return s;
+// Checks shared by the two tick entry points.
+static kie_status tick_checks(kie_engine *eng, int32_t n_sess, const int32_t *sids, int32_t steps) {
     if (!(eng->cfg.modes & KIE_MODE_TICK)) return eng->fail(KIE_ERR_UNSUPPORTED, "engine built without KIE_MODE_TICK");
-    if (n_sess < 1 || n_sess > 64 || steps < 1 || steps > 64 || !sids || !in_tokens || !out_tokens)
-        return eng->fail(KIE_ERR_ARG, "tick needs 1..64 sessions, 1..64 steps and host buffers");
+    if (n_sess < 1 || n_sess > 64 || steps < 1 || steps > 64 || !sids)
+        return eng->fail(KIE_ERR_ARG, "tick needs 1..64 sessions and 1..64 steps");
     std::vector<char> seen(eng->cfg.max_sessions, 0);
+    kie_status s;
     for (int i = 0; i < n_sess; i++) {
         if ((s = check_sid(eng, sids[i])) != KIE_OK) return s;
         if (seen[sids[i]]) return eng->fail(KIE_ERR_ARG, "session %d appears twice in one tick", sids[i]);
@@ -808,6 +807,47 @@ extern "C" kie_status kie_tick(kie_engine *eng, int32_t n_sess, const int32_t *s
         if ((int64_t)eng->sess_len[sids[i]] + steps > eng->cfg.max_ctx)
             return eng->fail(KIE_ERR_CAPACITY, "session %d: %d steps exceed max_ctx", sids[i], steps);
     }
+    return KIE_OK;
+}
+
+extern "C" kie_status kie_tick_launch(kie_engine *eng, int32_t n_sess, const int32_t *sids, const int32_t *in_tokens_dev,
+                                      int32_t steps, int32_t *out_tokens_dev, float *logits_dev, void *stream) {
+    kie_status s = check_live(eng);
+    if (s != KIE_OK) return s;
+    if (!in_tokens_dev || !out_tokens_dev) return eng->fail(KIE_ERR_ARG, "tick launch needs device buffers");
+    if ((s = tick_checks(eng, n_sess, sids, steps)) != KIE_OK) return s;
+    if ((s = stop_resident(eng)) != KIE_OK) return s;
+    cudaStream_t st = stream ? static_cast<cudaStream_t>(stream) : eng->stream;
+    // rows of the command: sessions and positions from the host (pageable: copied before return)
+    std::vector<int32_t> sp(2 * n_sess);
+    for (int i = 0; i < n_sess; i++) {
+        sp[i] = sids[i];
+        sp[n_sess + i] = eng->sess_len[sids[i]];
+    }
+    cudaError_t e = cudaMemcpyAsync(eng->P.mr_sid, sp.data(), (size_t)n_sess * 4, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(eng->P.mr_pos, sp.data() + n_sess, (size_t)n_sess * 4, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(eng->P.mr_tok, in_tokens_dev, (size_t)n_sess * 4, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(eng->P.bar, 0, 16, st);
+    KieCmd cmd{};
+    cmd.op = OP_TICK;
+    cmd.n = steps;
+    cmd.n_sess = n_sess;
+    cmd.out = out_tokens_dev;
+    cmd.logits = logits_dev;
+    if (e == cudaSuccess) e = kie_mr_launch(eng->P, cmd, 0, st);
+    if (e != cudaSuccess) return eng->cuda_fail(e, "launching the tick kernel");
+    for (int i = 0; i < n_sess; i++) eng->sess_len[sids[i]] += steps;
+    return KIE_OK;
+}
+
+extern "C" kie_status kie_tick(kie_engine *eng, int32_t n_sess, const int32_t *sids, const int32_t *in_tokens,
+                               int32_t steps, int32_t *out_tokens, float *logits_dev) {
+    kie_status s = check_live(eng);
+    if (s != KIE_OK) return s;
+    if (!in_tokens || !out_tokens) return eng->fail(KIE_ERR_ARG, "tick needs host buffers");
+    if ((s = tick_checks(eng, n_sess, sids, steps)) != KIE_OK) return s;
     if ((s = check_tokens(eng, in_tokens, n_sess)) != KIE_OK) return s;
     if ((s = ensure_kind(eng, KIND_MR)) != KIE_OK) return s;
     int32_t *io = eng->mbox_host->io;

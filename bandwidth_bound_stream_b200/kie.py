@@ -25,7 +25,7 @@ EXPORTS = ("kie_config_defaults", "kie_create", "kie_destroy", "kie_session_open
            "kie_session_length", "kie_session_rewind", "kie_session_kv", "kie_prefill", "kie_decode_step",
            "kie_generate", "kie_decode_launch", "kie_sync", "kie_tick", "kie_last_error", "kie_status_string",
            "kie_flash_decode", "kie_flash_decode_scratch_bytes", "kie_trace_enable", "kie_trace_read",
-           "kie_trace_events", "kie_flash_decode_noalloc")
+           "kie_trace_events", "kie_flash_decode_noalloc", "kie_tick_launch")
 
 
 class KieConfig(ctypes.Structure):
@@ -76,6 +76,7 @@ def _load():
         "kie_trace_read": (i32, [vp, vp, i64, P(i64)]),
         "kie_trace_events": (i32, [vp]),
         "kie_flash_decode_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, i64, i32, vp, vp]),
+        "kie_tick_launch": (i32, [vp, i32, vp, vp, i32, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(h, name)
@@ -184,6 +185,12 @@ class Engine:
                       logits_dev_ptr: int | None = None, stream_ptr: int | None = None):
         self._check(lib.kie_decode_launch(self.h, sid, in_tok_dev_ptr, n, out_dev_ptr, logits_dev_ptr, stream_ptr),
                     "kie_decode_launch")
+
+    def tick_launch(self, sids, in_tok_dev_ptr: int, steps: int, out_dev_ptr: int, logits_dev_ptr: int | None = None,
+                    stream_ptr: int | None = None):
+        s = np.ascontiguousarray(sids, dtype=np.int32)
+        self._check(lib.kie_tick_launch(self.h, s.size, _ptr(s), in_tok_dev_ptr, steps, out_dev_ptr, logits_dev_ptr,
+                                        stream_ptr), "kie_tick_launch")
 
     def trace_enable(self, tokens: int):
         self._check(lib.kie_trace_enable(self.h, tokens), "kie_trace_enable")

@@ -181,9 +181,22 @@ def main():
     ap.add_argument("--model", default="dense-1.9b", help="workload shape (profiling cases use smaller ones)")
     ap.add_argument("--prompt", type=int, default=PROMPT)
     ap.add_argument("--decode", type=int, default=DECODE)
+    ap.add_argument("--ticks", type=int, default=500, help="timed ticks of the 56-session workload (0 = skip)")
+    ap.add_argument("--tick-only", action="store_true", help="only the tick workload (its own JSON line)")
+    ap.add_argument("--tick-model", default="dense-10.8b")
+    ap.add_argument("--tick-prompt", type=int, default=0, help="fixed prompt length per session (0 = seeded 1000-1500)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank, world, local = dist_setup()
+    if args.tick_only:
+        import torch
+        torch.cuda.set_device(local)
+        t = run_tick(args.ticks, args.warmup, local, clocks_for=local, model_name=args.tick_model,
+                     prompt_len=args.tick_prompt)
+        if rank == 0:
+            print(json.dumps({"metric": "p99 tick latency at 56 sessions", "value": t["p99_ms"], "unit": "ms",
+                              "higher_is_better": False, "n_gpus": world, "tick": t}), flush=True)
+        return
     if args.impl == "reference":
         run_reference(args, rank)
         if world > 1:
@@ -202,8 +215,9 @@ def main():
     want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
     dw = kie.DeviceWeights(m, seed=0, device=dev, host_copy=want_cpu)
     prompt = synth.prompt(m, prompt_len)
-    eng = kie.Engine(kie.config(m, max_ctx=prompt_len + decode_n, timeout_ms=10000, idle_ms=200, device=local),
-                     dw.kie)
+    # both kernels: the prompt is prefilled in chunks of 64 positions on the tensor cores
+    eng = kie.Engine(kie.config(m, max_ctx=prompt_len + decode_n, timeout_ms=10000, idle_ms=200, device=local,
+                                modes=kie.KIE_MODE_BATCH1 | kie.KIE_MODE_TICK), dw.kie)
     host_weights = dw.host
     dw.free()  # the engine keeps its own repacked copy
     torch.cuda.empty_cache()
@@ -226,6 +240,7 @@ def main():
         launch()
     eng.sync()
     ref_tokens = out_d.cpu().numpy().copy()
+    torch.cuda.nvtx.range_push("kie_decode_timed")
 
     def barrier():
         if world > 1:
@@ -244,6 +259,7 @@ def main():
         launch()
         ends[i].record(stream)
     t_all1.record(stream)
+    torch.cuda.nvtx.range_pop()
     eng.sync()
     torch.cuda.synchronize()
     clock_info = clocks.stop()
@@ -319,6 +335,8 @@ def main():
                     "itl_ms_p99": round(float(np.percentile(itl, 99)), 4),
                     "per_launch_ms": [round(x, 3) for x in per_launch]},
     }
+    if args.ticks > 0 and headline:
+        line["tick"] = run_tick(args.ticks, args.warmup, local, clocks_for=local)
     if want_cpu:
         line["cpu_baseline"] = oracle_baseline(m, host_weights, prompt_len + decode_n // 2)
     if rank == 0:
@@ -326,6 +344,89 @@ def main():
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+TICK_SESSIONS, TICK_STEPS, TICK_DEADLINE_MS = 56, 2, 160.0
+
+
+def run_tick(n_ticks: int, warmup: int, local: int, clocks_for: int, model_name: str = "dense-10.8b",
+             prompt_len: int = 0) -> dict:
+    """The continuous-inference workload: 56 sessions of the 10.8B bf16 model, each prefilled
+    with a seeded prompt of 1000-1500 tokens, then n_ticks ticks of 2 greedy steps per session
+    through kie_tick (one doorbell per tick). Tick latency is the host-side round trip of one
+    kie_tick call (doorbell written -> outputs read), as a server would see it."""
+    import torch
+
+    from bandwidth_bound_stream_b200 import kie, synth
+    m = synth.CONFIGS[model_name]
+    dev = f"cuda:{local}"
+    lens = [prompt_len or synth.tick_prompt_length(s) for s in range(TICK_SESSIONS)]
+    max_ctx = max(lens) + TICK_STEPS * (2 * n_ticks + 2 * warmup) + 8
+    t0 = time.perf_counter()
+    dw = kie.DeviceWeights(m, seed=0, device=dev)
+    eng = kie.Engine(kie.config(m, max_sessions=TICK_SESSIONS, max_ctx=max_ctx, timeout_ms=60000, idle_ms=500,
+                                device=local, modes=kie.KIE_MODE_TICK), dw.kie)
+    dw.free()
+    torch.cuda.empty_cache()
+    setup_s = time.perf_counter() - t0
+    sids = [eng.session_open() for _ in range(TICK_SESSIONS)]
+    t0 = time.perf_counter()
+    tokens = np.array([eng.prefill(sids[s], synth.prompt(m, lens[s], session=s)) for s in range(TICK_SESSIONS)],
+                      dtype=np.int32)
+    prefill_s = time.perf_counter() - t0
+    for _ in range(warmup):
+        tokens = eng.tick(sids, tokens, TICK_STEPS)[-1].copy()
+    ctx0 = [eng.session_length(s) for s in sids]
+    clocks = ClockSampler(clocks_for)
+    clocks.start()
+    lat = []
+    for _ in range(n_ticks):
+        a = time.perf_counter()
+        out = eng.tick(sids, tokens, TICK_STEPS)
+        lat.append((time.perf_counter() - a) * 1e3)
+        tokens = out[-1].copy()
+    clk = clocks.stop()
+    # the same ticks, stream-ordered on device buffers and timed with CUDA events (device time)
+    stream = torch.cuda.Stream(device=dev)
+    tok_d = torch.tensor(tokens, device=dev)
+    outs = [torch.zeros((TICK_STEPS, TICK_SESSIONS), dtype=torch.int32, device=dev) for _ in range(2)]
+    for k in range(warmup):
+        eng.tick_launch(sids, tok_d.data_ptr() if k == 0 else outs[(k - 1) % 2][-1].data_ptr(), TICK_STEPS,
+                        outs[k % 2].data_ptr(), None, stream.cuda_stream)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_ticks)]
+    torch.cuda.nvtx.range_push("kie_tick_timed")
+    for k in range(n_ticks):
+        src = outs[(warmup + k - 1) % 2][-1] if warmup + k > 0 else tok_d
+        ev[k][0].record(stream)
+        eng.tick_launch(sids, src.data_ptr(), TICK_STEPS, outs[(warmup + k) % 2].data_ptr(), None, stream.cuda_stream)
+        ev[k][1].record(stream)
+    torch.cuda.nvtx.range_pop()
+    eng.sync()
+    dev_ms = np.array([a.elapsed_time(b) for a, b in ev])
+    eng.close()
+    lat = np.array(lat)
+    # bytes one tick must move: all weights but the embedding table (plus one row per session) per
+    # step, each session's KV read over its attended positions, and its new K/V write
+    per_pos = m.kv_bytes_per_position()
+    tick_bytes = []
+    for k in range(n_ticks):
+        b = 0
+        for st in range(TICK_STEPS):
+            b += m.weight_bytes_per_token() + (TICK_SESSIONS - 1) * 2 * m.d_model
+            b += sum((c + TICK_STEPS * k + st + 1) * per_pos + per_pos for c in ctx0)
+        tick_bytes.append(b)
+    gbs = float(np.median(np.array(tick_bytes) / (lat / 1e3)) / 1e9)
+    misses = int((lat > TICK_DEADLINE_MS).sum())
+    return {"model": "dense-10.8b bf16 (48L d4096 32/8x128 F14336 V32000)", "sessions": TICK_SESSIONS,
+            "steps_per_tick": TICK_STEPS, "ticks": n_ticks, "session_ticks": TICK_SESSIONS * n_ticks,
+            "ctx_start_range": [min(lens), max(lens)], "p50_ms": round(float(np.percentile(lat, 50)), 3),
+            "p99_ms": round(float(np.percentile(lat, 99)), 3), "max_ms": round(float(lat.max()), 3),
+            "deadline_ms": TICK_DEADLINE_MS, "ticks_late": misses, "session_ticks_late": misses * TICK_SESSIONS,
+            "achieved_gbs_median": round(gbs, 1), "prefill_s": round(prefill_s, 2), "setup_s": round(setup_s, 1),
+            "device_ms_p50": round(float(np.percentile(dev_ms, 50)), 3),
+            "device_ms_p99": round(float(np.percentile(dev_ms, 99)), 3),
+            "device_launches": n_ticks,
+            "path": "kie_tick via the mapped-mailbox doorbell, host clock", "clocks": clk}
 
 
 def kernel_revision() -> str:

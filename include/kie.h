@@ -179,6 +179,17 @@ kie_status kie_trace_enable(kie_engine *eng, int32_t tokens);
 kie_status kie_trace_read(kie_engine *eng, uint64_t *host, int64_t max_elems, int64_t *n);
 int32_t kie_trace_events(kie_engine *eng);
 
+/*
+ * Stream-ordered form of kie_tick: one launch of the tick kernel on `stream` (cudaStream_t;
+ * NULL = the engine's own stream). sids (HOST, [n_sess]) as for kie_tick; in_tokens_dev
+ * (DEVICE, [n_sess]) the first inputs, out_tokens_dev (DEVICE, [steps][n_sess]) every argmax,
+ * logits_dev (DEVICE, nullable, [steps][n_sess][vocab]). The last step's outputs can be passed
+ * as the next call's inputs. Returns once the launch is queued; session lengths advance
+ * immediately; device errors surface at kie_sync.
+ */
+kie_status kie_tick_launch(kie_engine *eng, int32_t n_sess, const int32_t *sids, const int32_t *in_tokens_dev,
+                           int32_t steps, int32_t *out_tokens_dev, float *logits_dev, void *stream);
+
 /* Copies the engine's last error message (NUL-terminated, truncated to len). */
 kie_status kie_last_error(kie_engine *eng, char *buf, int32_t len);
 

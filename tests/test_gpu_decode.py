@@ -249,3 +249,15 @@ def test_resident_kernel_idles_out_and_relaunches(kie):
         eng.session_rewind(sid, len(prompt))
         b = eng.generate(sid, first, 5)
         assert np.array_equal(a, b)
+
+
+def test_tick_prefill_then_batch1_decode(kie):
+    """An engine with both kernels: the prompt goes through the tick kernel's chunked prefill (its
+    K/V land in the shared cache), then the batch-1 kernel decodes from that cache."""
+    from bandwidth_bound_stream_b200 import synth
+    from tests.parity import assert_reports
+    for m, plen, steps in [(synth.TINY, 100, 12), (synth.SLICE_1P9B, 70, 6)]:
+        dw, eng, orc = _setup(kie, m, plen + steps + 4, modes=kie.KIE_MODE_BATCH1 | kie.KIE_MODE_TICK)
+        with eng:
+            reps = _lockstep(kie, eng, orc, m, synth.prompt(m, plen, session=5), steps)
+        assert_reports(reps, m.dtype)

@@ -121,3 +121,30 @@ def test_tick_errors(kie):
         assert ei.value.status == kie.KIE_ERR_UNSUPPORTED
         out = eng.tick([a, b], [1, 2], 2)
         assert out.shape == (2, 2) and eng.session_length(a) == 6
+
+
+def test_tick_launch_matches_doorbell(kie):
+    """The stream-ordered launch (device buffers) computes the same tick as the doorbell path
+    (split-K partial sums meet through atomics, so compare logits to a tight tolerance)."""
+    from bandwidth_bound_stream_b200 import synth
+    m = synth.TINY
+    dw = kie.DeviceWeights(m)
+    n = 6
+    with kie.Engine(kie.config(m, max_sessions=n, max_ctx=64, timeout_ms=5000, idle_ms=50,
+                               modes=kie.KIE_MODE_TICK), dw.kie) as eng:
+        sids = [eng.session_open() for _ in range(n)]
+        lens = [5, 9, 17, 33, 2, 40]
+        firsts = np.array([eng.prefill(sids[i], synth.prompt(m, lens[i], session=i)) for i in range(n)],
+                          dtype=np.int32)
+        la = torch.empty((2, n, m.vocab), dtype=torch.float32, device="cuda")
+        lb = torch.empty_like(la)
+        out_a = eng.tick(sids, firsts, 2, la.data_ptr())
+        for i in range(n):
+            eng.session_rewind(sids[i], lens[i])
+        tok_d = torch.tensor(firsts, device="cuda")
+        out_d = torch.zeros((2, n), dtype=torch.int32, device="cuda")
+        eng.tick_launch(sids, tok_d.data_ptr(), 2, out_d.data_ptr(), lb.data_ptr())
+        eng.sync()
+        np.testing.assert_allclose(lb.cpu().numpy(), la.cpu().numpy(), rtol=0, atol=1e-3)
+        assert (out_d.cpu().numpy() == out_a).mean() > 0.9
+        assert all(eng.session_length(sids[i]) == lens[i] + 2 for i in range(n))
