@@ -59,6 +59,8 @@ extern "C" kie_status kie_flash_decode(const float *q_dev, const void *k_dev, co
     A.cnt = reinterpret_cast<unsigned *>(static_cast<char *>(scratch_dev) +
                                          fd_part_bytes(n_heads, n_kv_heads, head_dim, n_ctx));
     A.o = out_dev;
+    A.bpack = nullptr;
+    A.brow = 0;
     A.D = head_dim;
     A.Hkv = n_kv_heads;
     A.nsplit = fd_splits(G, n_ctx);

@@ -12,7 +12,8 @@
 // Position groups, then warps, are merged by rescaling to the common max. The last unit to
 // finish a kv head combines the splits the same way:
 //     o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s,
-// which equals the one-pass softmax over all positions for any split count.
+// which equals the one-pass softmax over all positions for any split count (the merge
+// issues each step's loads together, so it costs two L2 round trips for any split count).
 //
 // Contract for callers: NW warps (8 or 16, threads 0 .. 32*NW-1) execute attn_all_units
 // together and use named barrier 1.
@@ -27,7 +28,11 @@ struct AttnArgs {
     long long head_stride;   // elements between consecutive kv heads
     float *part;             // [Hkv * nsplit * G][D + 2] partials (m, l, acc)
     unsigned *cnt;           // [Hkv] finished-split counters (0 on entry, left at 0)
-    float *o;                // [Hq][D] output
+    float *o;                // [Hq][D] output (unused when bpack is set)
+    uint8_t *bpack;          // or null: the output goes, as 16-bit hi/lo halves, to row brow
+                             // (hi) and 64 + brow (lo) of the swizzled 128 x 64 tiles of the
+                             // tick kernel's B operand (column h * D + e)
+    int brow;
     int D, Hkv, nsplit, ctx;
 };
 
@@ -37,6 +42,7 @@ struct AttnSmem {
     float mrow[KIE_GMAX];
     float red[KIE_GMAX * 16];
     int is_last;
+    unsigned long long t_unit;  // globaltimer when this CTA's last unit finished its positions
 };
 
 // Asks L2 for the K and V rows units first, first + step, ... will read (a hint that may be
@@ -55,16 +61,50 @@ KIE_DEV void attn_prefetch(const uint16_t *k, const uint16_t *v, long long head_
     }
 }
 
+// positions per position group per batch (register budget)
+template <int GC, int NW>
+__host__ __device__ constexpr int attn_batch() {
+    return NW >= 16 ? (GC == 1 ? 4 : 2) : (GC == 1 ? 8 : GC == 2 ? 4 : 2);
+}
+
+// The first batch of K/V rows of a unit, loaded ahead of the barrier that publishes q (every
+// cached position but the newest is final before the QKV phase of a token).
+template <int B>
+struct AttnPre {
+    uint4 k[B], v[B];
+};
+
 // 2^(x - M) with 2^(-inf - M) = 0 (M >= x; M = -inf only when x = -inf)
 KIE_DEV float rescale(float x, float M) { return x == -CUDART_INF_F ? 0.f : exp2f(x - M); }
 
 // Query heads hoff .. hoff+nh-1 (nh <= GC) of the group of kv head `unit / nsplit`, whose
 // group has Gt query heads in all; a kv head with more than 4 query heads is done in chunks
 // of 4 (each chunk re-reads the split's K/V, mostly from L2).
+// Issues the loads of the first batch of `unit` (as attn_unit does), skipping position
+// `newest`, whose row may not be written yet; attn_unit<..., true> consumes them.
 template <int DT, int GC, int NW>
-__device__ void attn_unit(const AttnArgs &A, AttnSmem &S, int unit, int Gt, int hoff) {
+__device__ __forceinline__ void attn_preload(const AttnArgs &A, int unit, int newest, AttnPre<attn_batch<GC, NW>()> &pre) {
+    constexpr int B = attn_batch<GC, NW>();
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int D = A.D, lpp = D >> 3, ppw = 32 / lpp, sub = lane / lpp, sl = lane % lpp;
+    const int ngroups = NW * ppw, gi = w * ppw + sub;
+    const int g = unit / A.nsplit, s = unit % A.nsplit;
+    const int p0 = (int)((long long)s * A.ctx / A.nsplit), p1 = (int)((long long)(s + 1) * A.ctx / A.nsplit);
+    const size_t kvoff = (size_t)g * A.head_stride + (size_t)p0 * D + sl * 8;
+#pragma unroll
+    for (int b = 0; b < B; b++) {
+        const int j = gi + b * ngroups;
+        const bool ok = j < p1 - p0 && p0 + j != newest;
+        pre.k[b] = ok ? __ldcg(reinterpret_cast<const uint4 *>(A.k + kvoff + (size_t)j * D)) : make_uint4(0, 0, 0, 0);
+        pre.v[b] = ok ? __ldcg(reinterpret_cast<const uint4 *>(A.v + kvoff + (size_t)j * D)) : make_uint4(0, 0, 0, 0);
+    }
+}
+
+template <int DT, int GC, int NW, bool PRE = false>
+__device__ void attn_unit(const AttnArgs &A, AttnSmem &S, int unit, int Gt, int hoff,
+                          const AttnPre<attn_batch<GC, NW>()> *pre = nullptr) {
     constexpr int G = GC;
-    constexpr int B = NW >= 16 ? (G == 1 ? 4 : 2) : (G == 1 ? 8 : G == 2 ? 4 : 2);  // positions per group per batch (register budget)
+    constexpr int B = attn_batch<GC, NW>();
     constexpr int ATTN_WARPS = NW, ATTN_THREADS = NW * 32;
     const int nh = min(GC, Gt - hoff);
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
@@ -98,15 +138,8 @@ __device__ void attn_unit(const AttnArgs &A, AttnSmem &S, int unit, int Gt, int 
         for (int e = 0; e < 8; e++) acc[jj][e] = 0.f;
     }
 
-    for (int base = 0; base < np; base += ngroups * B) {  // uniform across the CTA
-        uint4 kv[B], vv[B];
-#pragma unroll
-        for (int b = 0; b < B; b++) {
-            const int j = base + gi + b * ngroups;
-            const bool ok = j < np;
-            kv[b] = ok ? __ldcg(reinterpret_cast<const uint4 *>(Kp + (size_t)j * D)) : make_uint4(0, 0, 0, 0);
-            vv[b] = ok ? __ldcg(reinterpret_cast<const uint4 *>(Vp + (size_t)j * D)) : make_uint4(0, 0, 0, 0);
-        }
+    // one batch: scores of B positions per group, then the running softmax update
+    auto batch = [&](int base, const uint4 (&kv)[B], const uint4 (&vv)[B]) {
         float sc[B][G];
 #pragma unroll
         for (int b = 0; b < B; b++) {
@@ -145,6 +178,30 @@ __device__ void attn_unit(const AttnArgs &A, AttnSmem &S, int unit, int Gt, int 
                 for (int e = 0; e < 8; e++) acc[jj][e] = fmaf(p, f[e], acc[jj][e]);
             }
         }
+    };
+    int base0 = 0;
+    if (PRE) {  // the first batch was loaded before q was published; only the newest row is read now
+        uint4 kv[B], vv[B];
+#pragma unroll
+        for (int b = 0; b < B; b++) {
+            const int j = gi + b * ngroups;
+            const bool late = j < np && p0 + j == ctx - 1;
+            kv[b] = late ? __ldcg(reinterpret_cast<const uint4 *>(Kp + (size_t)j * D)) : pre->k[b];
+            vv[b] = late ? __ldcg(reinterpret_cast<const uint4 *>(Vp + (size_t)j * D)) : pre->v[b];
+        }
+        batch(0, kv, vv);
+        base0 = ngroups * B;
+    }
+    for (int base = base0; base < np; base += ngroups * B) {  // uniform across the CTA
+        uint4 kv[B], vv[B];
+#pragma unroll
+        for (int b = 0; b < B; b++) {
+            const int j = base + gi + b * ngroups;
+            const bool ok = j < np;
+            kv[b] = ok ? __ldcg(reinterpret_cast<const uint4 *>(Kp + (size_t)j * D)) : make_uint4(0, 0, 0, 0);
+            vv[b] = ok ? __ldcg(reinterpret_cast<const uint4 *>(Vp + (size_t)j * D)) : make_uint4(0, 0, 0, 0);
+        }
+        batch(base, kv, vv);
     }
     // merge the position groups of each warp (lanes with the same sl hold the same dims)
 #pragma unroll
@@ -190,6 +247,7 @@ __device__ void attn_unit(const AttnArgs &A, AttnSmem &S, int unit, int Gt, int 
         named_bar_sync(1, ATTN_THREADS);
     }
 
+    if (tid == 0) S.t_unit = globaltimer();
     // publish this split's partial, then the last split of the kv head merges
     float *pp = A.part + ((size_t)unit * Gt + hoff) * (D + 2);
     for (int i = tid; i < nh * (D + 2) / 2; i += ATTN_THREADS) {  // float2 per thread (D + 2 is even)
@@ -215,19 +273,81 @@ __device__ void attn_unit(const AttnArgs &A, AttnSmem &S, int unit, int Gt, int 
     named_bar_sync(1, ATTN_THREADS);
     if (S.is_last) {
         __threadfence();
+        // All loads of a step are issued before any is used, so the merge costs two L2
+        // round trips whatever the split count: (1) every split's (m, l); (2) per query head
+        // M = max m_k, e_k = 2^(m_k - M) and den = sum e_k l_k; (3) per output pair
+        // num = sum e_k acc_k, the splits shared out over TPP adjacent lanes (each adds its
+        // splits in ascending order, then a fixed shuffle tree), o = num / den.
         const float *pg = A.part + (size_t)g * nsplit * Gt * (D + 2);
-        for (int i = tid; i < Gt * D; i += ATTN_THREADS) {
-            const int jj = i / D, e = i % D;
-            float mxs = -CUDART_INF_F;
-            for (int k = 0; k < nsplit; k++) mxs = fmaxf(mxs, __ldcg(pg + ((size_t)k * Gt + jj) * (D + 2)));
-            float num = 0.f, den = 0.f;
+        float *ek = &S.wacc[0][0];  // [nsplit][Gt] (the warp sums were published above)
+        float *lk = ek + nsplit * Gt;
+        for (int i = tid; i < nsplit * Gt; i += ATTN_THREADS) {
+            const float2 ml = __ldcg(reinterpret_cast<const float2 *>(pg + (size_t)i * (D + 2)));
+            ek[i] = ml.x;
+            lk[i] = ml.y;
+        }
+        named_bar_sync(1, ATTN_THREADS);
+        if (tid < Gt) {
+            float M = -CUDART_INF_F;
+            for (int k = 0; k < nsplit; k++) M = fmaxf(M, ek[k * Gt + tid]);
+            float den = 0.f;
             for (int k = 0; k < nsplit; k++) {
-                const float *pk = pg + ((size_t)k * Gt + jj) * (D + 2);
-                const float wk = rescale(__ldcg(pk), mxs);
-                den = fmaf(wk, __ldcg(pk + 1), den);
-                num = fmaf(wk, __ldcg(pk + 2 + e), num);
+                const float e = rescale(ek[k * Gt + tid], M);
+                ek[k * Gt + tid] = e;
+                den = fmaf(e, lk[k * Gt + tid], den);
             }
-            A.o[(size_t)(g * Gt + jj) * D + e] = num / den;
+            S.red[tid] = den;
+        }
+        named_bar_sync(1, ATTN_THREADS);
+        const int npairs = Gt * D / 2;
+        int tpp = 1;  // lanes per output pair: a power of two <= 16
+        while (tpp < 16 && tpp * 2 * npairs <= ATTN_THREADS) tpp <<= 1;
+        for (int i0 = 0; i0 < npairs * tpp; i0 += ATTN_THREADS) {  // uniform across the CTA
+            const int i = i0 + tid, pr = i / tpp, sub = i % tpp;
+            float2 num = make_float2(0.f, 0.f);
+            const int jj = (2 * pr) / D, e = (2 * pr) % D;
+            if (pr < npairs) {
+                const float *pe = pg + (size_t)jj * (D + 2) + 2 + e;
+                constexpr int MU = NW >= 16 ? 8 : 4;  // loads in flight per lane (register budget)
+                for (int kb = sub; kb < nsplit; kb += MU * tpp) {
+                    float2 v[MU];
+                    float wk[MU];
+#pragma unroll
+                    for (int u = 0; u < MU; u++) {
+                        const int k = kb + u * tpp;
+                        const bool ok = k < nsplit;
+                        v[u] = ok ? __ldcg(reinterpret_cast<const float2 *>(pe + (size_t)k * Gt * (D + 2)))
+                                  : make_float2(0.f, 0.f);
+                        wk[u] = ok ? ek[k * Gt + jj] : 0.f;
+                    }
+#pragma unroll
+                    for (int u = 0; u < MU; u++) {
+                        num.x = fmaf(wk[u], v[u].x, num.x);
+                        num.y = fmaf(wk[u], v[u].y, num.y);
+                    }
+                }
+            }
+            for (int o = 1; o < tpp; o <<= 1) {
+                num.x += __shfl_xor_sync(0xffffffffu, num.x, o);
+                num.y += __shfl_xor_sync(0xffffffffu, num.y, o);
+            }
+            if (pr < npairs && sub == 0) {
+                const float den = S.red[jj];
+                const float o0 = num.x / den, o1 = num.y / den;
+                const int col = (g * Gt + jj) * D + e;
+                if (A.bpack) {
+                    uint8_t *tile = A.bpack + (size_t)(col >> 6) * 16384;
+                    const uint32_t within = (uint32_t)(col & 7) * 2;
+                    const uint16_t h0 = store1<DT>(o0), h1 = store1<DT>(o1);
+                    const uint16_t l0 = store1<DT>(o0 - cvt1<DT>(h0)), l1 = store1<DT>(o1 - cvt1<DT>(h1));
+                    *reinterpret_cast<uint32_t *>(tile + sw128(A.brow, (col >> 3) & 7) + within) =
+                        (uint32_t)h0 | ((uint32_t)h1 << 16);
+                    *reinterpret_cast<uint32_t *>(tile + sw128(64 + A.brow, (col >> 3) & 7) + within) =
+                        (uint32_t)l0 | ((uint32_t)l1 << 16);
+                } else {
+                    *reinterpret_cast<float2 *>(A.o + col) = make_float2(o0, o1);
+                }
+            }
         }
         if (tid == 0) A.cnt[g] = 0u;
     }

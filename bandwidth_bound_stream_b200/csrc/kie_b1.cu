@@ -8,9 +8,11 @@
 //
 //  * Warp 16 (the producer) walks this CTA's fixed weight schedule for the whole command
 //    (all layers, all tokens) and copies it, chunk by chunk, into a 3 x 64 KB shared-memory
-//    ring with 1-D bulk async copies (TMA). An optional second cursor runs `pf_chunks`
-//    chunks further ahead and asks for the same chunks to be brought into L2 (off by
-//    default: measured on B200 it lowers throughput). The schedule is contiguous in HBM
+//    ring with 1-D bulk async copies (TMA). The ring holds 192 KB; while the consumers sit
+//    in attention (which reads no weights) it fills and HBM would idle, so when the producer
+//    reaches the O phase of a layer it also asks L2 for the next `pf_chunks` chunks beyond
+//    the ring (a one-shot prefetch into the bubble; a continuous lead was measured to lower
+//    throughput on B200). The schedule is contiguous in HBM
 //    because the weights were repacked at engine creation in exactly this order, so each SM
 //    streams one disjoint span (the aligned, topology-aware access of the same section).
 //    The producer never waits on grid barriers.
@@ -44,6 +46,8 @@
 namespace {
 
 constexpr int RING_BYTES = KIE_NSLOT * KIE_SLOT_BYTES;
+// phases whose first chunk triggers the one-shot L2 prefetch (the one after attention)
+constexpr unsigned PF_PHASES = 1u << PH_O;
 
 constexpr int WPART_FLOATS = 8 * KIE_ROWACC_MAX;  // column-slice partials: [slices][rows] flattened
 
@@ -143,6 +147,7 @@ __device__ bool grid_barrier(const KieParams &P, B1Shared &S, unsigned long long
 struct ChunkIter {
     const uint8_t *seg, *g;
     int t, l, ph, r;
+    bool first;  // the chunk just returned is the first of its phase
 };
 
 __device__ __forceinline__ void chunk_begin(ChunkIter &it, const uint8_t *seg) {
@@ -152,6 +157,7 @@ __device__ __forceinline__ void chunk_begin(ChunkIter &it, const uint8_t *seg) {
     it.l = 0;
     it.ph = 0;
     it.r = 0;
+    it.first = false;
 }
 
 // Next chunk (address, bytes); false when the command's schedule is exhausted.
@@ -164,6 +170,7 @@ __device__ bool chunk_next(const KieParams &P, const B1Shared &S, const KieCmd &
             const int nr = min(P.cr[it.ph], rows - it.r);
             bytes = (uint32_t)(nr * P.K[it.ph] * 2);
             addr = it.g;
+            it.first = (it.r == 0);
             it.g += bytes;
             it.r += nr;
             return true;
@@ -199,12 +206,10 @@ __device__ bool chunk_next(const KieParams &P, const B1Shared &S, const KieCmd &
 
 __device__ void produce(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint8_t *ring, const KieCmd &cmd) {
     const uint8_t *seg = P.wpack + P.seg_off[blockIdx.x];
-    ChunkIter fetch, pref;
+    ChunkIter fetch;
     chunk_begin(fetch, seg);
-    chunk_begin(pref, seg);
     const uint8_t *a;
     uint32_t b;
-    for (int k = 0; k < P.pf_chunks && chunk_next(P, S, cmd, pref, a, b); k++) bulk_prefetch_l2(a, b);
     unsigned long long waited = 0;
     int tok = 0;
     while (chunk_next(P, S, cmd, fetch, a, b)) {
@@ -229,9 +234,17 @@ __device__ void produce(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint
         mbar_arrive_expect_tx(&S.full[slot], b);
         bulk_g2s(ring + (size_t)slot * KIE_SLOT_BYTES, a, b, &S.full[slot]);
         ring_it++;
-        const uint8_t *a2;
-        uint32_t b2;
-        if (chunk_next(P, S, cmd, pref, a2, b2)) bulk_prefetch_l2(a2, b2);
+        if (P.pf_chunks > 0 && ((PF_PHASES >> fetch.ph) & 1u) && fetch.first) {
+            // the attention bubble: the ring takes this chunk and the next KIE_NSLOT - 1;
+            // the pf_chunks after those start moving into L2 now
+            ChunkIter pf = fetch;
+            const uint8_t *a2;
+            uint32_t b2;
+            bool more = true;
+            for (int k = 0; k < KIE_NSLOT - 1 && more; k++) more = chunk_next(P, S, cmd, pf, a2, b2);
+            for (int k = 0; k < P.pf_chunks && more; k++)
+                if ((more = chunk_next(P, S, cmd, pf, a2, b2))) bulk_prefetch_l2(a2, b2);
+        }
     }
     if (P.trace && tok < P.trace_tokens)
         P.trace[((size_t)blockIdx.x * P.trace_tokens + tok) * P.trace_events + P.trace_events - 1] = waited;
@@ -544,8 +557,13 @@ __device__ int final_argmax(const KieParams &P) {
 
 // --------------------------------------------------------------- consumer: attention
 
-template <int DT>
-__device__ void attention_layer(const KieParams &P, B1Shared &S, int l, int sid, int pos) {
+// The QKV -> attention barrier with this CTA's attention unit around it (at most one unit per
+// CTA: splits = nblk / Hkv). The unit's first batch of K/V rows is loaded before the barrier
+// (all but the newest position are final by then), so those loads overlap the barrier; the
+// query heads of a kv head are taken GC at a time.
+template <int DT, int GC>
+__device__ void attention_step(const KieParams &P, B1Shared &S, int l, int sid, int pos, unsigned long long &epoch,
+                               int t, int e) {
     AttnArgs A;
     A.q = P.q;
     A.k = P.kcache + (size_t)sid * P.sess_stride + (size_t)l * P.Hkv * P.max_ctx * P.D;
@@ -554,11 +572,24 @@ __device__ void attention_layer(const KieParams &P, B1Shared &S, int l, int sid,
     A.part = P.part;
     A.cnt = P.cnt;
     A.o = P.o;
+    A.bpack = nullptr;
+    A.brow = 0;
     A.D = P.D;
     A.Hkv = P.Hkv;
     A.nsplit = P.splits;
     A.ctx = pos + 1;
-    attn_all_units<DT, KIE_CONS_WARPS>(A, S.at, P.G, blockIdx.x, P.nblk);
+    const int unit = blockIdx.x;
+    const bool have = unit < P.Hkv * P.splits;
+    AttnPre<attn_batch<GC, KIE_CONS_WARPS>()> pre;
+    if (have) attn_preload<DT, GC, KIE_CONS_WARPS>(A, unit, pos, pre);
+    grid_barrier(P, S, epoch, P.timeout_ns, 1);
+    trace_mark(P, t, e + 2);
+    if (threadIdx.x == 0) S.at.t_unit = 0;
+    if (have && !S.abort) {
+        attn_unit<DT, GC, KIE_CONS_WARPS, true>(A, S.at, unit, P.G, 0, &pre);
+        for (int hoff = GC; hoff < P.G; hoff += GC) attn_unit<DT, GC, KIE_CONS_WARPS>(A, S.at, unit, P.G, hoff);
+    }
+    trace_mark(P, t, e + 3);
 }
 
 // --------------------------------------------------------------- consumer: one command
@@ -585,10 +616,9 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, cons
             trace_mark(P, t, e);
             epilogue_qkv<DT>(P, S, l, cmd.sid, pos, tok);
             trace_mark(P, t, e + 1);
-            grid_barrier(P, S, epoch, P.timeout_ns, 1);
-            trace_mark(P, t, e + 2);
-            if (!S.abort) attention_layer<DT>(P, S, l, cmd.sid, pos);
-            trace_mark(P, t, e + 3);
+            attention_step<DT, 2>(P, S, l, cmd.sid, pos, epoch, t, e);  // also serves G == 1 (one idle head slot)
+            if (P.trace && t < P.trace_tokens && threadIdx.x == 0)  // end of this CTA's positions (0: no unit)
+                P.trace[((size_t)blockIdx.x * P.trace_tokens + t) * P.trace_events + e + 15] = S.at.t_unit;
             grid_barrier(P, S, epoch, P.timeout_ns, 2);
             trace_mark(P, t, e + 4);
             gemv_dispatch<DT>(P, S, ring_it, ring, PH_O, l, tok, pos, t);

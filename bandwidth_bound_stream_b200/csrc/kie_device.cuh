@@ -144,6 +144,14 @@ KIE_DEV uint16_t store1(float f) {
     return __half_as_ushort(__float2half_rn(f));
 }
 
+// byte offset of 16-byte chunk c (0..7) of row r in a 128 x 64 16-bit tile stored K-major with
+// the 128-byte swizzle (8-row atoms of 1024 B; the MMA operand layout of the tick kernel)
+KIE_DEV uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+// make this thread's generic-proxy global writes visible to later async-proxy (bulk copy)
+// reads, and order its async-proxy reads after its earlier generic accesses
+KIE_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
 KIE_DEV float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

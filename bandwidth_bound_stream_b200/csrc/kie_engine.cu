@@ -396,8 +396,9 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
         CK(eng->alloc(&P.mr_yqkv, (size_t)R * (qd + 2 * kvd) * 4), "cudaMalloc tick scratch");
         CK(eng->alloc(&P.mr_ygu, (size_t)R * 2 * F * 4), "cudaMalloc tick scratch");
         CK(eng->alloc(&P.mr_q, (size_t)R * qd * 4), "cudaMalloc tick scratch");
-        CK(eng->alloc(&P.mr_o, (size_t)R * qd * 4), "cudaMalloc tick scratch");
-        CK(eng->alloc(&P.mr_rstd, (size_t)R * 4), "cudaMalloc tick scratch");
+        const size_t bpack = (size_t)std::max(std::max(d, qd), F) / 64 * 16384;  // one 16 KB tile per k-step
+        CK(eng->alloc(&P.mr_bpack, bpack), "cudaMalloc tick scratch");
+        CK(cudaMemset(P.mr_bpack, 0, bpack), "memset");
         CK(eng->alloc(&P.mr_logits, (size_t)R * V * 4), "cudaMalloc tick scratch");
         CK(eng->alloc(&P.mr_part, (size_t)R * Hkv * G * (D + 2) * 4), "cudaMalloc tick scratch");
         CK(eng->alloc(&P.mr_cnt, (size_t)R * Hkv * 4), "cudaMalloc tick scratch");

@@ -83,7 +83,7 @@ struct KieParams {
     unsigned *last_seq;             // last doorbell sequence processed
     KieCmd *cmd;                    // command broadcast slot
     long long timeout_ns, idle_ns;
-    int pf_chunks;                  // L2 prefetch lead of the weight stream, in ring chunks
+    int pf_chunks;                  // weight chunks beyond the ring requested into L2 at each attention phase
     float *ssq;                     // [nblk] per-CTA sums of squares of the residual rows it owns
     unsigned long long *trace;      // phase stamps (null = off)
     int trace_tokens, trace_events;
@@ -92,7 +92,10 @@ struct KieParams {
     const uint8_t *mr_wpack;
     const long long *mr_seg_off;
     const int *mr_a0;               // [5][nblk+1]
-    float *mr_x, *mr_yqkv, *mr_ygu, *mr_q, *mr_o, *mr_rstd, *mr_logits, *mr_part;
+    float *mr_x, *mr_yqkv, *mr_ygu, *mr_q, *mr_logits, *mr_part;
+    // the B operand of the running GEMM: one swizzled 128 x 64 16-bit tile per k-step (rows
+    // 0-63 hi, 64-127 lo of the activations), written by the phase that finalises them
+    uint8_t *mr_bpack;
     unsigned *mr_cnt;
     int *mr_sid, *mr_pos, *mr_tok;  // [64] rows of the current command
 };

@@ -13,16 +13,19 @@
 // the MMA reads, and streamed by the producer warp with 1-D bulk copies into an 8-slot ring.
 // B holds the activations split into two 16-bit halves: rows 0-63 carry hi(x) and rows
 // 64-127 carry lo(x) = x - hi(x), so D[:, s] + D[:, 64 + s] equals W x_s to about 16 bits of
-// the fp32 activation (the tensor cores take 16-bit operands only). Warps 0-3 build B tiles
-// from the fp32 activations (applying the RMSNorm scale, or silu(gate)*up for the down
-// projection), warp 8 issues tcgen05.mma and commits, warps 4-7 read the accumulator from
-// TMEM and add it into the fp32 outputs with atomics: the weight tiles of one phase are
-// split evenly over the SMs by k-steps, so partial sums of a row block from several SMs meet
-// in global memory.
+// the fp32 activation (the tensor cores take 16-bit operands only). The phase that finalises
+// an activation writes it once, already in that tile layout, to a small global buffer (one
+// tile per k-step: the RMSNorm phases for QKV, gate/up and the head, attention for O, the
+// activation phase silu(gate)*up for down); during the GEMM, thread 0 streams the tile of
+// each k-step from there (L2) into a 4-slot ring with bulk copies, beside the weight tiles.
+// Warp 8 issues tcgen05.mma and commits, warps 4-7 read the accumulator from TMEM and add
+// it into the fp32 outputs with atomics: the weight tiles of one phase are split evenly over
+// the SMs by k-steps, so partial sums of a row block from several SMs meet in global memory.
 //
-// Phases per layer, each ended by a grid barrier: NORM1 (per-row 1/rms, clear the QKV
-// accumulator) | QKV | ROPE (rotate q and k, append K and V) | ATTN | O (+= residual) |
-// NORM2 | GATE/UP | DOWN (+= residual); then NORMF | HEAD | ARGMAX per step.
+// Phases per layer, each ended by a grid barrier: NORM1 (per-row 1/rms -> QKV operand, clear
+// the QKV accumulator) | QKV | ROPE (rotate q and k, append K and V) | ATTN (-> O operand) |
+// O (+= residual) | NORM2 | GATE/UP | ACT | DOWN (+= residual); then NORMF | HEAD | ARGMAX
+// per step.
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
@@ -31,7 +34,7 @@
 
 namespace {
 
-constexpr int MR_THREADS = 320;           // warps 0-3 B builders, 4-7 epilogue, 8 MMA, 9 producer
+constexpr int MR_THREADS = 320;           // warps 0-3 (thread 0: B loads), 4-7 epilogue, 8 MMA, 9 producer
 constexpr int MR_WORKERS = 256;           // warps 0-7 also run the non-GEMM phases
 constexpr int A_SLOTS = 8, B_SLOTS = 4;
 constexpr int TILE = 16384;               // one 128 x 64 16-bit tile
@@ -119,9 +122,6 @@ __host__ __device__ constexpr uint32_t idesc_f16(int dtype) {
            ((128u >> 3) << 17) | ((128u >> 4) << 24);
 }
 
-// byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled tile
-KIE_DEV uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
-
 // ------------------------------------------------------------------ shared helpers
 
 struct Gemm {
@@ -156,6 +156,7 @@ __device__ __forceinline__ void copy_cmd(KieCmd *dst, const KieCmd *src, bool vo
 // grid barrier over warps 0-7 of every CTA (bounded; see the batch-1 kernel)
 __device__ bool mr_barrier(const KieParams &P, MrShared &S, unsigned long long &epoch, long long timeout_ns,
                            unsigned where) {
+    fence_proxy_async_global();  // B-operand tiles written before the barrier are read by bulk copies after it
     named_bar_sync(1, MR_WORKERS);
     if (threadIdx.x == 0) {
         int ok = !S.abort;
@@ -283,88 +284,41 @@ __device__ void mr_mma(const KieParams &P, MrShared &S, uint32_t &a_it, uint32_t
     umma_commit(&S.drain);
 }
 
-// ------------------------------------------------------------------ B-tile builders (warps 0-3)
+// ------------------------------------------------------------------ B operand
 
-// Builds the B tile of k-step ks of GEMM g: rows m < M of the 16-bit hi half, rows 64 + m of
-// the lo half, 64 columns, in the swizzled K-major layout.
+// hi/lo 16-bit halves of 8 consecutive activations -> chunk c of row m (hi) and 64 + m (lo)
+// of a swizzled B tile
 template <int DT>
-__device__ void build_b(const KieParams &P, uint8_t *tile, int g, int l, int ks, int M) {
-    const int t = threadIdx.x;  // 0..127
-    const int m = t >> 1, h = t & 1;
-    const int k0 = ks * 64 + h * 32;
-    float v[32];
-    if (m < M) {
-        if (g == G_O) {
-            const float4 *src = reinterpret_cast<const float4 *>(P.mr_o + (size_t)m * P.Hq * P.D + k0);
+__device__ __forceinline__ void put_b8(uint8_t *tile, int m, int c, const float (&v)[8]) {
+    uint32_t hw[4], lw[4];
 #pragma unroll
-            for (int i = 0; i < 8; i++) {
-                const float4 q = __ldcg(src + i);
-                v[4 * i] = q.x; v[4 * i + 1] = q.y; v[4 * i + 2] = q.z; v[4 * i + 3] = q.w;
-            }
-        } else if (g == G_DOWN) {
-            const float4 *gs = reinterpret_cast<const float4 *>(P.mr_ygu + (size_t)m * 2 * P.F + k0);
-            const float4 *us = reinterpret_cast<const float4 *>(P.mr_ygu + (size_t)m * 2 * P.F + P.F + k0);
-#pragma unroll
-            for (int i = 0; i < 8; i++) {
-                const float4 a = __ldcg(gs + i), b = __ldcg(us + i);
-                const float ga[4] = {a.x, a.y, a.z, a.w}, ub[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-                for (int e = 0; e < 4; e++) v[4 * i + e] = ga[e] / (1.f + expf(-ga[e])) * ub[e];
-            }
-        } else {  // normalised residual
-            const float r = __ldcg(P.mr_rstd + m);
-            const uint16_t *gain = P.gains + (size_t)(g == G_HEAD ? 2 * P.L : 2 * l + (g == G_GU ? 1 : 0)) * P.d;
-            const float4 *src = reinterpret_cast<const float4 *>(P.mr_x + (size_t)m * P.d + k0);
-#pragma unroll
-            for (int i = 0; i < 8; i++) {
-                const float4 q = __ldcg(src + i);
-                const uint2 gw = __ldg(reinterpret_cast<const uint2 *>(gain + k0 + 4 * i));
-                float g0, g1, g2, g3;
-                cvt2<DT>(gw.x, g0, g1);
-                cvt2<DT>(gw.y, g2, g3);
-                v[4 * i] = q.x * r * g0; v[4 * i + 1] = q.y * r * g1; v[4 * i + 2] = q.z * r * g2; v[4 * i + 3] = q.w * r * g3;
-            }
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 32; i++) v[i] = 0.f;
+    for (int j = 0; j < 4; j++) {
+        const float x0 = v[2 * j], x1 = v[2 * j + 1];
+        const uint16_t h0 = store1<DT>(x0), h1 = store1<DT>(x1);
+        const uint16_t l0 = store1<DT>(x0 - cvt1<DT>(h0)), l1 = store1<DT>(x1 - cvt1<DT>(h1));
+        hw[j] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+        lw[j] = (uint32_t)l0 | ((uint32_t)l1 << 16);
     }
-    // hi / lo halves, 8 values per 16-byte chunk
-#pragma unroll
-    for (int c = 0; c < 4; c++) {
-        uint32_t hw[4], lw[4];
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const float x0 = v[8 * c + 2 * j], x1 = v[8 * c + 2 * j + 1];
-            const uint16_t h0 = store1<DT>(x0), h1 = store1<DT>(x1);
-            const uint16_t l0 = store1<DT>(x0 - cvt1<DT>(h0)), l1 = store1<DT>(x1 - cvt1<DT>(h1));
-            hw[j] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-            lw[j] = (uint32_t)l0 | ((uint32_t)l1 << 16);
-        }
-        const int chunk = h * 4 + c;
-        *reinterpret_cast<uint4 *>(tile + sw128(m, chunk)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4 *>(tile + sw128(MAXR + m, chunk)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-    }
+    *reinterpret_cast<uint4 *>(tile + sw128(m, c)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4 *>(tile + sw128(MAXR + m, c)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
 }
 
-template <int DT>
-__device__ void mr_builders(const KieParams &P, MrShared &S, uint32_t &b_it, int g, int l, int M) {
+// Thread 0 during a GEMM phase: the B tile of every k-step this CTA multiplies, in atom
+// order, from the global operand buffer into the B ring (finished by the phase before, and
+// made visible by the grid barrier in between).
+__device__ void mr_bload(const KieParams &P, MrShared &S, uint32_t &b_it, int g) {
     const int nks = gemm_of(P, g).K / 64;
-    const int lane = threadIdx.x & 31;
+    fence_proxy_async_global();
     for (int a = S.a0[g]; a < S.a1[g]; a++) {
         const uint32_t bs = b_it % B_SLOTS;
-        bool ok = !S.abort && mbar_wait(&S.b_empty[bs], ((b_it / B_SLOTS) & 1u) ^ 1u, P.timeout_ns, &S.abort);
-        ok = __all_sync(0xffffffffu, ok);
-        b_it++;
-        if (!ok) {
+        if (S.abort || !mbar_wait(&S.b_empty[bs], ((b_it / B_SLOTS) & 1u) ^ 1u, P.timeout_ns, &S.abort)) {
             if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x92);
             S.abort = 1;
-            continue;
+            return;
         }
-        build_b<DT>(P, S.b[bs], g, l, a % nks, M);
-        fence_proxy_async_smem();  // generic-proxy writes become visible to the tensor cores
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.b_full[bs]);
+        mbar_arrive_expect_tx(&S.b_full[bs], TILE);
+        bulk_g2s(S.b[bs], P.mr_bpack + (size_t)(a % nks) * TILE, TILE, &S.b_full[bs]);
+        b_it++;
     }
 }
 
@@ -412,40 +366,78 @@ __device__ void mr_epilogue(const KieParams &P, MrShared &S, uint32_t &u_it, int
 
 // ------------------------------------------------------------------ worker phases (warps 0-7)
 
-// per-row 1/rms of the residual (one CTA per row), and clear the next GEMM's accumulator
+// Per row (one CTA per row): 1/rms of the residual, then the row of the next GEMM's B operand,
+// x * (1/rms) * gain, in 8-column chunks (the second pass re-reads the row from L2, which
+// keeps the register budget of the 10-warp CTA); also clears the next GEMM's accumulator.
 template <int DT>
-__device__ void phase_norm(const KieParams &P, MrShared &S, int g_next, bool load_emb, int M) {
+__device__ void phase_norm(const KieParams &P, MrShared &S, int g_next, int l, bool load_emb, int M) {
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     if (g_next != G_O) {  // clear rows 0..M-1 of the accumulator of the next GEMM
         const Gemm G = gemm_of(P, g_next);
         const size_t n = (size_t)M * G.ldy;
         for (size_t i = (size_t)blockIdx.x * MR_WORKERS + tid; i < n; i += (size_t)P.nblk * MR_WORKERS) G.y[i] = 0.f;
     }
+    const int nch = P.d >> 3;
+    const uint16_t *gain = P.gains + (size_t)(g_next == G_HEAD ? 2 * P.L : 2 * l + (g_next == G_GU ? 1 : 0)) * P.d;
     for (int m = blockIdx.x; m < M; m += P.nblk) {
         float *x = P.mr_x + (size_t)m * P.d;
         float ss = 0.f;
         if (load_emb) {  // a new step starts from the embedding rows of its input tokens
             const int tok = __ldcg(P.mr_tok + m);
-            for (int j = tid; j < P.d; j += MR_WORKERS) {
-                const float v = cvt1<DT>(P.emb[(size_t)tok * P.d + j]);
-                x[j] = v;
-                ss += v * v;
+            for (int c = tid; c < nch; c += MR_WORKERS) {
+                float v[8];
+                cvt8<DT>(__ldg(reinterpret_cast<const uint4 *>(P.emb + (size_t)tok * P.d + 8 * c)), v);
+                float4 *xd = reinterpret_cast<float4 *>(x + 8 * c);
+                xd[0] = make_float4(v[0], v[1], v[2], v[3]);
+                xd[1] = make_float4(v[4], v[5], v[6], v[7]);
+#pragma unroll
+                for (int e = 0; e < 8; e++) ss += v[e] * v[e];
             }
         } else {
-            for (int j = tid; j < P.d; j += MR_WORKERS) {
-                const float v = __ldcg(x + j);
-                ss += v * v;
+            for (int c = tid; c < nch; c += MR_WORKERS) {
+                const float4 a = __ldcg(reinterpret_cast<const float4 *>(x + 8 * c));
+                const float4 b = __ldcg(reinterpret_cast<const float4 *>(x + 8 * c + 4));
+                ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w + b.x * b.x + b.y * b.y + b.z * b.z + b.w * b.w;
             }
         }
         ss = warp_sum(ss);
         if (lane == 0) S.red[w] = ss;
         named_bar_sync(1, MR_WORKERS);
-        if (tid == 0) {
-            float v = 0.f;
-            for (int k = 0; k < MR_WORKERS / 32; k++) v += S.red[k];
-            P.mr_rstd[m] = rsqrtf(v / (float)P.d + P.eps);
-        }
+        float tot = 0.f;
+        for (int k = 0; k < MR_WORKERS / 32; k++) tot += S.red[k];
+        const float r = rsqrtf(tot / (float)P.d + P.eps);
         named_bar_sync(1, MR_WORKERS);
+        for (int c = tid; c < nch; c += MR_WORKERS) {
+            const float4 a = __ldcg(reinterpret_cast<const float4 *>(x + 8 * c));
+            const float4 b = __ldcg(reinterpret_cast<const float4 *>(x + 8 * c + 4));
+            float gv[8];
+            cvt8<DT>(__ldg(reinterpret_cast<const uint4 *>(gain + 8 * c)), gv);
+            const float v[8] = {a.x * r * gv[0], a.y * r * gv[1], a.z * r * gv[2], a.w * r * gv[3],
+                                b.x * r * gv[4], b.y * r * gv[5], b.z * r * gv[6], b.w * r * gv[7]};
+            put_b8<DT>(P.mr_bpack + (size_t)(c >> 3) * TILE, m, c & 7, v);
+        }
+    }
+}
+
+// the down projection's operand: u = silu(gate) * up, all rows, spread over every CTA
+template <int DT>
+__device__ void phase_act(const KieParams &P, int M) {
+    const int nch = P.F >> 3;
+    const long long n = (long long)M * nch;
+    for (long long i = (long long)blockIdx.x * MR_WORKERS + threadIdx.x; i < n; i += (long long)P.nblk * MR_WORKERS) {
+        const int m = (int)(i / nch), c = (int)(i % nch);
+        const float *gs = P.mr_ygu + (size_t)m * 2 * P.F + 8 * c;
+        const float *us = gs + P.F;
+        float v[8];
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            const float4 a = __ldcg(reinterpret_cast<const float4 *>(gs + 4 * h));
+            const float4 b = __ldcg(reinterpret_cast<const float4 *>(us + 4 * h));
+            const float ga[4] = {a.x, a.y, a.z, a.w}, ub[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int e = 0; e < 4; e++) v[4 * h + e] = ga[e] / (1.f + expf(-ga[e])) * ub[e];
+        }
+        put_b8<DT>(P.mr_bpack + (size_t)(c >> 3) * TILE, m, c & 7, v);
     }
 }
 
@@ -498,7 +490,9 @@ __device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M) {
         A.head_stride = (long long)P.max_ctx * P.D;
         A.part = P.mr_part + (size_t)m * P.Hkv * G * (P.D + 2);
         A.cnt = P.mr_cnt + (size_t)m * P.Hkv;
-        A.o = P.mr_o + (size_t)m * P.Hq * P.D;
+        A.o = nullptr;
+        A.bpack = P.mr_bpack;  // the output is the O projection's B operand, row m
+        A.brow = m;
         A.D = P.D;
         A.Hkv = P.Hkv;
         A.nsplit = 1;
@@ -562,40 +556,46 @@ __device__ void phase_argmax(const KieParams &P, MrShared &S, const KieCmd &cmd,
 
 // ------------------------------------------------------------------ one command, workers' view
 
+// a GEMM phase from the workers' side: thread 0 streams the B tiles, warps 4-7 drain TMEM
+__device__ __forceinline__ void mr_gemm(const KieParams &P, MrShared &S, uint32_t &b_it, uint32_t &u_it, int g, int M) {
+    if (threadIdx.x < 32) {
+        if (threadIdx.x == 0) mr_bload(P, S, b_it, g);
+        __syncwarp();  // warp 0 converges again before the grid barrier's bar.sync
+    } else if (threadIdx.x >= 128) {
+        mr_epilogue(P, S, u_it, g, M);
+    }
+}
+
 template <int DT>
 __device__ void mr_work(const KieParams &P, MrShared &S, uint32_t &b_it, uint32_t &u_it, const KieCmd &cmd,
                         unsigned long long &epoch) {
     const int M = cmd.n_sess;
-    const bool builder = threadIdx.x < 128;
     const int steps = steps_of(cmd);
     for (int st = 0; st < steps; st++) {
         for (int l = 0; l < P.L; l++) {
-            if (!S.abort) phase_norm<DT>(P, S, G_QKV, l == 0, M);
+            if (!S.abort) phase_norm<DT>(P, S, G_QKV, l, l == 0, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 1);
-            if (builder) mr_builders<DT>(P, S, b_it, G_QKV, l, M);
-            else mr_epilogue(P, S, u_it, G_QKV, M);
+            mr_gemm(P, S, b_it, u_it, G_QKV, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 2);
             if (!S.abort) phase_rope<DT>(P, l, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 3);
             if (!S.abort) phase_attn<DT>(P, S, l, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 4);
-            if (builder) mr_builders<DT>(P, S, b_it, G_O, l, M);
-            else mr_epilogue(P, S, u_it, G_O, M);
+            mr_gemm(P, S, b_it, u_it, G_O, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 5);
-            if (!S.abort) phase_norm<DT>(P, S, G_GU, false, M);
+            if (!S.abort) phase_norm<DT>(P, S, G_GU, l, false, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 6);
-            if (builder) mr_builders<DT>(P, S, b_it, G_GU, l, M);
-            else mr_epilogue(P, S, u_it, G_GU, M);
+            mr_gemm(P, S, b_it, u_it, G_GU, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 7);
-            if (builder) mr_builders<DT>(P, S, b_it, G_DOWN, l, M);
-            else mr_epilogue(P, S, u_it, G_DOWN, M);
+            if (!S.abort) phase_act<DT>(P, M);
+            mr_barrier(P, S, epoch, P.timeout_ns, 12);
+            mr_gemm(P, S, b_it, u_it, G_DOWN, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 8);
         }
         if (head_needed(cmd)) {
-            if (!S.abort) phase_norm<DT>(P, S, G_HEAD, false, M);
+            if (!S.abort) phase_norm<DT>(P, S, G_HEAD, P.L, false, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 9);
-            if (builder) mr_builders<DT>(P, S, b_it, G_HEAD, P.L, M);
-            else mr_epilogue(P, S, u_it, G_HEAD, M);
+            mr_gemm(P, S, b_it, u_it, G_HEAD, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 10);
             if (!S.abort) phase_argmax(P, S, cmd, st, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 11);
@@ -618,7 +618,7 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
             mbar_init(&S.a_empty[i], 1);
         }
         for (int i = 0; i < B_SLOTS; i++) {
-            mbar_init(&S.b_full[i], 4);
+            mbar_init(&S.b_full[i], 1);
             mbar_init(&S.b_empty[i], 1);
         }
         for (int i = 0; i < 2; i++) {
@@ -699,6 +699,11 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
             drains++;
         } else {
             mr_work<DT>(P, S, b_it, u_it, cmd, epoch);
+            if (tid == 0) {  // B copies still in flight (only after an abort) land before the CTA moves on
+                const uint32_t first = b_it > B_SLOTS ? b_it - B_SLOTS : 0;
+                for (uint32_t k = first; k < b_it; k++)
+                    mbar_wait(&S.b_full[k % B_SLOTS], (k / B_SLOTS) & 1u, P.timeout_ns, nullptr);
+            }
         }
         __syncthreads();
         if (resident && blockIdx.x == 0 && tid == 0) {

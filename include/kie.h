@@ -69,8 +69,11 @@ typedef struct {
     int32_t idle_ms;      /* the resident kernel exits after this long with no command */
     int32_t modes;        /* KIE_MODE_* bitmask                                        */
     int32_t device;       /* CUDA device ordinal                                       */
-    int32_t prefetch_kb;  /* per-SM lead of the weight stream requested into L2 ahead of
-                             the shared-memory ring, in KB (default 0 = ring only)       */
+    int32_t prefetch_kb;  /* batch-1 kernel: per SM, the KB of weights beyond its shared-
+                             memory ring that are requested into L2 when the consumers
+                             enter attention (which reads no weights), so HBM keeps
+                             streaming through that phase; 0 = ring only. Rounded up to
+                             64 KB ring chunks.                                          */
 } kie_config;
 
 /*
@@ -172,7 +175,8 @@ kie_status kie_tick(kie_engine *eng, int32_t n_sess, const int32_t *sids, const 
  *   0: token start; then per layer 16 slots: 11 phase ends (QKV rows, QKV epilogue, barrier,
  *   attention, barrier, O rows+epilogue, barrier, gate/up rows+epilogue, barrier, down
  *   rows+epilogue, barrier) and 5 inner stamps (input vectors ready in the QKV, O, gate/up
- *   and down phases; attention loads done); then 3 for the head (rows+argmax, barrier, final
+ *   and down phases; end of this CTA's attention positions, before its split is published,
+ *   0 if it had no unit); then 3 for the head (rows+argmax, barrier, final
  *   argmax); then the consumer's and the producer's total ring wait in ns.
  */
 kie_status kie_trace_enable(kie_engine *eng, int32_t tokens);
