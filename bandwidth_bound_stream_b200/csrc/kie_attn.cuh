@@ -67,42 +67,77 @@ __host__ __device__ constexpr int attn_batch() {
     return NW >= 16 ? (GC == 1 ? 4 : 2) : (GC == 1 ? 8 : GC == 2 ? 4 : 2);
 }
 
-// The first batch of K/V rows of a unit, loaded ahead of the barrier that publishes q (every
-// cached position but the newest is final before the QKV phase of a token).
-template <int B>
-struct AttnPre {
-    uint4 k[B], v[B];
-};
-
 // 2^(x - M) with 2^(-inf - M) = 0 (M >= x; M = -inf only when x = -inf)
 KIE_DEV float rescale(float x, float M) { return x == -CUDART_INF_F ? 0.f : exp2f(x - M); }
 
-// Query heads hoff .. hoff+nh-1 (nh <= GC) of the group of kv head `unit / nsplit`, whose
-// group has Gt query heads in all; a kv head with more than 4 query heads is done in chunks
-// of 4 (each chunk re-reads the split's K/V, mostly from L2).
-// Issues the loads of the first batch of `unit` (as attn_unit does), skipping position
-// `newest`, whose row may not be written yet; attn_unit<..., true> consumes them.
-template <int DT, int GC, int NW>
-__device__ __forceinline__ void attn_preload(const AttnArgs &A, int unit, int newest, AttnPre<attn_batch<GC, NW>()> &pre) {
-    constexpr int B = attn_batch<GC, NW>();
-    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-    const int D = A.D, lpp = D >> 3, ppw = 32 / lpp, sub = lane / lpp, sl = lane % lpp;
-    const int ngroups = NW * ppw, gi = w * ppw + sub;
-    const int g = unit / A.nsplit, s = unit % A.nsplit;
-    const int p0 = (int)((long long)s * A.ctx / A.nsplit), p1 = (int)((long long)(s + 1) * A.ctx / A.nsplit);
-    const size_t kvoff = (size_t)g * A.head_stride + (size_t)p0 * D + sl * 8;
+// One batch of a position group: the scores of its B positions base + gi + b * ngroups
+// (those >= np count as -inf) for the G query heads, then the running softmax update of
+// (m, l, acc); the D/8 lanes of a position hold 16-byte slices of its K and V rows.
+template <int DT, int G, int B>
+KIE_DEV void attn_update(const uint4 (&kv)[B], const uint4 (&vv)[B], int base, int np, int gi, int ngroups, int lpp,
+                         const float (&q)[G][8], float (&m)[G], float (&l)[G], float (&acc)[G][8]) {
+    float sc[B][G];
 #pragma unroll
     for (int b = 0; b < B; b++) {
-        const int j = gi + b * ngroups;
-        const bool ok = j < p1 - p0 && p0 + j != newest;
-        pre.k[b] = ok ? __ldcg(reinterpret_cast<const uint4 *>(A.k + kvoff + (size_t)j * D)) : make_uint4(0, 0, 0, 0);
-        pre.v[b] = ok ? __ldcg(reinterpret_cast<const uint4 *>(A.v + kvoff + (size_t)j * D)) : make_uint4(0, 0, 0, 0);
+        const bool ok = base + gi + b * ngroups < np;
+        float f[8];
+        cvt8<DT>(kv[b], f);
+#pragma unroll
+        for (int jj = 0; jj < G; jj++) {
+            float d = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; e++) d = fmaf(f[e], q[jj][e], d);
+            for (int o = lpp >> 1; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+            sc[b][jj] = ok ? d : -CUDART_INF_F;
+        }
+    }
+#pragma unroll
+    for (int jj = 0; jj < G; jj++) {
+        float mb = m[jj];
+#pragma unroll
+        for (int b = 0; b < B; b++) mb = fmaxf(mb, sc[b][jj]);
+        const float r = rescale(m[jj], mb);
+        l[jj] *= r;
+#pragma unroll
+        for (int e = 0; e < 8; e++) acc[jj][e] *= r;
+        m[jj] = mb;
+    }
+#pragma unroll
+    for (int b = 0; b < B; b++) {
+        float f[8];
+        cvt8<DT>(vv[b], f);
+#pragma unroll
+        for (int jj = 0; jj < G; jj++) {
+            const float p = rescale(sc[b][jj], m[jj]);
+            l[jj] += p;
+#pragma unroll
+            for (int e = 0; e < 8; e++) acc[jj][e] = fmaf(p, f[e], acc[jj][e]);
+        }
     }
 }
 
-template <int DT, int GC, int NW, bool PRE = false>
-__device__ void attn_unit(const AttnArgs &A, AttnSmem &S, int unit, int Gt, int hoff,
-                          const AttnPre<attn_batch<GC, NW>()> *pre = nullptr) {
+// output elements col, col + 1 (col even): fp32 to A.o, or hi/lo 16-bit halves into the packed
+// B operand of the tick kernel
+template <int DT>
+KIE_DEV void attn_out2(const AttnArgs &A, int col, float o0, float o1) {
+    if (A.bpack) {
+        uint8_t *tile = A.bpack + (size_t)(col >> 6) * 16384;
+        const uint32_t within = (uint32_t)(col & 7) * 2;
+        const uint16_t h0 = store1<DT>(o0), h1 = store1<DT>(o1);
+        const uint16_t l0 = store1<DT>(o0 - cvt1<DT>(h0)), l1 = store1<DT>(o1 - cvt1<DT>(h1));
+        *reinterpret_cast<uint32_t *>(tile + sw128(A.brow, (col >> 3) & 7) + within) = (uint32_t)h0 | ((uint32_t)h1 << 16);
+        *reinterpret_cast<uint32_t *>(tile + sw128(64 + A.brow, (col >> 3) & 7) + within) = (uint32_t)l0 | ((uint32_t)l1 << 16);
+    } else {
+        *reinterpret_cast<float2 *>(A.o + col) = make_float2(o0, o1);
+    }
+}
+
+template <int DT, int GC, int NW, bool DIRECT>
+__device__ __forceinline__ void attn_tail(const AttnArgs &A, AttnSmem &S, int unit, int Gt, int hoff, float (&m)[GC], float (&l)[GC],
+                          float (&acc)[GC][8]);
+
+template <int DT, int GC, int NW>
+__device__ void attn_unit(const AttnArgs &A, AttnSmem &S, int unit, int Gt, int hoff) {
     constexpr int G = GC;
     constexpr int B = attn_batch<GC, NW>();
     constexpr int ATTN_WARPS = NW, ATTN_THREADS = NW * 32;
@@ -138,61 +173,10 @@ __device__ void attn_unit(const AttnArgs &A, AttnSmem &S, int unit, int Gt, int 
         for (int e = 0; e < 8; e++) acc[jj][e] = 0.f;
     }
 
-    // one batch: scores of B positions per group, then the running softmax update
     auto batch = [&](int base, const uint4 (&kv)[B], const uint4 (&vv)[B]) {
-        float sc[B][G];
-#pragma unroll
-        for (int b = 0; b < B; b++) {
-            const bool ok = base + gi + b * ngroups < np;
-            float f[8];
-            cvt8<DT>(kv[b], f);
-#pragma unroll
-            for (int jj = 0; jj < G; jj++) {
-                float d = 0.f;
-#pragma unroll
-                for (int e = 0; e < 8; e++) d = fmaf(f[e], q[jj][e], d);
-                for (int o = lpp >> 1; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-                sc[b][jj] = ok ? d : -CUDART_INF_F;
-            }
-        }
-#pragma unroll
-        for (int jj = 0; jj < G; jj++) {
-            float mb = m[jj];
-#pragma unroll
-            for (int b = 0; b < B; b++) mb = fmaxf(mb, sc[b][jj]);
-            const float r = rescale(m[jj], mb);
-            l[jj] *= r;
-#pragma unroll
-            for (int e = 0; e < 8; e++) acc[jj][e] *= r;
-            m[jj] = mb;
-        }
-#pragma unroll
-        for (int b = 0; b < B; b++) {
-            float f[8];
-            cvt8<DT>(vv[b], f);
-#pragma unroll
-            for (int jj = 0; jj < G; jj++) {
-                const float p = rescale(sc[b][jj], m[jj]);
-                l[jj] += p;
-#pragma unroll
-                for (int e = 0; e < 8; e++) acc[jj][e] = fmaf(p, f[e], acc[jj][e]);
-            }
-        }
+        attn_update<DT, G, B>(kv, vv, base, np, gi, ngroups, lpp, q, m, l, acc);
     };
-    int base0 = 0;
-    if (PRE) {  // the first batch was loaded before q was published; only the newest row is read now
-        uint4 kv[B], vv[B];
-#pragma unroll
-        for (int b = 0; b < B; b++) {
-            const int j = gi + b * ngroups;
-            const bool late = j < np && p0 + j == ctx - 1;
-            kv[b] = late ? __ldcg(reinterpret_cast<const uint4 *>(Kp + (size_t)j * D)) : pre->k[b];
-            vv[b] = late ? __ldcg(reinterpret_cast<const uint4 *>(Vp + (size_t)j * D)) : pre->v[b];
-        }
-        batch(0, kv, vv);
-        base0 = ngroups * B;
-    }
-    for (int base = base0; base < np; base += ngroups * B) {  // uniform across the CTA
+    for (int base = 0; base < np; base += ngroups * B) {  // uniform across the CTA
         uint4 kv[B], vv[B];
 #pragma unroll
         for (int b = 0; b < B; b++) {
@@ -203,6 +187,24 @@ __device__ void attn_unit(const AttnArgs &A, AttnSmem &S, int unit, int Gt, int 
         }
         batch(base, kv, vv);
     }
+    attn_tail<DT, GC, NW, (NW < 16)>(A, S, unit, Gt, hoff, m, l, acc);
+}
+
+// The end of a unit: merge the position groups and warps of this CTA at their common max;
+// with one split the result is final (o = acc / l: written directly when DIRECT), otherwise
+// publish the split's partial and let the last split of the kv head merge all of them.
+// (The 16-warp batch-1 kernel, whose units always have several splits at its sizes, leaves
+// DIRECT out to keep registers for its main loop; the general merge is exact for one split.)
+template <int DT, int GC, int NW, bool DIRECT>
+__device__ __forceinline__ void attn_tail(const AttnArgs &A, AttnSmem &S, int unit, int Gt, int hoff, float (&m)[GC], float (&l)[GC],
+                          float (&acc)[GC][8]) {
+    constexpr int G = GC;
+    constexpr int ATTN_WARPS = NW, ATTN_THREADS = NW * 32;
+    const int nh = min(GC, Gt - hoff);
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int D = A.D, lpp = D >> 3, sub = lane / lpp, sl = lane % lpp;
+    const int nsplit = A.nsplit;
+    const int g = unit / nsplit;
     // merge the position groups of each warp (lanes with the same sl hold the same dims)
 #pragma unroll
     for (int jj = 0; jj < G; jj++) {
@@ -248,6 +250,17 @@ __device__ void attn_unit(const AttnArgs &A, AttnSmem &S, int unit, int Gt, int 
     }
 
     if (tid == 0) S.t_unit = globaltimer();
+    if (DIRECT && nsplit == 1) {  // the only split: o = acc / l
+        for (int i = tid; i < nh * D / 2; i += ATTN_THREADS) {
+            const int jj = (2 * i) / D, e = (2 * i) % D, k = jj * D + e;
+            const float den = ((S.wl[0][jj] + S.wl[1][jj]) + S.wl[2][jj]) + S.wl[3][jj];
+            const float n0 = ((S.wacc[0][k] + S.wacc[1][k]) + S.wacc[2][k]) + S.wacc[3][k];
+            const float n1 = ((S.wacc[0][k + 1] + S.wacc[1][k + 1]) + S.wacc[2][k + 1]) + S.wacc[3][k + 1];
+            attn_out2<DT>(A, (g * Gt + hoff + jj) * D + e, n0 / den, n1 / den);
+        }
+        named_bar_sync(1, ATTN_THREADS);
+        return;
+    }
     // publish this split's partial, then the last split of the kv head merges
     float *pp = A.part + ((size_t)unit * Gt + hoff) * (D + 2);
     for (int i = tid; i < nh * (D + 2) / 2; i += ATTN_THREADS) {  // float2 per thread (D + 2 is even)
@@ -333,20 +346,7 @@ __device__ void attn_unit(const AttnArgs &A, AttnSmem &S, int unit, int Gt, int 
             }
             if (pr < npairs && sub == 0) {
                 const float den = S.red[jj];
-                const float o0 = num.x / den, o1 = num.y / den;
-                const int col = (g * Gt + jj) * D + e;
-                if (A.bpack) {
-                    uint8_t *tile = A.bpack + (size_t)(col >> 6) * 16384;
-                    const uint32_t within = (uint32_t)(col & 7) * 2;
-                    const uint16_t h0 = store1<DT>(o0), h1 = store1<DT>(o1);
-                    const uint16_t l0 = store1<DT>(o0 - cvt1<DT>(h0)), l1 = store1<DT>(o1 - cvt1<DT>(h1));
-                    *reinterpret_cast<uint32_t *>(tile + sw128(A.brow, (col >> 3) & 7) + within) =
-                        (uint32_t)h0 | ((uint32_t)h1 << 16);
-                    *reinterpret_cast<uint32_t *>(tile + sw128(64 + A.brow, (col >> 3) & 7) + within) =
-                        (uint32_t)l0 | ((uint32_t)l1 << 16);
-                } else {
-                    *reinterpret_cast<float2 *>(A.o + col) = make_float2(o0, o1);
-                }
+                attn_out2<DT>(A, (g * Gt + jj) * D + e, num.x / den, num.y / den);
             }
         }
         if (tid == 0) A.cnt[g] = 0u;

@@ -9,10 +9,9 @@
 //  * Warp 16 (the producer) walks this CTA's fixed weight schedule for the whole command
 //    (all layers, all tokens) and copies it, chunk by chunk, into a 3 x 64 KB shared-memory
 //    ring with 1-D bulk async copies (TMA). The ring holds 192 KB; while the consumers sit
-//    in attention (which reads no weights) it fills and HBM would idle, so when the producer
-//    reaches the O phase of a layer it also asks L2 for the next `pf_chunks` chunks beyond
-//    the ring (a one-shot prefetch into the bubble; a continuous lead was measured to lower
-//    throughput on B200). The schedule is contiguous in HBM
+//    in attention (which reads no weights) it fills and HBM would idle, so a CTA that has
+//    finished its attention unit may ask L2 for the `pf_chunks` chunks beyond the ring (the
+//    producer publishes where it stands; off by default). The schedule is contiguous in HBM
 //    because the weights were repacked at engine creation in exactly this order, so each SM
 //    streams one disjoint span (the aligned, topology-aware access of the same section).
 //    The producer never waits on grid barriers.
@@ -46,8 +45,6 @@
 namespace {
 
 constexpr int RING_BYTES = KIE_NSLOT * KIE_SLOT_BYTES;
-// phases whose first chunk triggers the one-shot L2 prefetch (the one after attention)
-constexpr unsigned PF_PHASES = 1u << PH_O;
 
 constexpr int WPART_FLOATS = 8 * KIE_ROWACC_MAX;  // column-slice partials: [slices][rows] flattened
 
@@ -69,6 +66,8 @@ struct __align__(16) B1Shared {
     int gb_ok;
     int row0[KIE_NPH], row1[KIE_NPH];
     unsigned long long wait_cons;
+    const uint8_t *volatile pf_next;  // the producer's next unfetched byte of the segment
+    const uint8_t *seg_end;
 };
 
 // word-wise copies of the command record (volatile: it may live in mapped host memory)
@@ -147,7 +146,6 @@ __device__ bool grid_barrier(const KieParams &P, B1Shared &S, unsigned long long
 struct ChunkIter {
     const uint8_t *seg, *g;
     int t, l, ph, r;
-    bool first;  // the chunk just returned is the first of its phase
 };
 
 __device__ __forceinline__ void chunk_begin(ChunkIter &it, const uint8_t *seg) {
@@ -157,7 +155,6 @@ __device__ __forceinline__ void chunk_begin(ChunkIter &it, const uint8_t *seg) {
     it.l = 0;
     it.ph = 0;
     it.r = 0;
-    it.first = false;
 }
 
 // Next chunk (address, bytes); false when the command's schedule is exhausted.
@@ -170,7 +167,6 @@ __device__ bool chunk_next(const KieParams &P, const B1Shared &S, const KieCmd &
             const int nr = min(P.cr[it.ph], rows - it.r);
             bytes = (uint32_t)(nr * P.K[it.ph] * 2);
             addr = it.g;
-            it.first = (it.r == 0);
             it.g += bytes;
             it.r += nr;
             return true;
@@ -234,17 +230,7 @@ __device__ void produce(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint
         mbar_arrive_expect_tx(&S.full[slot], b);
         bulk_g2s(ring + (size_t)slot * KIE_SLOT_BYTES, a, b, &S.full[slot]);
         ring_it++;
-        if (P.pf_chunks > 0 && ((PF_PHASES >> fetch.ph) & 1u) && fetch.first) {
-            // the attention bubble: the ring takes this chunk and the next KIE_NSLOT - 1;
-            // the pf_chunks after those start moving into L2 now
-            ChunkIter pf = fetch;
-            const uint8_t *a2;
-            uint32_t b2;
-            bool more = true;
-            for (int k = 0; k < KIE_NSLOT - 1 && more; k++) more = chunk_next(P, S, cmd, pf, a2, b2);
-            for (int k = 0; k < P.pf_chunks && more; k++)
-                if ((more = chunk_next(P, S, cmd, pf, a2, b2))) bulk_prefetch_l2(a2, b2);
-        }
+        S.pf_next = a + b;
     }
     if (P.trace && tok < P.trace_tokens)
         P.trace[((size_t)blockIdx.x * P.trace_tokens + tok) * P.trace_events + P.trace_events - 1] = waited;
@@ -557,10 +543,10 @@ __device__ int final_argmax(const KieParams &P) {
 
 // --------------------------------------------------------------- consumer: attention
 
-// The QKV -> attention barrier with this CTA's attention unit around it (at most one unit per
-// CTA: splits = nblk / Hkv). The unit's first batch of K/V rows is loaded before the barrier
-// (all but the newest position are final by then), so those loads overlap the barrier; the
-// query heads of a kv head are taken GC at a time.
+// The QKV -> attention barrier, then this CTA's attention unit (at most one unit per CTA:
+// splits = nblk / Hkv); the query heads of a kv head are taken GC at a time. (Loading the
+// unit's first K/V batch before the barrier was measured slower: the barrier's release then
+// waits for those loads.)
 template <int DT, int GC>
 __device__ void attention_step(const KieParams &P, B1Shared &S, int l, int sid, int pos, unsigned long long &epoch,
                                int t, int e) {
@@ -580,14 +566,19 @@ __device__ void attention_step(const KieParams &P, B1Shared &S, int l, int sid, 
     A.ctx = pos + 1;
     const int unit = blockIdx.x;
     const bool have = unit < P.Hkv * P.splits;
-    AttnPre<attn_batch<GC, KIE_CONS_WARPS>()> pre;
-    if (have) attn_preload<DT, GC, KIE_CONS_WARPS>(A, unit, pos, pre);
     grid_barrier(P, S, epoch, P.timeout_ns, 1);
     trace_mark(P, t, e + 2);
     if (threadIdx.x == 0) S.at.t_unit = 0;
     if (have && !S.abort) {
-        attn_unit<DT, GC, KIE_CONS_WARPS, true>(A, S.at, unit, P.G, 0, &pre);
-        for (int hoff = GC; hoff < P.G; hoff += GC) attn_unit<DT, GC, KIE_CONS_WARPS>(A, S.at, unit, P.G, hoff);
+        for (int hoff = 0; hoff < P.G; hoff += GC) attn_unit<DT, GC, KIE_CONS_WARPS>(A, S.at, unit, P.G, hoff);
+    }
+    if (P.pf_chunks > 0 && threadIdx.x == 0) {
+        // this CTA's K/V reads are done; while the others finish theirs (and the ring sits full),
+        // the weights beyond the ring start moving into L2
+        const uint8_t *p = S.pf_next;
+        const long long n = min((long long)P.pf_chunks * KIE_SLOT_BYTES, (long long)(S.seg_end - p));
+        for (long long o = 0; o < n; o += KIE_SLOT_BYTES)
+            bulk_prefetch_l2(p + o, (uint32_t)min((long long)KIE_SLOT_BYTES, n - o));
     }
     trace_mark(P, t, e + 3);
 }
@@ -669,6 +660,8 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
         }
         fence_mbar_init();
         S.abort = 0;
+        S.pf_next = P.wpack + P.seg_off[blockIdx.x];
+        S.seg_end = P.wpack + P.seg_off[blockIdx.x + 1];
     }
     if (tid < KIE_NPH) {
         S.row0[tid] = P.row0[tid * (P.nblk + 1) + blockIdx.x];

@@ -49,6 +49,8 @@ struct __align__(1024) MrShared {
     AttnSmem at;
     uint64_t a_full[A_SLOTS], a_empty[A_SLOTS], b_full[B_SLOTS], b_empty[B_SLOTS];
     uint64_t acc_full[2], acc_empty[2], drain;
+    uint64_t k_full[B_SLOTS], k_empty[B_SLOTS];  // the B ring as a K/V chunk ring in attention
+    uint32_t k_iss;                              // K/V chunks issued so far (thread 0)
     uint32_t tmem_base;
     KieCmd cmd;
     volatile int abort;
@@ -309,6 +311,7 @@ __device__ __forceinline__ void put_b8(uint8_t *tile, int m, int c, const float 
 __device__ void mr_bload(const KieParams &P, MrShared &S, uint32_t &b_it, int g) {
     const int nks = gemm_of(P, g).K / 64;
     fence_proxy_async_global();
+    fence_proxy_async_smem();  // attention read the B ring through the generic proxy
     for (int a = S.a0[g]; a < S.a1[g]; a++) {
         const uint32_t bs = b_it % B_SLOTS;
         if (S.abort || !mbar_wait(&S.b_empty[bs], ((b_it / B_SLOTS) & 1u) ^ 1u, P.timeout_ns, &S.abort)) {
@@ -477,8 +480,89 @@ __device__ void phase_rope(const KieParams &P, int l, int M) {
     }
 }
 
+// One (row, kv head) unit of the tick's attention, over the row's whole cache range: thread 0
+// streams the K and V rows in chunks of CP positions with bulk copies into the B ring (idle
+// between GEMM phases; K in the first half of a slot, V in the second), 4 chunks in flight;
+// the 8 worker warps score and accumulate each chunk from shared memory. Query heads
+// hoff .. hoff + GC - 1 of the kv head's Gt.
+template <int DT, int GC>
+__device__ void tick_attn_unit(const KieParams &P, MrShared &S, const AttnArgs &A, int g, int Gt, int hoff,
+                               uint32_t &k_it) {
+    constexpr int NW = MR_WORKERS / 32, B = 2;
+    const int nh = min(GC, Gt - hoff);
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int D = A.D, lpp = D >> 3, ppw = 32 / lpp, sub = lane / lpp, sl = lane % lpp;
+    const int ngroups = NW * ppw, gi = w * ppw + sub;  // ngroups * B == CP for every D
+    const int rowb = D * 2, CP = (TILE / 2) / rowb;
+    const int ctx = A.ctx, nch = (ctx + CP - 1) / CP;
+    const uint8_t *kb = reinterpret_cast<const uint8_t *>(A.k + (size_t)g * A.head_stride);
+    const uint8_t *vb = reinterpret_cast<const uint8_t *>(A.v + (size_t)g * A.head_stride);
+    auto issue = [&](int c) {  // chunk c of this unit into its slot (thread 0)
+        const uint32_t it = k_it + c, slot = it % B_SLOTS;
+        if (S.abort || !mbar_wait(&S.k_empty[slot], ((it / B_SLOTS) & 1u) ^ 1u, P.timeout_ns, &S.abort)) {
+            if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x94);
+            S.abort = 1;
+            return;
+        }
+        const uint32_t bytes = (uint32_t)(min(CP, ctx - c * CP) * rowb);
+        mbar_arrive_expect_tx(&S.k_full[slot], 2 * bytes);
+        bulk_g2s(S.b[slot], kb + (size_t)c * CP * rowb, bytes, &S.k_full[slot]);
+        bulk_g2s(S.b[slot] + TILE / 2, vb + (size_t)c * CP * rowb, bytes, &S.k_full[slot]);
+        S.k_iss = it + 1;
+    };
+    if (tid == 0) {
+        fence_proxy_async_global();  // the newest rows were written (generic proxy) before the barrier
+        for (int c = 0; c < min(B_SLOTS, nch); c++) issue(c);
+    }
+    const float qscale = rsqrtf((float)D) * 1.4426950408889634f;
+    float q[GC][8];
+#pragma unroll
+    for (int jj = 0; jj < GC; jj++) {
+        const float *qp = A.q + (size_t)(g * Gt + hoff + min(jj, nh - 1)) * D + sl * 8;
+        const float4 a = __ldcg(reinterpret_cast<const float4 *>(qp));
+        const float4 b = __ldcg(reinterpret_cast<const float4 *>(qp + 4));
+        q[jj][0] = a.x * qscale; q[jj][1] = a.y * qscale; q[jj][2] = a.z * qscale; q[jj][3] = a.w * qscale;
+        q[jj][4] = b.x * qscale; q[jj][5] = b.y * qscale; q[jj][6] = b.z * qscale; q[jj][7] = b.w * qscale;
+    }
+    float m[GC], l[GC], acc[GC][8];
+#pragma unroll
+    for (int jj = 0; jj < GC; jj++) {
+        m[jj] = -CUDART_INF_F;
+        l[jj] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; e++) acc[jj][e] = 0.f;
+    }
+    for (int c = 0; c < nch; c++) {
+        const uint32_t it = k_it + c, slot = it % B_SLOTS;
+        const bool ok = __all_sync(0xffffffffu, !S.abort && mbar_wait(&S.k_full[slot], (it / B_SLOTS) & 1u,
+                                                                       P.timeout_ns, &S.abort));
+        if (!ok) {
+            if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x95);
+            S.abort = 1;
+            break;
+        }
+        uint4 kv[B], vv[B];
+#pragma unroll
+        for (int b = 0; b < B; b++) {
+            const int jl = gi + b * ngroups;
+            const bool in = c * CP + jl < ctx;
+            kv[b] = in ? *reinterpret_cast<const uint4 *>(S.b[slot] + jl * rowb + sl * 16) : make_uint4(0, 0, 0, 0);
+            vv[b] = in ? *reinterpret_cast<const uint4 *>(S.b[slot] + TILE / 2 + jl * rowb + sl * 16)
+                       : make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.k_empty[slot]);  // this warp's reads of the slot are done
+        attn_update<DT, GC, B>(kv, vv, c * CP, ctx, gi, ngroups, lpp, q, m, l, acc);
+        if (tid == 0 && c + B_SLOTS < nch) issue(c + B_SLOTS);
+    }
+    k_it += nch;
+    attn_tail<DT, GC, NW, true>(A, S.at, g, Gt, hoff, m, l, acc);
+}
+
+// Attention of every row (a tick's sessions or a prefill chunk's positions): one unit per
+// (row, kv head), the unit's output written into the O projection's B operand.
 template <int DT>
-__device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M) {
+__device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M, uint32_t &k_it) {
     const int G = P.G;
     for (int u = blockIdx.x; u < M * P.Hkv; u += P.nblk) {
         const int m = u / P.Hkv, g = u % P.Hkv;
@@ -488,8 +572,8 @@ __device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M) {
         A.k = P.kcache + (size_t)sid * P.sess_stride + (size_t)l * P.Hkv * P.max_ctx * P.D;
         A.v = P.vcache + (size_t)sid * P.sess_stride + (size_t)l * P.Hkv * P.max_ctx * P.D;
         A.head_stride = (long long)P.max_ctx * P.D;
-        A.part = P.mr_part + (size_t)m * P.Hkv * G * (P.D + 2);
-        A.cnt = P.mr_cnt + (size_t)m * P.Hkv;
+        A.part = nullptr;  // one split: the unit's result is final
+        A.cnt = nullptr;
         A.o = nullptr;
         A.bpack = P.mr_bpack;  // the output is the O projection's B operand, row m
         A.brow = m;
@@ -497,15 +581,12 @@ __device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M) {
         A.Hkv = P.Hkv;
         A.nsplit = 1;
         A.ctx = pos + 1;
-        if (G <= 4) {
-            switch (G) {
-                case 1: attn_unit<DT, 1, 8>(A, S.at, g, 1, 0); break;
-                case 2: attn_unit<DT, 2, 8>(A, S.at, g, 2, 0); break;
-                case 3: attn_unit<DT, 3, 8>(A, S.at, g, 3, 0); break;
-                default: attn_unit<DT, 4, 8>(A, S.at, g, 4, 0); break;
-            }
-        } else {
-            for (int hoff = 0; hoff < G; hoff += 4) attn_unit<DT, 4, 8>(A, S.at, g, G, hoff);
+        switch (G) {
+            case 1: tick_attn_unit<DT, 1>(P, S, A, g, 1, 0, k_it); break;
+            case 2: tick_attn_unit<DT, 2>(P, S, A, g, 2, 0, k_it); break;
+            case 3: tick_attn_unit<DT, 3>(P, S, A, g, 3, 0, k_it); break;
+            default:
+                for (int hoff = 0; hoff < G; hoff += 4) tick_attn_unit<DT, 4>(P, S, A, g, G, hoff, k_it);
         }
     }
 }
@@ -517,7 +598,8 @@ __device__ __forceinline__ void amax(float &v, int &i, float v2, int i2) {
     }
 }
 
-// argmax of each row's logits (one CTA per row); outputs and the next step's inputs
+// argmax of each row's logits (one CTA per row); outputs and the next step's inputs. The
+// row is read as float4 with 8 loads in flight per thread (lowest index wins ties).
 __device__ void phase_argmax(const KieParams &P, MrShared &S, const KieCmd &cmd, int step, int M) {
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     for (int m = blockIdx.x; m < M; m += P.nblk) {
@@ -527,12 +609,41 @@ __device__ void phase_argmax(const KieParams &P, MrShared &S, const KieCmd &cmd,
         const bool copy = cmd.logits && (cmd.op == OP_TICK || m == M - 1);
         float *dst = nullptr;
         if (copy) dst = cmd.logits + (cmd.op == OP_TICK ? ((size_t)step * M + m) * P.V : 0);
-        for (int r = tid; r < P.V; r += MR_WORKERS) {
+        // rows start 16-byte aligned when V % 4 == 0; otherwise take the scalar path
+        const int n4 = (P.V % 4 == 0) ? P.V / 4 : 0;
+        const float4 *lg4 = reinterpret_cast<const float4 *>(lg);
+        const bool dst4 = dst && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0;  // caller's buffer may be unaligned
+        for (int r0 = tid; r0 < n4; r0 += MR_WORKERS * 8) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                const int r = r0 + u * MR_WORKERS;
+                v[u] = r < n4 ? __ldcg(lg4 + r) : make_float4(-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                const int r = r0 + u * MR_WORKERS;
+                if (r < n4) {
+                    if (dst4) {
+                        reinterpret_cast<float4 *>(dst)[r] = v[u];
+                    } else if (dst) {
+                        dst[4 * r] = v[u].x;
+                        dst[4 * r + 1] = v[u].y;
+                        dst[4 * r + 2] = v[u].z;
+                        dst[4 * r + 3] = v[u].w;
+                    }
+                    amax(bv, bi, v[u].x, 4 * r);
+                    amax(bv, bi, v[u].y, 4 * r + 1);
+                    amax(bv, bi, v[u].z, 4 * r + 2);
+                    amax(bv, bi, v[u].w, 4 * r + 3);
+                }
+            }
+        }
+        for (int r = 4 * n4 + tid; r < P.V; r += MR_WORKERS) {
             const float v = __ldcg(lg + r);
             if (dst) dst[r] = v;
             amax(bv, bi, v, r);
         }
-#pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax(bv, bi, __shfl_xor_sync(0xffffffffu, bv, o), __shfl_xor_sync(0xffffffffu, bi, o));
         if (lane == 0) {
             S.red[w] = bv;
@@ -566,39 +677,63 @@ __device__ __forceinline__ void mr_gemm(const KieParams &P, MrShared &S, uint32_
     }
 }
 
+// phase trace (thread 0 of each CTA; same record layout as the batch-1 kernel, one record per
+// step of the command)
+__device__ __forceinline__ void mr_mark(const KieParams &P, int st, int ev) {
+    if (P.trace && st < P.trace_tokens && threadIdx.x == 0)
+        P.trace[((size_t)blockIdx.x * P.trace_tokens + st) * P.trace_events + ev] = globaltimer();
+}
+
 template <int DT>
-__device__ void mr_work(const KieParams &P, MrShared &S, uint32_t &b_it, uint32_t &u_it, const KieCmd &cmd,
-                        unsigned long long &epoch) {
+__device__ void mr_work(const KieParams &P, MrShared &S, uint32_t &b_it, uint32_t &u_it, uint32_t &k_it,
+                        const KieCmd &cmd, unsigned long long &epoch) {
     const int M = cmd.n_sess;
     const int steps = steps_of(cmd);
     for (int st = 0; st < steps; st++) {
+        mr_mark(P, st, 0);
         for (int l = 0; l < P.L; l++) {
+            const int e = 1 + 16 * l;
             if (!S.abort) phase_norm<DT>(P, S, G_QKV, l, l == 0, M);
+            mr_mark(P, st, e);
             mr_barrier(P, S, epoch, P.timeout_ns, 1);
+            mr_mark(P, st, e + 1);
             mr_gemm(P, S, b_it, u_it, G_QKV, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 2);
+            mr_mark(P, st, e + 3);
             if (!S.abort) phase_rope<DT>(P, l, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 3);
-            if (!S.abort) phase_attn<DT>(P, S, l, M);
+            mr_mark(P, st, e + 4);
+            if (!S.abort) phase_attn<DT>(P, S, l, M, k_it);
+            mr_mark(P, st, e + 5);
             mr_barrier(P, S, epoch, P.timeout_ns, 4);
+            mr_mark(P, st, e + 6);
             mr_gemm(P, S, b_it, u_it, G_O, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 5);
+            mr_mark(P, st, e + 7);
             if (!S.abort) phase_norm<DT>(P, S, G_GU, l, false, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 6);
+            mr_mark(P, st, e + 8);
             mr_gemm(P, S, b_it, u_it, G_GU, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 7);
+            mr_mark(P, st, e + 9);
             if (!S.abort) phase_act<DT>(P, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 12);
+            mr_mark(P, st, e + 10);
             mr_gemm(P, S, b_it, u_it, G_DOWN, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 8);
+            mr_mark(P, st, e + 11);
         }
         if (head_needed(cmd)) {
+            const int eh = 1 + 16 * P.L;
             if (!S.abort) phase_norm<DT>(P, S, G_HEAD, P.L, false, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 9);
+            mr_mark(P, st, eh);
             mr_gemm(P, S, b_it, u_it, G_HEAD, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 10);
+            mr_mark(P, st, eh + 1);
             if (!S.abort) phase_argmax(P, S, cmd, st, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 11);
+            mr_mark(P, st, eh + 2);
         }
     }
 }
@@ -626,6 +761,11 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
             mbar_init(&S.acc_empty[i], 4);
         }
         mbar_init(&S.drain, 1);
+        for (int i = 0; i < B_SLOTS; i++) {
+            mbar_init(&S.k_full[i], 1);
+            mbar_init(&S.k_empty[i], MR_WORKERS / 32);
+        }
+        S.k_iss = 0;
         fence_mbar_init();
         S.abort = 0;
     }
@@ -641,7 +781,7 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
     __syncthreads();
     tc_fence_after();
 
-    uint32_t a_it = 0, b_it = 0, u_it = 0, drains = 0;
+    uint32_t a_it = 0, b_it = 0, u_it = 0, k_it = 0, drains = 0;
     unsigned long long epoch = 0;
     for (;;) {
         if (tid < MR_WORKERS) {
@@ -698,11 +838,14 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
             }
             drains++;
         } else {
-            mr_work<DT>(P, S, b_it, u_it, cmd, epoch);
-            if (tid == 0) {  // B copies still in flight (only after an abort) land before the CTA moves on
+            mr_work<DT>(P, S, b_it, u_it, k_it, cmd, epoch);
+            if (tid == 0) {  // copies still in flight (only after an abort) land before the CTA moves on
                 const uint32_t first = b_it > B_SLOTS ? b_it - B_SLOTS : 0;
                 for (uint32_t k = first; k < b_it; k++)
                     mbar_wait(&S.b_full[k % B_SLOTS], (k / B_SLOTS) & 1u, P.timeout_ns, nullptr);
+                const uint32_t kfirst = S.k_iss > B_SLOTS ? S.k_iss - B_SLOTS : 0;
+                for (uint32_t k = kfirst; k < S.k_iss; k++)
+                    mbar_wait(&S.k_full[k % B_SLOTS], (k / B_SLOTS) & 1u, P.timeout_ns, nullptr);
             }
         }
         __syncthreads();

@@ -70,10 +70,10 @@ typedef struct {
     int32_t modes;        /* KIE_MODE_* bitmask                                        */
     int32_t device;       /* CUDA device ordinal                                       */
     int32_t prefetch_kb;  /* batch-1 kernel: per SM, the KB of weights beyond its shared-
-                             memory ring that are requested into L2 when the consumers
-                             enter attention (which reads no weights), so HBM keeps
-                             streaming through that phase; 0 = ring only. Rounded up to
-                             64 KB ring chunks.                                          */
+                             memory ring that a CTA requests into L2 once it has finished
+                             its attention unit (attention reads no weights, so HBM would
+                             otherwise idle while the other units finish); 0 = ring only.
+                             Rounded up to 64 KB ring chunks.                            */
 } kie_config;
 
 /*
@@ -167,17 +167,24 @@ kie_status kie_tick(kie_engine *eng, int32_t n_sess, const int32_t *sids, const 
                     int32_t *out_tokens, float *logits_dev);
 
 /*
- * Phase trace (observability). kie_trace_enable(eng, tokens) makes every later decode
- * command record, for its first `tokens` tokens, a globaltimer stamp (ns) per CTA at each
- * phase boundary, plus per-token ring wait totals; tokens = 0 turns it off. kie_trace_read
+ * Phase trace (observability). kie_trace_enable(eng, tokens) makes every later command
+ * record, for its first `tokens` tokens (batch-1 decode) or steps (tick, chunked prefill), a
+ * globaltimer stamp (ns) per CTA at each phase boundary; tokens = 0 turns it off. Each
+ * command overwrites the record of the one before. kie_trace_read
  * copies the record into `host` (uint64, at most max_elems) and returns the element count
  * through *n; layout [cta][token][event], events per token = kie_trace_events(eng):
+ * Batch-1 decode commands write one record per token:
  *   0: token start; then per layer 16 slots: 11 phase ends (QKV rows, QKV epilogue, barrier,
  *   attention, barrier, O rows+epilogue, barrier, gate/up rows+epilogue, barrier, down
  *   rows+epilogue, barrier) and 5 inner stamps (input vectors ready in the QKV, O, gate/up
  *   and down phases; end of this CTA's attention positions, before its split is published,
  *   0 if it had no unit); then 3 for the head (rows+argmax, barrier, final
  *   argmax); then the consumer's and the producer's total ring wait in ns.
+ * Tick and chunked-prefill commands write one record per step, in the same layout:
+ *   0: step start; per layer (slot 1 + 16 l + k): k = 0 first norm done, then the ends of
+ *   the grid barriers after: 1 first norm, 3 QKV, 4 RoPE, 6 attention (5: this CTA's
+ *   attention done, before the barrier), 7 O, 8 second norm, 9 gate/up, 10 activation,
+ *   11 down; head (slot 1 + 16 L + k): 0 final norm, 1 head rows, 2 argmax.
  */
 kie_status kie_trace_enable(kie_engine *eng, int32_t tokens);
 kie_status kie_trace_read(kie_engine *eng, uint64_t *host, int64_t max_elems, int64_t *n);
