@@ -70,7 +70,7 @@ def build_kie(force: bool = False, verbose_ptxas: bool = False) -> str:
             sys.stdout.write(log)
     if failed:
         raise RuntimeError("nvcc failed")
-    _run([NVCC, *ARCH, "-shared", "-o", out, *objs, "-lcuda"])
+    _run([NVCC, *ARCH, "-shared", "-o", out, *objs])  # the CUDA runtime only (no driver library at link time)
     return out
 
 

@@ -6,6 +6,7 @@
 // at run time ("实时AI推理为何贵56倍？…", section 把一切提前决定好). Per call the host only
 // writes input tokens into a mapped mailbox and reads output tokens back (same page,
 // section 让工作常驻 GPU).
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <emmintrin.h>
 
@@ -199,6 +200,12 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
         kie_destroy(eng);
         return s;
     };
+    // a failed CUDA call releases everything allocated so far
+#define CKC(expr, what)                                               \
+    do {                                                              \
+        cudaError_t _e = (expr);                                      \
+        if (_e != cudaSuccess) return bail(eng->cuda_fail(_e, what)); \
+    } while (0)
     const bool b1 = (c.modes & KIE_MODE_BATCH1) != 0, mr = (c.modes & KIE_MODE_TICK) != 0;
     cudaError_t e = cudaSetDevice(c.device);
     if (e != cudaSuccess) return bail(eng->cuda_fail(e, "cudaSetDevice"));
@@ -278,7 +285,7 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
         seg_off[cc + 1] = seg_off[cc] + (long long)L * lb + hb;
     }
     uint8_t *wpack = nullptr;
-    CK(eng->alloc(&wpack, (size_t)seg_off[nblk]), "cudaMalloc packed weights");
+    CKC(eng->alloc(&wpack, (size_t)seg_off[nblk]), "cudaMalloc packed weights");
     P.wpack = wpack;
     {
         std::vector<RowCopy> rc;
@@ -309,7 +316,7 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
             }
         }
         RowCopy *d_rc = nullptr;
-        CK(cudaMalloc(&d_rc, rc.size() * sizeof(RowCopy)), "cudaMalloc repack list");
+        CKC(cudaMalloc(&d_rc, rc.size() * sizeof(RowCopy)), "cudaMalloc repack list");
         e = cudaMemcpy(d_rc, rc.data(), rc.size() * sizeof(RowCopy), cudaMemcpyHostToDevice);
         if (e == cudaSuccess) {
             gather_rows_kernel<<<4 * nblk, 256>>>(d_rc, (long long)rc.size(), wpack);
@@ -321,10 +328,10 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
     }
     int *d_row0 = nullptr;
     long long *d_seg = nullptr;
-    CK(eng->alloc(&d_row0, row0.size() * sizeof(int)), "cudaMalloc plan");
-    CK(eng->alloc(&d_seg, seg_off.size() * sizeof(long long)), "cudaMalloc plan");
-    CK(cudaMemcpy(d_row0, row0.data(), row0.size() * sizeof(int), cudaMemcpyHostToDevice), "upload plan");
-    CK(cudaMemcpy(d_seg, seg_off.data(), seg_off.size() * sizeof(long long), cudaMemcpyHostToDevice), "upload plan");
+    CKC(eng->alloc(&d_row0, row0.size() * sizeof(int)), "cudaMalloc plan");
+    CKC(eng->alloc(&d_seg, seg_off.size() * sizeof(long long)), "cudaMalloc plan");
+    CKC(cudaMemcpy(d_row0, row0.data(), row0.size() * sizeof(int), cudaMemcpyHostToDevice), "upload plan");
+    CKC(cudaMemcpy(d_seg, seg_off.data(), seg_off.size() * sizeof(long long), cudaMemcpyHostToDevice), "upload plan");
     P.row0 = d_row0;
     P.seg_off = d_seg;
     }  // batch-1 kernel
@@ -348,7 +355,7 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
             mseg[cc + 1] = mseg[cc] + tiles * 16384;
         }
         uint8_t *mpack = nullptr;
-        CK(eng->alloc(&mpack, (size_t)mseg[nblk]), "cudaMalloc tick weights");
+        CKC(eng->alloc(&mpack, (size_t)mseg[nblk]), "cudaMalloc tick weights");
         const size_t tsz = kie_mr_tile_src_bytes();
         std::vector<uint8_t> desc((size_t)(mseg[nblk] / 16384) * tsz);
         size_t nt = 0;
@@ -376,7 +383,7 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
             }
         }
         void *d_desc = nullptr;
-        CK(cudaMalloc(&d_desc, desc.size()), "cudaMalloc tick repack list");
+        CKC(cudaMalloc(&d_desc, desc.size()), "cudaMalloc tick repack list");
         e = cudaMemcpy(d_desc, desc.data(), desc.size(), cudaMemcpyHostToDevice);
         if (e == cudaSuccess) e = kie_mr_repack(d_desc, (long long)nt, mpack, 0);
         if (e == cudaSuccess) e = cudaDeviceSynchronize();
@@ -384,41 +391,41 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
         if (e != cudaSuccess) return bail(eng->cuda_fail(e, "tick weight repack"));
         int *d_a0 = nullptr;
         long long *d_mseg = nullptr;
-        CK(eng->alloc(&d_a0, a0.size() * sizeof(int)), "cudaMalloc tick plan");
-        CK(eng->alloc(&d_mseg, mseg.size() * sizeof(long long)), "cudaMalloc tick plan");
-        CK(cudaMemcpy(d_a0, a0.data(), a0.size() * sizeof(int), cudaMemcpyHostToDevice), "upload tick plan");
-        CK(cudaMemcpy(d_mseg, mseg.data(), mseg.size() * sizeof(long long), cudaMemcpyHostToDevice), "upload tick plan");
+        CKC(eng->alloc(&d_a0, a0.size() * sizeof(int)), "cudaMalloc tick plan");
+        CKC(eng->alloc(&d_mseg, mseg.size() * sizeof(long long)), "cudaMalloc tick plan");
+        CKC(cudaMemcpy(d_a0, a0.data(), a0.size() * sizeof(int), cudaMemcpyHostToDevice), "upload tick plan");
+        CKC(cudaMemcpy(d_mseg, mseg.data(), mseg.size() * sizeof(long long), cudaMemcpyHostToDevice), "upload tick plan");
         P.mr_wpack = mpack;
         P.mr_a0 = d_a0;
         P.mr_seg_off = d_mseg;
         const int R = 64;  // rows per step
-        CK(eng->alloc(&P.mr_x, (size_t)R * d * 4), "cudaMalloc tick scratch");
-        CK(eng->alloc(&P.mr_yqkv, (size_t)R * (qd + 2 * kvd) * 4), "cudaMalloc tick scratch");
-        CK(eng->alloc(&P.mr_ygu, (size_t)R * 2 * F * 4), "cudaMalloc tick scratch");
-        CK(eng->alloc(&P.mr_q, (size_t)R * qd * 4), "cudaMalloc tick scratch");
+        CKC(eng->alloc(&P.mr_x, (size_t)R * d * 4), "cudaMalloc tick scratch");
+        CKC(eng->alloc(&P.mr_yqkv, (size_t)R * (qd + 2 * kvd) * 4), "cudaMalloc tick scratch");
+        CKC(eng->alloc(&P.mr_ygu, (size_t)R * 2 * F * 4), "cudaMalloc tick scratch");
+        CKC(eng->alloc(&P.mr_q, (size_t)R * qd * 4), "cudaMalloc tick scratch");
         const size_t bpack = (size_t)std::max(std::max(d, qd), F) / 64 * 16384;  // one 16 KB tile per k-step
-        CK(eng->alloc(&P.mr_bpack, bpack), "cudaMalloc tick scratch");
-        CK(cudaMemset(P.mr_bpack, 0, bpack), "memset");
-        CK(eng->alloc(&P.mr_logits, (size_t)R * V * 4), "cudaMalloc tick scratch");
-        CK(eng->alloc(&P.mr_part, (size_t)R * Hkv * G * (D + 2) * 4), "cudaMalloc tick scratch");
-        CK(eng->alloc(&P.mr_cnt, (size_t)R * Hkv * 4), "cudaMalloc tick scratch");
-        CK(eng->alloc(&P.mr_sid, (size_t)R * 4), "cudaMalloc tick scratch");
-        CK(eng->alloc(&P.mr_pos, (size_t)R * 4), "cudaMalloc tick scratch");
-        CK(eng->alloc(&P.mr_tok, (size_t)R * 4), "cudaMalloc tick scratch");
-        CK(cudaMemset(P.mr_cnt, 0, (size_t)R * Hkv * 4), "memset");
-        CK(cudaMemset(P.mr_x, 0, (size_t)R * d * 4), "memset");
+        CKC(eng->alloc(&P.mr_bpack, bpack), "cudaMalloc tick scratch");
+        CKC(cudaMemset(P.mr_bpack, 0, bpack), "memset");
+        CKC(eng->alloc(&P.mr_logits, (size_t)R * V * 4), "cudaMalloc tick scratch");
+        CKC(eng->alloc(&P.mr_part, (size_t)R * Hkv * G * (D + 2) * 4), "cudaMalloc tick scratch");
+        CKC(eng->alloc(&P.mr_cnt, (size_t)R * Hkv * 4), "cudaMalloc tick scratch");
+        CKC(eng->alloc(&P.mr_sid, (size_t)R * 4), "cudaMalloc tick scratch");
+        CKC(eng->alloc(&P.mr_pos, (size_t)R * 4), "cudaMalloc tick scratch");
+        CKC(eng->alloc(&P.mr_tok, (size_t)R * 4), "cudaMalloc tick scratch");
+        CKC(cudaMemset(P.mr_cnt, 0, (size_t)R * Hkv * 4), "memset");
+        CKC(cudaMemset(P.mr_x, 0, (size_t)R * d * 4), "memset");
     }
 
     // ---- small weights: embedding table and norm gains
     uint16_t *emb = nullptr, *gains = nullptr;
-    CK(eng->alloc(&emb, (size_t)V * d * 2), "cudaMalloc embedding");
-    CK(cudaMemcpy(emb, w->tok_emb, (size_t)V * d * 2, cudaMemcpyDeviceToDevice), "copy embedding");
-    CK(eng->alloc(&gains, (size_t)(2 * L + 1) * d * 2), "cudaMalloc gains");
+    CKC(eng->alloc(&emb, (size_t)V * d * 2), "cudaMalloc embedding");
+    CKC(cudaMemcpy(emb, w->tok_emb, (size_t)V * d * 2, cudaMemcpyDeviceToDevice), "copy embedding");
+    CKC(eng->alloc(&gains, (size_t)(2 * L + 1) * d * 2), "cudaMalloc gains");
     for (int l = 0; l < L; l++) {
-        CK(cudaMemcpy(gains + (size_t)(2 * l) * d, w->layers[9 * l + 0], (size_t)d * 2, cudaMemcpyDeviceToDevice), "gains");
-        CK(cudaMemcpy(gains + (size_t)(2 * l + 1) * d, w->layers[9 * l + 5], (size_t)d * 2, cudaMemcpyDeviceToDevice), "gains");
+        CKC(cudaMemcpy(gains + (size_t)(2 * l) * d, w->layers[9 * l + 0], (size_t)d * 2, cudaMemcpyDeviceToDevice), "gains");
+        CKC(cudaMemcpy(gains + (size_t)(2 * l + 1) * d, w->layers[9 * l + 5], (size_t)d * 2, cudaMemcpyDeviceToDevice), "gains");
     }
-    CK(cudaMemcpy(gains + (size_t)(2 * L) * d, w->final_norm, (size_t)d * 2, cudaMemcpyDeviceToDevice), "gains");
+    CKC(cudaMemcpy(gains + (size_t)(2 * L) * d, w->final_norm, (size_t)d * 2, cudaMemcpyDeviceToDevice), "gains");
     P.emb = emb;
     P.gains = gains;
 
@@ -431,55 +438,91 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
                 rope[(size_t)p * (D / 2) + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
             }
         float2 *d_rope = nullptr;
-        CK(eng->alloc(&d_rope, rope.size() * sizeof(float2)), "cudaMalloc rope");
-        CK(cudaMemcpy(d_rope, rope.data(), rope.size() * sizeof(float2), cudaMemcpyHostToDevice), "upload rope");
+        CKC(eng->alloc(&d_rope, rope.size() * sizeof(float2)), "cudaMalloc rope");
+        CKC(cudaMemcpy(d_rope, rope.data(), rope.size() * sizeof(float2), cudaMemcpyHostToDevice), "upload rope");
         P.rope = d_rope;
     }
 
     // ---- KV cache for every session slot
     P.sess_stride = (long long)L * Hkv * c.max_ctx * D;
-    CK(eng->alloc(&P.kcache, (size_t)c.max_sessions * P.sess_stride * 2), "cudaMalloc K cache");
-    CK(eng->alloc(&P.vcache, (size_t)c.max_sessions * P.sess_stride * 2), "cudaMalloc V cache");
+    CKC(eng->alloc(&P.kcache, (size_t)c.max_sessions * P.sess_stride * 2), "cudaMalloc K cache");
+    CKC(eng->alloc(&P.vcache, (size_t)c.max_sessions * P.sess_stride * 2), "cudaMalloc V cache");
+    // the tick kernel's attention reads K tiles by 2-D TMA: the K arena as [rows][D], rows =
+    // sessions * L * Hkv * max_ctx (one per cached position), boxes of 128 rows x 64 dims,
+    // 128-byte swizzled (the MMA operand layout); head_dim not a multiple of 64 keeps the
+    // CUDA-core attention
+    P.mr_kmap = nullptr;
+    const unsigned long long kv_rows = (unsigned long long)c.max_sessions * L * Hkv * c.max_ctx;
+    if (mr && D % 64 == 0 && kv_rows < (1ull << 31)) {
+        // the driver's encoder, looked up through the runtime (no link-time driver dependency)
+        typedef CUresult (*EncodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                        const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                        CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        CKC(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q), "driver entry point");
+        if (!fn || q != cudaDriverEntryPointSuccess) {
+            eng->fail(KIE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+            return bail(KIE_ERR_CUDA);
+        }
+        CUtensorMap tm;
+        const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)kv_rows};
+        const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+        const cuuint32_t box[2] = {64, 128}, estr[2] = {1, 1};
+        const CUresult r = reinterpret_cast<EncodeTiled>(fn)(
+            &tm, c.dtype == KIE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, P.kcache, dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            eng->fail(KIE_ERR_CUDA, "cuTensorMapEncodeTiled (K arena) failed: %d", (int)r);
+            return bail(KIE_ERR_CUDA);
+        }
+        void *d_map = nullptr;
+        CKC(eng->alloc(&d_map, sizeof(CUtensorMap)), "cudaMalloc tensor map");
+        CKC(cudaMemcpy(d_map, &tm, sizeof(CUtensorMap), cudaMemcpyHostToDevice), "upload tensor map");
+        P.mr_kmap = d_map;
+    }
 
     // ---- activations and scratch
-    CK(eng->alloc(&P.x, (size_t)d * 4), "cudaMalloc x");
-    CK(eng->alloc(&P.q, (size_t)qd * 4), "cudaMalloc q");
-    CK(eng->alloc(&P.o, (size_t)qd * 4), "cudaMalloc o");
-    CK(eng->alloc(&P.u, (size_t)F * 4), "cudaMalloc u");
-    CK(eng->alloc(&P.part, (size_t)Hkv * P.splits * G * (D + 2) * 4), "cudaMalloc partials");
-    CK(eng->alloc(&P.cnt, (size_t)Hkv * 4), "cudaMalloc counters");
-    CK(eng->alloc(&P.cand_val, (size_t)nblk * 4), "cudaMalloc candidates");
-    CK(eng->alloc(&P.cand_idx, (size_t)nblk * 4), "cudaMalloc candidates");
-    CK(eng->alloc(&P.tokbuf, (size_t)c.max_ctx * 4), "cudaMalloc token buffer");
-    CK(eng->alloc(&P.bar, 16), "cudaMalloc barrier");
-    CK(eng->alloc(&P.err, 16), "cudaMalloc error word");
-    CK(eng->alloc(&P.last_seq, 16), "cudaMalloc sequence");
-    CK(eng->alloc(&P.cmd, sizeof(KieCmd)), "cudaMalloc command");
-    CK(eng->alloc(&P.ssq, (size_t)nblk * 4), "cudaMalloc norm partials");
-    CK(cudaMemset(P.ssq, 0, (size_t)nblk * 4), "memset");
-    CK(cudaMemset(P.cnt, 0, (size_t)Hkv * 4), "memset");
-    CK(cudaMemset(P.bar, 0, 16), "memset");
-    CK(cudaMemset(P.err, 0, 16), "memset");
-    CK(cudaMemset(P.last_seq, 0, 16), "memset");
-    CK(cudaMemset(P.x, 0, (size_t)d * 4), "memset");
+    CKC(eng->alloc(&P.x, (size_t)d * 4), "cudaMalloc x");
+    CKC(eng->alloc(&P.q, (size_t)qd * 4), "cudaMalloc q");
+    CKC(eng->alloc(&P.o, (size_t)qd * 4), "cudaMalloc o");
+    CKC(eng->alloc(&P.u, (size_t)F * 4), "cudaMalloc u");
+    CKC(eng->alloc(&P.part, (size_t)Hkv * P.splits * G * (D + 2) * 4), "cudaMalloc partials");
+    CKC(eng->alloc(&P.cnt, (size_t)Hkv * 4), "cudaMalloc counters");
+    CKC(eng->alloc(&P.cand_val, (size_t)nblk * 4), "cudaMalloc candidates");
+    CKC(eng->alloc(&P.cand_idx, (size_t)nblk * 4), "cudaMalloc candidates");
+    CKC(eng->alloc(&P.tokbuf, (size_t)c.max_ctx * 4), "cudaMalloc token buffer");
+    CKC(eng->alloc(&P.bar, 16), "cudaMalloc barrier");
+    CKC(eng->alloc(&P.err, 16), "cudaMalloc error word");
+    CKC(eng->alloc(&P.last_seq, 16), "cudaMalloc sequence");
+    CKC(eng->alloc(&P.cmd, sizeof(KieCmd)), "cudaMalloc command");
+    CKC(eng->alloc(&P.ssq, (size_t)nblk * 4), "cudaMalloc norm partials");
+    CKC(cudaMemset(P.ssq, 0, (size_t)nblk * 4), "memset");
+    CKC(cudaMemset(P.cnt, 0, (size_t)Hkv * 4), "memset");
+    CKC(cudaMemset(P.bar, 0, 16), "memset");
+    CKC(cudaMemset(P.err, 0, 16), "memset");
+    CKC(cudaMemset(P.last_seq, 0, 16), "memset");
+    CKC(cudaMemset(P.x, 0, (size_t)d * 4), "memset");
 
     // ---- the doorbell: mapped, pinned host memory
     eng->io_ints = 2 * (int64_t)c.max_ctx + 3 * 64 + 64 * 64;
     const size_t mb_bytes = sizeof(KieMailbox) + (size_t)eng->io_ints * 4;
-    CK(cudaHostAlloc((void **)&eng->mbox_host, mb_bytes, cudaHostAllocMapped | cudaHostAllocPortable), "cudaHostAlloc mailbox");
+    CKC(cudaHostAlloc((void **)&eng->mbox_host, mb_bytes, cudaHostAllocMapped | cudaHostAllocPortable), "cudaHostAlloc mailbox");
     memset(eng->mbox_host, 0, mb_bytes);
-    CK(cudaHostGetDevicePointer((void **)&eng->mbox_dev, eng->mbox_host, 0), "mailbox device alias");
+    CKC(cudaHostGetDevicePointer((void **)&eng->mbox_dev, eng->mbox_host, 0), "mailbox device alias");
     P.mbox = eng->mbox_dev;
 
-    CK(cudaStreamCreateWithFlags(&eng->stream, cudaStreamNonBlocking), "cudaStreamCreate");
-    CK(cudaEventCreateWithFlags(&eng->ev_done, cudaEventDisableTiming), "cudaEventCreate");
-    CK(cudaDeviceSynchronize(), "create");
+    CKC(cudaStreamCreateWithFlags(&eng->stream, cudaStreamNonBlocking), "cudaStreamCreate");
+    CKC(cudaEventCreateWithFlags(&eng->ev_done, cudaEventDisableTiming), "cudaEventCreate");
+    CKC(cudaDeviceSynchronize(), "create");
     eng->sess_len.assign(c.max_sessions, 0);
     eng->sess_used.assign(c.max_sessions, 0);
     (void)st;
     *out = eng;
     return KIE_OK;
 }
+#undef CKC
 
 // ---------------------------------------------------------------- resident kernel control
 

@@ -51,6 +51,8 @@ struct __align__(1024) MrShared {
     uint64_t acc_full[2], acc_empty[2], drain;
     uint64_t k_full[B_SLOTS], k_empty[B_SLOTS];  // the B ring as a K/V chunk ring in attention
     uint32_t k_iss;                              // K/V chunks issued so far (thread 0)
+    uint64_t at_k, at_v, at_s;                   // tensor-core attention: K tile, V tile, scores
+    uint32_t tk_iss, tv_iss, ts_iss;             // tiles issued (thread 0)
     uint32_t tmem_base;
     KieCmd cmd;
     volatile int abort;
@@ -74,7 +76,17 @@ KIE_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync
 KIE_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 KIE_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// D[tmem] (+)= A(desc) * B(desc)^T, M = N = 128, K = 16 (16-bit inputs, fp32 accumulate)
+// 2-D tiled bulk tensor copy (TMA, no multicast) of box (x, y) of the tensor map into shared
+// memory, completion as transaction bytes on `bar`
+KIE_DEV void tma_load_2d(void *dst, const void *tmap, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(dst)),
+        "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// D[tmem] (+)= A(desc) * B(desc)^T, M = 128, N from the instruction descriptor, K = 16 (16-bit inputs, fp32 accumulate)
 KIE_DEV void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
@@ -118,10 +130,10 @@ KIE_DEV uint64_t smem_desc_sw128(uint32_t saddr) {
     return d;
 }
 
-// Instruction descriptor: fp32 accumulate, A and B 16-bit (f16 or bf16), both K-major, M = N = 128.
-__host__ __device__ constexpr uint32_t idesc_f16(int dtype) {
+// Instruction descriptor: fp32 accumulate, A and B 16-bit (f16 or bf16), both K-major, M = 128, N = n.
+__host__ __device__ constexpr uint32_t idesc_f16(int dtype, uint32_t n = 128) {
     return (1u << 4) | ((uint32_t)(dtype == KIE_BF16) << 7) | ((uint32_t)(dtype == KIE_BF16) << 10) |
-           ((128u >> 3) << 17) | ((128u >> 4) << 24);
+           ((n >> 3) << 17) | ((128u >> 4) << 24);
 }
 
 // ------------------------------------------------------------------ shared helpers
@@ -559,10 +571,180 @@ __device__ void tick_attn_unit(const KieParams &P, MrShared &S, const AttnArgs &
     attn_tail<DT, GC, NW, true>(A, S.at, g, Gt, hoff, m, l, acc);
 }
 
+// One (row, kv head) unit on the tensor cores (head_dim a multiple of 64), 128 positions per
+// tile:
+//   scores  S[p][c] = K[p] . Qt[c]  by tcgen05.mma (M = 128 positions, N = 16, K = head_dim):
+//           columns c < 8 hold the 16-bit hi part of the scaled query heads, c >= 8 the lo part,
+//           so S[p][h] + S[p][8 + h] is the score of head h to ~16 bits of the fp32 query;
+//   K tile  2-D TMA copy of 128 cached rows x 64 dims per box, 128-byte swizzled (the MMA's
+//           K-major operand layout), from a tensor map over the whole K arena;
+//   softmax warps 0-3 read a position each from TMEM, keep the running max M and sum L per
+//           head (the same values in every thread) and write p = 2^(s - M) to shared memory;
+//   P V     all 8 warps on the CUDA cores from the V tile (1-D bulk copy), D/8 lanes per row.
+// The K buffer is refilled as soon as the MMA has read it, the V buffer once P V is done.
+template <int DT, int GC>
+__device__ void tick_attn_mma(const KieParams &P, MrShared &S, const AttnArgs &A, int g, int Gt, int hoff,
+                              long long row0, uint32_t &t_it) {
+    constexpr int NW = MR_WORKERS / 32;
+    const int nh = min(GC, Gt - hoff);
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int D = A.D, nks = D >> 6, lpp = D >> 3, ppw = 32 / lpp, sub = lane / lpp, sl = lane % lpp;
+    const int ngroups = NW * ppw, gi = w * ppw + sub;
+    const int ctx = A.ctx, ntile = (ctx + 127) >> 7;
+    uint8_t *Ks = S.b[0];  // [nks][128 rows][128 B], swizzled
+    uint8_t *Vs = S.b[2];  // [128][D] row-major
+    uint8_t *Qt = reinterpret_cast<uint8_t *>(S.at.wacc);                          // [nks][16][128 B], swizzled
+    float *Ps = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(S.at.wacc) + 4096);  // [128][4]
+    const uint8_t *vsrc = reinterpret_cast<const uint8_t *>(A.v + (size_t)g * A.head_stride);
+    const uint32_t idesc = idesc_f16(DT, 16);
+    auto load_k = [&](int t) {  // thread 0
+        mbar_arrive_expect_tx(&S.at_k, (uint32_t)nks * 16384u);
+        for (int ks = 0; ks < nks; ks++) tma_load_2d(Ks + ks * 16384, P.mr_kmap, ks * 64, (int)(row0 + t * 128), &S.at_k);
+        S.tk_iss++;
+    };
+    auto load_v = [&](int t) {  // thread 0
+        const uint32_t bytes = (uint32_t)(min(128, ctx - t * 128) * D * 2);
+        mbar_arrive_expect_tx(&S.at_v, bytes);
+        bulk_g2s(Vs, vsrc + (size_t)t * 128 * D * 2, bytes, &S.at_v);
+        S.tv_iss++;
+    };
+    if (tid == 0 && !S.abort) {
+        fence_proxy_async_global();  // the newest rows were written (generic proxy) before the barrier
+        load_k(0);
+        load_v(0);
+    }
+    // the query operand: rows h (hi) and 8 + h (lo) of the scaled query heads, other rows zero
+    const float qscale = rsqrtf((float)D) * 1.4426950408889634f;
+    for (int i = tid; i < 16 * (D >> 3); i += MR_WORKERS) {
+        const int row = i / (D >> 3), ch = i % (D >> 3), h = row & 7;
+        uint32_t pk[4] = {0u, 0u, 0u, 0u};
+        if (h < nh) {
+            const float *qp = A.q + (size_t)(g * Gt + hoff + h) * D + ch * 8;
+            const float4 a = __ldcg(reinterpret_cast<const float4 *>(qp));
+            const float4 b = __ldcg(reinterpret_cast<const float4 *>(qp + 4));
+            const float v[8] = {a.x * qscale, a.y * qscale, a.z * qscale, a.w * qscale,
+                                b.x * qscale, b.y * qscale, b.z * qscale, b.w * qscale};
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                uint16_t e0 = store1<DT>(v[2 * j]), e1 = store1<DT>(v[2 * j + 1]);
+                if (row >= 8) {
+                    e0 = store1<DT>(v[2 * j] - cvt1<DT>(e0));
+                    e1 = store1<DT>(v[2 * j + 1] - cvt1<DT>(e1));
+                }
+                pk[j] = (uint32_t)e0 | ((uint32_t)e1 << 16);
+            }
+        }
+        *reinterpret_cast<uint4 *>(Qt + (ch >> 3) * 2048 + sw128(row, ch & 7)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+    fence_proxy_async_smem();  // generic writes of the query tile -> tensor-core reads
+    named_bar_sync(1, MR_WORKERS);
+
+    float M[GC], L[GC], acc[GC][8];
+#pragma unroll
+    for (int h = 0; h < GC; h++) {
+        M[h] = -CUDART_INF_F;
+        L[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; e++) acc[h][e] = 0.f;
+    }
+    for (int t = 0; t < ntile; t++) {  // uniform control flow: every thread reaches every barrier
+        const uint32_t par = t_it & 1u;
+        const int p0 = t * 128, np = min(128, ctx - p0);
+        if (tid == 0 && !S.abort) {
+            if (mbar_wait(&S.at_k, par, P.timeout_ns, &S.abort)) {
+                tc_fence_after();
+                const uint32_t sk = smem_u32(Ks), sq = smem_u32(Qt);
+                for (int ks = 0; ks < nks; ks++)
+#pragma unroll
+                    for (int kk = 0; kk < 4; kk++)
+                        umma_f16(S.tmem_base, smem_desc_sw128(sk + ks * 16384 + kk * 32),
+                                 smem_desc_sw128(sq + ks * 2048 + kk * 32), idesc, (ks | kk) ? 1u : 0u);
+                umma_commit(&S.at_s);
+                S.ts_iss++;
+            } else {
+                if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x96);
+                S.abort = 1;
+            }
+        }
+        float sc[GC];
+        if (w < 4) {
+            const bool ok = __all_sync(0xffffffffu, !S.abort && mbar_wait(&S.at_s, par, P.timeout_ns, &S.abort));
+            const int pos = p0 + w * 32 + lane;
+            float v[32];
+            if (ok) {
+                tc_fence_after();
+                tmem_ld32(S.tmem_base + ((uint32_t)(w * 32) << 16), v);
+                tc_fence_before();
+            }
+#pragma unroll
+            for (int h = 0; h < GC; h++) sc[h] = (ok && pos < ctx && h < nh) ? v[h] + v[8 + h] : -CUDART_INF_F;
+#pragma unroll
+            for (int h = 0; h < GC; h++) {
+                const float mx = warp_max(sc[h]);
+                if (lane == 0) S.at.red[w * 8 + h] = mx;
+            }
+            if (tid == 0 && ok && t + 1 < ntile) load_k(t + 1);  // the MMA has read the K buffer
+        }
+        named_bar_sync(1, MR_WORKERS);
+        float corr[GC];
+#pragma unroll
+        for (int h = 0; h < GC; h++) {
+            const float mt = fmaxf(fmaxf(S.at.red[h], S.at.red[8 + h]), fmaxf(S.at.red[16 + h], S.at.red[24 + h]));
+            const float mn = fmaxf(M[h], mt);
+            corr[h] = rescale(M[h], mn);
+            M[h] = mn;
+        }
+        if (w < 4) {
+            float pv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int h = 0; h < GC; h++) pv[h] = rescale(sc[h], M[h]);
+            *reinterpret_cast<float4 *>(Ps + (w * 32 + lane) * 4) = make_float4(pv[0], pv[1], pv[2], pv[3]);
+#pragma unroll
+            for (int h = 0; h < GC; h++) {
+                const float sm = warp_sum(pv[h]);
+                if (lane == 0) S.at.red[32 + w * 8 + h] = sm;
+            }
+        }
+        named_bar_sync(1, MR_WORKERS);
+#pragma unroll
+        for (int h = 0; h < GC; h++) {
+            L[h] = L[h] * corr[h] + ((S.at.red[32 + h] + S.at.red[40 + h]) + (S.at.red[48 + h] + S.at.red[56 + h]));
+#pragma unroll
+            for (int e = 0; e < 8; e++) acc[h][e] *= corr[h];
+        }
+        if (!S.abort && mbar_wait(&S.at_v, par, P.timeout_ns, &S.abort)) {
+            for (int j = gi; j < np; j += ngroups) {
+                float f[8];
+                cvt8<DT>(*reinterpret_cast<const uint4 *>(Vs + (size_t)j * D * 2 + sl * 16), f);
+                const float4 pj = *reinterpret_cast<const float4 *>(Ps + j * 4);
+                const float pp[4] = {pj.x, pj.y, pj.z, pj.w};
+#pragma unroll
+                for (int h = 0; h < GC; h++)
+#pragma unroll
+                    for (int e = 0; e < 8; e++) acc[h][e] = fmaf(pp[h], f[e], acc[h][e]);
+            }
+        } else if (tid == 0 && !S.abort) {
+            set_error(P.err, DERR_RING_TIMEOUT, 0x97);
+            S.abort = 1;
+        }
+        named_bar_sync(1, MR_WORKERS);  // the V buffer and P are consumed
+        if (tid == 0 && !S.abort && t + 1 < ntile) {
+            fence_proxy_async_smem();  // generic reads of the V buffer before the bulk copy refills it
+            load_v(t + 1);
+        }
+        t_it++;
+    }
+    // hand the unit to the common tail: every thread holds the final M; L is counted once
+    float lsh[GC];
+#pragma unroll
+    for (int h = 0; h < GC; h++) lsh[h] = gi == 0 ? L[h] : 0.f;
+    attn_tail<DT, GC, NW, true>(A, S.at, g, Gt, hoff, M, lsh, acc);
+}
+
 // Attention of every row (a tick's sessions or a prefill chunk's positions): one unit per
 // (row, kv head), the unit's output written into the O projection's B operand.
 template <int DT>
-__device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M, uint32_t &k_it) {
+__device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M, uint32_t &k_it, uint32_t &t_it) {
     const int G = P.G;
     for (int u = blockIdx.x; u < M * P.Hkv; u += P.nblk) {
         const int m = u / P.Hkv, g = u % P.Hkv;
@@ -581,13 +763,13 @@ __device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M, uint32
         A.Hkv = P.Hkv;
         A.nsplit = 1;
         A.ctx = pos + 1;
-        switch (G) {
-            case 1: tick_attn_unit<DT, 1>(P, S, A, g, 1, 0, k_it); break;
-            case 2: tick_attn_unit<DT, 2>(P, S, A, g, 2, 0, k_it); break;
-            case 3: tick_attn_unit<DT, 3>(P, S, A, g, 3, 0, k_it); break;
-            default:
-                for (int hoff = 0; hoff < G; hoff += 4) tick_attn_unit<DT, 4>(P, S, A, g, G, hoff, k_it);
+        if (P.mr_kmap) {  // head_dim a multiple of 64: scores on the tensor cores
+            const long long row0 = (((long long)sid * P.L + l) * P.Hkv + g) * P.max_ctx;
+            // up to 4 query heads per pass (fewer heads leave rows of the query operand zero)
+            for (int hoff = 0; hoff < G; hoff += 4) tick_attn_mma<DT, 4>(P, S, A, g, G, hoff, row0, t_it);
+            continue;
         }
+        for (int hoff = 0; hoff < G; hoff += 4) tick_attn_unit<DT, 4>(P, S, A, g, G, hoff, k_it);
     }
 }
 
@@ -686,7 +868,7 @@ __device__ __forceinline__ void mr_mark(const KieParams &P, int st, int ev) {
 
 template <int DT>
 __device__ void mr_work(const KieParams &P, MrShared &S, uint32_t &b_it, uint32_t &u_it, uint32_t &k_it,
-                        const KieCmd &cmd, unsigned long long &epoch) {
+                        uint32_t &t_it, const KieCmd &cmd, unsigned long long &epoch) {
     const int M = cmd.n_sess;
     const int steps = steps_of(cmd);
     for (int st = 0; st < steps; st++) {
@@ -703,7 +885,7 @@ __device__ void mr_work(const KieParams &P, MrShared &S, uint32_t &b_it, uint32_
             if (!S.abort) phase_rope<DT>(P, l, M);
             mr_barrier(P, S, epoch, P.timeout_ns, 3);
             mr_mark(P, st, e + 4);
-            if (!S.abort) phase_attn<DT>(P, S, l, M, k_it);
+            if (!S.abort) phase_attn<DT>(P, S, l, M, k_it, t_it);
             mr_mark(P, st, e + 5);
             mr_barrier(P, S, epoch, P.timeout_ns, 4);
             mr_mark(P, st, e + 6);
@@ -766,6 +948,10 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
             mbar_init(&S.k_empty[i], MR_WORKERS / 32);
         }
         S.k_iss = 0;
+        mbar_init(&S.at_k, 1);
+        mbar_init(&S.at_v, 1);
+        mbar_init(&S.at_s, 1);
+        S.tk_iss = S.tv_iss = S.ts_iss = 0;
         fence_mbar_init();
         S.abort = 0;
     }
@@ -781,7 +967,7 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
     __syncthreads();
     tc_fence_after();
 
-    uint32_t a_it = 0, b_it = 0, u_it = 0, k_it = 0, drains = 0;
+    uint32_t a_it = 0, b_it = 0, u_it = 0, k_it = 0, t_it = 0, drains = 0;
     unsigned long long epoch = 0;
     for (;;) {
         if (tid < MR_WORKERS) {
@@ -838,7 +1024,7 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
             }
             drains++;
         } else {
-            mr_work<DT>(P, S, b_it, u_it, k_it, cmd, epoch);
+            mr_work<DT>(P, S, b_it, u_it, k_it, t_it, cmd, epoch);
             if (tid == 0) {  // copies still in flight (only after an abort) land before the CTA moves on
                 const uint32_t first = b_it > B_SLOTS ? b_it - B_SLOTS : 0;
                 for (uint32_t k = first; k < b_it; k++)
@@ -846,6 +1032,10 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
                 const uint32_t kfirst = S.k_iss > B_SLOTS ? S.k_iss - B_SLOTS : 0;
                 for (uint32_t k = kfirst; k < S.k_iss; k++)
                     mbar_wait(&S.k_full[k % B_SLOTS], (k / B_SLOTS) & 1u, P.timeout_ns, nullptr);
+                // the tensor-core attention's last K, V loads and score MMA (one of each in flight at most)
+                if (S.tk_iss) mbar_wait(&S.at_k, (S.tk_iss - 1) & 1u, P.timeout_ns, nullptr);
+                if (S.tv_iss) mbar_wait(&S.at_v, (S.tv_iss - 1) & 1u, P.timeout_ns, nullptr);
+                if (S.ts_iss) mbar_wait(&S.at_s, (S.ts_iss - 1) & 1u, P.timeout_ns, nullptr);
             }
         }
         __syncthreads();
