@@ -340,16 +340,23 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
         const int NGm = 5;
         const int Nm[NGm] = {qd + 2 * kvd, d, 2 * F, d, V};
         const int Km[NGm] = {d, qd, d, F, d};
+        // work unit ("atom"): the tiles of two consecutive 64-wide k-steps of a 128-row block (the
+        // odd last k-step of a block alone), moved by one bulk copy; atoms are split evenly over
+        // the SMs, phase by phase
+        auto natk = [&](int g) { return (Km[g] / 64 + 1) / 2; };
+        auto atom_tiles = [&](int g, long long a) { return std::min(2, Km[g] / 64 - 2 * (int)(a % natk(g))); };
         std::vector<int> a0((size_t)NGm * (nblk + 1));
         for (int g = 0; g < NGm; g++) {
-            const long long atoms = (long long)((Nm[g] + 127) / 128) * (Km[g] / 64);
+            const long long atoms = (long long)((Nm[g] + 127) / 128) * natk(g);
             for (int cc = 0; cc <= nblk; cc++) a0[(size_t)g * (nblk + 1) + cc] = (int)(cc * atoms / nblk);
         }
         std::vector<long long> mseg(nblk + 1, 0);
         for (int cc = 0; cc < nblk; cc++) {
             long long tiles = 0;
             for (int g = 0; g < NGm; g++) {
-                const long long n = a0[(size_t)g * (nblk + 1) + cc + 1] - a0[(size_t)g * (nblk + 1) + cc];
+                long long n = 0;
+                for (long long a = a0[(size_t)g * (nblk + 1) + cc]; a < a0[(size_t)g * (nblk + 1) + cc + 1]; a++)
+                    n += atom_tiles(g, a);
                 tiles += g < 4 ? n * L : n;
             }
             mseg[cc + 1] = mseg[cc] + tiles * 16384;
@@ -373,12 +380,13 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
                         case 3: src3[0] = Lw[8]; break;
                         default: src3[0] = w->lm_head; break;
                     }
-                    const int nks = Km[g] / 64;
-                    for (int a = a0[(size_t)g * (nblk + 1) + cc]; a < a0[(size_t)g * (nblk + 1) + cc + 1]; a++) {
-                        kie_mr_tile_src(&desc[nt * tsz], src3, n0, n1, off, Nm[g], Km[g], a / nks, a % nks);
-                        nt++;
-                        off += 16384;
-                    }
+                    for (int a = a0[(size_t)g * (nblk + 1) + cc]; a < a0[(size_t)g * (nblk + 1) + cc + 1]; a++)
+                        for (int t = 0; t < atom_tiles(g, a); t++) {
+                            kie_mr_tile_src(&desc[nt * tsz], src3, n0, n1, off, Nm[g], Km[g], a / natk(g),
+                                            2 * (a % natk(g)) + t);
+                            nt++;
+                            off += 16384;
+                        }
                 }
             }
         }

@@ -36,20 +36,25 @@ namespace {
 
 constexpr int MR_THREADS = 320;           // warps 0-3 (thread 0: B loads), 4-7 epilogue, 8 MMA, 9 producer
 constexpr int MR_WORKERS = 256;           // warps 0-7 also run the non-GEMM phases
-constexpr int A_SLOTS = 8, B_SLOTS = 4;
 constexpr int TILE = 16384;               // one 128 x 64 16-bit tile
+// A GEMM "atom" is the tiles of two consecutive 64-wide k-steps of one 128-row block (one when
+// it is the odd last k-step of the block), moved with one 32 KB bulk copy: on B200 a ring of
+// 4 x 32 KB copies streams ~7.3 TB/s where 8 x 16 KB copies stream ~5.8 TB/s.
+constexpr int ATOM = 2 * TILE;
+constexpr int A_SLOTS = 4, B_SLOTS = 2;   // atoms in flight: weights (HBM), activations (L2)
+constexpr int KV_SLOTS = 4;               // 16 KB K/V chunks of the CUDA-core attention, in the B ring
 constexpr int MAXR = 64;                  // rows per step (hi half of B; lo half at +64)
 constexpr int TMEM_COLS = 256;            // two 128-column fp32 accumulators
 
 enum { G_QKV = 0, G_O = 1, G_GU = 2, G_DOWN = 3, G_HEAD = 4, NG = 5 };
 
 struct __align__(1024) MrShared {
-    uint8_t a[A_SLOTS][TILE];
-    uint8_t b[B_SLOTS][TILE];
+    uint8_t a[A_SLOTS][ATOM];
+    uint8_t b[B_SLOTS][ATOM];
     AttnSmem at;
     uint64_t a_full[A_SLOTS], a_empty[A_SLOTS], b_full[B_SLOTS], b_empty[B_SLOTS];
     uint64_t acc_full[2], acc_empty[2], drain;
-    uint64_t k_full[B_SLOTS], k_empty[B_SLOTS];  // the B ring as a K/V chunk ring in attention
+    uint64_t k_full[KV_SLOTS], k_empty[KV_SLOTS];  // the B ring as a K/V chunk ring in attention
     uint32_t k_iss;                              // K/V chunks issued so far (thread 0)
     uint64_t at_k, at_v, at_s;                   // tensor-core attention: K tile, V tile, scores
     uint32_t tk_iss, tv_iss, ts_iss;             // tiles issued (thread 0)
@@ -155,6 +160,10 @@ __device__ __forceinline__ Gemm gemm_of(const KieParams &P, int g) {
     return G;
 }
 
+// atoms per row block of a K-long contraction, and the tiles (1 or 2) of atom a
+__device__ __forceinline__ int atoms_per_rb(int K) { return (K / 64 + 1) / 2; }
+__device__ __forceinline__ int atom_tiles(int K, int a) { return min(2, K / 64 - 2 * (a % atoms_per_rb(K))); }
+
 // words of a command record (volatile: it may live in mapped host memory)
 __device__ __forceinline__ void copy_cmd(KieCmd *dst, const KieCmd *src, bool vol) {
     uint32_t *d = reinterpret_cast<uint32_t *>(dst);
@@ -210,24 +219,24 @@ __device__ __forceinline__ int steps_of(const KieCmd &cmd) { return cmd.op == OP
 
 __device__ void mr_produce(const KieParams &P, MrShared &S, uint32_t &a_it, const KieCmd &cmd) {
     const uint8_t *seg = P.mr_wpack + P.mr_seg_off[blockIdx.x];
-    long long layer_bytes = 0;
-    for (int g = 0; g < G_HEAD; g++) layer_bytes += (long long)(S.a1[g] - S.a0[g]) * TILE;
     const int steps = steps_of(cmd);
     for (int st = 0; st < steps && !S.abort; st++) {
         const uint8_t *src = seg;
         for (int l = 0; l <= P.L && !S.abort; l++) {
             if (l == P.L && !head_needed(cmd)) break;
             for (int g = (l < P.L ? 0 : G_HEAD); g < (l < P.L ? G_HEAD : NG); g++) {
+                const int K = gemm_of(P, g).K;
                 for (int a = S.a0[g]; a < S.a1[g]; a++) {
                     const uint32_t slot = a_it % A_SLOTS, par = (a_it / A_SLOTS) & 1u;
+                    const uint32_t bytes = (uint32_t)atom_tiles(K, a) * TILE;
                     if (S.abort || !mbar_wait(&S.a_empty[slot], par ^ 1u, P.timeout_ns, &S.abort)) {
                         if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x90);
                         S.abort = 1;
                         break;
                     }
-                    mbar_arrive_expect_tx(&S.a_full[slot], TILE);
-                    bulk_g2s(S.a[slot], src, TILE, &S.a_full[slot]);
-                    src += TILE;
+                    mbar_arrive_expect_tx(&S.a_full[slot], bytes);
+                    bulk_g2s(S.a[slot], src, bytes, &S.a_full[slot]);
+                    src += bytes;
                     a_it++;
                 }
             }
@@ -249,11 +258,11 @@ __device__ void mr_mma(const KieParams &P, MrShared &S, uint32_t &a_it, uint32_t
         for (int l = 0; l <= P.L && ok; l++) {
             if (l == P.L && !head_needed(cmd)) break;
             for (int g = (l < P.L ? 0 : G_HEAD); g < (l < P.L ? G_HEAD : NG) && ok; g++) {
-                const int nks = gemm_of(P, g).K / 64;
+                const int K = gemm_of(P, g).K, natk = atoms_per_rb(K);
                 int cur_rb = -1;
                 uint32_t ab = 0;
                 for (int a = S.a0[g]; a < S.a1[g] && ok; a++) {
-                    const int rb = a / nks;
+                    const int rb = a / natk, nt = atom_tiles(K, a);
                     const bool first = (rb != cur_rb);
                     if (first) {  // new unit: take a free accumulator
                         cur_rb = rb;
@@ -273,15 +282,16 @@ __device__ void mr_mma(const KieParams &P, MrShared &S, uint32_t &a_it, uint32_t
                     tc_fence_after();
                     const uint32_t sa = smem_u32(S.a[as]), sb = smem_u32(S.b[bs]);
                     const uint32_t tmem_d = S.tmem_base + ab * 128u;
+                    for (int t = 0; t < nt; t++)
 #pragma unroll
-                    for (int kk = 0; kk < 4; kk++)
-                        umma_f16(tmem_d, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32), idesc,
-                                 (first && kk == 0) ? 0u : 1u);
+                        for (int kk = 0; kk < 4; kk++)
+                            umma_f16(tmem_d, smem_desc_sw128(sa + t * TILE + kk * 32), smem_desc_sw128(sb + t * TILE + kk * 32),
+                                     idesc, (first && t == 0 && kk == 0) ? 0u : 1u);
                     umma_commit(&S.a_empty[as]);
                     umma_commit(&S.b_empty[bs]);
                     a_it++;
                     b_it++;
-                    const bool last = (a + 1 == S.a1[g]) || ((a + 1) / nks != rb);
+                    const bool last = (a + 1 == S.a1[g]) || ((a + 1) / natk != rb);
                     if (last) {
                         umma_commit(&S.acc_full[ab]);
                         u_it++;
@@ -321,7 +331,7 @@ __device__ __forceinline__ void put_b8(uint8_t *tile, int m, int c, const float 
 // order, from the global operand buffer into the B ring (finished by the phase before, and
 // made visible by the grid barrier in between).
 __device__ void mr_bload(const KieParams &P, MrShared &S, uint32_t &b_it, int g) {
-    const int nks = gemm_of(P, g).K / 64;
+    const int K = gemm_of(P, g).K, natk = atoms_per_rb(K);
     fence_proxy_async_global();
     fence_proxy_async_smem();  // attention read the B ring through the generic proxy
     for (int a = S.a0[g]; a < S.a1[g]; a++) {
@@ -331,8 +341,9 @@ __device__ void mr_bload(const KieParams &P, MrShared &S, uint32_t &b_it, int g)
             S.abort = 1;
             return;
         }
-        mbar_arrive_expect_tx(&S.b_full[bs], TILE);
-        bulk_g2s(S.b[bs], P.mr_bpack + (size_t)(a % nks) * TILE, TILE, &S.b_full[bs]);
+        const uint32_t bytes = (uint32_t)atom_tiles(K, a) * TILE;
+        mbar_arrive_expect_tx(&S.b_full[bs], bytes);
+        bulk_g2s(S.b[bs], P.mr_bpack + (size_t)(2 * (a % natk)) * TILE, bytes, &S.b_full[bs]);
         b_it++;
     }
 }
@@ -341,11 +352,11 @@ __device__ void mr_bload(const KieParams &P, MrShared &S, uint32_t &b_it, int g)
 
 __device__ void mr_epilogue(const KieParams &P, MrShared &S, uint32_t &u_it, int g, int M) {
     const Gemm G = gemm_of(P, g);
-    const int nks = G.K / 64;
+    const int natk = atoms_per_rb(G.K);
     const int wq = (threadIdx.x >> 5) & 3, lane = threadIdx.x & 31;
     int cur_rb = -1;
     for (int a = S.a0[g]; a < S.a1[g]; a++) {
-        const int rb = a / nks;
+        const int rb = a / natk;
         if (rb == cur_rb) continue;
         cur_rb = rb;
         const uint32_t ab = u_it & 1u;
@@ -398,7 +409,12 @@ __device__ void phase_norm(const KieParams &P, MrShared &S, int g_next, int l, b
         float *x = P.mr_x + (size_t)m * P.d;
         float ss = 0.f;
         if (load_emb) {  // a new step starts from the embedding rows of its input tokens
-            const int tok = __ldcg(P.mr_tok + m);
+            int tok = __ldcg(P.mr_tok + m);
+            if (tok < 0 || tok >= P.V) {  // e.g. an argmax over non-finite logits: fail the command
+                if (tid == 0) set_error(P.err, DERR_BAD_TOKEN, 0x40);
+                S.abort = 1;
+                tok = 0;
+            }
             for (int c = tid; c < nch; c += MR_WORKERS) {
                 float v[8];
                 cvt8<DT>(__ldg(reinterpret_cast<const uint4 *>(P.emb + (size_t)tok * P.d + 8 * c)), v);
@@ -509,22 +525,23 @@ __device__ void tick_attn_unit(const KieParams &P, MrShared &S, const AttnArgs &
     const int ctx = A.ctx, nch = (ctx + CP - 1) / CP;
     const uint8_t *kb = reinterpret_cast<const uint8_t *>(A.k + (size_t)g * A.head_stride);
     const uint8_t *vb = reinterpret_cast<const uint8_t *>(A.v + (size_t)g * A.head_stride);
+    uint8_t *ring = S.b[0];    // KV_SLOTS chunk slots of TILE bytes over the B ring
     auto issue = [&](int c) {  // chunk c of this unit into its slot (thread 0)
-        const uint32_t it = k_it + c, slot = it % B_SLOTS;
-        if (S.abort || !mbar_wait(&S.k_empty[slot], ((it / B_SLOTS) & 1u) ^ 1u, P.timeout_ns, &S.abort)) {
+        const uint32_t it = k_it + c, slot = it % KV_SLOTS;
+        if (S.abort || !mbar_wait(&S.k_empty[slot], ((it / KV_SLOTS) & 1u) ^ 1u, P.timeout_ns, &S.abort)) {
             if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x94);
             S.abort = 1;
             return;
         }
         const uint32_t bytes = (uint32_t)(min(CP, ctx - c * CP) * rowb);
         mbar_arrive_expect_tx(&S.k_full[slot], 2 * bytes);
-        bulk_g2s(S.b[slot], kb + (size_t)c * CP * rowb, bytes, &S.k_full[slot]);
-        bulk_g2s(S.b[slot] + TILE / 2, vb + (size_t)c * CP * rowb, bytes, &S.k_full[slot]);
+        bulk_g2s(ring + slot * TILE, kb + (size_t)c * CP * rowb, bytes, &S.k_full[slot]);
+        bulk_g2s(ring + slot * TILE + TILE / 2, vb + (size_t)c * CP * rowb, bytes, &S.k_full[slot]);
         S.k_iss = it + 1;
     };
     if (tid == 0) {
         fence_proxy_async_global();  // the newest rows were written (generic proxy) before the barrier
-        for (int c = 0; c < min(B_SLOTS, nch); c++) issue(c);
+        for (int c = 0; c < min(KV_SLOTS, nch); c++) issue(c);
     }
     const float qscale = rsqrtf((float)D) * 1.4426950408889634f;
     float q[GC][8];
@@ -545,8 +562,8 @@ __device__ void tick_attn_unit(const KieParams &P, MrShared &S, const AttnArgs &
         for (int e = 0; e < 8; e++) acc[jj][e] = 0.f;
     }
     for (int c = 0; c < nch; c++) {
-        const uint32_t it = k_it + c, slot = it % B_SLOTS;
-        const bool ok = __all_sync(0xffffffffu, !S.abort && mbar_wait(&S.k_full[slot], (it / B_SLOTS) & 1u,
+        const uint32_t it = k_it + c, slot = it % KV_SLOTS;
+        const bool ok = __all_sync(0xffffffffu, !S.abort && mbar_wait(&S.k_full[slot], (it / KV_SLOTS) & 1u,
                                                                        P.timeout_ns, &S.abort));
         if (!ok) {
             if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x95);
@@ -558,14 +575,14 @@ __device__ void tick_attn_unit(const KieParams &P, MrShared &S, const AttnArgs &
         for (int b = 0; b < B; b++) {
             const int jl = gi + b * ngroups;
             const bool in = c * CP + jl < ctx;
-            kv[b] = in ? *reinterpret_cast<const uint4 *>(S.b[slot] + jl * rowb + sl * 16) : make_uint4(0, 0, 0, 0);
-            vv[b] = in ? *reinterpret_cast<const uint4 *>(S.b[slot] + TILE / 2 + jl * rowb + sl * 16)
+            kv[b] = in ? *reinterpret_cast<const uint4 *>(ring + slot * TILE + jl * rowb + sl * 16) : make_uint4(0, 0, 0, 0);
+            vv[b] = in ? *reinterpret_cast<const uint4 *>(ring + slot * TILE + TILE / 2 + jl * rowb + sl * 16)
                        : make_uint4(0, 0, 0, 0);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.k_empty[slot]);  // this warp's reads of the slot are done
         attn_update<DT, GC, B>(kv, vv, c * CP, ctx, gi, ngroups, lpp, q, m, l, acc);
-        if (tid == 0 && c + B_SLOTS < nch) issue(c + B_SLOTS);
+        if (tid == 0 && c + KV_SLOTS < nch) issue(c + KV_SLOTS);
     }
     k_it += nch;
     attn_tail<DT, GC, NW, true>(A, S.at, g, Gt, hoff, m, l, acc);
@@ -591,8 +608,8 @@ __device__ void tick_attn_mma(const KieParams &P, MrShared &S, const AttnArgs &A
     const int D = A.D, nks = D >> 6, lpp = D >> 3, ppw = 32 / lpp, sub = lane / lpp, sl = lane % lpp;
     const int ngroups = NW * ppw, gi = w * ppw + sub;
     const int ctx = A.ctx, ntile = (ctx + 127) >> 7;
-    uint8_t *Ks = S.b[0];  // [nks][128 rows][128 B], swizzled
-    uint8_t *Vs = S.b[2];  // [128][D] row-major
+    uint8_t *Ks = S.b[0];  // [nks][128 rows][128 B], swizzled (32 KB)
+    uint8_t *Vs = S.b[1];  // [128][D] row-major (32 KB)
     uint8_t *Qt = reinterpret_cast<uint8_t *>(S.at.wacc);                          // [nks][16][128 B], swizzled
     float *Ps = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(S.at.wacc) + 4096);  // [128][4]
     const uint8_t *vsrc = reinterpret_cast<const uint8_t *>(A.v + (size_t)g * A.head_stride);
@@ -943,7 +960,7 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
             mbar_init(&S.acc_empty[i], 4);
         }
         mbar_init(&S.drain, 1);
-        for (int i = 0; i < B_SLOTS; i++) {
+        for (int i = 0; i < KV_SLOTS; i++) {
             mbar_init(&S.k_full[i], 1);
             mbar_init(&S.k_empty[i], MR_WORKERS / 32);
         }
@@ -1029,9 +1046,9 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
                 const uint32_t first = b_it > B_SLOTS ? b_it - B_SLOTS : 0;
                 for (uint32_t k = first; k < b_it; k++)
                     mbar_wait(&S.b_full[k % B_SLOTS], (k / B_SLOTS) & 1u, P.timeout_ns, nullptr);
-                const uint32_t kfirst = S.k_iss > B_SLOTS ? S.k_iss - B_SLOTS : 0;
+                const uint32_t kfirst = S.k_iss > KV_SLOTS ? S.k_iss - KV_SLOTS : 0;
                 for (uint32_t k = kfirst; k < S.k_iss; k++)
-                    mbar_wait(&S.k_full[k % B_SLOTS], (k / B_SLOTS) & 1u, P.timeout_ns, nullptr);
+                    mbar_wait(&S.k_full[k % KV_SLOTS], (k / KV_SLOTS) & 1u, P.timeout_ns, nullptr);
                 // the tensor-core attention's last K, V loads and score MMA (one of each in flight at most)
                 if (S.tk_iss) mbar_wait(&S.at_k, (S.tk_iss - 1) & 1u, P.timeout_ns, nullptr);
                 if (S.tv_iss) mbar_wait(&S.at_v, (S.tv_iss - 1) & 1u, P.timeout_ns, nullptr);

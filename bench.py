@@ -314,15 +314,17 @@ def main():
             tr = json.load(f)
         if headline and tr.get("kernel_rev") == kernel_revision():
             traffic = tr.get("bytes_per_launch")
+    dtype_name = "bf16" if m.dtype == 1 else "fp16"
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype_name, "data": "synthetic",
         "config": {"workload": WORKLOAD if headline else f"{m.name} batch-1: prompt {prompt_len}, decode {decode_n}",
                    "prompt": prompt_len, "decode": decode_n, "batch": 1,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "inputs larger than L2 (3.65 GB of weights streamed per token); no flush needed",
-                   "weights": "seeded N(0,0.02) fp16, norms 1"},
+                   "l2": f"inputs larger than L2 ({m.weight_bytes_per_token() / 1e9:.2f} GB of weights streamed per token);"
+                         " no flush needed",
+                   "weights": f"seeded N(0,0.02) {dtype_name}, norms 1"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": peak_kind,
                      "bytes_per_launch": bytes_launch, "kernel": f"kie_b1_kernel (one launch = {decode_n} tokens)"},
