@@ -61,6 +61,7 @@ extern "C" kie_status kie_flash_decode(const float *q_dev, const void *k_dev, co
     A.o = out_dev;
     A.bpack = nullptr;
     A.brow = 0;
+    A.gout = -1;
     A.D = head_dim;
     A.Hkv = n_kv_heads;
     A.nsplit = fd_splits(G, n_ctx);

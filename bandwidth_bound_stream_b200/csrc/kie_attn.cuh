@@ -33,6 +33,7 @@ struct AttnArgs {
                              // (hi) and 64 + brow (lo) of the swizzled 128 x 64 tiles of the
                              // tick kernel's B operand (column h * D + e)
     int brow;
+    int gout;                // kv head whose output columns a unit writes; -1: unit / nsplit
     int D, Hkv, nsplit, ctx;
 };
 
@@ -205,6 +206,7 @@ __device__ __forceinline__ void attn_tail(const AttnArgs &A, AttnSmem &S, int un
     const int D = A.D, lpp = D >> 3, sub = lane / lpp, sl = lane % lpp;
     const int nsplit = A.nsplit;
     const int g = unit / nsplit;
+    const int go = A.gout >= 0 ? A.gout : g;  // the kv head of the output columns
     // merge the position groups of each warp (lanes with the same sl hold the same dims)
 #pragma unroll
     for (int jj = 0; jj < G; jj++) {
@@ -256,7 +258,7 @@ __device__ __forceinline__ void attn_tail(const AttnArgs &A, AttnSmem &S, int un
             const float den = ((S.wl[0][jj] + S.wl[1][jj]) + S.wl[2][jj]) + S.wl[3][jj];
             const float n0 = ((S.wacc[0][k] + S.wacc[1][k]) + S.wacc[2][k]) + S.wacc[3][k];
             const float n1 = ((S.wacc[0][k + 1] + S.wacc[1][k + 1]) + S.wacc[2][k + 1]) + S.wacc[3][k + 1];
-            attn_out2<DT>(A, (g * Gt + hoff + jj) * D + e, n0 / den, n1 / den);
+            attn_out2<DT>(A, (go * Gt + hoff + jj) * D + e, n0 / den, n1 / den);
         }
         named_bar_sync(1, ATTN_THREADS);
         return;
@@ -346,7 +348,7 @@ __device__ __forceinline__ void attn_tail(const AttnArgs &A, AttnSmem &S, int un
             }
             if (pr < npairs && sub == 0) {
                 const float den = S.red[jj];
-                attn_out2<DT>(A, (g * Gt + jj) * D + e, num.x / den, num.y / den);
+                attn_out2<DT>(A, (go * Gt + jj) * D + e, num.x / den, num.y / den);
             }
         }
         if (tid == 0) A.cnt[g] = 0u;

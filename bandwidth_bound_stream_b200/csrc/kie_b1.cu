@@ -560,6 +560,7 @@ __device__ void attention_step(const KieParams &P, B1Shared &S, int l, int sid, 
     A.o = P.o;
     A.bpack = nullptr;
     A.brow = 0;
+    A.gout = -1;
     A.D = P.D;
     A.Hkv = P.Hkv;
     A.nsplit = P.splits;

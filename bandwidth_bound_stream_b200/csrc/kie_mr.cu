@@ -776,6 +776,7 @@ __device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M, uint32
         A.o = nullptr;
         A.bpack = P.mr_bpack;  // the output is the O projection's B operand, row m
         A.brow = m;
+        A.gout = g;
         A.D = P.D;
         A.Hkv = P.Hkv;
         A.nsplit = 1;

@@ -89,8 +89,10 @@ SLICE_1P9B = dataclasses.replace(DENSE_1P9B, name="slice-1.9b", n_layers=2)
 SLICE_8B = dataclasses.replace(DENSE_8B, name="slice-8b", n_layers=2)
 SLICE_TICK = dataclasses.replace(TICK_10P8B, name="slice-10.8b", n_layers=2)
 RAGGED = ModelConfig("ragged", 3, 384, 6, 2, 64, 1216, 5003, BF16, rope_theta=1e4)
+# head_dim 32, 5 query heads per kv head, odd k-step counts (d = 320, F = 576), odd vocabulary
+SMALL_HEAD = ModelConfig("small-head", 2, 320, 10, 2, 32, 576, 3001, FP16, rope_theta=1e4)
 CONFIGS = {c.name: c for c in (TINY, DENSE_1P9B, DENSE_8B, TICK_10P8B, SLICE_1P9B, SLICE_8B,
-                                SLICE_TICK, RAGGED)}
+                                SLICE_TICK, RAGGED, SMALL_HEAD)}
 
 
 def _lib():

@@ -93,6 +93,14 @@ def test_tick_ragged_parity(kie):
     _run_tick_parity(kie, synth.RAGGED, 7, [5, 12, 64, 65, 3, 30, 20], checked=[0, 3, 6], ticks=2, max_ctx=96)
 
 
+def test_tick_small_head_parity(kie):
+    """head_dim 32 (the CUDA-core attention path, contexts spanning several K/V chunks), 5 query
+    heads per kv head (two passes), odd k-step counts (single-tile atoms), fp16, odd vocabulary."""
+    from bandwidth_bound_stream_b200 import synth
+    _run_tick_parity(kie, synth.SMALL_HEAD, 6, [5, 40, 100, 129, 7, 250], checked=[0, 2, 3, 5], ticks=2,
+                     max_ctx=280)
+
+
 def test_tick_slice_10p8b_56_sessions(kie):
     """Two layers of the 10.8B tick shape at full width (bf16, GQA 4), 56 sessions; 5 sampled
     sessions are checked against the oracle."""
