@@ -137,6 +137,23 @@ def dist_setup():
     return rank, world, local
 
 
+def max_over_ranks(x: float, world: int, device="cpu") -> float:
+    """The largest of every rank's x (each rank passes its own time; all ranks get the max).
+    `device` is where the reduction runs: the rank's GPU under NCCL, the CPU under gloo."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, max_seconds: float) -> float:
+    """Throughput of the whole job: the units all ranks processed over the slowest rank's time."""
+    return world * units_per_rank / max_seconds
+
+
 def run_reference(args, rank):
     """The CPU oracle on this workload: each step is a bounded sample, one greedy decode token of the
     full 1.9B model at the workload's mean context length, timed on the host cores."""
@@ -267,11 +284,7 @@ def main():
     total_ms = t_all0.elapsed_time(t_all1)
     per_launch = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     assert np.array_equal(out_d.cpu().numpy(), ref_tokens), "decode is not deterministic across launches"
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
 
     # end to end through the doorbell with host buffers
     out_h = np.empty(decode_n, dtype=np.int32)
@@ -285,11 +298,7 @@ def main():
         eng.generate(sid, first, decode_n, out_h)
     e_s = time.perf_counter() - e0
     assert np.array_equal(out_h, ref_tokens), "doorbell and launch paths disagree"
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([e_s], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_s = float(t.item())
+    e_s = max_over_ranks(e_s, world, dev)
 
     # inter-token latency of single doorbell steps (host clock)
     eng.session_rewind(sid, prompt_len)
@@ -301,8 +310,7 @@ def main():
         itl.append((time.perf_counter() - a) * 1e3)
     eng.close()
 
-    tokens = world * decode_n * args.steps
-    value = tokens / (total_ms / 1e3)
+    value = whole_job_rate(decode_n * args.steps, world, total_ms / 1e3)
     peak, peak_kind = measured_peaks()
     bytes_launch = algorithmic_bytes(m, prompt_len, decode_n)
     mean_launch_s = statistics.mean(per_launch) / 1e3

@@ -8,8 +8,8 @@
  *  - Every weight byte and the KV cache are streamed once per generated token; decode is
  *    bound by memory bandwidth, not compute ("Kog 3000 tok/s 实时推理：内存带宽优化与请求级并发的
  *    工程权衡", section 内存带宽优化的三层策略; the HN digest of Kog's inference engine,
- *    section 技术原理, "内存带宽是关键瓶颈").
- *  - One resident kernel replaces per-op launches (the same digest, 技术原理, 持久化单内核运行时;
+ *    section 技术原理).
+ *  - One resident kernel replaces per-op launches (the same digest, section 技术原理;
  *    "实时AI推理为何贵56倍？持续推理与常驻内核的破局之道", section 让工作常驻 GPU). The host only
  *    writes input tokens into a mapped mailbox (the doorbell) and reads output tokens.
  *  - Sessions due on the same tick advance as one batch, so the weights are read once for
