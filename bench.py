@@ -155,14 +155,17 @@ def whole_job_rate(units_per_rank: float, world: int, max_seconds: float) -> flo
 
 
 def run_reference(args, rank):
-    """The CPU oracle on this workload: each step is a bounded sample, one greedy decode token of the
-    full 1.9B model at the workload's mean context length, timed on the host cores."""
+    """The CPU oracle on this arm's workload (the same --model / --prompt / --decode as the engine
+    arm): each step is a bounded sample, one greedy decode token of the full model at the
+    workload's mean context length, timed on the host cores."""
     if rank != 0:
         return
     from bandwidth_bound_stream_b200 import synth
     from oracle.oracle import OracleModel, num_threads
-    m = synth.DENSE_1P9B
-    ctx0 = PROMPT + DECODE // 2
+    m = synth.CONFIGS[args.model]
+    prompt_len, decode_n = args.prompt, args.decode
+    headline = (args.model == "dense-1.9b" and prompt_len == PROMPT and decode_n == DECODE)
+    ctx0 = prompt_len + decode_n // 2
     orc = OracleModel(m, synth.model_weights(m), ctx0 + args.warmup + args.steps + 1)
     orc.pos = ctx0
     tok = 1
@@ -173,14 +176,14 @@ def run_reference(args, rank):
         tok = int(np.argmax(orc.step(tok)))
     el = time.perf_counter() - t0
     value = args.steps / el
-    sample = (f"{args.steps} timed oracle decode steps (after {args.warmup} warm-up) of the full 1.9B model at "
+    sample = (f"{args.steps} timed oracle decode steps (after {args.warmup} warm-up) of the full {m.name} model at "
               f"positions {ctx0 + args.warmup}.. (KV cache of that length, zero contents)")
     cb = {"value": value, "unit": "tokens/s", "cores": num_threads(), "kind": "oracle", "sample": sample}
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD if headline else f"{m.name} batch-1: prompt {prompt_len}, decode {decode_n}",
-                   "prompt": prompt_len, "decode": decode_n, "batch": 1,
+                       "prompt": prompt_len, "decode": decode_n, "batch": 1,
                        "parallelism": "CPU oracle, OpenMP over output rows",
                        "step": "one decode token of the workload per step (bounded sample)"},
             "cpu_baseline": cb,
