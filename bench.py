@@ -216,6 +216,9 @@ def main():
         if rank == 0:
             print(json.dumps({"metric": "p99 tick latency at 56 sessions", "value": t["p99_ms"], "unit": "ms",
                               "higher_is_better": False, "n_gpus": world, "tick": t}), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
         return
     if args.impl == "reference":
         run_reference(args, rank)
