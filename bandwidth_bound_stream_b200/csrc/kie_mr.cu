@@ -56,8 +56,9 @@ struct __align__(1024) MrShared {
     uint64_t acc_full[2], acc_empty[2], drain;
     uint64_t k_full[KV_SLOTS], k_empty[KV_SLOTS];  // the B ring as a K/V chunk ring in attention
     uint32_t k_iss;                              // K/V chunks issued so far (thread 0)
-    uint64_t at_k, at_v, at_s;                   // tensor-core attention: K tile, V tile, scores
-    uint32_t tk_iss, tv_iss, ts_iss;             // tiles issued (thread 0)
+    uint64_t at_k[2], at_v[2], at_s;             // tensor-core attention: K, V tiles per stage; scores
+    uint32_t tk_iss[2], tv_iss[2], ts_iss;       // copies / MMA groups issued (thread 0)
+    volatile uint32_t att_seq;                   // attention phases finished (the producer waits on it)
     uint32_t tmem_base;
     KieCmd cmd;
     volatile int abort;
@@ -217,7 +218,7 @@ __device__ __forceinline__ int steps_of(const KieCmd &cmd) { return cmd.op == OP
 
 // ------------------------------------------------------------------ producer (warp 9)
 
-__device__ void mr_produce(const KieParams &P, MrShared &S, uint32_t &a_it, const KieCmd &cmd) {
+__device__ void mr_produce(const KieParams &P, MrShared &S, uint32_t &a_it, uint32_t &o_seq, const KieCmd &cmd) {
     const uint8_t *seg = P.mr_wpack + P.mr_seg_off[blockIdx.x];
     const int steps = steps_of(cmd);
     for (int st = 0; st < steps && !S.abort; st++) {
@@ -226,6 +227,18 @@ __device__ void mr_produce(const KieParams &P, MrShared &S, uint32_t &a_it, cons
             if (l == P.L && !head_needed(cmd)) break;
             for (int g = (l < P.L ? 0 : G_HEAD); g < (l < P.L ? G_HEAD : NG); g++) {
                 const int K = gemm_of(P, g).K;
+                if (g == G_O) {  // attention uses the ring as its K/V buffers: wait until it is done
+                    const uint64_t t0 = globaltimer();
+                    while (S.att_seq <= o_seq && !S.abort) {
+                        if ((long long)(globaltimer() - t0) > P.timeout_ns) {
+                            set_error(P.err, DERR_RING_TIMEOUT, 0x98);
+                            S.abort = 1;
+                        }
+                        __nanosleep(64);
+                    }
+                    o_seq++;
+                    fence_proxy_async_smem();  // attention's generic reads of the ring, then these copies
+                }
                 for (int a = S.a0[g]; a < S.a1[g]; a++) {
                     const uint32_t slot = a_it % A_SLOTS, par = (a_it / A_SLOTS) & 1u;
                     const uint32_t bytes = (uint32_t)atom_tiles(K, a) * TILE;
@@ -598,7 +611,10 @@ __device__ void tick_attn_unit(const KieParams &P, MrShared &S, const AttnArgs &
 //   softmax warps 0-3 read a position each from TMEM, keep the running max M and sum L per
 //           head (the same values in every thread) and write p = 2^(s - M) to shared memory;
 //   P V     all 8 warps on the CUDA cores from the V tile (1-D bulk copy), D/8 lanes per row.
-// The K buffer is refilled as soon as the MMA has read it, the V buffer once P V is done.
+// K and V tiles are double-buffered in the weight ring (4 x 32 KB), which the producer leaves
+// to attention (it holds the O projection's weights back until attention is done): the
+// copies of tile t + 2 are issued as soon as tile t is consumed, so a tile's loads overlap
+// the work on the tile before it.
 template <int DT, int GC>
 __device__ void tick_attn_mma(const KieParams &P, MrShared &S, const AttnArgs &A, int g, int Gt, int hoff,
                               long long row0, uint32_t &t_it) {
@@ -608,27 +624,28 @@ __device__ void tick_attn_mma(const KieParams &P, MrShared &S, const AttnArgs &A
     const int D = A.D, nks = D >> 6, lpp = D >> 3, ppw = 32 / lpp, sub = lane / lpp, sl = lane % lpp;
     const int ngroups = NW * ppw, gi = w * ppw + sub;
     const int ctx = A.ctx, ntile = (ctx + 127) >> 7;
-    uint8_t *Ks = S.b[0];  // [nks][128 rows][128 B], swizzled (32 KB)
-    uint8_t *Vs = S.b[1];  // [128][D] row-major (32 KB)
+    // stage s: K in a[2s] ([nks][128 rows][128 B], swizzled), V in a[2s + 1] ([128][D] row-major)
     uint8_t *Qt = reinterpret_cast<uint8_t *>(S.at.wacc);                          // [nks][16][128 B], swizzled
     float *Ps = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(S.at.wacc) + 4096);  // [128][4]
     const uint8_t *vsrc = reinterpret_cast<const uint8_t *>(A.v + (size_t)g * A.head_stride);
     const uint32_t idesc = idesc_f16(DT, 16);
-    auto load_k = [&](int t) {  // thread 0
-        mbar_arrive_expect_tx(&S.at_k, (uint32_t)nks * 16384u);
-        for (int ks = 0; ks < nks; ks++) tma_load_2d(Ks + ks * 16384, P.mr_kmap, ks * 64, (int)(row0 + t * 128), &S.at_k);
-        S.tk_iss++;
-    };
-    auto load_v = [&](int t) {  // thread 0
+    const uint32_t q0 = t_it;  // global index of this unit's first tile (stage = index & 1)
+    auto load_tile = [&](int t) {  // thread 0: K and V of tile t into its stage
+        const int st = (int)((q0 + t) & 1u);
+        mbar_arrive_expect_tx(&S.at_k[st], (uint32_t)nks * 16384u);
+        for (int ks = 0; ks < nks; ks++)
+            tma_load_2d(S.a[2 * st] + ks * 16384, P.mr_kmap, ks * 64, (int)(row0 + t * 128), &S.at_k[st]);
+        S.tk_iss[st]++;
         const uint32_t bytes = (uint32_t)(min(128, ctx - t * 128) * D * 2);
-        mbar_arrive_expect_tx(&S.at_v, bytes);
-        bulk_g2s(Vs, vsrc + (size_t)t * 128 * D * 2, bytes, &S.at_v);
-        S.tv_iss++;
+        mbar_arrive_expect_tx(&S.at_v[st], bytes);
+        bulk_g2s(S.a[2 * st + 1], vsrc + (size_t)t * 128 * D * 2, bytes, &S.at_v[st]);
+        S.tv_iss[st]++;
     };
     if (tid == 0 && !S.abort) {
         fence_proxy_async_global();  // the newest rows were written (generic proxy) before the barrier
-        load_k(0);
-        load_v(0);
+        fence_proxy_async_smem();    // earlier generic reads of the ring before the copies refill it
+        load_tile(0);
+        if (ntile > 1) load_tile(1);
     }
     // the query operand: rows h (hi) and 8 + h (lo) of the scaled query heads, other rows zero
     const float qscale = rsqrtf((float)D) * 1.4426950408889634f;
@@ -665,12 +682,15 @@ __device__ void tick_attn_mma(const KieParams &P, MrShared &S, const AttnArgs &A
         for (int e = 0; e < 8; e++) acc[h][e] = 0.f;
     }
     for (int t = 0; t < ntile; t++) {  // uniform control flow: every thread reaches every barrier
-        const uint32_t par = t_it & 1u;
+        const uint32_t par = t_it & 1u;                 // the scores barrier completes once per tile
+        const int st = (int)(t_it & 1u);                // this tile's stage
+        const uint32_t spar = (t_it >> 1) & 1u;         // ... whose barriers complete every other tile
+        const uint8_t *Vs = S.a[2 * st + 1];
         const int p0 = t * 128, np = min(128, ctx - p0);
         if (tid == 0 && !S.abort) {
-            if (mbar_wait(&S.at_k, par, P.timeout_ns, &S.abort)) {
+            if (mbar_wait(&S.at_k[st], spar, P.timeout_ns, &S.abort)) {
                 tc_fence_after();
-                const uint32_t sk = smem_u32(Ks), sq = smem_u32(Qt);
+                const uint32_t sk = smem_u32(S.a[2 * st]), sq = smem_u32(Qt);
                 for (int ks = 0; ks < nks; ks++)
 #pragma unroll
                     for (int kk = 0; kk < 4; kk++)
@@ -700,7 +720,6 @@ __device__ void tick_attn_mma(const KieParams &P, MrShared &S, const AttnArgs &A
                 const float mx = warp_max(sc[h]);
                 if (lane == 0) S.at.red[w * 8 + h] = mx;
             }
-            if (tid == 0 && ok && t + 1 < ntile) load_k(t + 1);  // the MMA has read the K buffer
         }
         named_bar_sync(1, MR_WORKERS);
         float corr[GC];
@@ -729,7 +748,7 @@ __device__ void tick_attn_mma(const KieParams &P, MrShared &S, const AttnArgs &A
 #pragma unroll
             for (int e = 0; e < 8; e++) acc[h][e] *= corr[h];
         }
-        if (!S.abort && mbar_wait(&S.at_v, par, P.timeout_ns, &S.abort)) {
+        if (!S.abort && mbar_wait(&S.at_v[st], spar, P.timeout_ns, &S.abort)) {
             for (int j = gi; j < np; j += ngroups) {
                 float f[8];
                 cvt8<DT>(*reinterpret_cast<const uint4 *>(Vs + (size_t)j * D * 2 + sl * 16), f);
@@ -744,10 +763,10 @@ __device__ void tick_attn_mma(const KieParams &P, MrShared &S, const AttnArgs &A
             set_error(P.err, DERR_RING_TIMEOUT, 0x97);
             S.abort = 1;
         }
-        named_bar_sync(1, MR_WORKERS);  // the V buffer and P are consumed
-        if (tid == 0 && !S.abort && t + 1 < ntile) {
+        named_bar_sync(1, MR_WORKERS);  // this stage's K (the MMA is done) and V, and P, are consumed
+        if (tid == 0 && !S.abort && t + 2 < ntile) {
             fence_proxy_async_smem();  // generic reads of the V buffer before the bulk copy refills it
-            load_v(t + 1);
+            load_tile(t + 2);
         }
         t_it++;
     }
@@ -904,6 +923,11 @@ __device__ void mr_work(const KieParams &P, MrShared &S, uint32_t &b_it, uint32_
             mr_barrier(P, S, epoch, P.timeout_ns, 3);
             mr_mark(P, st, e + 4);
             if (!S.abort) phase_attn<DT>(P, S, l, M, k_it, t_it);
+            named_bar_sync(1, MR_WORKERS);  // every worker is done with the ring
+            if (threadIdx.x == 0) {
+                __threadfence_block();
+                S.att_seq = S.att_seq + 1;  // the producer may now fill the ring with the O weights
+            }
             mr_mark(P, st, e + 5);
             mr_barrier(P, S, epoch, P.timeout_ns, 4);
             mr_mark(P, st, e + 6);
@@ -966,10 +990,14 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
             mbar_init(&S.k_empty[i], MR_WORKERS / 32);
         }
         S.k_iss = 0;
-        mbar_init(&S.at_k, 1);
-        mbar_init(&S.at_v, 1);
+        for (int i = 0; i < 2; i++) {
+            mbar_init(&S.at_k[i], 1);
+            mbar_init(&S.at_v[i], 1);
+            S.tk_iss[i] = S.tv_iss[i] = 0;
+        }
         mbar_init(&S.at_s, 1);
-        S.tk_iss = S.tv_iss = S.ts_iss = 0;
+        S.ts_iss = 0;
+        S.att_seq = 0;
         fence_mbar_init();
         S.abort = 0;
     }
@@ -985,7 +1013,7 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
     __syncthreads();
     tc_fence_after();
 
-    uint32_t a_it = 0, b_it = 0, u_it = 0, k_it = 0, t_it = 0, drains = 0;
+    uint32_t a_it = 0, b_it = 0, u_it = 0, k_it = 0, t_it = 0, o_seq = 0, drains = 0;
     unsigned long long epoch = 0;
     for (;;) {
         if (tid < MR_WORKERS) {
@@ -1034,7 +1062,7 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
         const KieCmd cmd = S.cmd;
         if (cmd.op != OP_TICK && cmd.op != OP_PREFILL) break;
         if (warp == 9) {
-            if ((tid & 31) == 0) mr_produce(P, S, a_it, cmd);
+            if ((tid & 31) == 0) mr_produce(P, S, a_it, o_seq, cmd);
         } else if (warp == 8) {
             if ((tid & 31) == 0) {
                 mr_mma(P, S, a_it, b_it, u_it, cmd);
@@ -1051,8 +1079,10 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
                 for (uint32_t k = kfirst; k < S.k_iss; k++)
                     mbar_wait(&S.k_full[k % KV_SLOTS], (k / KV_SLOTS) & 1u, P.timeout_ns, nullptr);
                 // the tensor-core attention's last K, V loads and score MMA (one of each in flight at most)
-                if (S.tk_iss) mbar_wait(&S.at_k, (S.tk_iss - 1) & 1u, P.timeout_ns, nullptr);
-                if (S.tv_iss) mbar_wait(&S.at_v, (S.tv_iss - 1) & 1u, P.timeout_ns, nullptr);
+                for (int i = 0; i < 2; i++) {  // per stage: its k-th copy completes phase k - 1
+                    if (S.tk_iss[i]) mbar_wait(&S.at_k[i], (S.tk_iss[i] - 1) & 1u, P.timeout_ns, nullptr);
+                    if (S.tv_iss[i]) mbar_wait(&S.at_v[i], (S.tv_iss[i] - 1) & 1u, P.timeout_ns, nullptr);
+                }
                 if (S.ts_iss) mbar_wait(&S.at_s, (S.ts_iss - 1) & 1u, P.timeout_ns, nullptr);
             }
         }
