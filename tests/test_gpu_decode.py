@@ -154,47 +154,67 @@ def test_full_1p9b_parity_short_context(kie):
     assert_reports(reps, m.dtype)
 
 
-def test_full_1p9b_bench_launch_layer0_cache(kie):
-    """The benchmark's configuration (1.9B, prompt 1024, one launch of 512 steps): layer-0 K/V at sampled
-    positions equal the oracle's projection of that position's token (they depend on it alone)."""
+def _bench_launch_layer0_check(kie, m, prompt_len, decode_n, positions, modes):
+    """One launch of the bench's configuration; layer-0 K/V at sampled positions must equal the
+    oracle's projection of that position's token (they depend on that token alone)."""
     from bandwidth_bound_stream_b200 import synth
     from oracle import oracle as orc
-    m = synth.DENSE_1P9B
+    max_ctx = prompt_len + decode_n
     dw = kie.DeviceWeights(m, host_copy=True)
-    prompt = synth.prompt(m, 1024)
-    with kie.Engine(kie.config(m, max_ctx=1536, timeout_ms=5000, idle_ms=50), dw.kie) as eng:
+    prompt = synth.prompt(m, prompt_len)
+    with kie.Engine(kie.config(m, max_ctx=max_ctx, timeout_ms=20000, idle_ms=50, modes=modes), dw.kie) as eng:
         sid = eng.session_open()
         first = eng.prefill(sid, prompt)
         tok_d = torch.tensor([first], dtype=torch.int32, device="cuda")
-        out_d = torch.zeros(512, dtype=torch.int32, device="cuda")
-        eng.decode_launch(sid, tok_d.data_ptr(), 512, out_d.data_ptr())
+        out_d = torch.zeros(decode_n, dtype=torch.int32, device="cuda")
+        eng.decode_launch(sid, tok_d.data_ptr(), decode_n, out_d.data_ptr())
         eng.sync()
         gen = out_d.cpu().numpy()
         assert gen.min() >= 0 and gen.max() < m.vocab
         kp, vp = eng.session_kv(sid)
-        n = m.n_kv_heads * 1536 * m.head_dim
+        n = m.n_kv_heads * max_ctx * m.head_dim
         # copy layer 0 of the cache through a torch view of the engine's buffer
-        kt = _device_view(kp, n)
-        vt = _device_view(vp, n)
-        K0 = kt.cpu().numpy().view(np.uint16).reshape(m.n_kv_heads, 1536, m.head_dim)
-        V0 = vt.cpu().numpy().view(np.uint16).reshape(m.n_kv_heads, 1536, m.head_dim)
+        K0 = _device_view(kp, n).cpu().numpy().view(np.uint16).reshape(m.n_kv_heads, max_ctx, m.head_dim)
+        V0 = _device_view(vp, n).cpu().numpy().view(np.uint16).reshape(m.n_kv_heads, max_ctx, m.head_dim)
     seq = np.concatenate([prompt, [first], gen[:-1]])
     L0 = dw.host["layers"][0]
-    for p in (0, 1, 777, 1023, 1024, 1300, 1535):
+    D = m.head_dim
+    for p in positions:
         e = orc.value(dw.host["tok_emb"][seq[p]], m.dtype)
         h = orc.rmsnorm(e, L0["attn_norm"], m.dtype, m.rms_eps)
         k = orc.matvec(L0["wk"], m.dtype, h)
         v = orc.matvec(L0["wv"], m.dtype, h)
-        D = m.head_dim
         for g in range(m.n_kv_heads):
             kr = orc.rope(k[g * D:(g + 1) * D], p, m.rope_theta)
             want_k = orc.value(orc.store(kr, m.dtype), m.dtype)
             want_v = orc.value(orc.store(v[g * D:(g + 1) * D], m.dtype), m.dtype)
-            got_k = orc.value(K0[g, p], m.dtype)
-            got_v = orc.value(V0[g, p], m.dtype)
             # fp32 accumulation vs fp64: at most one rounding step of the stored value apart
-            np.testing.assert_allclose(got_k, want_k, rtol=2e-3, atol=1e-4)
-            np.testing.assert_allclose(got_v, want_v, rtol=2e-3, atol=1e-4)
+            np.testing.assert_allclose(orc.value(K0[g, p], m.dtype), want_k, rtol=2e-3, atol=1e-4)
+            np.testing.assert_allclose(orc.value(V0[g, p], m.dtype), want_v, rtol=2e-3, atol=1e-4)
+
+
+def test_full_1p9b_bench_launch_layer0_cache(kie):
+    """The benchmark's configuration (1.9B, prompt 1024, one launch of 512 steps), prompt
+    prefilled by the batch-1 kernel."""
+    from bandwidth_bound_stream_b200 import synth
+    _bench_launch_layer0_check(kie, synth.DENSE_1P9B, 1024, 512, (0, 1, 777, 1023, 1024, 1300, 1535),
+                               kie.KIE_MODE_BATCH1)
+
+
+def test_full_8b_bench_launch_layer0_cache(kie):
+    """The 8B (Llama-3-8B shape, bf16, theta 5e5) configuration: prompt 4096 prefilled in tick-kernel
+    chunks, one launch of 256 decode steps."""
+    from bandwidth_bound_stream_b200 import synth
+    _bench_launch_layer0_check(kie, synth.DENSE_8B, 4096, 256, (0, 63, 64, 2049, 4095, 4096, 4351),
+                               kie.KIE_MODE_BATCH1 | kie.KIE_MODE_TICK)
+
+
+def test_full_1p9b_32k_bench_launch_layer0_cache(kie):
+    """The long-context configuration: 1.9B, prompt 32768 prefilled in tick-kernel chunks, one
+    launch of 256 decode steps (attention over a 32K cache)."""
+    from bandwidth_bound_stream_b200 import synth
+    _bench_launch_layer0_check(kie, synth.DENSE_1P9B, 32768, 256, (0, 4095, 16384, 32703, 32767, 32768, 33023),
+                               kie.KIE_MODE_BATCH1 | kie.KIE_MODE_TICK)
 
 
 def _device_view(ptr, n):
