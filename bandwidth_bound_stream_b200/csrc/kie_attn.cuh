@@ -34,6 +34,11 @@ struct AttnArgs {
                              // tick kernel's B operand (column h * D + e)
     int brow;
     int gout;                // kv head whose output columns a unit writes; -1: unit / nsplit
+    uint32_t cnt_target;     // 0: the last split merges. Else every split merges a slice of its kv
+                             // head's output once cnt[kv head] reaches this value (the counters
+                             // then only count up; fp32 output A.o only)
+    long long timeout_ns;    // bound of that wait; on expiry err gets an error code
+    unsigned *err;
     int D, Hkv, nsplit, ctx;
 };
 
@@ -280,6 +285,65 @@ __device__ __forceinline__ void attn_tail(const AttnArgs &A, AttnSmem &S, int un
     }
     __threadfence();
     named_bar_sync(1, ATTN_THREADS);
+    if (A.cnt_target) {
+        // Every split merges its own slice of the kv head's output once all splits have
+        // published (after its last pass over the query heads): one (m, l) + partial-sum load
+        // for all splits, in a single round trip, and no single CTA merging everything.
+        const bool last_pass = hoff + GC >= Gt;
+        if (tid == 0) {
+            atomicAdd(A.cnt + g, 1u);
+            const uint64_t t0 = globaltimer();
+            unsigned spins = 0;
+            while (last_pass && (int)(ld_acquire_gpu_u32(A.cnt + g) - A.cnt_target) < 0) {
+                if ((++spins & 63u) == 0) {
+                    if (ld_volatile_u32(A.err) != 0u) break;  // another CTA failed: give up
+                    if ((long long)(globaltimer() - t0) > A.timeout_ns) {
+                        set_error(A.err, DERR_BARRIER_TIMEOUT, 0x50);
+                        break;
+                    }
+                }
+            }
+        }
+        named_bar_sync(1, ATTN_THREADS);
+        if (!last_pass) return;
+        const int s = unit % nsplit, E = Gt * D;
+        const int e0 = (int)((long long)s * E / nsplit), e1 = (int)((long long)(s + 1) * E / nsplit), ne = e1 - e0;
+        const float *pg = A.part + (size_t)g * nsplit * Gt * (D + 2);
+        float *ek = &S.wacc[0][0];   // [nsplit][Gt] max, then weights
+        float *lk = ek + nsplit * Gt;  // [nsplit][Gt] sums
+        float *ak = lk + nsplit * Gt;  // [nsplit][ne] partial sums of this slice
+        for (int i = tid; i < nsplit * Gt + nsplit * ne; i += ATTN_THREADS) {
+            if (i < nsplit * Gt) {
+                const float2 ml = __ldcg(reinterpret_cast<const float2 *>(pg + (size_t)i * (D + 2)));
+                ek[i] = ml.x;
+                lk[i] = ml.y;
+            } else {
+                const int j = i - nsplit * Gt, k = j / ne, ee = e0 + j % ne;
+                ak[j] = __ldcg(pg + ((size_t)k * Gt + ee / D) * (D + 2) + 2 + ee % D);
+            }
+        }
+        named_bar_sync(1, ATTN_THREADS);
+        if (tid < Gt) {
+            float M = -CUDART_INF_F;
+            for (int k = 0; k < nsplit; k++) M = fmaxf(M, ek[k * Gt + tid]);
+            float den = 0.f;
+            for (int k = 0; k < nsplit; k++) {
+                const float e = rescale(ek[k * Gt + tid], M);
+                ek[k * Gt + tid] = e;
+                den = fmaf(e, lk[k * Gt + tid], den);
+            }
+            S.red[tid] = den;
+        }
+        named_bar_sync(1, ATTN_THREADS);
+        for (int j = tid; j < ne; j += ATTN_THREADS) {  // splits added in ascending order
+            const int ee = e0 + j, jj = ee / D;
+            float num = 0.f;
+            for (int k = 0; k < nsplit; k++) num = fmaf(ek[k * Gt + jj], ak[k * ne + j], num);
+            A.o[(size_t)(go * Gt + jj) * D + ee % D] = num / S.red[jj];
+        }
+        named_bar_sync(1, ATTN_THREADS);
+        return;
+    }
     if (tid == 0) {
         const unsigned chunks = (unsigned)((Gt + GC - 1) / GC);
         const unsigned prev = atomicAdd(A.cnt + g, 1u);

@@ -549,7 +549,7 @@ __device__ int final_argmax(const KieParams &P) {
 // waits for those loads.)
 template <int DT, int GC>
 __device__ void attention_step(const KieParams &P, B1Shared &S, int l, int sid, int pos, unsigned long long &epoch,
-                               int t, int e) {
+                               int t, int e, uint32_t &att_use) {
     AttnArgs A;
     A.q = P.q;
     A.k = P.kcache + (size_t)sid * P.sess_stride + (size_t)l * P.Hkv * P.max_ctx * P.D;
@@ -561,6 +561,12 @@ __device__ void attention_step(const KieParams &P, B1Shared &S, int l, int sid, 
     A.bpack = nullptr;
     A.brow = 0;
     A.gout = -1;
+    // every split merges a slice once all splits of its kv head have published; each split
+    // adds one per pass over the query heads, and the counters only count up within a launch
+    A.cnt_target = (att_use + 1u) * (uint32_t)P.splits * (uint32_t)((P.G + GC - 1) / GC);
+    A.timeout_ns = P.timeout_ns;
+    A.err = P.err;
+    att_use++;
     A.D = P.D;
     A.Hkv = P.Hkv;
     A.nsplit = P.splits;
@@ -588,7 +594,7 @@ __device__ void attention_step(const KieParams &P, B1Shared &S, int l, int sid, 
 
 template <int DT>
 __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring, const KieCmd &cmd,
-                        unsigned long long &epoch) {
+                        unsigned long long &epoch, uint32_t &att_use) {
     int tok = cmd.in_tok;
     if (cmd.op == OP_DECODE && cmd.tok_dev) tok = __ldcg(cmd.tok_dev);
     const int L = P.L;
@@ -608,7 +614,7 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, cons
             trace_mark(P, t, e);
             epilogue_qkv<DT>(P, S, l, cmd.sid, pos, tok);
             trace_mark(P, t, e + 1);
-            attention_step<DT, 2>(P, S, l, cmd.sid, pos, epoch, t, e);  // also serves G == 1 (one idle head slot)
+            attention_step<DT, 2>(P, S, l, cmd.sid, pos, epoch, t, e, att_use);  // also serves G == 1 (one idle head slot)
             if (P.trace && t < P.trace_tokens && threadIdx.x == 0)  // end of this CTA's positions (0: no unit)
                 P.trace[((size_t)blockIdx.x * P.trace_tokens + t) * P.trace_events + e + 15] = S.at.t_unit;
             grid_barrier(P, S, epoch, P.timeout_ns, 2);
@@ -672,6 +678,7 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
 
     uint32_t ring_it = 0;  // chunks consumed (consumers) / issued (producer); both advance identically
     unsigned long long epoch = 0;
+    uint32_t att_use = 0;  // attention phases so far in this launch (the merge counters' targets)
     for (;;) {
         if (tid < KIE_CONS_THREADS) {
             if (!resident) {
@@ -717,7 +724,7 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
         if (tid >= KIE_CONS_THREADS) {
             if (tid == KIE_CONS_THREADS) produce(P, S, ring_it, smem, cmd);
         } else {
-            consume<DT>(P, S, ring_it, smem, cmd, epoch);
+            consume<DT>(P, S, ring_it, smem, cmd, epoch, att_use);
         }
         __syncthreads();
         if (resident && blockIdx.x == 0 && tid == 0) {
@@ -756,6 +763,9 @@ cudaError_t kie_b1_occupancy(int dtype, int *blocks_per_sm) {
 }
 
 cudaError_t kie_b1_launch(const KieParams &P, const KieCmd &one, int resident, cudaStream_t stream) {
+    // the attention merge counters count up from zero within a launch
+    const cudaError_t e = cudaMemsetAsync(P.cnt, 0, (size_t)P.Hkv * sizeof(unsigned), stream);
+    if (e != cudaSuccess) return e;
     KieParams p = P;
     KieCmd c = one;
     int r = resident;

@@ -43,6 +43,12 @@ KIE_DEV void st_release_sys_u32(volatile uint32_t *p, uint32_t v) {
 
 KIE_DEV unsigned ld_volatile_u32(const unsigned *p) { return *(const volatile unsigned *)p; }
 
+KIE_DEV unsigned ld_acquire_gpu_u32(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // Records the first device error (code, where). Later errors keep the first.
 KIE_DEV void set_error(unsigned *err, unsigned code, unsigned where) {
     atomicCAS(err, 0u, (code << 8) | (where & 0xFFu));

@@ -796,6 +796,9 @@ __device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M, uint32
         A.bpack = P.mr_bpack;  // the output is the O projection's B operand, row m
         A.brow = m;
         A.gout = g;
+        A.cnt_target = 0;
+        A.timeout_ns = 0;
+        A.err = nullptr;
         A.D = P.D;
         A.Hkv = P.Hkv;
         A.nsplit = 1;
