@@ -195,7 +195,6 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
     kie_engine *eng = new kie_engine();
     eng->cfg = *cfg;
     const kie_config &c = eng->cfg;
-    kie_status st = KIE_OK;
     auto bail = [&](kie_status s) {
         kie_destroy(eng);
         return s;
@@ -526,7 +525,6 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
     CKC(cudaDeviceSynchronize(), "create");
     eng->sess_len.assign(c.max_sessions, 0);
     eng->sess_used.assign(c.max_sessions, 0);
-    (void)st;
     *out = eng;
     return KIE_OK;
 }
