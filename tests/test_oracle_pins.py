@@ -137,6 +137,17 @@ def test_attention_matches_scipy_softmax():
         np.testing.assert_allclose(orc.attention(q, K, V, dt), w @ Vf, rtol=1e-11, atol=1e-13)
 
 
+def test_attention_weights_sum_to_one():
+    # with every value row equal to 1 the output is the sum of the softmax weights, whatever
+    # the scores (peaked, flat or spread over many positions)
+    rng = np.random.default_rng(12)
+    for n, D, dt, scale in [(1, 32, FP16, 1.0), (7, 64, BF16, 30.0), (513, 128, FP16, 0.1)]:
+        K, _ = _kv(rng, n, D, dt)
+        ones = orc.store(np.ones((n, D)), dt)
+        out = orc.attention(rng.normal(size=D) * scale, K, ones, dt)
+        np.testing.assert_allclose(out, np.ones(D), rtol=0, atol=1e-13)
+
+
 def test_attention_uniform_scores_average_values():
     rng = np.random.default_rng(8)
     _, V = _kv(rng, 9, 64, FP16)
