@@ -266,6 +266,52 @@ def test_errors_are_reported_not_fatal(kie):
         assert ei.value.status == kie.KIE_ERR_CAPACITY
 
 
+def test_empty_inputs_and_a_cache_filled_to_max_ctx(kie):
+    """Empty inputs are argument errors that change nothing. A session fills its cache to exactly
+    max_ctx in parity with the oracle at every position, after which one more token is a capacity
+    error from every entry point. A tick may end on the last position."""
+    from bandwidth_bound_stream_b200 import synth
+    from oracle.oracle import OracleModel
+    from tests.parity import assert_reports, compare_step
+    m = synth.TINY
+    max_ctx = 40
+    dw, eng, orc = _setup(kie, m, max_ctx, max_sessions=2, modes=kie.KIE_MODE_BATCH1 | kie.KIE_MODE_TICK)
+    with eng:
+        # prefill 24 (tick kernel chunks), then batch-1 decode up to position max_ctx - 1
+        assert_reports(_lockstep(kie, eng, orc, m, synth.prompt(m, 24), max_ctx - 24), m.dtype)
+        sid = eng.session_open()
+        full = 1 - sid  # the two slots are 0 and 1; the other one holds the full session
+        assert eng.session_length(full) == max_ctx
+        for call in (lambda: eng.decode_step(full, 1), lambda: eng.generate(full, 1, 1),
+                     lambda: eng.prefill(full, [1]), lambda: eng.tick([full], [1], 1)):
+            with pytest.raises(kie.KieError) as ei:
+                call()
+            assert ei.value.status == kie.KIE_ERR_CAPACITY
+        assert eng.session_length(full) == max_ctx
+        for call in (lambda: eng.prefill(sid, np.zeros(0, dtype=np.int32)), lambda: eng.generate(sid, 1, 0),
+                     lambda: eng.tick([], np.zeros(0, dtype=np.int32), 1), lambda: eng.tick([sid], [1], 0)):
+            with pytest.raises(kie.KieError) as ei:
+                call()
+            assert ei.value.status == kie.KIE_ERR_ARG
+        assert eng.session_length(sid) == 0
+        # a two-step tick that writes positions max_ctx - 2 and max_ctx - 1
+        o2 = OracleModel(m, dw.host, max_ctx)
+        p2 = synth.prompt(m, max_ctx - 2, session=3)
+        first = eng.prefill(sid, p2)
+        ref = o2.prefill(p2)
+        reps = [compare_step(ref, first, ref, m.dtype)]
+        t0 = int(np.argmax(ref))
+        logits = torch.empty((2, 1, m.vocab), dtype=torch.float32, device="cuda")
+        out = eng.tick([sid], [t0], 2, logits.data_ptr())
+        got = logits.cpu().numpy()
+        ref1 = o2.step(t0)
+        reps.append(compare_step(got[0, 0], int(out[0, 0]), ref1, m.dtype))
+        if int(out[0, 0]) == int(np.argmax(ref1)):  # else a low-margin step: the chains part here
+            reps.append(compare_step(got[1, 0], int(out[1, 0]), o2.step(int(out[0, 0])), m.dtype))
+        assert_reports(reps, m.dtype)
+        assert eng.session_length(sid) == max_ctx
+
+
 def test_resident_kernel_idles_out_and_relaunches(kie):
     """With no command the resident kernel gives up waiting after idle_ms and exits cleanly; the
     next call relaunches it and the results are unchanged."""
