@@ -266,6 +266,75 @@ def test_cache_append_at_later_position_uses_that_position():
     assert np.array_equal(m.k_cache[0, :, p].ravel(), k_rot.astype(np.float32).astype(np.float16).view(np.uint16))
 
 
+def _torch_values(bits, dt):
+    """Stored fp16/bf16 bits -> float64 tensor, decoded by numpy / torch (not by the oracle)."""
+    if dt == FP16:
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.float16).astype(np.float64))
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(torch.float64)
+
+
+def _torch_bits(values, dt):
+    """float64 array -> storage bits (fp32 first, then round to nearest even), by numpy / torch."""
+    f32 = np.asarray(values, dtype=np.float64).astype(np.float32)
+    if dt == FP16:
+        return f32.astype(np.float16).view(np.uint16)
+    return torch.from_numpy(f32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_whole_network_matches_torch_library_formulation():
+    """Every decode step of the chain against the same network written over the whole sequence
+    with torch library routines: F.rms_norm, rotation as complex multiplication, causal
+    scaled_dot_product_attention on kv heads repeated per query group, F.silu. Random norm gains
+    and a scaled-up Wq/Wk (peaked attention) pin the wiring that the building-block pins leave
+    open: which gain goes where, gate vs up, the query's rotation at later positions, the score
+    scale and the kv-head map."""
+    import torch.nn.functional as F
+    rng = np.random.default_rng(21)
+    for cfg in (MINI, dataclasses.replace(MINI, dtype=BF16, n_heads=6, n_kv_heads=2, head_dim=16, rope_theta=5e5)):
+        dt, d, Hq, Hkv, D = cfg.dtype, cfg.d_model, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+        w = _weights(cfg)
+        for L in w["layers"]:
+            for name in ("wq", "wk"):
+                L[name] = _torch_bits(8.0 * _torch_values(L[name], dt).numpy(), dt)
+            for name in ("attn_norm", "mlp_norm"):
+                L[name] = _torch_bits(rng.uniform(0.5, 1.5, d), dt)
+        w["final_norm"] = _torch_bits(rng.uniform(0.5, 1.5, d), dt)
+        toks = synth.prompt(cfg, 9)
+        n = len(toks)
+
+        store = torch.float16 if dt == FP16 else torch.bfloat16
+        half = D // 2
+        ang = torch.arange(n, dtype=torch.float64)[:, None] * cfg.rope_theta ** (
+            -2.0 * torch.arange(half, dtype=torch.float64) / D)
+        turn = torch.polar(torch.ones_like(ang), ang)[:, None, :]  # [position, 1, D/2]
+
+        def rotate(t):  # [position, head, D]: the pair (i, i + D/2) as one complex number
+            z = torch.complex(t[..., :half], t[..., half:]) * turn
+            return torch.cat([z.real, z.imag], dim=-1)
+
+        def val(bits):
+            return _torch_values(bits, dt)
+
+        x = val(w["tok_emb"])[torch.from_numpy(toks.astype(np.int64))]
+        for L in w["layers"]:
+            h = F.rms_norm(x, (d,), weight=val(L["attn_norm"]), eps=cfg.rms_eps)
+            q = rotate((h @ val(L["wq"]).T).view(n, Hq, D))
+            k = rotate((h @ val(L["wk"]).T).view(n, Hkv, D)).to(torch.float32).to(store).to(torch.float64)
+            v = (h @ val(L["wv"]).T).view(n, Hkv, D).to(torch.float32).to(store).to(torch.float64)
+            rep = Hq // Hkv
+            o = F.scaled_dot_product_attention(q.transpose(0, 1), k.repeat_interleave(rep, 1).transpose(0, 1),
+                                               v.repeat_interleave(rep, 1).transpose(0, 1), is_causal=True)
+            x = x + o.transpose(0, 1).reshape(n, Hq * D) @ val(L["wo"]).T
+            h = F.rms_norm(x, (d,), weight=val(L["mlp_norm"]), eps=cfg.rms_eps)
+            x = x + (F.silu(h @ val(L["w_gate"]).T) * (h @ val(L["w_up"]).T)) @ val(L["w_down"]).T
+        want = (F.rms_norm(x, (d,), weight=val(w["final_norm"]), eps=cfg.rms_eps) @ val(w["lm_head"]).T).numpy()
+
+        m = orc.OracleModel(cfg, w, n)
+        got = np.stack([m.step(t) for t in toks])
+        assert np.abs(want).max() > 0.1  # logits of a visible size
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-10)
+
+
 def test_bad_arguments_rejected():
     m = orc.OracleModel(MINI, _weights(MINI), 2)
     with pytest.raises(ValueError):
