@@ -312,6 +312,65 @@ def test_empty_inputs_and_a_cache_filled_to_max_ctx(kie):
         assert eng.session_length(sid) == max_ctx
 
 
+def _randomize_gains(dw, model, seed):
+    """Norm gains from U(0.5, 1.5), rounded to the storage dtype by numpy / torch, written to
+    the device tensors and to the host copy the oracle reads (before the engine is created)."""
+    rng = np.random.default_rng(seed)
+    for (name, layer), t in dw.tensors.items():
+        if name not in ("attn_norm", "mlp_norm", "final_norm"):
+            continue
+        f32 = rng.uniform(0.5, 1.5, model.d_model).astype(np.float32)
+        if model.dtype == 0:
+            bits = f32.astype(np.float16).view(np.uint16)
+        else:
+            bits = torch.from_numpy(f32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        t.copy_(torch.from_numpy(bits.view(np.int16)))
+        if layer >= 0:
+            dw.host["layers"][layer][name] = bits
+        else:
+            dw.host[name] = bits
+
+
+def test_random_norm_gains_parity(kie):
+    """The synthetic models' gains are all 1.0, which cannot show a gain applied in the wrong
+    place. With random gains: the prompt through the tick kernel's chunks, decode steps
+    through the batch-1 kernel, then two-step ticks, each against the oracle on the same gains."""
+    from bandwidth_bound_stream_b200 import synth
+    from oracle.oracle import OracleModel
+    from tests.parity import assert_reports, compare_step
+    for i, m in enumerate((synth.TINY, synth.RAGGED)):
+        max_ctx = 48
+        dw = kie.DeviceWeights(m, host_copy=True)
+        _randomize_gains(dw, m, 40 + i)
+        orc = OracleModel(m, dw.host, max_ctx)
+        cfg = kie.config(m, max_ctx=max_ctx, max_sessions=2, timeout_ms=5000, idle_ms=50,
+                         modes=kie.KIE_MODE_BATCH1 | kie.KIE_MODE_TICK)
+        with kie.Engine(cfg, dw.kie) as eng:
+            reps = _lockstep(kie, eng, orc, m, synth.prompt(m, 20), 8)
+            sid = eng.session_open()
+            o2 = OracleModel(m, dw.host, max_ctx)
+            p2 = synth.prompt(m, 12, session=4)
+            first = eng.prefill(sid, p2)
+            ref = o2.prefill(p2)
+            reps.append(compare_step(ref, first, ref, m.dtype))
+            tok = int(np.argmax(ref))
+            logits = torch.empty((2, 1, m.vocab), dtype=torch.float32, device="cuda")
+            for _ in range(3):
+                out = eng.tick([sid], [tok], 2, logits.data_ptr())
+                got = logits.cpu().numpy()
+                ref1 = o2.step(tok)
+                reps.append(compare_step(got[0, 0], int(out[0, 0]), ref1, m.dtype))
+                if int(out[0, 0]) != int(np.argmax(ref1)):
+                    break  # a low-margin step (accepted above): the two chains part here
+                ref2 = o2.step(int(out[0, 0]))
+                reps.append(compare_step(got[1, 0], int(out[1, 0]), ref2, m.dtype))
+                if int(out[1, 0]) != int(np.argmax(ref2)):
+                    break
+                tok = int(out[1, 0])
+        assert_reports(reps, m.dtype)
+        dw.free()
+
+
 def test_resident_kernel_idles_out_and_relaunches(kie):
     """With no command the resident kernel gives up waiting after idle_ms and exits cleanly; the
     next call relaunches it and the results are unchanged."""
