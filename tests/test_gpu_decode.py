@@ -313,13 +313,21 @@ def test_empty_inputs_and_a_cache_filled_to_max_ctx(kie):
 
 
 def _randomize_gains(dw, model, seed):
-    """Norm gains from U(0.5, 1.5), rounded to the storage dtype by numpy / torch, written to
-    the device tensors and to the host copy the oracle reads (before the engine is created)."""
+    """Norm gains from U(0.5, 1.5) and Wq, Wk scaled by 8 (peaked attention), rounded to the
+    storage dtype by numpy / torch, written to the device tensors and to the host copy the
+    oracle reads (before the engine is created)."""
     rng = np.random.default_rng(seed)
     for (name, layer), t in dw.tensors.items():
-        if name not in ("attn_norm", "mlp_norm", "final_norm"):
+        if name in ("attn_norm", "mlp_norm", "final_norm"):
+            f32 = rng.uniform(0.5, 1.5, model.d_model).astype(np.float32)
+        elif name in ("wq", "wk"):
+            old = t.cpu().numpy().view(np.uint16)
+            if model.dtype == 0:
+                f32 = 8.0 * old.view(np.float16).astype(np.float32)
+            else:
+                f32 = 8.0 * torch.from_numpy(old.view(np.int16)).view(torch.bfloat16).float().numpy()
+        else:
             continue
-        f32 = rng.uniform(0.5, 1.5, model.d_model).astype(np.float32)
         if model.dtype == 0:
             bits = f32.astype(np.float16).view(np.uint16)
         else:
@@ -331,10 +339,12 @@ def _randomize_gains(dw, model, seed):
             dw.host[name] = bits
 
 
-def test_random_norm_gains_parity(kie):
+def test_random_norm_gains_and_peaked_attention_parity(kie):
     """The synthetic models' gains are all 1.0, which cannot show a gain applied in the wrong
-    place. With random gains: the prompt through the tick kernel's chunks, decode steps
-    through the batch-1 kernel, then two-step ticks, each against the oracle on the same gains."""
+    place, and their small models attend almost uniformly, which hides a wrong score scale.
+    With random gains and Wq, Wk scaled by 8: the prompt through the tick kernel's chunks
+    (tensor-core scores), decode steps through the batch-1 kernel, then two-step ticks, each
+    against the oracle on the same weights."""
     from bandwidth_bound_stream_b200 import synth
     from oracle.oracle import OracleModel
     from tests.parity import assert_reports, compare_step
