@@ -205,6 +205,9 @@ def main():
     ap.add_argument("--tick-only", action="store_true", help="only the tick workload (its own JSON line)")
     ap.add_argument("--tick-model", default="dense-10.8b")
     ap.add_argument("--tick-prompt", type=int, default=0, help="fixed prompt length per session (0 = seeded 1000-1500)")
+    ap.add_argument("--trace", type=int, default=0,
+                    help="after the timed region, trace this many tokens (<= 8) of one more launch and add the "
+                         "batch-1 kernel's per-phase durations as phase_us (0 = off)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank, world, local = dist_setup()
@@ -314,6 +317,16 @@ def main():
         a = time.perf_counter()
         tok = eng.decode_step(sid, tok)
         itl.append((time.perf_counter() - a) * 1e3)
+    phase_us = None
+    if args.trace > 0:  # untimed: one more launch with the phase trace on, at the same context
+        from bandwidth_bound_stream_b200 import trace
+        n_tr = min(args.trace, 8, decode_n)
+        eng.trace_enable(n_tr)
+        eng.session_rewind(sid, prompt_len)
+        eng.decode_launch(sid, tok_d.data_ptr(), n_tr, out_d.data_ptr(), None, stream.cuda_stream)
+        eng.sync()
+        phase_us = trace.batch1_phase_us(eng.trace_read(n_tr), m.n_layers)
+        eng.trace_enable(0)
     eng.close()
 
     value = whole_job_rate(decode_n * args.steps, world, total_ms / 1e3)
@@ -351,6 +364,8 @@ def main():
                     "itl_ms_p99": round(float(np.percentile(itl, 99)), 4),
                     "per_launch_ms": [round(x, 3) for x in per_launch]},
     }
+    if phase_us is not None:
+        line["phase_us"] = phase_us
     if args.ticks > 0 and headline:
         line["tick"] = run_tick(args.ticks, args.warmup, local, clocks_for=local)
     if want_cpu:
