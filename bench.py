@@ -125,15 +125,22 @@ def oracle_baseline(model, host_weights, ctx0: int, min_s=10.0, max_s=30.0):
 
 
 def dist_setup():
+    """Rank, world size and local device index under torchrun (one process per GPU): NCCL on
+    the rank's GPU, or gloo on a host without CUDA (where only the reference arm can run)."""
     if "RANK" not in os.environ:
         return 0, 1, 0
+    import datetime
+
     import torch
     import torch.distributed as dist
     rank, world = int(os.environ["RANK"]), int(os.environ["WORLD_SIZE"])
     local = int(os.environ.get("LOCAL_RANK", rank))
-    torch.cuda.set_device(local)
-    import datetime
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+    timeout = datetime.timedelta(seconds=300)
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+    else:
+        dist.init_process_group("gloo", timeout=timeout)
     return rank, world, local
 
 
