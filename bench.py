@@ -84,6 +84,12 @@ class ClockSampler:
             return None
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=10)
+        return self.summarise(out)
+
+    @staticmethod
+    def summarise(out: str):
+        """Median SM clock of the loaded samples (above half the highest), the max clock, and every
+        throttle reason seen Active, from `nvidia-smi --format=csv,noheader,nounits` lines of FIELDS."""
         sm, mx, reasons = [], 0.0, set()
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         for line in out.strip().splitlines():
@@ -96,7 +102,7 @@ class ClockSampler:
             except ValueError:
                 continue
             for name, v in zip(names, parts[4:8]):
-                if v.lower().startswith("active"):
+                if v.lower().startswith("active"):  # "Not Active" does not count
                     reasons.add(name)
         if not sm:
             return None
