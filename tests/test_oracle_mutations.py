@@ -58,7 +58,22 @@ SLIPS = {
     "lm_head_is_the_embedding": [("orc_matvec(c->vocab, d, w->lm_head,", "orc_matvec(c->vocab, d, w->tok_emb,")],
     "embedding_row_off_by_one": [("x[i] = orc_value(w->tok_emb[(int64_t)token * d + i], dt);",
                                   "x[i] = orc_value(w->tok_emb[(int64_t)(token + (token + 1 < c->vocab)) * d + i], dt);")],
+    "rope_position_off_by_one": [("orc_rope(D, pos, c->rope_theta, q + hh * D);", "orc_rope(D, pos + 1, c->rope_theta, q + hh * D);"),
+                                 ("orc_rope(D, pos, c->rope_theta, k + g * D);", "orc_rope(D, pos + 1, c->rope_theta, k + g * D);"),
+                                 ("orc_rope(D, t, c->rope_theta, Q + ((int64_t)t * Hq + hh) * D);",
+                                  "orc_rope(D, t + 1, c->rope_theta, Q + ((int64_t)t * Hq + hh) * D);"),
+                                 ("orc_rope(D, t, c->rope_theta, Kf + g * D);", "orc_rope(D, t + 1, c->rope_theta, Kf + g * D);")],
+    "attention_skips_position_zero": [
+        ("orc_attention(D, pos + 1, q + hh * D, kcache + kv_index(c, max_ctx, l, g, 0),\n"
+         "                          vcache + kv_index(c, max_ctx, l, g, 0), dt, o + hh * D);",
+         "orc_attention(D, pos > 0 ? pos : 1, q + hh * D, kcache + kv_index(c, max_ctx, l, g, pos > 0 ? 1 : 0),\n"
+         "                          vcache + kv_index(c, max_ctx, l, g, pos > 0 ? 1 : 0), dt, o + hh * D);"),
+        ("orc_attention(D, t + 1, Q + ((int64_t)t * Hq + hh) * D, Ks + (int64_t)g * n * D,\n"
+         "                              Vs + (int64_t)g * n * D, dt, O + ((int64_t)t * Hq + hh) * D);",
+         "orc_attention(D, t > 0 ? t : 1, Q + ((int64_t)t * Hq + hh) * D, Ks + ((int64_t)g * n + (t > 0)) * D,\n"
+         "                              Vs + ((int64_t)g * n + (t > 0)) * D, dt, O + ((int64_t)t * Hq + hh) * D);")],
     # building blocks
+    "rmsnorm_fixed_eps": [("double r = 1.0 / sqrt(ss / n + eps);", "double r = 1.0 / sqrt(ss / n + 1e-6);")],
     "score_scale_missing": [("double scale = 1.0 / sqrt((double)D)", "double scale = 1.0")],
     "softmax_denominator_wrong": [("s[j] = exp(s[j] - m); sum += s[j];",
                                    "s[j] = exp(s[j] - m); sum += s[j] * 0.5 + 0.5 * s[j] * (j == 0);")],
