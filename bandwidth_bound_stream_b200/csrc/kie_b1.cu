@@ -9,12 +9,12 @@
 //  * Warp 16 (the producer) walks this CTA's fixed weight schedule for the whole command
 //    (all layers, all tokens) and copies it, chunk by chunk, into a 3 x 64 KB shared-memory
 //    ring with 1-D bulk async copies (TMA). The ring holds 192 KB; while the consumers sit
-//    in attention (which reads no weights) it fills and HBM would idle, so a CTA that has
-//    finished its attention unit may ask L2 for the `pf_chunks` chunks beyond the ring (the
-//    producer publishes where it stands; off by default). The schedule is contiguous in HBM
-//    because the weights were repacked at engine creation in exactly this order, so each SM
-//    streams one disjoint span (the aligned, topology-aware access of the same section).
-//    The producer never waits on grid barriers.
+//    in attention (which reads no weights) it fills and HBM would idle, so the producer also
+//    keeps the `pf_chunks` chunks after the one it copies requested into L2 (an L2 lead of a
+//    fixed size). The schedule is contiguous in HBM because the weights were repacked at
+//    engine creation in exactly this order, so each SM streams one disjoint span (the
+//    aligned, topology-aware access of the same section). The producer never waits on grid
+//    barriers.
 //  * Warps 0-15 (consumers) run the phases of each layer on the staged chunks:
 //      QKV  : RMSNorm -> [Wq;Wk;Wv] rows -> RoPE -> q, and the K/V append to the cache
 //      ATTN : split-K single-query attention over the cache, last split merges (LSE)
@@ -66,8 +66,6 @@ struct __align__(16) B1Shared {
     int gb_ok;
     int row0[KIE_NPH], row1[KIE_NPH];
     unsigned long long wait_cons;
-    const uint8_t *volatile pf_next;  // the producer's next unfetched byte of the segment
-    const uint8_t *seg_end;
 };
 
 // word-wise copies of the command record (volatile: it may live in mapped host memory)
@@ -202,13 +200,28 @@ __device__ bool chunk_next(const KieParams &P, const B1Shared &S, const KieCmd &
 
 __device__ void produce(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint8_t *ring, const KieCmd &cmd) {
     const uint8_t *seg = P.wpack + P.seg_off[blockIdx.x];
-    ChunkIter fetch;
+    ChunkIter fetch, lead;
     chunk_begin(fetch, seg);
+    chunk_begin(lead, seg);
     const uint8_t *a;
     uint32_t b;
     unsigned long long waited = 0;
     int tok = 0;
+    // The L2 lead: the pf_chunks chunks after the one being copied into the ring are requested
+    // into L2 as well, so HBM keeps streaming while the ring is full and the consumers sit in
+    // latency-bound work (attention, barriers); the ring then refills from L2.
+    int ahead = 0;  // chunks the lead iterator has passed beyond the fetch iterator
+    bool lead_live = P.pf_chunks > 0 && chunk_next(P, S, cmd, lead, a, b);  // skip chunk 0 (fetched now)
     while (chunk_next(P, S, cmd, fetch, a, b)) {
+        if (ahead > 0) ahead--;
+        while (lead_live && ahead < P.pf_chunks) {
+            const uint8_t *la;
+            uint32_t lb;
+            lead_live = chunk_next(P, S, cmd, lead, la, lb);
+            if (!lead_live) break;
+            bulk_prefetch_l2(la, lb);
+            ahead++;
+        }
         if (fetch.t != tok) {
             if (P.trace && tok < P.trace_tokens)
                 P.trace[((size_t)blockIdx.x * P.trace_tokens + tok) * P.trace_events + P.trace_events - 1] = waited;
@@ -230,7 +243,6 @@ __device__ void produce(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint
         mbar_arrive_expect_tx(&S.full[slot], b);
         bulk_g2s(ring + (size_t)slot * KIE_SLOT_BYTES, a, b, &S.full[slot]);
         ring_it++;
-        S.pf_next = a + b;
     }
     if (P.trace && tok < P.trace_tokens)
         P.trace[((size_t)blockIdx.x * P.trace_tokens + tok) * P.trace_events + P.trace_events - 1] = waited;
@@ -579,14 +591,6 @@ __device__ void attention_step(const KieParams &P, B1Shared &S, int l, int sid, 
     if (have && !S.abort) {
         for (int hoff = 0; hoff < P.G; hoff += GC) attn_unit<DT, GC, KIE_CONS_WARPS>(A, S.at, unit, P.G, hoff);
     }
-    if (P.pf_chunks > 0 && threadIdx.x == 0) {
-        // this CTA's K/V reads are done; while the others finish theirs (and the ring sits full),
-        // the weights beyond the ring start moving into L2
-        const uint8_t *p = S.pf_next;
-        const long long n = min((long long)P.pf_chunks * KIE_SLOT_BYTES, (long long)(S.seg_end - p));
-        for (long long o = 0; o < n; o += KIE_SLOT_BYTES)
-            bulk_prefetch_l2(p + o, (uint32_t)min((long long)KIE_SLOT_BYTES, n - o));
-    }
     trace_mark(P, t, e + 3);
 }
 
@@ -602,8 +606,11 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, cons
         const int pos = cmd.pos0 + t;
         if (cmd.op == OP_PREFILL) tok = __ldcg(P.tokbuf + t);
         if (tok < 0 || tok >= P.V) {
+            // e.g. a caller's device token, or an argmax over non-finite logits: fail the
+            // command, and read no row outside the embedding table on the way out
             if (threadIdx.x == 0) set_error(P.err, DERR_BAD_TOKEN, 0);
             S.abort = 1;
+            tok = 0;
         }
         if (threadIdx.x == 0) S.wait_cons = 0;
         trace_mark(P, t, 0);
@@ -645,7 +652,12 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, cons
             grid_barrier(P, S, epoch, P.timeout_ns, 6);
             trace_mark(P, t, eh + 1);
             tok = final_argmax(P);
-            if (blockIdx.x == 0 && threadIdx.x == 0 && cmd.out) cmd.out[cmd.op == OP_PREFILL ? 0 : t] = tok;
+            if (blockIdx.x == 0 && threadIdx.x == 0) {
+                if (cmd.out) cmd.out[cmd.op == OP_PREFILL ? 0 : t] = tok;
+                // no index wins an argmax over non-finite logits: the command fails (a later
+                // step of it also stops at the token check above)
+                if (tok < 0 || tok >= P.V) set_error(P.err, DERR_BAD_TOKEN, 1);
+            }
             trace_mark(P, t, eh + 2);
         }
         if (P.trace && t < P.trace_tokens && threadIdx.x == 0)
@@ -667,8 +679,6 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
         }
         fence_mbar_init();
         S.abort = 0;
-        S.pf_next = P.wpack + P.seg_off[blockIdx.x];
-        S.seg_end = P.wpack + P.seg_off[blockIdx.x + 1];
     }
     if (tid < KIE_NPH) {
         S.row0[tid] = P.row0[tid * (P.nblk + 1) + blockIdx.x];
@@ -729,7 +739,7 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
         __syncthreads();
         if (resident && blockIdx.x == 0 && tid == 0) {
             __threadfence_system();
-            P.mbox->status = S.abort ? -1 : 0;
+            P.mbox->status = (S.abort || ld_volatile_u32(P.err) != 0u) ? -1 : 0;
             st_release_sys_u32(&P.mbox->done_seq, cmd.seq);
         }
         if (!resident || S.abort) break;

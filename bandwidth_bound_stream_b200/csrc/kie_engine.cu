@@ -76,7 +76,18 @@ struct kie_engine {
     std::vector<int> sess_len;
     std::vector<char> sess_used;
     bool poisoned = false;
+    int pending_fault = KIE_FAULT_NONE;  // kie_inject_fault: applied to the next kernel launch
     std::string err;
+
+    // Clears the grid-barrier counter before a launch. With KIE_FAULT_BARRIER_SHORT pending it
+    // starts one arrival short instead (all ones: the first arrival wraps it to zero, so after
+    // every CTA has arrived it reads nblk - 1), and the first grid barrier of the launch cannot
+    // complete.
+    cudaError_t reset_barrier(cudaStream_t st) {
+        const int fill = pending_fault == KIE_FAULT_BARRIER_SHORT ? 0xFF : 0;
+        pending_fault = KIE_FAULT_NONE;
+        return cudaMemsetAsync(P.bar, fill, 16, st);
+    }
 
     kie_status fail(kie_status s, const char *fmt, ...) {
         char buf[512];
@@ -560,7 +571,7 @@ static kie_status check_device_error(kie_engine *eng) {
 }
 
 static kie_status launch_resident(kie_engine *eng, int kind) {
-    cudaError_t e = cudaMemsetAsync(eng->P.bar, 0, 16, eng->stream);
+    cudaError_t e = eng->reset_barrier(eng->stream);
     if (e == cudaSuccess) {
         KieCmd none{};
         e = kind == KIND_MR ? kie_mr_launch(eng->P, none, 1, eng->stream) : kie_b1_launch(eng->P, none, 1, eng->stream);
@@ -587,7 +598,8 @@ static kie_status doorbell(kie_engine *eng, const KieCmd &cmd_in, int kind) {
     memcpy((void *)&mb->cmd, &cmd, sizeof cmd);
     std::atomic_thread_fence(std::memory_order_release);
     mb->cmd_seq = s;
-    const double t0 = now_s(), limit = eng->cfg.timeout_ms * 1e-3 + (cmd.op == OP_EXIT ? 0.0 : 0.0);
+    // the device's first wait of a command (the broadcast barrier) is bounded by idle + timeout
+    const double t0 = now_s(), limit = (eng->cfg.timeout_ms + eng->cfg.idle_ms) * 1e-3;
     unsigned spins = 0;
     for (;;) {
         if (mb->done_seq == s) break;
@@ -603,8 +615,9 @@ static kie_status doorbell(kie_engine *eng, const KieCmd &cmd_in, int kind) {
                 kie_status ls = launch_resident(eng, kind);  // it went idle before taking the command
                 if (ls != KIE_OK) return ls;
             }
-            // the time limit scales with the work of the command
-            const double budget = limit * (1.0 + (cmd.n > 0 ? cmd.n / 64.0 : 0.0));
+            // the time limit scales with the work of the command, with room for the device to
+            // report its own timeout first
+            const double budget = 1.5 * limit * (1.0 + (cmd.n > 0 ? cmd.n / 64.0 : 0.0));
             if (now_s() - t0 > budget) {
                 return eng->fail(KIE_ERR_TIMEOUT, "no answer from the device after %.1f s", now_s() - t0);
             }
@@ -828,7 +841,7 @@ extern "C" kie_status kie_decode_launch(kie_engine *eng, int32_t sid, const int3
     cmd.tok_dev = in_token_dev;
     cmd.out = out_tokens_dev;
     cmd.logits = logits_dev;
-    cudaError_t e = cudaMemsetAsync(eng->P.bar, 0, 16, st);
+    cudaError_t e = eng->reset_barrier(st);
     if (e == cudaSuccess) e = kie_b1_launch(eng->P, cmd, 0, st);
     if (e != cudaSuccess) return eng->cuda_fail(e, "launching the decode kernel");
     eng->sess_len[sid] = ctx + n;
@@ -879,7 +892,7 @@ extern "C" kie_status kie_tick_launch(kie_engine *eng, int32_t n_sess, const int
         e = cudaMemcpyAsync(eng->P.mr_pos, sp.data() + n_sess, (size_t)n_sess * 4, cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(eng->P.mr_tok, in_tokens_dev, (size_t)n_sess * 4, cudaMemcpyDeviceToDevice, st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(eng->P.bar, 0, 16, st);
+    if (e == cudaSuccess) e = eng->reset_barrier(st);
     KieCmd cmd{};
     cmd.op = OP_TICK;
     cmd.n = steps;
@@ -918,6 +931,17 @@ extern "C" kie_status kie_tick(kie_engine *eng, int32_t n_sess, const int32_t *s
     const volatile int32_t *out = eng->mbox_host->io + 192;
     for (int i = 0; i < steps * n_sess; i++) out_tokens[i] = out[i];
     for (int i = 0; i < n_sess; i++) eng->sess_len[sids[i]] += steps;
+    return KIE_OK;
+}
+
+// ---------------------------------------------------------------- fault injection (tests)
+
+extern "C" kie_status kie_inject_fault(kie_engine *eng, int32_t fault) {
+    kie_status s = check_live(eng);
+    if (s != KIE_OK) return s;
+    if (fault != KIE_FAULT_NONE && fault != KIE_FAULT_BARRIER_SHORT) return eng->fail(KIE_ERR_ARG, "unknown fault %d", fault);
+    if ((s = stop_resident(eng)) != KIE_OK) return s;  // the fault applies to a fresh launch
+    eng->pending_fault = fault;
     return KIE_OK;
 }
 

@@ -83,7 +83,7 @@ struct KieParams {
     unsigned *last_seq;             // last doorbell sequence processed
     KieCmd *cmd;                    // command broadcast slot
     long long timeout_ns, idle_ns;
-    int pf_chunks;                  // weight chunks beyond the ring requested into L2 after each attention unit
+    int pf_chunks;                  // L2 lead: weight chunks after the one being copied that are kept requested into L2
     float *ssq;                     // [nblk] per-CTA sums of squares of the residual rows it owns
     unsigned long long *trace;      // phase stamps (null = off)
     int trace_tokens, trace_events;

@@ -876,6 +876,10 @@ __device__ void phase_argmax(const KieParams &P, MrShared &S, const KieCmd &cmd,
             float v = S.red[0];
             int i = __float_as_int(S.red[8]);
             for (int k = 1; k < MR_WORKERS / 32; k++) amax(v, i, S.red[k], __float_as_int(S.red[8 + k]));
+            if (i < 0 || i >= P.V) {  // non-finite logits (no index wins): fail the command
+                set_error(P.err, DERR_BAD_TOKEN, 0x41);
+                S.abort = 1;
+            }
             P.mr_tok[m] = i;                          // input of the next step
             P.mr_pos[m] = __ldcg(P.mr_pos + m) + 1;
             if (cmd.out) {

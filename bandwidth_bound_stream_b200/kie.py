@@ -25,7 +25,8 @@ EXPORTS = ("kie_config_defaults", "kie_create", "kie_destroy", "kie_session_open
            "kie_session_length", "kie_session_rewind", "kie_session_kv", "kie_prefill", "kie_decode_step",
            "kie_generate", "kie_decode_launch", "kie_sync", "kie_tick", "kie_last_error", "kie_status_string",
            "kie_flash_decode", "kie_flash_decode_scratch_bytes", "kie_trace_enable", "kie_trace_read",
-           "kie_trace_events", "kie_flash_decode_noalloc", "kie_tick_launch")
+           "kie_trace_events", "kie_flash_decode_noalloc", "kie_tick_launch", "kie_inject_fault")
+KIE_FAULT_NONE, KIE_FAULT_BARRIER_SHORT = 0, 1
 
 
 class KieConfig(ctypes.Structure):
@@ -77,6 +78,7 @@ def _load():
         "kie_trace_events": (i32, [vp]),
         "kie_flash_decode_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, i64, i32, vp, vp]),
         "kie_tick_launch": (i32, [vp, i32, vp, vp, i32, vp, vp, vp]),
+        "kie_inject_fault": (i32, [vp, i32]),
     }
     for name, (res, args) in sig.items():
         f = getattr(h, name)
@@ -204,6 +206,9 @@ class Engine:
         if n.value:
             self._check(lib.kie_trace_read(self.h, out.ctypes.data, n.value, ctypes.byref(n)), "kie_trace_read")
         return out.reshape(-1, tokens, ev)
+
+    def inject_fault(self, fault: int):
+        self._check(lib.kie_inject_fault(self.h, fault), "kie_inject_fault")
 
     def sync(self):
         self._check(lib.kie_sync(self.h), "kie_sync")

@@ -69,11 +69,12 @@ typedef struct {
     int32_t idle_ms;      /* the resident kernel exits after this long with no command */
     int32_t modes;        /* KIE_MODE_* bitmask                                        */
     int32_t device;       /* CUDA device ordinal                                       */
-    int32_t prefetch_kb;  /* batch-1 kernel: per SM, the KB of weights beyond its shared-
-                             memory ring that a CTA requests into L2 once it has finished
-                             its attention unit (attention reads no weights, so HBM would
-                             otherwise idle while the other units finish); 0 = ring only.
-                             Rounded up to 64 KB ring chunks.                            */
+    int32_t prefetch_kb;  /* batch-1 kernel: per SM, the KB of weights after the chunk
+                             being copied into the shared-memory ring that are kept
+                             requested into L2 (an L2 lead of fixed size, so HBM keeps
+                             streaming while the ring is full and the kernel sits in
+                             attention or at a barrier); 0 = ring only. Rounded up to
+                             64 KB ring chunks.                                          */
 } kie_config;
 
 /*
@@ -201,6 +202,20 @@ int32_t kie_trace_events(kie_engine *eng);
 kie_status kie_tick_launch(kie_engine *eng, int32_t n_sess, const int32_t *sids, const int32_t *in_tokens_dev,
                            int32_t steps, int32_t *out_tokens_dev, float *logits_dev, void *stream);
 
+/*
+ * Fault injection for tests of the failure paths, made on the host (no GPU fault, trap or
+ * hang): with KIE_FAULT_BARRIER_SHORT the next kernel launch of this engine (resident or
+ * stream-ordered, either kernel) starts its grid-barrier counter one arrival short. The
+ * first grid barrier of that launch then cannot complete: every CTA's bounded wait runs out
+ * after timeout_ms (the resident kernel's first barrier: idle_ms + timeout_ms), the kernel
+ * records the timeout in its error word, waits for its own copies in flight, releases its
+ * tensor memory and returns. The call that owns the launch reports KIE_ERR_TIMEOUT and the
+ * engine is poisoned (KIE_ERR_STATE afterwards). A resident kernel is stopped first, so the
+ * fault always meets a fresh launch. KIE_FAULT_NONE cancels a pending fault.
+ */
+enum { KIE_FAULT_NONE = 0, KIE_FAULT_BARRIER_SHORT = 1 };
+kie_status kie_inject_fault(kie_engine *eng, int32_t fault);
+
 /* Copies the engine's last error message (NUL-terminated, truncated to len). */
 kie_status kie_last_error(kie_engine *eng, char *buf, int32_t len);
 
@@ -217,7 +232,8 @@ const char *kie_status_string(kie_status s);
  * scratch_dev: caller-owned DEVICE buffer of at least kie_flash_decode_scratch_bytes(...)
  * bytes (split partials and merge counters; contents on entry are ignored).
  * All DEVICE, stream-ordered on `stream` (cudaStream_t, NULL = legacy default stream).
- * n_ctx >= 1, head_dim even <= 128, n_heads/n_kv_heads <= 8. Returns KIE_ERR_ARG on bad shapes.
+ * n_ctx >= 1, head_dim one of 8, 16, 32, 64, 128, n_heads a multiple of n_kv_heads with
+ * n_heads/n_kv_heads <= 8. Returns KIE_ERR_ARG on other shapes.
  */
 kie_status kie_flash_decode(const float *q_dev, const void *k_dev, const void *v_dev, int32_t n_heads,
                             int32_t n_kv_heads, int32_t head_dim, int32_t n_ctx, int64_t kv_stride, int32_t dtype,
@@ -241,6 +257,9 @@ int64_t kie_flash_decode_scratch_bytes(int32_t n_heads, int32_t n_kv_heads, int3
  * different streams, or from host threads without ordering between them) race with each
  * other and must be serialised by the caller; calls ordered on one stream are safe (each
  * call clears the merge counters it needs before its kernel runs).
+ * The address looked up on a device's first call stays cached for the life of the process:
+ * after cudaDeviceReset on that device it is stale, so a process that resets a device must
+ * not call this entry point on it again. Accepted shapes are those of kie_flash_decode.
  * Returns KIE_ERR_CAPACITY when kie_flash_decode_scratch_bytes(...) for this shape exceeds
  * KIE_FLASH_DECODE_NOALLOC_MAX_BYTES, KIE_ERR_ARG for bad shapes or pointers, KIE_ERR_CUDA
  * if the address lookup or the launch fails.

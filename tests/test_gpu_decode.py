@@ -154,12 +154,25 @@ def test_full_1p9b_parity_short_context(kie):
     assert_reports(reps, m.dtype)
 
 
-def _bench_launch_layer0_check(kie, m, prompt_len, decode_n, positions, modes):
-    """One launch of the bench's configuration; layer-0 K/V at sampled positions must equal the
-    oracle's projection of that position's token (they depend on that token alone)."""
+INJECTED_STEPS = 3
+
+
+def _bench_launch_layer0_check(kie, m, prompt_len, decode_n, positions, modes, prompt_checks=()):
+    """One launch of the bench's configuration, then:
+    * layer-0 K/V at sampled positions equal the oracle's projection of that position's token
+      (they depend on that token alone);
+    * the prefill's K/V of every layer at `prompt_checks` positions, recomputed by the oracle
+      from the engine's cache below each (tests/inject.py);
+    * INJECTED_STEPS more decode steps at the end of the launch's context, each compared with
+      the oracle's full-depth step from the engine's cache: logits, argmax and the appended K/V
+      of every layer. This checks the megakernel's attention (every split of every kv head and
+      their merge) at the context lengths the benchmark runs."""
     from bandwidth_bound_stream_b200 import synth
     from oracle import oracle as orc
-    max_ctx = prompt_len + decode_n
+    from oracle.oracle import OracleModel
+    from tests import inject
+    from tests.parity import assert_reports
+    max_ctx = prompt_len + decode_n + INJECTED_STEPS
     dw = kie.DeviceWeights(m, host_copy=True)
     prompt = synth.prompt(m, prompt_len)
     with kie.Engine(kie.config(m, max_ctx=max_ctx, timeout_ms=20000, idle_ms=50, modes=modes), dw.kie) as eng:
@@ -176,6 +189,13 @@ def _bench_launch_layer0_check(kie, m, prompt_len, decode_n, positions, modes):
         # copy layer 0 of the cache through a torch view of the engine's buffer
         K0 = _device_view(kp, n).cpu().numpy().view(np.uint16).reshape(m.n_kv_heads, max_ctx, m.head_dim)
         V0 = _device_view(vp, n).cpu().numpy().view(np.uint16).reshape(m.n_kv_heads, max_ctx, m.head_dim)
+        o = OracleModel(m, dw.host, max_ctx)
+        if prompt_checks:
+            inject.check_prompt_positions(eng, sid, m, max_ctx, o, prompt, prompt_checks)
+        logits = torch.empty(m.vocab, dtype=torch.float32, device="cuda")
+        reps = inject.injected_decode_steps(eng, sid, m, max_ctx, o, int(gen[-1]), INJECTED_STEPS, logits)
+        assert_reports(reps, m.dtype)
+        assert eng.session_length(sid) == max_ctx
     seq = np.concatenate([prompt, [first], gen[:-1]])
     L0 = dw.host["layers"][0]
     D = m.head_dim
@@ -208,26 +228,30 @@ def _within_one_ulp(got, want, dtype):
 
 def test_full_1p9b_bench_launch_layer0_cache(kie):
     """The benchmark's configuration (1.9B, prompt 1024, one launch of 512 steps), prompt
-    prefilled by the batch-1 kernel."""
+    prefilled by the batch-1 kernel; then full-depth steps at contexts 1536-1538 against the
+    oracle from the engine's cache (about 85 positions per attention split)."""
     from bandwidth_bound_stream_b200 import synth
     _bench_launch_layer0_check(kie, synth.DENSE_1P9B, 1024, 512, (0, 1, 777, 1023, 1024, 1300, 1535),
-                               kie.KIE_MODE_BATCH1)
+                               kie.KIE_MODE_BATCH1, prompt_checks=(700, 1023))
 
 
 def test_full_8b_bench_launch_layer0_cache(kie):
     """The 8B (Llama-3-8B shape, bf16, theta 5e5) configuration: prompt 4096 prefilled in tick-kernel
-    chunks, one launch of 256 decode steps."""
+    chunks, one launch of 256 decode steps; prefill K/V of every layer at two prompt positions and
+    full-depth steps at contexts 4352-4354, against the oracle from the engine's cache."""
     from bandwidth_bound_stream_b200 import synth
     _bench_launch_layer0_check(kie, synth.DENSE_8B, 4096, 256, (0, 63, 64, 2049, 4095, 4096, 4351),
-                               kie.KIE_MODE_BATCH1 | kie.KIE_MODE_TICK)
+                               kie.KIE_MODE_BATCH1 | kie.KIE_MODE_TICK, prompt_checks=(1500, 4095))
 
 
 def test_full_1p9b_32k_bench_launch_layer0_cache(kie):
     """The long-context configuration: 1.9B, prompt 32768 prefilled in tick-kernel chunks, one
-    launch of 256 decode steps (attention over a 32K cache)."""
+    launch of 256 decode steps (attention over a 32K cache); prefill K/V of every layer at two
+    prompt positions and full-depth steps at contexts 33024-33026 (about 1,835 positions per
+    attention split), against the oracle from the engine's cache."""
     from bandwidth_bound_stream_b200 import synth
     _bench_launch_layer0_check(kie, synth.DENSE_1P9B, 32768, 256, (0, 4095, 16384, 32703, 32767, 32768, 33023),
-                               kie.KIE_MODE_BATCH1 | kie.KIE_MODE_TICK)
+                               kie.KIE_MODE_BATCH1 | kie.KIE_MODE_TICK, prompt_checks=(20000, 32767))
 
 
 def _device_view(ptr, n):
