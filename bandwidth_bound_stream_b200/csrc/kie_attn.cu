@@ -62,7 +62,8 @@ extern "C" kie_status kie_flash_decode(const float *q_dev, const void *k_dev, co
     A.bpack = nullptr;
     A.brow = 0;
     A.gout = -1;
-    A.cnt_target = 0;  // the last split merges
+    A.cnt_target = 0;
+    A.oslice = nullptr;  // the last split merges
     A.timeout_ns = 0;
     A.err = nullptr;
     A.D = head_dim;

@@ -36,7 +36,10 @@ struct AttnArgs {
     int gout;                // kv head whose output columns a unit writes; -1: unit / nsplit
     uint32_t cnt_target;     // 0: the last split merges. Else every split merges a slice of its kv
                              // head's output once cnt[kv head] reaches this value (the counters
-                             // then only count up; fp32 output A.o only)
+                             // then only count up): elements [8 q0, 8 q1) of the kv head's Gt * D
+                             // outputs, q0 = s * (Gt * D / 8) / nsplit (8-element groups), written
+                             // to oslice[0 .. 8 (q1 - q0)) (shared memory)
+    float *oslice;
     long long timeout_ns;    // bound of that wait; on expiry err gets an error code
     unsigned *err;
     int D, Hkv, nsplit, ctx;
@@ -306,8 +309,10 @@ __device__ __forceinline__ void attn_tail(const AttnArgs &A, AttnSmem &S, int un
         }
         named_bar_sync(1, ATTN_THREADS);
         if (!last_pass) return;
-        const int s = unit % nsplit, E = Gt * D;
-        const int e0 = (int)((long long)s * E / nsplit), e1 = (int)((long long)(s + 1) * E / nsplit), ne = e1 - e0;
+        const int s = unit % nsplit, E = Gt * D, nq = E / 8;
+        const int e0 = 8 * (int)((long long)s * nq / nsplit), e1 = 8 * (int)((long long)(s + 1) * nq / nsplit);
+        const int ne = e1 - e0;
+        if (ne == 0) return;  // more splits than 8-element groups: this split owns no slice
         const float *pg = A.part + (size_t)g * nsplit * Gt * (D + 2);
         float *ek = &S.wacc[0][0];   // [nsplit][Gt] max, then weights
         float *lk = ek + nsplit * Gt;  // [nsplit][Gt] sums
@@ -339,7 +344,7 @@ __device__ __forceinline__ void attn_tail(const AttnArgs &A, AttnSmem &S, int un
             const int ee = e0 + j, jj = ee / D;
             float num = 0.f;
             for (int k = 0; k < nsplit; k++) num = fmaf(ek[k * Gt + jj], ak[k * ne + j], num);
-            A.o[(size_t)(go * Gt + jj) * D + ee % D] = num / S.red[jj];
+            A.oslice[j] = num / S.red[jj];
         }
         named_bar_sync(1, ATTN_THREADS);
         return;

@@ -8,34 +8,38 @@
 //
 //  * Warp 16 (the producer) walks this CTA's fixed weight schedule for the whole command
 //    (all layers, all tokens) and copies it, chunk by chunk, into a 3 x 64 KB shared-memory
-//    ring with 1-D bulk async copies (TMA). The ring holds 192 KB; while the consumers sit
-//    in attention (which reads no weights) it fills and HBM would idle, so the producer also
-//    keeps the `pf_chunks` chunks after the one it copies requested into L2 (an L2 lead of a
-//    fixed size). The schedule is contiguous in HBM because the weights were repacked at
-//    engine creation in exactly this order, so each SM streams one disjoint span (the
-//    aligned, topology-aware access of the same section). The producer never waits on grid
-//    barriers.
-//  * Warps 0-15 (consumers) run the phases of each layer on the staged chunks:
-//      QKV  : RMSNorm -> [Wq;Wk;Wv] rows -> RoPE -> q, and the K/V append to the cache
-//      ATTN : split-K single-query attention over the cache, last split merges (LSE)
-//      O    : x += Wo o
-//      GU   : RMSNorm -> gate/up rows -> u = silu(gate) * up
-//      DOWN : x += Wd u
+//    ring with 1-D bulk async copies (TMA). The schedule is contiguous in HBM because the
+//    weights were repacked at engine creation in exactly this order, so each SM streams one
+//    disjoint span (the aligned, topology-aware access of the same section). The producer
+//    never waits on grid barriers.
+//  * Warps 0-15 (consumers) run each layer as three phases, each ended by a grid barrier:
+//      A  QKV : RMSNorm -> [Wq;Wk;Wv] rows -> RoPE -> q, and the K/V append to the cache
+//      B  ATTN: split-K single-query attention; each split merges its slice of its kv head's
+//               output (log-sum-exp), then folds it through its own columns of Wo into the
+//               residual: x += Wo[:, slice] o[slice]
+//      C  MLP : RMSNorm -> gate/up rows -> u = silu(gate) * up for this CTA's pairs, then the
+//               same pairs' columns of Wd: x += Wd[:, pairs] u[pairs]
 //    then, per token, HEAD: final RMSNorm -> LM-head rows -> block argmax -> grid argmax.
-//    Phases are separated by a grid-wide barrier with a time limit.
+//    The two folds add into the residual with fp32 atomics, so no CTA has to wait for all of
+//    o or u: that removes two of the five grid barriers a row-partitioned O and down
+//    projection would need, and the gate/up and down weights stream back to back. In phase
+//    C a CTA may add into x only after every CTA has read x for its RMSNorm: a split barrier
+//    (arrive after the read, wait before the add) that is long complete when it is checked.
 //
-// GEMV mapping: a ring chunk holds 2*CR whole rows of length K. The 16 consumer warps form
-// two groups of 8; group g takes rows [g*CR, (g+1)*CR) of every chunk. In a group, warp w
-// owns the column slice
-// [w*K/8, (w+1)*K/8); lane l owns 16-byte vectors l, l+32, ... of that slice, so a lane's
-// slice of the input vector sits in registers for the whole phase and each staged weight
-// byte is read from shared memory exactly once. Row sums are reduced across the warp with
-// a shuffle butterfly over the CR rows; the 8 column-slice partials of a row are added in
-// a fixed order by the phase epilogue, so results are bit-reproducible.
+// GEMV mapping (QKV, gate/up, head): a ring chunk holds 2*CR whole rows of length K. The 16
+// consumer warps form two groups of 8; group g takes rows [g*CR, (g+1)*CR) of every chunk.
+// In a group, warp w owns the column slice [w*K/8, (w+1)*K/8); lane l owns 16-byte vectors
+// l, l+32, ... of that slice, so a lane's slice of the input vector sits in registers for
+// the whole phase and each staged weight byte is read from shared memory exactly once. Row
+// sums are reduced across the warp with a shuffle butterfly over the CR rows; the 8
+// column-slice partials of a row are added in a fixed order by the phase epilogue.
 //
-// RMSNorm: the residual rows are owned by the CTA that updates them (O and DOWN phases);
-// each CTA publishes the sum of squares of its rows when it arrives at the next grid
-// barrier, and every reader adds the per-CTA sums in CTA order.
+// Fold mapping (O and down): the CTA's columns arrive as [8-column group][d rows][8]
+// (16 bytes per row and group); thread t owns rows t, t + 512, ... for the whole fold and
+// accumulates them over its column groups, then adds them into x.
+//
+// RMSNorm: every CTA reads all of x for a normed phase, so each computes the sum of squares
+// itself (one CTA-wide reduction) instead of publishing partial sums.
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
@@ -53,10 +57,9 @@ struct __align__(16) B1Shared {
         float wpart[WPART_FLOATS];  // column-slice partials of this phase's row sums
         AttnSmem at;
     };
+    float fold_in[KIE_FOLD_MAX];  // the current fold's inputs: this CTA's slice of o, or of u
     float red[64];
     int redi[32];
-    float ssqw[KIE_CONS_WARPS];
-    float xown[KIE_XOWN_MAX];  // this CTA's residual rows (O and DOWN phases own the same rows)
     float2 rope_s[KIE_DMAX / 2];  // rotation of the current position, loaded at the start of QKV
     uint64_t full[KIE_NSLOT];
     uint64_t empty[KIE_NSLOT];
@@ -86,7 +89,6 @@ __device__ __forceinline__ void copy_words_cg(KieCmd *dst, const KieCmd *src) {
 // different rows of a chunk; 16: all warps share each row), 16-byte vectors per lane, and
 // rows per group in one ring chunk. K <= 14336.
 __host__ __device__ inline int col_slices(int K) { return K <= 8192 ? 8 : 16; }
-__host__ __device__ inline int vec_per_lane(int K) { return K <= 2048 ? 1 : K <= 4096 ? 2 : 4; }
 __host__ __device__ inline int rows_per_group(int K) { return K <= 2048 ? 8 : K <= 4096 ? 4 : 2; }
 
 __device__ __forceinline__ void trace_mark(const KieParams &P, int t, int ev, float after = 0.f) {
@@ -96,20 +98,13 @@ __device__ __forceinline__ void trace_mark(const KieParams &P, int t, int ev, fl
 
 // --------------------------------------------------------------- grid barrier
 
-// All consumer threads call this. Returns false if this CTA is aborting. With
-// publish_ssq, the sum of squares of the residual rows this CTA just wrote (per-warp
-// partials in S.ssqw) is published before arriving.
+// All consumer threads call this. Returns false if this CTA is aborting.
 __device__ bool grid_barrier(const KieParams &P, B1Shared &S, unsigned long long &epoch, long long timeout_ns,
-                             unsigned where, bool publish_ssq = false) {
+                             unsigned where) {
     named_bar_sync(1, KIE_CONS_THREADS);
     if (threadIdx.x == 0) {
         int ok = !S.abort;
         if (ok) {
-            if (publish_ssq) {
-                float v = 0.f;
-                for (int k = 0; k < KIE_CONS_WARPS; k++) v += S.ssqw[k];
-                P.ssq[blockIdx.x] = v;
-            }
             epoch += 1;
             const unsigned long long target = epoch * (unsigned long long)P.nblk;
             // release: this CTA's writes (ordered before by the named barrier) become visible
@@ -137,10 +132,41 @@ __device__ bool grid_barrier(const KieParams &P, B1Shared &S, unsigned long long
     return S.gb_ok != 0;
 }
 
+// The split barrier of phase C. Thread 0 announces that this CTA has read the residual (its
+// earlier reads are ordered before the release)...
+__device__ __forceinline__ void residual_read_arrive(const KieParams &P, const B1Shared &S) {
+    if (threadIdx.x == 0 && !S.abort) red_release_gpu_add_u64(P.rd, 1ull);
+}
+
+// ... and before the first add into it waits until every CTA has done so (`epoch`: this
+// CTA's arrivals so far, including the current one). All consumer threads call this.
+__device__ void residual_read_wait(const KieParams &P, B1Shared &S, unsigned long long epoch) {
+    if (threadIdx.x == 0 && !S.abort) {
+        const unsigned long long target = epoch * (unsigned long long)P.nblk;
+        const uint64_t t0 = globaltimer();
+        unsigned spins = 0;
+        while (ld_acquire_gpu_u64(P.rd) < target) {
+            if ((++spins & 255u) == 0) {
+                if (ld_volatile_u32(P.err) != 0u) {
+                    S.abort = 1;
+                    break;
+                }
+                if ((long long)(globaltimer() - t0) > P.timeout_ns) {
+                    set_error(P.err, DERR_BARRIER_TIMEOUT, 7);
+                    S.abort = 1;
+                    break;
+                }
+            }
+        }
+    }
+    named_bar_sync(1, KIE_CONS_THREADS);
+}
+
 // --------------------------------------------------------------- the weight schedule
 
-// Walks this CTA's chunks in stream order: per token, every layer's QKV, O, GU, DOWN rows,
-// then (when the token needs logits) the LM-head rows. A token restarts at the segment base.
+// Walks this CTA's chunks in stream order: per token, every layer's QKV rows, O-fold column
+// groups, gate/up rows and down-fold column groups, then (when the token needs logits) the
+// LM-head rows. A token restarts at the segment base.
 struct ChunkIter {
     const uint8_t *seg, *g;
     int t, l, ph, r;
@@ -155,15 +181,18 @@ __device__ __forceinline__ void chunk_begin(ChunkIter &it, const uint8_t *seg) {
     it.r = 0;
 }
 
-// Next chunk (address, bytes); false when the command's schedule is exhausted.
+__device__ __forceinline__ bool is_fold(int ph) { return ph == PH_OF || ph == PH_DF; }
+
+// Next chunk (address, bytes); false when the command's schedule is exhausted. A GEMV chunk
+// is cr rows of K elements; a fold chunk is cr column groups of d rows x 16 bytes.
 __device__ bool chunk_next(const KieParams &P, const B1Shared &S, const KieCmd &cmd, ChunkIter &it,
                            const uint8_t *&addr, uint32_t &bytes) {
     for (;;) {
         if (it.t >= cmd.n) return false;
-        const int rows = S.row1[it.ph] - S.row0[it.ph];
-        if (it.r < rows) {
-            const int nr = min(P.cr[it.ph], rows - it.r);
-            bytes = (uint32_t)(nr * P.K[it.ph] * 2);
+        const int n = S.row1[it.ph] - S.row0[it.ph];
+        if (it.r < n) {
+            const int nr = min(P.cr[it.ph], n - it.r);
+            bytes = (uint32_t)(is_fold(it.ph) ? nr * P.d * 16 : nr * P.K[it.ph] * 2);
             addr = it.g;
             it.g += bytes;
             it.r += nr;
@@ -176,7 +205,7 @@ __device__ bool chunk_next(const KieParams &P, const B1Shared &S, const KieCmd &
             it.l = 0;
             it.ph = 0;
             it.g = it.seg;
-        } else if (it.ph == PH_DOWN) {
+        } else if (it.ph == PH_DF) {
             if (++it.l == P.L) {
                 const bool head = (cmd.op != OP_PREFILL) || (it.t == cmd.n - 1);
                 if (head) {
@@ -200,28 +229,13 @@ __device__ bool chunk_next(const KieParams &P, const B1Shared &S, const KieCmd &
 
 __device__ void produce(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint8_t *ring, const KieCmd &cmd) {
     const uint8_t *seg = P.wpack + P.seg_off[blockIdx.x];
-    ChunkIter fetch, lead;
+    ChunkIter fetch;
     chunk_begin(fetch, seg);
-    chunk_begin(lead, seg);
     const uint8_t *a;
     uint32_t b;
     unsigned long long waited = 0;
     int tok = 0;
-    // The L2 lead: the pf_chunks chunks after the one being copied into the ring are requested
-    // into L2 as well, so HBM keeps streaming while the ring is full and the consumers sit in
-    // latency-bound work (attention, barriers); the ring then refills from L2.
-    int ahead = 0;  // chunks the lead iterator has passed beyond the fetch iterator
-    bool lead_live = P.pf_chunks > 0 && chunk_next(P, S, cmd, lead, a, b);  // skip chunk 0 (fetched now)
     while (chunk_next(P, S, cmd, fetch, a, b)) {
-        if (ahead > 0) ahead--;
-        while (lead_live && ahead < P.pf_chunks) {
-            const uint8_t *la;
-            uint32_t lb;
-            lead_live = chunk_next(P, S, cmd, lead, la, lb);
-            if (!lead_live) break;
-            bulk_prefetch_l2(la, lb);
-            ahead++;
-        }
         if (fetch.t != tok) {
             if (P.trace && tok < P.trace_tokens)
                 P.trace[((size_t)blockIdx.x * P.trace_tokens + tok) * P.trace_events + P.trace_events - 1] = waited;
@@ -254,43 +268,25 @@ __device__ void produce(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint
 
 // --------------------------------------------------------------- consumer: GEMV phases
 
-// element j of a phase's input vector (before the norm)
-template <int DT>
-__device__ __forceinline__ float phase_input(const KieParams &P, int ph, bool from_emb, int tok, int j) {
-    if (ph == PH_O) return __ldcg(P.o + j);
-    if (ph == PH_DOWN) return __ldcg(P.u + j);
-    if (from_emb) return cvt1<DT>(P.emb[(size_t)tok * P.d + j]);
-    return __ldcg(P.x + j);
-}
-
-// 1/sqrt(mean(x^2) + eps) of the residual, from the per-CTA partial sums (every warp
-// computes the same value in the same order).
-__device__ __forceinline__ float rstd_from_partials(const KieParams &P) {
-    const int lane = threadIdx.x & 31;
-    float v = 0.f;
-    for (int c = lane; c < P.nblk; c += 32) v += __ldcg(P.ssq + c);
-    v = warp_sum(v);
-    return rsqrtf(v / (float)P.d + P.eps);
-}
-
-// Runs one GEMV phase over this CTA's rows; row partials land in S.wpart (see rowsum).
+// Runs one GEMV phase (QKV, gate/up or head) over this CTA's rows: the RMSNorm of its input
+// (the embedding row at layer 0, else the residual x), then the rows; row partials land in
+// S.wpart (see rowsum).
 template <int DT, int NV, int CR, int CS>
 __device__ void gemv_phase(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring, int ph, int l,
                            int tok, int pos, int t) {
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int K = P.K[ph];
     const int rows = S.row1[ph] - S.row0[ph];
-    const bool norm = (ph == PH_QKV || ph == PH_GU || ph == PH_HEAD);
     const bool from_emb = (ph == PH_QKV && l == 0);
 
     // the QKV epilogue needs this position's rotation: fetch it now, under the row work
     if (ph == PH_QKV && tid < (P.D >> 1)) S.rope_s[tid] = P.rope[(size_t)pos * (P.D >> 1) + tid];
-    // raw inputs first (one round trip together with the norm partials below)
     const uint16_t *gain = P.gains + (size_t)(ph == PH_HEAD ? 2 * P.L : 2 * l + (ph == PH_GU ? 1 : 0)) * P.d;
     constexpr int GROUPS = KIE_CONS_WARPS / CS;  // warp groups, each taking CR rows of a chunk
     const int kslice = K / CS;  // columns per warp
     const int nvec = kslice >> 3;  // 16-byte vectors per warp slice
     float h[NV][8];
+    float ss = 0.f;
 #pragma unroll
     for (int i = 0; i < NV; i++) {
         const int v = lane + 32 * i;
@@ -301,44 +297,34 @@ __device__ void gemv_phase(const KieParams &P, B1Shared &S, uint32_t &ring_it, c
             if (from_emb) {
                 cvt8<DT>(__ldg(reinterpret_cast<const uint4 *>(P.emb + (size_t)tok * P.d + col0)), h[i]);
             } else {
-                const float *src = ph == PH_O ? P.o : ph == PH_DOWN ? P.u : P.x;
-                const float4 a = __ldcg(reinterpret_cast<const float4 *>(src + col0));
-                const float4 b = __ldcg(reinterpret_cast<const float4 *>(src + col0 + 4));
+                const float4 a = __ldcg(reinterpret_cast<const float4 *>(P.x + col0));
+                const float4 b = __ldcg(reinterpret_cast<const float4 *>(P.x + col0 + 4));
                 h[i][0] = a.x; h[i][1] = a.y; h[i][2] = a.z; h[i][3] = a.w;
                 h[i][4] = b.x; h[i][5] = b.y; h[i][6] = b.z; h[i][7] = b.w;
             }
-            if (norm) {
-                float g[8];
-                cvt8<DT>(__ldg(reinterpret_cast<const uint4 *>(gain + col0)), g);
+            float g[8];
+            cvt8<DT>(__ldg(reinterpret_cast<const uint4 *>(gain + col0)), g);
 #pragma unroll
-                for (int e = 0; e < 8; e++) h[i][e] *= g[e];
+            for (int e = 0; e < 8; e++) {
+                ss = fmaf(h[i][e], h[i][e], ss);
+                h[i][e] *= g[e];
             }
         }
     }
-    if (norm) {
-        float rstd;
-        if (from_emb) {
-            float ss = 0.f;
-            for (int j = tid; j < P.d; j += KIE_CONS_THREADS) {
-                const float v = cvt1<DT>(P.emb[(size_t)tok * P.d + j]);
-                ss += v * v;
-            }
-            ss = warp_sum(ss);
-            if (lane == 0) S.red[w] = ss;
-            named_bar_sync(1, KIE_CONS_THREADS);
-            float v = lane < KIE_CONS_WARPS ? S.red[lane] : 0.f;
-            v = warp_sum(v);
-            rstd = rsqrtf(v / (float)P.d + P.eps);
-            named_bar_sync(1, KIE_CONS_THREADS);
-        } else {
-            rstd = rstd_from_partials(P);
-        }
+    // 1/sqrt(mean(x^2) + eps) of the whole input: the CS warps of the first group cover every
+    // column once; their sums are added in warp order, so every thread gets the same value
+    ss = warp_sum(ss);
+    if (lane == 0 && w < CS) S.red[w] = ss;
+    named_bar_sync(1, KIE_CONS_THREADS);
+    float tot = 0.f;
 #pragma unroll
-        for (int i = 0; i < NV; i++)
+    for (int k = 0; k < CS; k++) tot += S.red[k];
+    const float rstd = rsqrtf(tot / (float)P.d + P.eps);
 #pragma unroll
-            for (int e = 0; e < 8; e++) h[i][e] *= rstd;
-    }
-    if (l < P.L) trace_mark(P, t, 1 + 16 * l + 11 + (ph == PH_QKV ? 0 : ph == PH_O ? 1 : ph == PH_GU ? 2 : 3), h[0][0]);
+    for (int i = 0; i < NV; i++)
+#pragma unroll
+        for (int e = 0; e < 8; e++) h[i][e] *= rstd;
+    if (l < P.L) trace_mark(P, t, 1 + 16 * l + (ph == PH_QKV ? 11 : 12), h[0][0]);
 
     unsigned long long waited = 0;
     const int grp = w / CS, ws = w % CS;
@@ -404,9 +390,63 @@ __device__ __forceinline__ void gemv_dispatch(const KieParams &P, B1Shared &S, u
                               int tok, int pos, int t) {
     const int K = P.K[ph];
     if (K <= 2048) gemv_phase<DT, 1, 8, 8>(P, S, ring_it, ring, ph, l, tok, pos, t);
-    else if (K <= 4096) gemv_phase<DT, 2, 4, 8>(P, S, ring_it, ring, ph, l, tok, pos, t);
-    else if (K <= 8192) gemv_phase<DT, 4, 2, 8>(P, S, ring_it, ring, ph, l, tok, pos, t);
-    else gemv_phase<DT, 4, 2, 16>(P, S, ring_it, ring, ph, l, tok, pos, t);
+    else gemv_phase<DT, 2, 4, 8>(P, S, ring_it, ring, ph, l, tok, pos, t);  // K <= 4096
+}
+
+// --------------------------------------------------------------- consumer: folds
+
+// One fold (O or down): this CTA's 8-column groups of W arrive as [group][d rows][8], and
+// S.fold_in holds 8 inputs per group. Thread t accumulates rows t + 512 j over all groups.
+template <int DT, int RPT>
+__device__ void fold_rows(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring, int ph,
+                          float (&acc)[RPT]) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int d = P.d, ng = S.row1[ph] - S.row0[ph], cpc = P.cr[ph];
+#pragma unroll
+    for (int j = 0; j < RPT; j++) acc[j] = 0.f;
+    named_bar_sync(1, KIE_CONS_THREADS);  // S.fold_in was written by other warps of this CTA
+    for (int g0 = 0; g0 < ng; g0 += cpc) {
+        const int n = min(cpc, ng - g0);
+        const uint32_t slot = ring_it % KIE_NSLOT, par = (ring_it / KIE_NSLOT) & 1u;
+        ring_it++;
+        bool have = !S.abort && mbar_try_wait(&S.full[slot], par);
+        if (!have && !S.abort) have = mbar_wait(&S.full[slot], par, P.timeout_ns, &S.abort);
+        have = __all_sync(0xffffffffu, have);
+        if (!have) {
+            if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, (unsigned)ph);
+            S.abort = 1;
+            continue;
+        }
+        const uint8_t *base = ring + (size_t)slot * KIE_SLOT_BYTES;
+        for (int gi = 0; gi < n; gi++) {
+            const float4 a = *reinterpret_cast<const float4 *>(&S.fold_in[(g0 + gi) * 8]);
+            const float4 b = *reinterpret_cast<const float4 *>(&S.fold_in[(g0 + gi) * 8 + 4]);
+            const float in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int j = 0; j < RPT; j++) {
+                const int r = tid + KIE_CONS_THREADS * j;
+                if (r < d) {
+                    float f[8];
+                    cvt8<DT>(*reinterpret_cast<const uint4 *>(base + ((size_t)gi * d + r) * 16), f);
+#pragma unroll
+                    for (int e = 0; e < 8; e++) acc[j] = fmaf(f[e], in[e], acc[j]);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.empty[slot]);
+    }
+}
+
+// x[r] += acc for this thread's rows (fp32 atomics: the folds of all CTAs meet in x)
+template <int RPT>
+__device__ __forceinline__ void fold_commit(const KieParams &P, const B1Shared &S, const float (&acc)[RPT], int ph) {
+    if (S.abort || S.row1[ph] == S.row0[ph]) return;
+#pragma unroll
+    for (int j = 0; j < RPT; j++) {
+        const int r = threadIdx.x + KIE_CONS_THREADS * j;
+        if (r < P.d) atomicAdd(P.x + r, acc[j]);
+    }
 }
 
 // --------------------------------------------------------------- consumer: epilogues
@@ -444,57 +484,39 @@ __device__ void epilogue_qkv(const KieParams &P, B1Shared &S, int l, int sid, in
             vp[i + half] = store1<DT>(b);
         }
     }
-    if (l == 0) {  // the residual starts as the embedding row (rows this CTA owns in the O phase)
-        for (int r = S.row0[PH_O] + threadIdx.x; r < S.row1[PH_O]; r += KIE_CONS_THREADS) {
-            const float v = cvt1<DT>(P.emb[(size_t)tok * P.d + r]);
-            S.xown[r - S.row0[PH_O]] = v;
-            P.x[r] = v;
-        }
+    if (l == 0) {  // the residual starts as the embedding row (each CTA writes a 1/nblk share)
+        const int r0 = (int)((long long)blockIdx.x * P.d / P.nblk), r1 = (int)((long long)(blockIdx.x + 1) * P.d / P.nblk);
+        for (int r = r0 + threadIdx.x; r < r1; r += KIE_CONS_THREADS) P.x[r] = cvt1<DT>(P.emb[(size_t)tok * P.d + r]);
+        attention_prefetch(P, l, sid, pos);
     }
-    if (l == 0) attention_prefetch(P, l, sid, pos);
 }
 
-// The cache rows this CTA's attention units will read in layer l start moving into L2
+// The cache rows this CTA's attention unit will read in layer l start moving into L2
 // (older positions are final; L2 stays coherent for the one written in this token).
 __device__ __forceinline__ void attention_prefetch(const KieParams &P, int l, int sid, int pos) {
     const int D = P.D;
     const size_t sess = (size_t)sid * P.sess_stride;
-    {
-        const int ctx = pos + 1;
-        for (int unit = blockIdx.x; unit < P.Hkv * P.splits; unit += P.nblk) {
-            const int g = unit / P.splits, s = unit % P.splits;
-            const long long p0 = (long long)s * ctx / P.splits, p1 = (long long)(s + 1) * ctx / P.splits;
-            const size_t off = sess + ((size_t)(l * P.Hkv + g) * P.max_ctx + p0) * D;
-            const int lines = (int)(((p1 - p0) * D * 2 + 127) / 128);
-            for (int j = threadIdx.x; j < 2 * lines; j += KIE_CONS_THREADS) {
-                const uint16_t *base = (j < lines ? P.kcache : P.vcache) + off;
-                prefetch_l2(reinterpret_cast<const uint8_t *>(base) + (size_t)(j % lines) * 128);
-            }
+    const int ctx = pos + 1;
+    for (int unit = blockIdx.x; unit < P.Hkv * P.splits; unit += P.nblk) {
+        const int g = unit / P.splits, s = unit % P.splits;
+        const long long p0 = (long long)s * ctx / P.splits, p1 = (long long)(s + 1) * ctx / P.splits;
+        const size_t off = sess + ((size_t)(l * P.Hkv + g) * P.max_ctx + p0) * D;
+        const int lines = (int)(((p1 - p0) * D * 2 + 127) / 128);
+        for (int j = threadIdx.x; j < 2 * lines; j += KIE_CONS_THREADS) {
+            const uint16_t *base = (j < lines ? P.kcache : P.vcache) + off;
+            prefetch_l2(reinterpret_cast<const uint8_t *>(base) + (size_t)(j % lines) * 128);
         }
     }
 }
 
-// x += row sums on the rows this CTA owns; per-warp sums of squares of the new rows
-__device__ void epilogue_residual(const KieParams &P, B1Shared &S, int ph) {
-    const int rbeg = S.row0[ph], n = S.row1[ph] - rbeg;
-    float ss = 0.f;
-    for (int r = threadIdx.x; r < n; r += KIE_CONS_THREADS) {
-        const float v = S.xown[r] + rowsum(S, r, col_slices(P.K[ph]));
-        S.xown[r] = v;
-        P.x[rbeg + r] = v;
-        ss += v * v;
-    }
-    ss = warp_sum(ss);
-    if ((threadIdx.x & 31) == 0) S.ssqw[threadIdx.x >> 5] = ss;
-}
-
+// u = silu(gate) * up for this CTA's pairs, into the down fold's inputs
 __device__ void epilogue_gu(const KieParams &P, B1Shared &S, int l, int sid, int pos) {
     if (l + 1 < P.L) attention_prefetch(P, l + 1, sid, pos);
-    const int rbeg = S.row0[PH_GU], npair = (S.row1[PH_GU] - rbeg) >> 1;
+    const int npair = (S.row1[PH_GU] - S.row0[PH_GU]) >> 1;
+    const int cs = col_slices(P.K[PH_GU]);
     for (int p = threadIdx.x; p < npair; p += KIE_CONS_THREADS) {
-        const int cs = col_slices(P.K[PH_GU]);
         const float g = rowsum(S, 2 * p, cs), up = rowsum(S, 2 * p + 1, cs);
-        P.u[(rbeg >> 1) + p] = g / (1.f + expf(-g)) * up;
+        S.fold_in[p] = g / (1.f + expf(-g)) * up;
     }
 }
 
@@ -556,9 +578,8 @@ __device__ int final_argmax(const KieParams &P) {
 // --------------------------------------------------------------- consumer: attention
 
 // The QKV -> attention barrier, then this CTA's attention unit (at most one unit per CTA:
-// splits = nblk / Hkv); the query heads of a kv head are taken GC at a time. (Loading the
-// unit's first K/V batch before the barrier was measured slower: the barrier's release then
-// waits for those loads.)
+// splits = nblk / Hkv); the query heads of a kv head are taken GC at a time. Each split merges
+// its slice of the kv head's output into S.fold_in (the O fold's inputs).
 template <int DT, int GC>
 __device__ void attention_step(const KieParams &P, B1Shared &S, int l, int sid, int pos, unsigned long long &epoch,
                                int t, int e, uint32_t &att_use) {
@@ -569,13 +590,14 @@ __device__ void attention_step(const KieParams &P, B1Shared &S, int l, int sid, 
     A.head_stride = (long long)P.max_ctx * P.D;
     A.part = P.part;
     A.cnt = P.cnt;
-    A.o = P.o;
+    A.o = nullptr;
     A.bpack = nullptr;
     A.brow = 0;
     A.gout = -1;
     // every split merges a slice once all splits of its kv head have published; each split
     // adds one per pass over the query heads, and the counters only count up within a launch
     A.cnt_target = (att_use + 1u) * (uint32_t)P.splits * (uint32_t)((P.G + GC - 1) / GC);
+    A.oslice = S.fold_in;
     A.timeout_ns = P.timeout_ns;
     A.err = P.err;
     att_use++;
@@ -591,14 +613,49 @@ __device__ void attention_step(const KieParams &P, B1Shared &S, int l, int sid, 
     if (have && !S.abort) {
         for (int hoff = 0; hoff < P.G; hoff += GC) attn_unit<DT, GC, KIE_CONS_WARPS>(A, S.at, unit, P.G, hoff);
     }
-    trace_mark(P, t, e + 3);
+}
+
+// the two folds of a layer and the down fold's split barrier, by rows per thread
+template <int DT, int RPT>
+__device__ __forceinline__ void o_fold(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring) {
+    float acc[RPT];
+    fold_rows<DT, RPT>(P, S, ring_it, ring, PH_OF, acc);
+    fold_commit<RPT>(P, S, acc, PH_OF);
+}
+
+template <int DT, int RPT>
+__device__ __forceinline__ void down_fold(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring,
+                                          unsigned long long rd_epoch, int t, int e) {
+    float acc[RPT];
+    fold_rows<DT, RPT>(P, S, ring_it, ring, PH_DF, acc);
+    residual_read_wait(P, S, rd_epoch);  // every CTA has read x for its gate/up norm
+    trace_mark(P, t, e + 10);
+    fold_commit<RPT>(P, S, acc, PH_DF);
+}
+
+// rows per thread of a fold (d <= 4096): 1, 2, 4 or 8
+template <int DT>
+__device__ __forceinline__ void o_fold_any(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring) {
+    if (P.d <= 512) o_fold<DT, 1>(P, S, ring_it, ring);
+    else if (P.d <= 1024) o_fold<DT, 2>(P, S, ring_it, ring);
+    else if (P.d <= 2048) o_fold<DT, 4>(P, S, ring_it, ring);
+    else o_fold<DT, 8>(P, S, ring_it, ring);
+}
+
+template <int DT>
+__device__ __forceinline__ void down_fold_any(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring,
+                                              unsigned long long rd_epoch, int t, int e) {
+    if (P.d <= 512) down_fold<DT, 1>(P, S, ring_it, ring, rd_epoch, t, e);
+    else if (P.d <= 1024) down_fold<DT, 2>(P, S, ring_it, ring, rd_epoch, t, e);
+    else if (P.d <= 2048) down_fold<DT, 4>(P, S, ring_it, ring, rd_epoch, t, e);
+    else down_fold<DT, 8>(P, S, ring_it, ring, rd_epoch, t, e);
 }
 
 // --------------------------------------------------------------- consumer: one command
 
 template <int DT>
 __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring, const KieCmd &cmd,
-                        unsigned long long &epoch, uint32_t &att_use) {
+                        unsigned long long &epoch, unsigned long long &rd_epoch, uint32_t &att_use) {
     int tok = cmd.in_tok;
     if (cmd.op == OP_DECODE && cmd.tok_dev) tok = __ldcg(cmd.tok_dev);
     const int L = P.L;
@@ -617,30 +674,31 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, cons
         const bool head = (cmd.op != OP_PREFILL) || (t == cmd.n - 1);
         for (int l = 0; l < L; l++) {
             const int e = 1 + 16 * l;
+            // A: QKV
             gemv_dispatch<DT>(P, S, ring_it, ring, PH_QKV, l, tok, pos, t);
             trace_mark(P, t, e);
             epilogue_qkv<DT>(P, S, l, cmd.sid, pos, tok);
             trace_mark(P, t, e + 1);
-            attention_step<DT, 2>(P, S, l, cmd.sid, pos, epoch, t, e, att_use);  // also serves G == 1 (one idle head slot)
+            // B: attention, then the O fold
+            attention_step<DT, 2>(P, S, l, cmd.sid, pos, epoch, t, e, att_use);  // also serves G == 1
             if (P.trace && t < P.trace_tokens && threadIdx.x == 0)  // end of this CTA's positions (0: no unit)
                 P.trace[((size_t)blockIdx.x * P.trace_tokens + t) * P.trace_events + e + 15] = S.at.t_unit;
-            grid_barrier(P, S, epoch, P.timeout_ns, 2);
+            trace_mark(P, t, e + 3);
+            o_fold_any<DT>(P, S, ring_it, ring);
             trace_mark(P, t, e + 4);
-            gemv_dispatch<DT>(P, S, ring_it, ring, PH_O, l, tok, pos, t);
-            epilogue_residual(P, S, PH_O);
+            grid_barrier(P, S, epoch, P.timeout_ns, 2);
             trace_mark(P, t, e + 5);
-            grid_barrier(P, S, epoch, P.timeout_ns, 3, true);
-            trace_mark(P, t, e + 6);
+            // C: gate/up, then the down fold
             gemv_dispatch<DT>(P, S, ring_it, ring, PH_GU, l, tok, pos, t);
+            residual_read_arrive(P, S);  // this CTA's reads of x are done
+            rd_epoch++;
+            trace_mark(P, t, e + 6);
             epilogue_gu(P, S, l, cmd.sid, pos);
             trace_mark(P, t, e + 7);
-            grid_barrier(P, S, epoch, P.timeout_ns, 4);
+            down_fold_any<DT>(P, S, ring_it, ring, rd_epoch, t, e);
             trace_mark(P, t, e + 8);
-            gemv_dispatch<DT>(P, S, ring_it, ring, PH_DOWN, l, tok, pos, t);
-            epilogue_residual(P, S, PH_DOWN);
+            grid_barrier(P, S, epoch, P.timeout_ns, 3);
             trace_mark(P, t, e + 9);
-            grid_barrier(P, S, epoch, P.timeout_ns, 5, true);
-            trace_mark(P, t, e + 10);
         }
         const int eh = 1 + 16 * L;
         if (head) {
@@ -688,6 +746,7 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
 
     uint32_t ring_it = 0;  // chunks consumed (consumers) / issued (producer); both advance identically
     unsigned long long epoch = 0;
+    unsigned long long rd_epoch = 0;  // split-barrier arrivals of this CTA so far in this launch
     uint32_t att_use = 0;  // attention phases so far in this launch (the merge counters' targets)
     for (;;) {
         if (tid < KIE_CONS_THREADS) {
@@ -734,7 +793,7 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
         if (tid >= KIE_CONS_THREADS) {
             if (tid == KIE_CONS_THREADS) produce(P, S, ring_it, smem, cmd);
         } else {
-            consume<DT>(P, S, ring_it, smem, cmd, epoch, att_use);
+            consume<DT>(P, S, ring_it, smem, cmd, epoch, rd_epoch, att_use);
         }
         __syncthreads();
         if (resident && blockIdx.x == 0 && tid == 0) {

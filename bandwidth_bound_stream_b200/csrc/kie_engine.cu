@@ -53,6 +53,27 @@ __global__ void gather_rows_kernel(const RowCopy *rc, long long n, uint8_t *aren
     }
 }
 
+// One fold block of the batch-1 stream: columns [col0, col0 + 8 ng) of a row-major matrix with
+// rows of `ld` bytes, written as [ng][rows][8] (16 bytes per row and column group).
+struct FoldCopy {
+    long long dst;
+    const uint8_t *src;
+    long long ld;
+    int col0, ng, rows;
+};
+
+__global__ void fold_pack_kernel(const FoldCopy *fc, long long n, uint8_t *arena) {
+    for (long long i = blockIdx.x; i < n; i += gridDim.x) {
+        const FoldCopy f = fc[i];
+        const long long vecs = (long long)f.ng * f.rows;
+        for (long long v = threadIdx.x; v < vecs; v += blockDim.x) {
+            const long long g = v / f.rows, r = v % f.rows;
+            *reinterpret_cast<uint4 *>(arena + f.dst + v * 16) =
+                *reinterpret_cast<const uint4 *>(f.src + r * f.ld + (f.col0 + 8 * g) * 2);
+        }
+    }
+}
+
 enum { KIND_NONE = 0, KIND_B1 = 1, KIND_MR = 2 };
 
 double now_s() {
@@ -86,7 +107,8 @@ struct kie_engine {
     cudaError_t reset_barrier(cudaStream_t st) {
         const int fill = pending_fault == KIE_FAULT_BARRIER_SHORT ? 0xFF : 0;
         pending_fault = KIE_FAULT_NONE;
-        return cudaMemsetAsync(P.bar, fill, 16, st);
+        cudaError_t e = cudaMemsetAsync(P.bar, fill, 16, st);
+        return e == cudaSuccess ? cudaMemsetAsync(P.rd, 0, 8, st) : e;
     }
 
     kie_status fail(kie_status s, const char *fmt, ...) {
@@ -134,7 +156,6 @@ extern "C" void kie_config_defaults(kie_config *c) {
     c->idle_ms = 200;
     c->modes = KIE_MODE_BATCH1;
     c->device = 0;
-    c->prefetch_kb = 0;
 }
 
 extern "C" const char *kie_status_string(kie_status s) {
@@ -177,7 +198,6 @@ static const char *shape_error(const kie_config &c) {
     if (c.max_sessions <= 0 || c.max_ctx <= 0) return "max_sessions and max_ctx must be positive";
     if (c.timeout_ms <= 0 || c.idle_ms <= 0) return "timeouts must be positive";
     if (!(c.modes & (KIE_MODE_BATCH1 | KIE_MODE_TICK))) return "modes must enable at least one kernel";
-    if (c.prefetch_kb < 0 || c.prefetch_kb > 65536) return "prefetch_kb must be in [0, 65536]";
     return nullptr;
 }
 
@@ -260,59 +280,74 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
 
     P.splits = 1;
     if (b1) {  // ---- batch-1 kernel: static schedule and packed weights
-    const int Kph[KIE_NPH] = {d, qd, d, F, d};
-    std::vector<int> row0((size_t)KIE_NPH * (nblk + 1));
-    partition(&row0[PH_QKV * (nblk + 1)], (qd + 2 * kvd) / 2, 2, nblk);
-    partition(&row0[PH_O * (nblk + 1)], d, 1, nblk);
-    partition(&row0[PH_GU * (nblk + 1)], F, 2, nblk);
-    partition(&row0[PH_DOWN * (nblk + 1)], d, 1, nblk);
-    partition(&row0[PH_HEAD * (nblk + 1)], V, 1, nblk);
-    for (int ph = 0; ph < KIE_NPH; ph++) {
-        P.K[ph] = Kph[ph];
-        P.cr[ph] = kie_b1_chunk_rows(Kph[ph]);  // rows per ring chunk (even for the paired phases)
-        if (ph == PH_O && (d + nblk - 1) / nblk > KIE_XOWN_MAX) {
-            eng->fail(KIE_ERR_ARG, "d_model too large for %d SMs", nblk);
-            return bail(KIE_ERR_ARG);
-        }
-        const int max_rows = kie_b1_max_rows(Kph[ph]);
-        for (int cc = 0; cc < nblk; cc++)
-            if (row0[ph * (nblk + 1) + cc + 1] - row0[ph * (nblk + 1) + cc] > max_rows) {
-                eng->fail(KIE_ERR_ARG, "phase %d gives a CTA more than %d rows", ph, max_rows);
-                return bail(KIE_ERR_ARG);
-            }
+    if (d > KIE_B1_DMAX) {
+        eng->fail(KIE_ERR_ARG, "the batch-1 kernel supports d_model <= %d", KIE_B1_DMAX);
+        return bail(KIE_ERR_ARG);
     }
     // attention splits: about one (kv head, split) unit per CTA
     P.splits = std::max(1, nblk / Hkv);
-    P.pf_chunks = (int)(((long long)c.prefetch_kb * 1024 + KIE_SLOT_BYTES - 1) / KIE_SLOT_BYTES);
+    const int E = G * D;  // attention outputs of one kv head (its query heads)
+    const int Kph[KIE_NPH] = {d, 8, d, 8, d};
+    std::vector<int> row0((size_t)KIE_NPH * (nblk + 1));
+    partition(&row0[PH_QKV * (nblk + 1)], (qd + 2 * kvd) / 2, 2, nblk);  // rotation pairs
+    // O fold: CTA c = g * splits + s holds 8-column groups [s (E/8) / splits, (s+1) (E/8) / splits)
+    // of kv head g's outputs, i.e. global groups g (E/8) + that; the CTAs past Hkv * splits none
+    for (int cc = 0; cc <= nblk; cc++) {
+        const int u = std::min(cc, Hkv * P.splits), g = u / P.splits, sp = u % P.splits;
+        row0[PH_OF * (nblk + 1) + cc] = g * (E / 8) + (int)((long long)sp * (E / 8) / P.splits);
+    }
+    partition(&row0[PH_GU * (nblk + 1)], F / 8, 16, nblk);  // 8 gate/up pairs (16 rows) at a time
+    partition(&row0[PH_DF * (nblk + 1)], F / 8, 1, nblk);   // the same pairs: 8-column groups of Wd
+    partition(&row0[PH_HEAD * (nblk + 1)], V, 1, nblk);
+    auto range = [&](int ph, int cc) { return row0[ph * (nblk + 1) + cc + 1] - row0[ph * (nblk + 1) + cc]; };
+    for (int ph = 0; ph < KIE_NPH; ph++) {
+        P.K[ph] = Kph[ph];
+        const bool fold = (ph == PH_OF || ph == PH_DF);
+        // rows per ring chunk (even for the paired phases), or 8-column groups per chunk of a fold
+        P.cr[ph] = fold ? KIE_SLOT_BYTES / (d * 16) : kie_b1_chunk_rows(Kph[ph]);
+        const int lim = fold ? KIE_FOLD_MAX / 8 : kie_b1_max_rows(Kph[ph]);
+        for (int cc = 0; cc < nblk; cc++)
+            if (range(ph, cc) > lim) {
+                eng->fail(KIE_ERR_ARG, "phase %d gives a CTA more than %d %s", ph, lim, fold ? "column groups" : "rows");
+                return bail(KIE_ERR_ARG);
+            }
+    }
 
-    // ---- packed weights: CTA c's stream is one contiguous segment
+    // ---- packed weights: CTA c's stream is one contiguous segment (per layer: QKV rows, its Wo
+    // column groups, its gate/up rows, its Wd column groups; then its LM-head rows)
     std::vector<long long> seg_off(nblk + 1, 0);
     for (int cc = 0; cc < nblk; cc++) {
-        long long lb = 0;
-        for (int ph = 0; ph < PH_HEAD; ph++)
-            lb += (long long)(row0[ph * (nblk + 1) + cc + 1] - row0[ph * (nblk + 1) + cc]) * Kph[ph] * 2;
-        const long long hb = (long long)(row0[PH_HEAD * (nblk + 1) + cc + 1] - row0[PH_HEAD * (nblk + 1) + cc]) * d * 2;
-        seg_off[cc + 1] = seg_off[cc] + (long long)L * lb + hb;
+        const long long lb = (long long)range(PH_QKV, cc) * d * 2 + (long long)range(PH_OF, cc) * d * 16 +
+                             (long long)range(PH_GU, cc) * d * 2 + (long long)range(PH_DF, cc) * d * 16;
+        seg_off[cc + 1] = seg_off[cc] + (long long)L * lb + (long long)range(PH_HEAD, cc) * d * 2;
     }
     uint8_t *wpack = nullptr;
     CKC(eng->alloc(&wpack, (size_t)seg_off[nblk]), "cudaMalloc packed weights");
     P.wpack = wpack;
     {
-        std::vector<RowCopy> rc;
-        rc.reserve((size_t)L * (qd + 2 * kvd + d + 2 * F + d) + V);
+        std::vector<RowCopy> rc;   // whole rows (GEMV phases)
+        std::vector<FoldCopy> fc;  // column-group blocks (folds)
+        rc.reserve((size_t)L * (qd + 2 * kvd + 2 * F) + V);
         for (int cc = 0; cc < nblk; cc++) {
             long long off = seg_off[cc];
             for (int l = 0; l <= L; l++) {
                 const void *const *Lw = w->layers + (size_t)9 * (l < L ? l : 0);
                 for (int ph = (l < L ? 0 : PH_HEAD); ph < (l < L ? PH_HEAD : KIE_NPH); ph++) {
+                    const int a = row0[ph * (nblk + 1) + cc], n = range(ph, cc);
+                    if (ph == PH_OF || ph == PH_DF) {
+                        if (n > 0) {
+                            const uint8_t *src = static_cast<const uint8_t *>(Lw[ph == PH_OF ? 4 : 8]);
+                            fc.push_back({off, src, (long long)(ph == PH_OF ? qd : F) * 2, 8 * a, n, d});
+                        }
+                        off += (long long)n * d * 16;
+                        continue;
+                    }
                     const int K = Kph[ph];
-                    for (int r = row0[ph * (nblk + 1) + cc]; r < row0[ph * (nblk + 1) + cc + 1]; r++) {
+                    for (int r = a; r < a + n; r++) {
                         const uint8_t *src;
                         switch (ph) {
                             case PH_QKV: src = qkv_src(c, Lw, r); break;
-                            case PH_O: src = static_cast<const uint8_t *>(Lw[4]) + (size_t)r * K * 2; break;
                             case PH_GU: src = static_cast<const uint8_t *>(Lw[(r & 1) ? 7 : 6]) + (size_t)(r >> 1) * K * 2; break;
-                            case PH_DOWN: src = static_cast<const uint8_t *>(Lw[8]) + (size_t)r * K * 2; break;
                             default: src = static_cast<const uint8_t *>(w->lm_head) + (size_t)r * K * 2; break;
                         }
                         rc.push_back({off, src, (long long)K * 2});
@@ -326,14 +361,20 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
             }
         }
         RowCopy *d_rc = nullptr;
+        FoldCopy *d_fc = nullptr;
         CKC(cudaMalloc(&d_rc, rc.size() * sizeof(RowCopy)), "cudaMalloc repack list");
-        e = cudaMemcpy(d_rc, rc.data(), rc.size() * sizeof(RowCopy), cudaMemcpyHostToDevice);
+        e = cudaMalloc(&d_fc, std::max<size_t>(1, fc.size()) * sizeof(FoldCopy));
+        if (e == cudaSuccess) e = cudaMemcpy(d_rc, rc.data(), rc.size() * sizeof(RowCopy), cudaMemcpyHostToDevice);
+        if (e == cudaSuccess && !fc.empty())
+            e = cudaMemcpy(d_fc, fc.data(), fc.size() * sizeof(FoldCopy), cudaMemcpyHostToDevice);
         if (e == cudaSuccess) {
             gather_rows_kernel<<<4 * nblk, 256>>>(d_rc, (long long)rc.size(), wpack);
+            if (!fc.empty()) fold_pack_kernel<<<4 * nblk, 256>>>(d_fc, (long long)fc.size(), wpack);
             e = cudaGetLastError();
         }
         if (e == cudaSuccess) e = cudaDeviceSynchronize();
         cudaFree(d_rc);
+        cudaFree(d_fc);
         if (e != cudaSuccess) return bail(eng->cuda_fail(e, "weight repack"));
     }
     int *d_row0 = nullptr;
@@ -504,21 +545,18 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
     // ---- activations and scratch
     CKC(eng->alloc(&P.x, (size_t)d * 4), "cudaMalloc x");
     CKC(eng->alloc(&P.q, (size_t)qd * 4), "cudaMalloc q");
-    CKC(eng->alloc(&P.o, (size_t)qd * 4), "cudaMalloc o");
-    CKC(eng->alloc(&P.u, (size_t)F * 4), "cudaMalloc u");
     CKC(eng->alloc(&P.part, (size_t)Hkv * P.splits * G * (D + 2) * 4), "cudaMalloc partials");
     CKC(eng->alloc(&P.cnt, (size_t)Hkv * 4), "cudaMalloc counters");
     CKC(eng->alloc(&P.cand_val, (size_t)nblk * 4), "cudaMalloc candidates");
     CKC(eng->alloc(&P.cand_idx, (size_t)nblk * 4), "cudaMalloc candidates");
     CKC(eng->alloc(&P.tokbuf, (size_t)c.max_ctx * 4), "cudaMalloc token buffer");
-    CKC(eng->alloc(&P.bar, 16), "cudaMalloc barrier");
+    CKC(eng->alloc(&P.bar, 32), "cudaMalloc barrier");  // [0]: grid barrier, [2]: the residual-read split barrier
+    P.rd = P.bar + 2;
     CKC(eng->alloc(&P.err, 16), "cudaMalloc error word");
     CKC(eng->alloc(&P.last_seq, 16), "cudaMalloc sequence");
     CKC(eng->alloc(&P.cmd, sizeof(KieCmd)), "cudaMalloc command");
-    CKC(eng->alloc(&P.ssq, (size_t)nblk * 4), "cudaMalloc norm partials");
-    CKC(cudaMemset(P.ssq, 0, (size_t)nblk * 4), "memset");
     CKC(cudaMemset(P.cnt, 0, (size_t)Hkv * 4), "memset");
-    CKC(cudaMemset(P.bar, 0, 16), "memset");
+    CKC(cudaMemset(P.bar, 0, 32), "memset");
     CKC(cudaMemset(P.err, 0, 16), "memset");
     CKC(cudaMemset(P.last_seq, 0, 16), "memset");
     CKC(cudaMemset(P.x, 0, (size_t)d * 4), "memset");

@@ -13,10 +13,15 @@
 #define KIE_ROWACC_MAX 1024                   // output rows one CTA may own in one phase
 #define KIE_GMAX 8                            // query heads per kv head
 #define KIE_DMAX 128                          // head_dim
-#define KIE_XOWN_MAX 64                       // residual rows one CTA may own (d_model / SMs)
+#define KIE_FOLD_MAX 256                      // inputs one CTA folds into the residual in one phase
+#define KIE_B1_DMAX 4096                      // d_model the batch-1 kernel's folds support
 
-// Phases of the batch-1 weight stream, in stream order within a layer; the LM head follows the last layer.
-enum { PH_QKV = 0, PH_O = 1, PH_GU = 2, PH_DOWN = 3, PH_HEAD = 4, KIE_NPH = 5 };
+// Phases of the batch-1 weight stream, in stream order within a layer; the LM head follows the
+// last layer. QKV, GU and HEAD are row GEMVs (whole rows of W, a CTA owns a row range). OF and DF
+// are folds: a CTA owns 8-column groups of Wo (its attention split's slice of the output) or of
+// Wd (the gate/up pairs it computed), streamed as [group][d rows][8 columns], and adds
+// W[:, its columns] * its inputs into the residual.
+enum { PH_QKV = 0, PH_OF = 1, PH_GU = 2, PH_DF = 3, PH_HEAD = 4, KIE_NPH = 5 };
 
 // Commands of the resident kernel.
 enum { OP_NONE = 0, OP_DECODE = 1, OP_PREFILL = 2, OP_TICK = 3, OP_EXIT = 4 };
@@ -57,11 +62,11 @@ struct KieParams {
     float eps;
     int max_ctx, max_sessions, nblk;
     int splits;                     // attention splits per kv head (batch-1)
-    int cr[KIE_NPH];                // rows per ring chunk, per phase
-    int K[KIE_NPH];                 // row length (elements) per phase
+    int cr[KIE_NPH];                // rows per ring chunk (GEMV phases) or 8-column groups per chunk (folds)
+    int K[KIE_NPH];                 // row length (elements) per phase (8 for folds)
     // batch-1 packed weights: CTA c streams [seg_off[c], seg_off[c+1]) once per token
     const uint8_t *wpack;
-    const int *row0;                // [KIE_NPH][nblk+1] logical row partition
+    const int *row0;                // [KIE_NPH][nblk+1] partition: rows (GEMV phases), 8-column groups (folds)
     const long long *seg_off;       // [nblk+1]
     // unpacked small weights
     const uint16_t *emb;            // [V][d]
@@ -71,20 +76,19 @@ struct KieParams {
     uint16_t *kcache, *vcache;
     long long sess_stride;
     // activations and scratch
-    float *x, *q, *o, *u;
+    float *x, *q;                   // residual [d] (folds add into it), rotated queries [Hq*D]
     float *part;                    // [Hkv*splits*G][D+2]
     unsigned *cnt;                  // [Hkv]
     float *cand_val;
     int *cand_idx;                  // [nblk]
     int *tokbuf;                    // [max_ctx] device copy of command inputs
     unsigned long long *bar;        // grid barrier counter
+    unsigned long long *rd;         // CTAs that have read the residual for the gate/up phase (split barrier)
     unsigned *err;                  // first device error
     KieMailbox *mbox;               // device alias of the mapped mailbox
     unsigned *last_seq;             // last doorbell sequence processed
     KieCmd *cmd;                    // command broadcast slot
     long long timeout_ns, idle_ns;
-    int pf_chunks;                  // L2 lead: weight chunks after the one being copied that are kept requested into L2
-    float *ssq;                     // [nblk] per-CTA sums of squares of the residual rows it owns
     unsigned long long *trace;      // phase stamps (null = off)
     int trace_tokens, trace_events;
     // multi-row (tick / chunked prefill) kernel: swizzled 128 x 64 weight tiles, CTA c streams

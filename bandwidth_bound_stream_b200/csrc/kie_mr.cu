@@ -797,6 +797,7 @@ __device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M, uint32
         A.brow = m;
         A.gout = g;
         A.cnt_target = 0;
+        A.oslice = nullptr;
         A.timeout_ns = 0;
         A.err = nullptr;
         A.D = P.D;

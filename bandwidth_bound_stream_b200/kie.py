@@ -34,7 +34,7 @@ class KieConfig(ctypes.Structure):
                                                "vocab")] + \
                [("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float)] + \
                [(n, ctypes.c_int32) for n in ("dtype", "max_sessions", "max_ctx", "timeout_ms", "idle_ms", "modes",
-                                               "device", "prefetch_kb")]
+                                               "device")]
 
 
 class KieWeights(ctypes.Structure):
@@ -96,7 +96,7 @@ def _ptr(a: np.ndarray):
 
 
 def config(model, max_sessions: int = 1, max_ctx: int = 4096, timeout_ms: int = 10000, idle_ms: int = 200,
-           modes: int = KIE_MODE_BATCH1, device: int = 0, prefetch_kb: int | None = None) -> KieConfig:
+           modes: int = KIE_MODE_BATCH1, device: int = 0) -> KieConfig:
     """A kie_config for a model shape (any object with the shape attributes of synth.ModelConfig)."""
     c = KieConfig()
     lib.kie_config_defaults(ctypes.byref(c))
@@ -105,8 +105,6 @@ def config(model, max_sessions: int = 1, max_ctx: int = 4096, timeout_ms: int = 
     c.rms_eps, c.rope_theta = model.rms_eps, model.rope_theta
     c.max_sessions, c.max_ctx, c.timeout_ms, c.idle_ms, c.modes, c.device = (max_sessions, max_ctx, timeout_ms,
                                                                                 idle_ms, modes, device)
-    if prefetch_kb is not None:
-        c.prefetch_kb = prefetch_kb
     return c
 
 

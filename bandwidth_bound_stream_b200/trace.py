@@ -2,8 +2,9 @@
 
 ``kie_trace_enable`` / ``kie_trace_read`` (layout in ``include/kie.h``) give, per CTA and
 token, globaltimer stamps (ns). Slot 0 is the token's start. Each layer l then has 16 slots
-from 1 + 16 l: the ends of its 11 phases, the input-ready stamps of the QKV, O, gate/up and
-down phases, and the end of this CTA's attention positions (0 when it owns no unit). After
+from 1 + 16 l: the ends of its 10 phases (slots 0-9), the end of the down fold's wait for
+every CTA's read of the residual (10), the input-ready stamps of the QKV and gate/up phases
+(11, 12), and the end of this CTA's attention positions (15; 0 when it owns no unit). After
 the layers come the LM head's rows, its barrier and the final argmax, then two ring-wait
 totals. Host-side arithmetic only.
 """
@@ -11,8 +12,9 @@ from __future__ import annotations
 
 import numpy as np
 
-LAYER_PHASES = ("qkv_rows", "qkv_epilogue", "barrier_qkv_attn", "attention", "barrier_attn_o", "o_rows_epilogue",
-                "barrier_o_gu", "gate_up_rows_epilogue", "barrier_gu_down", "down_rows_epilogue", "barrier_down_next")
+LAYER_PHASES = ("qkv_rows", "qkv_epilogue", "barrier_qkv_attn", "attention", "o_fold", "barrier_o_gu",
+                "gate_up_rows", "gate_up_epilogue", "down_fold", "barrier_down_next")
+LAYER_END = len(LAYER_PHASES) - 1  # slot of the layer's last phase end
 
 
 def batch1_events(n_layers: int) -> int:
@@ -43,7 +45,7 @@ def batch1_phase_us(trace: np.ndarray, n_layers: int, first_token: int = 1) -> d
         s = x[:, t, :]
         for l in layers:
             base = 1 + 16 * l
-            prev = s[:, base - 6] if l > 0 else s[:, 0]  # the end of the previous layer (or the token start)
+            prev = s[:, base - 16 + LAYER_END] if l > 0 else s[:, 0]  # the end of the previous layer (or the token start)
             for i, p in enumerate(LAYER_PHASES):
                 dur[p].append(s[:, base + i] - prev)
                 prev = s[:, base + i]
@@ -52,11 +54,11 @@ def batch1_phase_us(trace: np.ndarray, n_layers: int, first_token: int = 1) -> d
             positions.extend((tu - s[:, base + 2])[own])
             merge.extend((s[:, base + 3] - tu)[own])
         eh = 1 + 16 * n_layers
-        head["lm_head_rows"].append(s[:, eh] - s[:, eh - 6])
+        head["lm_head_rows"].append(s[:, eh] - s[:, eh - 16 + LAYER_END])
         head["lm_head_barrier"].append(s[:, eh + 1] - s[:, eh])
         head["argmax"].append(s[:, eh + 2] - s[:, eh + 1])
         if n_layers > 1:
-            per_layer.append((s[:, 1 + 16 * (n_layers - 1) + 10] - s[:, 1 + 10]) / (n_layers - 1))
+            per_layer.append((s[:, 1 + 16 * (n_layers - 1) + LAYER_END] - s[:, 1 + LAYER_END]) / (n_layers - 1))
 
     def us(arrays):  # mean over every CTA of every entry, ns -> µs
         return round(float(np.mean(np.concatenate([np.ravel(a) for a in arrays]))) / 1e3, 2)

@@ -69,12 +69,6 @@ typedef struct {
     int32_t idle_ms;      /* the resident kernel exits after this long with no command */
     int32_t modes;        /* KIE_MODE_* bitmask                                        */
     int32_t device;       /* CUDA device ordinal                                       */
-    int32_t prefetch_kb;  /* batch-1 kernel: per SM, the KB of weights after the chunk
-                             being copied into the shared-memory ring that are kept
-                             requested into L2 (an L2 lead of fixed size, so HBM keeps
-                             streaming while the ring is full and the kernel sits in
-                             attention or at a barrier); 0 = ring only. Rounded up to
-                             64 KB ring chunks.                                          */
 } kie_config;
 
 /*
@@ -95,7 +89,7 @@ typedef struct {
 
 /* Fills a config with the shape fields zeroed and defaults for the rest
    (eps 1e-5, theta 1e4, fp16, 1 session, 4096 positions, timeouts 10 s / 200 ms,
-   batch-1 mode, device 0, no L2 lead). */
+   batch-1 mode, device 0). */
 void kie_config_defaults(kie_config *cfg);
 
 /*
@@ -103,7 +97,7 @@ void kie_config_defaults(kie_config *cfg);
  * (packed weights, KV cache of max_sessions x max_ctx, activations, split-K scratch,
  * mapped host mailbox), computes the static work partition for this GPU's SM count and
  * repacks the weights. Constraints: d_model, n_heads*head_dim and ffn multiples of 64,
- * d_model <= 8192, ffn and n_heads*head_dim <= 14336;
+ * d_model <= 8192 (<= 4096 with KIE_MODE_BATCH1), ffn and n_heads*head_dim <= 14336;
  * head_dim even and <= 128; n_heads a multiple of n_kv_heads with n_heads/n_kv_heads <= 8.
  * Errors: KIE_ERR_ARG (shape), KIE_ERR_CUDA (allocation or launch). On error *out is NULL.
  */
@@ -175,12 +169,13 @@ kie_status kie_tick(kie_engine *eng, int32_t n_sess, const int32_t *sids, const 
  * copies the record into `host` (uint64, at most max_elems) and returns the element count
  * through *n; layout [cta][token][event], events per token = kie_trace_events(eng):
  * Batch-1 decode commands write one record per token:
- *   0: token start; then per layer 16 slots: 11 phase ends (QKV rows, QKV epilogue, barrier,
- *   attention, barrier, O rows+epilogue, barrier, gate/up rows+epilogue, barrier, down
- *   rows+epilogue, barrier) and 5 inner stamps (input vectors ready in the QKV, O, gate/up
- *   and down phases; end of this CTA's attention positions, before its split is published,
- *   0 if it had no unit); then 3 for the head (rows+argmax, barrier, final
- *   argmax); then the consumer's and the producer's total ring wait in ns.
+ *   0: token start; then per layer 16 slots: 10 phase ends (0 QKV rows, 1 QKV epilogue,
+ *   2 barrier, 3 attention with its slice merge, 4 O fold, 5 barrier, 6 gate/up rows,
+ *   7 gate/up epilogue, 8 down fold, 9 barrier), then 10 the end of the down fold's wait for
+ *   every CTA's read of the residual, 11 and 12 input vectors ready in the QKV and gate/up
+ *   phases, 15 the end of this CTA's attention positions (before its split is published; 0
+ *   if it had no unit); then 3 for the head (rows+argmax, barrier, final argmax); then the
+ *   consumer's and the producer's total ring wait in ns.
  * Tick and chunked-prefill commands write one record per step, in the same layout:
  *   0: step start; per layer (slot 1 + 16 l + k): k = 0 first norm done, then the ends of
  *   the grid barriers after: 1 first norm, 3 QKV, 4 RoPE, 6 attention (5: this CTA's

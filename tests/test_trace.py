@@ -28,7 +28,7 @@ def _synthetic(n_cta, n_tok, L, phase_ns, pos_ns, head_ns):
 
 
 def test_phase_breakdown_recovers_known_durations():
-    phase = [4200, 840, 2970, 9080, 1740, 1900, 2500, 11230, 3120, 5750, 2550]
+    phase = [4200, 840, 2970, 9080, 1740, 1900, 2500, 11230, 3120, 5750]
     x = _synthetic(4, 3, 5, phase, pos_ns=4720, head_ns=(20320, 2700, 1570))
     out = tr.batch1_phase_us(x, 5)
     for name, d in zip(tr.LAYER_PHASES, phase):
@@ -43,7 +43,7 @@ def test_phase_breakdown_recovers_known_durations():
 
 
 def test_phase_breakdown_single_layer_and_shape_check():
-    x = _synthetic(2, 1, 1, [10] * 11, pos_ns=3, head_ns=(5, 6, 7))
+    x = _synthetic(2, 1, 1, [10] * 10, pos_ns=3, head_ns=(5, 6, 7))
     out = tr.batch1_phase_us(x, 1)
     assert out["qkv_rows"] == pytest.approx(0.01) and out["tokens"] == 1 and "per_layer" not in out
     with pytest.raises(ValueError):
