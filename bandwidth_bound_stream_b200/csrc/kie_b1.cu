@@ -69,6 +69,7 @@ struct __align__(16) B1Shared {
     int gb_ok;
     int row0[KIE_NPH], row1[KIE_NPH];
     unsigned long long wait_cons;
+    __align__(16) uint8_t warm_sink[512];  // destination of the K/V reads into L2 (16 bytes per lane; never read)
 };
 
 // word-wise copies of the command record (volatile: it may live in mapped host memory)
@@ -451,7 +452,7 @@ __device__ __forceinline__ void fold_commit(const KieParams &P, const B1Shared &
 
 // --------------------------------------------------------------- consumer: epilogues
 
-__device__ __forceinline__ void attention_prefetch(const KieParams &P, int l, int sid, int pos);
+__device__ __forceinline__ void attention_prefetch(const KieParams &P, B1Shared &S, int l, int sid, int pos);
 
 // q/k rows come in rotation pairs (dim i, dim i + D/2); v rows use the same pairing.
 template <int DT>
@@ -487,13 +488,13 @@ __device__ void epilogue_qkv(const KieParams &P, B1Shared &S, int l, int sid, in
     if (l == 0) {  // the residual starts as the embedding row (each CTA writes a 1/nblk share)
         const int r0 = (int)((long long)blockIdx.x * P.d / P.nblk), r1 = (int)((long long)(blockIdx.x + 1) * P.d / P.nblk);
         for (int r = r0 + threadIdx.x; r < r1; r += KIE_CONS_THREADS) P.x[r] = cvt1<DT>(P.emb[(size_t)tok * P.d + r]);
-        attention_prefetch(P, l, sid, pos);
+        attention_prefetch(P, S, l, sid, pos);
     }
 }
 
-// The cache rows this CTA's attention unit will read in layer l start moving into L2
-// (older positions are final; L2 stays coherent for the one written in this token).
-__device__ __forceinline__ void attention_prefetch(const KieParams &P, int l, int sid, int pos) {
+// The cache rows this CTA's attention unit will read in layer l are read into L2 ahead of
+// time (older positions are final; L2 stays coherent for the one written in this token).
+__device__ __forceinline__ void attention_prefetch(const KieParams &P, B1Shared &S, int l, int sid, int pos) {
     const int D = P.D;
     const size_t sess = (size_t)sid * P.sess_stride;
     const int ctx = pos + 1;
@@ -501,17 +502,20 @@ __device__ __forceinline__ void attention_prefetch(const KieParams &P, int l, in
         const int g = unit / P.splits, s = unit % P.splits;
         const long long p0 = (long long)s * ctx / P.splits, p1 = (long long)(s + 1) * ctx / P.splits;
         const size_t off = sess + ((size_t)(l * P.Hkv + g) * P.max_ctx + p0) * D;
-        const int lines = (int)(((p1 - p0) * D * 2 + 127) / 128);
+        // whole lines (a partial one is left to the loads), at most 256 KB per unit: at long
+        // contexts a layer's cache outgrows L2, and reading it all ahead would evict itself and
+        // compete with the weight stream of the phase that issues the reads
+        const int lines = (int)min((p1 - p0) * D * 2 / 128, (long long)KIE_KV_WARM_LINES);
         for (int j = threadIdx.x; j < 2 * lines; j += KIE_CONS_THREADS) {
             const uint16_t *base = (j < lines ? P.kcache : P.vcache) + off;
-            prefetch_l2(reinterpret_cast<const uint8_t *>(base) + (size_t)(j % lines) * 128);
+            l2_warm_line(S.warm_sink + (threadIdx.x & 31) * 16, reinterpret_cast<const uint8_t *>(base) + (size_t)(j % lines) * 128);
         }
     }
 }
 
 // u = silu(gate) * up for this CTA's pairs, into the down fold's inputs
 __device__ void epilogue_gu(const KieParams &P, B1Shared &S, int l, int sid, int pos) {
-    if (l + 1 < P.L) attention_prefetch(P, l + 1, sid, pos);
+    if (l + 1 < P.L) attention_prefetch(P, S, l + 1, sid, pos);
     const int npair = (S.row1[PH_GU] - S.row0[PH_GU]) >> 1;
     const int cs = col_slices(P.K[PH_GU]);
     for (int p = threadIdx.x; p < npair; p += KIE_CONS_THREADS) {
@@ -721,6 +725,7 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, cons
         if (P.trace && t < P.trace_tokens && threadIdx.x == 0)
             P.trace[((size_t)blockIdx.x * P.trace_tokens + t) * P.trace_events + P.trace_events - 2] = S.wait_cons;
     }
+    cp_async_wait_all();  // the L2 reads into warm_sink have landed
 }
 
 // --------------------------------------------------------------- the kernel
@@ -743,7 +748,6 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
         S.row1[tid] = P.row0[tid * (P.nblk + 1) + blockIdx.x + 1];
     }
     __syncthreads();
-
     uint32_t ring_it = 0;  // chunks consumed (consumers) / issued (producer); both advance identically
     unsigned long long epoch = 0;
     unsigned long long rd_epoch = 0;  // split-barrier arrivals of this CTA so far in this launch

@@ -106,6 +106,15 @@ KIE_DEV void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
                  : "memory");
 }
 
+// Reads 16 bytes at src into shared memory at dst asynchronously, with the 128-byte L2 fetch
+// size: the line lands in L2 and stays there for a later bulk copy (on B200 the L2 prefetch
+// instructions leave much of the data out of L2). The caller never reads dst; it waits for
+// these copies (cp_async_wait_all) before its shared memory goes away.
+KIE_DEV void l2_warm_line(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global.L2::128B [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+KIE_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Hint: bring the 128-byte line holding p into L2 (through the load/store unit).
 KIE_DEV void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 

@@ -15,6 +15,7 @@
 #define KIE_DMAX 128                          // head_dim
 #define KIE_FOLD_MAX 256                      // inputs one CTA folds into the residual in one phase
 #define KIE_B1_DMAX 4096                      // d_model the batch-1 kernel's folds support
+#define KIE_KV_WARM_LINES 1024                // 128-byte lines each of K and V an attention unit reads into L2 ahead
 
 // Phases of the batch-1 weight stream, in stream order within a layer; the LM head follows the
 // last layer. QKV, GU and HEAD are row GEMVs (whole rows of W, a CTA owns a row range). OF and DF
