@@ -23,6 +23,10 @@
  *     x   += Wd (silu(Wg h) * (Wu h)),  silu(z) = z / (1 + exp(-z))
  *   logits = W_lm (x / sqrt(mean(x^2) + eps) * g_final);  token = argmax (lowest index on ties)
  *
+ * The sampling variant (orc_sample, at the end) replaces the argmax by temperature / top-k
+ * sampling with one counter-based uniform draw per step (splitmix64 keyed by a seed and the
+ * step's position).
+ *
  * Arithmetic is fp64 throughout; weights are read as exact fp16/bf16 values. The only
  * rounding besides fp64's own is the one the method defines: K and V are stored in the
  * weight dtype (rounded fp64 -> fp32 -> storage, both round-to-nearest-even).
@@ -306,3 +310,81 @@ int32_t orc_forward_sequence(const orc_config *c, const orc_weights *w, int32_t 
 }
 
 int32_t orc_num_threads(void) { return omp_get_max_threads(); }
+
+/* ---------------------------------------------------------------- sampling
+ *
+ * The variant beside greedy decoding: temperature and top-k sampling of the next token, with
+ * one uniform draw per decode step taken from a counter-based generator, so a step's token is
+ * a function of (logits, temperature, top_k, seed, position) alone.
+ */
+
+/* splitmix64: the state advances by the golden-ratio increment 0x9E3779B97F4A7C15 and each
+   output is the new state through the finalizer below (two xor-shift-multiply rounds and a
+   final xor-shift). Output n >= 1 of the generator started from state s is mix(s + n * inc). */
+uint64_t orc_splitmix64(uint64_t seed, uint64_t n) {
+    uint64_t z = seed + n * 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+/* The draw of the decode step at position pos: the top 24 bits of output pos + 1 of the
+   generator started from `seed`, as a multiple of 2^-24 in [0, 1). */
+double orc_uniform(uint64_t seed, int32_t pos) {
+    return (double)(orc_splitmix64(seed, (uint64_t)pos + 1) >> 40) / 16777216.0;
+}
+
+/*
+ * One sampled token. The candidates are the top_k largest logits, in order of value
+ * (descending) and, for equal values, of index (ascending). Candidate k weighs
+ * w_k = exp((z_k - z_0) / temperature); the token is the first candidate whose cumulative
+ * weight exceeds u * (total weight). top_k = 1 is the greedy argmax.
+ * Returns the token; -1 on bad arguments; -2 if a candidate's logit is not finite.
+ * *margin (nullable) receives the distance from u * total to the nearest boundary between
+ * candidates, divided by the total (1 when there is no boundary).
+ */
+int32_t orc_sample(int32_t n, const double *logits, double temperature, int32_t top_k, double u, double *margin) {
+    if (n <= 0 || top_k < 1 || top_k > n || !(temperature > 0.0) || !(u >= 0.0 && u < 1.0)) return -1;
+    int32_t *cand = (int32_t *)malloc(sizeof(int32_t) * top_k);
+    char *taken = (char *)calloc(n, 1);
+    /* the candidates in order: repeatedly the largest remaining value, lowest index first */
+    for (int k = 0; k < top_k; k++) {
+        int best = -1;
+        for (int i = 0; i < n; i++) {
+            if (taken[i]) continue;
+            const double v = isnan(logits[i]) ? -INFINITY : logits[i];
+            if (best < 0 || v > (isnan(logits[best]) ? -INFINITY : logits[best])) best = i;
+        }
+        cand[k] = best;
+        taken[best] = 1;
+    }
+    int32_t tok = -2;
+    int finite = 1;
+    for (int k = 0; k < top_k; k++) finite &= isfinite(logits[cand[k]]) != 0;
+    if (finite) {
+        double *cum = (double *)malloc(sizeof(double) * top_k);
+        double total = 0.0;
+        for (int k = 0; k < top_k; k++) {
+            total += exp((logits[cand[k]] - logits[cand[0]]) / temperature);
+            cum[k] = total;
+        }
+        const double r = u * total;
+        int pick = top_k - 1;
+        for (int k = 0; k < top_k; k++)
+            if (cum[k] > r) {
+                pick = k;
+                break;
+            }
+        tok = cand[pick];
+        if (margin) {
+            double m = 1.0;
+            if (pick > 0) m = fmin(m, (r - cum[pick - 1]) / total);
+            if (pick < top_k - 1) m = fmin(m, (cum[pick] - r) / total);
+            *margin = m;
+        }
+        free(cum);
+    }
+    free(cand);
+    free(taken);
+    return tok;
+}

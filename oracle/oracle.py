@@ -47,6 +47,12 @@ def lib():
         h.orc_forward_sequence.restype = i32
         h.orc_forward_sequence.argtypes = [ctypes.POINTER(_Config), ctypes.POINTER(_Weights), i32, vp, vp]
         h.orc_num_threads.restype = i32
+        h.orc_splitmix64.restype = ctypes.c_uint64
+        h.orc_splitmix64.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
+        h.orc_uniform.restype = ctypes.c_double
+        h.orc_uniform.argtypes = [ctypes.c_uint64, i32]
+        h.orc_sample.restype = i32
+        h.orc_sample.argtypes = [i32, vp, ctypes.c_double, i32, ctypes.c_double, vp]
         del dp
         lib.h = h
     return lib.h
@@ -109,6 +115,25 @@ def silu(z: float) -> float:
 def argmax(v: np.ndarray) -> int:
     v = np.ascontiguousarray(v, dtype=np.float64)
     return int(lib().orc_argmax(v.size, _ptr(v)))
+
+
+def splitmix64(seed: int, n: int) -> int:
+    """Output n >= 1 of the splitmix64 generator started from state `seed`."""
+    return int(lib().orc_splitmix64(seed & (2 ** 64 - 1), n))
+
+
+def uniform(seed: int, pos: int) -> float:
+    """The sampling draw of the decode step at position `pos`."""
+    return float(lib().orc_uniform(seed & (2 ** 64 - 1), pos))
+
+
+def sample(logits, temperature: float, top_k: int, u: float):
+    """(token, margin) of temperature / top-k sampling with draw u (token -1: bad arguments,
+    -2: a candidate's logit is not finite)."""
+    v = np.ascontiguousarray(logits, dtype=np.float64)
+    m = np.zeros(1)
+    tok = int(lib().orc_sample(v.size, _ptr(v), float(temperature), int(top_k), float(u), _ptr(m)))
+    return tok, float(m[0])
 
 
 def num_threads() -> int:

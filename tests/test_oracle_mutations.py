@@ -90,6 +90,16 @@ SLIPS = {
     "matvec_transposed": [("const uint16_t *row = W + (int64_t)n * K;", "const uint16_t *row = W + (int64_t)n;"),
                           ("for (int k = 0; k < K; k++) acc += tv[row[k]] * x[k];",
                            "for (int k = 0; k < K; k++) acc += tv[row[(int64_t)k * N]] * x[k];")],
+    # sampling
+    "sample_temperature_multiplies": [("total += exp((logits[cand[k]] - logits[cand[0]]) / temperature);",
+                                       "total += exp((logits[cand[k]] - logits[cand[0]]) * temperature);")],
+    "sample_ties_to_highest_index": [("if (best < 0 || v > (isnan(logits[best]) ? -INFINITY : logits[best])) best = i;",
+                                      "if (best < 0 || v >= (isnan(logits[best]) ? -INFINITY : logits[best])) best = i;")],
+    "sample_boundary_inclusive": [("            if (cum[k] > r) {", "            if (cum[k] >= r) {")],
+    "sample_draw_uses_output_pos": [("return (double)(orc_splitmix64(seed, (uint64_t)pos + 1) >> 40) / 16777216.0;",
+                                     "return (double)(orc_splitmix64(seed, (uint64_t)pos) >> 40) / 16777216.0;")],
+    "sample_cumulative_from_last_candidate": [("        const double r = u * total;", "        const double r = (1.0 - u) * total;")],
+    "splitmix64_second_shift": [("z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;", "z = (z ^ (z >> 28)) * 0x94D049BB133111EBull;")],
     # storage types
     "bf16_store_truncates": [("return (uint16_t)((x + 0x7FFFu + lsb) >> 16);", "return (uint16_t)(x >> 16);")],
     "fp16_store_rounds_half_up": [("if (rem > 0.5 || (rem == 0.5 && (qi & 1u))) qi++;", "if (rem >= 0.5) qi++;")],

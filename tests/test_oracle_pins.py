@@ -5,6 +5,7 @@ or an independent formulation, chosen so that a plausible slip (a dropped term, 
 a transposed operand, an off-by-one position, a wrong head mapping) fails.
 """
 import dataclasses
+import os
 
 import numpy as np
 import pytest
@@ -15,6 +16,7 @@ from bandwidth_bound_stream_b200 import synth
 from oracle import oracle as orc
 
 FP16, BF16 = 0, 1
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 
 # ---------------------------------------------------------------- storage types
@@ -349,3 +351,71 @@ def test_logit_scale_of_synthetic_model():
     m = orc.OracleModel(cfg, _weights(cfg), 4)
     lg = m.step(int(synth.prompt(cfg, 1)[0]))
     assert 0.5 * 0.02 * np.sqrt(cfg.d_model) < lg.std() < 2.0 * 0.02 * np.sqrt(cfg.d_model)
+
+
+# ------------------------------------------------------------------ sampling (the variant beside argmax)
+
+def test_splitmix64_and_draw_match_the_published_vector():
+    """The oracle's own splitmix64 reproduces the published first five outputs from state
+    1234567, and a step's draw is the top 24 bits of output pos + 1 over 2^24."""
+    want = [int(l) for l in open(os.path.join(GOLDEN, "splitmix64_1234567.txt")) if not l.startswith("#")]
+    assert [orc.splitmix64(1234567, n) for n in range(1, 6)] == want
+    for pos, w in enumerate(want):
+        assert orc.uniform(1234567, pos) == (w >> 40) / 2.0 ** 24
+
+
+def test_sample_top1_is_argmax_for_any_temperature_and_draw():
+    rng = np.random.default_rng(5)
+    for _ in range(50):
+        z = rng.normal(size=37)
+        for T, u in ((0.1, 0.0), (1.0, 0.5), (7.0, 0.999)):
+            tok, m = orc.sample(z, T, 1, u)
+            assert tok == int(np.argmax(z)) and m == 1.0
+
+
+def test_sample_two_candidates_closed_form():
+    """Top-2 of (a, b, much smaller...): the first is chosen iff u < 1 / (1 + e^{(b - a) / T})."""
+    a, b, T = 1.3, 0.4, 0.7
+    z = np.array([-5.0, b, -9.0, a, -7.0])
+    p_first = 1.0 / (1.0 + np.exp((b - a) / T))
+    for u in np.linspace(0.0, 0.9999, 97):
+        tok, m = orc.sample(z, T, 2, u)
+        assert tok == (3 if u < p_first else 1)
+        assert m == pytest.approx(abs(u - p_first), abs=1e-12)
+
+
+def test_sample_frequencies_equal_the_tempered_top_k_softmax():
+    """Draws spread evenly over [0, 1) pick each candidate with its probability, and never a
+    token outside the top k: the temperature, the restriction and the order all enter."""
+    rng = np.random.default_rng(9)
+    z = rng.normal(size=64) * 2.0
+    T, k, N = 0.7, 10, 20000
+    top = np.argsort(-z, kind="stable")[:k]
+    w = np.exp((z[top] - z[top[0]]) / T)
+    p = w / w.sum()
+    counts = np.zeros(64)
+    for i in range(N):
+        tok, _ = orc.sample(z, T, k, (i + 0.5) / N)
+        counts[tok] += 1
+    assert counts[np.setdiff1d(np.arange(64), top)].sum() == 0
+    np.testing.assert_allclose(counts[top] / N, p, atol=1.5 / N)
+
+
+def test_sample_order_breaks_ties_by_index():
+    z = np.array([1.0, 5.0, 5.0, 0.0])
+    assert orc.sample(z, 1.0, 2, 0.49)[0] == 1 and orc.sample(z, 1.0, 2, 0.51)[0] == 2
+    # a draw exactly on a boundary (u * total = 1 = the first weight) goes to the next candidate:
+    # the token is the first whose cumulative weight exceeds the draw
+    assert orc.sample(z, 1.0, 2, 0.5) == (2, 0.0)
+    # third candidate: weights 1, 1, e^-4, so it takes draws above 2 / (2 + e^-4) = 0.99093
+    assert orc.sample(z, 1.0, 3, 0.995)[0] == 0 and orc.sample(z, 1.0, 3, 0.99)[0] == 2
+
+
+def test_sample_rejects_bad_arguments_and_non_finite_candidates():
+    z = np.array([0.5, 2.0, 1.0])
+    assert orc.sample(z, 0.0, 2, 0.5)[0] == -1
+    assert orc.sample(z, 1.0, 4, 0.5)[0] == -1
+    assert orc.sample(z, 1.0, 2, 1.0)[0] == -1
+    assert orc.sample(np.array([np.nan, 1.0, 0.0]), 1.0, 3, 0.2)[0] == -2
+    assert orc.sample(np.array([np.inf, 1.0, 0.0]), 1.0, 2, 0.2)[0] == -2
+    assert orc.sample(np.array([np.nan, 1.0, 0.0]), 1.0, 2, 0.2)[0] in (1, 2)  # NaN ranks below every number
