@@ -45,6 +45,7 @@
 
 #include "kie_attn.cuh"
 #include "kie_device.cuh"
+#include "kie_sample.cuh"
 
 namespace {
 
@@ -56,6 +57,10 @@ struct __align__(16) B1Shared {
     union {
         float wpart[WPART_FLOATS];  // column-slice partials of this phase's row sums
         AttnSmem at;
+        struct {
+            float vals[KIE_SAMPLE_VALS];  // the values a top-k selection reads
+            SampleScratch ss;
+        } samp;
     };
     float fold_in[KIE_FOLD_MAX];  // the current fold's inputs: this CTA's slice of o, or of u
     float red[64];
@@ -579,6 +584,62 @@ __device__ int final_argmax(const KieParams &P) {
     return i;
 }
 
+// Sampling head, first stage: this CTA's logits (rows rbeg .. rbeg + n) -> optional output,
+// then its top-k (value, token) into the candidate slots cand_tv/cand_ti[cta][0..k); slots past
+// the CTA's row count hold NaN, which ranks below every number.
+// (Arguments by value: a reference to the kernel's parameter block would make the kernel keep
+// a copy of it in local memory.)
+__device__ __noinline__ void sample_local(B1Shared &S, float *logits, int k, int cs, float *cand_tv, int *cand_ti,
+                                          int V) {
+    const int tid = threadIdx.x;
+    const int rbeg = S.row0[PH_HEAD], n = S.row1[PH_HEAD] - rbeg;
+    float v0 = 0.f, v1 = 0.f;  // rows tid and tid + 512 (n <= 1024)
+    if (tid < n) v0 = rowsum(S, tid, cs);
+    if (tid + KIE_CONS_THREADS < n) v1 = rowsum(S, tid + KIE_CONS_THREADS, cs);
+    if (logits) {
+        if (tid < n) logits[rbeg + tid] = v0;
+        if (tid + KIE_CONS_THREADS < n) logits[rbeg + tid + KIE_CONS_THREADS] = v1;
+    }
+    named_bar_sync(1, KIE_CONS_THREADS);  // the row partials are read: their space takes the values
+    if (tid < n) S.samp.vals[tid] = v0;
+    if (tid + KIE_CONS_THREADS < n) S.samp.vals[tid + KIE_CONS_THREADS] = v1;
+    const int kl = min(k, n);
+    if (kl > 0) {
+        const float *vals = S.samp.vals;
+        block_topk<KIE_CONS_THREADS>(S.samp.ss, n, kl, [&](int p) { return vals[p]; }, [&](int p) { return rbeg + p; });
+    } else {
+        named_bar_sync(1, KIE_CONS_THREADS);
+    }
+    if (tid < KIE_TOPK_MAX) {
+        const bool have = tid < kl;
+        cand_tv[blockIdx.x * KIE_TOPK_MAX + tid] = have ? S.samp.ss.top_v[tid] : CUDART_NAN_F;
+        cand_ti[blockIdx.x * KIE_TOPK_MAX + tid] = have ? S.samp.ss.top_i[tid] : V + tid;
+    }
+}
+
+// Sampling head, second stage (after the head barrier, in every CTA): the top-k of all CTAs'
+// candidates (CTA c's at positions c*k .. c*k + k - 1: equal values keep the token order), the
+// draw of position pos, the token. Returns the same token in every thread.
+__device__ __noinline__ int sample_global(B1Shared &S, int nblk, const float *cand_tv, const int *cand_ti, float inv_t,
+                                         int k, unsigned long long seed, int pos) {
+    const int tid = threadIdx.x, n = nblk * k;
+    for (int p = tid; p < n; p += KIE_CONS_THREADS)
+        S.samp.vals[p] = __ldcg(cand_tv + (p / k) * KIE_TOPK_MAX + p % k);
+    named_bar_sync(1, KIE_CONS_THREADS);
+    const float *vals = S.samp.vals;
+    const int *ti = cand_ti;
+    block_topk<KIE_CONS_THREADS>(S.samp.ss, n, k, [&](int p) { return vals[p]; },
+                                 [&](int p) { return __ldcg(ti + (p / k) * KIE_TOPK_MAX + p % k); });
+    if (tid < 32) {
+        const int tok = sample_pick(S.samp.ss, k, inv_t, sample_uniform(seed, pos));
+        if (tid == 0) S.token = tok;
+    }
+    named_bar_sync(1, KIE_CONS_THREADS);
+    const int tok = S.token;
+    named_bar_sync(1, KIE_CONS_THREADS);  // S.token is read before anyone reuses the space
+    return tok;
+}
+
 // --------------------------------------------------------------- consumer: attention
 
 // The QKV -> attention barrier, then this CTA's attention unit (at most one unit per CTA:
@@ -663,6 +724,10 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, cons
     int tok = cmd.in_tok;
     if (cmd.op == OP_DECODE && cmd.tok_dev) tok = __ldcg(cmd.tok_dev);
     const int L = P.L;
+    SampleCfg sc;
+    sc.inv_t = __ldcg(&P.samp[cmd.sid].inv_t);
+    sc.top_k = __ldcg(&P.samp[cmd.sid].top_k);
+    sc.seed = __ldcg(&P.samp[cmd.sid].seed);
     for (int t = 0; t < cmd.n; t++) {
         const int pos = cmd.pos0 + t;
         if (cmd.op == OP_PREFILL) tok = __ldcg(P.tokbuf + t);
@@ -709,11 +774,13 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, cons
             gemv_dispatch<DT>(P, S, ring_it, ring, PH_HEAD, L, tok, pos, t);
             float *lg = nullptr;
             if (cmd.logits) lg = cmd.logits + (cmd.op == OP_PREFILL ? 0 : (size_t)t * P.V);
-            epilogue_head(P, S, lg);
+            if (sc.top_k > 1) sample_local(S, lg, sc.top_k, col_slices(P.K[PH_HEAD]), P.cand_tv, P.cand_ti, P.V);
+            else epilogue_head(P, S, lg);
             trace_mark(P, t, eh);
             grid_barrier(P, S, epoch, P.timeout_ns, 6);
             trace_mark(P, t, eh + 1);
-            tok = final_argmax(P);
+            tok = sc.top_k > 1 ? sample_global(S, P.nblk, P.cand_tv, P.cand_ti, sc.inv_t, sc.top_k, sc.seed, pos)
+                               : final_argmax(P);
             if (blockIdx.x == 0 && threadIdx.x == 0) {
                 if (cmd.out) cmd.out[cmd.op == OP_PREFILL ? 0 : t] = tok;
                 // no index wins an argmax over non-finite logits: the command fails (a later

@@ -280,6 +280,10 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
 
     P.splits = 1;
     if (b1) {  // ---- batch-1 kernel: static schedule and packed weights
+    if (nblk * KIE_TOPK_MAX > KIE_SAMPLE_VALS) {
+        eng->fail(KIE_ERR_ARG, "the batch-1 kernel's sampling supports at most %d SMs", KIE_SAMPLE_VALS / KIE_TOPK_MAX);
+        return bail(KIE_ERR_ARG);
+    }
     if (d > KIE_B1_DMAX) {
         eng->fail(KIE_ERR_ARG, "the batch-1 kernel supports d_model <= %d", KIE_B1_DMAX);
         return bail(KIE_ERR_ARG);
@@ -549,6 +553,15 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
     CKC(eng->alloc(&P.cnt, (size_t)Hkv * 4), "cudaMalloc counters");
     CKC(eng->alloc(&P.cand_val, (size_t)nblk * 4), "cudaMalloc candidates");
     CKC(eng->alloc(&P.cand_idx, (size_t)nblk * 4), "cudaMalloc candidates");
+    CKC(eng->alloc(&P.cand_tv, (size_t)nblk * KIE_TOPK_MAX * 4), "cudaMalloc sampling candidates");
+    CKC(eng->alloc(&P.cand_ti, (size_t)nblk * KIE_TOPK_MAX * 4), "cudaMalloc sampling candidates");
+    {
+        SampleCfg *samp = nullptr;
+        CKC(eng->alloc(&samp, (size_t)c.max_sessions * sizeof(SampleCfg)), "cudaMalloc sampling settings");
+        std::vector<SampleCfg> greedy(c.max_sessions, SampleCfg{1.f, 1, 0ull});
+        CKC(cudaMemcpy(samp, greedy.data(), greedy.size() * sizeof(SampleCfg), cudaMemcpyHostToDevice), "sampling settings");
+        P.samp = samp;
+    }
     CKC(eng->alloc(&P.tokbuf, (size_t)c.max_ctx * 4), "cudaMalloc token buffer");
     CKC(eng->alloc(&P.bar, 32), "cudaMalloc barrier");  // [0]: grid barrier, [2]: the residual-read split barrier
     P.rd = P.bar + 2;
@@ -709,18 +722,45 @@ static kie_status check_sid(kie_engine *eng, int32_t sid) {
     return KIE_OK;
 }
 
+static kie_status set_sampling(kie_engine *eng, int32_t sid, const SampleCfg &sc);
+
 extern "C" kie_status kie_session_open(kie_engine *eng, int32_t *sid) {
     kie_status s = check_live(eng);
     if (s != KIE_OK) return s;
     if (!sid) return KIE_ERR_ARG;
     for (int i = 0; i < eng->cfg.max_sessions; i++)
         if (!eng->sess_used[i]) {
+            if ((s = set_sampling(eng, i, SampleCfg{1.f, 1, 0ull})) != KIE_OK) return s;  // greedy
             eng->sess_used[i] = 1;
             eng->sess_len[i] = 0;
             *sid = i;
             return KIE_OK;
         }
     return eng->fail(KIE_ERR_CAPACITY, "all %d session slots are open", eng->cfg.max_sessions);
+}
+
+static kie_status set_sampling(kie_engine *eng, int32_t sid, const SampleCfg &sc) {
+    // the legacy default stream: it does not wait for the engine's (non-blocking) stream, where
+    // a resident kernel may sit idle between commands
+    const cudaError_t e = cudaMemcpy(const_cast<SampleCfg *>(eng->P.samp) + sid, &sc, sizeof sc, cudaMemcpyHostToDevice);
+    return e == cudaSuccess ? KIE_OK : eng->cuda_fail(e, "sampling settings");
+}
+
+extern "C" kie_status kie_session_sampling(kie_engine *eng, int32_t sid, const kie_sampling *sp) {
+    kie_status s = check_live(eng);
+    if (s != KIE_OK) return s;
+    if ((s = check_sid(eng, sid)) != KIE_OK) return s;
+    SampleCfg sc{1.f, 1, 0ull};
+    if (sp) {
+        if (sp->top_k < 1 || sp->top_k > std::min(KIE_TOPK_MAX, eng->cfg.vocab))
+            return eng->fail(KIE_ERR_ARG, "top_k must be in [1, %d]", std::min(KIE_TOPK_MAX, eng->cfg.vocab));
+        if (sp->top_k > 1) {
+            if (!(sp->temperature > 0.f) || !std::isfinite(sp->temperature) || !std::isfinite(1.f / sp->temperature))
+                return eng->fail(KIE_ERR_ARG, "temperature must be a positive finite number");
+            sc = SampleCfg{1.f / sp->temperature, sp->top_k, (unsigned long long)sp->seed};
+        }
+    }
+    return set_sampling(eng, sid, sc);
 }
 
 extern "C" kie_status kie_session_close(kie_engine *eng, int32_t sid) {

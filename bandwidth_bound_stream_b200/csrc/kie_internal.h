@@ -24,6 +24,14 @@
 // W[:, its columns] * its inputs into the residual.
 enum { PH_QKV = 0, PH_OF = 1, PH_GU = 2, PH_DF = 3, PH_HEAD = 4, KIE_NPH = 5 };
 
+// Per-session sampling of the next token (top_k <= 1: greedy argmax).
+struct SampleCfg {
+    float inv_t;               // 1 / temperature
+    int top_k;
+    unsigned long long seed;
+};
+#define KIE_SAMPLE_VALS 6144   // values one CTA selects from in shared memory (batch-1 kernel)
+
 // Commands of the resident kernel.
 enum { OP_NONE = 0, OP_DECODE = 1, OP_PREFILL = 2, OP_TICK = 3, OP_EXIT = 4 };
 
@@ -82,6 +90,9 @@ struct KieParams {
     unsigned *cnt;                  // [Hkv]
     float *cand_val;
     int *cand_idx;                  // [nblk]
+    const SampleCfg *samp;          // [max_sessions]
+    float *cand_tv;                 // [nblk][KIE_TOPK_MAX] each CTA's top-k logits (sampling)
+    int *cand_ti;                   // [nblk][KIE_TOPK_MAX] and their token ids
     int *tokbuf;                    // [max_ctx] device copy of command inputs
     unsigned long long *bar;        // grid barrier counter
     unsigned long long *rd;         // CTAs that have read the residual for the gate/up phase (split barrier)

@@ -31,6 +31,7 @@
 
 #include "kie_attn.cuh"
 #include "kie_device.cuh"
+#include "kie_sample.cuh"
 
 namespace {
 
@@ -873,10 +874,24 @@ __device__ void phase_argmax(const KieParams &P, MrShared &S, const KieCmd &cmd,
             S.red[8 + w] = __int_as_float(bi);
         }
         named_bar_sync(1, MR_WORKERS);
+        // the session's sampling (the variant beside argmax): top-k of the row's logits, then the
+        // draw of the step's position (attention's shared memory is free in this phase)
+        const int sid = __ldcg(P.mr_sid + m);
+        const int topk = __ldcg(&P.samp[sid].top_k);
+        const bool sample = topk > 1 && (cmd.op == OP_TICK || m == M - 1);
+        int sampled = 0;
+        if (sample) {
+            SampleScratch &SS = *reinterpret_cast<SampleScratch *>(&S.at);
+            block_topk<MR_WORKERS>(SS, P.V, topk, [&](int p) { return __ldcg(lg + p); }, [&](int p) { return p; });
+            if (tid < 32)
+                sampled = sample_pick(SS, topk, __ldcg(&P.samp[sid].inv_t),
+                                      sample_uniform(__ldcg(&P.samp[sid].seed), __ldcg(P.mr_pos + m)));
+        }
         if (tid == 0) {
             float v = S.red[0];
             int i = __float_as_int(S.red[8]);
             for (int k = 1; k < MR_WORKERS / 32; k++) amax(v, i, S.red[k], __float_as_int(S.red[8 + k]));
+            if (sample) i = sampled;
             if (i < 0 || i >= P.V) {  // non-finite logits (no index wins): fail the command
                 set_error(P.err, DERR_BAD_TOKEN, 0x41);
                 S.abort = 1;

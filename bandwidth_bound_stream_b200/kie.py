@@ -25,7 +25,9 @@ EXPORTS = ("kie_config_defaults", "kie_create", "kie_destroy", "kie_session_open
            "kie_session_length", "kie_session_rewind", "kie_session_kv", "kie_prefill", "kie_decode_step",
            "kie_generate", "kie_decode_launch", "kie_sync", "kie_tick", "kie_last_error", "kie_status_string",
            "kie_flash_decode", "kie_flash_decode_scratch_bytes", "kie_trace_enable", "kie_trace_read",
-           "kie_trace_events", "kie_flash_decode_noalloc", "kie_tick_launch", "kie_inject_fault")
+           "kie_trace_events", "kie_flash_decode_noalloc", "kie_tick_launch", "kie_inject_fault",
+           "kie_session_sampling")
+KIE_TOPK_MAX = 32
 KIE_FAULT_NONE, KIE_FAULT_BARRIER_SHORT = 0, 1
 
 
@@ -40,6 +42,10 @@ class KieConfig(ctypes.Structure):
 class KieWeights(ctypes.Structure):
     _fields_ = [("tok_emb", ctypes.c_void_p), ("layers", ctypes.POINTER(ctypes.c_void_p)),
                 ("final_norm", ctypes.c_void_p), ("lm_head", ctypes.c_void_p)]
+
+
+class KieSampling(ctypes.Structure):
+    _fields_ = [("temperature", ctypes.c_float), ("top_k", ctypes.c_int32), ("seed", ctypes.c_uint64)]
 
 
 class KieError(RuntimeError):
@@ -79,6 +85,7 @@ def _load():
         "kie_flash_decode_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, i64, i32, vp, vp]),
         "kie_tick_launch": (i32, [vp, i32, vp, vp, i32, vp, vp, vp]),
         "kie_inject_fault": (i32, [vp, i32]),
+        "kie_session_sampling": (i32, [vp, i32, P(KieSampling)]),
     }
     for name, (res, args) in sig.items():
         f = getattr(h, name)
@@ -157,6 +164,14 @@ class Engine:
 
     def session_rewind(self, sid: int, ctx: int):
         self._check(lib.kie_session_rewind(self.h, sid, ctx), "kie_session_rewind")
+
+    def session_sampling(self, sid: int, temperature: float = 1.0, top_k: int = 1, seed: int = 0, greedy: bool = False):
+        """Temperature / top-k sampling for a session (greedy=True restores argmax decoding)."""
+        if greedy:
+            self._check(lib.kie_session_sampling(self.h, sid, None), "kie_session_sampling")
+            return
+        sp = KieSampling(float(temperature), int(top_k), int(seed) & (2 ** 64 - 1))
+        self._check(lib.kie_session_sampling(self.h, sid, ctypes.byref(sp)), "kie_session_sampling")
 
     def session_kv(self, sid: int):
         k, v = ctypes.c_void_p(), ctypes.c_void_p()

@@ -211,6 +211,29 @@ kie_status kie_tick_launch(kie_engine *eng, int32_t n_sess, const int32_t *sids,
 enum { KIE_FAULT_NONE = 0, KIE_FAULT_BARRIER_SHORT = 1 };
 kie_status kie_inject_fault(kie_engine *eng, int32_t fault);
 
+/*
+ * Sampling of one session's next tokens, the variant beside greedy argmax (used by every call
+ * that produces its tokens: kie_prefill's first token, kie_decode_step, kie_generate,
+ * kie_decode_launch, kie_tick, kie_tick_launch). A step's token is a function of its logits
+ * and (temperature, top_k, seed, the step's position) alone:
+ *   candidates: the top_k largest logits, ordered by value (descending), then index (ascending);
+ *   weights:    exp((z_k - z_0) / temperature);
+ *   draw:       u = (output pos + 1 of splitmix64 started from state `seed`) >> 40, / 2^24, where
+ *               pos is the position of the step's input token;
+ *   token:      the first candidate whose cumulative weight exceeds u * (total weight).
+ * top_k = 1 is greedy argmax (temperature and seed unused). s = NULL restores greedy decoding;
+ * kie_session_open starts every session greedy. Errors: KIE_ERR_ARG for top_k outside
+ * [1, min(KIE_TOPK_MAX, vocab)] or, with top_k > 1, a temperature that is not a positive
+ * finite number. Non-finite candidate logits fail the command with KIE_ERR_DEVICE.
+ */
+#define KIE_TOPK_MAX 32
+typedef struct {
+    float temperature;
+    int32_t top_k;
+    uint64_t seed;
+} kie_sampling;
+kie_status kie_session_sampling(kie_engine *eng, int32_t sid, const kie_sampling *s);
+
 /* Copies the engine's last error message (NUL-terminated, truncated to len). */
 kie_status kie_last_error(kie_engine *eng, char *buf, int32_t len);
 
