@@ -50,6 +50,13 @@ typedef struct {
     const uint16_t *final_norm;       /* [d_model]         */
     const uint16_t *lm_head;          /* [vocab][d_model]  */
     const uint16_t *const *layers;    /* [n_layers * 9], order of the enum above */
+    /* Optional FP8 weights (all NULL for the 16-bit model): E4M3 codes and per-row scales of
+       every matrix (entries of the norm gains unused) and of the LM head; when q8 is set, every
+       matrix-vector product uses value(code) * scale[row] instead of the 16-bit weights. */
+    const uint8_t *const *q8;         /* [n_layers * 9] */
+    const float *const *q8_scale;     /* [n_layers * 9] */
+    const uint8_t *q8_head;
+    const float *q8_head_scale;
 } orc_weights;
 
 /* ---------------------------------------------------------------- storage types */
@@ -141,6 +148,90 @@ void orc_matvec(int32_t N, int32_t K, const uint16_t *W, int32_t dtype, const do
     }
 }
 
+/* ---------------------------------------------------------------- FP8 (E4M3) weights
+ *
+ * E4M3 (the "fn" variant of the OCP FP8 formats): 1 sign bit, 4 exponent bits with bias 7,
+ * 3 fraction bits; exponent 0 holds the subnormals m/8 * 2^-6; the all-ones exponent with
+ * fraction 111 is NaN and there are no infinities, so the largest finite value is
+ * 1.75 * 2^8 = 448.
+ */
+
+/* Exact value of an E4M3 code. */
+double orc_e4m3_value(uint8_t b) {
+    const int sign = b >> 7, e = (b >> 3) & 0xF, m = b & 7;
+    double v;
+    if (e == 0xF && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);            /* m/8 * 2^-6 */
+    else v = ldexp((double)(8 + m), e - 10);          /* (1 + m/8) * 2^(e-7) */
+    return sign ? -v : v;
+}
+
+/* fp32 value -> nearest E4M3 code, ties to the even code, finite results saturated at +-448
+   (a value beyond the largest finite code encodes as that code); NaN -> 0x7F. */
+uint8_t orc_e4m3_encode(float f) {
+    if (f != f) return 0x7F;
+    const uint8_t sign = signbit(f) ? 0x80 : 0;
+    double a = fabs((double)f);
+    if (a >= 448.0) return sign | 0x7E;
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e);                        /* a = fr * 2^e, fr in [0.5, 1) */
+    int exp8 = e - 1;                    /* a = 1.xxx * 2^exp8 */
+    if (exp8 < -6) exp8 = -6;            /* subnormal range: fixed step 2^-9 */
+    const double step = ldexp(1.0, exp8 - 3);
+    const double q = a / step;           /* exact: a has 24 bits, step a power of two */
+    const double fl = floor(q), rem = q - fl;
+    uint32_t qi = (uint32_t)fl;
+    if (rem > 0.5 || (rem == 0.5 && (qi & 1u))) qi++;
+    if (exp8 == -6 && qi < 8) return sign | (uint8_t)qi;   /* subnormal (or zero) */
+    if (qi == 16) { qi = 8; exp8++; }                       /* rounding carried */
+    if (exp8 > 8 || (exp8 == 8 && qi > 14)) return sign | 0x7E;
+    return sign | (uint8_t)(((exp8 + 7) << 3) | (qi & 7));
+}
+
+/* Per-row quantisation of a 16-bit matrix [N][K]: scale[n] = max_k |W[n][k]| / 448 (fp32; 1 for
+   an all-zero row) and q[n][k] = encode(W[n][k] / scale[n]), the quotient in fp32. */
+void orc_quantize_rows(int32_t N, int32_t K, const uint16_t *W, int32_t dtype, uint8_t *q, float *scale) {
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; n++) {
+        const uint16_t *row = W + (int64_t)n * K;
+        float amax = 0.f;
+        for (int k = 0; k < K; k++) {
+            const float a = (float)fabs(orc_value(row[k], dtype));
+            if (a > amax) amax = a;
+        }
+        const float s = amax > 0.f ? amax / 448.0f : 1.0f;
+        scale[n] = s;
+        for (int k = 0; k < K; k++) q[(int64_t)n * K + k] = orc_e4m3_encode((float)orc_value(row[k], dtype) / s);
+    }
+}
+
+/* y = (scale * Q) x for E4M3 codes Q [N][K] with per-row scales. */
+void orc_matvec_q8(int32_t N, int32_t K, const uint8_t *Q, const float *scale, const double *x, double *y) {
+    double tv[256];
+    for (int i = 0; i < 256; i++) tv[i] = orc_e4m3_value((uint8_t)i);
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; n++) {
+        const uint8_t *row = Q + (int64_t)n * K;
+        double acc = 0.0;
+        for (int k = 0; k < K; k++) acc += tv[row[k]] * x[k];
+        y[n] = (double)scale[n] * acc;
+    }
+}
+
+/* Matrix j of layer l (an enum index above) times x: the FP8 codes when the model has them. */
+static void layer_matvec(const orc_config *c, const orc_weights *w, int l, int j, int32_t N, int32_t K,
+                         const double *x, double *y) {
+    const int64_t i = (int64_t)l * W_PER_LAYER + j;
+    if (w->q8) orc_matvec_q8(N, K, w->q8[i], w->q8_scale[i], x, y);
+    else orc_matvec(N, K, w->layers[i], c->dtype, x, y);
+}
+
+static void head_matvec(const orc_config *c, const orc_weights *w, const double *x, double *y) {
+    if (w->q8) orc_matvec_q8(c->vocab, c->d_model, w->q8_head, w->q8_head_scale, x, y);
+    else orc_matvec(c->vocab, c->d_model, w->lm_head, c->dtype, x, y);
+}
+
 /* Rotary position embedding, rotate-half form: for i < D/2 the pair (v_i, v_{i+D/2})
    turns by the angle pos * theta^(-2i/D). */
 void orc_rope(int32_t D, int32_t pos, double theta, double *v) {
@@ -211,9 +302,9 @@ int32_t orc_step(const orc_config *c, const orc_weights *w, uint16_t *kcache, ui
     for (int l = 0; l < c->n_layers; l++) {
         const uint16_t *const *L = w->layers + (int64_t)l * W_PER_LAYER;
         orc_rmsnorm(d, x, L[W_ATTN_NORM], dt, c->rms_eps, h);
-        orc_matvec(Hq * D, d, L[W_Q], dt, h, q);
-        orc_matvec(Hkv * D, d, L[W_K], dt, h, k);
-        orc_matvec(Hkv * D, d, L[W_V], dt, h, v);
+        layer_matvec(c, w, l, W_Q, Hq * D, d, h, q);
+        layer_matvec(c, w, l, W_K, Hkv * D, d, h, k);
+        layer_matvec(c, w, l, W_V, Hkv * D, d, h, v);
         for (int hh = 0; hh < Hq; hh++) orc_rope(D, pos, c->rope_theta, q + hh * D);
         for (int g = 0; g < Hkv; g++) orc_rope(D, pos, c->rope_theta, k + g * D);
         for (int g = 0; g < Hkv; g++)
@@ -226,19 +317,19 @@ int32_t orc_step(const orc_config *c, const orc_weights *w, uint16_t *kcache, ui
             orc_attention(D, pos + 1, q + hh * D, kcache + kv_index(c, max_ctx, l, g, 0),
                           vcache + kv_index(c, max_ctx, l, g, 0), dt, o + hh * D);
         }
-        orc_matvec(d, Hq * D, L[W_O], dt, o, y);
+        layer_matvec(c, w, l, W_O, d, Hq * D, o, y);
         for (int i = 0; i < d; i++) x[i] += y[i];
         orc_rmsnorm(d, x, L[W_MLP_NORM], dt, c->rms_eps, h);
-        orc_matvec(F, d, L[W_GATE], dt, h, gt);
-        orc_matvec(F, d, L[W_UP], dt, h, up);
+        layer_matvec(c, w, l, W_GATE, F, d, h, gt);
+        layer_matvec(c, w, l, W_UP, F, d, h, up);
         for (int i = 0; i < F; i++) gt[i] = orc_silu(gt[i]) * up[i];
-        orc_matvec(d, F, L[W_DOWN], dt, gt, y);
+        layer_matvec(c, w, l, W_DOWN, d, F, gt, y);
         for (int i = 0; i < d; i++) x[i] += y[i];
     }
     int32_t tok = -2;
     if (logits) {
         orc_rmsnorm(d, x, w->final_norm, dt, c->rms_eps, h);
-        orc_matvec(c->vocab, d, w->lm_head, dt, h, logits);
+        head_matvec(c, w, h, logits);
         tok = orc_argmax(c->vocab, logits);
     }
     free(x); free(h); free(q); free(k); free(v); free(o); free(y); free(gt); free(up);
@@ -270,9 +361,9 @@ int32_t orc_forward_sequence(const orc_config *c, const orc_weights *w, int32_t 
         /* projections of every position; keys/values laid out [kv head][position][D] */
         for (int t = 0; t < n; t++) {
             orc_rmsnorm(d, X + (int64_t)t * d, L[W_ATTN_NORM], dt, c->rms_eps, H + (int64_t)t * d);
-            orc_matvec(Hq * D, d, L[W_Q], dt, H + (int64_t)t * d, Q + (int64_t)t * Hq * D);
-            orc_matvec(Hkv * D, d, L[W_K], dt, H + (int64_t)t * d, Kf);
-            orc_matvec(Hkv * D, d, L[W_V], dt, H + (int64_t)t * d, Vf);
+            layer_matvec(c, w, l, W_Q, Hq * D, d, H + (int64_t)t * d, Q + (int64_t)t * Hq * D);
+            layer_matvec(c, w, l, W_K, Hkv * D, d, H + (int64_t)t * d, Kf);
+            layer_matvec(c, w, l, W_V, Hkv * D, d, H + (int64_t)t * d, Vf);
             for (int hh = 0; hh < Hq; hh++) orc_rope(D, t, c->rope_theta, Q + ((int64_t)t * Hq + hh) * D);
             for (int g = 0; g < Hkv; g++) {
                 orc_rope(D, t, c->rope_theta, Kf + g * D);
@@ -291,19 +382,19 @@ int32_t orc_forward_sequence(const orc_config *c, const orc_weights *w, int32_t 
             }
         for (int t = 0; t < n; t++) {
             double *x = X + (int64_t)t * d;
-            orc_matvec(d, Hq * D, L[W_O], dt, O + (int64_t)t * Hq * D, Y);
+            layer_matvec(c, w, l, W_O, d, Hq * D, O + (int64_t)t * Hq * D, Y);
             for (int i = 0; i < d; i++) x[i] += Y[i];
             orc_rmsnorm(d, x, L[W_MLP_NORM], dt, c->rms_eps, H + (int64_t)t * d);
-            orc_matvec(F, d, L[W_GATE], dt, H + (int64_t)t * d, G);
-            orc_matvec(F, d, L[W_UP], dt, H + (int64_t)t * d, U);
+            layer_matvec(c, w, l, W_GATE, F, d, H + (int64_t)t * d, G);
+            layer_matvec(c, w, l, W_UP, F, d, H + (int64_t)t * d, U);
             for (int i = 0; i < F; i++) G[i] = orc_silu(G[i]) * U[i];
-            orc_matvec(d, F, L[W_DOWN], dt, G, Y);
+            layer_matvec(c, w, l, W_DOWN, d, F, G, Y);
             for (int i = 0; i < d; i++) x[i] += Y[i];
         }
     }
     for (int t = 0; t < n; t++) {
         orc_rmsnorm(d, X + (int64_t)t * d, w->final_norm, dt, c->rms_eps, H + (int64_t)t * d);
-        orc_matvec(c->vocab, d, w->lm_head, dt, H + (int64_t)t * d, logits + (int64_t)t * c->vocab);
+        head_matvec(c, w, H + (int64_t)t * d, logits + (int64_t)t * c->vocab);
     }
     free(X); free(H); free(Q); free(O); free(Kf); free(Vf); free(Ks); free(Vs); free(Y); free(G); free(U);
     return 0;

@@ -23,7 +23,9 @@ class _Config(ctypes.Structure):
 
 class _Weights(ctypes.Structure):
     _fields_ = [("tok_emb", ctypes.c_void_p), ("final_norm", ctypes.c_void_p), ("lm_head", ctypes.c_void_p),
-                ("layers", ctypes.POINTER(ctypes.c_void_p))]
+                ("layers", ctypes.POINTER(ctypes.c_void_p)), ("q8", ctypes.POINTER(ctypes.c_void_p)),
+                ("q8_scale", ctypes.POINTER(ctypes.c_void_p)), ("q8_head", ctypes.c_void_p),
+                ("q8_head_scale", ctypes.c_void_p)]
 
 
 def lib():
@@ -53,6 +55,12 @@ def lib():
         h.orc_uniform.argtypes = [ctypes.c_uint64, i32]
         h.orc_sample.restype = i32
         h.orc_sample.argtypes = [i32, vp, ctypes.c_double, i32, ctypes.c_double, vp]
+        h.orc_e4m3_value.restype = ctypes.c_double
+        h.orc_e4m3_value.argtypes = [ctypes.c_uint8]
+        h.orc_e4m3_encode.restype = ctypes.c_uint8
+        h.orc_e4m3_encode.argtypes = [ctypes.c_float]
+        h.orc_quantize_rows.argtypes = [i32, i32, vp, i32, vp, vp]
+        h.orc_matvec_q8.argtypes = [i32, i32, vp, vp, vp, vp]
         del dp
         lib.h = h
     return lib.h
@@ -136,6 +144,47 @@ def sample(logits, temperature: float, top_k: int, u: float):
     return tok, float(m[0])
 
 
+def e4m3_value(codes) -> np.ndarray:
+    c = np.atleast_1d(np.asarray(codes, dtype=np.uint8))
+    return np.array([lib().orc_e4m3_value(int(x)) for x in c.ravel()]).reshape(c.shape)
+
+
+def e4m3_encode(values) -> np.ndarray:
+    """fp32 values (given as any floats, converted to fp32 first) -> E4M3 codes."""
+    v = np.atleast_1d(np.asarray(values, dtype=np.float32))
+    return np.array([lib().orc_e4m3_encode(float(x)) for x in v.ravel()], dtype=np.uint8).reshape(v.shape)
+
+
+def quantize_rows(W_bits: np.ndarray, dtype: int):
+    """Per-row E4M3 quantisation of a 16-bit matrix: (codes [N][K] uint8, scales [N] fp32)."""
+    W = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    N, K = W.shape
+    q = np.empty((N, K), dtype=np.uint8)
+    sc = np.empty(N, dtype=np.float32)
+    lib().orc_quantize_rows(N, K, _ptr(W), dtype, _ptr(q), _ptr(sc))
+    return q, sc
+
+
+def matvec_q8(Q: np.ndarray, scale: np.ndarray, x: np.ndarray) -> np.ndarray:
+    Q = np.ascontiguousarray(Q, dtype=np.uint8)
+    sc = np.ascontiguousarray(scale, dtype=np.float32)
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    N, K = Q.shape
+    y = np.empty(N)
+    lib().orc_matvec_q8(N, K, _ptr(Q), _ptr(sc), _ptr(x), _ptr(y))
+    return y
+
+
+FP8_MATRICES = ("wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down")
+
+
+def quantize_model(cfg, weights: dict) -> dict:
+    """The FP8 form of a model's weights: every matrix of every layer and the LM head quantised
+    per row ({"layers": [{name: (codes, scales)}], "lm_head": (codes, scales)})."""
+    return {"layers": [{n: quantize_rows(layer[n], cfg.dtype) for n in FP8_MATRICES} for layer in weights["layers"]],
+            "lm_head": quantize_rows(weights["lm_head"], cfg.dtype)}
+
+
 def num_threads() -> int:
     return int(lib().orc_num_threads())
 
@@ -150,7 +199,9 @@ class OracleModel:
     {"tok_emb", "final_norm", "lm_head", "layers": [ {name: array} per layer ]}.
     """
 
-    def __init__(self, cfg, weights: dict, max_ctx: int):
+    def __init__(self, cfg, weights: dict, max_ctx: int, q8: dict | None = None):
+        """q8 (optional): the FP8 form of the weights (quantize_model); every matrix-vector
+        product then uses the E4M3 codes times their row scales."""
         self.cfg = cfg
         self.max_ctx = max_ctx
         self._c = _Config(cfg.n_layers, cfg.d_model, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, cfg.ffn,
@@ -169,6 +220,28 @@ class OracleModel:
         self._keep += [emb, fin, head]
         self._w = _Weights(_ptr(emb), _ptr(fin), _ptr(head),
                            ctypes.cast(self._layer_ptrs, ctypes.POINTER(ctypes.c_void_p)))
+        if q8 is not None:
+            qp, sp = [], []
+            for layer in q8["layers"]:
+                for name in LAYER_TENSORS:
+                    if name in layer:
+                        qa = np.ascontiguousarray(layer[name][0], dtype=np.uint8)
+                        sa = np.ascontiguousarray(layer[name][1], dtype=np.float32)
+                        self._keep += [qa, sa]
+                        qp.append(_ptr(qa))
+                        sp.append(_ptr(sa))
+                    else:
+                        qp.append(None)
+                        sp.append(None)
+            self._q8_ptrs = (ctypes.c_void_p * len(qp))(*qp)
+            self._q8_sc = (ctypes.c_void_p * len(sp))(*sp)
+            hq = np.ascontiguousarray(q8["lm_head"][0], dtype=np.uint8)
+            hs = np.ascontiguousarray(q8["lm_head"][1], dtype=np.float32)
+            self._keep += [hq, hs]
+            self._w.q8 = ctypes.cast(self._q8_ptrs, ctypes.POINTER(ctypes.c_void_p))
+            self._w.q8_scale = ctypes.cast(self._q8_sc, ctypes.POINTER(ctypes.c_void_p))
+            self._w.q8_head = _ptr(hq)
+            self._w.q8_head_scale = _ptr(hs)
         shape = (cfg.n_layers, cfg.n_kv_heads, max_ctx, cfg.head_dim)
         self.k_cache = np.zeros(shape, dtype=np.uint16)
         self.v_cache = np.zeros(shape, dtype=np.uint16)

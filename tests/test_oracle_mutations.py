@@ -46,16 +46,26 @@ SLIPS = {
         ("orc_rmsnorm(d, X + (int64_t)t * d, w->final_norm,",
          "orc_rmsnorm(d, X + (int64_t)t * d, w->layers[(int64_t)(c->n_layers - 1) * W_PER_LAYER + W_MLP_NORM],")],
     "no_final_norm": [("        orc_rmsnorm(d, x, w->final_norm, dt, c->rms_eps, h);\n"
-                       "        orc_matvec(c->vocab, d, w->lm_head, dt, h, logits);",
-                       "        orc_matvec(c->vocab, d, w->lm_head, dt, x, logits);"),
-                      ("        orc_matvec(c->vocab, d, w->lm_head, dt, H + (int64_t)t * d, logits + (int64_t)t * c->vocab);",
-                       "        orc_matvec(c->vocab, d, w->lm_head, dt, X + (int64_t)t * d, logits + (int64_t)t * c->vocab);")],
+                       "        head_matvec(c, w, h, logits);",
+                       "        head_matvec(c, w, x, logits);"),
+                      ("        head_matvec(c, w, H + (int64_t)t * d, logits + (int64_t)t * c->vocab);",
+                       "        head_matvec(c, w, X + (int64_t)t * d, logits + (int64_t)t * c->vocab);")],
     "residual_overwritten_after_attention": [
-        ("        orc_matvec(d, Hq * D, L[W_O], dt, o, y);\n        for (int i = 0; i < d; i++) x[i] += y[i];",
-         "        orc_matvec(d, Hq * D, L[W_O], dt, o, y);\n        for (int i = 0; i < d; i++) x[i] = y[i];"),
+        ("        layer_matvec(c, w, l, W_O, d, Hq * D, o, y);\n        for (int i = 0; i < d; i++) x[i] += y[i];",
+         "        layer_matvec(c, w, l, W_O, d, Hq * D, o, y);\n        for (int i = 0; i < d; i++) x[i] = y[i];"),
         ("            for (int i = 0; i < d; i++) x[i] += Y[i];\n            orc_rmsnorm",
          "            for (int i = 0; i < d; i++) x[i] = Y[i];\n            orc_rmsnorm")],
-    "lm_head_is_the_embedding": [("orc_matvec(c->vocab, d, w->lm_head,", "orc_matvec(c->vocab, d, w->tok_emb,")],
+    "lm_head_is_the_embedding": [("else orc_matvec(c->vocab, c->d_model, w->lm_head,", "else orc_matvec(c->vocab, c->d_model, w->tok_emb,")],
+    # FP8 weights
+    "e4m3_exponent_bias": [("else v = ldexp((double)(8 + m), e - 10);", "else v = ldexp((double)(8 + m), e - 11);")],
+    "e4m3_encode_rounds_half_up": [("    if (rem > 0.5 || (rem == 0.5 && (qi & 1u))) qi++;\n    if (exp8 == -6",
+                                    "    if (rem >= 0.5) qi++;\n    if (exp8 == -6")],
+    "e4m3_scale_from_mean": [("const float s = amax > 0.f ? amax / 448.0f : 1.0f;", "const float s = amax > 0.f ? amax / 440.0f : 1.0f;")],
+    "q8_scale_divides": [("y[n] = (double)scale[n] * acc;", "y[n] = acc / (double)scale[n];")],
+    "q8_gate_is_up": [("    if (w->q8) orc_matvec_q8(N, K, w->q8[i], w->q8_scale[i], x, y);",
+                       "    if (w->q8) orc_matvec_q8(N, K, w->q8[j == W_GATE ? i + 1 : i], w->q8_scale[j == W_GATE ? i + 1 : i], x, y);")],
+    "q8_head_reads_16bit_weights": [("if (w->q8) orc_matvec_q8(c->vocab, c->d_model, w->q8_head, w->q8_head_scale, x, y);",
+                                     "if (0 && w->q8) orc_matvec_q8(c->vocab, c->d_model, w->q8_head, w->q8_head_scale, x, y);")],
     "embedding_row_off_by_one": [("x[i] = orc_value(w->tok_emb[(int64_t)token * d + i], dt);",
                                   "x[i] = orc_value(w->tok_emb[(int64_t)(token + (token + 1 < c->vocab)) * d + i], dt);")],
     "rope_position_off_by_one": [("orc_rope(D, pos, c->rope_theta, q + hh * D);", "orc_rope(D, pos + 1, c->rope_theta, q + hh * D);"),

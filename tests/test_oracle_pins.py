@@ -419,3 +419,114 @@ def test_sample_rejects_bad_arguments_and_non_finite_candidates():
     assert orc.sample(np.array([np.nan, 1.0, 0.0]), 1.0, 3, 0.2)[0] == -2
     assert orc.sample(np.array([np.inf, 1.0, 0.0]), 1.0, 2, 0.2)[0] == -2
     assert orc.sample(np.array([np.nan, 1.0, 0.0]), 1.0, 2, 0.2)[0] in (1, 2)  # NaN ranks below every number
+
+
+# ------------------------------------------------------------------ FP8 (E4M3) weights
+
+def test_e4m3_values_match_torch_for_every_pattern():
+    want = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    got = orc.e4m3_value(np.arange(256))
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    assert np.array_equal(got[~np.isnan(got)], want[~np.isnan(want)])
+
+
+def test_e4m3_encode_matches_torch_rounding_and_saturates():
+    """Round to nearest, ties to the even code, against torch's conversion for values in range,
+    including every exact midpoint between neighbouring codes (ties) and the subnormals; beyond
+    the largest finite value (448) the encoding saturates (torch's conversion returns NaN past
+    464, so that part is pinned by value)."""
+    codes = np.arange(256, dtype=np.uint8)
+    vals = orc.e4m3_value(codes)
+    fin = np.sort(np.unique(vals[np.isfinite(vals)]))
+    mids = (fin[:-1] + fin[1:]) / 2
+    rng = np.random.default_rng(3)
+    x = np.concatenate([fin, mids, rng.normal(size=5000) * 60, rng.normal(size=2000) * 0.01]).astype(np.float32)
+    x = x[np.abs(x) <= 448]
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(orc.e4m3_encode(x), want)
+    assert list(orc.e4m3_encode([449.0, 463.9, 1e6, -1e6, float("inf")])) == [0x7E, 0x7E, 0x7E, 0xFE, 0x7E]
+    assert orc.e4m3_encode([float("nan")])[0] == 0x7F
+
+
+def test_quantize_rows_closed_forms():
+    rng = np.random.default_rng(4)
+    for dtype in (FP16, BF16):
+        W = synth.normal_u16(77, 0x51, 24 * 96, dtype).reshape(24, 96)
+        W[5] = 0  # an all-zero row
+        q, s = orc.quantize_rows(W, dtype)
+        w = orc.value(W, dtype)
+        amax = np.abs(w).max(axis=1)
+        want_s = np.where(amax > 0, (amax.astype(np.float32) / np.float32(448.0)).astype(np.float32), np.float32(1.0))
+        assert np.array_equal(s, want_s)
+        assert (q[5] == 0).all() and s[5] == 1.0
+        deq = orc.e4m3_value(q) * s[:, None].astype(np.float64)
+        # each code is the nearest to w / s: within half a code step of it (steps: 2^-9 below 2^-6)
+        ratio = (w / s[:, None].astype(np.float64))
+        e = np.floor(np.log2(np.maximum(np.abs(ratio), 2.0 ** -6)))
+        half_step = 2.0 ** (e - 3) / 2
+        assert (np.abs(orc.e4m3_value(q) - ratio) <= half_step * (1 + 1e-6) + 1e-12).all()
+        # the largest element of each non-zero row encodes as +-448
+        rows = np.arange(24)[amax > 0]
+        top = np.abs(w[rows]).argmax(axis=1)
+        assert (np.abs(orc.e4m3_value(q[rows, top])) == 448.0).all()
+        assert np.isfinite(deq).all()
+    del rng
+
+
+def test_matvec_q8_matches_numpy():
+    rng = np.random.default_rng(6)
+    q = rng.integers(0, 256, size=(33, 70)).astype(np.uint8)
+    q[(q & 0x7F) == 0x7F] = 0x01  # no NaN codes
+    s = rng.uniform(0.01, 2.0, 33).astype(np.float32)
+    x = rng.normal(size=70)
+    want = (orc.e4m3_value(q) * s[:, None].astype(np.float64)) @ x
+    np.testing.assert_allclose(orc.matvec_q8(q, s, x), want, rtol=1e-13, atol=1e-13)
+
+
+def test_fp8_step_equals_the_16bit_step_on_the_same_values():
+    """A model whose 16-bit matrices equal value(code) * 2^k for E4M3 codes and power-of-two row
+    scales 2^k (exact in fp16): the FP8 path (codes and scales) gives the same logits, bit for
+    bit, at every step. A scale applied to the wrong rows, or a matrix taken from the wrong
+    slot, would differ."""
+    from oracle.oracle import OracleModel
+    m = synth.TINY
+    w = synth.model_weights(m)
+    rng = np.random.default_rng(12)
+
+    def on_grid(W):
+        codes = orc.e4m3_encode(orc.value(W, m.dtype) * 50.0)
+        codes[(codes & 0x7F) == 0x7F] = 0  # no NaN
+        k = rng.integers(-3, 4, size=W.shape[0]).astype(np.float64)
+        vals = orc.e4m3_value(codes) * np.exp2(k)[:, None] / 64.0
+        return codes, (np.exp2(k) / 64.0).astype(np.float32), orc.store(vals, m.dtype)
+
+    q8 = {"layers": [], "lm_head": None}
+    w16 = {"tok_emb": w["tok_emb"], "final_norm": w["final_norm"], "layers": []}
+    for layer in w["layers"]:
+        ql, wl = {}, dict(layer)
+        for name in orc.FP8_MATRICES:
+            c, sc, bits = on_grid(layer[name])
+            ql[name] = (c, sc)
+            wl[name] = bits
+        q8["layers"].append(ql)
+        w16["layers"].append(wl)
+    c, sc, bits = on_grid(w["lm_head"])
+    q8["lm_head"] = (c, sc)
+    w16["lm_head"] = bits
+    a, b = OracleModel(m, w16, 16), OracleModel(m, w16, 16, q8=q8)
+    prompt = synth.prompt(m, 6)
+    for t in prompt:
+        assert np.array_equal(a.step(int(t)), b.step(int(t)))
+    # and the FP8 path reads the codes of every matrix: changing one matrix's codes (same 16-bit
+    # weights) changes the logits (after a 6-token prompt: at position 0 the query and key
+    # matrices cannot show, attention over one position returns its value)
+    base = OracleModel(m, w16, 16, q8=q8).prefill(prompt)
+    for where in [(0, n) for n in orc.FP8_MATRICES] + [("head", None)]:
+        q = {"layers": [dict(l) for l in q8["layers"]], "lm_head": q8["lm_head"]}
+        if where[0] == "head":
+            c, sc = q["lm_head"]
+            q["lm_head"] = (c ^ 1, sc)
+        else:
+            c, sc = q["layers"][0][where[1]]
+            q["layers"][0][where[1]] = (c ^ 1, sc)
+        assert not np.array_equal(OracleModel(m, w16, 16, q8=q).prefill(prompt), base), where
