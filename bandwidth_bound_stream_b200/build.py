@@ -16,8 +16,8 @@ INCLUDE = os.path.join(ROOT, "include")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
-KIE_SOURCES = ["kie_engine.cu", "kie_b1.cu", "kie_mr.cu", "kie_attn.cu"]
-KIE_HEADERS = ["kie_device.cuh", "kie_internal.h", "kie_attn.cuh"]
+KIE_SOURCES = ["kie_engine.cu", "kie_b1.cu", "kie_mr.cu", "kie_attn.cu", "kie_fp8.cu"]
+KIE_HEADERS = ["kie_device.cuh", "kie_internal.h", "kie_attn.cuh", "kie_sample.cuh"]
 
 
 def _run(cmd):

@@ -40,6 +40,7 @@
 //
 // RMSNorm: every CTA reads all of x for a normed phase, so each computes the sum of squares
 // itself (one CTA-wide reduction) instead of publishing partial sums.
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
@@ -52,6 +53,40 @@ namespace {
 constexpr int RING_BYTES = KIE_NSLOT * KIE_SLOT_BYTES;
 
 constexpr int WPART_FLOATS = 8 * KIE_ROWACC_MAX;  // column-slice partials: [slices][rows] flattened
+
+// 8 streamed weights -> 8 floats: 16-byte vector of the storage dtype, or 8-byte vector of E4M3
+// codes (element 0 in the lowest byte)
+template <int DT, bool F8>
+struct WVec;
+template <int DT>
+struct WVec<DT, false> {
+    using T = uint4;
+    static constexpr int BYTES = 16;
+    static __device__ __forceinline__ void cvt(const T &w, float *f) { cvt8<DT>(w, f); }
+};
+template <int DT>
+struct WVec<DT, true> {
+    using T = uint2;
+    static constexpr int BYTES = 8;
+    static __device__ __forceinline__ void cvt(const T &w, float *f) {
+        const uint32_t u[2] = {w.x, w.y};
+#pragma unroll
+        for (int j = 0; j < 2; j++) {
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(u[j] >> (16 * h)), __NV_E4M3);
+                const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(&r));
+                f[4 * j + 2 * h] = v.x;
+                f[4 * j + 2 * h + 1] = v.y;
+            }
+        }
+    }
+};
+
+// offsets of a layer's phase blocks in the E4M3 row scales (P.wsc)
+__device__ __forceinline__ int sc_off_o(const KieParams &P) { return (P.Hq + 2 * P.Hkv) * P.D; }
+__device__ __forceinline__ int sc_off_gu(const KieParams &P) { return sc_off_o(P) + P.d; }
+__device__ __forceinline__ int sc_off_down(const KieParams &P) { return sc_off_gu(P) + 2 * P.F; }
 
 struct __align__(16) B1Shared {
     union {
@@ -198,7 +233,7 @@ __device__ bool chunk_next(const KieParams &P, const B1Shared &S, const KieCmd &
         const int n = S.row1[it.ph] - S.row0[it.ph];
         if (it.r < n) {
             const int nr = min(P.cr[it.ph], n - it.r);
-            bytes = (uint32_t)(is_fold(it.ph) ? nr * P.d * 16 : nr * P.K[it.ph] * 2);
+            bytes = (uint32_t)(is_fold(it.ph) ? nr * P.d * 8 * P.wesz : nr * P.K[it.ph] * P.wesz);
             addr = it.g;
             it.g += bytes;
             it.r += nr;
@@ -277,13 +312,25 @@ __device__ void produce(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint
 // Runs one GEMV phase (QKV, gate/up or head) over this CTA's rows: the RMSNorm of its input
 // (the embedding row at layer 0, else the residual x), then the rows; row partials land in
 // S.wpart (see rowsum).
-template <int DT, int NV, int CR, int CS>
+// With E4M3 weights, rsc receives the row scales the phase's epilogue applies: rows 2*tid and
+// 2*tid + 1 of this CTA (the QKV and gate/up pairs), or rows tid and tid + 512 (head).
+template <int DT, bool F8, int NV, int CR, int CS>
 __device__ void gemv_phase(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring, int ph, int l,
-                           int tok, int pos, int t) {
+                           int tok, int pos, int t, float2 &rsc) {
+    using WV = WVec<DT, F8>;
+    constexpr int ESZ = F8 ? 1 : 2;
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int K = P.K[ph];
     const int rows = S.row1[ph] - S.row0[ph];
     const bool from_emb = (ph == PH_QKV && l == 0);
+    rsc = make_float2(1.f, 1.f);
+    if (F8) {  // issued first: the loads complete under the row work
+        const float *sc = P.wsc + (ph == PH_HEAD ? (size_t)P.L * P.sc_stride
+                                                 : (size_t)l * P.sc_stride + (ph == PH_GU ? sc_off_gu(P) : 0)) + S.row0[ph];
+        const int r0 = ph == PH_HEAD ? tid : 2 * tid, r1 = ph == PH_HEAD ? tid + KIE_CONS_THREADS : 2 * tid + 1;
+        if (r0 < rows) rsc.x = __ldg(sc + r0);
+        if (r1 < rows) rsc.y = __ldg(sc + r1);
+    }
 
     // the QKV epilogue needs this position's rotation: fetch it now, under the row work
     if (ph == PH_QKV && tid < (P.D >> 1)) S.rope_s[tid] = P.rope[(size_t)pos * (P.D >> 1) + tid];
@@ -335,9 +382,9 @@ __device__ void gemv_phase(const KieParams &P, B1Shared &S, uint32_t &ring_it, c
     unsigned long long waited = 0;
     const int grp = w / CS, ws = w % CS;
     constexpr int STRIDE = WPART_FLOATS / CS;  // row capacity of one slice's partials
-    for (int c0 = 0; c0 < rows; c0 += GROUPS * CR) {
-        const int r0 = c0 + grp * CR;  // this group's first row in the chunk
-        const int nr = max(0, min(CR, rows - r0));
+    // a chunk holds SUB blocks of GROUPS * CR rows (two with one-byte weights)
+    constexpr int SUB = 2 / ESZ;
+    for (int c0 = 0; c0 < rows; c0 += SUB * GROUPS * CR) {
         const uint32_t slot = ring_it % KIE_NSLOT, par = (ring_it / KIE_NSLOT) & 1u;
         ring_it++;
         bool have = !S.abort && mbar_try_wait(&S.full[slot], par);
@@ -352,32 +399,39 @@ __device__ void gemv_phase(const KieParams &P, B1Shared &S, uint32_t &ring_it, c
             S.abort = 1;
             continue;  // keep the control flow; the command ends at the next barrier
         }
-        const uint8_t *base = ring + (size_t)slot * KIE_SLOT_BYTES + ((size_t)grp * CR * K + (size_t)ws * kslice) * 2;
-        float acc[8];
 #pragma unroll
-        for (int r = 0; r < 8; r++) acc[r] = 0.f;
+        for (int sub = 0; sub < SUB; sub++) {
+            const int r0 = c0 + (sub * GROUPS + grp) * CR;  // this group's first row in the block
+            const int nr = max(0, min(CR, rows - r0));
+            const uint8_t *base = ring + (size_t)slot * KIE_SLOT_BYTES +
+                                  ((size_t)(sub * GROUPS + grp) * CR * K + (size_t)ws * kslice) * ESZ;
+            float acc[8];
 #pragma unroll
-        for (int r = 0; r < CR; r++) {
-            if (r < nr) {
-                const uint8_t *rowp = base + (size_t)r * K * 2;
+            for (int r = 0; r < 8; r++) acc[r] = 0.f;
 #pragma unroll
-                for (int i = 0; i < NV; i++) {
-                    const int v = lane + 32 * i;
-                    if (v < nvec) {
-                        const uint4 wv = *reinterpret_cast<const uint4 *>(rowp + v * 16);
-                        float f[8];
-                        cvt8<DT>(wv, f);
+            for (int r = 0; r < CR; r++) {
+                if (r < nr) {
+                    const uint8_t *rowp = base + (size_t)r * K * ESZ;
 #pragma unroll
-                        for (int e = 0; e < 8; e++) acc[r] = fmaf(f[e], h[i][e], acc[r]);
+                    for (int i = 0; i < NV; i++) {
+                        const int v = lane + 32 * i;
+                        if (v < nvec) {
+                            float f[8];
+                            WV::cvt(*reinterpret_cast<const typename WV::T *>(rowp + v * WV::BYTES), f);
+#pragma unroll
+                            for (int e = 0; e < 8; e++) acc[r] = fmaf(f[e], h[i][e], acc[r]);
+                        }
                     }
                 }
             }
+            if (sub == SUB - 1) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.empty[slot]);  // shared-memory reads of the chunk are done
+            }
+            const float s = warp_reduce_rows<CR>(acc);
+            constexpr int LPR = 32 / CR;
+            if ((lane % LPR) == 0 && lane / LPR < nr) S.wpart[ws * STRIDE + r0 + lane / LPR] = s;
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.empty[slot]);  // shared-memory reads of the chunk are done
-        const float s = warp_reduce_rows<CR>(acc);
-        constexpr int LPR = 32 / CR;
-        if ((lane % LPR) == 0 && lane / LPR < nr) S.wpart[ws * STRIDE + r0 + lane / LPR] = s;
     }
     if (tid == 0) S.wait_cons += waited;
     named_bar_sync(1, KIE_CONS_THREADS);
@@ -391,21 +445,24 @@ __device__ __forceinline__ float rowsum(const B1Shared &S, int r, int cs) {
     return v;
 }
 
-template <int DT>
-__device__ __forceinline__ void gemv_dispatch(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring, int ph, int l,
-                              int tok, int pos, int t) {
+template <int DT, bool F8>
+__device__ __forceinline__ float2 gemv_dispatch(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring,
+                                                int ph, int l, int tok, int pos, int t) {
     const int K = P.K[ph];
-    if (K <= 2048) gemv_phase<DT, 1, 8, 8>(P, S, ring_it, ring, ph, l, tok, pos, t);
-    else gemv_phase<DT, 2, 4, 8>(P, S, ring_it, ring, ph, l, tok, pos, t);  // K <= 4096
+    float2 rsc;
+    if (K <= 2048) gemv_phase<DT, F8, 1, 8, 8>(P, S, ring_it, ring, ph, l, tok, pos, t, rsc);
+    else gemv_phase<DT, F8, 2, 4, 8>(P, S, ring_it, ring, ph, l, tok, pos, t, rsc);  // K <= 4096
+    return rsc;
 }
 
 // --------------------------------------------------------------- consumer: folds
 
 // One fold (O or down): this CTA's 8-column groups of W arrive as [group][d rows][8], and
 // S.fold_in holds 8 inputs per group. Thread t accumulates rows t + 512 j over all groups.
-template <int DT, int RPT>
+template <int DT, bool F8, int RPT>
 __device__ void fold_rows(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring, int ph,
                           float (&acc)[RPT]) {
+    using WV = WVec<DT, F8>;
     const int tid = threadIdx.x, lane = tid & 31;
     const int d = P.d, ng = S.row1[ph] - S.row0[ph], cpc = P.cr[ph];
 #pragma unroll
@@ -433,7 +490,7 @@ __device__ void fold_rows(const KieParams &P, B1Shared &S, uint32_t &ring_it, co
                 const int r = tid + KIE_CONS_THREADS * j;
                 if (r < d) {
                     float f[8];
-                    cvt8<DT>(*reinterpret_cast<const uint4 *>(base + ((size_t)gi * d + r) * 16), f);
+                    WV::cvt(*reinterpret_cast<const typename WV::T *>(base + ((size_t)gi * d + r) * WV::BYTES), f);
 #pragma unroll
                     for (int e = 0; e < 8; e++) acc[j] = fmaf(f[e], in[e], acc[j]);
                 }
@@ -444,14 +501,26 @@ __device__ void fold_rows(const KieParams &P, B1Shared &S, uint32_t &ring_it, co
     }
 }
 
-// x[r] += acc for this thread's rows (fp32 atomics: the folds of all CTAs meet in x)
+// x[r] += acc (times the row's scale with E4M3 weights) for this thread's rows (fp32 atomics:
+// the folds of all CTAs meet in x)
 template <int RPT>
-__device__ __forceinline__ void fold_commit(const KieParams &P, const B1Shared &S, const float (&acc)[RPT], int ph) {
+__device__ __forceinline__ void fold_commit(const KieParams &P, const B1Shared &S, const float (&acc)[RPT], int ph,
+                                            const float (&scl)[RPT]) {
     if (S.abort || S.row1[ph] == S.row0[ph]) return;
 #pragma unroll
     for (int j = 0; j < RPT; j++) {
         const int r = threadIdx.x + KIE_CONS_THREADS * j;
-        if (r < P.d) atomicAdd(P.x + r, acc[j]);
+        if (r < P.d) atomicAdd(P.x + r, acc[j] * scl[j]);
+    }
+}
+
+// the fold's row scales (E4M3 weights), loaded before the fold so they arrive under its work
+template <bool F8, int RPT>
+__device__ __forceinline__ void fold_scales(const KieParams &P, int l, int off, float (&scl)[RPT]) {
+#pragma unroll
+    for (int j = 0; j < RPT; j++) {
+        const int r = threadIdx.x + KIE_CONS_THREADS * j;
+        scl[j] = (F8 && r < P.d) ? __ldg(P.wsc + (size_t)l * P.sc_stride + off + r) : 1.f;
     }
 }
 
@@ -461,14 +530,14 @@ __device__ __forceinline__ void attention_prefetch(const KieParams &P, B1Shared 
 
 // q/k rows come in rotation pairs (dim i, dim i + D/2); v rows use the same pairing.
 template <int DT>
-__device__ void epilogue_qkv(const KieParams &P, B1Shared &S, int l, int sid, int pos, int tok) {
+__device__ void epilogue_qkv(const KieParams &P, B1Shared &S, int l, int sid, int pos, int tok, float2 rsc) {
     const int D = P.D, half = D >> 1, qd = P.Hq * D, kvd = P.Hkv * D;
     const int rbeg = S.row0[PH_QKV], npair = (S.row1[PH_QKV] - rbeg) >> 1;
     const size_t sess = (size_t)sid * P.sess_stride;
     for (int p = threadIdx.x; p < npair; p += KIE_CONS_THREADS) {
         const int r = rbeg + 2 * p;
         const int cs = col_slices(P.K[PH_QKV]);
-        const float a = rowsum(S, 2 * p, cs), b = rowsum(S, 2 * p + 1, cs);
+        const float a = rowsum(S, 2 * p, cs) * rsc.x, b = rowsum(S, 2 * p + 1, cs) * rsc.y;  // (p == tid)
         const int i = (r % D) >> 1;
         if (r < qd + kvd) {
             const float2 cs = S.rope_s[i];
@@ -519,12 +588,12 @@ __device__ __forceinline__ void attention_prefetch(const KieParams &P, B1Shared 
 }
 
 // u = silu(gate) * up for this CTA's pairs, into the down fold's inputs
-__device__ void epilogue_gu(const KieParams &P, B1Shared &S, int l, int sid, int pos) {
+__device__ void epilogue_gu(const KieParams &P, B1Shared &S, int l, int sid, int pos, float2 rsc) {
     if (l + 1 < P.L) attention_prefetch(P, S, l + 1, sid, pos);
     const int npair = (S.row1[PH_GU] - S.row0[PH_GU]) >> 1;
     const int cs = col_slices(P.K[PH_GU]);
     for (int p = threadIdx.x; p < npair; p += KIE_CONS_THREADS) {
-        const float g = rowsum(S, 2 * p, cs), up = rowsum(S, 2 * p + 1, cs);
+        const float g = rowsum(S, 2 * p, cs) * rsc.x, up = rowsum(S, 2 * p + 1, cs) * rsc.y;  // (p == tid)
         S.fold_in[p] = g / (1.f + expf(-g)) * up;
     }
 }
@@ -546,13 +615,13 @@ __device__ void warp_argmax(float &v, int &i) {
 }
 
 // logits of this CTA's rows -> optional output, local argmax -> candidate slot
-__device__ void epilogue_head(const KieParams &P, B1Shared &S, float *logits) {
+__device__ void epilogue_head(const KieParams &P, B1Shared &S, float *logits, float2 rsc) {
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int rbeg = S.row0[PH_HEAD], n = S.row1[PH_HEAD] - rbeg;
     float bv = -CUDART_INF_F;
     int bi = 0x7fffffff;
-    for (int r = tid; r < n; r += KIE_CONS_THREADS) {
-        const float v = rowsum(S, r, col_slices(P.K[PH_HEAD]));
+    for (int r = tid; r < n; r += KIE_CONS_THREADS) {  // rows tid and tid + 512 (n <= 1024)
+        const float v = rowsum(S, r, col_slices(P.K[PH_HEAD])) * (r == tid ? rsc.x : rsc.y);
         if (logits) logits[rbeg + r] = v;
         argmax_combine(bv, bi, v, rbeg + r);
     }
@@ -590,12 +659,12 @@ __device__ int final_argmax(const KieParams &P) {
 // (Arguments by value: a reference to the kernel's parameter block would make the kernel keep
 // a copy of it in local memory.)
 __device__ __noinline__ void sample_local(B1Shared &S, float *logits, int k, int cs, float *cand_tv, int *cand_ti,
-                                          int V) {
+                                          int V, float2 rsc) {
     const int tid = threadIdx.x;
     const int rbeg = S.row0[PH_HEAD], n = S.row1[PH_HEAD] - rbeg;
     float v0 = 0.f, v1 = 0.f;  // rows tid and tid + 512 (n <= 1024)
-    if (tid < n) v0 = rowsum(S, tid, cs);
-    if (tid + KIE_CONS_THREADS < n) v1 = rowsum(S, tid + KIE_CONS_THREADS, cs);
+    if (tid < n) v0 = rowsum(S, tid, cs) * rsc.x;
+    if (tid + KIE_CONS_THREADS < n) v1 = rowsum(S, tid + KIE_CONS_THREADS, cs) * rsc.y;
     if (logits) {
         if (tid < n) logits[rbeg + tid] = v0;
         if (tid + KIE_CONS_THREADS < n) logits[rbeg + tid + KIE_CONS_THREADS] = v1;
@@ -674,6 +743,9 @@ __device__ void attention_step(const KieParams &P, B1Shared &S, int l, int sid, 
     const bool have = unit < P.Hkv * P.splits;
     grid_barrier(P, S, epoch, P.timeout_ns, 1);
     trace_mark(P, t, e + 2);
+    if (P.wesz == 1)  // the O fold's row scales (E4M3 weights) wait in L1 through attention
+        for (int r = threadIdx.x; r < P.d; r += KIE_CONS_THREADS)
+            prefetch_l1(P.wsc + (size_t)l * P.sc_stride + sc_off_o(P) + r);
     if (threadIdx.x == 0) S.at.t_unit = 0;
     if (have && !S.abort) {
         for (int hoff = 0; hoff < P.G; hoff += GC) attn_unit<DT, GC, KIE_CONS_WARPS>(A, S.at, unit, P.G, hoff);
@@ -681,44 +753,47 @@ __device__ void attention_step(const KieParams &P, B1Shared &S, int l, int sid, 
 }
 
 // the two folds of a layer and the down fold's split barrier, by rows per thread
-template <int DT, int RPT>
-__device__ __forceinline__ void o_fold(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring) {
-    float acc[RPT];
-    fold_rows<DT, RPT>(P, S, ring_it, ring, PH_OF, acc);
-    fold_commit<RPT>(P, S, acc, PH_OF);
+template <int DT, bool F8, int RPT>
+__device__ __forceinline__ void o_fold(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring, int l) {
+    float acc[RPT], scl[RPT];
+    fold_scales<F8, RPT>(P, l, sc_off_o(P), scl);
+    fold_rows<DT, F8, RPT>(P, S, ring_it, ring, PH_OF, acc);
+    fold_commit<RPT>(P, S, acc, PH_OF, scl);
 }
 
-template <int DT, int RPT>
+template <int DT, bool F8, int RPT>
 __device__ __forceinline__ void down_fold(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring,
-                                          unsigned long long rd_epoch, int t, int e) {
-    float acc[RPT];
-    fold_rows<DT, RPT>(P, S, ring_it, ring, PH_DF, acc);
+                                          int l, unsigned long long rd_epoch, int t, int e) {
+    float acc[RPT], scl[RPT];
+    fold_scales<F8, RPT>(P, l, sc_off_down(P), scl);
+    fold_rows<DT, F8, RPT>(P, S, ring_it, ring, PH_DF, acc);
     residual_read_wait(P, S, rd_epoch);  // every CTA has read x for its gate/up norm
     trace_mark(P, t, e + 10);
-    fold_commit<RPT>(P, S, acc, PH_DF);
+    fold_commit<RPT>(P, S, acc, PH_DF, scl);
 }
 
 // rows per thread of a fold (d <= 4096): 1, 2, 4 or 8
-template <int DT>
-__device__ __forceinline__ void o_fold_any(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring) {
-    if (P.d <= 512) o_fold<DT, 1>(P, S, ring_it, ring);
-    else if (P.d <= 1024) o_fold<DT, 2>(P, S, ring_it, ring);
-    else if (P.d <= 2048) o_fold<DT, 4>(P, S, ring_it, ring);
-    else o_fold<DT, 8>(P, S, ring_it, ring);
+template <int DT, bool F8>
+__device__ __forceinline__ void o_fold_any(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring,
+                                           int l) {
+    if (P.d <= 512) o_fold<DT, F8, 1>(P, S, ring_it, ring, l);
+    else if (P.d <= 1024) o_fold<DT, F8, 2>(P, S, ring_it, ring, l);
+    else if (P.d <= 2048) o_fold<DT, F8, 4>(P, S, ring_it, ring, l);
+    else o_fold<DT, F8, 8>(P, S, ring_it, ring, l);
 }
 
-template <int DT>
+template <int DT, bool F8>
 __device__ __forceinline__ void down_fold_any(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring,
-                                              unsigned long long rd_epoch, int t, int e) {
-    if (P.d <= 512) down_fold<DT, 1>(P, S, ring_it, ring, rd_epoch, t, e);
-    else if (P.d <= 1024) down_fold<DT, 2>(P, S, ring_it, ring, rd_epoch, t, e);
-    else if (P.d <= 2048) down_fold<DT, 4>(P, S, ring_it, ring, rd_epoch, t, e);
-    else down_fold<DT, 8>(P, S, ring_it, ring, rd_epoch, t, e);
+                                              int l, unsigned long long rd_epoch, int t, int e) {
+    if (P.d <= 512) down_fold<DT, F8, 1>(P, S, ring_it, ring, l, rd_epoch, t, e);
+    else if (P.d <= 1024) down_fold<DT, F8, 2>(P, S, ring_it, ring, l, rd_epoch, t, e);
+    else if (P.d <= 2048) down_fold<DT, F8, 4>(P, S, ring_it, ring, l, rd_epoch, t, e);
+    else down_fold<DT, F8, 8>(P, S, ring_it, ring, l, rd_epoch, t, e);
 }
 
 // --------------------------------------------------------------- consumer: one command
 
-template <int DT>
+template <int DT, bool F8>
 __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring, const KieCmd &cmd,
                         unsigned long long &epoch, unsigned long long &rd_epoch, uint32_t &att_use) {
     int tok = cmd.in_tok;
@@ -744,38 +819,38 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, cons
         for (int l = 0; l < L; l++) {
             const int e = 1 + 16 * l;
             // A: QKV
-            gemv_dispatch<DT>(P, S, ring_it, ring, PH_QKV, l, tok, pos, t);
+            const float2 sq = gemv_dispatch<DT, F8>(P, S, ring_it, ring, PH_QKV, l, tok, pos, t);
             trace_mark(P, t, e);
-            epilogue_qkv<DT>(P, S, l, cmd.sid, pos, tok);
+            epilogue_qkv<DT>(P, S, l, cmd.sid, pos, tok, sq);
             trace_mark(P, t, e + 1);
             // B: attention, then the O fold
             attention_step<DT, 2>(P, S, l, cmd.sid, pos, epoch, t, e, att_use);  // also serves G == 1
             if (P.trace && t < P.trace_tokens && threadIdx.x == 0)  // end of this CTA's positions (0: no unit)
                 P.trace[((size_t)blockIdx.x * P.trace_tokens + t) * P.trace_events + e + 15] = S.at.t_unit;
             trace_mark(P, t, e + 3);
-            o_fold_any<DT>(P, S, ring_it, ring);
+            o_fold_any<DT, F8>(P, S, ring_it, ring, l);
             trace_mark(P, t, e + 4);
             grid_barrier(P, S, epoch, P.timeout_ns, 2);
             trace_mark(P, t, e + 5);
             // C: gate/up, then the down fold
-            gemv_dispatch<DT>(P, S, ring_it, ring, PH_GU, l, tok, pos, t);
+            const float2 sg = gemv_dispatch<DT, F8>(P, S, ring_it, ring, PH_GU, l, tok, pos, t);
             residual_read_arrive(P, S);  // this CTA's reads of x are done
             rd_epoch++;
             trace_mark(P, t, e + 6);
-            epilogue_gu(P, S, l, cmd.sid, pos);
+            epilogue_gu(P, S, l, cmd.sid, pos, sg);
             trace_mark(P, t, e + 7);
-            down_fold_any<DT>(P, S, ring_it, ring, rd_epoch, t, e);
+            down_fold_any<DT, F8>(P, S, ring_it, ring, l, rd_epoch, t, e);
             trace_mark(P, t, e + 8);
             grid_barrier(P, S, epoch, P.timeout_ns, 3);
             trace_mark(P, t, e + 9);
         }
         const int eh = 1 + 16 * L;
         if (head) {
-            gemv_dispatch<DT>(P, S, ring_it, ring, PH_HEAD, L, tok, pos, t);
+            const float2 sh = gemv_dispatch<DT, F8>(P, S, ring_it, ring, PH_HEAD, L, tok, pos, t);
             float *lg = nullptr;
             if (cmd.logits) lg = cmd.logits + (cmd.op == OP_PREFILL ? 0 : (size_t)t * P.V);
-            if (sc.top_k > 1) sample_local(S, lg, sc.top_k, col_slices(P.K[PH_HEAD]), P.cand_tv, P.cand_ti, P.V);
-            else epilogue_head(P, S, lg);
+            if (sc.top_k > 1) sample_local(S, lg, sc.top_k, col_slices(P.K[PH_HEAD]), P.cand_tv, P.cand_ti, P.V, sh);
+            else epilogue_head(P, S, lg, sh);
             trace_mark(P, t, eh);
             grid_barrier(P, S, epoch, P.timeout_ns, 6);
             trace_mark(P, t, eh + 1);
@@ -797,7 +872,7 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, cons
 
 // --------------------------------------------------------------- the kernel
 
-template <int DT>
+template <int DT, bool F8>
 __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, KieCmd one, int resident) {
     extern __shared__ __align__(1024) uint8_t smem[];
     B1Shared &S = *reinterpret_cast<B1Shared *>(smem + RING_BYTES);
@@ -864,7 +939,7 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
         if (tid >= KIE_CONS_THREADS) {
             if (tid == KIE_CONS_THREADS) produce(P, S, ring_it, smem, cmd);
         } else {
-            consume<DT>(P, S, ring_it, smem, cmd, epoch, rd_epoch, att_use);
+            consume<DT, F8>(P, S, ring_it, smem, cmd, epoch, rd_epoch, att_use);
         }
         __syncthreads();
         if (resident && blockIdx.x == 0 && tid == 0) {
@@ -888,18 +963,18 @@ size_t kie_b1_smem_bytes() { return RING_BYTES + sizeof(B1Shared); }
 int kie_b1_chunk_rows(int K) { return (KIE_CONS_WARPS / col_slices(K)) * rows_per_group(K); }
 int kie_b1_max_rows(int K) { return WPART_FLOATS / col_slices(K); }
 
-cudaError_t kie_b1_prepare(int dtype) {
-    const int smem = (int)kie_b1_smem_bytes();
-    return dtype == KIE_BF16
-               ? cudaFuncSetAttribute(kie_b1_kernel<KIE_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
-               : cudaFuncSetAttribute(kie_b1_kernel<KIE_FP16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+// the kernel instantiation for a storage dtype and weight format
+static const void *b1_fn(int dtype, bool f8) {
+    if (dtype == KIE_BF16) return f8 ? (const void *)kie_b1_kernel<KIE_BF16, true> : (const void *)kie_b1_kernel<KIE_BF16, false>;
+    return f8 ? (const void *)kie_b1_kernel<KIE_FP16, true> : (const void *)kie_b1_kernel<KIE_FP16, false>;
 }
 
-cudaError_t kie_b1_occupancy(int dtype, int *blocks_per_sm) {
-    const size_t smem = kie_b1_smem_bytes();
-    return dtype == KIE_BF16
-               ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, kie_b1_kernel<KIE_BF16>, KIE_THREADS, smem)
-               : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, kie_b1_kernel<KIE_FP16>, KIE_THREADS, smem);
+cudaError_t kie_b1_prepare(int dtype, bool f8) {
+    return cudaFuncSetAttribute(b1_fn(dtype, f8), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kie_b1_smem_bytes());
+}
+
+cudaError_t kie_b1_occupancy(int dtype, bool f8, int *blocks_per_sm) {
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, b1_fn(dtype, f8), KIE_THREADS, kie_b1_smem_bytes());
 }
 
 cudaError_t kie_b1_launch(const KieParams &P, const KieCmd &one, int resident, cudaStream_t stream) {
@@ -910,8 +985,8 @@ cudaError_t kie_b1_launch(const KieParams &P, const KieCmd &one, int resident, c
     KieCmd c = one;
     int r = resident;
     void *args[] = {&p, &c, &r};
-    const void *fn = P.dtype == KIE_BF16 ? (const void *)kie_b1_kernel<KIE_BF16> : (const void *)kie_b1_kernel<KIE_FP16>;
-    return cudaLaunchCooperativeKernel(fn, dim3(P.nblk), dim3(KIE_THREADS), args, kie_b1_smem_bytes(), stream);
+    return cudaLaunchCooperativeKernel(b1_fn(P.dtype, P.wesz == 1), dim3(P.nblk), dim3(KIE_THREADS), args,
+                                       kie_b1_smem_bytes(), stream);
 }
 
 }  // extern "C++"

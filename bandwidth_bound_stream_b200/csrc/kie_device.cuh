@@ -115,6 +115,9 @@ KIE_DEV void l2_warm_line(void *dst, const void *src) {
 }
 KIE_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+// Hint: bring the line holding p into this SM's L1.
+KIE_DEV void prefetch_l1(const void *p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
+
 // Hint: bring the 128-byte line holding p into L2 (through the load/store unit).
 KIE_DEV void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 

@@ -26,14 +26,16 @@
 size_t kie_b1_smem_bytes();
 int kie_b1_chunk_rows(int K);
 int kie_b1_max_rows(int K);
-cudaError_t kie_b1_prepare(int dtype);
-cudaError_t kie_b1_occupancy(int dtype, int *blocks_per_sm);
+cudaError_t kie_b1_prepare(int dtype, bool f8);
+cudaError_t kie_b1_occupancy(int dtype, bool f8, int *blocks_per_sm);
 cudaError_t kie_b1_launch(const KieParams &P, const KieCmd &one, int resident, cudaStream_t stream);
 size_t kie_mr_smem_bytes();
 cudaError_t kie_mr_prepare(int dtype);
 cudaError_t kie_mr_occupancy(int dtype, int *blocks_per_sm);
 cudaError_t kie_mr_launch(const KieParams &P, const KieCmd &one, int resident, cudaStream_t stream);
 cudaError_t kie_mr_repack(const void *tiles, long long n, uint8_t *arena, cudaStream_t stream);
+cudaError_t kie_fp8_quantize(const void *w, long long rows, int cols, int dtype, uint8_t *q, float *scale,
+                             cudaStream_t stream);
 size_t kie_mr_tile_src_bytes();
 void kie_mr_tile_src(void *dst, const void *const *src3, int n0, int n1, long long off, int N, int K, int rb, int ks);
 
@@ -59,7 +61,7 @@ struct FoldCopy {
     long long dst;
     const uint8_t *src;
     long long ld;
-    int col0, ng, rows;
+    int col0, ng, rows, esz;  // esz: bytes per element (2, or 1 for E4M3 codes)
 };
 
 __global__ void fold_pack_kernel(const FoldCopy *fc, long long n, uint8_t *arena) {
@@ -68,8 +70,9 @@ __global__ void fold_pack_kernel(const FoldCopy *fc, long long n, uint8_t *arena
         const long long vecs = (long long)f.ng * f.rows;
         for (long long v = threadIdx.x; v < vecs; v += blockDim.x) {
             const long long g = v / f.rows, r = v % f.rows;
-            *reinterpret_cast<uint4 *>(arena + f.dst + v * 16) =
-                *reinterpret_cast<const uint4 *>(f.src + r * f.ld + (f.col0 + 8 * g) * 2);
+            const uint8_t *src = f.src + r * f.ld + (long long)(f.col0 + 8 * g) * f.esz;
+            if (f.esz == 2) *reinterpret_cast<uint4 *>(arena + f.dst + v * 16) = *reinterpret_cast<const uint4 *>(src);
+            else *reinterpret_cast<uint2 *>(arena + f.dst + v * 8) = *reinterpret_cast<const uint2 *>(src);
         }
     }
 }
@@ -198,6 +201,8 @@ static const char *shape_error(const kie_config &c) {
     if (c.max_sessions <= 0 || c.max_ctx <= 0) return "max_sessions and max_ctx must be positive";
     if (c.timeout_ms <= 0 || c.idle_ms <= 0) return "timeouts must be positive";
     if (!(c.modes & (KIE_MODE_BATCH1 | KIE_MODE_TICK))) return "modes must enable at least one kernel";
+    if (c.weight_fp8 != 0 && (c.weight_fp8 != 1 || c.modes != KIE_MODE_BATCH1))
+        return "weight_fp8 must be 0 or 1, and 1 needs modes == KIE_MODE_BATCH1";
     return nullptr;
 }
 
@@ -206,16 +211,16 @@ static void partition(int *row0, int n_units, int unit, int nblk) {
     for (int c = 0; c <= nblk; c++) row0[c] = (int)((long long)c * n_units / nblk) * unit;
 }
 
-// Source row of logical row r of each phase (rotation pairs and gate/up pairs interleaved).
-static const uint8_t *qkv_src(const kie_config &c, const void *const *L, int r) {
+// Logical row r of the QKV phase (rotation pairs (i, i + D/2) adjacent, v rows paired the same
+// way): its matrix (1 = wq, 2 = wk, 3 = wv in a layer's weight list) and row in that matrix.
+static void qkv_row(const kie_config &c, int r, int *mat, int *row) {
     const int D = c.head_dim, qd = c.n_heads * D, kvd = c.n_kv_heads * D;
     const int j = r % D, dim = (j >> 1) + (j & 1) * (D >> 1);
-    const void *m;
     int head;
-    if (r < qd) { m = L[1]; head = r / D; }
-    else if (r < qd + kvd) { m = L[2]; head = (r - qd) / D; }
-    else { m = L[3]; head = (r - qd - kvd) / D; }
-    return static_cast<const uint8_t *>(m) + ((size_t)head * D + dim) * c.d_model * 2;
+    if (r < qd) { *mat = 1; head = r / D; }
+    else if (r < qd + kvd) { *mat = 2; head = (r - qd) / D; }
+    else { *mat = 3; head = (r - qd - kvd) / D; }
+    *row = head * D + dim;
 }
 
 extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, kie_engine **out) {
@@ -247,10 +252,10 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
         return bail(KIE_ERR_CUDA);
     }
     if (b1) {
-        e = kie_b1_prepare(c.dtype);
+        e = kie_b1_prepare(c.dtype, c.weight_fp8 != 0);
         if (e != cudaSuccess) return bail(eng->cuda_fail(e, "kernel attributes"));
         int occ = 0;
-        e = kie_b1_occupancy(c.dtype, &occ);
+        e = kie_b1_occupancy(c.dtype, c.weight_fp8 != 0, &occ);
         if (e != cudaSuccess || occ < 1)
             return bail(eng->cuda_fail(e == cudaSuccess ? cudaErrorInvalidConfiguration : e,
                                        "batch-1 megakernel does not fit on an SM"));
@@ -291,6 +296,9 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
     // attention splits: about one (kv head, split) unit per CTA
     P.splits = std::max(1, nblk / Hkv);
     const int E = G * D;  // attention outputs of one kv head (its query heads)
+    const bool f8 = c.weight_fp8 != 0;
+    const int esz = f8 ? 1 : 2;
+    P.wesz = esz;
     const int Kph[KIE_NPH] = {d, 8, d, 8, d};
     std::vector<int> row0((size_t)KIE_NPH * (nblk + 1));
     partition(&row0[PH_QKV * (nblk + 1)], (qd + 2 * kvd) / 2, 2, nblk);  // rotation pairs
@@ -308,7 +316,7 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
         P.K[ph] = Kph[ph];
         const bool fold = (ph == PH_OF || ph == PH_DF);
         // rows per ring chunk (even for the paired phases), or 8-column groups per chunk of a fold
-        P.cr[ph] = fold ? KIE_SLOT_BYTES / (d * 16) : kie_b1_chunk_rows(Kph[ph]);
+        P.cr[ph] = fold ? KIE_SLOT_BYTES / (d * 8 * esz) : kie_b1_chunk_rows(Kph[ph]) * (2 / esz);
         const int lim = fold ? KIE_FOLD_MAX / 8 : kie_b1_max_rows(Kph[ph]);
         for (int cc = 0; cc < nblk; cc++)
             if (range(ph, cc) > lim) {
@@ -321,13 +329,93 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
     // column groups, its gate/up rows, its Wd column groups; then its LM-head rows)
     std::vector<long long> seg_off(nblk + 1, 0);
     for (int cc = 0; cc < nblk; cc++) {
-        const long long lb = (long long)range(PH_QKV, cc) * d * 2 + (long long)range(PH_OF, cc) * d * 16 +
-                             (long long)range(PH_GU, cc) * d * 2 + (long long)range(PH_DF, cc) * d * 16;
-        seg_off[cc + 1] = seg_off[cc] + (long long)L * lb + (long long)range(PH_HEAD, cc) * d * 2;
+        const long long lb = ((long long)range(PH_QKV, cc) * d + (long long)range(PH_OF, cc) * d * 8 +
+                              (long long)range(PH_GU, cc) * d + (long long)range(PH_DF, cc) * d * 8) * esz;
+        seg_off[cc + 1] = seg_off[cc] + (long long)L * lb + (long long)range(PH_HEAD, cc) * d * esz;
     }
     uint8_t *wpack = nullptr;
     CKC(eng->alloc(&wpack, (size_t)seg_off[nblk]), "cudaMalloc packed weights");
     P.wpack = wpack;
+    // E4M3 codes and row scales of every matrix (layer l, list index j; the LM head at [L][0]),
+    // made once here and freed after the repack
+    std::vector<uint8_t *> qcodes((size_t)(L + 1) * 9, nullptr);
+    std::vector<float *> qscale((size_t)(L + 1) * 9, nullptr);
+    auto free_q = [&]() {
+        for (auto p : qcodes) cudaFree(p);
+        for (auto p : qscale) cudaFree(p);
+    };
+    auto mat_shape = [&](int j, int *N, int *K) {
+        switch (j) {
+            case 1: *N = qd; *K = d; break;
+            case 2: case 3: *N = kvd; *K = d; break;
+            case 4: *N = d; *K = qd; break;
+            case 6: case 7: *N = F; *K = d; break;
+            default: *N = d; *K = F; break;  // 8: w_down
+        }
+    };
+    if (f8) {
+        for (int l = 0; l <= L && e == cudaSuccess; l++)
+            for (int j = (l < L ? 1 : 0); j < (l < L ? 9 : 1) && e == cudaSuccess; j++) {
+                if (j == 5) continue;  // the MLP norm gain
+                int N = V, K = d;
+                if (l < L) mat_shape(j, &N, &K);
+                const void *src = l < L ? w->layers[(size_t)9 * l + j] : w->lm_head;
+                e = cudaMalloc(&qcodes[(size_t)9 * l + j], (size_t)N * K);
+                if (e == cudaSuccess) e = cudaMalloc(&qscale[(size_t)9 * l + j], (size_t)N * 4);
+                if (e == cudaSuccess) e = kie_fp8_quantize(src, N, K, c.dtype, qcodes[(size_t)9 * l + j],
+                                                           qscale[(size_t)9 * l + j], 0);
+            }
+        if (e == cudaSuccess) e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) {
+            free_q();
+            return bail(eng->cuda_fail(e, "weight quantisation"));
+        }
+        // the row scales in each phase's logical row order: per layer [QKV | O | gate/up | down],
+        // then the LM head
+        P.sc_stride = qd + 2 * kvd + d + 2 * F + d;
+        std::vector<float> sc((size_t)L * P.sc_stride + V);
+        std::vector<std::vector<float>> hs((size_t)(L + 1) * 9);
+        for (int l = 0; l <= L && e == cudaSuccess; l++)
+            for (int j = (l < L ? 1 : 0); j < (l < L ? 9 : 1) && e == cudaSuccess; j++) {
+                if (j == 5) continue;
+                int N = V, K = d;
+                if (l < L) mat_shape(j, &N, &K);
+                hs[(size_t)9 * l + j].resize(N);
+                e = cudaMemcpy(hs[(size_t)9 * l + j].data(), qscale[(size_t)9 * l + j], (size_t)N * 4, cudaMemcpyDeviceToHost);
+            }
+        if (e != cudaSuccess) {
+            free_q();
+            return bail(eng->cuda_fail(e, "reading the row scales"));
+        }
+        for (int l = 0; l < L; l++) {
+            float *o = sc.data() + (size_t)l * P.sc_stride;
+            for (int r = 0; r < qd + 2 * kvd; r++) {
+                int m, row;
+                qkv_row(c, r, &m, &row);
+                o[r] = hs[(size_t)9 * l + m][row];
+            }
+            o += qd + 2 * kvd;
+            for (int r = 0; r < d; r++) o[r] = hs[(size_t)9 * l + 4][r];
+            o += d;
+            for (int r = 0; r < 2 * F; r++) o[r] = hs[(size_t)9 * l + ((r & 1) ? 7 : 6)][r >> 1];
+            o += 2 * F;
+            for (int r = 0; r < d; r++) o[r] = hs[(size_t)9 * l + 8][r];
+        }
+        for (int r = 0; r < V; r++) sc[(size_t)L * P.sc_stride + r] = hs[(size_t)9 * L][r];
+        float *d_sc = nullptr;
+        e = eng->alloc(&d_sc, sc.size() * 4);
+        if (e == cudaSuccess) e = cudaMemcpy(d_sc, sc.data(), sc.size() * 4, cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) {
+            free_q();
+            return bail(eng->cuda_fail(e, "row scales"));
+        }
+        P.wsc = d_sc;
+    }
+    // a matrix's rows as the repack reads them: the 16-bit weights, or their codes
+    auto mat_src = [&](int l, int j) -> const uint8_t * {
+        if (f8) return qcodes[(size_t)9 * l + j];
+        return static_cast<const uint8_t *>(l < L ? w->layers[(size_t)9 * l + j] : w->lm_head);
+    };
     {
         std::vector<RowCopy> rc;   // whole rows (GEMV phases)
         std::vector<FoldCopy> fc;  // column-group blocks (folds)
@@ -340,34 +428,39 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
                     const int a = row0[ph * (nblk + 1) + cc], n = range(ph, cc);
                     if (ph == PH_OF || ph == PH_DF) {
                         if (n > 0) {
-                            const uint8_t *src = static_cast<const uint8_t *>(Lw[ph == PH_OF ? 4 : 8]);
-                            fc.push_back({off, src, (long long)(ph == PH_OF ? qd : F) * 2, 8 * a, n, d});
+                            const uint8_t *src = mat_src(l, ph == PH_OF ? 4 : 8);
+                            fc.push_back({off, src, (long long)(ph == PH_OF ? qd : F) * esz, 8 * a, n, d, esz});
                         }
-                        off += (long long)n * d * 16;
+                        off += (long long)n * d * 8 * esz;
                         continue;
                     }
                     const int K = Kph[ph];
                     for (int r = a; r < a + n; r++) {
                         const uint8_t *src;
-                        switch (ph) {
-                            case PH_QKV: src = qkv_src(c, Lw, r); break;
-                            case PH_GU: src = static_cast<const uint8_t *>(Lw[(r & 1) ? 7 : 6]) + (size_t)(r >> 1) * K * 2; break;
-                            default: src = static_cast<const uint8_t *>(w->lm_head) + (size_t)r * K * 2; break;
+                        if (ph == PH_QKV) {
+                            int m, row;
+                            qkv_row(c, r, &m, &row);
+                            src = mat_src(l, m) + (size_t)row * K * esz;
+                        } else if (ph == PH_GU) {
+                            src = mat_src(l, (r & 1) ? 7 : 6) + (size_t)(r >> 1) * K * esz;
+                        } else {
+                            src = mat_src(L, 0) + (size_t)r * K * esz;
                         }
-                        rc.push_back({off, src, (long long)K * 2});
-                        off += (long long)K * 2;
+                        rc.push_back({off, src, (long long)K * esz});
+                        off += (long long)K * esz;
                     }
                 }
             }
             if (off != seg_off[cc + 1]) {
+                free_q();
                 eng->fail(KIE_ERR_ARG, "internal: segment size mismatch");
                 return bail(KIE_ERR_ARG);
             }
         }
         RowCopy *d_rc = nullptr;
         FoldCopy *d_fc = nullptr;
-        CKC(cudaMalloc(&d_rc, rc.size() * sizeof(RowCopy)), "cudaMalloc repack list");
-        e = cudaMalloc(&d_fc, std::max<size_t>(1, fc.size()) * sizeof(FoldCopy));
+        e = cudaMalloc(&d_rc, rc.size() * sizeof(RowCopy));
+        if (e == cudaSuccess) e = cudaMalloc(&d_fc, std::max<size_t>(1, fc.size()) * sizeof(FoldCopy));
         if (e == cudaSuccess) e = cudaMemcpy(d_rc, rc.data(), rc.size() * sizeof(RowCopy), cudaMemcpyHostToDevice);
         if (e == cudaSuccess && !fc.empty())
             e = cudaMemcpy(d_fc, fc.data(), fc.size() * sizeof(FoldCopy), cudaMemcpyHostToDevice);
@@ -379,6 +472,7 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
         if (e == cudaSuccess) e = cudaDeviceSynchronize();
         cudaFree(d_rc);
         cudaFree(d_fc);
+        free_q();
         if (e != cudaSuccess) return bail(eng->cuda_fail(e, "weight repack"));
     }
     int *d_row0 = nullptr;

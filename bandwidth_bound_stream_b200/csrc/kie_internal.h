@@ -75,6 +75,9 @@ struct KieParams {
     int K[KIE_NPH];                 // row length (elements) per phase (8 for folds)
     // batch-1 packed weights: CTA c streams [seg_off[c], seg_off[c+1]) once per token
     const uint8_t *wpack;
+    int wesz;                       // bytes per streamed weight: 2 (dtype), or 1 (E4M3 codes)
+    const float *wsc;               // E4M3 row scales: per layer [QKV rows | d | gate/up rows | d], then [V]
+    int sc_stride;                  // floats per layer in wsc
     const int *row0;                // [KIE_NPH][nblk+1] partition: rows (GEMV phases), 8-column groups (folds)
     const long long *seg_off;       // [nblk+1]
     // unpacked small weights

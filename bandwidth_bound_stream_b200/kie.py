@@ -26,7 +26,7 @@ EXPORTS = ("kie_config_defaults", "kie_create", "kie_destroy", "kie_session_open
            "kie_generate", "kie_decode_launch", "kie_sync", "kie_tick", "kie_last_error", "kie_status_string",
            "kie_flash_decode", "kie_flash_decode_scratch_bytes", "kie_trace_enable", "kie_trace_read",
            "kie_trace_events", "kie_flash_decode_noalloc", "kie_tick_launch", "kie_inject_fault",
-           "kie_session_sampling")
+           "kie_session_sampling", "kie_quantize_e4m3")
 KIE_TOPK_MAX = 32
 KIE_FAULT_NONE, KIE_FAULT_BARRIER_SHORT = 0, 1
 
@@ -36,7 +36,7 @@ class KieConfig(ctypes.Structure):
                                                "vocab")] + \
                [("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float)] + \
                [(n, ctypes.c_int32) for n in ("dtype", "max_sessions", "max_ctx", "timeout_ms", "idle_ms", "modes",
-                                               "device")]
+                                               "device", "weight_fp8")]
 
 
 class KieWeights(ctypes.Structure):
@@ -86,6 +86,7 @@ def _load():
         "kie_tick_launch": (i32, [vp, i32, vp, vp, i32, vp, vp, vp]),
         "kie_inject_fault": (i32, [vp, i32]),
         "kie_session_sampling": (i32, [vp, i32, P(KieSampling)]),
+        "kie_quantize_e4m3": (i32, [vp, i64, i32, i32, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(h, name)
@@ -103,7 +104,7 @@ def _ptr(a: np.ndarray):
 
 
 def config(model, max_sessions: int = 1, max_ctx: int = 4096, timeout_ms: int = 10000, idle_ms: int = 200,
-           modes: int = KIE_MODE_BATCH1, device: int = 0) -> KieConfig:
+           modes: int = KIE_MODE_BATCH1, device: int = 0, weight_fp8: bool = False) -> KieConfig:
     """A kie_config for a model shape (any object with the shape attributes of synth.ModelConfig)."""
     c = KieConfig()
     lib.kie_config_defaults(ctypes.byref(c))
@@ -112,6 +113,7 @@ def config(model, max_sessions: int = 1, max_ctx: int = 4096, timeout_ms: int = 
     c.rms_eps, c.rope_theta = model.rms_eps, model.rope_theta
     c.max_sessions, c.max_ctx, c.timeout_ms, c.idle_ms, c.modes, c.device = (max_sessions, max_ctx, timeout_ms,
                                                                                 idle_ms, modes, device)
+    c.weight_fp8 = 1 if weight_fp8 else 0
     return c
 
 
@@ -248,6 +250,10 @@ def flash_decode_noalloc(q_ptr, k_ptr, v_ptr, n_heads, n_kv_heads, head_dim, n_c
 
 
 FLASH_DECODE_NOALLOC_MAX_BYTES = 4 << 20
+
+
+def quantize_e4m3(w_ptr, rows, cols, dtype, q_ptr, scale_ptr, stream_ptr=None) -> int:
+    return lib.kie_quantize_e4m3(w_ptr, rows, cols, dtype, q_ptr, scale_ptr, stream_ptr)
 
 
 def flash_decode_scratch_bytes(n_heads, n_kv_heads, head_dim, n_ctx) -> int:

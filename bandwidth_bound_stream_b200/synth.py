@@ -70,9 +70,16 @@ class ModelConfig:
         return (self.n_layers * per_layer + int(np.prod(self.shape("tok_emb")))
                 + int(np.prod(self.shape("lm_head"))) + self.d_model)
 
-    def weight_bytes_per_token(self) -> int:
-        """Bytes one decode step must stream: every weight except the embedding table, plus one embedding row."""
-        return 2 * (self.n_params() - self.vocab * self.d_model + self.d_model)
+    def weight_bytes_per_token(self, fp8: bool = False) -> int:
+        """Bytes one decode step must stream: every weight except the embedding table, plus one
+        embedding row. With fp8, the matrices and the LM head stream as one-byte E4M3 codes plus
+        a 4-byte scale per row; the norm gains and the embedding row stay 16-bit."""
+        if not fp8:
+            return 2 * (self.n_params() - self.vocab * self.d_model + self.d_model)
+        d, q, kv, f, V, L = self.d_model, self.q_dim, self.kv_dim, self.ffn, self.vocab, self.n_layers
+        elems = L * (q * d + 2 * kv * d + d * q + 2 * f * d + d * f) + V * d
+        rows = L * (q + 2 * kv + d + 2 * f + d) + V
+        return elems + 4 * rows + 2 * (2 * L + 1) * d + 2 * d
 
     def kv_bytes_per_position(self) -> int:
         """K and V bytes of one context position over all layers."""

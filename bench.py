@@ -47,14 +47,15 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def algorithmic_bytes(model, ctx0: int, n: int) -> int:
+def algorithmic_bytes(model, ctx0: int, n: int, fp8: bool = False) -> int:
     """Bytes one launch must move: all weights except the embedding table plus one embedding row per token,
-    the KV cache read over the attended positions, and the new position's K/V write."""
+    the KV cache read over the attended positions, and the new position's K/V write (fp8: the
+    matrices as E4M3 codes plus row scales)."""
     per_pos = model.kv_bytes_per_position()
     total = 0
     for t in range(n):
         attended = ctx0 + t + 1
-        total += model.weight_bytes_per_token() + attended * per_pos + per_pos
+        total += model.weight_bytes_per_token(fp8) + attended * per_pos + per_pos
     return total
 
 
@@ -389,8 +390,8 @@ def main():
     if args.ticks > 0 and headline:
         line["tick"] = run_tick(args.ticks, args.warmup, local, clocks_for=local)
     if headline and not args.no_extra and world == 1:
-        line["configs"] = {f"{n}@{p}+{d}": run_extra(n, p, d, args.extra_steps, 3, local, peak)
-                           for n, p, d in EXTRA_CONFIGS}
+        line["configs"] = {f"{n}{'-fp8' if f8 else ''}@{p}+{d}": run_extra(n, p, d, f8, args.extra_steps, 3, local, peak)
+                           for n, p, d, f8 in EXTRA_CONFIGS}
     if want_cpu:
         line["cpu_baseline"] = oracle_baseline(m, host_weights, prompt_len + decode_n // 2)
     if rank == 0:
@@ -402,11 +403,14 @@ def main():
 
 # The other batch-1 workloads of the method's configurations, measured after the headline in
 # the same run (each: its own engine, the prompt prefilled before timing, device-timed launches).
-EXTRA_CONFIGS = (("dense-8b", 4096, 256), ("dense-1.9b", 32768, 256))
+EXTRA_CONFIGS = (("dense-8b", 4096, 256, False), ("dense-1.9b", 32768, 256, False), ("dense-1.9b", 1024, 512, True))
 
 
-def run_extra(name: str, prompt_len: int, decode_n: int, steps: int, warmup: int, local: int, peak: float) -> dict:
-    """tokens/s and the roofline of one more batch-1 workload (steps launches of decode_n tokens)."""
+def run_extra(name: str, prompt_len: int, decode_n: int, fp8: bool, steps: int, warmup: int, local: int,
+              peak: float) -> dict:
+    """tokens/s and the roofline of one more batch-1 workload (steps launches of decode_n tokens);
+    fp8: the engine streams E4M3 weights with row scales (the prompt then goes through the
+    batch-1 kernel as well)."""
     import torch
 
     from bandwidth_bound_stream_b200 import kie, synth
@@ -414,8 +418,9 @@ def run_extra(name: str, prompt_len: int, decode_n: int, steps: int, warmup: int
     dev = f"cuda:{local}"
     t0 = time.perf_counter()
     dw = kie.DeviceWeights(m, seed=0, device=dev)
+    modes = kie.KIE_MODE_BATCH1 if fp8 else kie.KIE_MODE_BATCH1 | kie.KIE_MODE_TICK
     eng = kie.Engine(kie.config(m, max_ctx=prompt_len + decode_n, timeout_ms=20000, idle_ms=200, device=local,
-                                modes=kie.KIE_MODE_BATCH1 | kie.KIE_MODE_TICK), dw.kie)
+                                modes=modes, weight_fp8=fp8), dw.kie)
     dw.free()
     torch.cuda.empty_cache()
     setup_s = time.perf_counter() - t0
@@ -447,10 +452,11 @@ def run_extra(name: str, prompt_len: int, decode_n: int, steps: int, warmup: int
     clk = clocks.stop()
     per = [a.elapsed_time(b) for a, b in ev]
     eng.close()
-    bytes_launch = algorithmic_bytes(m, prompt_len, decode_n)
+    bytes_launch = algorithmic_bytes(m, prompt_len, decode_n, fp8)
     mean_s = statistics.mean(per) / 1e3
     achieved = bytes_launch / mean_s / 1e9
-    return {"workload": f"{name} {'bf16' if m.dtype else 'fp16'} batch-1: prompt {prompt_len}, greedy decode {decode_n}",
+    wt = "E4M3 weights with fp32 row scales, " if fp8 else ""
+    return {"workload": f"{name} {wt}{'bf16' if m.dtype else 'fp16'} batch-1: prompt {prompt_len}, greedy decode {decode_n}",
             "tokens_per_s": round(decode_n * steps / (sum(per) / 1e3), 2), "steps": steps, "warmup": warmup,
             "per_launch_ms": [round(x, 3) for x in per],
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",

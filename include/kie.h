@@ -69,6 +69,13 @@ typedef struct {
     int32_t idle_ms;      /* the resident kernel exits after this long with no command */
     int32_t modes;        /* KIE_MODE_* bitmask                                        */
     int32_t device;       /* CUDA device ordinal                                       */
+    int32_t weight_fp8;   /* 1: the batch-1 kernel streams its matrices (and the LM head) as
+                             E4M3 codes with a per-row fp32 scale, quantised by kie_create
+                             from the given 16-bit weights as kie_quantize_e4m3 does; half
+                             the bytes per token. Needs modes == KIE_MODE_BATCH1 (the tick
+                             kernel's tensor-core contractions take 16-bit operands), and
+                             prompts then go through the batch-1 kernel too. 0: weights
+                             stream in `dtype`.                                           */
 } kie_config;
 
 /*
@@ -233,6 +240,17 @@ typedef struct {
     uint64_t seed;
 } kie_sampling;
 kie_status kie_session_sampling(kie_engine *eng, int32_t sid, const kie_sampling *s);
+
+/*
+ * Per-row E4M3 quantisation of a 16-bit matrix (w_dev: [rows][cols] of dtype, DEVICE), as
+ * kie_create does for a weight_fp8 engine: scale_dev[n] (DEVICE, fp32) = max_k |w[n][k]| / 448
+ * (1 for an all-zero row) and q_dev[n][k] (DEVICE, one byte each) = the E4M3 code nearest to the
+ * fp32 quotient w[n][k] / scale[n] (ties to the even code), saturated at +-448. E4M3: sign, 4
+ * exponent bits with bias 7, 3 fraction bits, no infinities, 0x7F / 0xFF NaN. Stream-ordered on
+ * `stream` (cudaStream_t; NULL = legacy default stream). KIE_ERR_ARG on bad arguments.
+ */
+kie_status kie_quantize_e4m3(const void *w_dev, int64_t rows, int32_t cols, int32_t dtype, uint8_t *q_dev,
+                             float *scale_dev, void *stream);
 
 /* Copies the engine's last error message (NUL-terminated, truncated to len). */
 kie_status kie_last_error(kie_engine *eng, char *buf, int32_t len);

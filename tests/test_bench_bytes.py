@@ -19,3 +19,13 @@ def test_algorithmic_bytes_grow_with_context():
     m = synth.DENSE_8B
     a, b = bench.algorithmic_bytes(m, 4096, 1), bench.algorithmic_bytes(m, 4097, 1)
     assert b - a == m.kv_bytes_per_position() == 32 * 8 * 128 * 2 * 2
+
+
+def test_fp8_weight_bytes():
+    """E4M3 codes (one byte) for every matrix and the LM head, a 4-byte scale per row, 16-bit
+    norms and embedding row."""
+    L, d, Hq, Hkv, D, F, V = 28, 2048, 16, 8, 128, 8192, 32000
+    elems = L * (Hq * D * d + 2 * Hkv * D * d + d * Hq * D + 3 * F * d) + V * d
+    rows = L * (Hq * D + 2 * Hkv * D + d + 2 * F + d) + V
+    assert synth.DENSE_1P9B.weight_bytes_per_token(fp8=True) == elems + 4 * rows + 2 * (2 * L + 1) * d + 2 * d
+    assert abs(synth.DENSE_1P9B.weight_bytes_per_token(fp8=True) / synth.DENSE_1P9B.weight_bytes_per_token() - 0.5) < 0.001
