@@ -504,13 +504,20 @@ def run_tick(n_ticks: int, warmup: int, local: int, clocks_for: int, model_name:
         lat.append((time.perf_counter() - a) * 1e3)
         tokens = out[-1].copy()
     clk = clocks.stop()
-    # the same ticks, stream-ordered on device buffers and timed with CUDA events (device time)
+    # the same ticks, stream-ordered on device buffers and timed with CUDA events (device time),
+    # from the same contexts: the sessions are rewound to where the doorbell ticks started (else
+    # every tick would attend ~2 * n_ticks more positions)
+    for s, c in zip(sids, ctx0):
+        eng.session_rewind(s, c)
     stream = torch.cuda.Stream(device=dev)
     tok_d = torch.tensor(tokens, device=dev)
     outs = [torch.zeros((TICK_STEPS, TICK_SESSIONS), dtype=torch.int32, device=dev) for _ in range(2)]
     for k in range(warmup):
         eng.tick_launch(sids, tok_d.data_ptr() if k == 0 else outs[(k - 1) % 2][-1].data_ptr(), TICK_STEPS,
                         outs[k % 2].data_ptr(), None, stream.cuda_stream)
+    eng.sync()
+    for s, c in zip(sids, ctx0):
+        eng.session_rewind(s, c)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_ticks)]
     torch.cuda.nvtx.range_push("kie_tick_timed")
     for k in range(n_ticks):
@@ -553,7 +560,8 @@ def kernel_revision() -> str:
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "bandwidth_bound_stream_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.startswith("kie_b1") or name in ("kie_device.cuh", "kie_attn.cuh", "kie_internal.h"):
+        if name.startswith("kie_b1") or name in ("kie_device.cuh", "kie_attn.cuh", "kie_internal.h",
+                                                  "kie_sample.cuh"):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(f.read())
     return h.hexdigest()[:12]
