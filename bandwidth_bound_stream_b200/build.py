@@ -17,6 +17,9 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 KIE_SOURCES = ["kie_engine.cu", "kie_b1.cu", "kie_mr.cu", "kie_attn.cu", "kie_fp8.cu"]
+# build variants of the engine library: the product ("") and a diagnostic build, each its own
+# file (selected at import by KIE_VARIANT): "profile" times the GEMV consumer warps per chunk
+VARIANTS = {"": [], "profile": ["-DKIE_PROFILE_GEMV"]}
 KIE_HEADERS = ["kie_device.cuh", "kie_internal.h", "kie_attn.cuh", "kie_sample.cuh"]
 
 
@@ -43,19 +46,25 @@ def build_synth(force: bool = False) -> str:
     return out
 
 
-def build_kie(force: bool = False, verbose_ptxas: bool = False) -> str:
-    out = os.path.join(HERE, "libkie.so")
+def lib_name(variant: str = "") -> str:
+    if variant not in VARIANTS:
+        raise ValueError(f"unknown build variant {variant!r} (one of {sorted(VARIANTS)})")
+    return "libkie.so" if not variant else f"libkie_{variant}.so"
+
+
+def build_kie(force: bool = False, verbose_ptxas: bool = False, variant: str = "") -> str:
+    out = os.path.join(HERE, lib_name(variant))
     srcs = [os.path.join(CSRC, s) for s in KIE_SOURCES]
     deps = srcs + [os.path.join(CSRC, h) for h in KIE_HEADERS] + [os.path.join(INCLUDE, "kie.h")]
     if not (force or verbose_ptxas or _stale(out, deps)):
         return out
-    objdir = os.path.join(HERE, "_build")
+    objdir = os.path.join(HERE, "_build" + (f"_{variant}" if variant else ""))
     os.makedirs(objdir, exist_ok=True)
     objs, procs = [], []
     for s in srcs:
         o = os.path.join(objdir, os.path.basename(s) + ".o")
         cmd = [NVCC, *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-rdc=false",
-               "-I", INCLUDE, "-I", CSRC, "-c", s, "-o", o]
+               "-I", INCLUDE, "-I", CSRC, *VARIANTS[variant], "-c", s, "-o", o]
         if verbose_ptxas:
             cmd.insert(1, "-Xptxas=-v")
         procs.append((cmd, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)))
@@ -83,3 +92,5 @@ if __name__ == "__main__":
     build_all(force="--force" in sys.argv)
     if "--ptxas" in sys.argv:
         build_kie(verbose_ptxas=True)
+    if "--variant" in sys.argv:  # e.g. --variant profile
+        build_kie(force="--force" in sys.argv, variant=sys.argv[sys.argv.index("--variant") + 1])

@@ -108,7 +108,7 @@ struct __align__(16) B1Shared {
     int token;
     int gb_ok;
     int row0[KIE_NPH], row1[KIE_NPH];
-    unsigned long long wait_cons;
+    unsigned long long wait_ph[KIE_NPH];  // consumer ring waits of this token per phase (ns, traced runs)
     __align__(16) uint8_t warm_sink[512];  // destination of the K/V reads into L2 (16 bytes per lane; never read)
 };
 
@@ -266,6 +266,19 @@ __device__ bool chunk_next(const KieParams &P, const B1Shared &S, const KieCmd &
     }
 }
 
+// --------------------------------------------------------------- ring
+
+// A consumer's wait for the data of ring slot `slot` (phase parity `par`). With the trace on,
+// thread 0 adds the time it was blocked to the phase's total.
+__device__ __forceinline__ bool ring_take(const KieParams &P, B1Shared &S, uint32_t slot, uint32_t par, int ph) {
+    if (S.abort) return false;
+    if (mbar_test_wait(&S.full[slot], par)) return true;
+    const uint64_t w0 = globaltimer();
+    const bool ok = mbar_wait(&S.full[slot], par, P.timeout_ns, &S.abort);
+    if (P.trace && threadIdx.x == 0) S.wait_ph[ph] += globaltimer() - w0;
+    return ok;
+}
+
 // --------------------------------------------------------------- producer
 
 __device__ void produce(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint8_t *ring, const KieCmd &cmd) {
@@ -284,7 +297,7 @@ __device__ void produce(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint
             tok = fetch.t;
         }
         const uint32_t slot = ring_it % KIE_NSLOT, par = (ring_it / KIE_NSLOT) & 1u;
-        if (!mbar_try_wait(&S.empty[slot], par ^ 1u)) {
+        if (!mbar_test_wait(&S.empty[slot], par ^ 1u)) {
             const uint64_t w0 = globaltimer();
             const bool ok = !S.abort && mbar_wait(&S.empty[slot], par ^ 1u, P.timeout_ns, &S.abort);
             waited += globaltimer() - w0;
@@ -379,21 +392,23 @@ __device__ void gemv_phase(const KieParams &P, B1Shared &S, uint32_t &ring_it, c
         for (int e = 0; e < 8; e++) h[i][e] *= rstd;
     if (l < P.L) trace_mark(P, t, 1 + 16 * l + (ph == PH_QKV ? 11 : 12), h[0][0]);
 
-    unsigned long long waited = 0;
     const int grp = w / CS, ws = w % CS;
     constexpr int STRIDE = WPART_FLOATS / CS;  // row capacity of one slice's partials
+#ifdef KIE_PROFILE_GEMV
+    // diagnostic build: SM cycles from a chunk's data being ready to this warp's release of
+    // it, summed over the gate/up chunks, for the first warp of each row group
+    long long busy = 0, c_ready = 0;
+#endif
     // a chunk holds SUB blocks of GROUPS * CR rows (two with one-byte weights)
     constexpr int SUB = 2 / ESZ;
     for (int c0 = 0; c0 < rows; c0 += SUB * GROUPS * CR) {
         const uint32_t slot = ring_it % KIE_NSLOT, par = (ring_it / KIE_NSLOT) & 1u;
         ring_it++;
-        bool have = !S.abort && mbar_try_wait(&S.full[slot], par);
-        if (!have && !S.abort) {
-            const uint64_t w0 = globaltimer();
-            have = mbar_wait(&S.full[slot], par, P.timeout_ns, &S.abort);
-            waited += globaltimer() - w0;
-        }
+        bool have = ring_take(P, S, slot, par, ph);
         have = __all_sync(0xffffffffu, have);  // one decision per warp (the reduction needs all lanes)
+#ifdef KIE_PROFILE_GEMV
+        c_ready = clock64();
+#endif
         if (!have) {
             if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, (unsigned)ph);
             S.abort = 1;
@@ -427,13 +442,19 @@ __device__ void gemv_phase(const KieParams &P, B1Shared &S, uint32_t &ring_it, c
             if (sub == SUB - 1) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.empty[slot]);  // shared-memory reads of the chunk are done
+#ifdef KIE_PROFILE_GEMV
+                busy += clock64() - c_ready;
+#endif
             }
             const float s = warp_reduce_rows<CR>(acc);
             constexpr int LPR = 32 / CR;
             if ((lane % LPR) == 0 && lane / LPR < nr) S.wpart[ws * STRIDE + r0 + lane / LPR] = s;
         }
     }
-    if (tid == 0) S.wait_cons += waited;
+#ifdef KIE_PROFILE_GEMV
+    if (P.trace && t < P.trace_tokens && l < P.L && ph == PH_GU && lane == 0 && ws == 0)
+        P.trace[((size_t)blockIdx.x * P.trace_tokens + t) * P.trace_events + 1 + 16 * l + 13 + grp] = busy;
+#endif
     named_bar_sync(1, KIE_CONS_THREADS);
 }
 
@@ -472,8 +493,7 @@ __device__ void fold_rows(const KieParams &P, B1Shared &S, uint32_t &ring_it, co
         const int n = min(cpc, ng - g0);
         const uint32_t slot = ring_it % KIE_NSLOT, par = (ring_it / KIE_NSLOT) & 1u;
         ring_it++;
-        bool have = !S.abort && mbar_try_wait(&S.full[slot], par);
-        if (!have && !S.abort) have = mbar_wait(&S.full[slot], par, P.timeout_ns, &S.abort);
+        bool have = ring_take(P, S, slot, par, ph);
         have = __all_sync(0xffffffffu, have);
         if (!have) {
             if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, (unsigned)ph);
@@ -813,7 +833,7 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, cons
             S.abort = 1;
             tok = 0;
         }
-        if (threadIdx.x == 0) S.wait_cons = 0;
+        if (threadIdx.x < KIE_NPH) S.wait_ph[threadIdx.x] = 0;
         trace_mark(P, t, 0);
         const bool head = (cmd.op != OP_PREFILL) || (t == cmd.n - 1);
         for (int l = 0; l < L; l++) {
@@ -864,8 +884,9 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, cons
             }
             trace_mark(P, t, eh + 2);
         }
-        if (P.trace && t < P.trace_tokens && threadIdx.x == 0)
-            P.trace[((size_t)blockIdx.x * P.trace_tokens + t) * P.trace_events + P.trace_events - 2] = S.wait_cons;
+        if (P.trace && t < P.trace_tokens && threadIdx.x < KIE_NPH)
+            P.trace[((size_t)blockIdx.x * P.trace_tokens + t) * P.trace_events + P.trace_events - 1 - KIE_NPH +
+                    threadIdx.x] = S.wait_ph[threadIdx.x];
     }
     cp_async_wait_all();  // the L2 reads into warm_sink have landed
 }

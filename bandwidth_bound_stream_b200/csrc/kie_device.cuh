@@ -74,6 +74,19 @@ KIE_DEV void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
                  : "memory");
 }
 
+// Non-blocking test of an mbarrier phase (returns at once).
+KIE_DEV bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Potentially blocking test: the thread may be suspended in hardware (up to the 1 ms hint)
+// until the phase completes.
 KIE_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(

@@ -1121,7 +1121,7 @@ extern "C" kie_status kie_inject_fault(kie_engine *eng, int32_t fault) {
 
 extern "C" int32_t kie_trace_events(kie_engine *eng) {
     if (!eng) return 0;
-    return 1 + 16 * eng->cfg.n_layers + 3 + 2;
+    return 1 + 16 * eng->cfg.n_layers + 3 + KIE_NPH + 1;
 }
 
 extern "C" kie_status kie_trace_enable(kie_engine *eng, int32_t tokens) {

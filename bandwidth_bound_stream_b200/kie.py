@@ -13,7 +13,12 @@ import os
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libkie.so")
+# KIE_VARIANT selects a diagnostic build of the same library ("profile": GEMV consumer timing
+# in the phase trace); unset means the product build
+VARIANT = os.environ.get("KIE_VARIANT", "")
+if VARIANT not in ("", "profile"):
+    raise ImportError(f"KIE_VARIANT={VARIANT!r}: expected unset or 'profile'")
+LIB_PATH = os.path.join(_HERE, "libkie.so" if not VARIANT else f"libkie_{VARIANT}.so")
 
 KIE_OK, KIE_ERR_ARG, KIE_ERR_CAPACITY, KIE_ERR_CUDA = 0, -1, -2, -3
 KIE_ERR_TIMEOUT, KIE_ERR_STATE, KIE_ERR_DEVICE, KIE_ERR_UNSUPPORTED = -4, -5, -6, -7
@@ -56,7 +61,8 @@ class KieError(RuntimeError):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libkie.so not built ({LIB_PATH}); run __graft_entry__.build()")
+        raise ImportError(f"{os.path.basename(LIB_PATH)} not built ({LIB_PATH}); run __graft_entry__.build()"
+                          + (f" or build.build_kie(variant={VARIANT!r})" if VARIANT else ""))
     h = ctypes.CDLL(LIB_PATH)
     i32, vp, i64 = ctypes.c_int32, ctypes.c_void_p, ctypes.c_int64
     P = ctypes.POINTER
@@ -213,7 +219,7 @@ class Engine:
         self._check(lib.kie_trace_enable(self.h, tokens), "kie_trace_enable")
 
     def trace_read(self, tokens: int) -> np.ndarray:
-        """Phase stamps as [cta][token][event] (uint64 ns; the last two events are ring wait totals)."""
+        """Phase stamps as [cta][token][event] (uint64 ns; the last six events are ring wait totals)."""
         ev = lib.kie_trace_events(self.h)
         n = ctypes.c_int64()
         self._check(lib.kie_trace_read(self.h, None, 0, ctypes.byref(n)), "kie_trace_read")

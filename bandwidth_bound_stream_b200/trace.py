@@ -5,8 +5,9 @@ token, globaltimer stamps (ns). Slot 0 is the token's start. Each layer l then h
 from 1 + 16 l: the ends of its 10 phases (slots 0-9), the end of the down fold's wait for
 every CTA's read of the residual (10), the input-ready stamps of the QKV and gate/up phases
 (11, 12), and the end of this CTA's attention positions (15; 0 when it owns no unit). After
-the layers come the LM head's rows, its barrier and the final argmax, then two ring-wait
-totals. Host-side arithmetic only.
+the layers come the LM head's rows, its barrier and the final argmax, then the consumer
+warps' ring waits of the token per weight phase (QKV rows, O fold, gate/up rows, down fold,
+LM head) and the producer's total wait for free ring slots (ns). Host-side arithmetic only.
 """
 from __future__ import annotations
 
@@ -15,11 +16,12 @@ import numpy as np
 LAYER_PHASES = ("qkv_rows", "qkv_epilogue", "barrier_qkv_attn", "attention", "o_fold", "barrier_o_gu",
                 "gate_up_rows", "gate_up_epilogue", "down_fold", "barrier_down_next")
 LAYER_END = len(LAYER_PHASES) - 1  # slot of the layer's last phase end
+RING_PHASES = ("qkv_rows", "o_fold", "gate_up_rows", "down_fold", "lm_head_rows")  # consumer wait slots
 
 
 def batch1_events(n_layers: int) -> int:
     """Trace slots per token of the batch-1 kernel."""
-    return 1 + 16 * n_layers + 3 + 2
+    return 1 + 16 * n_layers + 3 + len(RING_PHASES) + 1
 
 
 def batch1_phase_us(trace: np.ndarray, n_layers: int, first_token: int = 1) -> dict:
@@ -41,6 +43,9 @@ def batch1_phase_us(trace: np.ndarray, n_layers: int, first_token: int = 1) -> d
     dur = {p: [] for p in LAYER_PHASES}
     positions, merge, per_layer = [], [], []
     head = {"lm_head_rows": [], "lm_head_barrier": [], "argmax": []}
+    nr = len(RING_PHASES)
+    ring = {p: [] for p in RING_PHASES}
+    producer = []
     for t in toks:
         s = x[:, t, :]
         for l in layers:
@@ -57,6 +62,9 @@ def batch1_phase_us(trace: np.ndarray, n_layers: int, first_token: int = 1) -> d
         head["lm_head_rows"].append(s[:, eh] - s[:, eh - 16 + LAYER_END])
         head["lm_head_barrier"].append(s[:, eh + 1] - s[:, eh])
         head["argmax"].append(s[:, eh + 2] - s[:, eh + 1])
+        for k, p in enumerate(RING_PHASES):  # per token; the layer phases spread over the layers
+            ring[p].append(s[:, n_ev - 1 - nr + k] / (1 if p == "lm_head_rows" else n_layers))
+        producer.append(s[:, n_ev - 1])
         if n_layers > 1:
             per_layer.append((s[:, 1 + 16 * (n_layers - 1) + LAYER_END] - s[:, 1 + LAYER_END]) / (n_layers - 1))
 
@@ -70,6 +78,9 @@ def batch1_phase_us(trace: np.ndarray, n_layers: int, first_token: int = 1) -> d
     out.update({k: us(v) for k, v in head.items()})
     if per_layer:
         out["per_layer"] = us(per_layer)
+    # consumer time blocked on weights that had not arrived: per layer (per token for the head)
+    out["ring_wait"] = {p: us(v) for p, v in ring.items()}
+    out["producer_wait_per_token"] = us(producer)
     out["tokens"] = len(toks)
     out["layers_averaged"] = len(layers)
     return out

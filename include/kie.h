@@ -182,7 +182,9 @@ kie_status kie_tick(kie_engine *eng, int32_t n_sess, const int32_t *sids, const 
  *   every CTA's read of the residual, 11 and 12 input vectors ready in the QKV and gate/up
  *   phases, 15 the end of this CTA's attention positions (before its split is published; 0
  *   if it had no unit); then 3 for the head (rows+argmax, barrier, final argmax); then the
- *   consumer's and the producer's total ring wait in ns.
+ *   token's consumer ring waits in ns per weight phase (QKV rows, O fold, gate/up rows, down
+ *   fold, LM head: the time thread 0 was blocked on a weight chunk that had not landed), and
+ *   the producer's total wait for a free ring slot in ns.
  * Tick and chunked-prefill commands write one record per step, in the same layout:
  *   0: step start; per layer (slot 1 + 16 l + k): k = 0 first norm done, then the ends of
  *   the grid barriers after: 1 first norm, 3 QKV, 4 RoPE, 6 attention (5: this CTA's

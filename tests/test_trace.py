@@ -24,6 +24,9 @@ def _synthetic(n_cta, n_tok, L, phase_ns, pos_ns, head_ns):
             for k, d in enumerate(head_ns):
                 now += d
                 x[c, t, eh + k] = now
+            for k in range(len(tr.RING_PHASES)):  # ring waits: (k + 1) us per layer, head 9 us
+                x[c, t, ev - 1 - len(tr.RING_PHASES) + k] = 9000 if k == 4 else (k + 1) * 1000 * L
+            x[c, t, ev - 1] = 123_000
     return x
 
 
@@ -40,6 +43,9 @@ def test_phase_breakdown_recovers_known_durations():
     assert out["argmax"] == pytest.approx(1.57)
     assert out["per_layer"] == pytest.approx(sum(phase) / 1e3)
     assert out["tokens"] == 2 and out["layers_averaged"] == 4
+    assert out["ring_wait"] == pytest.approx({"qkv_rows": 1.0, "o_fold": 2.0, "gate_up_rows": 3.0, "down_fold": 4.0,
+                                              "lm_head_rows": 9.0})
+    assert out["producer_wait_per_token"] == pytest.approx(123.0)
 
 
 def test_phase_breakdown_single_layer_and_shape_check():
