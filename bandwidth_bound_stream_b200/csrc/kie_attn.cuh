@@ -51,6 +51,7 @@ struct AttnSmem {
     float mrow[KIE_GMAX];
     float red[KIE_GMAX * 16];
     int is_last;
+    uint32_t pub_sink;          // scratch word of pub_wait
     unsigned long long t_unit;  // globaltimer when this CTA's last unit finished its positions
 };
 
@@ -271,8 +272,11 @@ __device__ __forceinline__ void attn_tail(const AttnArgs &A, AttnSmem &S, int un
         named_bar_sync(1, ATTN_THREADS);
         return;
     }
-    // publish this split's partial, then the last split of the kv head merges
+    // publish this split's partial, then the last split of the kv head merges. With cnt_target
+    // (the batch-1 megakernel, whose weight stream keeps bulk copies in flight) the partial is
+    // published by completion and the split's count is a relaxed add; else by a fence.
     float *pp = A.part + ((size_t)unit * Gt + hoff) * (D + 2);
+    uint32_t ptok = 0;
     for (int i = tid; i < nh * (D + 2) / 2; i += ATTN_THREADS) {  // float2 per thread (D + 2 is even)
         const int jj = (2 * i) / (D + 2), e = (2 * i) % (D + 2);
         float2 val;
@@ -284,9 +288,11 @@ __device__ __forceinline__ void attn_tail(const AttnArgs &A, AttnSmem &S, int un
             val.x = ((S.wacc[0][k] + S.wacc[1][k]) + S.wacc[2][k]) + S.wacc[3][k];
             val.y = ((S.wacc[0][k + 1] + S.wacc[1][k + 1]) + S.wacc[2][k + 1]) + S.wacc[3][k + 1];
         }
-        reinterpret_cast<float2 *>(pp)[i] = val;
+        if (A.cnt_target) pub_f32x2(pp + 2 * i, val.x, val.y, ptok);
+        else reinterpret_cast<float2 *>(pp)[i] = val;
     }
-    __threadfence();
+    if (A.cnt_target) pub_wait(ptok, &S.pub_sink);
+    else __threadfence();
     named_bar_sync(1, ATTN_THREADS);
     if (A.cnt_target) {
         // Every split merges its own slice of the kv head's output once all splits have
@@ -294,7 +300,7 @@ __device__ __forceinline__ void attn_tail(const AttnArgs &A, AttnSmem &S, int un
         // for all splits, in a single round trip, and no single CTA merging everything.
         const bool last_pass = hoff + GC >= Gt;
         if (tid == 0) {
-            atomicAdd(A.cnt + g, 1u);
+            red_relaxed_gpu_add_u32(A.cnt + g, 1u);
             const uint64_t t0 = globaltimer();
             unsigned spins = 0;
             while (last_pass && (int)(ld_acquire_gpu_u32(A.cnt + g) - A.cnt_target) < 0) {

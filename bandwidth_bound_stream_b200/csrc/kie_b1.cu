@@ -52,6 +52,84 @@ namespace {
 
 constexpr int RING_BYTES = KIE_NSLOT * KIE_SLOT_BYTES;
 
+// ------------------------------------------------------------------ tensor memory (TMEM) staging
+//
+// With 16-bit weights and d_model 2048 or 4096, every 64 KB ring chunk gives each of the 512
+// consumer threads exactly 8 pieces of 16 bytes (rows of its column slice, or rows of its fold
+// columns), and within each piece index the 16-byte pieces of the warps' lanes lie at a uniform
+// 16-byte stride, 512 bytes per warp. So the producer can move a landed chunk on from shared
+// memory into one of 4 TMEM slots (128 columns each; all 512 columns of the SM) with 16
+// tcgen05.cp copies of 128 lanes x 32 bytes that read the ring's own layout: copy j fills
+// columns 8j..8j+7, i.e. pieces 2(j%4) and 2(j%4)+1 of warps 4(j/4) .. 4(j/4)+3, lane 32(w%4)+l
+// holding thread (w, l)'s pieces. A consumer warp then takes its 8 pieces with one tcgen05.ld
+// (32 lanes x 32 columns) of its lane quarter. The ring slot is free once the copies are done.
+// The producer moves the chunks it fetches while the consumers are in the attention step and
+// its grid barriers (produce_tmem), so there the weight stream runs 7 chunks (448 KB per SM)
+// ahead of the consumers instead of 3.
+
+constexpr uint32_t TMEM_COLS = 512;
+
+KIE_DEV void tm_alloc(uint32_t *dst_smem) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+KIE_DEV void tm_dealloc(uint32_t taddr) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(TMEM_COLS) : "memory");
+}
+KIE_DEV void tm_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+KIE_DEV void tm_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// arrive on `bar` once every tcgen05 operation this thread issued so far has completed
+KIE_DEV void tm_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+// shared-memory descriptor, no swizzle: 8-row core matrices of 16-byte rows, `lbo` bytes between
+// the two 16-byte halves of a 32-byte row, `sbo` bytes between consecutive 8-row groups
+KIE_DEV uint64_t tm_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1u << 46);
+}
+KIE_DEV void tm_cp(uint32_t taddr, uint64_t desc) {
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+// this warp's lane quarter, 32 consecutive columns -> 32 registers per thread
+KIE_DEV void tm_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+          "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+          "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+KIE_DEV uint4 tm_piece(const uint32_t (&r)[32], int k) { return make_uint4(r[4 * k], r[4 * k + 1], r[4 * k + 2], r[4 * k + 3]); }
+
+// byte offset in the ring chunk, and distance between the two 16-byte halves, of copy j (0..15)
+// of a chunk of phase ph. GEMV chunks hold rows of d 16-bit weights: with d = 2048 piece k of
+// warp w is row 8 (w / 8) + k of the chunk; with d = 4096 it is row 4 (w / 8) + k / 2, in column
+// half k % 2 of the row (the halves 4096 bytes apart). Fold chunks: piece k is column group
+// k / R, row tid + 512 (k % R), with R = d / 512 pieces per group.
+KIE_DEV void tm_copy_src(int ph, int d, int j, uint32_t &off, uint32_t &lbo) {
+    const uint32_t cg = (uint32_t)j >> 2, p = (uint32_t)j & 3u;
+    if (ph == PH_OF || ph == PH_DF) {
+        const uint32_t R = (uint32_t)d / 512u, k0 = 2u * p;
+        off = (k0 / R) * (uint32_t)d * 16u + (k0 % R) * 8192u + cg * 2048u;
+        lbo = 8192u;
+    } else if (d == 2048) {
+        off = ((cg >> 1) * 8u + 2u * p) * 4096u + (cg & 1u) * 2048u;
+        lbo = 4096u;
+    } else {
+        off = ((cg >> 1) * 4u + p) * 8192u + (cg & 1u) * 2048u;
+        lbo = 4096u;
+    }
+}
+
 constexpr int WPART_FLOATS = 8 * KIE_ROWACC_MAX;  // column-slice partials: [slices][rows] flattened
 
 // 8 streamed weights -> 8 floats: 16-byte vector of the storage dtype, or 8-byte vector of E4M3
@@ -103,6 +181,10 @@ struct __align__(16) B1Shared {
     float2 rope_s[KIE_DMAX / 2];  // rotation of the current position, loaded at the start of QKV
     uint64_t full[KIE_NSLOT];
     uint64_t empty[KIE_NSLOT];
+    uint64_t tfull[KIE_NTS];   // TMEM staging: slot t holds its chunk (tcgen05.commit)
+    uint64_t tempty[KIE_NTS];  // every consumer warp has read slot t
+    uint32_t tmem_base;
+    uint32_t pub_sink;         // scratch word of pub_wait
     KieCmd cmd;
     volatile int abort;
     int token;
@@ -140,16 +222,20 @@ __device__ __forceinline__ void trace_mark(const KieParams &P, int t, int ev, fl
 // --------------------------------------------------------------- grid barrier
 
 // All consumer threads call this. Returns false if this CTA is aborting.
+// fenced: the arrive is a release (the command broadcast, written with plain stores while no
+// weight copies are in flight). Otherwise the values other CTAs read afterwards were published
+// by completion (pub_*; every thread waited for them before the named barrier below), so the
+// arrive is relaxed and does not wait for the weight stream's copies in flight.
 __device__ bool grid_barrier(const KieParams &P, B1Shared &S, unsigned long long &epoch, long long timeout_ns,
-                             unsigned where) {
+                             unsigned where, bool fenced = false) {
     named_bar_sync(1, KIE_CONS_THREADS);
     if (threadIdx.x == 0) {
         int ok = !S.abort;
         if (ok) {
             epoch += 1;
             const unsigned long long target = epoch * (unsigned long long)P.nblk;
-            // release: this CTA's writes (ordered before by the named barrier) become visible
-            red_release_gpu_add_u64(P.bar, 1ull);
+            if (fenced) red_release_gpu_add_u64(P.bar, 1ull);
+            else red_relaxed_gpu_add_u64(P.bar, 1ull);
             uint64_t t0 = globaltimer();
             unsigned spins = 0;
             while (ld_acquire_gpu_u64(P.bar) < target) {
@@ -173,10 +259,10 @@ __device__ bool grid_barrier(const KieParams &P, B1Shared &S, unsigned long long
     return S.gb_ok != 0;
 }
 
-// The split barrier of phase C. Thread 0 announces that this CTA has read the residual (its
-// earlier reads are ordered before the release)...
+// The split barrier of phase C. Thread 0 announces that this CTA has read the residual (the
+// reads have returned: their values were used before the phase's last named barrier)...
 __device__ __forceinline__ void residual_read_arrive(const KieParams &P, const B1Shared &S) {
-    if (threadIdx.x == 0 && !S.abort) red_release_gpu_add_u64(P.rd, 1ull);
+    if (threadIdx.x == 0 && !S.abort) red_relaxed_gpu_add_u64(P.rd, 1ull);
 }
 
 // ... and before the first add into it waits until every CTA has done so (`epoch`: this
@@ -211,6 +297,8 @@ __device__ void residual_read_wait(const KieParams &P, B1Shared &S, unsigned lon
 struct ChunkIter {
     const uint8_t *seg, *g;
     int t, l, ph, r;
+    int qn;  // chunks of this layer's O fold, gate/up and down fold returned so far
+    int cq;  // the returned chunk's index among them (-1: a QKV or LM-head chunk)
 };
 
 __device__ __forceinline__ void chunk_begin(ChunkIter &it, const uint8_t *seg) {
@@ -220,6 +308,8 @@ __device__ __forceinline__ void chunk_begin(ChunkIter &it, const uint8_t *seg) {
     it.l = 0;
     it.ph = 0;
     it.r = 0;
+    it.qn = 0;
+    it.cq = -1;
 }
 
 __device__ __forceinline__ bool is_fold(int ph) { return ph == PH_OF || ph == PH_DF; }
@@ -237,10 +327,12 @@ __device__ bool chunk_next(const KieParams &P, const B1Shared &S, const KieCmd &
             addr = it.g;
             it.g += bytes;
             it.r += nr;
+            it.cq = (it.ph == PH_QKV || it.ph == PH_HEAD) ? -1 : it.qn++;
             return true;
         }
         // phase exhausted: advance
         it.r = 0;
+        if (it.ph == PH_DF) it.qn = 0;
         if (it.ph == PH_HEAD) {
             it.t++;
             it.l = 0;
@@ -279,9 +371,37 @@ __device__ __forceinline__ bool ring_take(const KieParams &P, B1Shared &S, uint3
     return ok;
 }
 
+// The TMEM counterpart: wait until TMEM slot `ts` (phase parity `par`) holds its chunk.
+__device__ __forceinline__ bool tmem_take(const KieParams &P, B1Shared &S, uint32_t ts, uint32_t par, int ph) {
+    if (S.abort) return false;
+    if (mbar_test_wait(&S.tfull[ts], par)) return true;
+    const uint64_t w0 = globaltimer();
+    const bool ok = mbar_wait(&S.tfull[ts], par, P.timeout_ns, &S.abort);
+    if (P.trace && threadIdx.x == 0) S.wait_ph[ph] += globaltimer() - w0;
+    return ok;
+}
+
+// A consumer warp's 8 pieces of the chunk in TMEM slot ts (see the staging layout above);
+// the slot is released as soon as they are in registers.
+__device__ __forceinline__ void tmem_read_chunk(B1Shared &S, uint32_t ts, uint32_t (&r)[32]) {
+    const int w = threadIdx.x >> 5;
+    tm_fence_after();
+    tm_ld32(S.tmem_base + ((uint32_t)(32 * (w & 3)) << 16) + ts * 128u + 32u * (uint32_t)(w >> 2), r);
+    tm_fence_before();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&S.tempty[ts]);
+}
+
 // --------------------------------------------------------------- producer
 
-__device__ void produce(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint8_t *ring, const KieCmd &cmd) {
+// Writes the producer's wait for this token into its trace slot.
+__device__ __forceinline__ void trace_producer_wait(const KieParams &P, int tok, unsigned long long waited) {
+    if (P.trace && tok < P.trace_tokens)
+        P.trace[((size_t)blockIdx.x * P.trace_tokens + tok) * P.trace_events + P.trace_events - 1] = waited;
+}
+
+// Shared-memory ring only: chunk i goes to slot i % 3, and the consumers read it there.
+__device__ void produce_ring(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint8_t *ring, const KieCmd &cmd) {
     const uint8_t *seg = P.wpack + P.seg_off[blockIdx.x];
     ChunkIter fetch;
     chunk_begin(fetch, seg);
@@ -291,8 +411,7 @@ __device__ void produce(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint
     int tok = 0;
     while (chunk_next(P, S, cmd, fetch, a, b)) {
         if (fetch.t != tok) {
-            if (P.trace && tok < P.trace_tokens)
-                P.trace[((size_t)blockIdx.x * P.trace_tokens + tok) * P.trace_events + P.trace_events - 1] = waited;
+            trace_producer_wait(P, tok, waited);
             waited = 0;
             tok = fetch.t;
         }
@@ -312,12 +431,122 @@ __device__ void produce(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint
         bulk_g2s(ring + (size_t)slot * KIE_SLOT_BYTES, a, b, &S.full[slot]);
         ring_it++;
     }
-    if (P.trace && tok < P.trace_tokens)
-        P.trace[((size_t)blockIdx.x * P.trace_tokens + tok) * P.trace_events + P.trace_events - 1] = waited;
+    trace_producer_wait(P, tok, waited);
     // Wait until every copy issued into the ring has landed before anyone may leave.
     const uint32_t first = ring_it > KIE_NSLOT ? ring_it - KIE_NSLOT : 0;
     for (uint32_t k = first; k < ring_it; k++)
         mbar_wait(&S.full[k % KIE_NSLOT], (k / KIE_NSLOT) & 1u, P.timeout_ns, nullptr);
+}
+
+// With TMEM staging, the first KIE_NTS chunks after each layer's QKV rows (its O-fold columns,
+// then gate/up rows) move on from their ring slot into TMEM slot (m % KIE_NTS), m counting the
+// moved chunks. Those are the chunks the producer fetches while the consumers are in the
+// attention step and its grid barriers; moving them frees their ring slots for the next chunks,
+// so the stream runs 7 chunks ahead there instead of 3. Every other chunk is read from the ring
+// as without staging (the steady stream keeps its rate). A ring slot is free once its chunk
+// has been read (16 consumer warps) or moved (the producer's 15 arrivals plus the copies'
+// completion). Moves are issued in order; one waits for its chunk to land and for the
+// consumers to be done with the TMEM slot's previous chunk, while the bulk copies run ahead.
+__device__ __forceinline__ bool via_tmem(int cq) { return cq >= 0 && cq < KIE_NTS; }
+
+__device__ void produce_tmem(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint32_t &tm_it, uint8_t *ring,
+                             const KieCmd &cmd) {
+    const uint8_t *seg = P.wpack + P.seg_off[blockIdx.x];
+    ChunkIter fetch;
+    chunk_begin(fetch, seg);
+    const uint8_t *a = nullptr;
+    uint32_t b = 0;
+    bool more = chunk_next(P, S, cmd, fetch, a, b);
+    // moves waiting for their chunk to land or their TMEM slot: (chunk, phase), at most one per ring slot
+    uint32_t mv_chunk[KIE_NSLOT];
+    int mv_ph[KIE_NSLOT];
+    int mv_n = 0, mv_head = 0;
+    int tok = 0;
+    unsigned long long waited = 0;
+    uint64_t stall0 = 0;  // start of the current stall (0: making progress)
+    const uint32_t ring_s = smem_u32(ring);
+    const uint32_t tbase = S.tmem_base;
+    while (more || mv_n > 0) {
+        bool progress = false;
+        if (more) {
+            const uint32_t slot = ring_it % KIE_NSLOT, par = (ring_it / KIE_NSLOT) & 1u;
+            if (mbar_test_wait(&S.empty[slot], par ^ 1u)) {
+                if (fetch.t != tok) {
+                    trace_producer_wait(P, tok, waited);
+                    waited = 0;
+                    tok = fetch.t;
+                }
+                mbar_arrive_expect_tx(&S.full[slot], b);
+                bulk_g2s(ring + (size_t)slot * KIE_SLOT_BYTES, a, b, &S.full[slot]);
+                if (via_tmem(fetch.cq)) {
+                    const int q = (mv_head + mv_n) % KIE_NSLOT;
+                    mv_chunk[q] = ring_it;
+                    mv_ph[q] = fetch.ph;
+                    mv_n++;
+                }
+                ring_it++;
+                more = chunk_next(P, S, cmd, fetch, a, b);
+                progress = true;
+            }
+        }
+        if (mv_n > 0) {
+            const uint32_t c = mv_chunk[mv_head];
+            const uint32_t slot = c % KIE_NSLOT, par = (c / KIE_NSLOT) & 1u;
+            const uint32_t ts = tm_it % KIE_NTS, tpar = (tm_it / KIE_NTS) & 1u;
+            if (mbar_test_wait(&S.full[slot], par) && mbar_test_wait(&S.tempty[ts], tpar ^ 1u)) {
+                tm_fence_after();
+                const int ph = mv_ph[mv_head];
+#pragma unroll 4
+                for (int j = 0; j < 16; j++) {
+                    uint32_t off, lbo;
+                    tm_copy_src(ph, P.d, j, off, lbo);
+                    tm_cp(tbase + ts * 128u + 8u * (uint32_t)j,
+                          tm_desc(ring_s + slot * (uint32_t)KIE_SLOT_BYTES + off, lbo, 128u));
+                }
+                tm_commit(&S.tfull[ts]);
+                tm_commit(&S.empty[slot]);                     // the last arrival: the copies are done
+                mbar_arrive_n(&S.empty[slot], KIE_CONS_WARPS - 1);  // in place of the consumer warps
+                tm_it++;
+                mv_head = (mv_head + 1) % KIE_NSLOT;
+                mv_n--;
+                progress = true;
+            }
+        }
+        if (progress) {
+            if (stall0) waited += globaltimer() - stall0;
+            stall0 = 0;
+            continue;
+        }
+        const uint64_t now = globaltimer();
+        if (!stall0) stall0 = now;
+        if (S.abort) break;
+        if ((long long)(now - stall0) > P.timeout_ns) {
+            set_error(P.err, DERR_RING_TIMEOUT, 0x81);
+            S.abort = 1;
+            break;
+        }
+        // nothing to issue: sleep in hardware on the event most likely to come next (bounded, so
+        // that the other stage is looked at again soon), leaving the issue slots to the consumers
+        if (mv_n > 0) {
+            const uint32_t c = mv_chunk[mv_head];
+            if (!mbar_test_wait(&S.full[c % KIE_NSLOT], (c / KIE_NSLOT) & 1u))
+                mbar_try_wait_ns(&S.full[c % KIE_NSLOT], (c / KIE_NSLOT) & 1u, 256);
+            else
+                mbar_try_wait_ns(&S.tempty[tm_it % KIE_NTS], ((tm_it / KIE_NTS) & 1u) ^ 1u, 256);
+        } else if (more) {
+            mbar_try_wait_ns(&S.empty[ring_it % KIE_NSLOT], ((ring_it / KIE_NSLOT) & 1u) ^ 1u, 256);
+        }
+    }
+    if (stall0) waited += globaltimer() - stall0;
+    trace_producer_wait(P, tok, waited);
+    // Before anyone may leave: every bulk copy issued has landed, and every move has completed
+    // (a move's commit is the last arrival on its ring slot's empty barrier).
+    for (uint32_t k = (ring_it > KIE_NSLOT ? ring_it - KIE_NSLOT : 0); k < ring_it; k++)
+        mbar_wait(&S.full[k % KIE_NSLOT], (k / KIE_NSLOT) & 1u, P.timeout_ns, nullptr);
+    for (uint32_t k = 0; k < KIE_NTS && k < tm_it; k++) {
+        const uint32_t m = tm_it - 1 - k;
+        mbar_wait(&S.tfull[m % KIE_NTS], (m / KIE_NTS) & 1u, P.timeout_ns, nullptr);
+    }
 }
 
 // --------------------------------------------------------------- consumer: GEMV phases
@@ -327,9 +556,9 @@ __device__ void produce(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint
 // S.wpart (see rowsum).
 // With E4M3 weights, rsc receives the row scales the phase's epilogue applies: rows 2*tid and
 // 2*tid + 1 of this CTA (the QKV and gate/up pairs), or rows tid and tid + 512 (head).
-template <int DT, bool F8, int NV, int CR, int CS>
-__device__ void gemv_phase(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring, int ph, int l,
-                           int tok, int pos, int t, float2 &rsc) {
+template <int DT, bool F8, bool TM, int NV, int CR, int CS>
+__device__ void gemv_phase(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint32_t &tm_it, int &lq,
+                           const uint8_t *ring, int ph, int l, int tok, int pos, int t, float2 &rsc) {
     using WV = WVec<DT, F8>;
     constexpr int ESZ = F8 ? 1 : 2;
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
@@ -359,7 +588,10 @@ __device__ void gemv_phase(const KieParams &P, B1Shared &S, uint32_t &ring_it, c
 #pragma unroll
         for (int e = 0; e < 8; e++) h[i][e] = 0.f;
         if (v < nvec) {
-            const int col0 = (w % CS) * kslice + 8 * v;  // 8 consecutive columns, 32-byte aligned
+            // 8 consecutive columns, 32-byte aligned. With TMEM staging and two vectors per lane,
+            // vector i covers columns i K/2 + (w % CS) K/16 + 8 lane (the staging layout's column
+            // halves); else the slice's columns in order.
+            const int col0 = (TM && NV == 2) ? i * (K / 2) + (w % CS) * (K / 16) + 8 * lane : (w % CS) * kslice + 8 * v;
             if (from_emb) {
                 cvt8<DT>(__ldg(reinterpret_cast<const uint4 *>(P.emb + (size_t)tok * P.d + col0)), h[i]);
             } else {
@@ -401,10 +633,27 @@ __device__ void gemv_phase(const KieParams &P, B1Shared &S, uint32_t &ring_it, c
 #endif
     // a chunk holds SUB blocks of GROUPS * CR rows (two with one-byte weights)
     constexpr int SUB = 2 / ESZ;
-    for (int c0 = 0; c0 < rows; c0 += SUB * GROUPS * CR) {
+    constexpr int CH = SUB * GROUPS * CR;
+    // with TMEM staging, the chunks among the layer's first KIE_NTS after its QKV rows were
+    // moved into TMEM (lq: chunks of the layer seen so far; -1 for the QKV and head phases)
+    int ntm = 0;
+    if (TM && lq >= 0) {
+        const int nch = (rows + CH - 1) / CH;
+        ntm = min(max(KIE_NTS - lq, 0), nch);
+        lq += nch;
+    }
+    // byte offset of vector i of this lane within a row: with TMEM staging and two vectors per
+    // lane the staging layout's column halves, else the slice's columns in order
+    auto colb = [&](int i) {
+        return ((TM && NV == 2) ? i * (K / 2) + ws * (K / 16) + 8 * lane : ws * kslice + 8 * (lane + 32 * i)) * ESZ;
+    };
+    for (int c0 = 0, ci = 0; c0 < rows; c0 += CH, ci++) {
+        const bool via = TM && ci < ntm;
         const uint32_t slot = ring_it % KIE_NSLOT, par = (ring_it / KIE_NSLOT) & 1u;
+        const uint32_t ts = tm_it % KIE_NTS, tpar = (tm_it / KIE_NTS) & 1u;
         ring_it++;
-        bool have = ring_take(P, S, slot, par, ph);
+        if (via) tm_it++;
+        bool have = via ? tmem_take(P, S, ts, tpar, ph) : ring_take(P, S, slot, par, ph);
         have = __all_sync(0xffffffffu, have);  // one decision per warp (the reduction needs all lanes)
 #ifdef KIE_PROFILE_GEMV
         c_ready = clock64();
@@ -414,12 +663,38 @@ __device__ void gemv_phase(const KieParams &P, B1Shared &S, uint32_t &ring_it, c
             S.abort = 1;
             continue;  // keep the control flow; the command ends at the next barrier
         }
+        if constexpr (TM) {
+            if (via) {  // 16-bit weights: one block of GROUPS * CR rows; piece r NV + i is row r, vector i
+                uint32_t tw[32];
+                tmem_read_chunk(S, ts, tw);
+                const int r0 = c0 + grp * CR;
+                const int nr = max(0, min(CR, rows - r0));
+                float acc[8];
+#pragma unroll
+                for (int r = 0; r < 8; r++) acc[r] = 0.f;
+#pragma unroll
+                for (int r = 0; r < CR; r++) {
+                    if (r < nr) {
+#pragma unroll
+                        for (int i = 0; i < NV; i++) {
+                            float f[8];
+                            cvt8<DT>(tm_piece(tw, r * NV + i), f);
+#pragma unroll
+                            for (int e = 0; e < 8; e++) acc[r] = fmaf(f[e], h[i][e], acc[r]);
+                        }
+                    }
+                }
+                const float s = warp_reduce_rows<CR>(acc);
+                constexpr int LPR = 32 / CR;
+                if ((lane % LPR) == 0 && lane / LPR < nr) S.wpart[ws * STRIDE + r0 + lane / LPR] = s;
+                continue;
+            }
+        }
 #pragma unroll
         for (int sub = 0; sub < SUB; sub++) {
             const int r0 = c0 + (sub * GROUPS + grp) * CR;  // this group's first row in the block
             const int nr = max(0, min(CR, rows - r0));
-            const uint8_t *base = ring + (size_t)slot * KIE_SLOT_BYTES +
-                                  ((size_t)(sub * GROUPS + grp) * CR * K + (size_t)ws * kslice) * ESZ;
+            const uint8_t *base = ring + (size_t)slot * KIE_SLOT_BYTES + (size_t)(sub * GROUPS + grp) * CR * K * ESZ;
             float acc[8];
 #pragma unroll
             for (int r = 0; r < 8; r++) acc[r] = 0.f;
@@ -432,7 +707,7 @@ __device__ void gemv_phase(const KieParams &P, B1Shared &S, uint32_t &ring_it, c
                         const int v = lane + 32 * i;
                         if (v < nvec) {
                             float f[8];
-                            WV::cvt(*reinterpret_cast<const typename WV::T *>(rowp + v * WV::BYTES), f);
+                            WV::cvt(*reinterpret_cast<const typename WV::T *>(rowp + colb(i)), f);
 #pragma unroll
                             for (int e = 0; e < 8; e++) acc[r] = fmaf(f[e], h[i][e], acc[r]);
                         }
@@ -466,13 +741,13 @@ __device__ __forceinline__ float rowsum(const B1Shared &S, int r, int cs) {
     return v;
 }
 
-template <int DT, bool F8>
-__device__ __forceinline__ float2 gemv_dispatch(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring,
-                                                int ph, int l, int tok, int pos, int t) {
+template <int DT, bool F8, bool TM>
+__device__ __forceinline__ float2 gemv_dispatch(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint32_t &tm_it,
+                                                int &lq, const uint8_t *ring, int ph, int l, int tok, int pos, int t) {
     const int K = P.K[ph];
     float2 rsc;
-    if (K <= 2048) gemv_phase<DT, F8, 1, 8, 8>(P, S, ring_it, ring, ph, l, tok, pos, t, rsc);
-    else gemv_phase<DT, F8, 2, 4, 8>(P, S, ring_it, ring, ph, l, tok, pos, t, rsc);  // K <= 4096
+    if (K <= 2048) gemv_phase<DT, F8, TM, 1, 8, 8>(P, S, ring_it, tm_it, lq, ring, ph, l, tok, pos, t, rsc);
+    else gemv_phase<DT, F8, TM, 2, 4, 8>(P, S, ring_it, tm_it, lq, ring, ph, l, tok, pos, t, rsc);  // K <= 4096
     return rsc;
 }
 
@@ -480,58 +755,90 @@ __device__ __forceinline__ float2 gemv_dispatch(const KieParams &P, B1Shared &S,
 
 // One fold (O or down): this CTA's 8-column groups of W arrive as [group][d rows][8], and
 // S.fold_in holds 8 inputs per group. Thread t accumulates rows t + 512 j over all groups.
-template <int DT, bool F8, int RPT>
-__device__ void fold_rows(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring, int ph,
-                          float (&acc)[RPT]) {
+template <int DT, bool F8, bool TM, int RPT>
+__device__ void fold_rows(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint32_t &tm_it, int &lq,
+                          const uint8_t *ring, int ph, float (&acc)[RPT]) {
     using WV = WVec<DT, F8>;
     const int tid = threadIdx.x, lane = tid & 31;
     const int d = P.d, ng = S.row1[ph] - S.row0[ph], cpc = P.cr[ph];
 #pragma unroll
     for (int j = 0; j < RPT; j++) acc[j] = 0.f;
     named_bar_sync(1, KIE_CONS_THREADS);  // S.fold_in was written by other warps of this CTA
-    for (int g0 = 0; g0 < ng; g0 += cpc) {
+    int ntm = 0;  // leading chunks staged in TMEM (see gemv_phase)
+    if (TM && lq >= 0) {
+        const int nch = (ng + cpc - 1) / cpc;
+        ntm = min(max(KIE_NTS - lq, 0), nch);
+        lq += nch;
+    }
+    for (int g0 = 0, ci = 0; g0 < ng; g0 += cpc, ci++) {
         const int n = min(cpc, ng - g0);
+        const bool via = TM && ci < ntm;
         const uint32_t slot = ring_it % KIE_NSLOT, par = (ring_it / KIE_NSLOT) & 1u;
+        const uint32_t ts = tm_it % KIE_NTS, tpar = (tm_it / KIE_NTS) & 1u;
         ring_it++;
-        bool have = ring_take(P, S, slot, par, ph);
+        if (via) tm_it++;
+        bool have = via ? tmem_take(P, S, ts, tpar, ph) : ring_take(P, S, slot, par, ph);
         have = __all_sync(0xffffffffu, have);
         if (!have) {
             if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, (unsigned)ph);
             S.abort = 1;
             continue;
         }
-        const uint8_t *base = ring + (size_t)slot * KIE_SLOT_BYTES;
-        for (int gi = 0; gi < n; gi++) {
-            const float4 a = *reinterpret_cast<const float4 *>(&S.fold_in[(g0 + gi) * 8]);
-            const float4 b = *reinterpret_cast<const float4 *>(&S.fold_in[(g0 + gi) * 8 + 4]);
-            const float in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        if (TM && via) {
+            // the chunk's cpc = 8 / RPT column groups: piece k = gi RPT + j is row tid + 512 j of group gi
+            uint32_t tw[32];
+            tmem_read_chunk(S, ts, tw);
 #pragma unroll
-            for (int j = 0; j < RPT; j++) {
-                const int r = tid + KIE_CONS_THREADS * j;
-                if (r < d) {
-                    float f[8];
-                    WV::cvt(*reinterpret_cast<const typename WV::T *>(base + ((size_t)gi * d + r) * WV::BYTES), f);
+            for (int gi = 0; gi < 8 / RPT; gi++) {
+                if (gi < n) {
+                    const float4 a = *reinterpret_cast<const float4 *>(&S.fold_in[(g0 + gi) * 8]);
+                    const float4 b = *reinterpret_cast<const float4 *>(&S.fold_in[(g0 + gi) * 8 + 4]);
+                    const float in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-                    for (int e = 0; e < 8; e++) acc[j] = fmaf(f[e], in[e], acc[j]);
+                    for (int j = 0; j < RPT; j++) {
+                        float f[8];
+                        cvt8<DT>(tm_piece(tw, gi * RPT + j), f);
+#pragma unroll
+                        for (int e = 0; e < 8; e++) acc[j] = fmaf(f[e], in[e], acc[j]);
+                    }
                 }
             }
+        } else {
+            const uint8_t *base = ring + (size_t)slot * KIE_SLOT_BYTES;
+            for (int gi = 0; gi < n; gi++) {
+                const float4 a = *reinterpret_cast<const float4 *>(&S.fold_in[(g0 + gi) * 8]);
+                const float4 b = *reinterpret_cast<const float4 *>(&S.fold_in[(g0 + gi) * 8 + 4]);
+                const float in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int j = 0; j < RPT; j++) {
+                    const int r = tid + KIE_CONS_THREADS * j;
+                    if (r < d) {
+                        float f[8];
+                        WV::cvt(*reinterpret_cast<const typename WV::T *>(base + ((size_t)gi * d + r) * WV::BYTES), f);
+#pragma unroll
+                        for (int e = 0; e < 8; e++) acc[j] = fmaf(f[e], in[e], acc[j]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.empty[slot]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.empty[slot]);
     }
 }
 
 // x[r] += acc (times the row's scale with E4M3 weights) for this thread's rows (fp32 atomics:
 // the folds of all CTAs meet in x)
 template <int RPT>
-__device__ __forceinline__ void fold_commit(const KieParams &P, const B1Shared &S, const float (&acc)[RPT], int ph,
+__device__ __forceinline__ void fold_commit(const KieParams &P, B1Shared &S, const float (&acc)[RPT], int ph,
                                             const float (&scl)[RPT]) {
     if (S.abort || S.row1[ph] == S.row0[ph]) return;
+    uint32_t tok = 0;
 #pragma unroll
     for (int j = 0; j < RPT; j++) {
         const int r = threadIdx.x + KIE_CONS_THREADS * j;
-        if (r < P.d) atomicAdd(P.x + r, acc[j] * scl[j]);
+        if (r < P.d) pub_add_f32(P.x + r, acc[j] * scl[j], tok);
     }
+    pub_wait(tok, &S.pub_sink);  // the next grid barrier's arrive follows these adds' completion
 }
 
 // the fold's row scales (E4M3 weights), loaded before the fold so they arrive under its work
@@ -548,42 +855,54 @@ __device__ __forceinline__ void fold_scales(const KieParams &P, int l, int off, 
 
 __device__ __forceinline__ void attention_prefetch(const KieParams &P, B1Shared &S, int l, int sid, int pos);
 
-// q/k rows come in rotation pairs (dim i, dim i + D/2); v rows use the same pairing.
+// q/k rows come in rotation pairs (dim i, dim i + D/2); v rows use the same pairing. Thread p
+// takes pair p (npair <= 512); the CTA's pairs come two at a time as dims (i, i + 1), i even, of
+// one head, so the even thread of each two writes both dims as one word (q: two fp32 values,
+// k and v: two 16-bit values), published by completion for the attention step.
 template <int DT>
 __device__ void epilogue_qkv(const KieParams &P, B1Shared &S, int l, int sid, int pos, int tok, float2 rsc) {
     const int D = P.D, half = D >> 1, qd = P.Hq * D, kvd = P.Hkv * D;
     const int rbeg = S.row0[PH_QKV], npair = (S.row1[PH_QKV] - rbeg) >> 1;
     const size_t sess = (size_t)sid * P.sess_stride;
-    for (int p = threadIdx.x; p < npair; p += KIE_CONS_THREADS) {
-        const int r = rbeg + 2 * p;
+    const int p = threadIdx.x;
+    const int r = rbeg + 2 * p;
+    const int i = (r % D) >> 1;
+    const bool act = p < npair;
+    float ra = 0.f, rb = 0.f;
+    if (act) {
         const int cs = col_slices(P.K[PH_QKV]);
-        const float a = rowsum(S, 2 * p, cs) * rsc.x, b = rowsum(S, 2 * p + 1, cs) * rsc.y;  // (p == tid)
-        const int i = (r % D) >> 1;
-        if (r < qd + kvd) {
-            const float2 cs = S.rope_s[i];
-            const float ra = a * cs.x - b * cs.y, rb = b * cs.x + a * cs.y;
-            if (r < qd) {
-                const int hh = r / D;
-                P.q[hh * D + i] = ra;
-                P.q[hh * D + i + half] = rb;
-            } else {
-                const int g = (r - qd) / D;
-                uint16_t *kp = P.kcache + sess + ((size_t)(l * P.Hkv + g) * P.max_ctx + pos) * D;
-                kp[i] = store1<DT>(ra);
-                kp[i + half] = store1<DT>(rb);
-            }
+        const float a = rowsum(S, 2 * p, cs) * rsc.x, b = rowsum(S, 2 * p + 1, cs) * rsc.y;
+        if (r < qd + kvd) {  // rotate q and k
+            const float2 c = S.rope_s[i];
+            ra = a * c.x - b * c.y;
+            rb = b * c.x + a * c.y;
         } else {
-            const int g = (r - qd - kvd) / D;
-            uint16_t *vp = P.vcache + sess + ((size_t)(l * P.Hkv + g) * P.max_ctx + pos) * D;
-            vp[i] = store1<DT>(a);
-            vp[i + half] = store1<DT>(b);
+            ra = a;
+            rb = b;
+        }
+    }
+    const float ra1 = __shfl_down_sync(0xffffffffu, ra, 1), rb1 = __shfl_down_sync(0xffffffffu, rb, 1);
+    uint32_t tk = 0;
+    if (act && (p & 1) == 0) {
+        auto pack = [](float x0, float x1) { return (uint32_t)store1<DT>(x0) | ((uint32_t)store1<DT>(x1) << 16); };
+        if (r < qd) {
+            float *qp = P.q + (r / D) * D;
+            pub_f32x2(qp + i, ra, ra1, tk);
+            pub_f32x2(qp + i + half, rb, rb1, tk);
+        } else {
+            const bool isk = r < qd + kvd;
+            const int g = (r - qd - (isk ? 0 : kvd)) / D;
+            uint16_t *cp = (isk ? P.kcache : P.vcache) + sess + ((size_t)(l * P.Hkv + g) * P.max_ctx + pos) * D;
+            pub_u32(cp + i, pack(ra, ra1), tk);
+            pub_u32(cp + i + half, pack(rb, rb1), tk);
         }
     }
     if (l == 0) {  // the residual starts as the embedding row (each CTA writes a 1/nblk share)
         const int r0 = (int)((long long)blockIdx.x * P.d / P.nblk), r1 = (int)((long long)(blockIdx.x + 1) * P.d / P.nblk);
-        for (int r = r0 + threadIdx.x; r < r1; r += KIE_CONS_THREADS) P.x[r] = cvt1<DT>(P.emb[(size_t)tok * P.d + r]);
+        for (int rr = r0 + threadIdx.x; rr < r1; rr += KIE_CONS_THREADS) pub_f32(P.x + rr, cvt1<DT>(P.emb[(size_t)tok * P.d + rr]), tk);
         attention_prefetch(P, S, l, sid, pos);
     }
+    pub_wait(tk, &S.pub_sink);
 }
 
 // The cache rows this CTA's attention unit will read in layer l are read into L2 ahead of
@@ -655,9 +974,11 @@ __device__ void epilogue_head(const KieParams &P, B1Shared &S, float *logits, fl
         float v = lane < KIE_CONS_WARPS ? S.red[lane] : -CUDART_INF_F;
         int i = lane < KIE_CONS_WARPS ? S.redi[lane] : 0x7fffffff;
         warp_argmax(v, i);
-        if (lane == 0) {
-            P.cand_val[blockIdx.x] = v;
-            P.cand_idx[blockIdx.x] = i;
+        if (lane == 0) {  // published by completion for the head's grid barrier
+            uint32_t tk = 0;
+            pub_f32(P.cand_val + blockIdx.x, v, tk);
+            pub_u32(P.cand_idx + blockIdx.x, (uint32_t)i, tk);
+            pub_wait(tk, &S.pub_sink);
         }
     }
 }
@@ -699,10 +1020,12 @@ __device__ __noinline__ void sample_local(B1Shared &S, float *logits, int k, int
     } else {
         named_bar_sync(1, KIE_CONS_THREADS);
     }
-    if (tid < KIE_TOPK_MAX) {
+    if (tid < KIE_TOPK_MAX) {  // published by completion for the head's grid barrier
         const bool have = tid < kl;
-        cand_tv[blockIdx.x * KIE_TOPK_MAX + tid] = have ? S.samp.ss.top_v[tid] : CUDART_NAN_F;
-        cand_ti[blockIdx.x * KIE_TOPK_MAX + tid] = have ? S.samp.ss.top_i[tid] : V + tid;
+        uint32_t tk = 0;
+        pub_f32(cand_tv + blockIdx.x * KIE_TOPK_MAX + tid, have ? S.samp.ss.top_v[tid] : CUDART_NAN_F, tk);
+        pub_u32(cand_ti + blockIdx.x * KIE_TOPK_MAX + tid, (uint32_t)(have ? S.samp.ss.top_i[tid] : V + tid), tk);
+        pub_wait(tk, &S.pub_sink);
     }
 }
 
@@ -773,49 +1096,61 @@ __device__ void attention_step(const KieParams &P, B1Shared &S, int l, int sid, 
 }
 
 // the two folds of a layer and the down fold's split barrier, by rows per thread
-template <int DT, bool F8, int RPT>
-__device__ __forceinline__ void o_fold(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring, int l) {
+template <int DT, bool F8, bool TM, int RPT>
+__device__ __forceinline__ void o_fold(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint32_t &tm_it, int &lq,
+                                       const uint8_t *ring, int l) {
     float acc[RPT], scl[RPT];
     fold_scales<F8, RPT>(P, l, sc_off_o(P), scl);
-    fold_rows<DT, F8, RPT>(P, S, ring_it, ring, PH_OF, acc);
+    fold_rows<DT, F8, TM, RPT>(P, S, ring_it, tm_it, lq, ring, PH_OF, acc);
     fold_commit<RPT>(P, S, acc, PH_OF, scl);
 }
 
-template <int DT, bool F8, int RPT>
-__device__ __forceinline__ void down_fold(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring,
-                                          int l, unsigned long long rd_epoch, int t, int e) {
+template <int DT, bool F8, bool TM, int RPT>
+__device__ __forceinline__ void down_fold(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint32_t &tm_it, int &lq,
+                                          const uint8_t *ring, int l, unsigned long long rd_epoch, int t, int e) {
     float acc[RPT], scl[RPT];
     fold_scales<F8, RPT>(P, l, sc_off_down(P), scl);
-    fold_rows<DT, F8, RPT>(P, S, ring_it, ring, PH_DF, acc);
+    fold_rows<DT, F8, TM, RPT>(P, S, ring_it, tm_it, lq, ring, PH_DF, acc);
     residual_read_wait(P, S, rd_epoch);  // every CTA has read x for its gate/up norm
     trace_mark(P, t, e + 10);
     fold_commit<RPT>(P, S, acc, PH_DF, scl);
 }
 
 // rows per thread of a fold (d <= 4096): 1, 2, 4 or 8
-template <int DT, bool F8>
-__device__ __forceinline__ void o_fold_any(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring,
-                                           int l) {
-    if (P.d <= 512) o_fold<DT, F8, 1>(P, S, ring_it, ring, l);
-    else if (P.d <= 1024) o_fold<DT, F8, 2>(P, S, ring_it, ring, l);
-    else if (P.d <= 2048) o_fold<DT, F8, 4>(P, S, ring_it, ring, l);
-    else o_fold<DT, F8, 8>(P, S, ring_it, ring, l);
+template <int DT, bool F8, bool TM>
+__device__ __forceinline__ void o_fold_any(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint32_t &tm_it,
+                                           int &lq, const uint8_t *ring, int l) {
+    if constexpr (TM) {  // d is 2048 or 4096
+        if (P.d <= 2048) o_fold<DT, F8, TM, 4>(P, S, ring_it, tm_it, lq, ring, l);
+        else o_fold<DT, F8, TM, 8>(P, S, ring_it, tm_it, lq, ring, l);
+        return;
+    }
+    if (P.d <= 512) o_fold<DT, F8, TM, 1>(P, S, ring_it, tm_it, lq, ring, l);
+    else if (P.d <= 1024) o_fold<DT, F8, TM, 2>(P, S, ring_it, tm_it, lq, ring, l);
+    else if (P.d <= 2048) o_fold<DT, F8, TM, 4>(P, S, ring_it, tm_it, lq, ring, l);
+    else o_fold<DT, F8, TM, 8>(P, S, ring_it, tm_it, lq, ring, l);
 }
 
-template <int DT, bool F8>
-__device__ __forceinline__ void down_fold_any(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring,
-                                              int l, unsigned long long rd_epoch, int t, int e) {
-    if (P.d <= 512) down_fold<DT, F8, 1>(P, S, ring_it, ring, l, rd_epoch, t, e);
-    else if (P.d <= 1024) down_fold<DT, F8, 2>(P, S, ring_it, ring, l, rd_epoch, t, e);
-    else if (P.d <= 2048) down_fold<DT, F8, 4>(P, S, ring_it, ring, l, rd_epoch, t, e);
-    else down_fold<DT, F8, 8>(P, S, ring_it, ring, l, rd_epoch, t, e);
+template <int DT, bool F8, bool TM>
+__device__ __forceinline__ void down_fold_any(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint32_t &tm_it,
+                                              int &lq, const uint8_t *ring, int l, unsigned long long rd_epoch, int t,
+                                              int e) {
+    if constexpr (TM) {  // d is 2048 or 4096
+        if (P.d <= 2048) down_fold<DT, F8, TM, 4>(P, S, ring_it, tm_it, lq, ring, l, rd_epoch, t, e);
+        else down_fold<DT, F8, TM, 8>(P, S, ring_it, tm_it, lq, ring, l, rd_epoch, t, e);
+        return;
+    }
+    if (P.d <= 512) down_fold<DT, F8, TM, 1>(P, S, ring_it, tm_it, lq, ring, l, rd_epoch, t, e);
+    else if (P.d <= 1024) down_fold<DT, F8, TM, 2>(P, S, ring_it, tm_it, lq, ring, l, rd_epoch, t, e);
+    else if (P.d <= 2048) down_fold<DT, F8, TM, 4>(P, S, ring_it, tm_it, lq, ring, l, rd_epoch, t, e);
+    else down_fold<DT, F8, TM, 8>(P, S, ring_it, tm_it, lq, ring, l, rd_epoch, t, e);
 }
 
 // --------------------------------------------------------------- consumer: one command
 
-template <int DT, bool F8>
-__device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, const uint8_t *ring, const KieCmd &cmd,
-                        unsigned long long &epoch, unsigned long long &rd_epoch, uint32_t &att_use) {
+template <int DT, bool F8, bool TM>
+__device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint32_t &tm_it, const uint8_t *ring,
+                        const KieCmd &cmd, unsigned long long &epoch, unsigned long long &rd_epoch, uint32_t &att_use) {
     int tok = cmd.in_tok;
     if (cmd.op == OP_DECODE && cmd.tok_dev) tok = __ldcg(cmd.tok_dev);
     const int L = P.L;
@@ -839,7 +1174,9 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, cons
         for (int l = 0; l < L; l++) {
             const int e = 1 + 16 * l;
             // A: QKV
-            const float2 sq = gemv_dispatch<DT, F8>(P, S, ring_it, ring, PH_QKV, l, tok, pos, t);
+            int lq = -1;  // the QKV rows are never staged in TMEM
+            const float2 sq = gemv_dispatch<DT, F8, TM>(P, S, ring_it, tm_it, lq, ring, PH_QKV, l, tok, pos, t);
+            lq = 0;  // the chunks of the O fold, gate/up rows and down fold, counted from here
             trace_mark(P, t, e);
             epilogue_qkv<DT>(P, S, l, cmd.sid, pos, tok, sq);
             trace_mark(P, t, e + 1);
@@ -848,25 +1185,26 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, cons
             if (P.trace && t < P.trace_tokens && threadIdx.x == 0)  // end of this CTA's positions (0: no unit)
                 P.trace[((size_t)blockIdx.x * P.trace_tokens + t) * P.trace_events + e + 15] = S.at.t_unit;
             trace_mark(P, t, e + 3);
-            o_fold_any<DT, F8>(P, S, ring_it, ring, l);
+            o_fold_any<DT, F8, TM>(P, S, ring_it, tm_it, lq, ring, l);
             trace_mark(P, t, e + 4);
             grid_barrier(P, S, epoch, P.timeout_ns, 2);
             trace_mark(P, t, e + 5);
             // C: gate/up, then the down fold
-            const float2 sg = gemv_dispatch<DT, F8>(P, S, ring_it, ring, PH_GU, l, tok, pos, t);
+            const float2 sg = gemv_dispatch<DT, F8, TM>(P, S, ring_it, tm_it, lq, ring, PH_GU, l, tok, pos, t);
             residual_read_arrive(P, S);  // this CTA's reads of x are done
             rd_epoch++;
             trace_mark(P, t, e + 6);
             epilogue_gu(P, S, l, cmd.sid, pos, sg);
             trace_mark(P, t, e + 7);
-            down_fold_any<DT, F8>(P, S, ring_it, ring, l, rd_epoch, t, e);
+            down_fold_any<DT, F8, TM>(P, S, ring_it, tm_it, lq, ring, l, rd_epoch, t, e);
             trace_mark(P, t, e + 8);
             grid_barrier(P, S, epoch, P.timeout_ns, 3);
             trace_mark(P, t, e + 9);
         }
         const int eh = 1 + 16 * L;
         if (head) {
-            const float2 sh = gemv_dispatch<DT, F8>(P, S, ring_it, ring, PH_HEAD, L, tok, pos, t);
+            int lq = -1;
+            const float2 sh = gemv_dispatch<DT, F8, TM>(P, S, ring_it, tm_it, lq, ring, PH_HEAD, L, tok, pos, t);
             float *lg = nullptr;
             if (cmd.logits) lg = cmd.logits + (cmd.op == OP_PREFILL ? 0 : (size_t)t * P.V);
             if (sc.top_k > 1) sample_local(S, lg, sc.top_k, col_slices(P.K[PH_HEAD]), P.cand_tv, P.cand_ti, P.V, sh);
@@ -893,7 +1231,7 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, cons
 
 // --------------------------------------------------------------- the kernel
 
-template <int DT, bool F8>
+template <int DT, bool F8, bool TM>
 __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, KieCmd one, int resident) {
     extern __shared__ __align__(1024) uint8_t smem[];
     B1Shared &S = *reinterpret_cast<B1Shared *>(smem + RING_BYTES);
@@ -901,7 +1239,13 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
     if (tid == 0) {
         for (int i = 0; i < KIE_NSLOT; i++) {
             mbar_init(&S.full[i], 1);
-            mbar_init(&S.empty[i], KIE_CONS_WARPS);  // both groups read every chunk
+            // a chunk's 16 consumer warps, or (moved into TMEM) the producer's 15 arrivals and
+            // the commit of the copies
+            mbar_init(&S.empty[i], KIE_CONS_WARPS);
+        }
+        for (int i = 0; i < KIE_NTS; i++) {
+            mbar_init(&S.tfull[i], 1);
+            mbar_init(&S.tempty[i], KIE_CONS_WARPS);
         }
         fence_mbar_init();
         S.abort = 0;
@@ -910,8 +1254,12 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
         S.row0[tid] = P.row0[tid * (P.nblk + 1) + blockIdx.x];
         S.row1[tid] = P.row0[tid * (P.nblk + 1) + blockIdx.x + 1];
     }
+    if (TM && tid < 32) tm_alloc(&S.tmem_base);  // all 512 columns (one CTA per SM); freed at exit
+    tm_fence_before();
     __syncthreads();
+    tm_fence_after();
     uint32_t ring_it = 0;  // chunks consumed (consumers) / issued (producer); both advance identically
+    uint32_t tm_it = 0;    // chunks staged in TMEM, counted the same way on both sides
     unsigned long long epoch = 0;
     unsigned long long rd_epoch = 0;  // split-barrier arrivals of this CTA so far in this launch
     uint32_t att_use = 0;  // attention phases so far in this launch (the merge counters' targets)
@@ -947,7 +1295,7 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
                         for (int j = tid; j < S.cmd.n; j += KIE_CONS_THREADS)
                             P.tokbuf[j] = ((const volatile int32_t *)S.cmd.tokens)[j];
                 }
-                grid_barrier(P, S, epoch, P.idle_ns + P.timeout_ns, 0);
+                grid_barrier(P, S, epoch, P.idle_ns + P.timeout_ns, 0, true);
                 if (tid == 0) {
                     copy_words_cg(&S.cmd, P.cmd);
                     if (S.abort) S.cmd.op = OP_EXIT;
@@ -958,9 +1306,12 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
         const KieCmd cmd = S.cmd;
         if (cmd.op != OP_DECODE && cmd.op != OP_PREFILL) break;
         if (tid >= KIE_CONS_THREADS) {
-            if (tid == KIE_CONS_THREADS) produce(P, S, ring_it, smem, cmd);
+            if (tid == KIE_CONS_THREADS) {
+                if constexpr (TM) produce_tmem(P, S, ring_it, tm_it, smem, cmd);
+                else produce_ring(P, S, ring_it, smem, cmd);
+            }
         } else {
-            consume<DT, F8>(P, S, ring_it, smem, cmd, epoch, rd_epoch, att_use);
+            consume<DT, F8, TM>(P, S, ring_it, tm_it, smem, cmd, epoch, rd_epoch, att_use);
         }
         __syncthreads();
         if (resident && blockIdx.x == 0 && tid == 0) {
@@ -969,6 +1320,12 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
             st_release_sys_u32(&P.mbox->done_seq, cmd.seq);
         }
         if (!resident || S.abort) break;
+    }
+    if constexpr (TM) {  // every move has completed and every consumer read has returned
+        tm_fence_before();
+        __syncthreads();
+        tm_fence_after();
+        if (tid < 32) tm_dealloc(S.tmem_base);
     }
 }
 
@@ -984,18 +1341,27 @@ size_t kie_b1_smem_bytes() { return RING_BYTES + sizeof(B1Shared); }
 int kie_b1_chunk_rows(int K) { return (KIE_CONS_WARPS / col_slices(K)) * rows_per_group(K); }
 int kie_b1_max_rows(int K) { return WPART_FLOATS / col_slices(K); }
 
-// the kernel instantiation for a storage dtype and weight format
-static const void *b1_fn(int dtype, bool f8) {
-    if (dtype == KIE_BF16) return f8 ? (const void *)kie_b1_kernel<KIE_BF16, true> : (const void *)kie_b1_kernel<KIE_BF16, false>;
-    return f8 ? (const void *)kie_b1_kernel<KIE_FP16, true> : (const void *)kie_b1_kernel<KIE_FP16, false>;
+// TMEM staging needs the layouts its copies assume: 16-bit weights, d_model 2048 or 4096
+bool kie_b1_tmem_ok(int d, bool f8) { return !f8 && (d == 2048 || d == 4096); }
+
+// the kernel instantiation for a storage dtype, weight format and staging
+static const void *b1_fn(int dtype, bool f8, bool tm) {
+    if (dtype == KIE_BF16) {
+        if (f8) return (const void *)kie_b1_kernel<KIE_BF16, true, false>;
+        return tm ? (const void *)kie_b1_kernel<KIE_BF16, false, true> : (const void *)kie_b1_kernel<KIE_BF16, false, false>;
+    }
+    if (f8) return (const void *)kie_b1_kernel<KIE_FP16, true, false>;
+    return tm ? (const void *)kie_b1_kernel<KIE_FP16, false, true> : (const void *)kie_b1_kernel<KIE_FP16, false, false>;
 }
 
-cudaError_t kie_b1_prepare(int dtype, bool f8) {
-    return cudaFuncSetAttribute(b1_fn(dtype, f8), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kie_b1_smem_bytes());
+cudaError_t kie_b1_prepare(int dtype, bool f8, bool tm) {
+    return cudaFuncSetAttribute(b1_fn(dtype, f8, tm), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kie_b1_smem_bytes());
 }
 
-cudaError_t kie_b1_occupancy(int dtype, bool f8, int *blocks_per_sm) {
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, b1_fn(dtype, f8), KIE_THREADS, kie_b1_smem_bytes());
+cudaError_t kie_b1_occupancy(int dtype, bool f8, bool tm, int *blocks_per_sm) {
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, b1_fn(dtype, f8, tm), KIE_THREADS,
+                                                         kie_b1_smem_bytes());
 }
 
 cudaError_t kie_b1_launch(const KieParams &P, const KieCmd &one, int resident, cudaStream_t stream) {
@@ -1006,7 +1372,7 @@ cudaError_t kie_b1_launch(const KieParams &P, const KieCmd &one, int resident, c
     KieCmd c = one;
     int r = resident;
     void *args[] = {&p, &c, &r};
-    return cudaLaunchCooperativeKernel(b1_fn(P.dtype, P.wesz == 1), dim3(P.nblk), dim3(KIE_THREADS), args,
+    return cudaLaunchCooperativeKernel(b1_fn(P.dtype, P.wesz == 1, P.b1_tmem != 0), dim3(P.nblk), dim3(KIE_THREADS), args,
                                        kie_b1_smem_bytes(), stream);
 }
 

@@ -26,8 +26,9 @@
 size_t kie_b1_smem_bytes();
 int kie_b1_chunk_rows(int K);
 int kie_b1_max_rows(int K);
-cudaError_t kie_b1_prepare(int dtype, bool f8);
-cudaError_t kie_b1_occupancy(int dtype, bool f8, int *blocks_per_sm);
+bool kie_b1_tmem_ok(int d, bool f8);
+cudaError_t kie_b1_prepare(int dtype, bool f8, bool tm);
+cudaError_t kie_b1_occupancy(int dtype, bool f8, bool tm, int *blocks_per_sm);
 cudaError_t kie_b1_launch(const KieParams &P, const KieCmd &one, int resident, cudaStream_t stream);
 size_t kie_mr_smem_bytes();
 cudaError_t kie_mr_prepare(int dtype);
@@ -203,6 +204,7 @@ static const char *shape_error(const kie_config &c) {
     if (!(c.modes & (KIE_MODE_BATCH1 | KIE_MODE_TICK))) return "modes must enable at least one kernel";
     if (c.weight_fp8 != 0 && (c.weight_fp8 != 1 || c.modes != KIE_MODE_BATCH1))
         return "weight_fp8 must be 0 or 1, and 1 needs modes == KIE_MODE_BATCH1";
+    if (c.b1_staging != 0 && c.b1_staging != 1) return "b1_staging must be 0 or 1";
     return nullptr;
 }
 
@@ -251,11 +253,13 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
         eng->fail(KIE_ERR_CUDA, "device lacks cooperative launch");
         return bail(KIE_ERR_CUDA);
     }
+    // batch-1 weights staged on into TMEM where the kernel's chunk layouts allow it
+    const bool b1_tm = c.b1_staging == 1 && kie_b1_tmem_ok(c.d_model, c.weight_fp8 != 0);
     if (b1) {
-        e = kie_b1_prepare(c.dtype, c.weight_fp8 != 0);
+        e = kie_b1_prepare(c.dtype, c.weight_fp8 != 0, b1_tm);
         if (e != cudaSuccess) return bail(eng->cuda_fail(e, "kernel attributes"));
         int occ = 0;
-        e = kie_b1_occupancy(c.dtype, c.weight_fp8 != 0, &occ);
+        e = kie_b1_occupancy(c.dtype, c.weight_fp8 != 0, b1_tm, &occ);
         if (e != cudaSuccess || occ < 1)
             return bail(eng->cuda_fail(e == cudaSuccess ? cudaErrorInvalidConfiguration : e,
                                        "batch-1 megakernel does not fit on an SM"));
@@ -299,9 +303,12 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
     const bool f8 = c.weight_fp8 != 0;
     const int esz = f8 ? 1 : 2;
     P.wesz = esz;
+    P.b1_tmem = b1_tm ? 1 : 0;
     const int Kph[KIE_NPH] = {d, 8, d, 8, d};
     std::vector<int> row0((size_t)KIE_NPH * (nblk + 1));
-    partition(&row0[PH_QKV * (nblk + 1)], (qd + 2 * kvd) / 2, 2, nblk);  // rotation pairs
+    // two rotation pairs at a time: a CTA's pairs then come as (dims i, i + 1), i even, of one
+    // head, which its epilogue writes as single 32- or 64-bit words
+    partition(&row0[PH_QKV * (nblk + 1)], (qd + 2 * kvd) / 4, 4, nblk);
     // O fold: CTA c = g * splits + s holds 8-column groups [s (E/8) / splits, (s+1) (E/8) / splits)
     // of kv head g's outputs, i.e. global groups g (E/8) + that; the CTAs past Hkv * splits none
     for (int cc = 0; cc <= nblk; cc++) {

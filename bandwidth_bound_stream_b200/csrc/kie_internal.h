@@ -10,6 +10,7 @@
 #define KIE_THREADS (KIE_CONS_THREADS + 32)   // + one producer warp
 #define KIE_NSLOT 3                           // weight ring depth
 #define KIE_SLOT_BYTES 65536                  // one ring slot (large bulk copies stream best)
+#define KIE_NTS 4                             // TMEM weight slots (128 columns = one 64 KB chunk each)
 #define KIE_ROWACC_MAX 1024                   // output rows one CTA may own in one phase
 #define KIE_GMAX 8                            // query heads per kv head
 #define KIE_DMAX 128                          // head_dim
@@ -76,6 +77,7 @@ struct KieParams {
     // batch-1 packed weights: CTA c streams [seg_off[c], seg_off[c+1]) once per token
     const uint8_t *wpack;
     int wesz;                       // bytes per streamed weight: 2 (dtype), or 1 (E4M3 codes)
+    int b1_tmem;                    // 1: ring chunks are moved on into TMEM and read from there
     const float *wsc;               // E4M3 row scales: per layer [QKV rows | d | gate/up rows | d], then [V]
     int sc_stride;                  // floats per layer in wsc
     const int *row0;                // [KIE_NPH][nblk+1] partition: rows (GEMV phases), 8-column groups (folds)

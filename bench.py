@@ -218,6 +218,8 @@ def main():
     ap.add_argument("--ticks", type=int, default=500, help="timed ticks of the 56-session workload (0 = skip)")
     ap.add_argument("--tick-only", action="store_true", help="only the tick workload (its own JSON line)")
     ap.add_argument("--no-extra", action="store_true", help="skip the 8B and 32K-context batch-1 workloads")
+    ap.add_argument("--b1-staging", type=int, default=0, choices=[0, 1],
+                    help="batch-1 weight staging: 0 = shared-memory ring, 1 = ring plus TMEM slots for the attention step")
     ap.add_argument("--extra-steps", type=int, default=3, help="timed launches of each extra workload")
     ap.add_argument("--tick-model", default="dense-10.8b")
     ap.add_argument("--tick-prompt", type=int, default=0, help="fixed prompt length per session (0 = seeded 1000-1500)")
@@ -259,7 +261,7 @@ def main():
     prompt = synth.prompt(m, prompt_len)
     # both kernels: the prompt is prefilled in chunks of 64 positions on the tensor cores
     eng = kie.Engine(kie.config(m, max_ctx=prompt_len + decode_n, timeout_ms=10000, idle_ms=200, device=local,
-                                modes=kie.KIE_MODE_BATCH1 | kie.KIE_MODE_TICK), dw.kie)
+                                modes=kie.KIE_MODE_BATCH1 | kie.KIE_MODE_TICK, b1_staging=args.b1_staging), dw.kie)
     host_weights = dw.host
     dw.free()  # the engine keeps its own repacked copy
     torch.cuda.empty_cache()
@@ -390,7 +392,8 @@ def main():
     if args.ticks > 0 and headline:
         line["tick"] = run_tick(args.ticks, args.warmup, local, clocks_for=local)
     if headline and not args.no_extra and world == 1:
-        line["configs"] = {f"{n}{'-fp8' if f8 else ''}@{p}+{d}": run_extra(n, p, d, f8, args.extra_steps, 3, local, peak)
+        line["configs"] = {f"{n}{'-fp8' if f8 else ''}@{p}+{d}": run_extra(n, p, d, f8, args.extra_steps, 3, local, peak,
+                                                                             args.b1_staging)
                            for n, p, d, f8 in EXTRA_CONFIGS}
     if want_cpu:
         line["cpu_baseline"] = oracle_baseline(m, host_weights, prompt_len + decode_n // 2)
@@ -407,7 +410,7 @@ EXTRA_CONFIGS = (("dense-8b", 4096, 256, False), ("dense-1.9b", 32768, 256, Fals
 
 
 def run_extra(name: str, prompt_len: int, decode_n: int, fp8: bool, steps: int, warmup: int, local: int,
-              peak: float) -> dict:
+              peak: float, staging: int = 0) -> dict:
     """tokens/s and the roofline of one more batch-1 workload (steps launches of decode_n tokens);
     fp8: the engine streams E4M3 weights with row scales (the prompt then goes through the
     batch-1 kernel as well)."""
@@ -420,7 +423,7 @@ def run_extra(name: str, prompt_len: int, decode_n: int, fp8: bool, steps: int, 
     dw = kie.DeviceWeights(m, seed=0, device=dev)
     modes = kie.KIE_MODE_BATCH1 if fp8 else kie.KIE_MODE_BATCH1 | kie.KIE_MODE_TICK
     eng = kie.Engine(kie.config(m, max_ctx=prompt_len + decode_n, timeout_ms=20000, idle_ms=200, device=local,
-                                modes=modes, weight_fp8=fp8), dw.kie)
+                                modes=modes, weight_fp8=fp8, b1_staging=staging), dw.kie)
     dw.free()
     torch.cuda.empty_cache()
     setup_s = time.perf_counter() - t0

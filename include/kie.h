@@ -76,6 +76,15 @@ typedef struct {
                              kernel's tensor-core contractions take 16-bit operands), and
                              prompts then go through the batch-1 kernel too. 0: weights
                              stream in `dtype`.                                           */
+    int32_t b1_staging;   /* where the batch-1 kernel stages streamed weights:
+                             0 (default): the 3-slot shared-memory ring (64 KB slots).
+                             1: the ring, plus 4 slots of tensor memory (TMEM) per SM for
+                             the first 4 chunks after each layer's QKV rows, so the stream
+                             runs 7 chunks ahead through the attention step; 16-bit weights
+                             and d_model 2048 or 4096 only (else as 0). Same results; on
+                             one B200 about as fast as 0 on the 8B shape and 4 % slower on
+                             the 1.9B shape, since streaming through the attention step
+                             and the grid barriers lengthens their L2 round trips.        */
 } kie_config;
 
 /*

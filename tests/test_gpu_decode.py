@@ -130,14 +130,18 @@ def test_tiny_generate_and_launch_match_oracle_chain(kie):
         assert np.array_equal(out_d.cpu().numpy(), gen)
 
 
-@pytest.mark.parametrize("name,prompt_len,steps", [("slice-1.9b", 40, 8), ("slice-8b", 24, 6), ("ragged", 33, 10)])
-def test_sliced_shapes_parity(kie, name, prompt_len, steps):
+@pytest.mark.parametrize("name,prompt_len,steps,staging", [
+    ("slice-1.9b", 40, 8, 0), ("slice-8b", 24, 6, 0), ("ragged", 33, 10, 0),
+    ("slice-1.9b", 150, 8, 1), ("slice-8b", 90, 6, 1),
+])
+def test_sliced_shapes_parity(kie, name, prompt_len, steps, staging):
     """Two-layer slices of the 1.9B (fp16, GQA 2) and 8B (bf16, GQA 4) shapes at full width, and a ragged
-    shape (odd vocab, GQA 3, rows not divisible by the SM count)."""
+    shape (odd vocab, GQA 3, rows not divisible by the SM count). staging 1: the slices again with
+    the weight chunks of the attention step staged in TMEM (d_model 2048 and 4096 take it)."""
     from bandwidth_bound_stream_b200 import synth
     from tests.parity import assert_reports
     m = synth.CONFIGS[name]
-    dw, eng, orc = _setup(kie, m, prompt_len + steps + 4)
+    dw, eng, orc = _setup(kie, m, prompt_len + steps + 4, b1_staging=staging)
     with eng:
         reps = _lockstep(kie, eng, orc, m, synth.prompt(m, prompt_len), steps)
     assert_reports(reps, m.dtype)
