@@ -169,7 +169,10 @@ __device__ __forceinline__ int sc_off_down(const KieParams &P) { return sc_off_g
 struct __align__(16) B1Shared {
     union {
         float wpart[WPART_FLOATS];  // column-slice partials of this phase's row sums
-        AttnSmem at;
+        struct {
+            AttnSmem at;
+            uint4 kvcur[2][KIE_DMAX / 8];       // K and V rows of the current position (last split)
+        };
         struct {
             float vals[KIE_SAMPLE_VALS];  // the values a top-k selection reads
             SampleScratch ss;
@@ -185,6 +188,7 @@ struct __align__(16) B1Shared {
     uint64_t tempty[KIE_NTS];  // every consumer warp has read slot t
     uint32_t tmem_base;
     uint32_t pub_sink;         // scratch word of pub_wait
+    volatile uint32_t att_done;  // QKV -> attention barriers this CTA has passed in this launch
     KieCmd cmd;
     volatile int abort;
     int token;
@@ -294,11 +298,38 @@ __device__ void residual_read_wait(const KieParams &P, B1Shared &S, unsigned lon
 // Walks this CTA's chunks in stream order: per token, every layer's QKV rows, O-fold column
 // groups, gate/up rows and down-fold column groups, then (when the token needs logits) the
 // LM-head rows. A token restarts at the segment base.
+// K/V chunks (the attention unit's cache rows, when they stream through the ring) sit between
+// a layer's QKV rows and its O-fold columns: positions [p0, p0 + n) of the unit's split other
+// than the current one (final since earlier steps), KV_CHUNK_POS at a time, K rows at slot
+// offset 0 and V rows at KIE_SLOT_BYTES / 2.
+constexpr int PH_KV = KIE_NPH;
+__host__ __device__ inline int kv_chunk_pos(int D) { return KIE_SLOT_BYTES / 4 / D; }
+// query heads of a kv head the attention takes in one pass over the span (their queries and
+// running sums are held in registers: the register budget of the 16 consumer warps allows two);
+// more heads take more passes, each with the span streamed again
+constexpr int ATT_GC = 2;
+__host__ __device__ inline int kv_passes(const KieParams &P) { return (P.G + ATT_GC - 1) / ATT_GC; }
+
+// The cache positions of this CTA's attention unit at context ctx that the ring carries:
+// [p0, p0 + n), all of the split but the current position ctx - 1. false: no unit.
+__device__ __forceinline__ bool kv_ring_span(const KieParams &P, int ctx, int &g, int &p0, int &n) {
+    const int unit = blockIdx.x;
+    if (unit >= P.Hkv * P.splits) return false;
+    g = unit / P.splits;
+    const int s = unit % P.splits;
+    p0 = (int)((long long)s * ctx / P.splits);
+    const int p1 = (int)((long long)(s + 1) * ctx / P.splits);
+    n = max(0, min(p1, ctx - 1) - p0);
+    return true;
+}
+
 struct ChunkIter {
     const uint8_t *seg, *g;
     int t, l, ph, r;
     int qn;  // chunks of this layer's O fold, gate/up and down fold returned so far
-    int cq;  // the returned chunk's index among them (-1: a QKV or LM-head chunk)
+    int cq;  // the returned chunk's index among them (-1: a QKV, K/V or LM-head chunk)
+    int kv_g, kv_p0, kv_n;  // K/V span of the current layer (PH_KV)
+    int kv_pass;            // pass over the span (one per ATT_GC query heads)
 };
 
 __device__ __forceinline__ void chunk_begin(ChunkIter &it, const uint8_t *seg) {
@@ -315,11 +346,30 @@ __device__ __forceinline__ void chunk_begin(ChunkIter &it, const uint8_t *seg) {
 __device__ __forceinline__ bool is_fold(int ph) { return ph == PH_OF || ph == PH_DF; }
 
 // Next chunk (address, bytes); false when the command's schedule is exhausted. A GEMV chunk
-// is cr rows of K elements; a fold chunk is cr column groups of d rows x 16 bytes.
+// is cr rows of K elements; a fold chunk is cr column groups of d rows x 16 bytes; a K/V
+// chunk is K rows at addr and as many V rows at addr2 (bytes covers both).
+template <bool KVR>
 __device__ bool chunk_next(const KieParams &P, const B1Shared &S, const KieCmd &cmd, ChunkIter &it,
-                           const uint8_t *&addr, uint32_t &bytes) {
+                           const uint8_t *&addr, uint32_t &bytes, const uint8_t **addr2 = nullptr) {
     for (;;) {
         if (it.t >= cmd.n) return false;
+        if (it.ph == PH_KV) {
+            if (it.r < it.kv_n) {
+                const int nr = min(kv_chunk_pos(P.D), it.kv_n - it.r);
+                const size_t off = (size_t)cmd.sid * P.sess_stride +
+                                   ((size_t)(it.l * P.Hkv + it.kv_g) * P.max_ctx + it.kv_p0 + it.r) * P.D;
+                addr = reinterpret_cast<const uint8_t *>(P.kcache + off);
+                if (addr2) *addr2 = reinterpret_cast<const uint8_t *>(P.vcache + off);
+                bytes = (uint32_t)(2 * nr * P.D * 2);
+                it.r += nr;
+                it.cq = -1;
+                return true;
+            }
+            it.r = 0;
+            if (it.kv_n > 0 && ++it.kv_pass < kv_passes(P)) continue;  // the span again for the next query heads
+            it.ph = PH_OF;
+            continue;
+        }
         const int n = S.row1[it.ph] - S.row0[it.ph];
         if (it.r < n) {
             const int nr = min(P.cr[it.ph], n - it.r);
@@ -352,6 +402,10 @@ __device__ bool chunk_next(const KieParams &P, const B1Shared &S, const KieCmd &
             } else {
                 it.ph = 0;
             }
+        } else if (KVR && it.ph == PH_QKV) {
+            it.ph = PH_KV;
+            it.kv_pass = 0;
+            if (!kv_ring_span(P, cmd.pos0 + it.t + 1, it.kv_g, it.kv_p0, it.kv_n)) it.kv_n = 0;
         } else {
             it.ph++;
         }
@@ -394,6 +448,31 @@ __device__ __forceinline__ void tmem_read_chunk(B1Shared &S, uint32_t ts, uint32
 
 // --------------------------------------------------------------- producer
 
+// A K/V chunk of step t (t > 0 in the command), layer l, carries position pos - 1, which the
+// previous step's QKV epilogues wrote in layer l: it may be copied once this CTA's consumers
+// have passed that step's QKV -> attention barrier, the ((t - 1) L + l + 1)-th of the command
+// (att0: barriers passed before the command). Earlier positions, and every position of step 0,
+// were complete before. (With few chunks per step, as in small models, the stream can run
+// that far ahead.)
+__device__ __forceinline__ bool kv_chunk_ready(const KieParams &P, const B1Shared &S, const ChunkIter &it,
+                                               uint32_t att0) {
+    return it.t == 0 || (int)(S.att_done - (att0 + (uint32_t)((it.t - 1) * P.L + it.l + 1))) >= 0;
+}
+
+// Issues the bulk copies of one chunk into ring slot `slot`: a weight chunk in one piece, a K/V
+// chunk as its K rows at the slot's start and its V rows at the slot's middle.
+__device__ __forceinline__ void issue_chunk(B1Shared &S, uint8_t *ring, uint32_t slot, int ph, const uint8_t *a,
+                                            const uint8_t *a2, uint32_t b) {
+    uint8_t *dst = ring + (size_t)slot * KIE_SLOT_BYTES;
+    mbar_arrive_expect_tx(&S.full[slot], b);
+    if (ph == PH_KV) {
+        bulk_g2s(dst, a, b / 2, &S.full[slot]);
+        bulk_g2s(dst + KIE_SLOT_BYTES / 2, a2, b / 2, &S.full[slot]);
+    } else {
+        bulk_g2s(dst, a, b, &S.full[slot]);
+    }
+}
+
 // Writes the producer's wait for this token into its trace slot.
 __device__ __forceinline__ void trace_producer_wait(const KieParams &P, int tok, unsigned long long waited) {
     if (P.trace && tok < P.trace_tokens)
@@ -401,15 +480,17 @@ __device__ __forceinline__ void trace_producer_wait(const KieParams &P, int tok,
 }
 
 // Shared-memory ring only: chunk i goes to slot i % 3, and the consumers read it there.
+template <bool KVR>
 __device__ void produce_ring(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint8_t *ring, const KieCmd &cmd) {
+    const uint32_t att0 = S.att_done;
     const uint8_t *seg = P.wpack + P.seg_off[blockIdx.x];
     ChunkIter fetch;
     chunk_begin(fetch, seg);
-    const uint8_t *a;
+    const uint8_t *a, *a2 = nullptr;
     uint32_t b;
     unsigned long long waited = 0;
     int tok = 0;
-    while (chunk_next(P, S, cmd, fetch, a, b)) {
+    while (chunk_next<KVR>(P, S, cmd, fetch, a, b, &a2)) {
         if (fetch.t != tok) {
             trace_producer_wait(P, tok, waited);
             waited = 0;
@@ -426,9 +507,19 @@ __device__ void produce_ring(const KieParams &P, B1Shared &S, uint32_t &ring_it,
                 break;
             }
         }
+        if (fetch.ph == PH_KV && !kv_chunk_ready(P, S, fetch, att0)) {
+            const uint64_t w0 = globaltimer();
+            while (!kv_chunk_ready(P, S, fetch, att0) && !S.abort) {
+                if ((long long)(globaltimer() - w0) > P.timeout_ns) {
+                    set_error(P.err, DERR_RING_TIMEOUT, 0x82);
+                    S.abort = 1;
+                }
+                __nanosleep(64);
+            }
+            waited += globaltimer() - w0;
+        }
         if (S.abort) break;
-        mbar_arrive_expect_tx(&S.full[slot], b);
-        bulk_g2s(ring + (size_t)slot * KIE_SLOT_BYTES, a, b, &S.full[slot]);
+        issue_chunk(S, ring, slot, fetch.ph, a, a2, b);
         ring_it++;
     }
     trace_producer_wait(P, tok, waited);
@@ -449,14 +540,16 @@ __device__ void produce_ring(const KieParams &P, B1Shared &S, uint32_t &ring_it,
 // consumers to be done with the TMEM slot's previous chunk, while the bulk copies run ahead.
 __device__ __forceinline__ bool via_tmem(int cq) { return cq >= 0 && cq < KIE_NTS; }
 
+template <bool KVR>
 __device__ void produce_tmem(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint32_t &tm_it, uint8_t *ring,
                              const KieCmd &cmd) {
+    const uint32_t att0 = S.att_done;
     const uint8_t *seg = P.wpack + P.seg_off[blockIdx.x];
     ChunkIter fetch;
     chunk_begin(fetch, seg);
-    const uint8_t *a = nullptr;
+    const uint8_t *a = nullptr, *a2 = nullptr;
     uint32_t b = 0;
-    bool more = chunk_next(P, S, cmd, fetch, a, b);
+    bool more = chunk_next<KVR>(P, S, cmd, fetch, a, b, &a2);
     // moves waiting for their chunk to land or their TMEM slot: (chunk, phase), at most one per ring slot
     uint32_t mv_chunk[KIE_NSLOT];
     int mv_ph[KIE_NSLOT];
@@ -468,7 +561,7 @@ __device__ void produce_tmem(const KieParams &P, B1Shared &S, uint32_t &ring_it,
     const uint32_t tbase = S.tmem_base;
     while (more || mv_n > 0) {
         bool progress = false;
-        if (more) {
+        if (more && (fetch.ph != PH_KV || kv_chunk_ready(P, S, fetch, att0))) {
             const uint32_t slot = ring_it % KIE_NSLOT, par = (ring_it / KIE_NSLOT) & 1u;
             if (mbar_test_wait(&S.empty[slot], par ^ 1u)) {
                 if (fetch.t != tok) {
@@ -476,8 +569,7 @@ __device__ void produce_tmem(const KieParams &P, B1Shared &S, uint32_t &ring_it,
                     waited = 0;
                     tok = fetch.t;
                 }
-                mbar_arrive_expect_tx(&S.full[slot], b);
-                bulk_g2s(ring + (size_t)slot * KIE_SLOT_BYTES, a, b, &S.full[slot]);
+                issue_chunk(S, ring, slot, fetch.ph, a, a2, b);
                 if (via_tmem(fetch.cq)) {
                     const int q = (mv_head + mv_n) % KIE_NSLOT;
                     mv_chunk[q] = ring_it;
@@ -485,7 +577,7 @@ __device__ void produce_tmem(const KieParams &P, B1Shared &S, uint32_t &ring_it,
                     mv_n++;
                 }
                 ring_it++;
-                more = chunk_next(P, S, cmd, fetch, a, b);
+                more = chunk_next<KVR>(P, S, cmd, fetch, a, b, &a2);
                 progress = true;
             }
         }
@@ -533,6 +625,8 @@ __device__ void produce_tmem(const KieParams &P, B1Shared &S, uint32_t &ring_it,
                 mbar_try_wait_ns(&S.full[c % KIE_NSLOT], (c / KIE_NSLOT) & 1u, 256);
             else
                 mbar_try_wait_ns(&S.tempty[tm_it % KIE_NTS], ((tm_it / KIE_NTS) & 1u) ^ 1u, 256);
+        } else if (more && fetch.ph == PH_KV) {
+            __nanosleep(64);
         } else if (more) {
             mbar_try_wait_ns(&S.empty[ring_it % KIE_NSLOT], ((ring_it / KIE_NSLOT) & 1u) ^ 1u, 256);
         }
@@ -859,7 +953,7 @@ __device__ __forceinline__ void attention_prefetch(const KieParams &P, B1Shared 
 // takes pair p (npair <= 512); the CTA's pairs come two at a time as dims (i, i + 1), i even, of
 // one head, so the even thread of each two writes both dims as one word (q: two fp32 values,
 // k and v: two 16-bit values), published by completion for the attention step.
-template <int DT>
+template <int DT, bool KVR>
 __device__ void epilogue_qkv(const KieParams &P, B1Shared &S, int l, int sid, int pos, int tok, float2 rsc) {
     const int D = P.D, half = D >> 1, qd = P.Hq * D, kvd = P.Hkv * D;
     const int rbeg = S.row0[PH_QKV], npair = (S.row1[PH_QKV] - rbeg) >> 1;
@@ -900,7 +994,7 @@ __device__ void epilogue_qkv(const KieParams &P, B1Shared &S, int l, int sid, in
     if (l == 0) {  // the residual starts as the embedding row (each CTA writes a 1/nblk share)
         const int r0 = (int)((long long)blockIdx.x * P.d / P.nblk), r1 = (int)((long long)(blockIdx.x + 1) * P.d / P.nblk);
         for (int rr = r0 + threadIdx.x; rr < r1; rr += KIE_CONS_THREADS) pub_f32(P.x + rr, cvt1<DT>(P.emb[(size_t)tok * P.d + rr]), tk);
-        attention_prefetch(P, S, l, sid, pos);
+        if (!KVR) attention_prefetch(P, S, l, sid, pos);
     }
     pub_wait(tk, &S.pub_sink);
 }
@@ -927,8 +1021,9 @@ __device__ __forceinline__ void attention_prefetch(const KieParams &P, B1Shared 
 }
 
 // u = silu(gate) * up for this CTA's pairs, into the down fold's inputs
+template <bool KVR>
 __device__ void epilogue_gu(const KieParams &P, B1Shared &S, int l, int sid, int pos, float2 rsc) {
-    if (l + 1 < P.L) attention_prefetch(P, S, l + 1, sid, pos);
+    if (!KVR && l + 1 < P.L) attention_prefetch(P, S, l + 1, sid, pos);
     const int npair = (S.row1[PH_GU] - S.row0[PH_GU]) >> 1;
     const int cs = col_slices(P.K[PH_GU]);
     for (int p = threadIdx.x; p < npair; p += KIE_CONS_THREADS) {
@@ -1057,9 +1152,90 @@ __device__ __noinline__ int sample_global(B1Shared &S, int nblk, const float *ca
 // The QKV -> attention barrier, then this CTA's attention unit (at most one unit per CTA:
 // splits = nblk / Hkv); the query heads of a kv head are taken GC at a time. Each split merges
 // its slice of the kv head's output into S.fold_in (the O fold's inputs).
+// This CTA's attention unit (kv head g, split s) for query heads [hoff, hoff + GC) of the kv
+// head: its cache rows arrive through the weight ring (positions [p0, p0 + n) of the split, in
+// chunks of kv_chunk_pos(D) positions, one pass of the span per GC query heads), and in the
+// last split the current position's row, written this step by the QKV epilogues and published
+// before the barrier, is read from the cache at the start and taken last by position group 0.
+// Then the split merge (attn_tail). Position groups of D/8 lanes, scores in log2 units, as in
+// attn_unit.
 template <int DT, int GC>
+__device__ void attn_unit_ring(const KieParams &P, B1Shared &S, const AttnArgs &A, uint32_t &ring_it,
+                               const uint8_t *ring, int ctx, int hoff) {
+    constexpr int NW = KIE_CONS_WARPS;
+    constexpr int B = 1;  // positions per group per batch (registers)
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int D = P.D, lpp = D >> 3, ppw = 32 / lpp, sub = lane / lpp, sl = lane % lpp;
+    const int ngroups = NW * ppw, gi = w * ppw + sub;
+    const int Gt = P.G, nh = min(GC, Gt - hoff);
+    const float qscale = rsqrtf((float)D) * 1.4426950408889634f;
+    int g, p0, n;
+    kv_ring_span(P, ctx, g, p0, n);  // the caller checked that this CTA has a unit
+    const bool last = (int)blockIdx.x % P.splits == P.splits - 1;
+    float q[GC][8];
+#pragma unroll
+    for (int jj = 0; jj < GC; jj++) {
+        const float *qp = P.q + (size_t)(g * Gt + hoff + min(jj, nh - 1)) * D + sl * 8;
+        const float4 a = __ldcg(reinterpret_cast<const float4 *>(qp));
+        const float4 b = __ldcg(reinterpret_cast<const float4 *>(qp + 4));
+        q[jj][0] = a.x * qscale; q[jj][1] = a.y * qscale; q[jj][2] = a.z * qscale; q[jj][3] = a.w * qscale;
+        q[jj][4] = b.x * qscale; q[jj][5] = b.y * qscale; q[jj][6] = b.z * qscale; q[jj][7] = b.w * qscale;
+    }
+    // the current position's K and V rows (last split), staged for position group 0
+    if (last && tid < 2 * (D / 8)) {
+        const int kvsel = tid / (D / 8), c = tid % (D / 8);
+        const size_t o = (size_t)g * A.head_stride + (size_t)(ctx - 1) * D + c * 8;
+        S.kvcur[kvsel][c] = __ldcg(reinterpret_cast<const uint4 *>((kvsel ? A.v : A.k) + o));
+    }
+    named_bar_sync(1, KIE_CONS_THREADS);
+    float m[GC], lsum[GC], acc[GC][8];
+#pragma unroll
+    for (int jj = 0; jj < GC; jj++) {
+        m[jj] = -CUDART_INF_F;
+        lsum[jj] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; e++) acc[jj][e] = 0.f;
+    }
+    const int PB = kv_chunk_pos(D);
+    for (int c0 = 0; c0 < n; c0 += PB) {
+        const int np = min(PB, n - c0);
+        const uint32_t slot = ring_it % KIE_NSLOT, par = (ring_it / KIE_NSLOT) & 1u;
+        ring_it++;
+        bool have = ring_take(P, S, slot, par, PH_OF);  // traced with the O fold's waits
+        have = __all_sync(0xffffffffu, have);
+        if (!have) {
+            if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, (unsigned)PH_KV);
+            S.abort = 1;
+            continue;
+        }
+        const uint8_t *kb = ring + (size_t)slot * KIE_SLOT_BYTES, *vb = kb + KIE_SLOT_BYTES / 2;
+        for (int base = 0; base < np; base += ngroups * B) {  // uniform across the CTA
+            uint4 kv[B], vv[B];
+#pragma unroll
+            for (int b = 0; b < B; b++) {
+                const int j = base + gi + b * ngroups;
+                const bool ok = j < np;
+                const size_t o = ((size_t)j * D + sl * 8) * 2;
+                kv[b] = ok ? *reinterpret_cast<const uint4 *>(kb + o) : make_uint4(0, 0, 0, 0);
+                vv[b] = ok ? *reinterpret_cast<const uint4 *>(vb + o) : make_uint4(0, 0, 0, 0);
+            }
+            attn_update<DT, GC, B>(kv, vv, base, np, gi, ngroups, lpp, q, m, lsum, acc);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.empty[slot]);
+    }
+    if (last) {
+        uint4 kv[1], vv[1];
+        kv[0] = gi == 0 ? S.kvcur[0][sl] : make_uint4(0, 0, 0, 0);
+        vv[0] = gi == 0 ? S.kvcur[1][sl] : make_uint4(0, 0, 0, 0);
+        attn_update<DT, GC, 1>(kv, vv, 0, 1, gi, ngroups, lpp, q, m, lsum, acc);
+    }
+    attn_tail<DT, GC, NW, false>(A, S.at, (int)blockIdx.x, Gt, hoff, m, lsum, acc);
+}
+
+template <int DT, int GC, bool KVR>
 __device__ void attention_step(const KieParams &P, B1Shared &S, int l, int sid, int pos, unsigned long long &epoch,
-                               int t, int e, uint32_t &att_use) {
+                               int t, int e, uint32_t &att_use, uint32_t &ring_it, const uint8_t *ring) {
     AttnArgs A;
     A.q = P.q;
     A.k = P.kcache + (size_t)sid * P.sess_stride + (size_t)l * P.Hkv * P.max_ctx * P.D;
@@ -1085,13 +1261,17 @@ __device__ void attention_step(const KieParams &P, B1Shared &S, int l, int sid, 
     const int unit = blockIdx.x;
     const bool have = unit < P.Hkv * P.splits;
     grid_barrier(P, S, epoch, P.timeout_ns, 1);
+    if (threadIdx.x == 0) S.att_done = S.att_done + 1u;  // this step's K/V rows are complete (see kv_chunk_ready)
     trace_mark(P, t, e + 2);
     if (P.wesz == 1)  // the O fold's row scales (E4M3 weights) wait in L1 through attention
         for (int r = threadIdx.x; r < P.d; r += KIE_CONS_THREADS)
             prefetch_l1(P.wsc + (size_t)l * P.sc_stride + sc_off_o(P) + r);
     if (threadIdx.x == 0) S.at.t_unit = 0;
     if (have && !S.abort) {
-        for (int hoff = 0; hoff < P.G; hoff += GC) attn_unit<DT, GC, KIE_CONS_WARPS>(A, S.at, unit, P.G, hoff);
+        for (int hoff = 0; hoff < P.G; hoff += GC) {
+            if constexpr (KVR) attn_unit_ring<DT, GC>(P, S, A, ring_it, ring, pos + 1, hoff);
+            else attn_unit<DT, GC, KIE_CONS_WARPS>(A, S.at, unit, P.G, hoff);  // K/V from L2 (read ahead)
+        }
     }
 }
 
@@ -1148,7 +1328,7 @@ __device__ __forceinline__ void down_fold_any(const KieParams &P, B1Shared &S, u
 
 // --------------------------------------------------------------- consumer: one command
 
-template <int DT, bool F8, bool TM>
+template <int DT, bool F8, bool TM, bool KVR>
 __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint32_t &tm_it, const uint8_t *ring,
                         const KieCmd &cmd, unsigned long long &epoch, unsigned long long &rd_epoch, uint32_t &att_use) {
     int tok = cmd.in_tok;
@@ -1178,10 +1358,10 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint
             const float2 sq = gemv_dispatch<DT, F8, TM>(P, S, ring_it, tm_it, lq, ring, PH_QKV, l, tok, pos, t);
             lq = 0;  // the chunks of the O fold, gate/up rows and down fold, counted from here
             trace_mark(P, t, e);
-            epilogue_qkv<DT>(P, S, l, cmd.sid, pos, tok, sq);
+            epilogue_qkv<DT, KVR>(P, S, l, cmd.sid, pos, tok, sq);
             trace_mark(P, t, e + 1);
             // B: attention, then the O fold
-            attention_step<DT, 2>(P, S, l, cmd.sid, pos, epoch, t, e, att_use);  // also serves G == 1
+            attention_step<DT, ATT_GC, KVR>(P, S, l, cmd.sid, pos, epoch, t, e, att_use, ring_it, ring);
             if (P.trace && t < P.trace_tokens && threadIdx.x == 0)  // end of this CTA's positions (0: no unit)
                 P.trace[((size_t)blockIdx.x * P.trace_tokens + t) * P.trace_events + e + 15] = S.at.t_unit;
             trace_mark(P, t, e + 3);
@@ -1194,7 +1374,7 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint
             residual_read_arrive(P, S);  // this CTA's reads of x are done
             rd_epoch++;
             trace_mark(P, t, e + 6);
-            epilogue_gu(P, S, l, cmd.sid, pos, sg);
+            epilogue_gu<KVR>(P, S, l, cmd.sid, pos, sg);
             trace_mark(P, t, e + 7);
             down_fold_any<DT, F8, TM>(P, S, ring_it, tm_it, lq, ring, l, rd_epoch, t, e);
             trace_mark(P, t, e + 8);
@@ -1226,12 +1406,12 @@ __device__ void consume(const KieParams &P, B1Shared &S, uint32_t &ring_it, uint
             P.trace[((size_t)blockIdx.x * P.trace_tokens + t) * P.trace_events + P.trace_events - 1 - KIE_NPH +
                     threadIdx.x] = S.wait_ph[threadIdx.x];
     }
-    cp_async_wait_all();  // the L2 reads into warm_sink have landed
+    if (!KVR) cp_async_wait_all();  // the L2 reads into warm_sink have landed
 }
 
 // --------------------------------------------------------------- the kernel
 
-template <int DT, bool F8, bool TM>
+template <int DT, bool F8, bool TM, bool KVR>
 __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, KieCmd one, int resident) {
     extern __shared__ __align__(1024) uint8_t smem[];
     B1Shared &S = *reinterpret_cast<B1Shared *>(smem + RING_BYTES);
@@ -1249,6 +1429,7 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
         }
         fence_mbar_init();
         S.abort = 0;
+        S.att_done = 0;
     }
     if (tid < KIE_NPH) {
         S.row0[tid] = P.row0[tid * (P.nblk + 1) + blockIdx.x];
@@ -1307,11 +1488,11 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
         if (cmd.op != OP_DECODE && cmd.op != OP_PREFILL) break;
         if (tid >= KIE_CONS_THREADS) {
             if (tid == KIE_CONS_THREADS) {
-                if constexpr (TM) produce_tmem(P, S, ring_it, tm_it, smem, cmd);
-                else produce_ring(P, S, ring_it, smem, cmd);
+                if constexpr (TM) produce_tmem<KVR>(P, S, ring_it, tm_it, smem, cmd);
+                else produce_ring<KVR>(P, S, ring_it, smem, cmd);
             }
         } else {
-            consume<DT, F8, TM>(P, S, ring_it, tm_it, smem, cmd, epoch, rd_epoch, att_use);
+            consume<DT, F8, TM, KVR>(P, S, ring_it, tm_it, smem, cmd, epoch, rd_epoch, att_use);
         }
         __syncthreads();
         if (resident && blockIdx.x == 0 && tid == 0) {
@@ -1344,23 +1525,24 @@ int kie_b1_max_rows(int K) { return WPART_FLOATS / col_slices(K); }
 // TMEM staging needs the layouts its copies assume: 16-bit weights, d_model 2048 or 4096
 bool kie_b1_tmem_ok(int d, bool f8) { return !f8 && (d == 2048 || d == 4096); }
 
-// the kernel instantiation for a storage dtype, weight format and staging
-static const void *b1_fn(int dtype, bool f8, bool tm) {
-    if (dtype == KIE_BF16) {
-        if (f8) return (const void *)kie_b1_kernel<KIE_BF16, true, false>;
-        return tm ? (const void *)kie_b1_kernel<KIE_BF16, false, true> : (const void *)kie_b1_kernel<KIE_BF16, false, false>;
-    }
-    if (f8) return (const void *)kie_b1_kernel<KIE_FP16, true, false>;
-    return tm ? (const void *)kie_b1_kernel<KIE_FP16, false, true> : (const void *)kie_b1_kernel<KIE_FP16, false, false>;
+// the kernel instantiation for a storage dtype, weight format, staging and K/V path
+template <int DT>
+static const void *b1_fn_dt(bool f8, bool tm, bool kvr) {
+    if (f8) return kvr ? (const void *)kie_b1_kernel<DT, true, false, true> : (const void *)kie_b1_kernel<DT, true, false, false>;
+    if (tm) return kvr ? (const void *)kie_b1_kernel<DT, false, true, true> : (const void *)kie_b1_kernel<DT, false, true, false>;
+    return kvr ? (const void *)kie_b1_kernel<DT, false, false, true> : (const void *)kie_b1_kernel<DT, false, false, false>;
+}
+static const void *b1_fn(int dtype, bool f8, bool tm, bool kvr) {
+    return dtype == KIE_BF16 ? b1_fn_dt<KIE_BF16>(f8, tm, kvr) : b1_fn_dt<KIE_FP16>(f8, tm, kvr);
 }
 
-cudaError_t kie_b1_prepare(int dtype, bool f8, bool tm) {
-    return cudaFuncSetAttribute(b1_fn(dtype, f8, tm), cudaFuncAttributeMaxDynamicSharedMemorySize,
+cudaError_t kie_b1_prepare(int dtype, bool f8, bool tm, bool kvr) {
+    return cudaFuncSetAttribute(b1_fn(dtype, f8, tm, kvr), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kie_b1_smem_bytes());
 }
 
-cudaError_t kie_b1_occupancy(int dtype, bool f8, bool tm, int *blocks_per_sm) {
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, b1_fn(dtype, f8, tm), KIE_THREADS,
+cudaError_t kie_b1_occupancy(int dtype, bool f8, bool tm, bool kvr, int *blocks_per_sm) {
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, b1_fn(dtype, f8, tm, kvr), KIE_THREADS,
                                                          kie_b1_smem_bytes());
 }
 
@@ -1372,7 +1554,7 @@ cudaError_t kie_b1_launch(const KieParams &P, const KieCmd &one, int resident, c
     KieCmd c = one;
     int r = resident;
     void *args[] = {&p, &c, &r};
-    return cudaLaunchCooperativeKernel(b1_fn(P.dtype, P.wesz == 1, P.b1_tmem != 0), dim3(P.nblk), dim3(KIE_THREADS), args,
+    return cudaLaunchCooperativeKernel(b1_fn(P.dtype, P.wesz == 1, P.b1_tmem != 0, P.b1_kvr != 0), dim3(P.nblk), dim3(KIE_THREADS), args,
                                        kie_b1_smem_bytes(), stream);
 }
 

@@ -27,8 +27,8 @@ size_t kie_b1_smem_bytes();
 int kie_b1_chunk_rows(int K);
 int kie_b1_max_rows(int K);
 bool kie_b1_tmem_ok(int d, bool f8);
-cudaError_t kie_b1_prepare(int dtype, bool f8, bool tm);
-cudaError_t kie_b1_occupancy(int dtype, bool f8, bool tm, int *blocks_per_sm);
+cudaError_t kie_b1_prepare(int dtype, bool f8, bool tm, bool kvr);
+cudaError_t kie_b1_occupancy(int dtype, bool f8, bool tm, bool kvr, int *blocks_per_sm);
 cudaError_t kie_b1_launch(const KieParams &P, const KieCmd &one, int resident, cudaStream_t stream);
 size_t kie_mr_smem_bytes();
 cudaError_t kie_mr_prepare(int dtype);
@@ -205,6 +205,7 @@ static const char *shape_error(const kie_config &c) {
     if (c.weight_fp8 != 0 && (c.weight_fp8 != 1 || c.modes != KIE_MODE_BATCH1))
         return "weight_fp8 must be 0 or 1, and 1 needs modes == KIE_MODE_BATCH1";
     if (c.b1_staging != 0 && c.b1_staging != 1) return "b1_staging must be 0 or 1";
+    if (c.b1_kv_path < 0 || c.b1_kv_path > 2) return "b1_kv_path must be 0, 1 or 2";
     return nullptr;
 }
 
@@ -255,11 +256,13 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
     }
     // batch-1 weights staged on into TMEM where the kernel's chunk layouts allow it
     const bool b1_tm = c.b1_staging == 1 && kie_b1_tmem_ok(c.d_model, c.weight_fp8 != 0);
+    // the attention's K/V through the weight ring at long contexts, from L2 otherwise
+    const bool b1_kvr = c.b1_kv_path == 2 || (c.b1_kv_path == 0 && c.max_ctx > 8192);
     if (b1) {
-        e = kie_b1_prepare(c.dtype, c.weight_fp8 != 0, b1_tm);
+        e = kie_b1_prepare(c.dtype, c.weight_fp8 != 0, b1_tm, b1_kvr);
         if (e != cudaSuccess) return bail(eng->cuda_fail(e, "kernel attributes"));
         int occ = 0;
-        e = kie_b1_occupancy(c.dtype, c.weight_fp8 != 0, b1_tm, &occ);
+        e = kie_b1_occupancy(c.dtype, c.weight_fp8 != 0, b1_tm, b1_kvr, &occ);
         if (e != cudaSuccess || occ < 1)
             return bail(eng->cuda_fail(e == cudaSuccess ? cudaErrorInvalidConfiguration : e,
                                        "batch-1 megakernel does not fit on an SM"));
@@ -299,11 +302,13 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
     }
     // attention splits: about one (kv head, split) unit per CTA
     P.splits = std::max(1, nblk / Hkv);
+
     const int E = G * D;  // attention outputs of one kv head (its query heads)
     const bool f8 = c.weight_fp8 != 0;
     const int esz = f8 ? 1 : 2;
     P.wesz = esz;
     P.b1_tmem = b1_tm ? 1 : 0;
+    P.b1_kvr = b1_kvr ? 1 : 0;
     const int Kph[KIE_NPH] = {d, 8, d, 8, d};
     std::vector<int> row0((size_t)KIE_NPH * (nblk + 1));
     // two rotation pairs at a time: a CTA's pairs then come as (dims i, i + 1), i even, of one

@@ -78,6 +78,7 @@ struct KieParams {
     const uint8_t *wpack;
     int wesz;                       // bytes per streamed weight: 2 (dtype), or 1 (E4M3 codes)
     int b1_tmem;                    // 1: ring chunks are moved on into TMEM and read from there
+    int b1_kvr;                     // 1: the attention units' K/V rows stream through the weight ring
     const float *wsc;               // E4M3 row scales: per layer [QKV rows | d | gate/up rows | d], then [V]
     int sc_stride;                  // floats per layer in wsc
     const int *row0;                // [KIE_NPH][nblk+1] partition: rows (GEMV phases), 8-column groups (folds)

@@ -41,7 +41,7 @@ class KieConfig(ctypes.Structure):
                                                "vocab")] + \
                [("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float)] + \
                [(n, ctypes.c_int32) for n in ("dtype", "max_sessions", "max_ctx", "timeout_ms", "idle_ms", "modes",
-                                               "device", "weight_fp8", "b1_staging")]
+                                               "device", "weight_fp8", "b1_staging", "b1_kv_path")]
 
 
 class KieWeights(ctypes.Structure):
@@ -111,12 +111,14 @@ def _ptr(a: np.ndarray):
 
 def config(model, max_sessions: int = 1, max_ctx: int = 4096, timeout_ms: int = 10000, idle_ms: int = 200,
            modes: int = KIE_MODE_BATCH1, device: int = 0, weight_fp8: bool = False,
-           b1_staging: int = 0) -> KieConfig:
+           b1_staging: int = 0, b1_kv_path: int = 0) -> KieConfig:
     """A kie_config for a model shape (any object with the shape attributes of synth.ModelConfig).
 
     b1_staging: 0 streams the batch-1 kernel's weights through the shared-memory ring alone;
     1 also stages the first chunks after each layer's QKV rows in TMEM where the shape allows it
-    (16-bit weights, d_model 2048 or 4096)."""
+    (16-bit weights, d_model 2048 or 4096).
+    b1_kv_path: 0 picks by max_ctx (the weight ring above 8192 positions), 1 reads the KV cache
+    from L2, 2 streams it through the weight ring."""
     c = KieConfig()
     lib.kie_config_defaults(ctypes.byref(c))
     for f in ("n_layers", "d_model", "n_heads", "n_kv_heads", "head_dim", "ffn", "vocab", "dtype"):
@@ -126,6 +128,7 @@ def config(model, max_sessions: int = 1, max_ctx: int = 4096, timeout_ms: int = 
                                                                                 idle_ms, modes, device)
     c.weight_fp8 = 1 if weight_fp8 else 0
     c.b1_staging = b1_staging
+    c.b1_kv_path = b1_kv_path
     return c
 
 

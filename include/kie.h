@@ -85,6 +85,13 @@ typedef struct {
                              one B200 about as fast as 0 on the 8B shape and 4 % slower on
                              the 1.9B shape, since streaming through the attention step
                              and the grid barriers lengthens their L2 round trips.        */
+    int32_t b1_kv_path;   /* how the batch-1 kernel's attention reads the KV cache:
+                             0 (default): 2 when max_ctx > 8192, else 1.
+                             1: plain loads from L2, the split's rows read into L2 during
+                             the previous phase (best at short contexts).
+                             2: bulk copies through the weight ring, 128 positions (64 KB)
+                             per copy (best at long contexts, where each split's rows no
+                             longer fit its read-ahead). Same results either way.          */
 } kie_config;
 
 /*

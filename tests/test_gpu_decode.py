@@ -130,18 +130,22 @@ def test_tiny_generate_and_launch_match_oracle_chain(kie):
         assert np.array_equal(out_d.cpu().numpy(), gen)
 
 
-@pytest.mark.parametrize("name,prompt_len,steps,staging", [
-    ("slice-1.9b", 40, 8, 0), ("slice-8b", 24, 6, 0), ("ragged", 33, 10, 0),
-    ("slice-1.9b", 150, 8, 1), ("slice-8b", 90, 6, 1),
+@pytest.mark.parametrize("name,prompt_len,steps,staging,kv_path", [
+    ("slice-1.9b", 40, 8, 0, 1), ("slice-8b", 24, 6, 0, 1), ("ragged", 33, 10, 0, 1),
+    ("slice-1.9b", 150, 8, 1, 1), ("slice-8b", 90, 6, 1, 1),
+    ("tiny", 16, 12, 0, 2), ("ragged", 33, 10, 0, 2), ("slice-1.9b", 40, 8, 0, 2), ("slice-8b", 24, 6, 0, 2),
+    ("slice-1.9b", 150, 8, 1, 2),
 ])
-def test_sliced_shapes_parity(kie, name, prompt_len, steps, staging):
+def test_sliced_shapes_parity(kie, name, prompt_len, steps, staging, kv_path):
     """Two-layer slices of the 1.9B (fp16, GQA 2) and 8B (bf16, GQA 4) shapes at full width, and a ragged
     shape (odd vocab, GQA 3, rows not divisible by the SM count). staging 1: the slices again with
-    the weight chunks of the attention step staged in TMEM (d_model 2048 and 4096 take it)."""
+    the weight chunks of the attention step staged in TMEM (d_model 2048 and 4096 take it).
+    kv_path 2: the attention's K/V rows stream through the weight ring (one pass per two query
+    heads: two passes on the 8B slice); 1: read from L2."""
     from bandwidth_bound_stream_b200 import synth
     from tests.parity import assert_reports
     m = synth.CONFIGS[name]
-    dw, eng, orc = _setup(kie, m, prompt_len + steps + 4, b1_staging=staging)
+    dw, eng, orc = _setup(kie, m, prompt_len + steps + 4, b1_staging=staging, b1_kv_path=kv_path)
     with eng:
         reps = _lockstep(kie, eng, orc, m, synth.prompt(m, prompt_len), steps)
     assert_reports(reps, m.dtype)
