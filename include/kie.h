@@ -121,7 +121,8 @@ void kie_config_defaults(kie_config *cfg);
  * mapped host mailbox), computes the static work partition for this GPU's SM count and
  * repacks the weights. Constraints: d_model, n_heads*head_dim and ffn multiples of 64,
  * d_model <= 8192 (<= 4096 with KIE_MODE_BATCH1), ffn and n_heads*head_dim <= 14336;
- * head_dim even and <= 128; n_heads a multiple of n_kv_heads with n_heads/n_kv_heads <= 8.
+ * head_dim one of 8, 16, 32, 64, 128; n_heads a multiple of n_kv_heads with
+ * n_heads/n_kv_heads <= 8.
  * Errors: KIE_ERR_ARG (shape), KIE_ERR_CUDA (allocation or launch). On error *out is NULL.
  */
 kie_status kie_create(const kie_config *cfg, const kie_weights *w, kie_engine **out);
@@ -141,6 +142,8 @@ kie_status kie_session_rewind(kie_engine *eng, int32_t sid, int32_t ctx);
 kie_status kie_session_kv(kie_engine *eng, int32_t sid, void **k_dev, void **v_dev);
 
 /*
+ * Prefill, the first call of the pages' request cycle (the prompt fills the KV cache that every
+ * later token reads: "Kog 3000 tok/s 实时推理…", section 内存带宽优化的三层策略).
  * Appends a prompt: tokens (HOST, n >= 1) are processed teacher-forced at positions
  * ctx..ctx+n-1, and *first_token (HOST) receives the argmax after the last one.
  * KIE_ERR_CAPACITY if ctx + n > max_ctx (nothing written). Uses the tick kernel's
@@ -149,14 +152,18 @@ kie_status kie_session_kv(kie_engine *eng, int32_t sid, void **k_dev, void **v_d
 kie_status kie_prefill(kie_engine *eng, int32_t sid, const int32_t *tokens, int32_t n, int32_t *first_token);
 
 /*
- * One decode step through the doorbell: in_token at position ctx, *out_token (HOST)
+ * One decode step (the pages' bandwidth-bound step: every weight byte and the KV cache read
+ * once per token, same section) through the doorbell of the resident kernel (the host only
+ * writes inputs and reads outputs: "实时AI推理为何贵56倍？…", section 让工作常驻 GPU):
+ * in_token at position ctx, *out_token (HOST)
  * receives the argmax. logits_dev (DEVICE, nullable) receives the fp32 logits [vocab].
  */
 kie_status kie_decode_step(kie_engine *eng, int32_t sid, int32_t in_token, int32_t *out_token, float *logits_dev);
 
 /*
  * n greedy steps through the doorbell, the argmax fed back on the GPU with no host round
- * trip per token: out_tokens (HOST, [n]) receives each step's argmax.
+ * trip per token (the persistent single-kernel runtime of the HN digest of Kog's inference
+ * engine, section 技术原理): out_tokens (HOST, [n]) receives each step's argmax.
  */
 kie_status kie_generate(kie_engine *eng, int32_t sid, int32_t in_token, int32_t n, int32_t *out_tokens);
 
@@ -174,9 +181,10 @@ kie_status kie_decode_launch(kie_engine *eng, int32_t sid, const int32_t *in_tok
 kie_status kie_sync(kie_engine *eng);
 
 /*
- * One tick of the continuous-inference workload: the n_sess sessions sids[] (HOST)
- * advance together by `steps` greedy tokens each, weights read once per step for all of
- * them. in_tokens (HOST, [n_sess]) are the first inputs; step s's argmax is the input of
+ * One tick of the continuous-inference workload ("实时AI推理为何贵56倍？…", sections
+ * 让所有活跃会话同步推进 and 实测数据: all due sessions advance as one batch on a fixed
+ * deadline): the n_sess sessions sids[] (HOST) advance together by `steps` greedy tokens
+ * each, weights read once per step for all of them. in_tokens (HOST, [n_sess]) are the first inputs; step s's argmax is the input of
  * step s+1 on the GPU. out_tokens (HOST, [steps][n_sess]) receive every argmax.
  * logits_dev (DEVICE, nullable) receives [steps][n_sess][vocab] fp32.
  * Needs KIE_MODE_TICK; n_sess <= 64, distinct sids.
