@@ -17,9 +17,12 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 KIE_SOURCES = ["kie_engine.cu", "kie_b1.cu", "kie_mr.cu", "kie_attn.cu", "kie_fp8.cu"]
-# build variants of the engine library: the product ("") and a diagnostic build, each its own
-# file (selected at import by KIE_VARIANT): "profile" times the GEMV consumer warps per chunk
-VARIANTS = {"": [], "profile": ["-DKIE_PROFILE_GEMV"]}
+# build variants of the engine library: the product ("") and two diagnostic builds, each its own
+# file (selected at import by KIE_VARIANT): "debug" checks the index of every kernel write to
+# global memory (recording an error instead of writing) and keeps guard words around every
+# engine buffer, which the host checks after each command; "profile" times the GEMV consumer
+# warps per chunk
+VARIANTS = {"": [], "debug": ["-DKIE_CHECK_BOUNDS"], "profile": ["-DKIE_PROFILE_GEMV"]}
 KIE_HEADERS = ["kie_device.cuh", "kie_internal.h", "kie_attn.cuh", "kie_sample.cuh"]
 
 

@@ -288,6 +288,8 @@ __device__ __forceinline__ void attn_tail(const AttnArgs &A, AttnSmem &S, int un
             val.x = ((S.wacc[0][k] + S.wacc[1][k]) + S.wacc[2][k]) + S.wacc[3][k];
             val.y = ((S.wacc[0][k + 1] + S.wacc[1][k + 1]) + S.wacc[2][k + 1]) + S.wacc[3][k + 1];
         }
+        if (!in_bounds(((size_t)unit * Gt + hoff) * (D + 2) + 2 * i + 1 < (size_t)A.Hkv * nsplit * Gt * (D + 2), A.err, 0x30))
+            continue;
         if (A.cnt_target) pub_f32x2(pp + 2 * i, val.x, val.y, ptok);
         else reinterpret_cast<float2 *>(pp)[i] = val;
     }

@@ -219,7 +219,7 @@ __host__ __device__ inline int col_slices(int K) { return K <= 8192 ? 8 : 16; }
 __host__ __device__ inline int rows_per_group(int K) { return K <= 2048 ? 8 : K <= 4096 ? 4 : 2; }
 
 __device__ __forceinline__ void trace_mark(const KieParams &P, int t, int ev, float after = 0.f) {
-    if (P.trace && t < P.trace_tokens && threadIdx.x == 0)
+    if (P.trace && t < P.trace_tokens && threadIdx.x == 0 && in_bounds(ev < P.trace_events, P.err, 0x14))
         P.trace[((size_t)blockIdx.x * P.trace_tokens + t) * P.trace_events + ev] = globaltimer() + (after != after);
 }
 
@@ -981,14 +981,18 @@ __device__ void epilogue_qkv(const KieParams &P, B1Shared &S, int l, int sid, in
         auto pack = [](float x0, float x1) { return (uint32_t)store1<DT>(x0) | ((uint32_t)store1<DT>(x1) << 16); };
         if (r < qd) {
             float *qp = P.q + (r / D) * D;
-            pub_f32x2(qp + i, ra, ra1, tk);
-            pub_f32x2(qp + i + half, rb, rb1, tk);
+            if (in_bounds((r / D) * D + i + half + 1 < qd, P.err, 0x10)) {
+                pub_f32x2(qp + i, ra, ra1, tk);
+                pub_f32x2(qp + i + half, rb, rb1, tk);
+            }
         } else {
             const bool isk = r < qd + kvd;
             const int g = (r - qd - (isk ? 0 : kvd)) / D;
             uint16_t *cp = (isk ? P.kcache : P.vcache) + sess + ((size_t)(l * P.Hkv + g) * P.max_ctx + pos) * D;
-            pub_u32(cp + i, pack(ra, ra1), tk);
-            pub_u32(cp + i + half, pack(rb, rb1), tk);
+            if (in_bounds(pos < P.max_ctx && g < P.Hkv && sid < P.max_sessions && i + half + 1 < D, P.err, 0x11)) {
+                pub_u32(cp + i, pack(ra, ra1), tk);
+                pub_u32(cp + i + half, pack(rb, rb1), tk);
+            }
         }
     }
     if (l == 0) {  // the residual starts as the embedding row (each CTA writes a 1/nblk share)
@@ -1056,7 +1060,7 @@ __device__ void epilogue_head(const KieParams &P, B1Shared &S, float *logits, fl
     int bi = 0x7fffffff;
     for (int r = tid; r < n; r += KIE_CONS_THREADS) {  // rows tid and tid + 512 (n <= 1024)
         const float v = rowsum(S, r, col_slices(P.K[PH_HEAD])) * (r == tid ? rsc.x : rsc.y);
-        if (logits) logits[rbeg + r] = v;
+        if (logits && in_bounds(rbeg + r < P.V, P.err, 0x12)) logits[rbeg + r] = v;
         argmax_combine(bv, bi, v, rbeg + r);
     }
     warp_argmax(bv, bi);
@@ -1474,7 +1478,7 @@ __global__ void __launch_bounds__(KIE_THREADS, 1) kie_b1_kernel(KieParams P, Kie
                     // a prompt arrives in the mailbox; stage it in device memory for all CTAs
                     if (S.cmd.op == OP_PREFILL)
                         for (int j = tid; j < S.cmd.n; j += KIE_CONS_THREADS)
-                            P.tokbuf[j] = ((const volatile int32_t *)S.cmd.tokens)[j];
+                            if (in_bounds(j < P.max_ctx, P.err, 0x13)) P.tokbuf[j] = ((const volatile int32_t *)S.cmd.tokens)[j];
                 }
                 grid_barrier(P, S, epoch, P.idle_ns + P.timeout_ns, 0, true);
                 if (tid == 0) {

@@ -49,6 +49,21 @@ KIE_DEV unsigned ld_acquire_gpu_u32(const unsigned *p) {
     return v;
 }
 
+// Index check of a global write (the diagnostic build with KIE_CHECK_BOUNDS, which stands in
+// for a memory checker): false, with DERR_BOUNDS and `where` recorded in the error word, when
+// the index is out of range; the caller then skips the write. The product build compiles it
+// to true.
+KIE_DEV bool in_bounds(bool ok, unsigned *err, unsigned where) {
+#ifdef KIE_CHECK_BOUNDS
+    if (!ok) atomicCAS(err, 0u, ((unsigned)DERR_BOUNDS << 8) | (where & 0xFFu));
+    return ok;
+#else
+    (void)err;
+    (void)where;
+    return true;
+#endif
+}
+
 // ------------------------------------------------------------------ completion-based publication
 //
 // A release (fence.release, red.release, fence.acq_rel) at GPU scope waits until every memory

@@ -128,6 +128,39 @@ struct kie_engine {
     kie_status cuda_fail(cudaError_t e, const char *what) {
         return fail(KIE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
     }
+#ifdef KIE_CHECK_BOUNDS
+    // Diagnostic build: every engine buffer sits between two guard regions of GUARD bytes
+    // filled with GUARD_BYTE; check_guards() reports any that a kernel (or anyone) overwrote.
+    static constexpr size_t GUARD = 256;
+    static constexpr int GUARD_BYTE = 0xA5;
+    std::vector<std::pair<uint8_t *, size_t>> guarded;  // user region, its bytes
+    template <class T>
+    cudaError_t alloc(T **p, size_t bytes) {
+        bytes = bytes < 16 ? 16 : bytes;
+        uint8_t *q = nullptr;
+        cudaError_t e = cudaMalloc(&q, bytes + 2 * GUARD);
+        if (e != cudaSuccess) return e;
+        dev_allocs.push_back(q);
+        e = cudaMemset(q, GUARD_BYTE, GUARD);
+        if (e == cudaSuccess) e = cudaMemset(q + GUARD + bytes, GUARD_BYTE, GUARD);
+        guarded.push_back({q + GUARD, bytes});
+        *p = reinterpret_cast<T *>(q + GUARD);
+        return e;
+    }
+    // index of the first buffer whose guard words changed, or -1
+    int check_guards() const {
+        std::vector<uint8_t> h(GUARD);
+        for (size_t i = 0; i < guarded.size(); i++) {
+            for (int side = 0; side < 2; side++) {
+                const uint8_t *g = side ? guarded[i].first + guarded[i].second : guarded[i].first - GUARD;
+                if (cudaMemcpy(h.data(), g, GUARD, cudaMemcpyDeviceToHost) != cudaSuccess) return (int)i;
+                for (uint8_t b : h)
+                    if (b != GUARD_BYTE) return (int)i;
+            }
+        }
+        return -1;
+    }
+#else
     template <class T>
     cudaError_t alloc(T **p, size_t bytes) {
         void *q = nullptr;
@@ -138,6 +171,7 @@ struct kie_engine {
         }
         return e;
     }
+#endif
 };
 
 #define CK(expr, what)                                        \
@@ -712,12 +746,19 @@ static kie_status check_device_error(kie_engine *eng) {
     unsigned err = 0;
     cudaError_t e = cudaMemcpy(&err, eng->P.err, 4, cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return eng->fail(KIE_ERR_DEVICE, "reading device status: %s", cudaGetErrorString(e));
+#ifdef KIE_CHECK_BOUNDS
+    if (!err) {
+        const int bad = eng->check_guards();
+        if (bad >= 0) return eng->fail(KIE_ERR_DEVICE, "guard words of engine buffer %d overwritten", bad);
+    }
+#endif
     if (err) {
         const unsigned code = err >> 8, where = err & 0xFF;
         const char *what = code == DERR_BARRIER_TIMEOUT ? "grid barrier timed out"
                            : code == DERR_RING_TIMEOUT  ? "weight ring wait timed out"
                            : code == DERR_BAD_TOKEN     ? "token id out of range"
                            : code == DERR_MMA_TIMEOUT   ? "tensor-core wait timed out"
+                           : code == DERR_BOUNDS        ? "write index out of range (diagnostic build)"
                                                         : "unknown device error";
         return eng->fail(code == DERR_BARRIER_TIMEOUT || code == DERR_RING_TIMEOUT || code == DERR_MMA_TIMEOUT
                              ? KIE_ERR_TIMEOUT

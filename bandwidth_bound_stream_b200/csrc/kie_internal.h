@@ -37,7 +37,7 @@ struct SampleCfg {
 enum { OP_NONE = 0, OP_DECODE = 1, OP_PREFILL = 2, OP_TICK = 3, OP_EXIT = 4 };
 
 // Device error codes (err word = code << 8 | where).
-enum { DERR_BARRIER_TIMEOUT = 1, DERR_RING_TIMEOUT = 2, DERR_BAD_TOKEN = 3, DERR_MMA_TIMEOUT = 4 };
+enum { DERR_BARRIER_TIMEOUT = 1, DERR_RING_TIMEOUT = 2, DERR_BAD_TOKEN = 3, DERR_MMA_TIMEOUT = 4, DERR_BOUNDS = 5 };
 
 struct KieCmd {
     int32_t op, sid, pos0, n;

@@ -394,7 +394,8 @@ __device__ void mr_epilogue(const KieParams &P, MrShared &S, uint32_t &u_it, int
 #pragma unroll
                 for (int j = 0; j < 32; j++) {
                     const int s = half * 32 + j;
-                    if (s < M) atomicAdd(G.y + (size_t)s * G.ldy + row, hi[j] + lo[j]);
+                    if (s < M && in_bounds(s < MAXR && row < G.ldy, P.err, 0x23))
+                        atomicAdd(G.y + (size_t)s * G.ldy + row, hi[j] + lo[j]);
                 }
             }
         }
@@ -459,7 +460,8 @@ __device__ void phase_norm(const KieParams &P, MrShared &S, int g_next, int l, b
             cvt8<DT>(__ldg(reinterpret_cast<const uint4 *>(gain + 8 * c)), gv);
             const float v[8] = {a.x * r * gv[0], a.y * r * gv[1], a.z * r * gv[2], a.w * r * gv[3],
                                 b.x * r * gv[4], b.y * r * gv[5], b.z * r * gv[6], b.w * r * gv[7]};
-            put_b8<DT>(P.mr_bpack + (size_t)(c >> 3) * TILE, m, c & 7, v);
+            if (in_bounds(m < MAXR && (c >> 3) < max(max(P.d, P.Hq * P.D), P.F) / 64, P.err, 0x24))
+                put_b8<DT>(P.mr_bpack + (size_t)(c >> 3) * TILE, m, c & 7, v);
         }
     }
 }
@@ -482,7 +484,8 @@ __device__ void phase_act(const KieParams &P, int M) {
 #pragma unroll
             for (int e = 0; e < 4; e++) v[4 * h + e] = ga[e] / (1.f + expf(-ga[e])) * ub[e];
         }
-        put_b8<DT>(P.mr_bpack + (size_t)(c >> 3) * TILE, m, c & 7, v);
+        if (in_bounds(m < MAXR && (c >> 3) < max(max(P.d, P.Hq * P.D), P.F) / 64, P.err, 0x25))
+            put_b8<DT>(P.mr_bpack + (size_t)(c >> 3) * TILE, m, c & 7, v);
     }
 }
 
@@ -504,19 +507,25 @@ __device__ void phase_rope(const KieParams &P, int l, int M) {
                 const float ra = a * cs.x - b * cs.y, rb = b * cs.x + a * cs.y;
                 if (head < P.Hq) {
                     float *q = P.mr_q + (size_t)m * qd + base;
-                    q[i] = ra;
-                    q[i + half] = rb;
+                    if (in_bounds(m < MAXR && base + i + half < qd, P.err, 0x20)) {
+                        q[i] = ra;
+                        q[i + half] = rb;
+                    }
                 } else {
                     const int g = head - P.Hq;
                     uint16_t *kp = P.kcache + sess + ((size_t)(l * P.Hkv + g) * P.max_ctx + pos) * D;
-                    kp[i] = store1<DT>(ra);
-                    kp[i + half] = store1<DT>(rb);
+                    if (in_bounds(pos < P.max_ctx && g < P.Hkv && i + half < D, P.err, 0x21)) {
+                        kp[i] = store1<DT>(ra);
+                        kp[i + half] = store1<DT>(rb);
+                    }
                 }
             } else {
                 const int g = head - P.Hq - P.Hkv;
                 uint16_t *vp = P.vcache + sess + ((size_t)(l * P.Hkv + g) * P.max_ctx + pos) * D;
-                vp[i] = store1<DT>(a);
-                vp[i + half] = store1<DT>(b);
+                if (in_bounds(pos < P.max_ctx && g < P.Hkv && i + half < D, P.err, 0x22)) {
+                    vp[i] = store1<DT>(a);
+                    vp[i + half] = store1<DT>(b);
+                }
             }
         }
     }

@@ -13,11 +13,12 @@ import os
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-# KIE_VARIANT selects a diagnostic build of the same library ("profile": GEMV consumer timing
-# in the phase trace); unset means the product build
+# KIE_VARIANT selects a diagnostic build of the same library ("debug": index checks on every
+# kernel write and guard words around the engine's buffers; "profile": GEMV consumer timing in
+# the phase trace); unset means the product build
 VARIANT = os.environ.get("KIE_VARIANT", "")
-if VARIANT not in ("", "profile"):
-    raise ImportError(f"KIE_VARIANT={VARIANT!r}: expected unset or 'profile'")
+if VARIANT not in ("", "debug", "profile"):
+    raise ImportError(f"KIE_VARIANT={VARIANT!r}: expected unset, 'debug' or 'profile'")
 LIB_PATH = os.path.join(_HERE, "libkie.so" if not VARIANT else f"libkie_{VARIANT}.so")
 
 KIE_OK, KIE_ERR_ARG, KIE_ERR_CAPACITY, KIE_ERR_CUDA = 0, -1, -2, -3
