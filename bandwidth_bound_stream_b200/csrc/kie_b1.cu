@@ -181,6 +181,7 @@ struct __align__(16) B1Shared {
     float fold_in[KIE_FOLD_MAX];  // the current fold's inputs: this CTA's slice of o, or of u
     float red[64];
     int redi[32];
+    float nrm[16];                // the RMSNorm's partial sums of squares (one per column slice)
     float2 rope_s[KIE_DMAX / 2];  // rotation of the current position, loaded at the start of QKV
     uint64_t full[KIE_NSLOT];
     uint64_t empty[KIE_NSLOT];
@@ -704,18 +705,11 @@ __device__ void gemv_phase(const KieParams &P, B1Shared &S, uint32_t &ring_it, u
         }
     }
     // 1/sqrt(mean(x^2) + eps) of the whole input: the CS warps of the first group cover every
-    // column once; their sums are added in warp order, so every thread gets the same value
+    // column once; their sums are added in warp order after the rows, so every thread gets the
+    // same value. It is one factor of every row sum, so the rows run on g * x and the factor
+    // joins the row scales the epilogue applies (the reduction overlaps the first chunks).
     ss = warp_sum(ss);
-    if (lane == 0 && w < CS) S.red[w] = ss;
-    named_bar_sync(1, KIE_CONS_THREADS);
-    float tot = 0.f;
-#pragma unroll
-    for (int k = 0; k < CS; k++) tot += S.red[k];
-    const float rstd = rsqrtf(tot / (float)P.d + P.eps);
-#pragma unroll
-    for (int i = 0; i < NV; i++)
-#pragma unroll
-        for (int e = 0; e < 8; e++) h[i][e] *= rstd;
+    if (lane == 0 && w < CS) S.nrm[w] = ss;
     if (l < P.L) trace_mark(P, t, 1 + 16 * l + (ph == PH_QKV ? 11 : 12), h[0][0]);
 
     const int grp = w / CS, ws = w % CS;
@@ -825,6 +819,12 @@ __device__ void gemv_phase(const KieParams &P, B1Shared &S, uint32_t &ring_it, u
         P.trace[((size_t)blockIdx.x * P.trace_tokens + t) * P.trace_events + 1 + 16 * l + 13 + grp] = busy;
 #endif
     named_bar_sync(1, KIE_CONS_THREADS);
+    float tot = 0.f;
+#pragma unroll
+    for (int k = 0; k < CS; k++) tot += S.nrm[k];
+    const float rstd = rsqrtf(tot / (float)P.d + P.eps);
+    rsc.x *= rstd;
+    rsc.y *= rstd;
 }
 
 // the row sum of row r of the current phase (column slices added in a fixed order)
