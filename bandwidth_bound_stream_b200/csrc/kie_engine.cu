@@ -650,13 +650,14 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
     P.sess_stride = (long long)L * Hkv * c.max_ctx * D;
     CKC(eng->alloc(&P.kcache, (size_t)c.max_sessions * P.sess_stride * 2), "cudaMalloc K cache");
     CKC(eng->alloc(&P.vcache, (size_t)c.max_sessions * P.sess_stride * 2), "cudaMalloc V cache");
-    // the tick kernel's attention reads K tiles by 2-D TMA: the K arena as [rows][D], rows =
-    // sessions * L * Hkv * max_ctx (one per cached position), boxes of 128 rows x 64 dims,
-    // 128-byte swizzled (the MMA operand layout); head_dim not a multiple of 64 keeps the
-    // CUDA-core attention
-    P.mr_kmap = nullptr;
+    // the tick kernel's attention reads K and V tiles by 2-D TMA: each arena as [rows][D], rows
+    // = sessions * L * Hkv * max_ctx (one per cached position), boxes of 128 rows x 64 dims,
+    // 128-byte swizzled (the MMA operand layouts); head_dim not a multiple of 64 keeps the
+    // CUDA-core attention. A tile's rows may run up to 127 past the last row (zero fill), so
+    // every coordinate stays below 2^31.
+    P.mr_kmap = P.mr_vmap = nullptr;
     const unsigned long long kv_rows = (unsigned long long)c.max_sessions * L * Hkv * c.max_ctx;
-    if (mr && D % 64 == 0 && kv_rows < (1ull << 31)) {
+    if (mr && D % 64 == 0 && kv_rows + 256 < (1ull << 31)) {
         // the driver's encoder, looked up through the runtime (no link-time driver dependency)
         typedef CUresult (*EncodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                         const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -668,22 +669,25 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
             eng->fail(KIE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
             return bail(KIE_ERR_CUDA);
         }
-        CUtensorMap tm;
+        CUtensorMap tm[2];
         const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)kv_rows};
         const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
         const cuuint32_t box[2] = {64, 128}, estr[2] = {1, 1};
-        const CUresult r = reinterpret_cast<EncodeTiled>(fn)(
-            &tm, c.dtype == KIE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, P.kcache, dims,
-            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) {
-            eng->fail(KIE_ERR_CUDA, "cuTensorMapEncodeTiled (K arena) failed: %d", (int)r);
-            return bail(KIE_ERR_CUDA);
+        for (int a = 0; a < 2; a++) {
+            const CUresult r = reinterpret_cast<EncodeTiled>(fn)(
+                &tm[a], c.dtype == KIE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                a == 0 ? P.kcache : P.vcache, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            if (r != CUDA_SUCCESS) {
+                eng->fail(KIE_ERR_CUDA, "cuTensorMapEncodeTiled (%s arena) failed: %d", a == 0 ? "K" : "V", (int)r);
+                return bail(KIE_ERR_CUDA);
+            }
         }
-        void *d_map = nullptr;
-        CKC(eng->alloc(&d_map, sizeof(CUtensorMap)), "cudaMalloc tensor map");
-        CKC(cudaMemcpy(d_map, &tm, sizeof(CUtensorMap), cudaMemcpyHostToDevice), "upload tensor map");
+        uint8_t *d_map = nullptr;
+        CKC(eng->alloc(&d_map, 2 * sizeof(CUtensorMap)), "cudaMalloc tensor maps");
+        CKC(cudaMemcpy(d_map, tm, 2 * sizeof(CUtensorMap), cudaMemcpyHostToDevice), "upload tensor maps");
         P.mr_kmap = d_map;
+        P.mr_vmap = d_map + sizeof(CUtensorMap);
     }
 
     // ---- activations and scratch

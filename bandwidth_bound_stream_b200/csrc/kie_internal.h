@@ -118,9 +118,10 @@ struct KieParams {
     // the B operand of the running GEMM: one swizzled 128 x 64 16-bit tile per k-step (rows
     // 0-63 hi, 64-127 lo of the activations), written by the phase that finalises them
     uint8_t *mr_bpack;
-    // tensor map (in device memory) of the K arena viewed as [sessions * L * Hkv * max_ctx][D],
-    // boxes of 128 rows x 64 dims with the 128-byte swizzle; null when D is not a multiple of 64
-    const void *mr_kmap;
+    // tensor maps (in device memory) of the K and V arenas viewed as [sessions * L * Hkv *
+    // max_ctx][D], boxes of 128 rows x 64 dims with the 128-byte swizzle; null when D is not a
+    // multiple of 64
+    const void *mr_kmap, *mr_vmap;
     unsigned *mr_cnt;
     int *mr_sid, *mr_pos, *mr_tok;  // [64] rows of the current command
 };

@@ -46,6 +46,8 @@ constexpr int A_SLOTS = 4, B_SLOTS = 2;   // atoms in flight: weights (HBM), act
 constexpr int KV_SLOTS = 4;               // 16 KB K/V chunks of the CUDA-core attention, in the B ring
 constexpr int MAXR = 64;                  // rows per step (hi half of B; lo half at +64)
 constexpr int TMEM_COLS = 256;            // two 128-column fp32 accumulators
+constexpr int NU_MAX = 16;                // units per attention stream (a CTA with more runs several)
+constexpr int AT_STAGES = 3;              // K/V tile stages of the tensor-core attention (A ring x 2, B ring)
 
 enum { G_QKV = 0, G_O = 1, G_GU = 2, G_DOWN = 3, G_HEAD = 4, NG = 5 };
 
@@ -57,8 +59,12 @@ struct __align__(1024) MrShared {
     uint64_t acc_full[2], acc_empty[2], drain;
     uint64_t k_full[KV_SLOTS], k_empty[KV_SLOTS];  // the B ring as a K/V chunk ring in attention
     uint32_t k_iss;                              // K/V chunks issued so far (thread 0)
-    uint64_t at_k[2], at_v[2], at_s;             // tensor-core attention: K, V tiles per stage; scores
-    uint32_t tk_iss[2], tv_iss[2], ts_iss;       // copies / MMA groups issued (thread 0)
+    uint64_t at_k[AT_STAGES], at_v[AT_STAGES], at_s, at_o;  // tensor-core attention: K, V per stage; scores; P.V
+    uint32_t tk_iss[AT_STAGES], tv_iss[AT_STAGES], ts_iss, to_iss;  // copies / MMA groups issued
+    float at_corr[2][KIE_GMAX];                  // per tile (two in flight): rescale of the running sums
+    float at_l[4][KIE_GMAX];                     // the softmax warps' shares of the sums
+    long long un_row0[NU_MAX];                   // the attention stream's units: first K/V arena row,
+    int un_ctx[NU_MAX], un_nt[NU_MAX];           // context, tiles
     volatile uint32_t att_seq;                   // attention phases finished (the producer waits on it)
     uint32_t tmem_base;
     KieCmd cmd;
@@ -126,12 +132,39 @@ KIE_DEV void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 lanes x 16 consecutive fp32 columns from TMEM
+KIE_DEV void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; i++) v[i] = __uint_as_float(r[i]);
+}
+
 // Shared-memory matrix descriptor of a K-major, 128-byte-swizzled tile (8-row atoms of 1024 B).
 KIE_DEV uint64_t smem_desc_sw128(uint32_t saddr) {
     uint64_t d = 0;
     d |= (uint64_t)((saddr >> 4) & 0x3FFFu);       // start address
     d |= (uint64_t)1u << 16;                        // leading byte offset (unused when swizzled)
     d |= (uint64_t)(1024u >> 4) << 32;              // stride byte offset: next 8-row atom
+    d |= (uint64_t)1u << 46;                        // descriptor version (sm_100)
+    d |= (uint64_t)2u << 61;                        // layout: 128-byte swizzle
+    return d;
+}
+
+// Shared-memory matrix descriptor of an MN-major, 128-byte-swizzled operand as a 2-D tile
+// copy of 64-element-wide boxes lands it: 128-byte rows of 64 consecutive M elements, one row
+// per k, 8-row atoms of 1024 B; the next 64 M elements lie one box (TILE bytes) further on.
+KIE_DEV uint64_t smem_desc_mn_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);       // start address
+    d |= (uint64_t)((TILE >> 4) & 0x3FFFu) << 16;   // leading byte offset: next 64 elements of M
+    d |= (uint64_t)(1024u >> 4) << 32;              // stride byte offset: next 8 rows of K
     d |= (uint64_t)1u << 46;                        // descriptor version (sm_100)
     d |= (uint64_t)2u << 61;                        // layout: 128-byte swizzle
     return d;
@@ -611,52 +644,88 @@ __device__ void tick_attn_unit(const KieParams &P, MrShared &S, const AttnArgs &
     attn_tail<DT, GC, NW, true>(A, S.at, g, Gt, hoff, m, l, acc);
 }
 
-// One (row, kv head) unit on the tensor cores (head_dim a multiple of 64), 128 positions per
-// tile:
-//   scores  S[p][c] = K[p] . Qt[c]  by tcgen05.mma (M = 128 positions, N = 16, K = head_dim):
-//           columns c < 8 hold the 16-bit hi part of the scaled query heads, c >= 8 the lo part,
-//           so S[p][h] + S[p][8 + h] is the score of head h to ~16 bits of the fp32 query;
-//   K tile  2-D TMA copy of 128 cached rows x 64 dims per box, 128-byte swizzled (the MMA's
-//           K-major operand layout), from a tensor map over the whole K arena;
-//   softmax warps 0-3 read a position each from TMEM, keep the running max M and sum L per
-//           head (the same values in every thread) and write p = 2^(s - M) to shared memory;
-//   P V     all 8 warps on the CUDA cores from the V tile (1-D bulk copy), D/8 lanes per row.
-// K and V tiles are double-buffered in the weight ring (4 x 32 KB), which the producer leaves
-// to attention (it holds the O projection's weights back until attention is done): the
-// copies of tile t + 2 are issued as soon as tile t is consumed, so a tile's loads overlap
-// the work on the tile before it.
+// Tensor-core attention of the tick and of chunked prefill (head_dim a multiple of 64). The
+// units (row, kv head) a CTA takes in one attention phase form one stream of 128-position
+// tiles, and every tile takes two tcgen05 products:
+//   scores  S[p][c] = K[p] . Qt[c]  (M = 128 positions, N = 16, K = head_dim). Columns c < 8
+//           hold the 16-bit hi part of the scaled query heads, c >= 8 the lo part, so
+//           S[p][h] + S[p][8 + h] is the score of head h to ~16 bits of the fp32 query.
+//   values  O[d][c] = sum_p V[p][d] Pt[c][p]  (M = 128 dims, N = 16, K = 128 positions). V is
+//           the MN-major operand just as the tile copy lands it; Pt holds p = 2^(s - M) of
+//           each head as 16-bit hi (row h) and lo (row 8 + h) parts, so O[d][h] + O[d][8 + h]
+//           is the tile's P.V of head h to ~16 bits of p.
+// K and V tiles are 2-D TMA copies (no multicast) of 128 positions x 64 dims per box,
+// 128-byte swizzled, from tensor maps over the whole K and V arenas, into two stages of the
+// weight ring and a third in the activation ring (the producer holds the O weights back until
+// attention is done, and no activation tile moves during it). The copies of stream tile k + 3
+// -- the next unit's first tiles near the end of a unit -- are issued as soon as tile k's
+// products are done, so loads run on across unit boundaries.
+// Warps 0-3 run the softmax: a position each from TMEM, the running max M per head (the same
+// in every thread) and each thread's share of the running sum. They write Pt, and thread 0
+// issues the next tile's score product as soon as its K tile is in, before the current
+// tile's P.V. Warps 4-7 fold each tile's P.V into the output one tile behind (a dim each
+// from TMEM, rescaled by the tile's correction), and issue the tile copies.
+
+// the K and V tile buffers of attention stage st: two stages in the weight ring, one in the
+// activation ring (both idle during attention)
+KIE_DEV uint8_t *at_kbuf(MrShared &S, int st) { return st < 2 ? S.a[2 * st] : S.b[0]; }
+KIE_DEV uint8_t *at_vbuf(MrShared &S, int st) { return st < 2 ? S.a[2 * st + 1] : S.b[1]; }
+
+// thread 0 or 128: the copies of stream tile k (tile k - (tiles of the units before) of its
+// unit) into stage st
+__device__ void attn_issue(const KieParams &P, MrShared &S, int k, int nunits, int st, int nks) {
+    int i = 0;
+    while (i < nunits && k >= S.un_nt[i]) k -= S.un_nt[i++];
+    if (i >= nunits) return;
+    const int y = (int)(S.un_row0[i] + (long long)k * 128);
+    mbar_arrive_expect_tx(&S.at_k[st], (uint32_t)(nks * TILE));
+    for (int ks = 0; ks < nks; ks++) tma_load_2d(at_kbuf(S, st) + ks * TILE, P.mr_kmap, ks * 64, y, &S.at_k[st]);
+    S.tk_iss[st]++;
+    mbar_arrive_expect_tx(&S.at_v[st], (uint32_t)(nks * TILE));
+    for (int ks = 0; ks < nks; ks++) tma_load_2d(at_vbuf(S, st) + ks * TILE, P.mr_vmap, ks * 64, y, &S.at_v[st]);
+    S.tv_iss[st]++;
+}
+
+// thread 0: the score product of the tile in stage st (K tile x query operand) into TMEM
+// columns 0-15
+KIE_DEV void attn_scores_mma(MrShared &S, const uint8_t *Qt, int st, int nks, uint32_t idesc) {
+    const uint32_t sk = smem_u32(at_kbuf(S, st)), sq = smem_u32(Qt);
+    for (int ks = 0; ks < nks; ks++)
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+            umma_f16(S.tmem_base, smem_desc_sw128(sk + ks * TILE + kk * 32), smem_desc_sw128(sq + ks * 2048 + kk * 32),
+                     idesc, (ks | kk) ? 1u : 0u);
+    umma_commit(&S.at_s);
+    S.ts_iss++;
+}
+
+// thread 0: the P.V product of the tile in stage st into TMEM columns col .. col + 15
+KIE_DEV void attn_pv_mma(MrShared &S, const uint8_t *Pt, int st, uint32_t col, uint32_t idesc) {
+    const uint32_t sv = smem_u32(at_vbuf(S, st)), sp = smem_u32(Pt);
+#pragma unroll
+    for (int kb = 0; kb < 2; kb++)
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+            umma_f16(S.tmem_base + col, smem_desc_mn_sw128(sv + kb * 8192 + kk * 2048),
+                     smem_desc_sw128(sp + kb * 2048 + kk * 32), idesc, (kb | kk) ? 1u : 0u);
+    umma_commit(&S.at_o);
+    S.to_iss++;
+}
+
+// One pass of a unit (row m, kv head g; query heads hoff .. hoff + GC - 1 of its Gt): stream
+// entry ui, tiles k0 .. k0 + ntile - 1 of the stream's ktot.
 template <int DT, int GC>
-__device__ void tick_attn_mma(const KieParams &P, MrShared &S, const AttnArgs &A, int g, int Gt, int hoff,
-                              long long row0, uint32_t &t_it) {
-    constexpr int NW = MR_WORKERS / 32;
+__device__ void tick_attn_tc(const KieParams &P, MrShared &S, const AttnArgs &A, int g, int Gt, int hoff, int ui,
+                             int nunits, int k0, int ktot, unsigned long long &t_it) {
+    static_assert(GC <= 8, "the query operand holds 8 heads (hi) + 8 (lo)");
     const int nh = min(GC, Gt - hoff);
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-    const int D = A.D, nks = D >> 6, lpp = D >> 3, ppw = 32 / lpp, sub = lane / lpp, sl = lane % lpp;
-    const int ngroups = NW * ppw, gi = w * ppw + sub;
-    const int ctx = A.ctx, ntile = (ctx + 127) >> 7;
-    // stage s: K in a[2s] ([nks][128 rows][128 B], swizzled), V in a[2s + 1] ([128][D] row-major)
-    uint8_t *Qt = reinterpret_cast<uint8_t *>(S.at.wacc);                          // [nks][16][128 B], swizzled
-    float *Ps = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(S.at.wacc) + 4096);  // [128][4]
-    const uint8_t *vsrc = reinterpret_cast<const uint8_t *>(A.v + (size_t)g * A.head_stride);
-    const uint32_t idesc = idesc_f16(DT, 16);
-    const uint32_t q0 = t_it;  // global index of this unit's first tile (stage = index & 1)
-    auto load_tile = [&](int t) {  // thread 0: K and V of tile t into its stage
-        const int st = (int)((q0 + t) & 1u);
-        mbar_arrive_expect_tx(&S.at_k[st], (uint32_t)nks * 16384u);
-        for (int ks = 0; ks < nks; ks++)
-            tma_load_2d(S.a[2 * st] + ks * 16384, P.mr_kmap, ks * 64, (int)(row0 + t * 128), &S.at_k[st]);
-        S.tk_iss[st]++;
-        const uint32_t bytes = (uint32_t)(min(128, ctx - t * 128) * D * 2);
-        mbar_arrive_expect_tx(&S.at_v[st], bytes);
-        bulk_g2s(S.a[2 * st + 1], vsrc + (size_t)t * 128 * D * 2, bytes, &S.at_v[st]);
-        S.tv_iss[st]++;
-    };
-    if (tid == 0 && !S.abort) {
-        fence_proxy_async_global();  // the newest rows were written (generic proxy) before the barrier
-        fence_proxy_async_smem();    // earlier generic reads of the ring before the copies refill it
-        load_tile(0);
-        if (ntile > 1) load_tile(1);
-    }
+    const int D = A.D, nks = D >> 6;
+    const int ctx = S.un_ctx[ui], ntile = S.un_nt[ui];
+    uint8_t *Qt = reinterpret_cast<uint8_t *>(S.at.wacc);  // [nks][16 rows][128 B], swizzled
+    uint8_t *Pt0 = Qt + 4096;                              // two tiles of [2][16 rows][128 B], swizzled
+    const uint32_t idesc_s = idesc_f16(DT, 16), idesc_o = idesc_f16(DT, 16) | (1u << 15);  // V MN-major
+
     // the query operand: rows h (hi) and 8 + h (lo) of the scaled query heads, other rows zero
     const float qscale = rsqrtf((float)D) * 1.4426950408889634f;
     for (int i = tid; i < 16 * (D >> 3); i += MR_WORKERS) {
@@ -683,115 +752,204 @@ __device__ void tick_attn_mma(const KieParams &P, MrShared &S, const AttnArgs &A
     fence_proxy_async_smem();  // generic writes of the query tile -> tensor-core reads
     named_bar_sync(1, MR_WORKERS);
 
-    float M[GC], L[GC], acc[GC][8];
+    if (w < 4) {  // ---- softmax warps
+        float M[GC], Ls[GC];
 #pragma unroll
-    for (int h = 0; h < GC; h++) {
-        M[h] = -CUDART_INF_F;
-        L[h] = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; e++) acc[h][e] = 0.f;
-    }
-    for (int t = 0; t < ntile; t++) {  // uniform control flow: every thread reaches every barrier
-        const uint32_t par = t_it & 1u;                 // the scores barrier completes once per tile
-        const int st = (int)(t_it & 1u);                // this tile's stage
-        const uint32_t spar = (t_it >> 1) & 1u;         // ... whose barriers complete every other tile
-        const uint8_t *Vs = S.a[2 * st + 1];
-        const int p0 = t * 128, np = min(128, ctx - p0);
-        if (tid == 0 && !S.abort) {
-            if (mbar_wait(&S.at_k[st], spar, P.timeout_ns, &S.abort)) {
-                tc_fence_after();
-                const uint32_t sk = smem_u32(S.a[2 * st]), sq = smem_u32(Qt);
-                for (int ks = 0; ks < nks; ks++)
-#pragma unroll
-                    for (int kk = 0; kk < 4; kk++)
-                        umma_f16(S.tmem_base, smem_desc_sw128(sk + ks * 16384 + kk * 32),
-                                 smem_desc_sw128(sq + ks * 2048 + kk * 32), idesc, (ks | kk) ? 1u : 0u);
-                umma_commit(&S.at_s);
-                S.ts_iss++;
-            } else {
-                if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x96);
-                S.abort = 1;
-            }
+        for (int h = 0; h < GC; h++) {
+            M[h] = -CUDART_INF_F;
+            Ls[h] = 0.f;
         }
-        float sc[GC];
-        if (w < 4) {
+        for (int t = 0; t < ntile; t++) {  // uniform control flow: every thread reaches every barrier
+            const int st = (int)(t_it % AT_STAGES);                   // this tile's K/V stage
+            const uint32_t spar = (uint32_t)(t_it / AT_STAGES) & 1u;  // ... whose barriers complete every third tile
+            const int pb = (int)(t_it & 1ull);                        // its Pt, correction and P.V buffers
+            const uint32_t par = (uint32_t)pb;                        // the score barrier completes once per tile
+            const int p0 = t * 128, np = min(128, ctx - p0);
+            uint8_t *Pt = Pt0 + pb * 4096;
+            if (t == 0 && tid == 0 && !S.abort) {
+                if (mbar_wait(&S.at_k[st], spar, P.timeout_ns, &S.abort)) {
+                    tc_fence_after();
+                    attn_scores_mma(S, Qt, st, nks, idesc_s);
+                } else {
+                    if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x96);
+                    S.abort = 1;
+                }
+            }
             const bool ok = __all_sync(0xffffffffu, !S.abort && mbar_wait(&S.at_s, par, P.timeout_ns, &S.abort));
-            const int pos = p0 + w * 32 + lane;
-            float v[32];
+            float v[16];
             if (ok) {
                 tc_fence_after();
-                tmem_ld32(S.tmem_base + ((uint32_t)(w * 32) << 16), v);
-                tc_fence_before();
+                tmem_ld16(S.tmem_base + ((uint32_t)(w * 32) << 16), v);
             }
+            tc_fence_before();
+            const int pw = w * 32 + lane;  // this thread's position in the tile
+            float sc[GC];
 #pragma unroll
-            for (int h = 0; h < GC; h++) sc[h] = (ok && pos < ctx && h < nh) ? v[h] + v[8 + h] : -CUDART_INF_F;
+            for (int h = 0; h < GC; h++) sc[h] = (ok && p0 + pw < ctx && h < nh) ? v[h] + v[8 + h] : -CUDART_INF_F;
 #pragma unroll
             for (int h = 0; h < GC; h++) {
                 const float mx = warp_max(sc[h]);
                 if (lane == 0) S.at.red[w * 8 + h] = mx;
             }
-        }
-        named_bar_sync(1, MR_WORKERS);
-        float corr[GC];
-#pragma unroll
-        for (int h = 0; h < GC; h++) {
-            const float mt = fmaxf(fmaxf(S.at.red[h], S.at.red[8 + h]), fmaxf(S.at.red[16 + h], S.at.red[24 + h]));
-            const float mn = fmaxf(M[h], mt);
-            corr[h] = rescale(M[h], mn);
-            M[h] = mn;
-        }
-        if (w < 4) {
-            float pv[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int h = 0; h < GC; h++) pv[h] = rescale(sc[h], M[h]);
-            *reinterpret_cast<float4 *>(Ps + (w * 32 + lane) * 4) = make_float4(pv[0], pv[1], pv[2], pv[3]);
+            named_bar_sync(2, 128);  // every score of the tile is read: TMEM columns 0-15 are free
+            bool issued = false;
+            if (tid == 0 && t + 1 < ntile && !S.abort) {
+                const unsigned long long n1 = t_it + 1;
+                if (mbar_test_wait(&S.at_k[n1 % AT_STAGES], (uint32_t)(n1 / AT_STAGES) & 1u)) {
+                    tc_fence_after();
+                    attn_scores_mma(S, Qt, (int)(n1 % AT_STAGES), nks, idesc_s);
+                    issued = true;
+                }
+            }
+            float corr[GC];
 #pragma unroll
             for (int h = 0; h < GC; h++) {
-                const float sm = warp_sum(pv[h]);
-                if (lane == 0) S.at.red[32 + w * 8 + h] = sm;
+                const float mt = fmaxf(fmaxf(S.at.red[h], S.at.red[8 + h]), fmaxf(S.at.red[16 + h], S.at.red[24 + h]));
+                const float mn = fmaxf(M[h], mt);
+                corr[h] = rescale(M[h], mn);
+                M[h] = mn;
+                if (tid == h) S.at_corr[pb][h] = corr[h];
             }
+            // Pt: this position's p of every head, hi in row h and lo in row 8 + h; even lanes
+            // store the pair (position, position + 1)
+            const int kb = pw >> 6, ch = (pw >> 3) & 7, within = (pw & 7) * 2;
+#pragma unroll
+            for (int h = 0; h < GC; h++) {
+                const float p = rescale(sc[h], M[h]);
+                Ls[h] = Ls[h] * corr[h] + p;
+                const uint32_t hi = store1<DT>(p), lo = store1<DT>(p - cvt1<DT>((uint16_t)hi));
+                const uint32_t hi1 = __shfl_down_sync(0xffffffffu, hi, 1), lo1 = __shfl_down_sync(0xffffffffu, lo, 1);
+                if (!(lane & 1)) {
+                    *reinterpret_cast<uint32_t *>(Pt + kb * 2048 + sw128(h, ch) + within) = hi | (hi1 << 16);
+                    *reinterpret_cast<uint32_t *>(Pt + kb * 2048 + sw128(8 + h, ch) + within) = lo | (lo1 << 16);
+                }
+            }
+            if (np < 128) {  // the last tile: V rows past the context (other positions' data) become zeros
+                const bool vok = __all_sync(0xffffffffu, !S.abort && mbar_wait(&S.at_v[st], spar, P.timeout_ns, &S.abort));
+                if (vok) {
+                    uint8_t *Vs = at_vbuf(S, st);
+                    const int per = (128 - np) * 8;  // 16-byte pieces per box
+                    for (int i = tid; i < nks * per; i += 128) {
+                        const int ks = i / per, r = np + (i % per) / 8, c = i % 8;
+                        *reinterpret_cast<uint4 *>(Vs + ks * TILE + r * 128 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                }
+            }
+            fence_proxy_async_smem();       // Pt (and the zeroed V rows) -> tensor-core reads
+            named_bar_sync(1, MR_WORKERS);  // the tile's Pt and correction are in (warps 4-7 join)
+            if (tid == 0 && !S.abort) {
+                if (mbar_wait(&S.at_v[st], spar, P.timeout_ns, &S.abort)) {
+                    tc_fence_after();
+                    attn_pv_mma(S, Pt, st, 32u + 16u * (uint32_t)pb, idesc_o);
+                } else {
+                    if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x97);
+                    S.abort = 1;
+                }
+                if (t + 1 < ntile && !issued && !S.abort) {
+                    const unsigned long long n1 = t_it + 1;
+                    if (mbar_wait(&S.at_k[n1 % AT_STAGES], (uint32_t)(n1 / AT_STAGES) & 1u, P.timeout_ns, &S.abort)) {
+                        tc_fence_after();
+                        attn_scores_mma(S, Qt, (int)(n1 % AT_STAGES), nks, idesc_s);
+                    } else {
+                        if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x98);
+                        S.abort = 1;
+                    }
+                }
+            }
+            t_it++;
         }
-        named_bar_sync(1, MR_WORKERS);
 #pragma unroll
         for (int h = 0; h < GC; h++) {
-            L[h] = L[h] * corr[h] + ((S.at.red[32 + h] + S.at.red[40 + h]) + (S.at.red[48 + h] + S.at.red[56 + h]));
-#pragma unroll
-            for (int e = 0; e < 8; e++) acc[h][e] *= corr[h];
+            const float s = warp_sum(Ls[h]);
+            if (lane == 0) S.at_l[w][h] = s;
         }
-        if (!S.abort && mbar_wait(&S.at_v[st], spar, P.timeout_ns, &S.abort)) {
-            for (int j = gi; j < np; j += ngroups) {
-                float f[8];
-                cvt8<DT>(*reinterpret_cast<const uint4 *>(Vs + (size_t)j * D * 2 + sl * 16), f);
-                const float4 pj = *reinterpret_cast<const float4 *>(Ps + j * 4);
-                const float pp[4] = {pj.x, pj.y, pj.z, pj.w};
+        named_bar_sync(1, MR_WORKERS);  // the sums' shares are in
+        named_bar_sync(1, MR_WORKERS);  // the unit's output is written
+    } else {  // ---- output warps
+        const int wq = w - 4;
+        float acc[GC];
 #pragma unroll
-                for (int h = 0; h < GC; h++)
+        for (int h = 0; h < GC; h++) acc[h] = 0.f;
+        for (int t = 0; t < ntile; t++) {
+            const int st = (int)(t_it % AT_STAGES), pb = (int)(t_it & 1ull);
+            const uint32_t par = (uint32_t)pb;  // the P.V barrier completes once per tile
+            named_bar_sync(1, MR_WORKERS);   // the tile's Pt and correction are in; its P.V follows
+            float corr[GC];
 #pragma unroll
-                    for (int e = 0; e < 8; e++) acc[h][e] = fmaf(pp[h], f[e], acc[h][e]);
+            for (int h = 0; h < GC; h++) corr[h] = S.at_corr[pb][h];
+            const bool ok = __all_sync(0xffffffffu, !S.abort && mbar_wait(&S.at_o, par, P.timeout_ns, &S.abort));
+            float v[16];
+            if (ok) {
+                tc_fence_after();
+                tmem_ld16(S.tmem_base + 32u + 16u * (uint32_t)pb + ((uint32_t)(wq * 32) << 16), v);
             }
-        } else if (tid == 0 && !S.abort) {
-            set_error(P.err, DERR_RING_TIMEOUT, 0x97);
-            S.abort = 1;
-        }
-        named_bar_sync(1, MR_WORKERS);  // this stage's K (the MMA is done) and V, and P, are consumed
-        if (tid == 0 && !S.abort && t + 2 < ntile) {
-            fence_proxy_async_smem();  // generic reads of the V buffer before the bulk copy refills it
-            load_tile(t + 2);
-        }
-        t_it++;
-    }
-    // hand the unit to the common tail: every thread holds the final M; L is counted once
-    float lsh[GC];
+            tc_fence_before();
+            if (ok) {
 #pragma unroll
-    for (int h = 0; h < GC; h++) lsh[h] = gi == 0 ? L[h] : 0.f;
-    attn_tail<DT, GC, NW, true>(A, S.at, g, Gt, hoff, M, lsh, acc);
+                for (int h = 0; h < GC; h++) acc[h] = acc[h] * corr[h] + (v[h] + v[8 + h]);
+            }
+            // the tile's K and V are consumed: its stage takes stream tile k + AT_STAGES
+            if (tid == 128 && !S.abort && k0 + t + AT_STAGES < ktot) {
+                fence_proxy_async_smem();
+                attn_issue(P, S, k0 + t + AT_STAGES, nunits, st, nks);
+            }
+            t_it++;
+        }
+        named_bar_sync(1, MR_WORKERS);  // the sums' shares are in
+        const int d = wq * 32 + lane;   // this thread's output dim
+#pragma unroll
+        for (int h = 0; h < GC; h++) {
+            const float L = ((S.at_l[0][h] + S.at_l[1][h]) + S.at_l[2][h]) + S.at_l[3][h];
+            const float o = acc[h] / L;
+            const float o1 = __shfl_down_sync(0xffffffffu, o, 1);
+            if (h < nh && d < D && !(lane & 1)) attn_out2<DT>(A, (g * Gt + hoff + h) * D + d, o, o1);
+        }
+        named_bar_sync(1, MR_WORKERS);  // the unit's output is written
+    }
 }
 
 // Attention of every row (a tick's sessions or a prefill chunk's positions): one unit per
 // (row, kv head), the unit's output written into the O projection's B operand.
 template <int DT>
-__device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M, uint32_t &k_it, uint32_t &t_it) {
+__device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M, uint32_t &k_it, unsigned long long &t_it) {
     const int G = P.G;
+    if (P.mr_kmap) {  // head_dim a multiple of 64: both products on the tensor cores
+        const int tid = threadIdx.x, nks = P.D >> 6, npass = (G + 3) / 4;
+        // this CTA's units, each as passes over 4 query heads at a time (one pass up to G = 4)
+        const int ne = (M * P.Hkv - (int)blockIdx.x + P.nblk - 1) / P.nblk * npass;
+        for (int b0 = 0; b0 < ne; b0 += NU_MAX) {  // streams of up to NU_MAX passes
+            const int nb = min(NU_MAX, ne - b0);
+            if (tid < nb) {
+                const int e = b0 + tid, u = blockIdx.x + (e / npass) * P.nblk, m = u / P.Hkv, g = u % P.Hkv;
+                const int sid = __ldcg(P.mr_sid + m), pos = __ldcg(P.mr_pos + m);
+                S.un_row0[tid] = (((long long)sid * P.L + l) * P.Hkv + g) * P.max_ctx;
+                S.un_ctx[tid] = pos + 1;
+                S.un_nt[tid] = (pos + 128) >> 7;
+            }
+            named_bar_sync(1, MR_WORKERS);
+            int ktot = 0;
+            for (int i = 0; i < nb; i++) ktot += S.un_nt[i];
+            if (tid == 0 || tid == 128) fence_proxy_async_global();  // the newest rows (written before the barrier)
+            if (tid == 0 && !S.abort) {
+                fence_proxy_async_smem();  // earlier reads of the ring before the copies refill it
+                for (int k = 0; k < AT_STAGES && k < ktot; k++) attn_issue(P, S, k, nb, (int)((t_it + k) % AT_STAGES), nks);
+            }
+            int k0 = 0;
+            for (int i = 0; i < nb; i++) {
+                const int e = b0 + i, u = blockIdx.x + (e / npass) * P.nblk, m = u / P.Hkv, g = u % P.Hkv;
+                const int hoff = 4 * (e % npass);
+                AttnArgs A;
+                A.q = P.mr_q + (size_t)m * P.Hq * P.D;
+                A.o = nullptr;
+                A.bpack = P.mr_bpack;  // the output is the O projection's B operand, row m
+                A.brow = m;
+                A.D = P.D;
+                tick_attn_tc<DT, 4>(P, S, A, g, G, hoff, i, nb, k0, ktot, t_it);
+                k0 += S.un_nt[i];
+            }
+        }
+        return;
+    }
     for (int u = blockIdx.x; u < M * P.Hkv; u += P.nblk) {
         const int m = u / P.Hkv, g = u % P.Hkv;
         const int sid = __ldcg(P.mr_sid + m), pos = __ldcg(P.mr_pos + m);
@@ -814,12 +972,6 @@ __device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M, uint32
         A.Hkv = P.Hkv;
         A.nsplit = 1;
         A.ctx = pos + 1;
-        if (P.mr_kmap) {  // head_dim a multiple of 64: scores on the tensor cores
-            const long long row0 = (((long long)sid * P.L + l) * P.Hkv + g) * P.max_ctx;
-            // up to 4 query heads per pass (fewer heads leave rows of the query operand zero)
-            for (int hoff = 0; hoff < G; hoff += 4) tick_attn_mma<DT, 4>(P, S, A, g, G, hoff, row0, t_it);
-            continue;
-        }
         for (int hoff = 0; hoff < G; hoff += 4) tick_attn_unit<DT, 4>(P, S, A, g, G, hoff, k_it);
     }
 }
@@ -937,7 +1089,7 @@ __device__ __forceinline__ void mr_mark(const KieParams &P, int st, int ev) {
 
 template <int DT>
 __device__ void mr_work(const KieParams &P, MrShared &S, uint32_t &b_it, uint32_t &u_it, uint32_t &k_it,
-                        uint32_t &t_it, const KieCmd &cmd, unsigned long long &epoch) {
+                        unsigned long long &t_it, const KieCmd &cmd, unsigned long long &epoch) {
     const int M = cmd.n_sess;
     const int steps = steps_of(cmd);
     for (int st = 0; st < steps; st++) {
@@ -1022,13 +1174,14 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
             mbar_init(&S.k_empty[i], MR_WORKERS / 32);
         }
         S.k_iss = 0;
-        for (int i = 0; i < 2; i++) {
+        for (int i = 0; i < AT_STAGES; i++) {
             mbar_init(&S.at_k[i], 1);
             mbar_init(&S.at_v[i], 1);
             S.tk_iss[i] = S.tv_iss[i] = 0;
         }
         mbar_init(&S.at_s, 1);
-        S.ts_iss = 0;
+        mbar_init(&S.at_o, 1);
+        S.ts_iss = S.to_iss = 0;
         S.att_seq = 0;
         fence_mbar_init();
         S.abort = 0;
@@ -1045,7 +1198,8 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
     __syncthreads();
     tc_fence_after();
 
-    uint32_t a_it = 0, b_it = 0, u_it = 0, k_it = 0, t_it = 0, o_seq = 0, drains = 0;
+    uint32_t a_it = 0, b_it = 0, u_it = 0, k_it = 0, o_seq = 0, drains = 0;
+    unsigned long long t_it = 0;  // attention tiles so far (stage = t_it mod 3 never jumps at a wrap)
     unsigned long long epoch = 0;
     for (;;) {
         if (tid < MR_WORKERS) {
@@ -1110,12 +1264,13 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
                 const uint32_t kfirst = S.k_iss > KV_SLOTS ? S.k_iss - KV_SLOTS : 0;
                 for (uint32_t k = kfirst; k < S.k_iss; k++)
                     mbar_wait(&S.k_full[k % KV_SLOTS], (k / KV_SLOTS) & 1u, P.timeout_ns, nullptr);
-                // the tensor-core attention's last K, V loads and score MMA (one of each in flight at most)
-                for (int i = 0; i < 2; i++) {  // per stage: its k-th copy completes phase k - 1
+                // the tensor-core attention's last K, V loads and products (one of each in flight at most)
+                for (int i = 0; i < AT_STAGES; i++) {  // per stage: its k-th copy completes phase k - 1
                     if (S.tk_iss[i]) mbar_wait(&S.at_k[i], (S.tk_iss[i] - 1) & 1u, P.timeout_ns, nullptr);
                     if (S.tv_iss[i]) mbar_wait(&S.at_v[i], (S.tv_iss[i] - 1) & 1u, P.timeout_ns, nullptr);
                 }
                 if (S.ts_iss) mbar_wait(&S.at_s, (S.ts_iss - 1) & 1u, P.timeout_ns, nullptr);
+                if (S.to_iss) mbar_wait(&S.at_o, (S.to_iss - 1) & 1u, P.timeout_ns, nullptr);
             }
         }
         __syncthreads();
