@@ -59,8 +59,11 @@ struct __align__(1024) MrShared {
     uint64_t acc_full[2], acc_empty[2], drain;
     uint64_t k_full[KV_SLOTS], k_empty[KV_SLOTS];  // the B ring as a K/V chunk ring in attention
     uint32_t k_iss;                              // K/V chunks issued so far (thread 0)
-    uint64_t at_k[AT_STAGES], at_v[AT_STAGES], at_s, at_o;  // tensor-core attention: K, V per stage; scores; P.V
-    uint32_t tk_iss[AT_STAGES], tv_iss[AT_STAGES], ts_iss, to_iss;  // copies / MMA groups issued
+    // tensor-core attention: K, V tile per stage; scores done; scores read (softmax threads);
+    // per P.V buffer: Pt and correction in (softmax threads), product done, product read
+    // (output threads); a unit's query operand in; a stream's table in
+    uint64_t at_k[AT_STAGES], at_v[AT_STAGES], at_s, at_sf, at_p[2], at_o[2], at_of[2], at_q, at_tab;
+    uint32_t tk_iss[AT_STAGES], tv_iss[AT_STAGES];  // tile copies issued
     float at_corr[2][KIE_GMAX];                  // per tile (two in flight): rescale of the running sums
     float at_l[4][KIE_GMAX];                     // the softmax warps' shares of the sums
     long long un_row0[NU_MAX];                   // the attention stream's units: first K/V arena row,
@@ -296,8 +299,11 @@ __device__ void mr_produce(const KieParams &P, MrShared &S, uint32_t &a_it, uint
 
 // ------------------------------------------------------------------ MMA issuer (warp 8, one lane)
 
+__device__ bool mr_attn_mma(const KieParams &P, MrShared &S, int M, unsigned long long &at_it, uint32_t &q_it,
+                            uint32_t &tab_it);
+
 __device__ void mr_mma(const KieParams &P, MrShared &S, uint32_t &a_it, uint32_t &b_it, uint32_t &u_it,
-                       const KieCmd &cmd) {
+                       unsigned long long &at_it, uint32_t &q_it, uint32_t &tab_it, const KieCmd &cmd) {
     const uint32_t idesc = idesc_f16(P.dtype);
     const int steps = steps_of(cmd);
     bool ok = true;
@@ -305,6 +311,11 @@ __device__ void mr_mma(const KieParams &P, MrShared &S, uint32_t &a_it, uint32_t
         for (int l = 0; l <= P.L && ok; l++) {
             if (l == P.L && !head_needed(cmd)) break;
             for (int g = (l < P.L ? 0 : G_HEAD); g < (l < P.L ? G_HEAD : NG) && ok; g++) {
+                // the tensor-core attention runs between the QKV and O projections
+                if (g == G_O && P.mr_kmap && !mr_attn_mma(P, S, cmd.n_sess, at_it, q_it, tab_it)) {
+                    ok = false;
+                    break;
+                }
                 const int K = gemm_of(P, g).K, natk = atoms_per_rb(K);
                 int cur_rb = -1;
                 uint32_t ab = 0;
@@ -686,7 +697,7 @@ __device__ void attn_issue(const KieParams &P, MrShared &S, int k, int nunits, i
     S.tv_iss[st]++;
 }
 
-// thread 0: the score product of the tile in stage st (K tile x query operand) into TMEM
+// the score product of the tile in stage st (K tile x query operand) into TMEM
 // columns 0-15
 KIE_DEV void attn_scores_mma(MrShared &S, const uint8_t *Qt, int st, int nks, uint32_t idesc) {
     const uint32_t sk = smem_u32(at_kbuf(S, st)), sq = smem_u32(Qt);
@@ -696,11 +707,11 @@ KIE_DEV void attn_scores_mma(MrShared &S, const uint8_t *Qt, int st, int nks, ui
             umma_f16(S.tmem_base, smem_desc_sw128(sk + ks * TILE + kk * 32), smem_desc_sw128(sq + ks * 2048 + kk * 32),
                      idesc, (ks | kk) ? 1u : 0u);
     umma_commit(&S.at_s);
-    S.ts_iss++;
 }
 
-// thread 0: the P.V product of the tile in stage st into TMEM columns col .. col + 15
-KIE_DEV void attn_pv_mma(MrShared &S, const uint8_t *Pt, int st, uint32_t col, uint32_t idesc) {
+// the P.V product of the tile in stage st into P.V buffer pb (TMEM columns 32 + 16 pb ..)
+KIE_DEV void attn_pv_mma(MrShared &S, const uint8_t *Pt, int st, int pb, uint32_t idesc) {
+    const uint32_t col = 32u + 16u * (uint32_t)pb;
     const uint32_t sv = smem_u32(at_vbuf(S, st)), sp = smem_u32(Pt);
 #pragma unroll
     for (int kb = 0; kb < 2; kb++)
@@ -708,12 +719,11 @@ KIE_DEV void attn_pv_mma(MrShared &S, const uint8_t *Pt, int st, uint32_t col, u
         for (int kk = 0; kk < 4; kk++)
             umma_f16(S.tmem_base + col, smem_desc_mn_sw128(sv + kb * 8192 + kk * 2048),
                      smem_desc_sw128(sp + kb * 2048 + kk * 32), idesc, (kb | kk) ? 1u : 0u);
-    umma_commit(&S.at_o);
-    S.to_iss++;
+    umma_commit(&S.at_o[pb]);
 }
 
 // One pass of a unit (row m, kv head g; query heads hoff .. hoff + GC - 1 of its Gt): stream
-// entry ui, tiles k0 .. k0 + ntile - 1 of the stream's ktot.
+// entry ui, tiles k0 .. k0 + ntile - 1 of the stream's ktot. Warp 8 issues the products.
 template <int DT, int GC>
 __device__ void tick_attn_tc(const KieParams &P, MrShared &S, const AttnArgs &A, int g, int Gt, int hoff, int ui,
                              int nunits, int k0, int ktot, unsigned long long &t_it) {
@@ -724,7 +734,6 @@ __device__ void tick_attn_tc(const KieParams &P, MrShared &S, const AttnArgs &A,
     const int ctx = S.un_ctx[ui], ntile = S.un_nt[ui];
     uint8_t *Qt = reinterpret_cast<uint8_t *>(S.at.wacc);  // [nks][16 rows][128 B], swizzled
     uint8_t *Pt0 = Qt + 4096;                              // two tiles of [2][16 rows][128 B], swizzled
-    const uint32_t idesc_s = idesc_f16(DT, 16), idesc_o = idesc_f16(DT, 16) | (1u << 15);  // V MN-major
 
     // the query operand: rows h (hi) and 8 + h (lo) of the scaled query heads, other rows zero
     const float qscale = rsqrtf((float)D) * 1.4426950408889634f;
@@ -751,6 +760,7 @@ __device__ void tick_attn_tc(const KieParams &P, MrShared &S, const AttnArgs &A,
     }
     fence_proxy_async_smem();  // generic writes of the query tile -> tensor-core reads
     named_bar_sync(1, MR_WORKERS);
+    if (tid == 0) mbar_arrive(&S.at_q);  // warp 8 may issue the unit's score products
 
     if (w < 4) {  // ---- softmax warps
         float M[GC], Ls[GC];
@@ -762,26 +772,19 @@ __device__ void tick_attn_tc(const KieParams &P, MrShared &S, const AttnArgs &A,
         for (int t = 0; t < ntile; t++) {  // uniform control flow: every thread reaches every barrier
             const int st = (int)(t_it % AT_STAGES);                   // this tile's K/V stage
             const uint32_t spar = (uint32_t)(t_it / AT_STAGES) & 1u;  // ... whose barriers complete every third tile
-            const int pb = (int)(t_it & 1ull);                        // its Pt, correction and P.V buffers
-            const uint32_t par = (uint32_t)pb;                        // the score barrier completes once per tile
+            const int pb = (int)(t_it & 1ull);                        // its Pt, correction, P.V and max buffers
+            const uint32_t prev = (uint32_t)((t_it >> 1) + 1) & 1u;   // the buffers' phase of tile t_it - 2
             const int p0 = t * 128, np = min(128, ctx - p0);
             uint8_t *Pt = Pt0 + pb * 4096;
-            if (t == 0 && tid == 0 && !S.abort) {
-                if (mbar_wait(&S.at_k[st], spar, P.timeout_ns, &S.abort)) {
-                    tc_fence_after();
-                    attn_scores_mma(S, Qt, st, nks, idesc_s);
-                } else {
-                    if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x96);
-                    S.abort = 1;
-                }
-            }
-            const bool ok = __all_sync(0xffffffffu, !S.abort && mbar_wait(&S.at_s, par, P.timeout_ns, &S.abort));
+            float *red = S.at.red + pb * 32;
+            const bool ok = __all_sync(0xffffffffu, !S.abort && mbar_wait(&S.at_s, (uint32_t)pb, P.timeout_ns, &S.abort));
             float v[16];
             if (ok) {
                 tc_fence_after();
                 tmem_ld16(S.tmem_base + ((uint32_t)(w * 32) << 16), v);
             }
             tc_fence_before();
+            mbar_arrive(&S.at_sf);  // this thread's scores are read: the next tile's product may follow
             const int pw = w * 32 + lane;  // this thread's position in the tile
             float sc[GC];
 #pragma unroll
@@ -789,27 +792,26 @@ __device__ void tick_attn_tc(const KieParams &P, MrShared &S, const AttnArgs &A,
 #pragma unroll
             for (int h = 0; h < GC; h++) {
                 const float mx = warp_max(sc[h]);
-                if (lane == 0) S.at.red[w * 8 + h] = mx;
+                if (lane == 0) red[w * 8 + h] = mx;
             }
-            named_bar_sync(2, 128);  // every score of the tile is read: TMEM columns 0-15 are free
-            bool issued = false;
-            if (tid == 0 && t + 1 < ntile && !S.abort) {
-                const unsigned long long n1 = t_it + 1;
-                if (mbar_test_wait(&S.at_k[n1 % AT_STAGES], (uint32_t)(n1 / AT_STAGES) & 1u)) {
-                    tc_fence_after();
-                    attn_scores_mma(S, Qt, (int)(n1 % AT_STAGES), nks, idesc_s);
-                    issued = true;
-                }
-            }
+            named_bar_sync(2, 128);
             float corr[GC];
 #pragma unroll
             for (int h = 0; h < GC; h++) {
-                const float mt = fmaxf(fmaxf(S.at.red[h], S.at.red[8 + h]), fmaxf(S.at.red[16 + h], S.at.red[24 + h]));
+                const float mt = fmaxf(fmaxf(red[h], red[8 + h]), fmaxf(red[16 + h], red[24 + h]));
                 const float mn = fmaxf(M[h], mt);
                 corr[h] = rescale(M[h], mn);
                 M[h] = mn;
-                if (tid == h) S.at_corr[pb][h] = corr[h];
             }
+            // the buffers' last tile (t_it - 2) is folded into the output: Pt, its correction and
+            // its P.V accumulator are free
+            if (t_it >= 2 && !__all_sync(0xffffffffu, !S.abort && mbar_wait(&S.at_of[pb], prev, P.timeout_ns, &S.abort))) {
+                if (lane == 0 && !S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x99);
+                if (lane == 0) S.abort = 1;
+            }
+#pragma unroll
+            for (int h = 0; h < GC; h++)
+                if (tid == h) S.at_corr[pb][h] = corr[h];
             // Pt: this position's p of every head, hi in row h and lo in row 8 + h; even lanes
             // store the pair (position, position + 1)
             const int kb = pw >> 6, ch = (pw >> 3) & 7, within = (pw & 7) * 2;
@@ -835,27 +837,8 @@ __device__ void tick_attn_tc(const KieParams &P, MrShared &S, const AttnArgs &A,
                     }
                 }
             }
-            fence_proxy_async_smem();       // Pt (and the zeroed V rows) -> tensor-core reads
-            named_bar_sync(1, MR_WORKERS);  // the tile's Pt and correction are in (warps 4-7 join)
-            if (tid == 0 && !S.abort) {
-                if (mbar_wait(&S.at_v[st], spar, P.timeout_ns, &S.abort)) {
-                    tc_fence_after();
-                    attn_pv_mma(S, Pt, st, 32u + 16u * (uint32_t)pb, idesc_o);
-                } else {
-                    if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x97);
-                    S.abort = 1;
-                }
-                if (t + 1 < ntile && !issued && !S.abort) {
-                    const unsigned long long n1 = t_it + 1;
-                    if (mbar_wait(&S.at_k[n1 % AT_STAGES], (uint32_t)(n1 / AT_STAGES) & 1u, P.timeout_ns, &S.abort)) {
-                        tc_fence_after();
-                        attn_scores_mma(S, Qt, (int)(n1 % AT_STAGES), nks, idesc_s);
-                    } else {
-                        if (!S.abort) set_error(P.err, DERR_RING_TIMEOUT, 0x98);
-                        S.abort = 1;
-                    }
-                }
-            }
+            fence_proxy_async_smem();  // Pt (and the zeroed V rows) -> tensor-core reads
+            mbar_arrive(&S.at_p[pb]);  // this thread's part of Pt and the correction are in
             t_it++;
         }
 #pragma unroll
@@ -872,18 +855,18 @@ __device__ void tick_attn_tc(const KieParams &P, MrShared &S, const AttnArgs &A,
         for (int h = 0; h < GC; h++) acc[h] = 0.f;
         for (int t = 0; t < ntile; t++) {
             const int st = (int)(t_it % AT_STAGES), pb = (int)(t_it & 1ull);
-            const uint32_t par = (uint32_t)pb;  // the P.V barrier completes once per tile
-            named_bar_sync(1, MR_WORKERS);   // the tile's Pt and correction are in; its P.V follows
-            float corr[GC];
+            const uint32_t ph = (uint32_t)(t_it >> 1) & 1u;  // the buffer's barriers complete every other tile
+            bool ok = __all_sync(0xffffffffu, !S.abort && mbar_wait(&S.at_p[pb], ph, P.timeout_ns, &S.abort));
+            ok = ok && __all_sync(0xffffffffu, !S.abort && mbar_wait(&S.at_o[pb], ph, P.timeout_ns, &S.abort));
+            float corr[GC], v[16];
 #pragma unroll
             for (int h = 0; h < GC; h++) corr[h] = S.at_corr[pb][h];
-            const bool ok = __all_sync(0xffffffffu, !S.abort && mbar_wait(&S.at_o, par, P.timeout_ns, &S.abort));
-            float v[16];
             if (ok) {
                 tc_fence_after();
                 tmem_ld16(S.tmem_base + 32u + 16u * (uint32_t)pb + ((uint32_t)(wq * 32) << 16), v);
             }
             tc_fence_before();
+            mbar_arrive(&S.at_of[pb]);  // this thread has read the product and the correction
             if (ok) {
 #pragma unroll
                 for (int h = 0; h < GC; h++) acc[h] = acc[h] * corr[h] + (v[h] + v[8 + h]);
@@ -908,6 +891,49 @@ __device__ void tick_attn_tc(const KieParams &P, MrShared &S, const AttnArgs &A,
     }
 }
 
+// Lane 0 of warp 8: the products of the tensor-core attention of one layer-step, in the order
+// the worker warps consume them: the score product of tile k as soon as its K tile is in and
+// the softmax threads have read tile k - 1's scores; the P.V of tile k once its Pt is written
+// (which also means the output threads are done with the buffer's tile k - 2) and its V is in.
+__device__ bool mr_attn_mma(const KieParams &P, MrShared &S, int M, unsigned long long &at_it, uint32_t &q_it,
+                            uint32_t &tab_it) {
+    const int nks = P.D >> 6, npass = (P.G + 3) / 4;
+    const uint32_t idesc_s = idesc_f16(P.dtype, 16), idesc_o = idesc_s | (1u << 15);  // V MN-major
+    const int ne = (M * P.Hkv - (int)blockIdx.x + P.nblk - 1) / P.nblk * npass;
+    const uint8_t *Qt = reinterpret_cast<const uint8_t *>(S.at.wacc), *Pt0 = Qt + 4096;
+    for (int b0 = 0; b0 < ne; b0 += NU_MAX) {
+        const int nb = min(NU_MAX, ne - b0);
+        if (!mbar_wait(&S.at_tab, tab_it & 1u, P.timeout_ns, &S.abort)) return false;
+        tab_it++;
+        for (int i = 0; i < nb; i++) {
+            const int ntile = S.un_nt[i];
+            if (!mbar_wait(&S.at_q, q_it & 1u, P.timeout_ns, &S.abort)) return false;
+            q_it++;
+            for (int t = 0; t <= ntile; t++) {
+                if (t < ntile) {
+                    const unsigned long long k = at_it + t;
+                    if (!mbar_wait(&S.at_k[k % AT_STAGES], (uint32_t)(k / AT_STAGES) & 1u, P.timeout_ns, &S.abort) ||
+                        (k > 0 && !mbar_wait(&S.at_sf, (uint32_t)((k - 1) & 1ull), P.timeout_ns, &S.abort)))
+                        return false;
+                    tc_fence_after();
+                    attn_scores_mma(S, Qt, (int)(k % AT_STAGES), nks, idesc_s);
+                }
+                if (t > 0) {
+                    const unsigned long long k = at_it + t - 1;
+                    const int pb = (int)(k & 1ull);
+                    if (!mbar_wait(&S.at_p[pb], (uint32_t)(k >> 1) & 1u, P.timeout_ns, &S.abort) ||
+                        !mbar_wait(&S.at_v[k % AT_STAGES], (uint32_t)(k / AT_STAGES) & 1u, P.timeout_ns, &S.abort))
+                        return false;
+                    tc_fence_after();
+                    attn_pv_mma(S, Pt0 + pb * 4096, (int)(k % AT_STAGES), pb, idesc_o);
+                }
+            }
+            at_it += ntile;
+        }
+    }
+    return true;
+}
+
 // Attention of every row (a tick's sessions or a prefill chunk's positions): one unit per
 // (row, kv head), the unit's output written into the O projection's B operand.
 template <int DT>
@@ -930,9 +956,12 @@ __device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M, uint32
             int ktot = 0;
             for (int i = 0; i < nb; i++) ktot += S.un_nt[i];
             if (tid == 0 || tid == 128) fence_proxy_async_global();  // the newest rows (written before the barrier)
-            if (tid == 0 && !S.abort) {
-                fence_proxy_async_smem();  // earlier reads of the ring before the copies refill it
-                for (int k = 0; k < AT_STAGES && k < ktot; k++) attn_issue(P, S, k, nb, (int)((t_it + k) % AT_STAGES), nks);
+            if (tid == 0) {
+                if (!S.abort) {
+                    fence_proxy_async_smem();  // earlier reads of the ring before the copies refill it
+                    for (int k = 0; k < AT_STAGES && k < ktot; k++) attn_issue(P, S, k, nb, (int)((t_it + k) % AT_STAGES), nks);
+                }
+                mbar_arrive(&S.at_tab);  // warp 8 may read the stream's table
             }
             int k0 = 0;
             for (int i = 0; i < nb; i++) {
@@ -1180,8 +1209,14 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
             S.tk_iss[i] = S.tv_iss[i] = 0;
         }
         mbar_init(&S.at_s, 1);
-        mbar_init(&S.at_o, 1);
-        S.ts_iss = S.to_iss = 0;
+        mbar_init(&S.at_sf, 128);
+        for (int i = 0; i < 2; i++) {
+            mbar_init(&S.at_p[i], 128);
+            mbar_init(&S.at_o[i], 1);
+            mbar_init(&S.at_of[i], 128);
+        }
+        mbar_init(&S.at_q, 1);
+        mbar_init(&S.at_tab, 1);
         S.att_seq = 0;
         fence_mbar_init();
         S.abort = 0;
@@ -1198,7 +1233,7 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
     __syncthreads();
     tc_fence_after();
 
-    uint32_t a_it = 0, b_it = 0, u_it = 0, k_it = 0, o_seq = 0, drains = 0;
+    uint32_t a_it = 0, b_it = 0, u_it = 0, k_it = 0, o_seq = 0, drains = 0, q_it = 0, tab_it = 0;
     unsigned long long t_it = 0;  // attention tiles so far (stage = t_it mod 3 never jumps at a wrap)
     unsigned long long epoch = 0;
     for (;;) {
@@ -1251,7 +1286,7 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
             if ((tid & 31) == 0) mr_produce(P, S, a_it, o_seq, cmd);
         } else if (warp == 8) {
             if ((tid & 31) == 0) {
-                mr_mma(P, S, a_it, b_it, u_it, cmd);
+                mr_mma(P, S, a_it, b_it, u_it, t_it, q_it, tab_it, cmd);
                 mbar_wait(&S.drain, drains & 1u, P.timeout_ns, nullptr);
             }
             drains++;
@@ -1264,13 +1299,11 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
                 const uint32_t kfirst = S.k_iss > KV_SLOTS ? S.k_iss - KV_SLOTS : 0;
                 for (uint32_t k = kfirst; k < S.k_iss; k++)
                     mbar_wait(&S.k_full[k % KV_SLOTS], (k / KV_SLOTS) & 1u, P.timeout_ns, nullptr);
-                // the tensor-core attention's last K, V loads and products (one of each in flight at most)
+                // the tensor-core attention's last K, V loads (its products drain with warp 8's)
                 for (int i = 0; i < AT_STAGES; i++) {  // per stage: its k-th copy completes phase k - 1
                     if (S.tk_iss[i]) mbar_wait(&S.at_k[i], (S.tk_iss[i] - 1) & 1u, P.timeout_ns, nullptr);
                     if (S.tv_iss[i]) mbar_wait(&S.at_v[i], (S.tv_iss[i] - 1) & 1u, P.timeout_ns, nullptr);
                 }
-                if (S.ts_iss) mbar_wait(&S.at_s, (S.ts_iss - 1) & 1u, P.timeout_ns, nullptr);
-                if (S.to_iss) mbar_wait(&S.at_o, (S.to_iss - 1) & 1u, P.timeout_ns, nullptr);
             }
         }
         __syncthreads();
