@@ -48,6 +48,8 @@ constexpr int MAXR = 64;                  // rows per step (hi half of B; lo hal
 constexpr int TMEM_COLS = 256;            // two 128-column fp32 accumulators
 constexpr int NU_MAX = 16;                // units per attention stream (a CTA with more runs several)
 constexpr int AT_STAGES = 3;              // K/V tile stages of the tensor-core attention (A ring x 2, B ring)
+constexpr int AS_MAX = 2048;              // (unit, pass) entries the longest-first assignment sorts
+constexpr int AS_LIST = 16;               // ... entries per CTA it can hand out (>= AS_MAX / 148, rounded up)
 
 enum { G_QKV = 0, G_O = 1, G_GU = 2, G_DOWN = 3, G_HEAD = 4, NG = 5 };
 
@@ -68,6 +70,9 @@ struct __align__(1024) MrShared {
     float at_l[4][KIE_GMAX];                     // the softmax warps' shares of the sums
     long long un_row0[NU_MAX];                   // the attention stream's units: first K/V arena row,
     int un_ctx[NU_MAX], un_nt[NU_MAX];           // context, tiles
+    int un_n, un_more;                           // units in the stream; another stream follows
+    int un_cnt;                                  // this CTA's (unit, pass) entries this step (-1: dealt in turn)
+    uint16_t un_list[AS_LIST];                   // ... and which, longest first
     volatile uint32_t att_seq;                   // attention phases finished (the producer waits on it)
     uint32_t tmem_base;
     KieCmd cmd;
@@ -700,25 +705,30 @@ __device__ void attn_issue(const KieParams &P, MrShared &S, int k, int nunits, i
 // the score product of the tile in stage st (K tile x query operand) into TMEM
 // columns 0-15
 KIE_DEV void attn_scores_mma(MrShared &S, const uint8_t *Qt, int st, int nks, uint32_t idesc) {
-    const uint32_t sk = smem_u32(at_kbuf(S, st)), sq = smem_u32(Qt);
-    for (int ks = 0; ks < nks; ks++)
+    // descriptors advance by their start-address field (16-byte units)
+    const uint64_t dk = smem_desc_sw128(smem_u32(at_kbuf(S, st))), dq = smem_desc_sw128(smem_u32(Qt));
+    const uint32_t tm = S.tmem_base;
+#pragma unroll
+    for (int ks = 0; ks < 2; ks++) {
+        if (ks == nks) break;
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
-            umma_f16(S.tmem_base, smem_desc_sw128(sk + ks * TILE + kk * 32), smem_desc_sw128(sq + ks * 2048 + kk * 32),
-                     idesc, (ks | kk) ? 1u : 0u);
+            umma_f16(tm, dk + (uint64_t)((ks * TILE + kk * 32) >> 4), dq + (uint64_t)((ks * 2048 + kk * 32) >> 4), idesc,
+                     (ks | kk) ? 1u : 0u);
+    }
     umma_commit(&S.at_s);
 }
 
 // the P.V product of the tile in stage st into P.V buffer pb (TMEM columns 32 + 16 pb ..)
 KIE_DEV void attn_pv_mma(MrShared &S, const uint8_t *Pt, int st, int pb, uint32_t idesc) {
-    const uint32_t col = 32u + 16u * (uint32_t)pb;
-    const uint32_t sv = smem_u32(at_vbuf(S, st)), sp = smem_u32(Pt);
+    const uint32_t tm = S.tmem_base + 32u + 16u * (uint32_t)pb;
+    const uint64_t dv = smem_desc_mn_sw128(smem_u32(at_vbuf(S, st))), dp = smem_desc_sw128(smem_u32(Pt));
 #pragma unroll
     for (int kb = 0; kb < 2; kb++)
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
-            umma_f16(S.tmem_base + col, smem_desc_mn_sw128(sv + kb * 8192 + kk * 2048),
-                     smem_desc_sw128(sp + kb * 2048 + kk * 32), idesc, (kb | kk) ? 1u : 0u);
+            umma_f16(tm, dv + (uint64_t)((kb * 8192 + kk * 2048) >> 4), dp + (uint64_t)((kb * 2048 + kk * 32) >> 4), idesc,
+                     (kb | kk) ? 1u : 0u);
     umma_commit(&S.at_o[pb]);
 }
 
@@ -784,7 +794,8 @@ __device__ void tick_attn_tc(const KieParams &P, MrShared &S, const AttnArgs &A,
                 tmem_ld16(S.tmem_base + ((uint32_t)(w * 32) << 16), v);
             }
             tc_fence_before();
-            mbar_arrive(&S.at_sf);  // this thread's scores are read: the next tile's product may follow
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.at_sf);  // the warp's scores are read: the next tile's product may follow
             const int pw = w * 32 + lane;  // this thread's position in the tile
             float sc[GC];
 #pragma unroll
@@ -838,7 +849,8 @@ __device__ void tick_attn_tc(const KieParams &P, MrShared &S, const AttnArgs &A,
                 }
             }
             fence_proxy_async_smem();  // Pt (and the zeroed V rows) -> tensor-core reads
-            mbar_arrive(&S.at_p[pb]);  // this thread's part of Pt and the correction are in
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.at_p[pb]);  // the warp's part of Pt (and the correction) is in
             t_it++;
         }
 #pragma unroll
@@ -866,7 +878,8 @@ __device__ void tick_attn_tc(const KieParams &P, MrShared &S, const AttnArgs &A,
                 tmem_ld16(S.tmem_base + 32u + 16u * (uint32_t)pb + ((uint32_t)(wq * 32) << 16), v);
             }
             tc_fence_before();
-            mbar_arrive(&S.at_of[pb]);  // this thread has read the product and the correction
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.at_of[pb]);  // the warp has read the product and the correction
             if (ok) {
 #pragma unroll
                 for (int h = 0; h < GC; h++) acc[h] = acc[h] * corr[h] + (v[h] + v[8 + h]);
@@ -897,14 +910,15 @@ __device__ void tick_attn_tc(const KieParams &P, MrShared &S, const AttnArgs &A,
 // (which also means the output threads are done with the buffer's tile k - 2) and its V is in.
 __device__ bool mr_attn_mma(const KieParams &P, MrShared &S, int M, unsigned long long &at_it, uint32_t &q_it,
                             uint32_t &tab_it) {
-    const int nks = P.D >> 6, npass = (P.G + 3) / 4;
+    const int nks = P.D >> 6;
     const uint32_t idesc_s = idesc_f16(P.dtype, 16), idesc_o = idesc_s | (1u << 15);  // V MN-major
-    const int ne = (M * P.Hkv - (int)blockIdx.x + P.nblk - 1) / P.nblk * npass;
     const uint8_t *Qt = reinterpret_cast<const uint8_t *>(S.at.wacc), *Pt0 = Qt + 4096;
-    for (int b0 = 0; b0 < ne; b0 += NU_MAX) {
-        const int nb = min(NU_MAX, ne - b0);
+    (void)M;
+    for (bool more = true; more;) {  // the worker warps hand over one stream table at a time
         if (!mbar_wait(&S.at_tab, tab_it & 1u, P.timeout_ns, &S.abort)) return false;
         tab_it++;
+        const int nb = S.un_n;
+        more = S.un_more != 0;
         for (int i = 0; i < nb; i++) {
             const int ntile = S.un_nt[i];
             if (!mbar_wait(&S.at_q, q_it & 1u, P.timeout_ns, &S.abort)) return false;
@@ -934,6 +948,79 @@ __device__ bool mr_attn_mma(const KieParams &P, MrShared &S, int M, unsigned lon
     return true;
 }
 
+// Balanced assignment of a step's attention entries (unit, pass of 4 query heads) to the
+// CTAs, computed alike in every CTA. With E entries on nblk CTAs, r = E mod nblk CTAs take
+// K + 1 = E / nblk + 1 entries and the others K; the entries, sorted by tiles (descending, then
+// by index), go largest first to the K-entry CTAs and the r * (K + 1) smallest to the others.
+// Within each group they are dealt in rounds of one per CTA, each round to the CTAs in order
+// of the tiles they hold so far (fewest first). Positions do not change within a step, so it
+// runs at the first layer; S.un_cnt = -1 leaves the entries dealt in turn (more entries than
+// it sorts, or loads past its key range).
+__device__ void attn_assign(const KieParams &P, MrShared &S, int M) {
+    const int tid = threadIdx.x, npass = (P.G + 3) / 4, E = M * P.Hkv * npass, nblk = P.nblk;
+    const int ntmax = (P.max_ctx + 127) >> 7;
+    if (E > AS_MAX || nblk > 256 || ntmax > 0xFFFF || (long long)ntmax * E >= (1ll << 23) ||
+        (E + nblk - 1) / nblk > AS_LIST) {
+        if (tid == 0) S.un_cnt = -1;
+        named_bar_sync(1, MR_WORKERS);
+        return;
+    }
+    // scratch in the activation ring (idle until the stream's first copies)
+    uint32_t *key = reinterpret_cast<uint32_t *>(S.b[0]);  // [ep] (65535 - tiles) << 16 | entry
+    uint32_t *ld = key + AS_MAX;                            // [256] tiles so far << 8 | CTA
+    int ep = 1;
+    while (ep < E) ep <<= 1;
+    for (int i = tid; i < ep; i += MR_WORKERS) {
+        uint32_t k = 0xFFFFFFFFu;
+        if (i < E) {
+            const int m = (i / npass) / P.Hkv;
+            const int nt = (__ldcg(P.mr_pos + m) + 128) >> 7;
+            k = ((uint32_t)(0xFFFF - nt) << 16) | (uint32_t)i;
+        }
+        key[i] = k;
+    }
+    if (tid == 0) S.un_cnt = 0;
+    auto bitonic = [&](uint32_t *a, int n) {  // ascending; one thread per compared pair
+        for (int k = 2; k <= n; k <<= 1)
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                named_bar_sync(1, MR_WORKERS);
+                for (int i = tid; i < n; i += MR_WORKERS) {
+                    const int x = i ^ j;
+                    if (x > i) {
+                        const uint32_t u = a[i], v = a[x];
+                        if ((u > v) == ((i & k) == 0)) {
+                            a[i] = v;
+                            a[x] = u;
+                        }
+                    }
+                }
+            }
+        named_bar_sync(1, MR_WORKERS);
+    };
+    bitonic(key, ep);
+    // entries [e0, e0 + n * rounds) to CTAs c0 .. c0 + n - 1, one per CTA per round
+    auto deal = [&](int e0, int c0, int n, int rounds) {
+        for (int i = tid; i < 256; i += MR_WORKERS) ld[i] = i < n ? (uint32_t)(c0 + i) : 0xFFFFFFFFu;
+        for (int r = 0; r < rounds; r++) {
+            named_bar_sync(1, MR_WORKERS);
+            for (int j = tid; j < n; j += MR_WORKERS) {
+                const uint32_t k = key[e0 + r * n + j];
+                const uint32_t nt = 0xFFFFu - (k >> 16), cta = ld[j] & 0xFFu;
+                ld[j] = (((ld[j] >> 8) + nt) << 8) | cta;
+                if ((int)cta == (int)blockIdx.x) {
+                    S.un_list[r] = (uint16_t)(k & 0xFFFFu);
+                    S.un_cnt = r + 1;
+                }
+            }
+            if (r + 1 < rounds) bitonic(ld, 256);
+        }
+        named_bar_sync(1, MR_WORKERS);
+    };
+    const int K = E / nblk, r = E % nblk;
+    if (K > 0) deal(0, r, nblk - r, K);               // the largest entries, K per CTA
+    if (r > 0) deal((nblk - r) * K, 0, r, K + 1);     // the smallest, K + 1 per CTA
+}
+
 // Attention of every row (a tick's sessions or a prefill chunk's positions): one unit per
 // (row, kv head), the unit's output written into the O projection's B operand.
 template <int DT>
@@ -941,16 +1028,30 @@ __device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M, uint32
     const int G = P.G;
     if (P.mr_kmap) {  // head_dim a multiple of 64: both products on the tensor cores
         const int tid = threadIdx.x, nks = P.D >> 6, npass = (G + 3) / 4;
-        // this CTA's units, each as passes over 4 query heads at a time (one pass up to G = 4)
-        const int ne = (M * P.Hkv - (int)blockIdx.x + P.nblk - 1) / P.nblk * npass;
-        for (int b0 = 0; b0 < ne; b0 += NU_MAX) {  // streams of up to NU_MAX passes
-            const int nb = min(NU_MAX, ne - b0);
+        if (l == 0) attn_assign(P, S, M);
+        // this CTA's entries (unit, pass over 4 query heads at a time; one pass up to G = 4)
+        const bool dealt = S.un_cnt >= 0;
+        const int ne = dealt ? S.un_cnt : (M * P.Hkv - (int)blockIdx.x + P.nblk - 1) / P.nblk * npass;
+        auto entry = [&](int i, int &u, int &hoff) {
+            const int e = dealt ? (int)S.un_list[i] : ((int)blockIdx.x + (i / npass) * P.nblk) * npass + i % npass;
+            u = e / npass;
+            hoff = 4 * (e % npass);
+        };
+        int b0 = 0;
+        do {  // streams of up to NU_MAX entries (at least one, maybe empty: warp 8 waits for it)
+            const int nb = max(0, min(NU_MAX, ne - b0));
             if (tid < nb) {
-                const int e = b0 + tid, u = blockIdx.x + (e / npass) * P.nblk, m = u / P.Hkv, g = u % P.Hkv;
+                int u, hoff;
+                entry(b0 + tid, u, hoff);
+                const int m = u / P.Hkv, g = u % P.Hkv;
                 const int sid = __ldcg(P.mr_sid + m), pos = __ldcg(P.mr_pos + m);
                 S.un_row0[tid] = (((long long)sid * P.L + l) * P.Hkv + g) * P.max_ctx;
                 S.un_ctx[tid] = pos + 1;
                 S.un_nt[tid] = (pos + 128) >> 7;
+            }
+            if (tid == 0) {
+                S.un_n = nb;
+                S.un_more = b0 + nb < ne;
             }
             named_bar_sync(1, MR_WORKERS);
             int ktot = 0;
@@ -965,8 +1066,9 @@ __device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M, uint32
             }
             int k0 = 0;
             for (int i = 0; i < nb; i++) {
-                const int e = b0 + i, u = blockIdx.x + (e / npass) * P.nblk, m = u / P.Hkv, g = u % P.Hkv;
-                const int hoff = 4 * (e % npass);
+                int u, hoff;
+                entry(b0 + i, u, hoff);
+                const int m = u / P.Hkv, g = u % P.Hkv;
                 AttnArgs A;
                 A.q = P.mr_q + (size_t)m * P.Hq * P.D;
                 A.o = nullptr;
@@ -976,7 +1078,8 @@ __device__ void phase_attn(const KieParams &P, MrShared &S, int l, int M, uint32
                 tick_attn_tc<DT, 4>(P, S, A, g, G, hoff, i, nb, k0, ktot, t_it);
                 k0 += S.un_nt[i];
             }
-        }
+            b0 += nb;
+        } while (b0 < ne);
         return;
     }
     for (int u = blockIdx.x; u < M * P.Hkv; u += P.nblk) {
@@ -1209,11 +1312,11 @@ __global__ void __launch_bounds__(MR_THREADS, 1) kie_mr_kernel(KieParams P, KieC
             S.tk_iss[i] = S.tv_iss[i] = 0;
         }
         mbar_init(&S.at_s, 1);
-        mbar_init(&S.at_sf, 128);
+        mbar_init(&S.at_sf, 4);  // one arrival per softmax warp
         for (int i = 0; i < 2; i++) {
-            mbar_init(&S.at_p[i], 128);
+            mbar_init(&S.at_p[i], 4);
             mbar_init(&S.at_o[i], 1);
-            mbar_init(&S.at_of[i], 128);
+            mbar_init(&S.at_of[i], 4);  // one arrival per output warp
         }
         mbar_init(&S.at_q, 1);
         mbar_init(&S.at_tab, 1);
