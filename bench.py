@@ -545,7 +545,9 @@ def run_tick(n_ticks: int, warmup: int, local: int, clocks_for: int, model_name:
         tick_bytes.append(b)
     gbs = float(np.median(np.array(tick_bytes) / (lat / 1e3)) / 1e9)
     misses = int((lat > TICK_DEADLINE_MS).sum())
-    return {"model": "dense-10.8b bf16 (48L d4096 32/8x128 F14336 V32000)", "sessions": TICK_SESSIONS,
+    shape = (f"{m.name} {'bf16' if m.dtype == 1 else 'fp16'} ({m.n_layers}L d{m.d_model} "
+             f"{m.n_heads}/{m.n_kv_heads}x{m.head_dim} F{m.ffn} V{m.vocab})")
+    return {"model": shape, "sessions": TICK_SESSIONS,
             "steps_per_tick": TICK_STEPS, "ticks": n_ticks, "session_ticks": TICK_SESSIONS * n_ticks,
             "ctx_start_range": [min(lens), max(lens)], "p50_ms": round(float(np.percentile(lat, 50)), 3),
             "p99_ms": round(float(np.percentile(lat, 99)), 3), "max_ms": round(float(lat.max()), 3),
