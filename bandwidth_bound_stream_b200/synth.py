@@ -98,8 +98,14 @@ SLICE_TICK = dataclasses.replace(TICK_10P8B, name="slice-10.8b", n_layers=2)
 RAGGED = ModelConfig("ragged", 3, 384, 6, 2, 64, 1216, 5003, BF16, rope_theta=1e4)
 # head_dim 32, 5 query heads per kv head, odd k-step counts (d = 320, F = 576), odd vocabulary
 SMALL_HEAD = ModelConfig("small-head", 2, 320, 10, 2, 32, 576, 3001, FP16, rope_theta=1e4)
+# head_dim 64 with 6 query heads per kv head: the tick's tensor-core attention takes two passes
+# per unit (4 heads, then 2)
+GQA6 = ModelConfig("gqa6", 2, 512, 12, 2, 64, 1024, 3001, BF16, rope_theta=1e4)
+# 32 kv heads of 5 query heads: a 64-position prefill chunk has 64 x 32 x 2 attention passes,
+# more than the tick kernel balances per step, and more than one stream of them per SM
+WIDE_KV = ModelConfig("wide-kv", 2, 256, 160, 32, 64, 512, 1031, FP16, rope_theta=1e4)
 CONFIGS = {c.name: c for c in (TINY, DENSE_1P9B, DENSE_8B, TICK_10P8B, SLICE_1P9B, SLICE_8B,
-                                SLICE_TICK, RAGGED, SMALL_HEAD)}
+                                SLICE_TICK, RAGGED, SMALL_HEAD, GQA6, WIDE_KV)}
 
 
 def _lib():

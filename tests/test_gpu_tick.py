@@ -189,6 +189,20 @@ def test_tick_ragged_parity_many_tiles(kie):
     _run_tick_parity(kie, synth.RAGGED, 3, [301, 480, 650], checked=[0, 1, 2], ticks=2, max_ctx=670)
 
 
+def test_tick_two_passes_per_unit(kie):
+    """bf16, head_dim 64, 6 query heads per kv head: every unit of the tensor-core attention is
+    two passes (4 heads, then 2) over the same K/V tiles; prompts end mid-tile and mid-chunk."""
+    from bandwidth_bound_stream_b200 import synth
+    _run_tick_parity(kie, synth.GQA6, 3, [300, 129, 517], checked=[0, 1, 2], ticks=2, max_ctx=540)
+
+
+def test_tick_wide_kv_many_passes(kie):
+    """32 kv heads of 5 query heads: a prefill chunk's 64 x 32 x 2 attention passes exceed the
+    per-step balancing (they are dealt in turn) and fill more than one stream per SM."""
+    from bandwidth_bound_stream_b200 import synth
+    _run_tick_parity(kie, synth.WIDE_KV, 2, [200, 70], checked=[0, 1], ticks=2, max_ctx=220)
+
+
 def _run_tick_injected(kie, model, lens, checked, ticks, prompt_checks=()):
     """Prefill every session (tick-kernel chunks), then `ticks` two-step ticks with logits. For
     each checked session the oracle continues from the engine's cache (tests/inject.py): both
