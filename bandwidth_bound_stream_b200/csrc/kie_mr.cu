@@ -10,14 +10,15 @@
 //   D[128 weight rows][128] (fp32, TMEM) += A[128 weight rows][64] * B[128][64]^T  per k-step
 //
 // A is a 128 x 64 weight tile, stored in HBM already in the K-major 128-byte-swizzled layout
-// the MMA reads, and streamed by the producer warp with 1-D bulk copies into an 8-slot ring.
+// the MMA reads, and streamed by the producer warp with 1-D bulk copies, two tiles (32 KB) per
+// copy, into a ring of four such atoms.
 // B holds the activations split into two 16-bit halves: rows 0-63 carry hi(x) and rows
 // 64-127 carry lo(x) = x - hi(x), so D[:, s] + D[:, 64 + s] equals W x_s to about 16 bits of
 // the fp32 activation (the tensor cores take 16-bit operands only). The phase that finalises
 // an activation writes it once, already in that tile layout, to a small global buffer (one
 // tile per k-step: the RMSNorm phases for QKV, gate/up and the head, attention for O, the
 // activation phase silu(gate)*up for down); during the GEMM, thread 0 streams the tile of
-// each k-step from there (L2) into a 4-slot ring with bulk copies, beside the weight tiles.
+// each k-step from there (L2) into a ring of two atoms with bulk copies, beside the weight tiles.
 // Warp 8 issues tcgen05.mma and commits, warps 4-7 read the accumulator from TMEM and add
 // it into the fp32 outputs with atomics: the weight tiles of one phase are split evenly over
 // the SMs by k-steps, so partial sums of a row block from several SMs meet in global memory.
@@ -25,7 +26,8 @@
 // Phases per layer, each ended by a grid barrier: NORM1 (per-row 1/rms -> QKV operand, clear
 // the QKV accumulator) | QKV | ROPE (rotate q and k, append K and V) | ATTN (-> O operand) |
 // O (+= residual) | NORM2 | GATE/UP | ACT | DOWN (+= residual); then NORMF | HEAD | ARGMAX
-// per step.
+// per step. Attention puts both of its products on the tensor cores as well (see the
+// tensor-core attention below), with warp 8 issuing them between the QKV and O projections.
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
@@ -676,11 +678,13 @@ __device__ void tick_attn_unit(const KieParams &P, MrShared &S, const AttnArgs &
 // attention is done, and no activation tile moves during it). The copies of stream tile k + 3
 // -- the next unit's first tiles near the end of a unit -- are issued as soon as tile k's
 // products are done, so loads run on across unit boundaries.
-// Warps 0-3 run the softmax: a position each from TMEM, the running max M per head (the same
-// in every thread) and each thread's share of the running sum. They write Pt, and thread 0
-// issues the next tile's score product as soon as its K tile is in, before the current
-// tile's P.V. Warps 4-7 fold each tile's P.V into the output one tile behind (a dim each
-// from TMEM, rescaled by the tile's correction), and issue the tile copies.
+// Warp 8 (the GEMM MMA warp, idle in this phase) issues both products of every tile: the
+// score product as soon as the tile's K is in and the softmax warps have read the previous
+// tile's scores, the P.V once the tile's Pt is written and its V is in. Warps 0-3 run the
+// softmax: a position each from TMEM, the running max M per head (the same in every thread)
+// and each thread's share of the running sum; they write Pt (two buffers). Warps 4-7 fold
+// each tile's P.V (two TMEM buffers) into the output, rescaled by the tile's correction, and
+// issue the tile copies. The three roles meet at mbarriers only (one arrival per warp).
 
 // the K and V tile buffers of attention stage st: two stages in the weight ring, one in the
 // activation ring (both idle during attention)
