@@ -469,7 +469,6 @@ extern "C" kie_status kie_create(const kie_config *cfg, const kie_weights *w, ki
         for (int cc = 0; cc < nblk; cc++) {
             long long off = seg_off[cc];
             for (int l = 0; l <= L; l++) {
-                const void *const *Lw = w->layers + (size_t)9 * (l < L ? l : 0);
                 for (int ph = (l < L ? 0 : PH_HEAD); ph < (l < L ? PH_HEAD : KIE_NPH); ph++) {
                     const int a = row0[ph * (nblk + 1) + cc], n = range(ph, cc);
                     if (ph == PH_OF || ph == PH_DF) {
