@@ -902,7 +902,9 @@ __device__ void tick_attn_tc(const KieParams &P, MrShared &S, const AttnArgs &A,
             const float L = ((S.at_l[0][h] + S.at_l[1][h]) + S.at_l[2][h]) + S.at_l[3][h];
             const float o = acc[h] / L;
             const float o1 = __shfl_down_sync(0xffffffffu, o, 1);
-            if (h < nh && d < D && !(lane & 1)) attn_out2<DT>(A, (g * Gt + hoff + h) * D + d, o, o1);
+            if (h < nh && d < D && !(lane & 1) &&
+                in_bounds(A.brow < MAXR && (g * Gt + hoff + h) * D + d + 1 < P.Hq * P.D, P.err, 0x28))
+                attn_out2<DT>(A, (g * Gt + hoff + h) * D + d, o, o1);
         }
         named_bar_sync(1, MR_WORKERS);  // the unit's output is written
     }
